@@ -1,0 +1,423 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the WKV-7 recurrence on B200 (synthetic inputs).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one pass of the hot path over one batch of the workload:
+  prefill-0.19b (default): wkv7_forward on B8 T1024 H12 N64, bf16 inputs, fp32
+      state carried in (S0 ~ N(0, 0.1^2)) and out, y fp32;
+  prefill-1.5b: B16 T4096 H32 with the fused group_norm + bonus epilogue;
+  long-context: B1 T65536 H40, decay logits ~ N(2, 1), snapshots every 4096 tokens;
+  decode: one wkv7_decode_step on B256 H40 (fp32 state in HBM).
+Prints ONE JSON line (rank 0). Under torchrun every rank runs its own independent
+batch (weak scaling over (b, h) units, no collective on the data path); the timed
+region is bracketed by a barrier and a device synchronisation, and the time is the
+max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_rnn_sequence_rwkv_b200 import inputs  # noqa: E402
+
+METRIC = "WKV-7 Mtokens·heads/s (prefill, decode) at N=64 bf16; % of HBM/FP32/TC roofline"
+UNIT = "Mtoken·heads/s"
+L2_BYTES = 126 * 2 ** 20
+NAMES = ("r", "w", "k", "v", "kk", "a")
+
+WORKLOADS = {
+    "prefill-0.19b": dict(cid=1, default_steps=200),
+    "prefill-1.5b": dict(cid=2, default_steps=20),
+    "long-context": dict(cid=4, default_steps=10),
+    "decode": dict(cid=3, default_steps=256),
+}
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+# ---- clocks sampled during the timed region (NVML, polled from a thread) -------------------------
+
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = torch.cuda.get_device_properties(device_index).uuid
+            self._h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if str(uuid) in u:
+                    self._h = h
+            if self._h is None:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - depends on the box
+            self._nv = None
+            self.error = str(e)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if self._nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "error", "")}
+        names = [n for n, bit in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ---- distributed plumbing -------------------------------------------------------------------------
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---- workload set-up ---------------------------------------------------------------------------
+
+def algorithmic_bytes(wl, B, T, H, dt_bytes, s0: bool, s_out: bool, snaps: int, epilogue: bool) -> int:
+    """Bytes one forward must move at minimum: inputs once, y once, states once."""
+    N = wl.N
+    per_tok = 6 * N * dt_bytes + N * 4
+    st = N * N * 4
+    extra = (H * N * 3 * 4) if epilogue else 0
+    return B * T * H * per_tok + B * H * st * (int(s0) + int(s_out) + snaps) + extra
+
+
+def run_gpu(args, world, rank, local):
+    from linear_rnn_sequence_rwkv_b200 import wkv7
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    spec = WORKLOADS[args.workload]
+    wl = inputs.WORKLOADS[spec["cid"]]
+    steps = args.steps if args.steps is not None else spec["default_steps"]
+    warmup = args.warmup
+    peaks, peak_kind = _peaks()
+    stream = torch.cuda.current_stream(dev)
+    decode = args.workload == "decode"
+    snap_every = wl.snap_every
+
+    # independent batches per rank (seed offset), rotating input sets larger than L2
+    seed0 = inputs.SEED_BASE + wl.cid + 1000 * rank
+    if decode:
+        n_tok = 128
+        d = inputs.make_inputs(wl, device=str(dev), seed=seed0, T=n_tok)
+        B, H, N = wl.B, wl.H, wl.N
+        steps_in = {n: d[n].transpose(0, 1).contiguous() for n in NAMES}      # [128, B, H, N]
+        S = torch.zeros(B, H, N, N, device=dev)
+        y = torch.empty(B, H, N, device=dev)
+        T = 1
+        n_sets = 1
+
+        def step(i):
+            j = i % n_tok
+            wkv7.decode_step(*(steps_in[n][j] for n in NAMES), S, y=y)
+        bytes_per_launch = B * H * (6 * N * 2 + N * 4 + 2 * N * N * 4)
+        launches_per_step = 1
+        epilogue = False
+    else:
+        B, T, H, N = wl.B, wl.T, wl.H, wl.N
+        set_bytes = B * T * H * N * (6 * 2)
+        n_sets = max(1, min(8, math.ceil(2 * L2_BYTES / set_bytes)))
+        sets = [inputs.make_inputs(wl, device=str(dev), seed=seed0 + 17 * i) for i in range(n_sets)]
+        y = torch.empty(B, T, H, N, device=dev)
+        S_T = torch.empty(B, H, N, N, device=dev)
+        snaps = torch.empty(B, T // snap_every, H, N, N, device=dev) if snap_every else None
+        epilogue = wl.epilogue
+        ws_need = wkv7.workspace_bytes(B, T, H, N, torch.bfloat16, algo=args.algo, chunk=args.chunk,
+                                       snap_every=snap_every)
+        ws = torch.empty(max(ws_need, 1), dtype=torch.uint8, device=dev)
+
+        def step(i):
+            s = sets[i % n_sets]
+            ep = dict(ln_w=s["ln_w"], ln_b=s["ln_b"], r_k=s["r_k"]) if epilogue else {}
+            wkv7.forward(*(s[n] for n in NAMES), s["S0"], algo=args.algo, chunk=args.chunk, y=y, S_T=S_T,
+                         snap_every=snap_every, snapshots=snaps, workspace=ws, **ep)
+        bytes_per_launch = algorithmic_bytes(wl, B, T, H, 2, sets[0]["S0"] is not None, True,
+                                             T // snap_every if snap_every else 0, epilogue)
+        launches_per_step = 1 + (1 if epilogue and args.algo in ("seq",) else 0)
+
+    units_per_step = B * T * H
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+
+    # timed region: K steps, one event pair per step on the launching stream
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        ev[0].record(stream)
+        for i in range(steps):
+            step(warmup + i)
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    per_step_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    total_ms = ev[0].elapsed_time(ev[steps])
+    total_ms = max_over_ranks(total_ms, world, dev)
+    value = units_per_step * steps * world / (total_ms * 1e-3) / 1e6
+    launch_ms = statistics.mean(per_step_ms)
+
+    # roofline of the dominant kernel
+    hbm_peak = float(peaks["hbm_gbs"])
+    achieved_gbs = bytes_per_launch / (launch_ms * 1e-3) / 1e9
+    flops_per_launch = 36864 * units_per_step   # 9 N^2 per token-head: the exact recurrence
+    path = "decode" if decode else _path_name(args)
+    if path == "seq":
+        sm_max = float(peaks.get("sm_max_mhz", 1965.0))
+        fp32_peak = 148 * 128 * 2 * sm_max * 1e6 / 1e12
+        achieved = flops_per_launch / (launch_ms * 1e-3) / 1e12
+        roof = {"bound": "alu", "achieved": round(achieved, 3), "peak": round(fp32_peak, 2),
+                "unit": "TFLOP/s", "frac": round(achieved / fp32_peak, 4),
+                "peak_source": f"148 SMs x 128 FP32 lanes x 2 flop x {sm_max:.0f} MHz (derived)",
+                "traffic": None, "kernel": "seq_kernel",
+                "hbm_gbs": round(achieved_gbs, 1), "hbm_frac": round(achieved_gbs / hbm_peak, 4)}
+    else:
+        roof = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(achieved_gbs / hbm_peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
+                "traffic": None, "kernel": "decode_kernel" if decode else path,
+                "recurrence_tflops": round(flops_per_launch / (launch_ms * 1e-3) / 1e12, 3)}
+    roof["algorithmic_bytes_per_launch"] = bytes_per_launch
+
+    # end to end through the public API with pinned host buffers (copies inside the timed region)
+    e2e = None
+    if not decode:
+        e2e = run_e2e(args, wl, dev, stream, B, T, H, N, seed0, epilogue, snap_every, warmup,
+                      max(1, min(steps, 10)), world)
+
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": round(total_ms / steps, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32" if path in ("seq", "decode") else "tf32+f32",
+        "data": "synthetic (seeded torch Philox; shapes and value ranges of the RWKV-7 pages' workloads)",
+        "config": {"workload": f"{args.workload}: {wl.name}", "B": B, "T": T, "H": H, "N": N,
+                   "input_dtype": "bf16", "path": path, "chunk": args.chunk or None,
+                   "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world} (independent (b,h) units)",
+                   "l2": (f"{n_sets} rotating input sets, {n_sets * B * T * H * N * 12 / 1e6:.0f} MB > 126 MB L2"
+                          if not decode else "fp32 state 168 MB > 126 MB L2, 128 rotating token inputs")},
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": steps * launches_per_step,
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, decode)
+    return out
+
+
+def _path_name(args):
+    from linear_rnn_sequence_rwkv_b200 import wkv7  # noqa: F401
+    return {"auto": "seq", "seq": "seq"}.get(args.algo, args.algo)
+
+
+def run_e2e(args, wl, dev, stream, B, T, H, N, seed, epilogue, snap_every, warmup, steps, world):
+    """Same metric through wkv7.forward with pinned HOST tensors: H2D of the inputs,
+    the kernels and D2H of y and S_T are all inside the timed region."""
+    from linear_rnn_sequence_rwkv_b200 import wkv7
+    d = inputs.make_inputs(wl, device="cpu", seed=seed + 999)
+    host = {n: (v.pin_memory() if isinstance(v, torch.Tensor) else v) for n, v in d.items()}
+    h2d = sum(host[n].numel() * host[n].element_size() for n in NAMES)
+    h2d += 0 if host["S0"] is None else host["S0"].numel() * 4
+    if epilogue:
+        h2d += 3 * H * N * 4
+    d2h = B * T * H * N * 4 + B * H * N * N * 4 + (B * (T // snap_every) * H * N * N * 4 if snap_every else 0)
+    y_h = torch.empty(B, T, H, N).pin_memory()
+    S_h = torch.empty(B, H, N, N).pin_memory()
+
+    def once():
+        ep = {n: host[n] for n in ("ln_w", "ln_b", "r_k")} if epilogue else {}
+        y, S, _ = wkv7.forward(*(host[n] for n in NAMES), host["S0"], algo=args.algo, chunk=args.chunk,
+                               snap_every=snap_every, out_host=(y_h, S_h), **ep)
+        return y, S
+
+    for _ in range(max(1, min(warmup, 3))):
+        once()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        once()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    return {"value": round(B * T * H * steps * world / (ms * 1e-3) / 1e6, 3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 4)}
+
+
+def cpu_baseline(wl, decode: bool, budget_s: float = 12.0):
+    """The fp64 oracle (plain C, threads over (b, h)) on a bounded sample of the workload."""
+    import numpy as np
+    from oracle import native
+    if decode:
+        B, T, H = 16, 1, wl.H
+        d = inputs.make_inputs(wl, B=B, T=T, H=H, s0="normal")
+        sample = f"{B * H} heads x 1 decode step (S0 ~ N(0, 0.1^2)), repeated"
+    else:
+        T = min(wl.T, 4096)
+        H = wl.H
+        B = max(1, min(wl.B, 2 if wl.T > 2048 else wl.B))
+        d = inputs.make_inputs(wl, B=B, T=T, H=H)
+        sample = f"B{B} T{T} H{H} of the workload's first batch rows"
+    arrs = {n: np.ascontiguousarray(d[n].to(torch.float64).numpy()) for n in NAMES}
+    s0 = None if d["S0"] is None else np.ascontiguousarray(d["S0"].to(torch.float64).numpy())
+    units = B * T * H
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        native.forward(*(arrs[n] for n in NAMES), s0)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el > budget_s / 4 or reps >= 200:
+            break
+    return {"value": round(units * reps / el / 1e6, 5), "unit": UNIT, "cores": native.host_threads(),
+            "kind": "oracle", "sample": f"{sample}; {reps} run(s), {el:.1f} s wall"}
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the fp64 CPU oracle, as it stands, on host cores (rank 0 only)."""
+    if rank != 0:
+        return None
+    spec = WORKLOADS[args.workload]
+    wl = inputs.WORKLOADS[spec["cid"]]
+    steps = args.steps if args.steps is not None else 3
+    decode = args.workload == "decode"
+    import numpy as np
+    from oracle import native
+    if decode:
+        B, T, H = 32, 1, wl.H
+    else:
+        B, T, H = min(wl.B, 2), min(wl.T, 1024), wl.H
+    d = inputs.make_inputs(wl, B=B, T=T, H=H)
+    arrs = {n: np.ascontiguousarray(d[n].to(torch.float64).numpy()) for n in NAMES}
+    s0 = None if d["S0"] is None else np.ascontiguousarray(d["S0"].to(torch.float64).numpy())
+    for _ in range(args.warmup):
+        native.forward(*(arrs[n] for n in NAMES), s0)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        native.forward(*(arrs[n] for n in NAMES), s0)
+    el = time.perf_counter() - t0
+    value = B * T * H * steps / el / 1e6
+    cores = native.host_threads()
+    sample = f"B{B} T{T} H{H} sample of {wl.name} per step"
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": world,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": round(el / steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": f"{args.workload}: {wl.name}", "sample": sample},
+            "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="prefill-0.19b")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--algo", choices=["auto", "seq", "chunk", "split"], default="auto")
+    ap.add_argument("--chunk", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out))
+        return 0
+
+    world, rank, local = dist_setup()
+    if world != args.gpus and rank == 0:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    try:
+        out = run_gpu(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(out))
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,150 @@
+/*
+ * wkv7.h -- C ABI of the B200 (sm_100a) WKV-7 library.
+ *
+ * The WKV-7 operator is the time-mixing recurrence of RWKV-7 "Goose". Per batch
+ * element b and head h it carries an N x N fp32 state S (row i = value channel,
+ * column j = key channel) through the tokens t = 0..T-1:
+ *
+ *     S_t = S_{t-1} diag(w_t) - (S_{t-1} kk_t)(kk_t * a_t)^T + v_t k_t^T
+ *     y_t = S_t r_t
+ *
+ * (RWKV-7 rebuttal page, numpy time_mixing listing: the update and readout lines;
+ * ARWKV verdict page, key_machinery: the same update in row-vector form.)
+ * The optional epilogue (same listing: group_norm lambda and the bonus line)
+ * replaces y_t, per head, by
+ *
+ *     (y_t - mean) / sqrt(var + gn_eps) * ln_w[h] + ln_b[h]
+ *       + (sum_j r_t[j] k_t[j] r_k[h][j]) * v_t
+ *
+ * with the population variance over the N channels of the head.
+ *
+ * Conventions for every entry point:
+ *   - N must be 64 (the head size the kernels are written for).
+ *   - Token tensors r, w, k, v, kk, a are [B][T][H][N] row-major (decode: [B][H][N]),
+ *     all of the dtype given by `dt`. States are [B][H][N][N] fp32 row-major.
+ *     y is fp32 with the layout of the token tensors.
+ *   - Every pointer is a device pointer (cudaMalloc / caching allocator / managed)
+ *     on the current device, 16-byte aligned. Host pointers are rejected before
+ *     any launch (WKV7_ERR_ARG), as are pointers whose allocation is too small
+ *     for the stated sizes (when the driver can report the allocation's range).
+ *   - The caller owns every buffer. The library never allocates device memory and
+ *     never synchronises; work is enqueued on `stream` (a cudaStream_t, NULL for
+ *     the legacy default stream). Asynchronous faults appear at the caller's next
+ *     synchronisation, as for any CUDA kernel.
+ *   - Input contract (not validated on the hot path): kk is already L2-normalised
+ *     per head, k is the replacement key, w is the decay multiplier in (0, 1],
+ *     a is the in-context learning rate (any finite value is accepted).
+ *   - Errors are returned as wkv7_status; nothing is thrown across the ABI.
+ *     wkv7_last_error() gives a human-readable detail for the calling thread.
+ */
+#ifndef WKV7_H
+#define WKV7_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define WKV7_API __attribute__((visibility("default")))
+#else
+#define WKV7_API
+#endif
+
+#define WKV7_ABI_VERSION 1
+#define WKV7_HEAD_SIZE 64
+
+typedef enum wkv7_status {
+    WKV7_OK = 0,
+    WKV7_ERR_ARG = 1,          /* null / host / too-small pointer, bad size or option   */
+    WKV7_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement (N != 64) */
+    WKV7_ERR_ALIGN = 3,        /* a pointer is not 16-byte aligned                       */
+    WKV7_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed                    */
+    WKV7_ERR_TIMEOUT = 5,      /* reserved: a bounded device-side wait gave up           */
+    WKV7_ERR_WORKSPACE = 6     /* workspace missing or smaller than wkv7_workspace_bytes */
+} wkv7_status;
+
+typedef enum wkv7_dtype {
+    WKV7_F32 = 0,
+    WKV7_BF16 = 1
+} wkv7_dtype;
+
+typedef enum wkv7_algo {
+    WKV7_ALGO_AUTO = 0,   /* pick from dtype, T and B*H                                  */
+    WKV7_ALGO_SEQ = 1,    /* token-by-token scan, fp32 FMA; any T, any dtype             */
+    WKV7_ALGO_CHUNK = 2,  /* chunked prefill on tcgen05 tensor cores, fp32 chunk carry   */
+    WKV7_ALGO_SPLIT = 3   /* chunked prefill with T split into segments across CTAs      */
+} wkv7_algo;
+
+/* Options of wkv7_forward. Obtain defaults with wkv7_opts_default(). */
+typedef struct wkv7_opts {
+    int algo;             /* wkv7_algo                                                   */
+    int chunk;            /* chunk length of the chunked algorithms; 0 = default         */
+    int snap_every;       /* 0 = no snapshots; else store S after every snap_every tokens */
+    float *snapshots;     /* [B][T / snap_every][H][N][N] fp32, required if snap_every>0 */
+    const float *ln_w;    /* epilogue: all three NULL (off) or all three [H][N] fp32     */
+    const float *ln_b;
+    const float *r_k;
+    float gn_eps;         /* epilogue epsilon added to the variance (default 64e-5)      */
+    int segments;         /* WKV7_ALGO_SPLIT: T segments per (b, h); 0 = automatic       */
+} wkv7_opts;
+
+/* Fills *opts with the defaults: AUTO, default chunk, no snapshots, no epilogue,
+ * gn_eps = 64e-5, automatic segments. */
+WKV7_API void wkv7_opts_default(wkv7_opts *opts);
+
+/*
+ * Prefill / full-sequence forward.
+ *
+ * Inputs  r, w, k, v, kk, a : [B][T][H][N] of dtype dt.
+ *         S0                : [B][H][N][N] fp32, or NULL for a zero initial state.
+ * Outputs y                 : [B][T][H][N] fp32 (epilogue applied when enabled).
+ *         S_T               : [B][H][N][N] fp32 final state, or NULL. May equal S0
+ *                             (in-place hand-off); must not otherwise overlap inputs.
+ *         opts->snapshots   : states after tokens snap_every * m, m = 1..T/snap_every.
+ * Workspace: device memory of at least wkv7_workspace_bytes(...) bytes for the same
+ *         arguments (0 bytes for most configurations; NULL is then allowed).
+ * B, H >= 1; T >= 0 (T = 0 copies S0 to S_T, or zeros when S0 is NULL).
+ * (RWKV-7 paper summary, section 8: chunked pre-fill with a user-chosen chunk,
+ * forward inference with and without state storage.)
+ */
+WKV7_API wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype dt,
+                         const void *r, const void *w, const void *k, const void *v,
+                         const void *kk, const void *a,
+                         const float *S0, float *y, float *S_T,
+                         const wkv7_opts *opts,
+                         void *workspace, size_t workspace_bytes,
+                         void *stream);
+
+/*
+ * One decode step for every (b, h): the recurrence for a single token, with the
+ * state read and written in place.
+ *
+ * Inputs  r, w, k, v, kk, a : [B][H][N] of dtype dt.
+ * In/out  S                 : [B][H][N][N] fp32, updated in place.
+ * Output  y                 : [B][H][N] fp32 readout of the updated state.
+ * (RWKV-7 paper summary, section 8: single-token inference at constant memory.)
+ */
+WKV7_API wkv7_status wkv7_decode_step(int B, int H, int N, wkv7_dtype dt,
+                             const void *r, const void *w, const void *k, const void *v,
+                             const void *kk, const void *a,
+                             float *S, float *y, void *stream);
+
+/* Bytes of device workspace wkv7_forward needs for these arguments (opts may be NULL). */
+WKV7_API size_t wkv7_workspace_bytes(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opts *opts);
+
+/* Static string naming a status. */
+WKV7_API const char *wkv7_status_string(wkv7_status status);
+
+/* Detail of the last error returned on the calling thread ("" if none). */
+WKV7_API const char *wkv7_last_error(void);
+
+/* WKV7_ABI_VERSION of the loaded library. */
+WKV7_API int wkv7_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WKV7_H */

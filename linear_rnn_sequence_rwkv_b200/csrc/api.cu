@@ -1,0 +1,273 @@
+// C ABI of the WKV-7 library: argument validation, workspace sizing, dispatch.
+//
+// Every check that can fail runs on the host before anything is enqueued, so a bad
+// argument never reaches a kernel. Launches go to the caller's stream; nothing here
+// allocates device memory or synchronises.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+wkv7_status fail(wkv7_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+wkv7_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(WKV7_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// cuMemGetAddressRange through the runtime's driver entry point (no -lcuda needed).
+typedef CUresult (*AddrRangeFn)(CUdeviceptr *, size_t *, CUdeviceptr);
+AddrRangeFn addr_range_fn() {
+    static std::once_flag once;
+    static AddrRangeFn fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<AddrRangeFn>(p);
+    });
+    return fn;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Buf {
+    const char *name;
+    const void *ptr;
+    size_t bytes;
+};
+
+// Device-side checks of one buffer: device memory of the current device, large enough.
+wkv7_status check_device_buffer(const Buf &b, int device) {
+    if (!b.ptr || b.bytes == 0) return WKV7_OK;
+    cudaPointerAttributes at;
+    cudaError_t e = cudaPointerGetAttributes(&at, b.ptr);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(WKV7_ERR_ARG, "%s: cannot query pointer attributes (%s)", b.name, cudaGetErrorName(e));
+    }
+    if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged)
+        return fail(WKV7_ERR_ARG, "%s: not device memory (memory type %d)", b.name, (int)at.type);
+    if (at.type == cudaMemoryTypeDevice && at.device != device)
+        return fail(WKV7_ERR_ARG, "%s: allocated on device %d, current device is %d", b.name, at.device, device);
+    if (AddrRangeFn fn = addr_range_fn()) {
+        CUdeviceptr base = 0;
+        size_t size = 0;
+        if (fn(&base, &size, reinterpret_cast<CUdeviceptr>(b.ptr)) == CUDA_SUCCESS) {
+            const uintptr_t end = reinterpret_cast<uintptr_t>(b.ptr) + b.bytes;
+            if (end > static_cast<uintptr_t>(base) + size)
+                return fail(WKV7_ERR_ARG, "%s: needs %zu bytes but its allocation ends %zu bytes after it",
+                            b.name, b.bytes, static_cast<size_t>(base + size - reinterpret_cast<uintptr_t>(b.ptr)));
+        }
+    }
+    return WKV7_OK;
+}
+
+bool overlaps(const Buf &x, const Buf &y) {
+    if (!x.ptr || !y.ptr || !x.bytes || !y.bytes) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(x.ptr), a1 = a0 + x.bytes;
+    const uintptr_t b0 = reinterpret_cast<uintptr_t>(y.ptr), b1 = b0 + y.bytes;
+    return a0 < b1 && b0 < a1;
+}
+
+size_t elem_bytes(wkv7_dtype dt) { return dt == WKV7_BF16 ? 2 : 4; }
+
+// Product of non-negative sizes with overflow detection (returns false on overflow).
+bool mul_ok(size_t &acc, long long f) {
+    if (f < 0) return false;
+    if (f != 0 && acc > SIZE_MAX / static_cast<size_t>(f)) return false;
+    acc *= static_cast<size_t>(f);
+    return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+void wkv7_opts_default(wkv7_opts *o) {
+    if (!o) return;
+    std::memset(o, 0, sizeof(*o));
+    o->algo = WKV7_ALGO_AUTO;
+    o->gn_eps = 64e-5f;
+}
+
+const char *wkv7_status_string(wkv7_status s) {
+    switch (s) {
+        case WKV7_OK: return "WKV7_OK";
+        case WKV7_ERR_ARG: return "WKV7_ERR_ARG";
+        case WKV7_ERR_UNSUPPORTED: return "WKV7_ERR_UNSUPPORTED";
+        case WKV7_ERR_ALIGN: return "WKV7_ERR_ALIGN";
+        case WKV7_ERR_CUDA: return "WKV7_ERR_CUDA";
+        case WKV7_ERR_TIMEOUT: return "WKV7_ERR_TIMEOUT";
+        case WKV7_ERR_WORKSPACE: return "WKV7_ERR_WORKSPACE";
+    }
+    return "WKV7_ERR_UNKNOWN";
+}
+
+const char *wkv7_last_error(void) { return g_err; }
+
+int wkv7_abi_version(void) { return WKV7_ABI_VERSION; }
+
+size_t wkv7_workspace_bytes(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opts *opts) {
+    (void)B; (void)T; (void)H; (void)N; (void)dt; (void)opts;
+    return 0;
+}
+
+wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype dt, const void *r, const void *w,
+                         const void *k, const void *v, const void *kk, const void *a, const float *S0,
+                         float *y, float *S_T, const wkv7_opts *opts_in, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+    g_err[0] = '\0';
+    if (N <= 0 || B <= 0 || H <= 0 || T < 0)
+        return fail(WKV7_ERR_ARG, "bad sizes B=%d T=%d H=%d N=%d (need B,H,N >= 1, T >= 0)", B, T, H, N);
+    if (N != wkv7::kN) return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: only N=64 is implemented", N);
+    if (dt != WKV7_F32 && dt != WKV7_BF16) return fail(WKV7_ERR_ARG, "unknown dtype %d", (int)dt);
+    wkv7_opts opts;
+    wkv7_opts_default(&opts);
+    if (opts_in) opts = *opts_in;
+    if (opts.algo < WKV7_ALGO_AUTO || opts.algo > WKV7_ALGO_SPLIT)
+        return fail(WKV7_ERR_ARG, "unknown algo %d", opts.algo);
+    if (!(opts.chunk == 0 || opts.chunk == 16 || opts.chunk == 32 || opts.chunk == 64))
+        return fail(WKV7_ERR_ARG, "chunk=%d: must be 0 (default), 16, 32 or 64", opts.chunk);
+    if (opts.snap_every < 0) return fail(WKV7_ERR_ARG, "snap_every=%d < 0", opts.snap_every);
+    if (opts.snap_every > 0 && !opts.snapshots && T >= opts.snap_every)
+        return fail(WKV7_ERR_ARG, "snap_every=%d but snapshots is NULL", opts.snap_every);
+    const int n_epi = (opts.ln_w != nullptr) + (opts.ln_b != nullptr) + (opts.r_k != nullptr);
+    if (n_epi != 0 && n_epi != 3) return fail(WKV7_ERR_ARG, "epilogue needs all of ln_w, ln_b, r_k (or none)");
+    if (n_epi == 3 && !(std::isfinite(opts.gn_eps) && opts.gn_eps >= 0.f))
+        return fail(WKV7_ERR_ARG, "gn_eps must be finite and >= 0");
+    if (opts.segments < 0) return fail(WKV7_ERR_ARG, "segments=%d < 0", opts.segments);
+
+    size_t tok = 1, st = 1;
+    if (!mul_ok(tok, B) || !mul_ok(tok, T) || !mul_ok(tok, H) || !mul_ok(tok, N) || !mul_ok(st, B) ||
+        !mul_ok(st, H) || !mul_ok(st, N) || !mul_ok(st, N) || tok > (size_t(1) << 40))
+        return fail(WKV7_ERR_ARG, "sizes overflow");
+    const size_t in_bytes = tok * elem_bytes(dt), y_bytes = tok * 4, st_bytes = st * 4;
+    const int n_snap = opts.snap_every > 0 ? T / opts.snap_every : 0;
+    const size_t snap_bytes = st_bytes * static_cast<size_t>(n_snap);
+
+    if (T > 0) {
+        const void *req[] = {r, w, k, v, kk, a, y};
+        const char *names[] = {"r", "w", "k", "v", "kk", "a", "y"};
+        for (int i = 0; i < 7; ++i)
+            if (!req[i]) return fail(WKV7_ERR_ARG, "%s is NULL", names[i]);
+    }
+    const Buf bufs[] = {{"r", r, T ? in_bytes : 0},      {"w", w, T ? in_bytes : 0},
+                        {"k", k, T ? in_bytes : 0},      {"v", v, T ? in_bytes : 0},
+                        {"kk", kk, T ? in_bytes : 0},    {"a", a, T ? in_bytes : 0},
+                        {"S0", S0, st_bytes},            {"y", y, T ? y_bytes : 0},
+                        {"S_T", S_T, st_bytes},          {"snapshots", n_snap ? opts.snapshots : nullptr, snap_bytes},
+                        {"ln_w", opts.ln_w, size_t(H) * N * 4}, {"ln_b", opts.ln_b, size_t(H) * N * 4},
+                        {"r_k", opts.r_k, size_t(H) * N * 4},   {"workspace", workspace, workspace_bytes}};
+    constexpr int nb = sizeof(bufs) / sizeof(bufs[0]);
+    for (int i = 0; i < nb; ++i)
+        if (bufs[i].ptr && !aligned16(bufs[i].ptr))
+            return fail(WKV7_ERR_ALIGN, "%s is not 16-byte aligned", bufs[i].name);
+    const size_t need_ws = wkv7_workspace_bytes(B, T, H, N, dt, &opts);
+    if (need_ws > 0 && (!workspace || workspace_bytes < need_ws))
+        return fail(WKV7_ERR_WORKSPACE, "workspace of %zu bytes required, %zu given", need_ws,
+                    workspace ? workspace_bytes : 0);
+    // Outputs must not overlap inputs (S_T == S0 exactly is the allowed in-place hand-off).
+    const Buf &yb = bufs[7], &sb = bufs[8], &snb = bufs[9];
+    for (int i = 0; i < 7; ++i) {
+        if (i < 6 && overlaps(yb, bufs[i])) return fail(WKV7_ERR_ARG, "y overlaps %s", bufs[i].name);
+        if (i < 6 && overlaps(sb, bufs[i])) return fail(WKV7_ERR_ARG, "S_T overlaps %s", bufs[i].name);
+        if (overlaps(snb, bufs[i])) return fail(WKV7_ERR_ARG, "snapshots overlap %s", bufs[i].name);
+    }
+    if (overlaps(yb, sb)) return fail(WKV7_ERR_ARG, "y overlaps S_T");
+    if (overlaps(sb, bufs[6]) && S_T != S0) return fail(WKV7_ERR_ARG, "S_T partially overlaps S0");
+    if (overlaps(snb, sb) || overlaps(snb, bufs[6])) return fail(WKV7_ERR_ARG, "snapshots overlap a state");
+
+    int device = 0;
+    cudaError_t e = cudaGetDevice(&device);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return cuda_fail(e, "cudaGetDevice");
+    }
+    for (int i = 0; i < nb; ++i) {
+        const wkv7_status s = check_device_buffer(bufs[i], device);
+        if (s != WKV7_OK) return s;
+    }
+
+    wkv7::FwdArgs p{};
+    p.B = B; p.T = T; p.H = H; p.dt = dt;
+    p.r = r; p.w = w; p.k = k; p.v = v; p.kk = kk; p.a = a;
+    p.S0 = S0; p.y = y; p.S_T = S_T;
+    p.snap_every = n_snap ? opts.snap_every : 0;
+    p.snaps = n_snap ? opts.snapshots : nullptr;
+    p.ln_w = opts.ln_w; p.ln_b = opts.ln_b; p.r_k = opts.r_k; p.gn_eps = opts.gn_eps;
+    p.chunk = opts.chunk; p.segments = opts.segments;
+    p.ws = workspace; p.ws_bytes = workspace_bytes;
+    p.stream = static_cast<cudaStream_t>(stream);
+
+    if (T == 0) {
+        if (!S_T || S_T == S0) return WKV7_OK;
+        e = wkv7::launch_copy_state(p);
+        return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "state copy launch");
+    }
+    e = wkv7::launch_seq(p);
+    if (e != cudaSuccess) return cuda_fail(e, "sequential-scan launch");
+    if (n_epi == 3) {
+        e = wkv7::launch_epilogue(p);
+        if (e != cudaSuccess) return cuda_fail(e, "epilogue launch");
+    }
+    return WKV7_OK;
+}
+
+wkv7_status wkv7_decode_step(int B, int H, int N, wkv7_dtype dt, const void *r, const void *w, const void *k,
+                             const void *v, const void *kk, const void *a, float *S, float *y, void *stream) {
+    g_err[0] = '\0';
+    if (N <= 0 || B <= 0 || H <= 0) return fail(WKV7_ERR_ARG, "bad sizes B=%d H=%d N=%d", B, H, N);
+    if (N != wkv7::kN) return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: only N=64 is implemented", N);
+    if (dt != WKV7_F32 && dt != WKV7_BF16) return fail(WKV7_ERR_ARG, "unknown dtype %d", (int)dt);
+    size_t tok = 1;
+    if (!mul_ok(tok, B) || !mul_ok(tok, H) || !mul_ok(tok, N) || tok > (size_t(1) << 36))
+        return fail(WKV7_ERR_ARG, "sizes overflow");
+    const void *req[] = {r, w, k, v, kk, a, S, y};
+    const char *names[] = {"r", "w", "k", "v", "kk", "a", "S", "y"};
+    const size_t in_bytes = tok * elem_bytes(dt);
+    const size_t bytes[] = {in_bytes, in_bytes, in_bytes, in_bytes, in_bytes, in_bytes, tok * N * 4, tok * 4};
+    for (int i = 0; i < 8; ++i) {
+        if (!req[i]) return fail(WKV7_ERR_ARG, "%s is NULL", names[i]);
+        if (!aligned16(req[i])) return fail(WKV7_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
+    }
+    const Buf sb{"S", S, bytes[6]}, yb{"y", y, bytes[7]};
+    for (int i = 0; i < 6; ++i) {
+        const Buf ib{names[i], req[i], in_bytes};
+        if (overlaps(sb, ib) || overlaps(yb, ib)) return fail(WKV7_ERR_ARG, "output overlaps %s", names[i]);
+    }
+    if (overlaps(sb, yb)) return fail(WKV7_ERR_ARG, "y overlaps S");
+    int device = 0;
+    cudaError_t e = cudaGetDevice(&device);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return cuda_fail(e, "cudaGetDevice");
+    }
+    for (int i = 0; i < 8; ++i) {
+        const wkv7_status s = check_device_buffer(Buf{names[i], req[i], bytes[i]}, device);
+        if (s != WKV7_OK) return s;
+    }
+    wkv7::DecArgs p{B, H, dt, r, w, k, v, kk, a, S, y, static_cast<cudaStream_t>(stream)};
+    e = wkv7::launch_decode(p);
+    return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "decode launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,66 @@
+// Shared device helpers and the internal launcher interface of the WKV-7 library.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "wkv7.h"
+
+namespace wkv7 {
+
+constexpr int kN = WKV7_HEAD_SIZE;   // head size: the state of one (b, h) is kN x kN fp32
+
+// Arguments of one forward call after validation (device pointers, caller's stream).
+struct FwdArgs {
+    int B, T, H;
+    wkv7_dtype dt;
+    const void *r, *w, *k, *v, *kk, *a;
+    const float *S0;       // nullable: zero initial state
+    float *y;
+    float *S_T;            // nullable
+    int snap_every;        // 0 = off
+    float *snaps;          // [B][T/snap_every][H][N][N]
+    const float *ln_w, *ln_b, *r_k;   // all null = no epilogue
+    float gn_eps;
+    int chunk;
+    int segments;
+    void *ws;
+    size_t ws_bytes;
+    cudaStream_t stream;
+};
+
+struct DecArgs {
+    int B, H;
+    wkv7_dtype dt;
+    const void *r, *w, *k, *v, *kk, *a;
+    float *S;
+    float *y;
+    cudaStream_t stream;
+};
+
+// Launchers (each returns the launch status; no synchronisation).
+cudaError_t launch_seq(const FwdArgs &p);
+cudaError_t launch_epilogue(const FwdArgs &p);
+cudaError_t launch_decode(const DecArgs &p);
+cudaError_t launch_copy_state(const FwdArgs &p);   // T == 0: S_T <- S0 (or zeros)
+
+// ---- device helpers -------------------------------------------------------------------------
+
+__device__ __forceinline__ float bf16_lo(uint32_t packed) { return __uint_as_float(packed << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t packed) { return __uint_as_float(packed & 0xffff0000u); }
+
+// Four consecutive elements starting at p (16-byte aligned for float, 8-byte for bf16).
+__device__ __forceinline__ float4 load4(const float *p) { return __ldg(reinterpret_cast<const float4 *>(p)); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
+    return make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
+}
+__device__ __forceinline__ float load1(const float *p) { return __ldg(p); }
+__device__ __forceinline__ float load1(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+
+__device__ __forceinline__ float dot4(float4 a, float4 b) {
+    return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
+}
+
+}  // namespace wkv7

@@ -1,0 +1,196 @@
+"""Python binding of the WKV-7 C ABI (include/wkv7.h), loaded with ctypes.
+
+Argument marshalling only: torch tensors supply device memory and the current
+CUDA stream; every step of the computation runs in the library's CUDA kernels.
+There is no CPU fallback: without the built library or a CUDA device these
+functions raise.
+
+Host (CPU) tensors are accepted by ``forward`` and ``decode_step`` for callers
+that keep their data on the host: the inputs are copied to the device, the
+kernels run, and the outputs are copied back (the end-to-end path).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libwkv7.so")
+HEAD_SIZE = 64
+
+# wkv7_status
+OK, ERR_ARG, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(7)
+# wkv7_dtype
+F32, BF16 = 0, 1
+# wkv7_algo
+ALGOS = {"auto": 0, "seq": 1, "chunk": 2, "split": 3}
+
+EXPORTED = ("wkv7_opts_default", "wkv7_forward", "wkv7_decode_step", "wkv7_workspace_bytes",
+            "wkv7_status_string", "wkv7_last_error", "wkv7_abi_version")
+
+
+class Wkv7Error(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__(f"{where}: status {status} ({detail})")
+        self.status = status
+
+
+class Opts(ctypes.Structure):
+    _fields_ = [("algo", ctypes.c_int), ("chunk", ctypes.c_int), ("snap_every", ctypes.c_int),
+                ("snapshots", ctypes.c_void_p), ("ln_w", ctypes.c_void_p), ("ln_b", ctypes.c_void_p),
+                ("r_k", ctypes.c_void_p), ("gn_eps", ctypes.c_float), ("segments", ctypes.c_int)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load libwkv7.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                               "`python -m linear_rnn_sequence_rwkv_b200.build`")
+        lib = ctypes.CDLL(_LIB_PATH)
+        vp, ci = ctypes.c_void_p, ctypes.c_int
+        lib.wkv7_opts_default.argtypes = [ctypes.POINTER(Opts)]
+        lib.wkv7_opts_default.restype = None
+        lib.wkv7_forward.argtypes = [ci, ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp, ctypes.POINTER(Opts),
+                                                                       vp, ctypes.c_size_t, vp]
+        lib.wkv7_forward.restype = ci
+        lib.wkv7_decode_step.argtypes = [ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp]
+        lib.wkv7_decode_step.restype = ci
+        lib.wkv7_workspace_bytes.argtypes = [ci, ci, ci, ci, ci, ctypes.POINTER(Opts)]
+        lib.wkv7_workspace_bytes.restype = ctypes.c_size_t
+        lib.wkv7_status_string.argtypes = [ci]
+        lib.wkv7_status_string.restype = ctypes.c_char_p
+        lib.wkv7_last_error.argtypes = []
+        lib.wkv7_last_error.restype = ctypes.c_char_p
+        lib.wkv7_abi_version.argtypes = []
+        lib.wkv7_abi_version.restype = ci
+        _lib = lib
+        return lib
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        lib = load()
+        detail = lib.wkv7_last_error().decode() or lib.wkv7_status_string(status).decode()
+        raise Wkv7Error(status, where, detail)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype}: use bfloat16 or float32")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(device, stream):
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_opts(algo="auto", chunk=0, snap_every=0, snapshots=None, ln_w=None, ln_b=None, r_k=None,
+              gn_eps=64e-5, segments=0) -> Opts:
+    o = Opts()
+    load().wkv7_opts_default(ctypes.byref(o))
+    o.algo = ALGOS[algo] if isinstance(algo, str) else int(algo)
+    o.chunk = int(chunk)
+    o.snap_every = int(snap_every)
+    o.snapshots = None if snapshots is None else snapshots.data_ptr()
+    o.ln_w = None if ln_w is None else ln_w.data_ptr()
+    o.ln_b = None if ln_b is None else ln_b.data_ptr()
+    o.r_k = None if r_k is None else r_k.data_ptr()
+    o.gn_eps = float(gn_eps)
+    o.segments = int(segments)
+    return o
+
+
+def workspace_bytes(B, T, H, N=HEAD_SIZE, dtype=torch.bfloat16, **opt_kw) -> int:
+    return int(load().wkv7_workspace_bytes(B, T, H, N, BF16 if dtype == torch.bfloat16 else F32,
+                                           ctypes.byref(make_opts(**opt_kw))))
+
+
+def forward(r, w, k, v, kk, a, S0=None, *, algo="auto", chunk=0, snap_every=0, ln_w=None, ln_b=None,
+            r_k=None, gn_eps=64e-5, segments=0, y=None, S_T=None, snapshots=None, workspace=None,
+            return_state=True, stream=None, out_host=None):
+    """WKV-7 forward over [B, T, H, 64] inputs (bf16 or fp32, all the same dtype).
+
+    Returns (y, S_T, snapshots): y [B, T, H, 64] fp32, S_T [B, H, 64, 64] fp32
+    (None if return_state is False), snapshots [B, T//snap_every, H, 64, 64] or None.
+    Output tensors may be passed in (y=, S_T=, snapshots=) to avoid allocation; S_T
+    may be S0 for an in-place hand-off. CPU inputs run the end-to-end path (pinned
+    host tensors make its copies asynchronous; ``out_host=(y_host, S_host)`` names
+    pinned destinations for the results).
+    """
+    if r.device.type == "cpu":
+        return _forward_host(r, w, k, v, kk, a, S0, algo=algo, chunk=chunk, snap_every=snap_every,
+                             ln_w=ln_w, ln_b=ln_b, r_k=r_k, gn_eps=gn_eps, segments=segments,
+                             return_state=return_state, out_host=out_host)
+    lib = load()
+    B, T, H, N = r.shape
+    dev = r.device
+    if y is None:
+        y = torch.empty((B, T, H, N), device=dev, dtype=torch.float32)
+    if S_T is None and return_state:
+        S_T = torch.empty((B, H, N, N), device=dev, dtype=torch.float32)
+    n_snap = T // snap_every if snap_every else 0
+    if snapshots is None and n_snap:
+        snapshots = torch.empty((B, n_snap, H, N, N), device=dev, dtype=torch.float32)
+    opts = make_opts(algo, chunk, snap_every, snapshots, ln_w, ln_b, r_k, gn_eps, segments)
+    need = int(lib.wkv7_workspace_bytes(B, T, H, N, _dt(r), ctypes.byref(opts)))
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = lib.wkv7_forward(B, T, H, N, _dt(r), _ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(kk), _ptr(a),
+                              _ptr(S0), _ptr(y), _ptr(S_T), ctypes.byref(opts), _ptr(workspace),
+                              ws_bytes, _stream_handle(dev, stream))
+    _check(st, "wkv7_forward")
+    return y, S_T, snapshots
+
+
+def decode_step(r, w, k, v, kk, a, S, *, y=None, stream=None):
+    """One decode step; inputs [B, H, 64]; S [B, H, 64, 64] fp32 updated in place. Returns y."""
+    lib = load()
+    B, H, N = r.shape
+    if y is None:
+        y = torch.empty((B, H, N), device=r.device, dtype=torch.float32)
+    with torch.cuda.device(r.device):
+        st = lib.wkv7_decode_step(B, H, N, _dt(r), _ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(kk), _ptr(a),
+                                  _ptr(S), _ptr(y), _stream_handle(r.device, stream))
+    _check(st, "wkv7_decode_step")
+    return y
+
+
+def _forward_host(r, w, k, v, kk, a, S0, *, return_state, out_host, **kw):
+    """End-to-end path for host tensors: H2D copies, the kernels, D2H copies, all on
+    the current stream, which is synchronised before returning."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    to = lambda t: None if t is None else t.to(dev, non_blocking=True)
+    ep = {n: to(kw.pop(n)) for n in ("ln_w", "ln_b", "r_k")}
+    y, S_T, snaps = forward(*(to(t) for t in (r, w, k, v, kk, a)), to(S0), return_state=return_state,
+                            **ep, **kw)
+    y_h, S_h = out_host if out_host is not None else (None, None)
+    y_h = y.to("cpu") if y_h is None else y_h.copy_(y, non_blocking=True)
+    if S_T is not None:
+        S_h = S_T.to("cpu") if S_h is None else S_h.copy_(S_T, non_blocking=True)
+    sn_h = None if snaps is None else snaps.to("cpu")
+    stream.synchronize()
+    return y_h, S_h, sn_h

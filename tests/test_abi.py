@@ -1,0 +1,116 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol that
+include/wkv7.h declares, and rejects bad arguments on the host before any CUDA
+call (these calls return before touching the device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_rnn_sequence_rwkv_b200 import build, wkv7
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return wkv7.load()
+
+
+def _declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"WKV7_API\s+[\w\s\*]*?\b(wkv7_\w+)\s*\(", text))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared_symbols()
+    assert {"wkv7_forward", "wkv7_decode_step", "wkv7_workspace_bytes"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+    assert set(wkv7.EXPORTED) <= declared
+
+
+def test_abi_version_and_strings(lib):
+    assert lib.wkv7_abi_version() == 1
+    assert lib.wkv7_status_string(0) == b"WKV7_OK"
+    assert lib.wkv7_status_string(3) == b"WKV7_ERR_ALIGN"
+    assert lib.wkv7_status_string(99) == b"WKV7_ERR_UNKNOWN"
+    o = wkv7.Opts()
+    lib.wkv7_opts_default(ctypes.byref(o))
+    assert o.algo == 0 and o.chunk == 0 and o.snap_every == 0 and abs(o.gn_eps - 64e-5) < 1e-9
+
+
+FAKE = 0x10000   # 16-byte aligned, never dereferenced: validation fails first
+
+
+def _fwd(lib, B=1, T=4, H=1, N=64, dt=1, ptrs=None, opts=None, ws=None, ws_bytes=0):
+    p = ptrs or {}
+    get = lambda n, d=FAKE: ctypes.c_void_p(p.get(n, d)) if p.get(n, d) is not None else None
+    return lib.wkv7_forward(B, T, H, N, dt, *(get(n) for n in ("r", "w", "k", "v", "kk", "a")),
+                            get("S0", None), get("y"), get("S_T", None),
+                            ctypes.byref(opts) if opts else None, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(N=63), wkv7.ERR_UNSUPPORTED),
+    (dict(N=128), wkv7.ERR_UNSUPPORTED),
+    (dict(N=0), wkv7.ERR_ARG),
+    (dict(B=0), wkv7.ERR_ARG),
+    (dict(H=-1), wkv7.ERR_ARG),
+    (dict(T=-1), wkv7.ERR_ARG),
+    (dict(dt=7), wkv7.ERR_ARG),
+    (dict(ptrs={"kk": None}), wkv7.ERR_ARG),
+    (dict(ptrs={"y": None}), wkv7.ERR_ARG),
+    (dict(ptrs={"r": FAKE + 8}), wkv7.ERR_ALIGN),
+    (dict(ptrs={"S0": FAKE + 4}), wkv7.ERR_ALIGN),
+    (dict(B=1 << 30, T=1 << 30, H=1 << 30), wkv7.ERR_ARG),
+])
+def test_forward_rejects_bad_arguments(lib, kw, status):
+    assert _fwd(lib, **kw) == status
+    assert lib.wkv7_last_error() != b""
+
+
+@pytest.mark.parametrize("field,value", [("algo", 9), ("chunk", 24), ("snap_every", -1), ("segments", -2)])
+def test_forward_rejects_bad_options(lib, field, value):
+    o = wkv7.Opts()
+    lib.wkv7_opts_default(ctypes.byref(o))
+    setattr(o, field, value)
+    assert _fwd(lib, opts=o) == wkv7.ERR_ARG
+
+
+def test_forward_rejects_partial_epilogue_and_missing_snapshots(lib):
+    o = wkv7.Opts()
+    lib.wkv7_opts_default(ctypes.byref(o))
+    o.ln_w = FAKE
+    assert _fwd(lib, opts=o) == wkv7.ERR_ARG
+    lib.wkv7_opts_default(ctypes.byref(o))
+    o.snap_every = 2
+    assert _fwd(lib, opts=o) == wkv7.ERR_ARG
+
+
+def test_forward_rejects_overlapping_outputs(lib):
+    # y overlapping an input is caught on the host (pure address arithmetic)
+    assert _fwd(lib, ptrs={"y": FAKE}) == wkv7.ERR_ARG
+    assert b"overlap" in lib.wkv7_last_error()
+
+
+def test_decode_rejects_bad_arguments(lib):
+    P = lambda x: ctypes.c_void_p(x) if x is not None else None
+    args = [P(FAKE + 0x1000 * i) for i in range(8)]
+    assert lib.wkv7_decode_step(1, 1, 32, 1, *args, None) == wkv7.ERR_UNSUPPORTED
+    assert lib.wkv7_decode_step(0, 1, 64, 1, *args, None) == wkv7.ERR_ARG
+    bad = list(args)
+    bad[3] = None
+    assert lib.wkv7_decode_step(1, 1, 64, 1, *bad, None) == wkv7.ERR_ARG
+    bad = list(args)
+    bad[6] = P(FAKE + 0x6000 + 4)
+    assert lib.wkv7_decode_step(1, 1, 64, 1, *bad, None) == wkv7.ERR_ALIGN
+
+
+def test_workspace_query_is_host_only(lib):
+    assert wkv7.workspace_bytes(2, 128, 4) >= 0
