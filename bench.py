@@ -207,7 +207,7 @@ def run_gpu(args, world, rank, local):
                          snap_every=snap_every, snapshots=snaps, workspace=ws, **ep)
         bytes_per_launch = algorithmic_bytes(wl, B, T, H, 2, sets[0]["S0"] is not None, True,
                                              T // snap_every if snap_every else 0, epilogue)
-        launches_per_step = 1 + (1 if epilogue and args.algo in ("seq",) else 0)
+        launches_per_step = 1 + (1 if epilogue and _path_name(args) == "seq" else 0)
 
     units_per_step = B * T * H
 
@@ -249,7 +249,7 @@ def run_gpu(args, world, rank, local):
     else:
         roof = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved_gbs / hbm_peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
-                "traffic": None, "kernel": "decode_kernel" if decode else path,
+                "traffic": None, "kernel": "decode_kernel" if decode else "chunk_kernel",
                 "recurrence_tflops": round(flops_per_launch / (launch_ms * 1e-3) / 1e12, 3)}
     roof["algorithmic_bytes_per_launch"] = bytes_per_launch
 
@@ -280,8 +280,8 @@ def run_gpu(args, world, rank, local):
 
 
 def _path_name(args):
-    from linear_rnn_sequence_rwkv_b200 import wkv7  # noqa: F401
-    return {"auto": "seq", "seq": "seq"}.get(args.algo, args.algo)
+    """Kernel the library dispatches to for the bf16 workloads (AUTO picks the chunked one)."""
+    return {"auto": "chunk", "seq": "seq", "chunk": "chunk", "split": "chunk"}[args.algo]
 
 
 def run_e2e(args, wl, dev, stream, B, T, H, N, seed, epilogue, snap_every, warmup, steps, world):

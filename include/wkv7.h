@@ -61,7 +61,7 @@ typedef enum wkv7_status {
     WKV7_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement (N != 64) */
     WKV7_ERR_ALIGN = 3,        /* a pointer is not 16-byte aligned                       */
     WKV7_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed                    */
-    WKV7_ERR_TIMEOUT = 5,      /* reserved: a bounded device-side wait gave up           */
+    WKV7_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up (see poll below)    */
     WKV7_ERR_WORKSPACE = 6     /* workspace missing or smaller than wkv7_workspace_bytes */
 } wkv7_status;
 
@@ -73,7 +73,8 @@ typedef enum wkv7_dtype {
 typedef enum wkv7_algo {
     WKV7_ALGO_AUTO = 0,   /* pick from dtype, T and B*H                                  */
     WKV7_ALGO_SEQ = 1,    /* token-by-token scan, fp32 FMA; any T, any dtype             */
-    WKV7_ALGO_CHUNK = 2,  /* chunked prefill on tcgen05 tensor cores, fp32 chunk carry   */
+    WKV7_ALGO_CHUNK = 2,  /* chunked prefill on tcgen05 tensor cores, fp32 chunk carry;  */
+                          /* bf16 inputs, chunk 64, w >= exp(-e^-1/2) as on the pages      */
     WKV7_ALGO_SPLIT = 3   /* chunked prefill with T split into segments across CTAs      */
 } wkv7_algo;
 
@@ -130,6 +131,14 @@ WKV7_API wkv7_status wkv7_decode_step(int B, int H, int N, wkv7_dtype dt,
                              const void *r, const void *w, const void *k, const void *v,
                              const void *kk, const void *a,
                              float *S, float *y, void *stream);
+
+/*
+ * Synchronises `stream`, then reports whether a kernel of this library gave up one
+ * of its bounded device-side waits since the last call (WKV7_ERR_TIMEOUT; the
+ * affected outputs are then incomplete) and clears the flag. Kernels never trap or
+ * spin forever: a wait that exceeds its limit (2 s) records the error and returns.
+ */
+WKV7_API wkv7_status wkv7_poll_device_error(void *stream);
 
 /* Bytes of device workspace wkv7_forward needs for these arguments (opts may be NULL). */
 WKV7_API size_t wkv7_workspace_bytes(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opts *opts);

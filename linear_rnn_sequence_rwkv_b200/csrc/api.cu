@@ -223,12 +223,36 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype dt, const void *
         e = wkv7::launch_copy_state(p);
         return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "state copy launch");
     }
+    const bool chunk_ok = wkv7::chunk_supported(p) && (opts.chunk == 0 || opts.chunk == 64);
+    bool use_chunk = false;
+    if (opts.algo == WKV7_ALGO_CHUNK || opts.algo == WKV7_ALGO_SPLIT) {
+        if (!chunk_ok)
+            return fail(WKV7_ERR_UNSUPPORTED,
+                        "chunked algorithm needs bf16 inputs, chunk 0 or 64 and snap_every a multiple of 64");
+        use_chunk = true;
+    } else if (opts.algo == WKV7_ALGO_AUTO) {
+        use_chunk = chunk_ok && T >= 16;
+    }
+    if (use_chunk) {
+        e = wkv7::launch_chunk(p);
+        if (e != cudaSuccess) return cuda_fail(e, "chunked-prefill launch");
+        return WKV7_OK;
+    }
     e = wkv7::launch_seq(p);
     if (e != cudaSuccess) return cuda_fail(e, "sequential-scan launch");
     if (n_epi == 3) {
         e = wkv7::launch_epilogue(p);
         if (e != cudaSuccess) return cuda_fail(e, "epilogue launch");
     }
+    return WKV7_OK;
+}
+
+wkv7_status wkv7_poll_device_error(void *stream) {
+    g_err[0] = '\0';
+    unsigned int v = 0;
+    const cudaError_t e = wkv7::read_device_error(static_cast<cudaStream_t>(stream), &v, true);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+    if (v) return fail(WKV7_ERR_TIMEOUT, "a bounded device-side wait gave up (code %u)", v);
     return WKV7_OK;
 }
 

@@ -1,0 +1,704 @@
+// Chunked WKV-7 prefill on tcgen05 tensor cores (tf32 operands, fp32 accumulation),
+// with the state carried from chunk to chunk in fp32.
+//
+// The recurrence (RWKV-7 rebuttal page, numpy time_mixing listing, update and
+// readout lines; the paper summary, section 4: the transition stays "diagonal plus
+// rank one", which keeps the model parallelisable over time) is, per (b, h),
+//     S_t = S_{t-1} diag(w_t) + u_t b_t^T + v_t k_t^T,  u_t = -S_{t-1} kk_t,  b_t = kk_t*a_t,
+//     y_t = S_t r_t.
+// Over a chunk of C tokens with start state S_0, let g_t = prod_{s<=t} w_s (per key
+// channel, g_{-1} = 1) and gC = g_{C-1}. Unrolling gives (rows of the C x N matrices
+// are tokens; the derivation is this file's own, the pages give no chunk formula):
+//     KKd = kk*g_{t-1}, Rd = r*g_t, Bi = b/g_s, Ki = k/g_s, Bc = b*gC/g_s, Kc = k*gC/g_s
+//     M_ab = tril(KKd Bi^T, -1), M_kb = tril(KKd Ki^T, -1), Q_b = tril(Rd Bi^T), Q_k = tril(Rd Ki^T)
+//     A = (I + M_ab)^{-1}                              (the removed values U = A(-KKd S_0^T - M_kb V))
+//     [Z] = [Bc^T; Q_b] A,   [X] = Z [KKd | M_kb]
+//     P  = diag(gC) - Bc^T A KKd      R~ = Rd  - Q_b A KKd
+//     K~ = Kc^T - Bc^T A M_kb         Q~ = Q_k - Q_b A M_kb
+//     [S_C^T; Y] = [P; R~] S_0^T + [K~; Q~] V
+// Only the last line depends on the state, so the chain from chunk to chunk is one
+// fused M=128 MMA; everything else is computed from the chunk's own inputs.
+//
+// Mapping onto one B200 SM (one CTA per SM, persistent over (b, h) heads):
+//  * TMA (no multicast) stages the six bf16 [64 x 64] input tiles of the next chunk
+//    (128-byte swizzle) while the current chunk is processed.
+//  * Every MMA is tcgen05.mma kind::tf32, M=128, with the A operand in tensor memory
+//    (lane = row) and the B operand in shared memory (K-major, 128-byte swizzle). Five
+//    MMA rounds per chunk: Grams, Z, X, then the two state rounds into one accumulator.
+//  * 256 threads = 8 warps. TMEM lanes 0-63 belong to warps 0,1,4,5 ("column group":
+//    a key channel j or a token t, by phase), lanes 64-127 to warps 2,3,6,7 ("row
+//    group": a token t); the two warps sharing a lane quarter split the 64 columns.
+//  * The unit-lower-triangular inverse is done in fp32 on the CUDA cores: 16x16
+//    diagonal blocks by warp-shuffle substitution, then two levels of block merges.
+//  * Operands are rounded to tf32 (round to nearest) before the tensor core sees them;
+//    the carried state, the accumulators and all element-wise work stay fp32.
+// Every wait is bounded; a wait that gives up sets the device error word, the CTA
+// drains what it issued (bounded), frees its tensor memory and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "tc_util.cuh"
+
+namespace wkv7 {
+
+__device__ unsigned int g_device_error;   // non-zero: a bounded wait in a kernel gave up
+
+namespace {
+
+using namespace tc;
+
+constexpr int C = 64;             // chunk length (tokens)
+constexpr int kThreads = 256;
+constexpr int GTS = 68;           // row stride (floats) of the decay table: conflict-free row reads
+constexpr int LWS = 65;           // row stride of the inverse workspaces
+
+// Shared-memory layout (byte offsets from a 1024-byte aligned base).
+constexpr uint32_t OFF_B1 = 0;        // [Bi; Ki] 128x64 tf32 (R1 B operand); later the inverse workspace
+constexpr uint32_t OFF_B3 = 32768;    // [KKd^T | M_kb^T] 128x64 (R3 B operand)
+constexpr uint32_t OFF_B2 = 65536;    // A^T 64x64 (R2 B operand)
+constexpr uint32_t OFF_B4 = 81920;    // V^T 64x64 (R4 B operand; exact bf16 values)
+constexpr uint32_t OFF_B5 = 98304;    // S 64x64, row = value channel (R5 B operand)
+constexpr uint32_t OFF_IN = 114688;   // six bf16 [64][64] input tiles, TMA destination (swizzled)
+constexpr uint32_t OFF_GT = 163840;   // decay table [65][GTS] fp32; later the inverse [64][LWS]
+constexpr uint32_t OFF_SMALL = OFF_GT + 65 * GTS * 4;
+
+struct Small {
+    float gC[C];
+    float tot[2][C];
+    float bon[2][C];
+    float dk[2][C];       // r_t . k_t, partial over each column half (exact current-token Gram entry)
+    float db[2][C];       // r_t . (kk_t * a_t)
+    float red[2][C];
+    float ln_w[C], ln_b[C], r_k[C];
+    uint64_t bar_tma;
+    uint64_t bar_mma;
+    uint32_t tmem_base;
+};
+constexpr uint32_t SMEM_BYTES = OFF_SMALL + sizeof(Small) + 1024;   // + alignment slack
+
+// TMEM columns (512 allocated).
+constexpr uint32_t T_A1 = 0;     // [KKd; Rd]
+constexpr uint32_t T_D1 = 64;    // Grams [M_ab | M_kb ; Q_b | Q_k] -> cols 0-63 become [Bc^T; Q_b]
+constexpr uint32_t T_D2 = 192;   // Z
+constexpr uint32_t T_D3 = 256;   // X -> [P; R~] (cols 0-63) and [K~; Q~] (cols 64-127)
+constexpr uint32_t T_D4 = 384;   // [S_C^T; Y]
+constexpr uint32_t T_KC = 448;   // Kc^T (lanes 0-63)
+
+enum { XR = 0, XW = 1, XK = 2, XV = 3, XKK = 4, XA = 5 };
+
+struct ChunkMaps {
+    CUtensorMap m[6];
+};
+
+struct ChunkArgs {
+    int B, T, H;
+    const float *S0;
+    float *y, *S_T, *snaps;
+    int snap_every, n_snap;
+    const float *ln_w, *ln_b, *r_k;
+    float gn_eps;
+    unsigned int *err;
+    unsigned long long timeout_ns;
+};
+
+// bf16 element (t, j) of a 128-byte-swizzled [64][64] tile.
+__device__ __forceinline__ float in_elem(const uint8_t *tile, int t, int j) {
+    const uint32_t off = t * 128 + ((((j >> 3) ^ (t & 7))) << 4) + ((j & 7) << 1);
+    return __uint_as_float(uint32_t(*reinterpret_cast<const uint16_t *>(tile + off)) << 16);
+}
+// Eight bf16 elements (t, j..j+7), j a multiple of 8.
+__device__ __forceinline__ void in_row8(const uint8_t *tile, int t, int j, float (&o)[8]) {
+    const uint32_t off = t * 128 + ((((j >> 3) ^ (t & 7))) << 4);
+    const uint4 u = *reinterpret_cast<const uint4 *>(tile + off);
+    o[0] = bf16_lo(u.x); o[1] = bf16_hi(u.x); o[2] = bf16_lo(u.y); o[3] = bf16_hi(u.y);
+    o[4] = bf16_lo(u.z); o[5] = bf16_hi(u.z); o[6] = bf16_lo(u.w); o[7] = bf16_hi(u.w);
+}
+__device__ __forceinline__ void st_f4(uint8_t *base, uint32_t off, float a, float b, float c, float d) {
+    *reinterpret_cast<float4 *>(base + off) = make_float4(a, b, c, d);
+}
+__device__ __forceinline__ void named_bar_rows() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constant__ ChunkMaps maps, const ChunkArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
+    Small &S = *reinterpret_cast<Small *>(sm + OFF_SMALL);
+    const uint8_t *IN = sm + OFF_IN;
+    float *GT = reinterpret_cast<float *>(sm + OFF_GT);
+    float *Lw = reinterpret_cast<float *>(sm + OFF_B1);      // strictly lower M_ab [64][LWS]
+    float *Tw = Lw + 64 * LWS;                               // level-1 temps [2][16][17]
+    float *Tw2 = Tw + 2 * 16 * 17;                           // level-2 temp [32][33]
+    float *Aw = reinterpret_cast<float *>(sm + OFF_GT);      // inverse [64][LWS]
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int Lq = (warp & 3) * 32;         // first TMEM lane of this warp's quarter
+    const int L = Lq + lane;                // this thread's TMEM lane
+    const int h = tid >> 7;                 // which half of the 64 columns / tokens
+    const bool colg = L < 64;
+    const int units = p.B * p.H;
+    const int nchunks = (p.T + C - 1) / C;
+    const bool epi = p.ln_w != nullptr;
+
+    if (tid == 0) {
+        mbar_init(&S.bar_tma, 1);
+        mbar_init(&S.bar_mma, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&S.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = S.tmem_base;
+    // matrix descriptors of the shared-memory B operands at K-step 0
+    const uint64_t dB1 = desc_sw128(smem_u32(sm + OFF_B1)), dB2 = desc_sw128(smem_u32(sm + OFF_B2));
+    const uint64_t dB3 = desc_sw128(smem_u32(sm + OFF_B3)), dB4 = desc_sw128(smem_u32(sm + OFF_B4));
+    const uint64_t dB5 = desc_sw128(smem_u32(sm + OFF_B5));
+    uint32_t tma_parity = 0, mma_parity = 0;
+    bool tma_pending = false, mma_pending = false, failed = false;
+
+    auto issue_tma = [&](int u, int c) {   // thread 0
+        const int b = u / p.H, hh = u % p.H;
+        mbar_arrive_expect_tx(&S.bar_tma, 6 * 8192);
+#pragma unroll
+        for (int x = 0; x < 6; ++x) tma_load_4d(sm + OFF_IN + x * 8192, &maps.m[x], &S.bar_tma, 0, hh, c * C, b);
+    };
+    auto wait_mma = [&]() -> bool {        // all threads; true on timeout (uniform across the CTA)
+        const bool to = !mbar_wait(&S.bar_mma, mma_parity, p.timeout_ns);
+        mma_parity ^= 1u;
+        mma_pending = false;
+        tc_fence_after();
+        return __syncthreads_or(to) != 0;
+    };
+    auto sync_for_mma = [&]() {            // writes to smem/TMEM -> visible to the next MMA
+        fence_proxy_async_smem();
+        tmem_st_wait();
+        tc_fence_before();
+        __syncthreads();
+    };
+
+    int unit = blockIdx.x;
+    if (tid == 0 && unit < units) issue_tma(unit, 0);
+    tma_pending = unit < units;
+
+    for (; unit < units && !failed; unit += gridDim.x) {
+        const int b = unit / p.H, hh = unit % p.H;
+        // state operand S_0 (row = value channel i, K = key channel j), tf32-rounded
+        for (int e = tid; e < 1024; e += kThreads) {
+            const int i = e >> 4, j4 = (e & 15) * 4;
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (p.S0) x = __ldg(reinterpret_cast<const float4 *>(p.S0 + size_t(unit) * 4096 + i * 64 + j4));
+            st_f4(sm + OFF_B5, sw128_off(i, j4, 64), to_tf32(x.x), to_tf32(x.y), to_tf32(x.z), to_tf32(x.w));
+        }
+        if (epi && tid < 64) {
+            S.ln_w[tid] = p.ln_w[hh * 64 + tid];
+            S.ln_b[tid] = p.ln_b[hh * 64 + tid];
+            S.r_k[tid] = p.r_k[hh * 64 + tid];
+        }
+
+        for (int c = 0; c < nchunks; ++c) {
+            const int c0 = c * C, Lc = min(C, p.T - c0);
+            const bool last = c == nchunks - 1;
+            {   // ---- inputs of this chunk
+                const bool to = !mbar_wait(&S.bar_tma, tma_parity, p.timeout_ns);
+                tma_parity ^= 1u;
+                tma_pending = false;
+                if (__syncthreads_or(to)) { failed = true; break; }
+            }
+            // ---- S1: running decay products within each half of the chunk (column group, j = L)
+            if (colg) {
+                const uint8_t *wt = IN + XW * 8192;
+                float run = 1.f;
+#pragma unroll 8
+                for (int i = 0; i < 32; ++i) {
+                    const int t = 32 * h + i;
+                    run *= (t < Lc) ? in_elem(wt, t, L) : 1.f;   // padded tokens: w = 1
+                    GT[(t + 1) * GTS + L] = run;
+                }
+                S.tot[h][L] = run;
+                if (h == 0) GT[L] = 1.f;
+            }
+            __syncthreads();
+            // ---- S2: products of the second half made absolute; column outputs Kc^T (TMEM),
+            //      KKd^T (B3 rows 0-63), V^T (B4)
+            if (colg) {
+                const int j = L;
+                const float pre = h ? S.tot[0][j] : 1.f;
+                const float gCj = S.tot[0][j] * S.tot[1][j];
+                if (h == 0) S.gC[j] = gCj;
+                float gprev = pre;   // g_{t-1} of the first token of this half
+#pragma unroll 1
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    const int t0 = 32 * h + 8 * g8;
+                    float kc[8], kkd[8], vv[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int t = t0 + e;
+                        const float graw = GT[(t + 1) * GTS + j];
+                        const float gt = h ? pre * graw : graw;
+                        if (h) GT[(t + 1) * GTS + j] = gt;
+                        kc[e] = to_tf32(in_elem(IN + XK * 8192, t, j) * __fdividef(gCj, gt));
+                        kkd[e] = to_tf32(in_elem(IN + XKK * 8192, t, j) * gprev);
+                        vv[e] = in_elem(IN + XV * 8192, t, j);
+                        gprev = gt;
+                    }
+                    tmem_st8(tmem_addr(tb, Lq, T_KC + t0), kc);
+                    st_f4(sm + OFF_B3, sw128_off(j, t0, 128), kkd[0], kkd[1], kkd[2], kkd[3]);
+                    st_f4(sm + OFF_B3, sw128_off(j, t0 + 4, 128), kkd[4], kkd[5], kkd[6], kkd[7]);
+                    st_f4(sm + OFF_B4, sw128_off(j, t0, 64), vv[0], vv[1], vv[2], vv[3]);
+                    st_f4(sm + OFF_B4, sw128_off(j, t0 + 4, 64), vv[4], vv[5], vv[6], vv[7]);
+                }
+            }
+            __syncthreads();
+            // ---- S3: row outputs
+            if (colg) {                 // token t = L: KKd row -> A1 lanes 0..63
+                const int t = L;
+                const float *gp = GT + t * GTS;   // g_{t-1}
+#pragma unroll 1
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    const int j0 = 32 * h + 8 * g8;
+                    float kk8[8], v[8];
+                    in_row8(IN + XKK * 8192, t, j0, kk8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[e] = to_tf32(kk8[e] * gp[j0 + e]);
+                    tmem_st8(tmem_addr(tb, Lq, T_A1 + j0), v);
+                }
+            } else {                    // token t = L - 64: Rd row -> A1 lanes 64..127; Bi, Ki rows -> B1
+                const int t = L - 64;
+                const float *gt = GT + (t + 1) * GTS;   // g_t
+                float bon = 0.f, dk = 0.f, db = 0.f;
+#pragma unroll 1
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    const int j0 = 32 * h + 8 * g8;
+                    float r8[8], kk8[8], a8[8], k8[8], rd[8], bi[8], ki[8];
+                    in_row8(IN + XR * 8192, t, j0, r8);
+                    in_row8(IN + XKK * 8192, t, j0, kk8);
+                    in_row8(IN + XA * 8192, t, j0, a8);
+                    in_row8(IN + XK * 8192, t, j0, k8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float gv = gt[j0 + e];
+                        const float ig = __fdividef(1.f, gv);
+                        const float b = kk8[e] * a8[e];
+                        rd[e] = to_tf32(r8[e] * gv);
+                        bi[e] = to_tf32(b * ig);
+                        ki[e] = to_tf32(k8[e] * ig);
+                        dk = fmaf(r8[e], k8[e], dk);
+                        db = fmaf(r8[e], b, db);
+                        if (epi) bon = fmaf(r8[e] * k8[e], S.r_k[j0 + e], bon);
+                    }
+                    tmem_st8(tmem_addr(tb, Lq, T_A1 + j0), rd);
+                    st_f4(sm + OFF_B1, sw128_off(t, j0, 128), bi[0], bi[1], bi[2], bi[3]);
+                    st_f4(sm + OFF_B1, sw128_off(t, j0 + 4, 128), bi[4], bi[5], bi[6], bi[7]);
+                    st_f4(sm + OFF_B1, sw128_off(64 + t, j0, 128), ki[0], ki[1], ki[2], ki[3]);
+                    st_f4(sm + OFF_B1, sw128_off(64 + t, j0 + 4, 128), ki[4], ki[5], ki[6], ki[7]);
+                }
+                S.dk[h][t] = dk;
+                S.db[h][t] = db;
+                if (epi) S.bon[h][t] = bon;
+            }
+            sync_for_mma();
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)   // R1: Grams = [KKd; Rd] [Bi; Ki]^T
+                    mma_tf32_ts(tb + T_D1, tb + T_A1 + 8 * ks, dB1 + kstep_off(ks, 128),
+                                idesc_tf32(128, 128), ks > 0);
+                mma_commit(&S.bar_mma);
+            }
+            mma_pending = true;
+            if (wait_mma()) { failed = true; break; }
+            // ---- masks; M_ab -> inverse workspace; M_kb^T -> B3; A2 = [Bc^T; Q_b] in TMEM
+            if (colg) {
+                const int t = L, j = L;   // D1 row t (token) is read before lane j receives Bc^T row j
+                const float gCj = S.gC[j];
+#pragma unroll 1
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    const int s0 = 32 * h + 8 * g8;
+                    float m[8], bc[8];
+                    tmem_ld8(tmem_addr(tb, Lq, T_D1 + s0), m);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) Lw[t * LWS + s0 + e] = (s0 + e < t) ? m[e] : 0.f;
+                    tmem_ld8(tmem_addr(tb, Lq, T_D1 + 64 + s0), m);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        *reinterpret_cast<float *>(sm + OFF_B3 + sw128_off(64 + s0 + e, t, 128)) =
+                            (s0 + e < t) ? to_tf32(m[e]) : 0.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int ss = s0 + e;
+                        const float b = in_elem(IN + XKK * 8192, ss, j) * in_elem(IN + XA * 8192, ss, j);
+                        bc[e] = to_tf32(b * __fdividef(gCj, GT[(ss + 1) * GTS + j]));
+                    }
+                    tmem_st8(tmem_addr(tb, Lq, T_D1 + s0), bc);
+                }
+            } else {
+                const int t = L - 64;
+                // the current-token entry is taken exactly in fp32: it dominates short sequences
+                const float diag = S.db[0][t] + S.db[1][t];
+#pragma unroll 1
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    const int s0 = 32 * h + 8 * g8;
+                    float m[8];
+                    tmem_ld8(tmem_addr(tb, Lq, T_D1 + s0), m);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int ss = s0 + e;
+                        m[e] = ss < t ? to_tf32(m[e]) : (ss == t ? to_tf32(diag) : 0.f);
+                    }
+                    tmem_st8(tmem_addr(tb, Lq, T_D1 + s0), m);
+                }
+            }
+            sync_for_mma();
+            if (tid == 0) {
+                // input tiles and decay table are consumed: prefetch the next chunk (or next head)
+                if (!last) issue_tma(unit, c + 1);
+                else if (unit + int(gridDim.x) < units) issue_tma(unit + gridDim.x, 0);
+            }
+            tma_pending = !last || unit + int(gridDim.x) < units;
+            // ---- A = (I + M_ab)^{-1}. Diagonal 16x16 blocks: one thread per (block, column)
+            //      solves (I + L_dd) x = e_c by forward substitution in registers.
+            if (tid < 64) {
+                const int d = tid >> 4, cc = tid & 15;
+                const float *Lb = Lw + 16 * d * LWS + 16 * d;
+                float x[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    float acc = (r == cc) ? 1.f : 0.f;
+#pragma unroll
+                    for (int k = 0; k < r; ++k) acc = fmaf(-Lb[r * LWS + k], x[k], acc);
+                    x[r] = acc;
+                }
+#pragma unroll
+                for (int r = 0; r < 16; ++r) Aw[(16 * d + r) * LWS + 16 * d + cc] = x[r];
+            } else {
+                // zero the blocks above the diagonal: (bi, bj) with bi < bj
+#pragma unroll 1
+                for (int e = tid - 64; e < 6 * 256; e += kThreads - 64) {
+                    const int blk = e >> 8, o = e & 255;
+                    const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+                    const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+                    Aw[(16 * bi + (o >> 4)) * LWS + 16 * bj + (o & 15)] = 0.f;
+                }
+            }
+            __syncthreads();
+            // level 1: X[2p+1][2p] = -X[2p+1] (L[2p+1][2p] X[2p]),  p = 0, 1
+            for (int o = tid; o < 512; o += kThreads) {
+                const int pp = o >> 8, i = (o >> 4) & 15, jj = o & 15;
+                float acc = 0.f;
+#pragma unroll
+                for (int kq = 0; kq < 16; ++kq)
+                    acc = fmaf(Lw[(32 * pp + 16 + i) * LWS + 32 * pp + kq], Aw[(32 * pp + kq) * LWS + 32 * pp + jj], acc);
+                Tw[(pp * 16 + i) * 17 + jj] = acc;
+            }
+            __syncthreads();
+            for (int o = tid; o < 512; o += kThreads) {
+                const int pp = o >> 8, i = (o >> 4) & 15, jj = o & 15;
+                float acc = 0.f;
+#pragma unroll
+                for (int kq = 0; kq < 16; ++kq)
+                    acc = fmaf(Aw[(32 * pp + 16 + i) * LWS + 32 * pp + 16 + kq], Tw[(pp * 16 + kq) * 17 + jj], acc);
+                Aw[(32 * pp + 16 + i) * LWS + 32 * pp + jj] = -acc;
+            }
+            __syncthreads();
+            // level 2: Y[1][0] = -Y1 (L[32:64][0:32] Y0). Y0, Y1 are lower triangular, so the
+            // fixed-length sums are exact; each thread keeps four independent accumulators.
+            {
+                const int i = tid >> 3, jg = tid & 7;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+                for (int kq = 0; kq < 32; ++kq) {
+                    const float lv = Lw[(32 + i) * LWS + kq];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) acc[m] = fmaf(lv, Aw[kq * LWS + jg + 8 * m], acc[m]);
+                }
+#pragma unroll
+                for (int m = 0; m < 4; ++m) Tw2[i * 33 + jg + 8 * m] = acc[m];
+            }
+            __syncthreads();
+            {
+                const int i = tid >> 3, jg = tid & 7;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+                for (int kq = 0; kq < 32; ++kq) {
+                    const float av = Aw[(32 + i) * LWS + 32 + kq];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) acc[m] = fmaf(av, Tw2[kq * 33 + jg + 8 * m], acc[m]);
+                }
+#pragma unroll
+                for (int m = 0; m < 4; ++m) Aw[(32 + i) * LWS + jg + 8 * m] = -acc[m];
+            }
+            __syncthreads();
+            // B2 = A^T (row s, K = t)
+            for (int e = tid; e < 1024; e += kThreads) {
+                const int s = e & 63, t4 = (e >> 6) * 4;
+                st_f4(sm + OFF_B2, sw128_off(s, t4, 64), to_tf32(Aw[t4 * LWS + s]), to_tf32(Aw[(t4 + 1) * LWS + s]),
+                      to_tf32(Aw[(t4 + 2) * LWS + s]), to_tf32(Aw[(t4 + 3) * LWS + s]));
+            }
+            sync_for_mma();
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)   // R2: Z = [Bc^T; Q_b] A
+                    mma_tf32_ts(tb + T_D2, tb + T_D1 + 8 * ks, dB2 + kstep_off(ks, 64),
+                                idesc_tf32(128, 64), ks > 0);
+                mma_commit(&S.bar_mma);
+            }
+            mma_pending = true;
+            if (wait_mma()) { failed = true; break; }
+            // round Z to tf32 in place (it is the next A operand)
+#pragma unroll 1
+            for (int g8 = 0; g8 < 4; ++g8) {
+                float z[8];
+                tmem_ld8(tmem_addr(tb, Lq, T_D2 + 32 * h + 8 * g8), z);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) z[e] = to_tf32(z[e]);
+                tmem_st8(tmem_addr(tb, Lq, T_D2 + 32 * h + 8 * g8), z);
+            }
+            sync_for_mma();
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)   // R3: X = Z [KKd | M_kb]
+                    mma_tf32_ts(tb + T_D3, tb + T_D2 + 8 * ks, dB3 + kstep_off(ks, 128),
+                                idesc_tf32(128, 128), ks > 0);
+                mma_commit(&S.bar_mma);
+            }
+            mma_pending = true;
+            if (wait_mma()) { failed = true; break; }
+            // ---- P, K~ (column group, key j) and R~, Q~ (row group, token t), in place
+            if (colg) {
+                const int j = L;
+                const float gCj = S.gC[j];
+#pragma unroll 1
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    const int c8 = 32 * h + 8 * g8;
+                    float d[8], e8[8];
+                    tmem_ld8(tmem_addr(tb, Lq, T_D3 + c8), d);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) d[e] = to_tf32((c8 + e == j ? gCj : 0.f) - d[e]);
+                    tmem_st8(tmem_addr(tb, Lq, T_D3 + c8), d);
+                    tmem_ld8(tmem_addr(tb, Lq, T_D3 + 64 + c8), d);
+                    tmem_ld8(tmem_addr(tb, Lq, T_KC + c8), e8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) d[e] = to_tf32(e8[e] - d[e]);
+                    tmem_st8(tmem_addr(tb, Lq, T_D3 + 64 + c8), d);
+                }
+            } else {
+                const int t = L - 64;
+                const float diag = S.dk[0][t] + S.dk[1][t];
+#pragma unroll 1
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    const int c8 = 32 * h + 8 * g8;
+                    float d[8], e8[8];
+                    tmem_ld8(tmem_addr(tb, Lq, T_D3 + c8), d);
+                    tmem_ld8(tmem_addr(tb, Lq, T_A1 + c8), e8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) d[e] = to_tf32(e8[e] - d[e]);
+                    tmem_st8(tmem_addr(tb, Lq, T_D3 + c8), d);
+                    tmem_ld8(tmem_addr(tb, Lq, T_D3 + 64 + c8), d);
+                    tmem_ld8(tmem_addr(tb, Lq, T_D1 + 64 + c8), e8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int ss = c8 + e;
+                        d[e] = to_tf32((ss < t ? e8[e] : (ss == t ? diag : 0.f)) - d[e]);
+                    }
+                    tmem_st8(tmem_addr(tb, Lq, T_D3 + 64 + c8), d);
+                }
+            }
+            sync_for_mma();
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)   // R4: [K~; Q~] V
+                    mma_tf32_ts(tb + T_D4, tb + T_D3 + 64 + 8 * ks, dB4 + kstep_off(ks, 64),
+                                idesc_tf32(128, 64), ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)   // R5: += [P; R~] S_0^T
+                    mma_tf32_ts(tb + T_D4, tb + T_D3 + 8 * ks, dB5 + kstep_off(ks, 64),
+                                idesc_tf32(128, 64), 1);
+                mma_commit(&S.bar_mma);
+            }
+            mma_pending = true;
+            if (wait_mma()) { failed = true; break; }
+            // ---- new state -> B5 (+ S_T / snapshot); readout -> epilogue -> y
+            const int done = c0 + Lc;
+            const bool snap = p.snap_every > 0 && done % p.snap_every == 0;
+            if (colg) {
+                const int j = L;
+#pragma unroll 1
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    const int i0 = 32 * h + 8 * g8;
+                    float s8[8];
+                    tmem_ld8(tmem_addr(tb, Lq, T_D4 + i0), s8);    // S[i0+e][j]
+                    if (last && p.S_T) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) p.S_T[size_t(unit) * 4096 + (i0 + e) * 64 + j] = s8[e];
+                    }
+                    if (snap) {
+                        float *dst = p.snaps + ((size_t(b) * p.n_snap + (done / p.snap_every - 1)) * p.H + hh) * 4096;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) dst[(i0 + e) * 64 + j] = s8[e];
+                    }
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        *reinterpret_cast<float *>(sm + OFF_B5 + sw128_off(i0 + e, j, 64)) = to_tf32(s8[e]);
+                }
+            } else {
+                const int t = L - 64;
+                float *dst = p.y + ((size_t(b) * p.T + c0 + t) * p.H + hh) * 64 + 32 * h;
+                float mean = 0.f, inv = 1.f, bon = 0.f;
+                if (epi) {
+                    float s1 = 0.f, s2 = 0.f;
+#pragma unroll 1
+                    for (int g8 = 0; g8 < 4; ++g8) {
+                        float y8[8];
+                        tmem_ld8(tmem_addr(tb, Lq, T_D4 + 32 * h + 8 * g8), y8);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) s1 += y8[e];
+                    }
+                    S.red[h][t] = s1;
+                    named_bar_rows();
+                    mean = (S.red[0][t] + S.red[1][t]) * (1.f / 64.f);
+                    named_bar_rows();
+#pragma unroll 1
+                    for (int g8 = 0; g8 < 4; ++g8) {
+                        float y8[8];
+                        tmem_ld8(tmem_addr(tb, Lq, T_D4 + 32 * h + 8 * g8), y8);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) s2 = fmaf(y8[e] - mean, y8[e] - mean, s2);
+                    }
+                    S.red[h][t] = s2;
+                    named_bar_rows();
+                    inv = 1.f / sqrtf((S.red[0][t] + S.red[1][t]) * (1.f / 64.f) + p.gn_eps);
+                    bon = S.bon[0][t] + S.bon[1][t];
+                }
+#pragma unroll 1
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    const int i0 = 32 * h + 8 * g8;
+                    float y8[8];
+                    tmem_ld8(tmem_addr(tb, Lq, T_D4 + i0), y8);   // y_t[i0 + e]
+                    if (epi) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float v = *reinterpret_cast<const float *>(sm + OFF_B4 + sw128_off(i0 + e, t, 64));
+                            y8[e] = fmaf((y8[e] - mean) * inv, S.ln_w[i0 + e], S.ln_b[i0 + e]) + bon * v;
+                        }
+                    }
+                    if (t < Lc) {
+                        *reinterpret_cast<float4 *>(dst + 8 * g8) = make_float4(y8[0], y8[1], y8[2], y8[3]);
+                        *reinterpret_cast<float4 *>(dst + 8 * g8 + 4) = make_float4(y8[4], y8[5], y8[6], y8[7]);
+                    }
+                }
+            }
+            sync_for_mma();
+        }
+    }
+
+    if (failed) {
+        if (tid == 0) atomicOr(p.err, 1u);
+        // drain what this CTA issued (bounded), then release tensor memory
+        if (mma_pending) mbar_wait(&S.bar_mma, mma_parity, p.timeout_ns);
+        if (tma_pending) mbar_wait(&S.bar_tma, tma_parity, p.timeout_ns);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tb, 512);
+}
+
+// ---- host side ---------------------------------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+struct DeviceInfo {
+    int sms = 0;
+    unsigned int *err = nullptr;
+    bool attr_set = false;
+};
+
+cudaError_t device_info(DeviceInfo *&out) {
+    static std::mutex mu;
+    static DeviceInfo info[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(mu);
+    DeviceInfo &d = info[dev];
+    if (!d.attr_set) {
+        if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_device_error)) != cudaSuccess) return e;
+        if ((e = cudaFuncSetAttribute(chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_BYTES))) !=
+            cudaSuccess)
+            return e;
+        d.attr_set = true;
+    }
+    out = &d;
+    return cudaSuccess;
+}
+
+}  // namespace
+
+bool chunk_supported(const FwdArgs &p) {
+    return p.dt == WKV7_BF16 && (p.snap_every == 0 || p.snap_every % C == 0);
+}
+
+cudaError_t launch_chunk(const FwdArgs &p) {
+    auto enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    DeviceInfo *di = nullptr;
+    cudaError_t e = device_info(di);
+    if (e != cudaSuccess) return e;
+    ChunkMaps maps;
+    const void *src[6] = {p.r, p.w, p.k, p.v, p.kk, p.a};
+    const cuuint64_t dims[4] = {cuuint64_t(kN), cuuint64_t(p.H), cuuint64_t(p.T), cuuint64_t(p.B)};
+    const cuuint64_t strides[3] = {cuuint64_t(kN) * 2, cuuint64_t(p.H) * kN * 2, cuuint64_t(p.T) * p.H * kN * 2};
+    const cuuint32_t box[4] = {cuuint32_t(kN), 1, cuuint32_t(C), 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    for (int x = 0; x < 6; ++x) {
+        const CUresult r = enc(&maps.m[x], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(src[x]), dims,
+                               strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
+    ChunkArgs a{};
+    a.B = p.B; a.T = p.T; a.H = p.H;
+    a.S0 = p.S0; a.y = p.y; a.S_T = p.S_T; a.snaps = p.snaps;
+    a.snap_every = p.snap_every;
+    a.n_snap = p.snap_every > 0 ? p.T / p.snap_every : 0;
+    a.ln_w = p.ln_w; a.ln_b = p.ln_b; a.r_k = p.r_k; a.gn_eps = p.gn_eps;
+    a.err = di->err;
+    a.timeout_ns = 2000000000ull;
+    const int units = p.B * p.H;
+    const int grid = units < di->sms ? units : di->sms;
+    chunk_kernel<<<grid, kThreads, SMEM_BYTES, p.stream>>>(maps, a);
+    return cudaGetLastError();
+}
+
+cudaError_t read_device_error(cudaStream_t stream, unsigned int *value, bool clear) {
+    DeviceInfo *di = nullptr;
+    cudaError_t e = device_info(di);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaStreamSynchronize(stream)) != cudaSuccess) return e;
+    if ((e = cudaMemcpy(value, di->err, sizeof(unsigned int), cudaMemcpyDeviceToHost)) != cudaSuccess) return e;
+    if (clear && *value) e = cudaMemset(di->err, 0, sizeof(unsigned int));
+    return e;
+}
+
+}  // namespace wkv7

@@ -28,7 +28,7 @@ F32, BF16 = 0, 1
 ALGOS = {"auto": 0, "seq": 1, "chunk": 2, "split": 3}
 
 EXPORTED = ("wkv7_opts_default", "wkv7_forward", "wkv7_decode_step", "wkv7_workspace_bytes",
-            "wkv7_status_string", "wkv7_last_error", "wkv7_abi_version")
+            "wkv7_status_string", "wkv7_last_error", "wkv7_abi_version", "wkv7_poll_device_error")
 
 
 class Wkv7Error(RuntimeError):
@@ -77,6 +77,8 @@ def load():
         lib.wkv7_last_error.restype = ctypes.c_char_p
         lib.wkv7_abi_version.argtypes = []
         lib.wkv7_abi_version.restype = ci
+        lib.wkv7_poll_device_error.argtypes = [vp]
+        lib.wkv7_poll_device_error.restype = ci
         _lib = lib
         return lib
 
@@ -176,6 +178,13 @@ def decode_step(r, w, k, v, kk, a, S, *, y=None, stream=None):
                                   _ptr(S), _ptr(y), _stream_handle(r.device, stream))
     _check(st, "wkv7_decode_step")
     return y
+
+
+def poll_device_error(stream=None):
+    """Synchronise the stream and raise Wkv7Error(ERR_TIMEOUT) if a kernel gave up a
+    bounded device-side wait since the last poll."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _check(load().wkv7_poll_device_error(_stream_handle(dev, stream)), "wkv7_poll_device_error")
 
 
 def _forward_host(r, w, k, v, kk, a, S0, *, return_state, out_host, **kw):

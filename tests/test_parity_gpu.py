@@ -12,7 +12,7 @@ from tests.parity_util import TOL, as_np, heads_slice, snaps_err, state_err, y_e
 
 pytestmark = pytest.mark.gpu
 
-ALGOS_ANY = ["seq"]
+ALGOS_ANY = ["seq", "chunk"]      # algorithms that accept bf16 inputs
 
 
 def _dev(d, device):
@@ -27,7 +27,7 @@ def _gpu(dd, **kw):
     return wkv7.forward(dd["r"], dd["w"], dd["k"], dd["v"], dd["kk"], dd["a"], dd.get("S0"), **kw)
 
 
-@pytest.mark.parametrize("algo", ALGOS_ANY)
+@pytest.mark.parametrize("algo", ["seq", "auto"])
 def test_tiny_fp32_workload(cuda_device, algo):
     """Tiny oracle check (B1 T64 H2, fp32 in/out, S0 = 0): error <= 1e-5."""
     wl = inputs.WORKLOADS[0]
@@ -43,6 +43,8 @@ def test_tiny_fp32_workload(cuda_device, algo):
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_ragged_lengths(cuda_device, algo, T, dtype):
     """Lengths that are not multiples of any tile, with a carried-in state."""
+    if dtype == "f32" and algo == "chunk":
+        pytest.skip("the chunked algorithm takes bf16 inputs")
     wl = inputs.WORKLOADS[1]
     d = inputs.make_inputs(wl, B=2, T=T, H=3, dtype=dtype, seed=1000 + T)
     y_ref, S_ref, _ = _oracle(d)
@@ -89,8 +91,11 @@ def test_state_handoff_split(cuda_device, algo, T1):
     y_ref, S_ref, _ = _oracle({k: v.cpu() if v is not None else None for k, v in d.items()})
     assert y_err(torch.cat([y1, y2], dim=1), y_ref) <= TOL["bf16"]
     assert state_err(S2, S_ref) <= TOL["bf16"]
-    assert y_err(torch.cat([y1, y2], dim=1), y) <= 1e-5
-    assert state_err(S2, S) <= 1e-5
+    # the fp32 scan is reproducible to rounding; the chunked path moves its chunk
+    # boundaries with the split, so the two runs differ at tf32 operand rounding
+    self_tol = 1e-5 if algo == "seq" else TOL["bf16"]
+    assert y_err(torch.cat([y1, y2], dim=1), y) <= self_tol
+    assert state_err(S2, S) <= self_tol
 
 
 def test_in_place_state_handoff(cuda_device):
@@ -259,3 +264,56 @@ def test_long_context_sampled_heads(cuda_device, algo):
     assert y_err(y_got, y_ref) <= TOL["bf16"]
     assert state_err(S_got, S_ref) <= TOL["bf16"]
     assert snaps_err(sn_got, sn_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("algo", ALGOS_ANY)
+def test_more_heads_than_sms(cuda_device, algo):
+    """200 (b, h) heads: the persistent chunked kernel walks several heads per CTA and
+    prefetches the next head's first chunk."""
+    wl = inputs.WORKLOADS[1]
+    d = inputs.make_inputs(wl, B=4, T=200, H=50, seed=21)
+    y_ref, S_ref, _ = _oracle(d)
+    y, S, _ = _gpu(_dev(d, cuda_device), algo=algo)
+    assert y_err(y, y_ref) <= TOL["bf16"]
+    assert state_err(S, S_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("algo", ALGOS_ANY)
+@pytest.mark.parametrize("case", ["linear_attention", "full_erase", "no_decay_a0", "slowest_decay"])
+def test_degenerate_inputs(cuda_device, algo, case):
+    """Edge cases of the method: w = 1 with a = 0 (linear attention), w = 1 with a = 1
+    (delta-rule erasure), all-zero removal keys, and decay at the lower end of its range."""
+    wl = inputs.WORKLOADS[1]
+    d = inputs.make_inputs(wl, B=2, T=130, H=3, seed=22)
+    one = torch.ones_like(d["w"])
+    if case == "linear_attention":
+        d["w"], d["a"] = one.clone(), torch.zeros_like(d["a"])
+    elif case == "full_erase":
+        d["w"], d["a"] = one.clone(), one.clone()
+    elif case == "no_decay_a0":
+        d["kk"] = torch.zeros_like(d["kk"])
+    else:
+        d["w"] = torch.full_like(d["w"], inputs.W_MIN).to(torch.float32).to(d["w"].dtype)
+    y_ref, S_ref, _ = _oracle(d)
+    y, S, _ = _gpu(_dev(d, cuda_device), algo=algo)
+    assert y_err(y, y_ref) <= TOL["bf16"]
+    assert state_err(S, S_ref) <= TOL["bf16"]
+
+
+def test_chunk_rejects_unsupported_requests(cuda_device):
+    d = _dev(inputs.make_inputs(inputs.WORKLOADS[0], B=1, T=70, H=1, seed=23), cuda_device)
+    with pytest.raises(wkv7.Wkv7Error) as e:
+        _gpu(d, algo="chunk")                       # fp32 inputs
+    assert e.value.status == wkv7.ERR_UNSUPPORTED
+    d = _dev(inputs.make_inputs(inputs.WORKLOADS[1], B=1, T=70, H=1, seed=23), cuda_device)
+    with pytest.raises(wkv7.Wkv7Error) as e:
+        _gpu(d, algo="chunk", snap_every=10)        # snapshot inside a chunk
+    assert e.value.status == wkv7.ERR_UNSUPPORTED
+    y, S, sn = _gpu(d, snap_every=10)               # auto falls back to the scan
+    assert sn.shape[1] == 7
+
+
+def test_no_device_error_after_runs(cuda_device):
+    d = _dev(inputs.make_inputs(inputs.WORKLOADS[1], B=1, T=64, H=2, seed=24), cuda_device)
+    _gpu(d, algo="chunk")
+    wkv7.poll_device_error()
