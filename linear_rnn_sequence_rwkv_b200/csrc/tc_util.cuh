@@ -161,10 +161,37 @@ __device__ __forceinline__ uint64_t kstep_off(int ks, int rows) {
     return uint64_t(((ks >> 2) * rows * 128 + (ks & 3) * 32) >> 4);
 }
 
+// ---- MN-major operand layout (128-byte swizzle, tf32) ----------------------------------------------
+// A K x MN operand stored "MN-major": for each K index (a "row" here) 32 consecutive MN elements
+// fill one 128-byte line; 8 consecutive K rows form a 1024-byte swizzle atom (16-byte chunk c of
+// row r at chunk position c ^ (r % 8)). Atoms of successive K groups are MN_SBO bytes apart and
+// blocks of 32 MN elements are `kdim/8 * 1024` bytes apart. A thread owning one K row writes its
+// MN elements with 16-byte stores.
+constexpr uint32_t MN_SBO = 1024;
+__device__ __forceinline__ uint32_t mn_off(int k, int n, int kdim) {
+    return uint32_t((n >> 5) * (kdim >> 3) * 1024 + (k >> 3) * 1024 + (k & 7) * 128 +
+                    ((((n & 31) >> 2) ^ (k & 7)) << 4) + ((n & 3) << 2));
+}
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t smem_addr, int kdim) {
+    uint64_t d = 0;
+    d |= uint64_t((smem_addr & 0x3FFFFu) >> 4);                 // start address
+    d |= uint64_t(((kdim >> 3) * 1024) >> 4) << 16;             // leading byte offset: next 32 MN elements
+    d |= uint64_t(MN_SBO >> 4) << 32;                           // stride byte offset: next 8 K rows
+    d |= uint64_t(1) << 46;
+    d |= uint64_t(2) << 61;
+    return d;
+}
+// Offset (16-byte units) of K-step `ks` (8 K rows) in an MN-major tile.
+__device__ __forceinline__ uint64_t mn_kstep_off(int ks) { return uint64_t(ks * MN_SBO >> 4); }
+
 // Instruction descriptor of kind::tf32 with fp32 accumulation, K-major A and B.
 __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
     return (1u << 4) | (2u << 7) | (2u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
+// Same with B stored MN-major.
+__host__ __device__ constexpr uint32_t idesc_tf32_bmn(int M, int N) { return idesc_tf32(M, N) | (1u << 16); }
+// Same with the A operand negated (D = D - A B when accumulating).
+__host__ __device__ constexpr uint32_t idesc_neg_a(uint32_t idesc) { return idesc | (1u << 13); }
 
 // ---- tcgen05.mma (issued by a single thread) -----------------------------------------------------
 __device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
