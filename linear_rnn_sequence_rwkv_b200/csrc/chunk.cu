@@ -53,21 +53,22 @@ using namespace tc;
 constexpr int C = 64;             // chunk length (tokens)
 constexpr int kThreads = 256;
 constexpr int GTS = 68;           // row stride (floats) of the decay table: conflict-free row reads
-constexpr int LWS = 65;           // row stride of the inverse workspaces
+constexpr int LWS = 68;           // row stride of the inverse workspaces (16-byte aligned rows)
 
 // Shared-memory layout (byte offsets from a 1024-byte aligned base).
-constexpr uint32_t OFF_B1 = 0;        // [Bi; Ki] 128x64 tf32 (R1 B operand); later the inverse workspace
+constexpr uint32_t OFF_B1 = 0;        // [Bi; Ki] 128x64 tf32 (R1 B operand, R1b A operand); later the inverse workspace
 constexpr uint32_t OFF_B3 = 32768;    // [KKd^T | M_kb^T] 128x64 (R3 B operand)
 constexpr uint32_t OFF_B2 = 65536;    // A^T 64x64 (R2 B operand)
 constexpr uint32_t OFF_B4 = 81920;    // V^T 64x64 (R4 B operand; exact bf16 values)
 constexpr uint32_t OFF_B5 = 98304;    // S 64x64, row = value channel (R5 B operand)
-constexpr uint32_t OFF_IN = 114688;   // six bf16 [64][64] input tiles, TMA destination (swizzled)
-constexpr uint32_t OFF_GT = 163840;   // decay table [65][GTS] fp32; later the inverse [64][LWS]
+constexpr uint32_t OFF_B6 = 114688;   // KKd 64x64, row = token (R1b B operand)
+constexpr uint32_t OFF_IN = 131072;   // six bf16 [64][64] input tiles, TMA destination (swizzled)
+constexpr uint32_t OFF_GT = 180224;   // decay table [65][GTS] fp32; later the inverse [64][LWS]
 constexpr uint32_t OFF_SMALL = OFF_GT + 65 * GTS * 4;
 
 struct Small {
     float gC[C];
-    float tot[2][C];
+    float tq[4][C];       // decay product over each quarter of the chunk, per key channel
     float bon[2][C];
     float dk[2][C];       // r_t . k_t, partial over each column half (exact current-token Gram entry)
     float db[2][C];       // r_t . (kk_t * a_t)
@@ -81,9 +82,9 @@ constexpr uint32_t SMEM_BYTES = OFF_SMALL + sizeof(Small) + 1024;   // + alignme
 
 // TMEM columns (512 allocated).
 constexpr uint32_t T_A1 = 0;     // [KKd; Rd]
-constexpr uint32_t T_D1 = 64;    // Grams [M_ab | M_kb ; Q_b | Q_k] -> cols 0-63 become [Bc^T; Q_b]
-constexpr uint32_t T_D2 = 192;   // Z
-constexpr uint32_t T_D3 = 256;   // X -> [P; R~] (cols 0-63) and [K~; Q~] (cols 64-127)
+constexpr uint32_t T_D1 = 64;    // Grams [M_ab | M_kb ; Q_b | Q_k]
+constexpr uint32_t T_D2 = 192;   // transposed Grams [M_ab^T; M_kb^T] (R1b), then Z
+constexpr uint32_t T_D3 = 256;   // A2 = [Bc^T; Q_b] (cols 0-63), then X -> [P; R~] and [K~; Q~]
 constexpr uint32_t T_D4 = 384;   // [S_C^T; Y]
 constexpr uint32_t T_KC = 448;   // Kc^T (lanes 0-63)
 
@@ -128,8 +129,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     const uint8_t *IN = sm + OFF_IN;
     float *GT = reinterpret_cast<float *>(sm + OFF_GT);
     float *Lw = reinterpret_cast<float *>(sm + OFF_B1);      // strictly lower M_ab [64][LWS]
-    float *Tw = Lw + 64 * LWS;                               // level-1 temps [2][16][17]
-    float *Tw2 = Tw + 2 * 16 * 17;                           // level-2 temp [32][33]
+    float *Tw = Lw + 64 * LWS;                               // level-1 temps [2][16][20]
+    float *Tw2 = Tw + 2 * 16 * 20;                           // level-2 temp [32][36]
     float *Aw = reinterpret_cast<float *>(sm + OFF_GT);      // inverse [64][LWS]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -157,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     // matrix descriptors of the shared-memory B operands at K-step 0
     const uint64_t dB1 = desc_sw128(smem_u32(sm + OFF_B1)), dB2 = desc_sw128(smem_u32(sm + OFF_B2));
     const uint64_t dB3 = desc_sw128(smem_u32(sm + OFF_B3)), dB4 = desc_sw128(smem_u32(sm + OFF_B4));
-    const uint64_t dB5 = desc_sw128(smem_u32(sm + OFF_B5));
+    const uint64_t dB5 = desc_sw128(smem_u32(sm + OFF_B5)), dB6 = desc_sw128(smem_u32(sm + OFF_B6));
     uint32_t tma_parity = 0, mma_parity = 0;
     bool tma_pending = false, mma_pending = false, failed = false;
 
@@ -209,93 +210,94 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 tma_pending = false;
                 if (__syncthreads_or(to)) { failed = true; break; }
             }
-            // ---- S1: running decay products within each half of the chunk (column group, j = L)
-            if (colg) {
+            // ---- P1: decay products per key channel j over each quarter of the chunk (all threads)
+            {
+                const int j = tid & 63, q = tid >> 6;
                 const uint8_t *wt = IN + XW * 8192;
                 float run = 1.f;
-#pragma unroll 8
-                for (int i = 0; i < 32; ++i) {
-                    const int t = 32 * h + i;
-                    run *= (t < Lc) ? in_elem(wt, t, L) : 1.f;   // padded tokens: w = 1
-                    GT[(t + 1) * GTS + L] = run;
-                }
-                S.tot[h][L] = run;
-                if (h == 0) GT[L] = 1.f;
-            }
-            __syncthreads();
-            // ---- S2: products of the second half made absolute; column outputs Kc^T (TMEM),
-            //      KKd^T (B3 rows 0-63), V^T (B4)
-            if (colg) {
-                const int j = L;
-                const float pre = h ? S.tot[0][j] : 1.f;
-                const float gCj = S.tot[0][j] * S.tot[1][j];
-                if (h == 0) S.gC[j] = gCj;
-                float gprev = pre;   // g_{t-1} of the first token of this half
-#pragma unroll 1
-                for (int g8 = 0; g8 < 4; ++g8) {
-                    const int t0 = 32 * h + 8 * g8;
-                    float kc[8], kkd[8], vv[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int t = t0 + e;
-                        const float graw = GT[(t + 1) * GTS + j];
-                        const float gt = h ? pre * graw : graw;
-                        if (h) GT[(t + 1) * GTS + j] = gt;
-                        kc[e] = to_tf32(in_elem(IN + XK * 8192, t, j) * __fdividef(gCj, gt));
-                        kkd[e] = to_tf32(in_elem(IN + XKK * 8192, t, j) * gprev);
-                        vv[e] = in_elem(IN + XV * 8192, t, j);
-                        gprev = gt;
-                    }
-                    tmem_st8(tmem_addr(tb, Lq, T_KC + t0), kc);
-                    st_f4(sm + OFF_B3, sw128_off(j, t0, 128), kkd[0], kkd[1], kkd[2], kkd[3]);
-                    st_f4(sm + OFF_B3, sw128_off(j, t0 + 4, 128), kkd[4], kkd[5], kkd[6], kkd[7]);
-                    st_f4(sm + OFF_B4, sw128_off(j, t0, 64), vv[0], vv[1], vv[2], vv[3]);
-                    st_f4(sm + OFF_B4, sw128_off(j, t0 + 4, 64), vv[4], vv[5], vv[6], vv[7]);
+                for (int e = 0; e < 16; ++e) {
+                    const int t = 16 * q + e;
+                    run *= (t < Lc) ? in_elem(wt, t, j) : 1.f;   // padded tokens: w = 1
+                    GT[(t + 1) * GTS + j] = run;
+                }
+                S.tq[q][j] = run;
+            }
+            __syncthreads();
+            // ---- P2: absolute products g_t (the quarters before this one as prefix)
+            {
+                const int j = tid & 63, q = tid >> 6;
+                float pre = 1.f;
+                for (int qq = 0; qq < q; ++qq) pre *= S.tq[qq][j];
+                if (q > 0) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) GT[(16 * q + e + 1) * GTS + j] *= pre;
+                } else {
+                    GT[j] = 1.f;
+                    S.gC[j] = S.tq[0][j] * S.tq[1][j] * S.tq[2][j] * S.tq[3][j];
                 }
             }
             __syncthreads();
-            // ---- S3: row outputs
-            if (colg) {                 // token t = L: KKd row -> A1 lanes 0..63
+            // ---- P3: token rows. Lanes 0-63: KKd row -> A1 (TMEM) and B6 (R1b operand); Ki row -> B1.
+            //      Lanes 64-127: Rd row -> A1; Bi row -> B1; exact current-token Grams.
+            if (colg) {                 // token t = L: KKd row -> A1 lanes 0-63 and B6; Ki row -> B1
                 const int t = L;
-                const float *gp = GT + t * GTS;   // g_{t-1}
+                const float *gp = GT + t * GTS;         // g_{t-1}
+                const float *gt = GT + (t + 1) * GTS;   // g_t
 #pragma unroll 1
                 for (int g8 = 0; g8 < 4; ++g8) {
                     const int j0 = 32 * h + 8 * g8;
-                    float kk8[8], v[8];
+                    float kk8[8], k8[8], v[8], ki[8];
                     in_row8(IN + XKK * 8192, t, j0, kk8);
+                    in_row8(IN + XK * 8192, t, j0, k8);
+                    const float4 ga = *reinterpret_cast<const float4 *>(gp + j0);
+                    const float4 gb = *reinterpret_cast<const float4 *>(gp + j0 + 4);
+                    const float4 gc = *reinterpret_cast<const float4 *>(gt + j0);
+                    const float4 gd = *reinterpret_cast<const float4 *>(gt + j0 + 4);
+                    const float gpv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                    const float gtv[8] = {gc.x, gc.y, gc.z, gc.w, gd.x, gd.y, gd.z, gd.w};
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] = to_tf32(kk8[e] * gp[j0 + e]);
+                    for (int e = 0; e < 8; ++e) {
+                        v[e] = to_tf32(kk8[e] * gpv[e]);
+                        ki[e] = to_tf32(k8[e] * __fdividef(1.f, gtv[e]));
+                    }
                     tmem_st8(tmem_addr(tb, Lq, T_A1 + j0), v);
+                    st_f4(sm + OFF_B6, sw128_off(t, j0, 64), v[0], v[1], v[2], v[3]);
+                    st_f4(sm + OFF_B6, sw128_off(t, j0 + 4, 64), v[4], v[5], v[6], v[7]);
+                    st_f4(sm + OFF_B1, sw128_off(64 + t, j0, 128), ki[0], ki[1], ki[2], ki[3]);
+                    st_f4(sm + OFF_B1, sw128_off(64 + t, j0 + 4, 128), ki[4], ki[5], ki[6], ki[7]);
                 }
-            } else {                    // token t = L - 64: Rd row -> A1 lanes 64..127; Bi, Ki rows -> B1
+            } else {
                 const int t = L - 64;
                 const float *gt = GT + (t + 1) * GTS;   // g_t
                 float bon = 0.f, dk = 0.f, db = 0.f;
 #pragma unroll 1
                 for (int g8 = 0; g8 < 4; ++g8) {
                     const int j0 = 32 * h + 8 * g8;
-                    float r8[8], kk8[8], a8[8], k8[8], rd[8], bi[8], ki[8];
+                    float r8[8], kk8[8], a8[8], k8[8], g8v[8], rd[8], bi[8];
                     in_row8(IN + XR * 8192, t, j0, r8);
                     in_row8(IN + XKK * 8192, t, j0, kk8);
                     in_row8(IN + XA * 8192, t, j0, a8);
                     in_row8(IN + XK * 8192, t, j0, k8);
+                    {
+                        const float4 ga = *reinterpret_cast<const float4 *>(gt + j0);
+                        const float4 gb = *reinterpret_cast<const float4 *>(gt + j0 + 4);
+                        g8v[0] = ga.x; g8v[1] = ga.y; g8v[2] = ga.z; g8v[3] = ga.w;
+                        g8v[4] = gb.x; g8v[5] = gb.y; g8v[6] = gb.z; g8v[7] = gb.w;
+                    }
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float gv = gt[j0 + e];
-                        const float ig = __fdividef(1.f, gv);
-                        const float b = kk8[e] * a8[e];
-                        rd[e] = to_tf32(r8[e] * gv);
-                        bi[e] = to_tf32(b * ig);
-                        ki[e] = to_tf32(k8[e] * ig);
+                        const float ig = __fdividef(1.f, g8v[e]);
+                        const float bb = kk8[e] * a8[e];
+                        rd[e] = to_tf32(r8[e] * g8v[e]);
+                        bi[e] = to_tf32(bb * ig);
                         dk = fmaf(r8[e], k8[e], dk);
-                        db = fmaf(r8[e], b, db);
+                        db = fmaf(r8[e], bb, db);
                         if (epi) bon = fmaf(r8[e] * k8[e], S.r_k[j0 + e], bon);
                     }
                     tmem_st8(tmem_addr(tb, Lq, T_A1 + j0), rd);
                     st_f4(sm + OFF_B1, sw128_off(t, j0, 128), bi[0], bi[1], bi[2], bi[3]);
                     st_f4(sm + OFF_B1, sw128_off(t, j0 + 4, 128), bi[4], bi[5], bi[6], bi[7]);
-                    st_f4(sm + OFF_B1, sw128_off(64 + t, j0, 128), ki[0], ki[1], ki[2], ki[3]);
-                    st_f4(sm + OFF_B1, sw128_off(64 + t, j0 + 4, 128), ki[4], ki[5], ki[6], ki[7]);
                 }
                 S.dk[h][t] = dk;
                 S.db[h][t] = db;
@@ -306,35 +308,65 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)   // R1: Grams = [KKd; Rd] [Bi; Ki]^T
-                    mma_tf32_ts(tb + T_D1, tb + T_A1 + 8 * ks, dB1 + kstep_off(ks, 128),
-                                idesc_tf32(128, 128), ks > 0);
+                    mma_tf32_ts(tb + T_D1, tb + T_A1 + 8 * ks, dB1 + kstep_off(ks, 128), idesc_tf32(128, 128), ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)   // R1b: transposed Grams [Bi; Ki] KKd^T
+                    mma_tf32_ss(tb + T_D2, dB1 + kstep_off(ks, 128), dB6 + kstep_off(ks, 64), idesc_tf32(128, 64), ks > 0);
                 mma_commit(&S.bar_mma);
             }
             mma_pending = true;
-            if (wait_mma()) { failed = true; break; }
-            // ---- masks; M_ab -> inverse workspace; M_kb^T -> B3; A2 = [Bc^T; Q_b] in TMEM
+            // ---- P4 (while the Gram MMAs run): key-channel columns over tokens 32h..32h+31.
+            //      Lanes 0-63: Bc^T -> A2 rows (TMEM, T_D3) and Kc^T -> T_KC.
+            //      Lanes 64-127 (key j = L - 64): KKd^T -> B3 rows 0-63, V^T -> B4.
             if (colg) {
-                const int t = L, j = L;   // D1 row t (token) is read before lane j receives Bc^T row j
+                const int j = L;
                 const float gCj = S.gC[j];
 #pragma unroll 1
                 for (int g8 = 0; g8 < 4; ++g8) {
-                    const int s0 = 32 * h + 8 * g8;
-                    float m[8], bc[8];
-                    tmem_ld8(tmem_addr(tb, Lq, T_D1 + s0), m);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) Lw[t * LWS + s0 + e] = (s0 + e < t) ? m[e] : 0.f;
-                    tmem_ld8(tmem_addr(tb, Lq, T_D1 + 64 + s0), m);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        *reinterpret_cast<float *>(sm + OFF_B3 + sw128_off(64 + s0 + e, t, 128)) =
-                            (s0 + e < t) ? to_tf32(m[e]) : 0.f;
+                    const int t0 = 32 * h + 8 * g8;
+                    float bc[8], kc[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const int ss = s0 + e;
-                        const float b = in_elem(IN + XKK * 8192, ss, j) * in_elem(IN + XA * 8192, ss, j);
-                        bc[e] = to_tf32(b * __fdividef(gCj, GT[(ss + 1) * GTS + j]));
+                        const int t = t0 + e;
+                        const float sc = __fdividef(gCj, GT[(t + 1) * GTS + j]);   // prod of w after t
+                        bc[e] = to_tf32(in_elem(IN + XKK * 8192, t, j) * in_elem(IN + XA * 8192, t, j) * sc);
+                        kc[e] = to_tf32(in_elem(IN + XK * 8192, t, j) * sc);
                     }
-                    tmem_st8(tmem_addr(tb, Lq, T_D1 + s0), bc);
+                    tmem_st8(tmem_addr(tb, Lq, T_D3 + t0), bc);
+                    tmem_st8(tmem_addr(tb, Lq, T_KC + t0), kc);
+                }
+            } else {
+                const int j = L - 64;
+#pragma unroll 1
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    const int t0 = 32 * h + 8 * g8;
+                    float kkd[8], vv[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int t = t0 + e;
+                        kkd[e] = to_tf32(in_elem(IN + XKK * 8192, t, j) * GT[t * GTS + j]);   // kk * g_{t-1}
+                        vv[e] = in_elem(IN + XV * 8192, t, j);
+                    }
+                    st_f4(sm + OFF_B3, sw128_off(j, t0, 128), kkd[0], kkd[1], kkd[2], kkd[3]);
+                    st_f4(sm + OFF_B3, sw128_off(j, t0 + 4, 128), kkd[4], kkd[5], kkd[6], kkd[7]);
+                    st_f4(sm + OFF_B4, sw128_off(j, t0, 64), vv[0], vv[1], vv[2], vv[3]);
+                    st_f4(sm + OFF_B4, sw128_off(j, t0 + 4, 64), vv[4], vv[5], vv[6], vv[7]);
+                }
+            }
+            if (wait_mma()) { failed = true; break; }
+            // ---- P5: masks. Lanes 0-63 (token t): M_ab row -> inverse workspace.
+            //      Lanes 64-127 (token t): Q_b row -> A2 rows 64-127 (T_D3); M_kb^T row t -> B3.
+            if (colg) {
+                const int t = L;
+#pragma unroll 1
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    const int s0 = 32 * h + 8 * g8;
+                    float m[8];
+                    tmem_ld8(tmem_addr(tb, Lq, T_D1 + s0), m);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) m[e] = (s0 + e < t) ? m[e] : 0.f;
+                    *reinterpret_cast<float4 *>(Lw + t * LWS + s0) = make_float4(m[0], m[1], m[2], m[3]);
+                    *reinterpret_cast<float4 *>(Lw + t * LWS + s0 + 4) = make_float4(m[4], m[5], m[6], m[7]);
                 }
             } else {
                 const int t = L - 64;
@@ -350,7 +382,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                         const int ss = s0 + e;
                         m[e] = ss < t ? to_tf32(m[e]) : (ss == t ? to_tf32(diag) : 0.f);
                     }
-                    tmem_st8(tmem_addr(tb, Lq, T_D1 + s0), m);
+                    tmem_st8(tmem_addr(tb, Lq, T_D3 + s0), m);
+                    // row t of M_kb^T: M_kb[t'][t] for tokens t' = s0..s0+7 (nonzero for t' > t)
+                    tmem_ld8(tmem_addr(tb, Lq, T_D2 + s0), m);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) m[e] = (s0 + e > t) ? to_tf32(m[e]) : 0.f;
+                    st_f4(sm + OFF_B3, sw128_off(64 + t, s0, 128), m[0], m[1], m[2], m[3]);
+                    st_f4(sm + OFF_B3, sw128_off(64 + t, s0 + 4, 128), m[4], m[5], m[6], m[7]);
                 }
             }
             sync_for_mma();
@@ -361,9 +399,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
             }
             tma_pending = !last || unit + int(gridDim.x) < units;
             // ---- A = (I + M_ab)^{-1}. Diagonal 16x16 blocks: one thread per (block, column)
-            //      solves (I + L_dd) x = e_c by forward substitution in registers.
-            if (tid < 64) {
-                const int d = tid >> 4, cc = tid & 15;
+            //      solves (I + L_dd) x = e_c by forward substitution in registers (warps 2, 3).
+            if (tid >= 64 && tid < 128) {
+                const int d = (tid - 64) >> 4, cc = tid & 15;
                 const float *Lb = Lw + 16 * d * LWS + 16 * d;
                 float x[16];
 #pragma unroll
@@ -377,8 +415,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 for (int r = 0; r < 16; ++r) Aw[(16 * d + r) * LWS + 16 * d + cc] = x[r];
             } else {
                 // zero the blocks above the diagonal: (bi, bj) with bi < bj
+                const int z0 = tid < 64 ? tid : tid - 64;
 #pragma unroll 1
-                for (int e = tid - 64; e < 6 * 256; e += kThreads - 64) {
+                for (int e = z0; e < 6 * 256; e += kThreads - 64) {
                     const int blk = e >> 8, o = e & 255;
                     const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
                     const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
@@ -386,51 +425,61 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 }
             }
             __syncthreads();
-            // level 1: X[2p+1][2p] = -X[2p+1] (L[2p+1][2p] X[2p]),  p = 0, 1
-            for (int o = tid; o < 512; o += kThreads) {
-                const int pp = o >> 8, i = (o >> 4) & 15, jj = o & 15;
-                float acc = 0.f;
+            // level 1: X[2p+1][2p] = -X[2p+1] (L[2p+1][2p] X[2p]), p = 0, 1. Threads 0-127 each
+            // compute four adjacent outputs from one broadcast scalar and one float4 per step.
+            if (tid < 128) {
+                const int pp = tid >> 6, i = (tid >> 2) & 15, j4 = (tid & 3) * 4;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int kq = 0; kq < 16; ++kq)
-                    acc = fmaf(Lw[(32 * pp + 16 + i) * LWS + 32 * pp + kq], Aw[(32 * pp + kq) * LWS + 32 * pp + jj], acc);
-                Tw[(pp * 16 + i) * 17 + jj] = acc;
+                for (int kq = 0; kq < 16; ++kq) {
+                    const float lv = Lw[(32 * pp + 16 + i) * LWS + 32 * pp + kq];
+                    const float4 xv = *reinterpret_cast<const float4 *>(Aw + (32 * pp + kq) * LWS + 32 * pp + j4);
+                    acc[0] = fmaf(lv, xv.x, acc[0]); acc[1] = fmaf(lv, xv.y, acc[1]);
+                    acc[2] = fmaf(lv, xv.z, acc[2]); acc[3] = fmaf(lv, xv.w, acc[3]);
+                }
+                *reinterpret_cast<float4 *>(Tw + (pp * 16 + i) * 20 + j4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
             }
             __syncthreads();
-            for (int o = tid; o < 512; o += kThreads) {
-                const int pp = o >> 8, i = (o >> 4) & 15, jj = o & 15;
-                float acc = 0.f;
+            if (tid < 128) {
+                const int pp = tid >> 6, i = (tid >> 2) & 15, j4 = (tid & 3) * 4;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int kq = 0; kq < 16; ++kq)
-                    acc = fmaf(Aw[(32 * pp + 16 + i) * LWS + 32 * pp + 16 + kq], Tw[(pp * 16 + kq) * 17 + jj], acc);
-                Aw[(32 * pp + 16 + i) * LWS + 32 * pp + jj] = -acc;
+                for (int kq = 0; kq < 16; ++kq) {
+                    const float xv = Aw[(32 * pp + 16 + i) * LWS + 32 * pp + 16 + kq];
+                    const float4 tv = *reinterpret_cast<const float4 *>(Tw + (pp * 16 + kq) * 20 + j4);
+                    acc[0] = fmaf(xv, tv.x, acc[0]); acc[1] = fmaf(xv, tv.y, acc[1]);
+                    acc[2] = fmaf(xv, tv.z, acc[2]); acc[3] = fmaf(xv, tv.w, acc[3]);
+                }
+                *reinterpret_cast<float4 *>(Aw + (32 * pp + 16 + i) * LWS + 32 * pp + j4) =
+                    make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
             }
             __syncthreads();
             // level 2: Y[1][0] = -Y1 (L[32:64][0:32] Y0). Y0, Y1 are lower triangular, so the
-            // fixed-length sums are exact; each thread keeps four independent accumulators.
+            // fixed-length sums are exact. Each thread: one row, four adjacent columns.
             {
-                const int i = tid >> 3, jg = tid & 7;
+                const int i = tid >> 3, j4 = (tid & 7) * 4;
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
                 for (int kq = 0; kq < 32; ++kq) {
                     const float lv = Lw[(32 + i) * LWS + kq];
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) acc[m] = fmaf(lv, Aw[kq * LWS + jg + 8 * m], acc[m]);
+                    const float4 yv = *reinterpret_cast<const float4 *>(Aw + kq * LWS + j4);
+                    acc[0] = fmaf(lv, yv.x, acc[0]); acc[1] = fmaf(lv, yv.y, acc[1]);
+                    acc[2] = fmaf(lv, yv.z, acc[2]); acc[3] = fmaf(lv, yv.w, acc[3]);
                 }
-#pragma unroll
-                for (int m = 0; m < 4; ++m) Tw2[i * 33 + jg + 8 * m] = acc[m];
+                *reinterpret_cast<float4 *>(Tw2 + i * 36 + j4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
             }
             __syncthreads();
             {
-                const int i = tid >> 3, jg = tid & 7;
+                const int i = tid >> 3, j4 = (tid & 7) * 4;
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
                 for (int kq = 0; kq < 32; ++kq) {
                     const float av = Aw[(32 + i) * LWS + 32 + kq];
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) acc[m] = fmaf(av, Tw2[kq * 33 + jg + 8 * m], acc[m]);
+                    const float4 tv = *reinterpret_cast<const float4 *>(Tw2 + kq * 36 + j4);
+                    acc[0] = fmaf(av, tv.x, acc[0]); acc[1] = fmaf(av, tv.y, acc[1]);
+                    acc[2] = fmaf(av, tv.z, acc[2]); acc[3] = fmaf(av, tv.w, acc[3]);
                 }
-#pragma unroll
-                for (int m = 0; m < 4; ++m) Aw[(32 + i) * LWS + jg + 8 * m] = -acc[m];
+                *reinterpret_cast<float4 *>(Aw + (32 + i) * LWS + j4) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
             }
             __syncthreads();
             // B2 = A^T (row s, K = t)
@@ -444,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)   // R2: Z = [Bc^T; Q_b] A
-                    mma_tf32_ts(tb + T_D2, tb + T_D1 + 8 * ks, dB2 + kstep_off(ks, 64),
+                    mma_tf32_ts(tb + T_D2, tb + T_D3 + 8 * ks, dB2 + kstep_off(ks, 64),
                                 idesc_tf32(128, 64), ks > 0);
                 mma_commit(&S.bar_mma);
             }

@@ -124,11 +124,13 @@ __device__ __forceinline__ uint32_t tmem_addr(uint32_t base, uint32_t lane, uint
 }
 
 // ---- tf32 rounding -----------------------------------------------------------------------------
-// Round to the nearest tf32 value (ties away from zero); the tensor core then reads it exactly.
+// Round a finite fp32 value to the nearest tf32 value (10 explicit mantissa bits), ties away
+// from zero: add half of the 13 dropped bits' range to the sign-magnitude pattern, then clear
+// them (a carry into the exponent is the correct round-up). The tensor core then reads the
+// operand exactly. Two integer instructions; the conversion instruction is several times
+// slower on this part.
 __device__ __forceinline__ float to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
+    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
 }
 
 // ---- shared-memory operand layout (K-major, 128-byte swizzle, tf32) -------------------------------
