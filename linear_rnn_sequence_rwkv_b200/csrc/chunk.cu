@@ -12,9 +12,10 @@
 //     KKd = kk*g_{t-1}, Rd = r*g_t, Bi = b/g_s, Ki = k/g_s, Bc = b*gC/g_s, Kc = k*gC/g_s
 //     M_ab = tril(KKd Bi^T, -1), M_kb = tril(KKd Ki^T, -1), Q_b = tril(Rd Bi^T), Q_k = tril(Rd Ki^T)
 //     A = (I + M_ab)^{-1}                              (the removed values U = A(-KKd S_0^T - M_kb V))
-//     [Z] = [Bc^T; Q_b] A,   [X] = Z [KKd | M_kb]
-//     P  = diag(gC) - Bc^T A KKd      R~ = Rd  - Q_b A KKd
-//     K~ = Kc^T - Bc^T A M_kb         Q~ = Q_k - Q_b A M_kb
+//     [Z] = [Bi^T; Q_b] A,   [X] = Z [KKd | M_kb]
+//     P  = diag(gC) (I - Bi^T A KKd)      R~ = Rd  - Q_b A KKd
+//     K~ = diag(gC) (Ki^T - Bi^T A M_kb)  Q~ = Q_k - Q_b A M_kb
+// (Bc = Bi*gC and Kc = Ki*gC column-wise, so gC is applied once, per key row of P and K~.)
 //     [S_C^T; Y] = [P; R~] S_0^T + [K~; Q~] V
 // Only the last line depends on the state, so the chain from chunk to chunk is one
 // fused M=128 MMA; everything else is computed from the chunk's own inputs.
@@ -25,9 +26,11 @@
 //  * Every MMA is tcgen05.mma kind::tf32, M=128, with the A operand in tensor memory
 //    (lane = row) and the B operand in shared memory (K-major, 128-byte swizzle). Five
 //    MMA rounds per chunk: Grams, Z, X, then the two state rounds into one accumulator.
-//  * 256 threads = 8 warps. TMEM lanes 0-63 belong to warps 0,1,4,5 ("column group":
-//    a key channel j or a token t, by phase), lanes 64-127 to warps 2,3,6,7 ("row
-//    group": a token t); the two warps sharing a lane quarter split the 64 columns.
+//  * 512 threads = 16 warps, four per SM sub-partition so that latency is hidden. A warp
+//    reaches only its quarter of the TMEM lanes: lanes 0-63 belong to warps w with w % 4 in
+//    {0, 1} ("column group": a key channel j or a token t, by phase), lanes 64-127 to the
+//    others ("row group": a token t or a key channel). The four warps sharing a lane quarter
+//    split the 64 columns (or tokens) into 16-wide parts.
 //  * The unit-lower-triangular inverse is done in fp32 on the CUDA cores: 16x16
 //    diagonal blocks by warp-shuffle substitution, then two levels of block merges.
 //  * Operands are rounded to tf32 (round to nearest) before the tensor core sees them;
@@ -51,42 +54,43 @@ namespace {
 using namespace tc;
 
 constexpr int C = 64;             // chunk length (tokens)
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;   // 16 warps: 4 per SM sub-partition
 constexpr int GTS = 68;           // row stride (floats) of the decay table: conflict-free row reads
 constexpr int LWS = 68;           // row stride of the inverse workspaces (16-byte aligned rows)
 
 // Shared-memory layout (byte offsets from a 1024-byte aligned base).
-constexpr uint32_t OFF_B1 = 0;        // [Bi; Ki] 128x64 tf32 (R1 B operand, R1b A operand); later the inverse workspace
-constexpr uint32_t OFF_B3 = 32768;    // [KKd^T | M_kb^T] 128x64 (R3 B operand)
-constexpr uint32_t OFF_B2 = 65536;    // A^T 64x64 (R2 B operand)
-constexpr uint32_t OFF_B4 = 81920;    // V^T 64x64 (R4 B operand; exact bf16 values)
-constexpr uint32_t OFF_B5 = 98304;    // S 64x64, row = value channel (R5 B operand)
-constexpr uint32_t OFF_B6 = 114688;   // KKd 64x64, row = token (R1b B operand)
-constexpr uint32_t OFF_IN = 131072;   // six bf16 [64][64] input tiles, TMA destination (swizzled)
-constexpr uint32_t OFF_GT = 180224;   // decay table [65][GTS] fp32; later the inverse [64][LWS]
+constexpr uint32_t OFF_B1 = 0;        // [Bi; Ki] 128x64 tf32 (B of R1, R1c, R1d; A of R1b); later the inverse workspace
+constexpr uint32_t OFF_B3 = 32768;    // [KKd^T | M_kb^T] 128x64 (B of R3)
+constexpr uint32_t OFF_B2 = 65536;    // A^T 64x64 (B of R2)
+constexpr uint32_t OFF_B4 = 81920;    // V^T 64x64 (B of R4; exact bf16 values)
+constexpr uint32_t OFF_B5 = 98304;    // S 64x64, row = value channel (B of R5)
+constexpr uint32_t OFF_A1 = 114688;   // [KKd; Rd] 128x64 (A of R1; rows 0-63 are the B of R1b)
+constexpr uint32_t OFF_IN = 147456;   // six bf16 [64][64] input tiles, TMA destination (swizzled)
+constexpr uint32_t OFF_GT = 196608;   // decay table [65][GTS] fp32; later the inverse [64][LWS]
 constexpr uint32_t OFF_SMALL = OFF_GT + 65 * GTS * 4;
 
 struct Small {
     float gC[C];
-    float tq[4][C];       // decay product over each quarter of the chunk, per key channel
-    float bon[2][C];
-    float dk[2][C];       // r_t . k_t, partial over each column half (exact current-token Gram entry)
-    float db[2][C];       // r_t . (kk_t * a_t)
-    float red[2][C];
+    float tq[8][C];       // decay product over each eighth of the chunk, per key channel
+    float bon[4][C];
+    float dk[4][C];       // r_t . k_t, partial over each column quarter (exact current-token Gram entry)
+    float db[4][C];       // r_t . (kk_t * a_t)
+    float red[4][C];
     float ln_w[C], ln_b[C], r_k[C];
     uint64_t bar_tma;
     uint64_t bar_mma;
     uint32_t tmem_base;
 };
 constexpr uint32_t SMEM_BYTES = OFF_SMALL + sizeof(Small) + 1024;   // + alignment slack
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 // TMEM columns (512 allocated).
-constexpr uint32_t T_A1 = 0;     // [KKd; Rd]
-constexpr uint32_t T_D1 = 64;    // Grams [M_ab | M_kb ; Q_b | Q_k]
-constexpr uint32_t T_D2 = 192;   // transposed Grams [M_ab^T; M_kb^T] (R1b), then Z
-constexpr uint32_t T_D3 = 256;   // A2 = [Bc^T; Q_b] (cols 0-63), then X -> [P; R~] and [K~; Q~]
-constexpr uint32_t T_D4 = 384;   // [S_C^T; Y]
-constexpr uint32_t T_KC = 448;   // Kc^T (lanes 0-63)
+constexpr uint32_t T_D1 = 0;     // Grams [M_ab | M_kb ; Q_b | Q_k] (R1)
+constexpr uint32_t T_D2 = 128;   // transposed Grams [M_ab^T; M_kb^T] (R1b), then Z (R2)
+constexpr uint32_t T_D3 = 192;   // [I | Ki^T ; Rd | Q_k] -> R3 subtracts Z [KKd | M_kb] -> [I - X | Ki^T - X ; R~ | Q~]
+constexpr uint32_t T_D4 = 320;   // [S'^T; Y] (R4 + R5); the new state is diag(gC) S'^T
+constexpr uint32_t T_A2 = 384;   // A of R2: [Bi^T (R1c); Q_b]
+constexpr uint32_t T_ID = 448;   // identity (lanes 0-63) over zeros: A of the transposes, written once
 
 enum { XR = 0, XW = 1, XK = 2, XV = 3, XKK = 4, XA = 5 };
 
@@ -110,6 +114,22 @@ __device__ __forceinline__ float in_elem(const uint8_t *tile, int t, int j) {
     const uint32_t off = t * 128 + ((((j >> 3) ^ (t & 7))) << 4) + ((j & 7) << 1);
     return __uint_as_float(uint32_t(*reinterpret_cast<const uint16_t *>(tile + off)) << 16);
 }
+// Byte offsets, within a token row, of key channel j in a 128-byte-swizzled bf16 tile, for
+// the eight row phases t % 8 (hoisted out of column walks).
+__device__ __forceinline__ void col_offsets(int j, uint32_t (&xo)[8]) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) xo[e] = ((((j >> 3) ^ e)) << 4) + ((j & 7) << 1);
+}
+__device__ __forceinline__ float in_col(const uint8_t *tile, int t, const uint32_t (&xo)[8], int e) {
+    return __uint_as_float(uint32_t(*reinterpret_cast<const uint16_t *>(tile + t * 128 + xo[e])) << 16);
+}
+// Byte offsets of column k of a K-major swizzled tf32 tile with `rows` rows, for the eight
+// row phases r % 8: element (r0 + e, k) with r0 a multiple of 8 is at r0 * 128 + e * 128 + xo[e].
+__device__ __forceinline__ void kcol_offsets(int k, int rows, uint32_t (&xo)[8]) {
+    const int kb = k >> 5, kk = k & 31;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) xo[e] = uint32_t(kb * rows * 128 + ((((kk >> 2) ^ e)) << 4) + ((kk & 3) << 2));
+}
 // Eight bf16 elements (t, j..j+7), j a multiple of 8.
 __device__ __forceinline__ void in_row8(const uint8_t *tile, int t, int j, float (&o)[8]) {
     const uint32_t off = t * 128 + ((((j >> 3) ^ (t & 7))) << 4);
@@ -120,7 +140,8 @@ __device__ __forceinline__ void in_row8(const uint8_t *tile, int t, int j, float
 __device__ __forceinline__ void st_f4(uint8_t *base, uint32_t off, float a, float b, float c, float d) {
     *reinterpret_cast<float4 *>(base + off) = make_float4(a, b, c, d);
 }
-__device__ __forceinline__ void named_bar_rows() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Barrier among the warps that own TMEM lanes 64-127 (8 warps).
+__device__ __forceinline__ void named_bar_rows() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constant__ ChunkMaps maps, const ChunkArgs p) {
     extern __shared__ uint8_t smem_raw[];
@@ -136,7 +157,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int Lq = (warp & 3) * 32;         // first TMEM lane of this warp's quarter
     const int L = Lq + lane;                // this thread's TMEM lane
-    const int h = tid >> 7;                 // which half of the 64 columns / tokens
+    const int pq = warp >> 2;               // which 16-wide part of the 64 columns / tokens
+    const int c16 = 16 * pq;
     const bool colg = L < 64;
     const int units = p.B * p.H;
     const int nchunks = (p.T + C - 1) / C;
@@ -155,10 +177,21 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tb = S.tmem_base;
-    // matrix descriptors of the shared-memory B operands at K-step 0
+    // matrix descriptors of the shared-memory operands at K-step 0
     const uint64_t dB1 = desc_sw128(smem_u32(sm + OFF_B1)), dB2 = desc_sw128(smem_u32(sm + OFF_B2));
     const uint64_t dB3 = desc_sw128(smem_u32(sm + OFF_B3)), dB4 = desc_sw128(smem_u32(sm + OFF_B4));
-    const uint64_t dB5 = desc_sw128(smem_u32(sm + OFF_B5)), dB6 = desc_sw128(smem_u32(sm + OFF_B6));
+    const uint64_t dB5 = desc_sw128(smem_u32(sm + OFF_B5)), dA1 = desc_sw128(smem_u32(sm + OFF_A1));
+    {   // identity over zeros in T_ID (A operand of the transposes; never overwritten)
+        float id8[8];
+#pragma unroll 1
+        for (int g = 0; g < 2; ++g) {
+            const int c8 = c16 + 8 * g;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) id8[e] = (c8 + e == L) ? 1.f : 0.f;
+            tmem_st8(tmem_addr(tb, Lq, T_ID + c8), id8);
+        }
+        tmem_st_wait();
+    }
     uint32_t tma_parity = 0, mma_parity = 0;
     bool tma_pending = false, mma_pending = false, failed = false;
 
@@ -210,43 +243,49 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 tma_pending = false;
                 if (__syncthreads_or(to)) { failed = true; break; }
             }
-            // ---- P1: decay products per key channel j over each quarter of the chunk (all threads)
+            // ---- P1: decay products per key channel j over each eighth of the chunk (all threads)
             {
                 const int j = tid & 63, q = tid >> 6;
                 const uint8_t *wt = IN + XW * 8192;
+                uint32_t xo[8];
+                col_offsets(j, xo);
                 float run = 1.f;
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int t = 16 * q + e;
-                    run *= (t < Lc) ? in_elem(wt, t, j) : 1.f;   // padded tokens: w = 1
+                for (int e = 0; e < 8; ++e) {
+                    const int t = 8 * q + e;
+                    run *= (t < Lc) ? in_col(wt, t, xo, e) : 1.f;   // padded tokens: w = 1
                     GT[(t + 1) * GTS + j] = run;
                 }
                 S.tq[q][j] = run;
             }
             __syncthreads();
-            // ---- P2: absolute products g_t (the quarters before this one as prefix)
+            // ---- P2: absolute products g_t (the eighths before this one as prefix)
             {
                 const int j = tid & 63, q = tid >> 6;
                 float pre = 1.f;
                 for (int qq = 0; qq < q; ++qq) pre *= S.tq[qq][j];
                 if (q > 0) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) GT[(16 * q + e + 1) * GTS + j] *= pre;
+                    for (int e = 0; e < 8; ++e) GT[(8 * q + e + 1) * GTS + j] *= pre;
                 } else {
                     GT[j] = 1.f;
-                    S.gC[j] = S.tq[0][j] * S.tq[1][j] * S.tq[2][j] * S.tq[3][j];
+                    float g = 1.f;
+#pragma unroll
+                    for (int qq = 0; qq < 8; ++qq) g *= S.tq[qq][j];
+                    S.gC[j] = g;
                 }
             }
             __syncthreads();
-            // ---- P3: token rows. Lanes 0-63: KKd row -> A1 (TMEM) and B6 (R1b operand); Ki row -> B1.
-            //      Lanes 64-127: Rd row -> A1; Bi row -> B1; exact current-token Grams.
-            if (colg) {                 // token t = L: KKd row -> A1 lanes 0-63 and B6; Ki row -> B1
+            // ---- P3: token rows. Lanes 0-63 (token t = L): KKd row -> A1 rows 0-63, Ki row -> B1,
+            //      identity row -> T_D3 (start of P). Lanes 64-127 (token t): Rd row -> A1 rows 64-127
+            //      and T_D3 (start of R~), Bi row -> B1, exact current-token Grams.
+            if (colg) {
                 const int t = L;
                 const float *gp = GT + t * GTS;         // g_{t-1}
                 const float *gt = GT + (t + 1) * GTS;   // g_t
 #pragma unroll 1
-                for (int g8 = 0; g8 < 4; ++g8) {
-                    const int j0 = 32 * h + 8 * g8;
+                for (int g = 0; g < 2; ++g) {
+                    const int j0 = c16 + 8 * g;
                     float kk8[8], k8[8], v[8], ki[8];
                     in_row8(IN + XKK * 8192, t, j0, kk8);
                     in_row8(IN + XK * 8192, t, j0, k8);
@@ -261,96 +300,98 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                         v[e] = to_tf32(kk8[e] * gpv[e]);
                         ki[e] = to_tf32(k8[e] * __fdividef(1.f, gtv[e]));
                     }
-                    tmem_st8(tmem_addr(tb, Lq, T_A1 + j0), v);
-                    st_f4(sm + OFF_B6, sw128_off(t, j0, 64), v[0], v[1], v[2], v[3]);
-                    st_f4(sm + OFF_B6, sw128_off(t, j0 + 4, 64), v[4], v[5], v[6], v[7]);
+                    st_f4(sm + OFF_A1, sw128_off(t, j0, 128), v[0], v[1], v[2], v[3]);
+                    st_f4(sm + OFF_A1, sw128_off(t, j0 + 4, 128), v[4], v[5], v[6], v[7]);
                     st_f4(sm + OFF_B1, sw128_off(64 + t, j0, 128), ki[0], ki[1], ki[2], ki[3]);
                     st_f4(sm + OFF_B1, sw128_off(64 + t, j0 + 4, 128), ki[4], ki[5], ki[6], ki[7]);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[e] = (j0 + e == t) ? 1.f : 0.f;
+                    tmem_st8(tmem_addr(tb, Lq, T_D3 + j0), v);
                 }
             } else {
                 const int t = L - 64;
                 const float *gt = GT + (t + 1) * GTS;   // g_t
                 float bon = 0.f, dk = 0.f, db = 0.f;
 #pragma unroll 1
-                for (int g8 = 0; g8 < 4; ++g8) {
-                    const int j0 = 32 * h + 8 * g8;
-                    float r8[8], kk8[8], a8[8], k8[8], g8v[8], rd[8], bi[8];
+                for (int g = 0; g < 2; ++g) {
+                    const int j0 = c16 + 8 * g;
+                    float r8[8], kk8[8], a8[8], k8[8], rd[8], bi[8];
                     in_row8(IN + XR * 8192, t, j0, r8);
                     in_row8(IN + XKK * 8192, t, j0, kk8);
                     in_row8(IN + XA * 8192, t, j0, a8);
                     in_row8(IN + XK * 8192, t, j0, k8);
-                    {
-                        const float4 ga = *reinterpret_cast<const float4 *>(gt + j0);
-                        const float4 gb = *reinterpret_cast<const float4 *>(gt + j0 + 4);
-                        g8v[0] = ga.x; g8v[1] = ga.y; g8v[2] = ga.z; g8v[3] = ga.w;
-                        g8v[4] = gb.x; g8v[5] = gb.y; g8v[6] = gb.z; g8v[7] = gb.w;
-                    }
+                    const float4 ga = *reinterpret_cast<const float4 *>(gt + j0);
+                    const float4 gb = *reinterpret_cast<const float4 *>(gt + j0 + 4);
+                    const float g8v[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float ig = __fdividef(1.f, g8v[e]);
                         const float bb = kk8[e] * a8[e];
                         rd[e] = to_tf32(r8[e] * g8v[e]);
-                        bi[e] = to_tf32(bb * ig);
+                        bi[e] = to_tf32(bb * __fdividef(1.f, g8v[e]));
                         dk = fmaf(r8[e], k8[e], dk);
                         db = fmaf(r8[e], bb, db);
                         if (epi) bon = fmaf(r8[e] * k8[e], S.r_k[j0 + e], bon);
                     }
-                    tmem_st8(tmem_addr(tb, Lq, T_A1 + j0), rd);
+                    st_f4(sm + OFF_A1, sw128_off(64 + t, j0, 128), rd[0], rd[1], rd[2], rd[3]);
+                    st_f4(sm + OFF_A1, sw128_off(64 + t, j0 + 4, 128), rd[4], rd[5], rd[6], rd[7]);
+                    tmem_st8(tmem_addr(tb, Lq, T_D3 + j0), rd);
                     st_f4(sm + OFF_B1, sw128_off(t, j0, 128), bi[0], bi[1], bi[2], bi[3]);
                     st_f4(sm + OFF_B1, sw128_off(t, j0 + 4, 128), bi[4], bi[5], bi[6], bi[7]);
                 }
-                S.dk[h][t] = dk;
-                S.db[h][t] = db;
-                if (epi) S.bon[h][t] = bon;
+                S.dk[pq][t] = dk;
+                S.db[pq][t] = db;
+                if (epi) S.bon[pq][t] = bon;
             }
             sync_for_mma();
             if (tid == 0) {
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)   // R1: Grams = [KKd; Rd] [Bi; Ki]^T
-                    mma_tf32_ts(tb + T_D1, tb + T_A1 + 8 * ks, dB1 + kstep_off(ks, 128), idesc_tf32(128, 128), ks > 0);
+                    mma_tf32_ss(tb + T_D1, dA1 + kstep_off(ks, 128), dB1 + kstep_off(ks, 128), idesc_tf32(128, 128), ks > 0);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)   // R1b: transposed Grams [Bi; Ki] KKd^T
-                    mma_tf32_ss(tb + T_D2, dB1 + kstep_off(ks, 128), dB6 + kstep_off(ks, 64), idesc_tf32(128, 64), ks > 0);
+                    mma_tf32_ss(tb + T_D2, dB1 + kstep_off(ks, 128), dA1 + kstep_off(ks, 128), idesc_tf32(128, 64), ks > 0);
+                // transposes on the tensor core (exact: identity times tf32 operands):
+                // lanes 0-63 of T_A2 <- Bi^T (A of R2), of T_D3 cols 64-127 <- Ki^T (start of K~)
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_tf32_ts(tb + T_A2, tb + T_ID + 8 * ks, dB1 + kstep_off(ks, 128), idesc_tf32(128, 64), ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_tf32_ts(tb + T_D3 + 64, tb + T_ID + 8 * ks, dB1 + (8192 >> 4) + kstep_off(ks, 128),
+                                idesc_tf32(128, 64), ks > 0);
                 mma_commit(&S.bar_mma);
             }
             mma_pending = true;
-            // ---- P4 (while the Gram MMAs run): key-channel columns over tokens 32h..32h+31.
-            //      Lanes 0-63: Bc^T -> A2 rows (TMEM, T_D3) and Kc^T -> T_KC.
-            //      Lanes 64-127 (key j = L - 64): KKd^T -> B3 rows 0-63, V^T -> B4.
+            // ---- P4 (while the MMAs run): transposes through shared memory, no arithmetic.
+            //      Lanes 0-63 (key/value channel j = L): V^T row j -> B4.
+            //      Lanes 64-127 (key j = L - 64): KKd^T row j -> B3 rows 0-63.
             if (colg) {
                 const int j = L;
-                const float gCj = S.gC[j];
+                uint32_t xo[8];
+                col_offsets(j, xo);
 #pragma unroll 1
-                for (int g8 = 0; g8 < 4; ++g8) {
-                    const int t0 = 32 * h + 8 * g8;
-                    float bc[8], kc[8];
+                for (int g = 0; g < 2; ++g) {
+                    const int t0 = c16 + 8 * g;
+                    float vv[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int t = t0 + e;
-                        const float sc = __fdividef(gCj, GT[(t + 1) * GTS + j]);   // prod of w after t
-                        bc[e] = to_tf32(in_elem(IN + XKK * 8192, t, j) * in_elem(IN + XA * 8192, t, j) * sc);
-                        kc[e] = to_tf32(in_elem(IN + XK * 8192, t, j) * sc);
-                    }
-                    tmem_st8(tmem_addr(tb, Lq, T_D3 + t0), bc);
-                    tmem_st8(tmem_addr(tb, Lq, T_KC + t0), kc);
+                    for (int e = 0; e < 8; ++e) vv[e] = in_col(IN + XV * 8192, t0 + e, xo, e);
+                    st_f4(sm + OFF_B4, sw128_off(j, t0, 64), vv[0], vv[1], vv[2], vv[3]);
+                    st_f4(sm + OFF_B4, sw128_off(j, t0 + 4, 64), vv[4], vv[5], vv[6], vv[7]);
                 }
             } else {
                 const int j = L - 64;
+                uint32_t xo[8];
+                kcol_offsets(j, 128, xo);
+                const uint8_t *b6 = sm + OFF_A1;
 #pragma unroll 1
-                for (int g8 = 0; g8 < 4; ++g8) {
-                    const int t0 = 32 * h + 8 * g8;
-                    float kkd[8], vv[8];
+                for (int g = 0; g < 2; ++g) {
+                    const int t0 = c16 + 8 * g;
+                    float kkd[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int t = t0 + e;
-                        kkd[e] = to_tf32(in_elem(IN + XKK * 8192, t, j) * GT[t * GTS + j]);   // kk * g_{t-1}
-                        vv[e] = in_elem(IN + XV * 8192, t, j);
-                    }
+                    for (int e = 0; e < 8; ++e) kkd[e] = *reinterpret_cast<const float *>(b6 + (t0 + e) * 128 + xo[e]);
                     st_f4(sm + OFF_B3, sw128_off(j, t0, 128), kkd[0], kkd[1], kkd[2], kkd[3]);
                     st_f4(sm + OFF_B3, sw128_off(j, t0 + 4, 128), kkd[4], kkd[5], kkd[6], kkd[7]);
-                    st_f4(sm + OFF_B4, sw128_off(j, t0, 64), vv[0], vv[1], vv[2], vv[3]);
-                    st_f4(sm + OFF_B4, sw128_off(j, t0 + 4, 64), vv[4], vv[5], vv[6], vv[7]);
                 }
             }
             if (wait_mma()) { failed = true; break; }
@@ -359,8 +400,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
             if (colg) {
                 const int t = L;
 #pragma unroll 1
-                for (int g8 = 0; g8 < 4; ++g8) {
-                    const int s0 = 32 * h + 8 * g8;
+                for (int g = 0; g < 2; ++g) {
+                    const int s0 = c16 + 8 * g;
                     float m[8];
                     tmem_ld8(tmem_addr(tb, Lq, T_D1 + s0), m);
 #pragma unroll
@@ -370,19 +411,27 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 }
             } else {
                 const int t = L - 64;
-                // the current-token entry is taken exactly in fp32: it dominates short sequences
-                const float diag = S.db[0][t] + S.db[1][t];
+                // the current-token entries are taken exactly in fp32: they dominate short sequences
+                const float dgb = to_tf32(S.db[0][t] + S.db[1][t] + S.db[2][t] + S.db[3][t]);
+                const float dgk = S.dk[0][t] + S.dk[1][t] + S.dk[2][t] + S.dk[3][t];
 #pragma unroll 1
-                for (int g8 = 0; g8 < 4; ++g8) {
-                    const int s0 = 32 * h + 8 * g8;
+                for (int g = 0; g < 2; ++g) {
+                    const int s0 = c16 + 8 * g;
                     float m[8];
-                    tmem_ld8(tmem_addr(tb, Lq, T_D1 + s0), m);
+                    tmem_ld8(tmem_addr(tb, Lq, T_D1 + s0), m);          // Q_b row t
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int ss = s0 + e;
-                        m[e] = ss < t ? to_tf32(m[e]) : (ss == t ? to_tf32(diag) : 0.f);
+                        m[e] = ss < t ? to_tf32(m[e]) : (ss == t ? dgb : 0.f);
                     }
-                    tmem_st8(tmem_addr(tb, Lq, T_D3 + s0), m);
+                    tmem_st8(tmem_addr(tb, Lq, T_A2 + s0), m);
+                    tmem_ld8(tmem_addr(tb, Lq, T_D1 + 64 + s0), m);     // Q_k row t
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int ss = s0 + e;
+                        m[e] = ss < t ? m[e] : (ss == t ? dgk : 0.f);
+                    }
+                    tmem_st8(tmem_addr(tb, Lq, T_D3 + 64 + s0), m);
                     // row t of M_kb^T: M_kb[t'][t] for tokens t' = s0..s0+7 (nonzero for t' > t)
                     tmem_ld8(tmem_addr(tb, Lq, T_D2 + s0), m);
 #pragma unroll
@@ -455,8 +504,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
             }
             __syncthreads();
             // level 2: Y[1][0] = -Y1 (L[32:64][0:32] Y0). Y0, Y1 are lower triangular, so the
-            // fixed-length sums are exact. Each thread: one row, four adjacent columns.
-            {
+            // fixed-length sums are exact. Threads 0-255: one row, four adjacent columns each.
+            if (tid < 256) {
                 const int i = tid >> 3, j4 = (tid & 7) * 4;
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
@@ -469,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 *reinterpret_cast<float4 *>(Tw2 + i * 36 + j4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
             }
             __syncthreads();
-            {
+            if (tid < 256) {
                 const int i = tid >> 3, j4 = (tid & 7) * 4;
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
@@ -492,84 +541,30 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
             if (tid == 0) {
                 tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)   // R2: Z = [Bc^T; Q_b] A
-                    mma_tf32_ts(tb + T_D2, tb + T_D3 + 8 * ks, dB2 + kstep_off(ks, 64),
-                                idesc_tf32(128, 64), ks > 0);
+                for (int ks = 0; ks < 8; ++ks)   // R2: Z = [Bi^T; Q_b] A
+                    mma_tf32_ts(tb + T_D2, tb + T_A2 + 8 * ks, dB2 + kstep_off(ks, 64), idesc_tf32(128, 64), ks > 0);
                 mma_commit(&S.bar_mma);
             }
             mma_pending = true;
             if (wait_mma()) { failed = true; break; }
-            // round Z to tf32 in place (it is the next A operand)
-#pragma unroll 1
-            for (int g8 = 0; g8 < 4; ++g8) {
-                float z[8];
-                tmem_ld8(tmem_addr(tb, Lq, T_D2 + 32 * h + 8 * g8), z);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) z[e] = to_tf32(z[e]);
-                tmem_st8(tmem_addr(tb, Lq, T_D2 + 32 * h + 8 * g8), z);
-            }
-            sync_for_mma();
             if (tid == 0) {
                 tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)   // R3: X = Z [KKd | M_kb]
+                for (int ks = 0; ks < 8; ++ks)   // R3: T_D3 -= Z [KKd | M_kb]
                     mma_tf32_ts(tb + T_D3, tb + T_D2 + 8 * ks, dB3 + kstep_off(ks, 128),
-                                idesc_tf32(128, 128), ks > 0);
+                                idesc_neg_a(idesc_tf32(128, 128)), 1);
                 mma_commit(&S.bar_mma);
             }
             mma_pending = true;
             if (wait_mma()) { failed = true; break; }
-            // ---- P, K~ (column group, key j) and R~, Q~ (row group, token t), in place
-            if (colg) {
-                const int j = L;
-                const float gCj = S.gC[j];
-#pragma unroll 1
-                for (int g8 = 0; g8 < 4; ++g8) {
-                    const int c8 = 32 * h + 8 * g8;
-                    float d[8], e8[8];
-                    tmem_ld8(tmem_addr(tb, Lq, T_D3 + c8), d);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) d[e] = to_tf32((c8 + e == j ? gCj : 0.f) - d[e]);
-                    tmem_st8(tmem_addr(tb, Lq, T_D3 + c8), d);
-                    tmem_ld8(tmem_addr(tb, Lq, T_D3 + 64 + c8), d);
-                    tmem_ld8(tmem_addr(tb, Lq, T_KC + c8), e8);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) d[e] = to_tf32(e8[e] - d[e]);
-                    tmem_st8(tmem_addr(tb, Lq, T_D3 + 64 + c8), d);
-                }
-            } else {
-                const int t = L - 64;
-                const float diag = S.dk[0][t] + S.dk[1][t];
-#pragma unroll 1
-                for (int g8 = 0; g8 < 4; ++g8) {
-                    const int c8 = 32 * h + 8 * g8;
-                    float d[8], e8[8];
-                    tmem_ld8(tmem_addr(tb, Lq, T_D3 + c8), d);
-                    tmem_ld8(tmem_addr(tb, Lq, T_A1 + c8), e8);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) d[e] = to_tf32(e8[e] - d[e]);
-                    tmem_st8(tmem_addr(tb, Lq, T_D3 + c8), d);
-                    tmem_ld8(tmem_addr(tb, Lq, T_D3 + 64 + c8), d);
-                    tmem_ld8(tmem_addr(tb, Lq, T_D1 + 64 + c8), e8);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int ss = c8 + e;
-                        d[e] = to_tf32((ss < t ? e8[e] : (ss == t ? diag : 0.f)) - d[e]);
-                    }
-                    tmem_st8(tmem_addr(tb, Lq, T_D3 + 64 + c8), d);
-                }
-            }
-            sync_for_mma();
             if (tid == 0) {
                 tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)   // R4: [K~; Q~] V
-                    mma_tf32_ts(tb + T_D4, tb + T_D3 + 64 + 8 * ks, dB4 + kstep_off(ks, 64),
-                                idesc_tf32(128, 64), ks > 0);
+                for (int ks = 0; ks < 8; ++ks)   // R4: [Ki^T - X; Q~] V
+                    mma_tf32_ts(tb + T_D4, tb + T_D3 + 64 + 8 * ks, dB4 + kstep_off(ks, 64), idesc_tf32(128, 64), ks > 0);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)   // R5: += [P; R~] S_0^T
-                    mma_tf32_ts(tb + T_D4, tb + T_D3 + 8 * ks, dB5 + kstep_off(ks, 64),
-                                idesc_tf32(128, 64), 1);
+                for (int ks = 0; ks < 8; ++ks)   // R5: += [I - X; R~] S_0^T
+                    mma_tf32_ts(tb + T_D4, tb + T_D3 + 8 * ks, dB5 + kstep_off(ks, 64), idesc_tf32(128, 64), 1);
                 mma_commit(&S.bar_mma);
             }
             mma_pending = true;
@@ -579,11 +574,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
             const bool snap = p.snap_every > 0 && done % p.snap_every == 0;
             if (colg) {
                 const int j = L;
+                const float gCj = S.gC[j];
+                uint32_t xo[8];
+                kcol_offsets(j, 64, xo);
+                uint8_t *b5 = sm + OFF_B5;
 #pragma unroll 1
-                for (int g8 = 0; g8 < 4; ++g8) {
-                    const int i0 = 32 * h + 8 * g8;
+                for (int g = 0; g < 2; ++g) {
+                    const int i0 = c16 + 8 * g;
                     float s8[8];
-                    tmem_ld8(tmem_addr(tb, Lq, T_D4 + i0), s8);    // S[i0+e][j]
+                    tmem_ld8(tmem_addr(tb, Lq, T_D4 + i0), s8);    // S'[i0+e][j]
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) s8[e] *= gCj;                // S_C = S' diag(gC)
                     if (last && p.S_T) {
 #pragma unroll
                         for (int e = 0; e < 8; ++e) p.S_T[size_t(unit) * 4096 + (i0 + e) * 64 + j] = s8[e];
@@ -594,54 +595,49 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                         for (int e = 0; e < 8; ++e) dst[(i0 + e) * 64 + j] = s8[e];
                     }
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        *reinterpret_cast<float *>(sm + OFF_B5 + sw128_off(i0 + e, j, 64)) = to_tf32(s8[e]);
+                    for (int e = 0; e < 8; ++e) *reinterpret_cast<float *>(b5 + (i0 + e) * 128 + xo[e]) = to_tf32(s8[e]);
                 }
             } else {
                 const int t = L - 64;
-                float *dst = p.y + ((size_t(b) * p.T + c0 + t) * p.H + hh) * 64 + 32 * h;
-                float mean = 0.f, inv = 1.f, bon = 0.f;
-                if (epi) {
-                    float s1 = 0.f, s2 = 0.f;
-#pragma unroll 1
-                    for (int g8 = 0; g8 < 4; ++g8) {
-                        float y8[8];
-                        tmem_ld8(tmem_addr(tb, Lq, T_D4 + 32 * h + 8 * g8), y8);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) s1 += y8[e];
-                    }
-                    S.red[h][t] = s1;
-                    named_bar_rows();
-                    mean = (S.red[0][t] + S.red[1][t]) * (1.f / 64.f);
-                    named_bar_rows();
-#pragma unroll 1
-                    for (int g8 = 0; g8 < 4; ++g8) {
-                        float y8[8];
-                        tmem_ld8(tmem_addr(tb, Lq, T_D4 + 32 * h + 8 * g8), y8);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) s2 = fmaf(y8[e] - mean, y8[e] - mean, s2);
-                    }
-                    S.red[h][t] = s2;
-                    named_bar_rows();
-                    inv = 1.f / sqrtf((S.red[0][t] + S.red[1][t]) * (1.f / 64.f) + p.gn_eps);
-                    bon = S.bon[0][t] + S.bon[1][t];
-                }
-#pragma unroll 1
-                for (int g8 = 0; g8 < 4; ++g8) {
-                    const int i0 = 32 * h + 8 * g8;
+                float *dst = p.y + ((size_t(b) * p.T + c0 + t) * p.H + hh) * 64 + c16;
+                float yv[16];
+                {
                     float y8[8];
-                    tmem_ld8(tmem_addr(tb, Lq, T_D4 + i0), y8);   // y_t[i0 + e]
-                    if (epi) {
+                    tmem_ld8(tmem_addr(tb, Lq, T_D4 + c16), y8);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float v = *reinterpret_cast<const float *>(sm + OFF_B4 + sw128_off(i0 + e, t, 64));
-                            y8[e] = fmaf((y8[e] - mean) * inv, S.ln_w[i0 + e], S.ln_b[i0 + e]) + bon * v;
-                        }
+                    for (int e = 0; e < 8; ++e) yv[e] = y8[e];
+                    tmem_ld8(tmem_addr(tb, Lq, T_D4 + c16 + 8), y8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) yv[8 + e] = y8[e];
+                }
+                if (epi) {
+                    uint32_t xo[8];
+                    kcol_offsets(t, 64, xo);
+                    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) s1 += yv[e];
+                    S.red[pq][t] = s1;
+                    named_bar_rows();
+                    const float mean = (S.red[0][t] + S.red[1][t] + S.red[2][t] + S.red[3][t]) * (1.f / 64.f);
+                    named_bar_rows();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) s2 = fmaf(yv[e] - mean, yv[e] - mean, s2);
+                    S.red[pq][t] = s2;
+                    named_bar_rows();
+                    const float inv =
+                        1.f / sqrtf((S.red[0][t] + S.red[1][t] + S.red[2][t] + S.red[3][t]) * (1.f / 64.f) + p.gn_eps);
+                    const float bon = S.bon[0][t] + S.bon[1][t] + S.bon[2][t] + S.bon[3][t];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int ii = c16 + e;
+                        const float v = *reinterpret_cast<const float *>(sm + OFF_B4 + ii * 128 + xo[e & 7]);
+                        yv[e] = fmaf((yv[e] - mean) * inv, S.ln_w[ii], S.ln_b[ii]) + bon * v;
                     }
-                    if (t < Lc) {
-                        *reinterpret_cast<float4 *>(dst + 8 * g8) = make_float4(y8[0], y8[1], y8[2], y8[3]);
-                        *reinterpret_cast<float4 *>(dst + 8 * g8 + 4) = make_float4(y8[4], y8[5], y8[6], y8[7]);
-                    }
+                }
+                if (t < Lc) {
+#pragma unroll
+                    for (int m = 0; m < 4; ++m)
+                        *reinterpret_cast<float4 *>(dst + 4 * m) = make_float4(yv[4 * m], yv[4 * m + 1], yv[4 * m + 2], yv[4 * m + 3]);
                 }
             }
             sync_for_mma();
