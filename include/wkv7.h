@@ -54,6 +54,7 @@ extern "C" {
 
 #define WKV7_ABI_VERSION 1
 #define WKV7_HEAD_SIZE 64
+#define WKV7_MAX_SEGMENTS 8   /* CTAs per (b, h) of WKV7_ALGO_SPLIT (one thread-block cluster) */
 
 typedef enum wkv7_status {
     WKV7_OK = 0,
@@ -75,7 +76,12 @@ typedef enum wkv7_algo {
     WKV7_ALGO_SEQ = 1,    /* token-by-token scan, fp32 FMA; any T, any dtype             */
     WKV7_ALGO_CHUNK = 2,  /* chunked prefill on tcgen05 tensor cores, fp32 chunk carry;  */
                           /* bf16 inputs, chunk 64, w >= exp(-e^-1/2) as on the pages      */
-    WKV7_ALGO_SPLIT = 3   /* chunked prefill with T split into segments across CTAs      */
+    WKV7_ALGO_SPLIT = 3   /* chunked prefill with the chunks of one (b, h) spread over   */
+                          /* `segments` CTAs of a thread-block cluster: CTA r takes      */
+                          /* chunks r, r + segments, ... and passes the fp32 state to    */
+                          /* CTA r + 1 through distributed shared memory (chunk carry    */
+                          /* S_{c+1} = S_c P_c + Q_c, the chain being the only serial    */
+                          /* part); same inputs and limits as CHUNK                      */
 } wkv7_algo;
 
 /* Options of wkv7_forward. Obtain defaults with wkv7_opts_default(). */
@@ -88,7 +94,8 @@ typedef struct wkv7_opts {
     const float *ln_b;
     const float *r_k;
     float gn_eps;         /* epilogue epsilon added to the variance (default 64e-5)      */
-    int segments;         /* WKV7_ALGO_SPLIT: T segments per (b, h); 0 = automatic       */
+    int segments;         /* WKV7_ALGO_SPLIT: CTAs per (b, h), 1..WKV7_MAX_SEGMENTS, or  */
+                          /* 0 = automatic (AUTO always chooses; CHUNK uses one)         */
 } wkv7_opts;
 
 /* Fills *opts with the defaults: AUTO, default chunk, no snapshots, no epilogue,

@@ -154,7 +154,8 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype dt, const void *
     if (n_epi != 0 && n_epi != 3) return fail(WKV7_ERR_ARG, "epilogue needs all of ln_w, ln_b, r_k (or none)");
     if (n_epi == 3 && !(std::isfinite(opts.gn_eps) && opts.gn_eps >= 0.f))
         return fail(WKV7_ERR_ARG, "gn_eps must be finite and >= 0");
-    if (opts.segments < 0) return fail(WKV7_ERR_ARG, "segments=%d < 0", opts.segments);
+    if (opts.segments < 0 || opts.segments > WKV7_MAX_SEGMENTS)
+        return fail(WKV7_ERR_ARG, "segments=%d outside 0..%d", opts.segments, WKV7_MAX_SEGMENTS);
 
     size_t tok = 1, st = 1;
     if (!mul_ok(tok, B) || !mul_ok(tok, T) || !mul_ok(tok, H) || !mul_ok(tok, N) || !mul_ok(st, B) ||
@@ -214,7 +215,8 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype dt, const void *
     p.snap_every = n_snap ? opts.snap_every : 0;
     p.snaps = n_snap ? opts.snapshots : nullptr;
     p.ln_w = opts.ln_w; p.ln_b = opts.ln_b; p.r_k = opts.r_k; p.gn_eps = opts.gn_eps;
-    p.chunk = opts.chunk; p.segments = opts.segments;
+    p.chunk = opts.chunk;
+    p.segments = opts.algo == WKV7_ALGO_CHUNK ? 1 : (opts.algo == WKV7_ALGO_SPLIT ? opts.segments : 0);
     p.ws = workspace; p.ws_bytes = workspace_bytes;
     p.stream = static_cast<cudaStream_t>(stream);
 

@@ -55,6 +55,8 @@ using namespace tc;
 
 constexpr int C = 64;             // chunk length (tokens)
 constexpr int kThreads = 512;   // 16 warps: 4 per SM sub-partition
+constexpr int kColThreads = 256;  // threads owning TMEM lanes 0-63: they write the next state
+constexpr int kMaxSegments = WKV7_MAX_SEGMENTS;   // CTAs per (b, h) in split mode (portable cluster size)
 constexpr int GTS = 68;           // row stride (floats) of the decay table: conflict-free row reads
 constexpr int LWS = 68;           // row stride of the inverse workspaces (16-byte aligned rows)
 
@@ -79,6 +81,7 @@ struct Small {
     float ln_w[C], ln_b[C], r_k[C];
     uint64_t bar_tma;
     uint64_t bar_mma;
+    uint64_t bar_state;   // split mode: the carried state has arrived in B5 (kColThreads remote arrivals)
     uint32_t tmem_base;
 };
 constexpr uint32_t SMEM_BYTES = OFF_SMALL + sizeof(Small) + 1024;   // + alignment slack
@@ -164,9 +167,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     const int nchunks = (p.T + C - 1) / C;
     const bool epi = p.ln_w != nullptr;
 
+    // Split mode: the CTAs of a cluster share each (b, h); CTA `rank` takes chunks rank,
+    // rank + cs, ... and hands the state after each of them to CTA rank + 1 (mod cs).
+    const int cs = int(cluster_size()), rank = int(cluster_rank());
+    const int cid = int(cluster_index()), ncl = int(cluster_count());
     if (tid == 0) {
         mbar_init(&S.bar_tma, 1);
         mbar_init(&S.bar_mma, 1);
+        mbar_init(&S.bar_state, kColThreads);
         mbar_fence_init();
     }
     if (warp == 0) {
@@ -175,8 +183,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     }
     tc_fence_before();
     __syncthreads();
+    if (cs > 1) cluster_sync();   // every CTA's barriers are initialised before anyone arrives remotely
     tc_fence_after();
     const uint32_t tb = S.tmem_base;
+    const int next_rank = rank + 1 == cs ? 0 : rank + 1;
+    const uint32_t next_b5 = map_to_rank(smem_u32(sm + OFF_B5), uint32_t(next_rank));
+    const uint32_t next_bar = map_to_rank(smem_u32(&S.bar_state), uint32_t(next_rank));
     // matrix descriptors of the shared-memory operands at K-step 0
     const uint64_t dB1 = desc_sw128(smem_u32(sm + OFF_B1)), dB2 = desc_sw128(smem_u32(sm + OFF_B2));
     const uint64_t dB3 = desc_sw128(smem_u32(sm + OFF_B3)), dB4 = desc_sw128(smem_u32(sm + OFF_B4));
@@ -192,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         }
         tmem_st_wait();
     }
-    uint32_t tma_parity = 0, mma_parity = 0;
+    uint32_t tma_parity = 0, mma_parity = 0, state_parity = 0;
     bool tma_pending = false, mma_pending = false, failed = false;
 
     auto issue_tma = [&](int u, int c) {   // thread 0
@@ -201,12 +213,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
 #pragma unroll
         for (int x = 0; x < 6; ++x) tma_load_4d(sm + OFF_IN + x * 8192, &maps.m[x], &S.bar_tma, 0, hh, c * C, b);
     };
-    auto wait_mma = [&]() -> bool {        // all threads; true on timeout (uniform across the CTA)
+    // all threads; true on timeout here or (`extra`) in any thread (uniform across the CTA)
+    auto wait_mma = [&](bool extra = false) -> bool {
         const bool to = !mbar_wait(&S.bar_mma, mma_parity, p.timeout_ns);
         mma_parity ^= 1u;
         mma_pending = false;
         tc_fence_after();
-        return __syncthreads_or(to) != 0;
+        return __syncthreads_or(to || extra) != 0;
     };
     auto sync_for_mma = [&]() {            // writes to smem/TMEM -> visible to the next MMA
         fence_proxy_async_smem();
@@ -215,14 +228,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         __syncthreads();
     };
 
-    int unit = blockIdx.x;
-    if (tid == 0 && unit < units) issue_tma(unit, 0);
-    tma_pending = unit < units;
+    int unit = cid;
+    tma_pending = unit < units && rank < nchunks;
+    if (tid == 0 && tma_pending) issue_tma(unit, rank);
 
-    for (; unit < units && !failed; unit += gridDim.x) {
+    for (; unit < units && !failed; unit += ncl) {
         const int b = unit / p.H, hh = unit % p.H;
-        // state operand S_0 (row = value channel i, K = key channel j), tf32-rounded
-        for (int e = tid; e < 1024; e += kThreads) {
+        // state operand S_0 (row = value channel i, K = key channel j), tf32-rounded; in split
+        // mode only the CTA that takes chunk 0 loads it, the others receive their states
+        for (int e = (rank == 0 ? tid : 1024); e < 1024; e += kThreads) {
             const int i = e >> 4, j4 = (e & 15) * 4;
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
             if (p.S0) x = __ldg(reinterpret_cast<const float4 *>(p.S0 + size_t(unit) * 4096 + i * 64 + j4));
@@ -234,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
             S.r_k[tid] = p.r_k[hh * 64 + tid];
         }
 
-        for (int c = 0; c < nchunks; ++c) {
+        for (int c = rank; c < nchunks && !failed; c += cs) {
             const int c0 = c * C, Lc = min(C, p.T - c0);
             const bool last = c == nchunks - 1;
             {   // ---- inputs of this chunk
@@ -441,12 +455,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 }
             }
             sync_for_mma();
-            if (tid == 0) {
-                // input tiles and decay table are consumed: prefetch the next chunk (or next head)
-                if (!last) issue_tma(unit, c + 1);
-                else if (unit + int(gridDim.x) < units) issue_tma(unit + gridDim.x, 0);
+            {   // input tiles and decay table are consumed: prefetch this CTA's next chunk
+                int nu = unit, nc = c + cs;
+                if (nc >= nchunks) { nu = unit + ncl; nc = rank; }
+                tma_pending = nu < units && nc < nchunks;
+                if (tid == 0 && tma_pending) issue_tma(nu, nc);
             }
-            tma_pending = !last || unit + int(gridDim.x) < units;
             // ---- A = (I + M_ab)^{-1}. Diagonal 16x16 blocks: one thread per (block, column)
             //      solves (I + L_dd) x = e_c by forward substitution in registers (warps 2, 3).
             if (tid >= 64 && tid < 128) {
@@ -557,18 +571,29 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
             }
             mma_pending = true;
             if (wait_mma()) { failed = true; break; }
+            const bool recv = cs > 1 && c > 0;   // split mode: this chunk's start state comes from CTA rank-1
+            bool state_to = false;
             if (tid == 0) {
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)   // R4: [Ki^T - X; Q~] V
                     mma_tf32_ts(tb + T_D4, tb + T_D3 + 64 + 8 * ks, dB4 + kstep_off(ks, 64), idesc_tf32(128, 64), ks > 0);
+                if (recv) {
+                    // the only wait on another CTA: everything above used this chunk's inputs only
+                    state_to = !mbar_wait_cluster(&S.bar_state, state_parity, p.timeout_ns);
+                    fence_proxy_async_smem();
+                    tc_fence_after();
+                }
+                if (!state_to) {
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)   // R5: += [I - X; R~] S_0^T
-                    mma_tf32_ts(tb + T_D4, tb + T_D3 + 8 * ks, dB5 + kstep_off(ks, 64), idesc_tf32(128, 64), 1);
+                    for (int ks = 0; ks < 8; ++ks)   // R5: += [I - X; R~] S_0^T
+                        mma_tf32_ts(tb + T_D4, tb + T_D3 + 8 * ks, dB5 + kstep_off(ks, 64), idesc_tf32(128, 64), 1);
+                }
                 mma_commit(&S.bar_mma);
             }
+            if (recv) state_parity ^= 1u;
             mma_pending = true;
-            if (wait_mma()) { failed = true; break; }
+            if (wait_mma(state_to)) { failed = true; break; }
             // ---- new state -> B5 (+ S_T / snapshot); readout -> epilogue -> y
             const int done = c0 + Lc;
             const bool snap = p.snap_every > 0 && done % p.snap_every == 0;
@@ -578,6 +603,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 uint32_t xo[8];
                 kcol_offsets(j, 64, xo);
                 uint8_t *b5 = sm + OFF_B5;
+                // split mode: the state goes straight into the next CTA's B5 (distributed shared memory)
+                const bool send = cs > 1 && c + 1 < nchunks;
 #pragma unroll 1
                 for (int g = 0; g < 2; ++g) {
                     const int i0 = c16 + 8 * g;
@@ -585,6 +612,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                     tmem_ld8(tmem_addr(tb, Lq, T_D4 + i0), s8);    // S'[i0+e][j]
 #pragma unroll
                     for (int e = 0; e < 8; ++e) s8[e] *= gCj;                // S_C = S' diag(gC)
+                    if (send) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) st_cluster(next_b5 + (i0 + e) * 128 + xo[e], to_tf32(s8[e]));
+                        if (g == 1) {
+                            fence_proxy_async_cluster();
+                            mbar_arrive_remote(next_bar);
+                        }
+                    }
                     if (last && p.S_T) {
 #pragma unroll
                         for (int e = 0; e < 8; ++e) p.S_T[size_t(unit) * 4096 + (i0 + e) * 64 + j] = s8[e];
@@ -594,8 +629,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
 #pragma unroll
                         for (int e = 0; e < 8; ++e) dst[(i0 + e) * 64 + j] = s8[e];
                     }
+                    if (cs == 1) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) *reinterpret_cast<float *>(b5 + (i0 + e) * 128 + xo[e]) = to_tf32(s8[e]);
+                        for (int e = 0; e < 8; ++e) *reinterpret_cast<float *>(b5 + (i0 + e) * 128 + xo[e]) = to_tf32(s8[e]);
+                    }
                 }
             } else {
                 const int t = L - 64;
@@ -653,6 +690,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tb, 512);
+    // no CTA leaves while another CTA of its cluster may still write to its shared memory
+    if (cs > 1) cluster_sync();
 }
 
 // ---- host side ---------------------------------------------------------------------------------------
@@ -675,7 +714,23 @@ struct DeviceInfo {
     int sms = 0;
     unsigned int *err = nullptr;
     bool attr_set = false;
+    int clusters[kMaxSegments + 1] = {};   // co-resident clusters of each size (0: that size does not fit)
 };
+
+cudaLaunchConfig_t launch_config(int grid, int cs, cudaStream_t stream, cudaLaunchAttribute *attr) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(unsigned(grid), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = stream;
+    attr->id = cudaLaunchAttributeClusterDimension;
+    attr->val.clusterDim.x = unsigned(cs);
+    attr->val.clusterDim.y = 1;
+    attr->val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+}
 
 cudaError_t device_info(DeviceInfo *&out) {
     static std::mutex mu;
@@ -692,10 +747,41 @@ cudaError_t device_info(DeviceInfo *&out) {
         if ((e = cudaFuncSetAttribute(chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_BYTES))) !=
             cudaSuccess)
             return e;
+        d.clusters[1] = d.sms;
+        for (int cs = 2; cs <= kMaxSegments; ++cs) {
+            cudaLaunchAttribute attr;
+            const cudaLaunchConfig_t cfg = launch_config(cs * (d.sms / cs), cs, nullptr, &attr);
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, chunk_kernel, &cfg) != cudaSuccess) {
+                cudaGetLastError();
+                n = 0;
+            }
+            d.clusters[cs] = n;
+        }
         d.attr_set = true;
     }
     out = &d;
     return cudaSuccess;
+}
+
+// CTAs per (b, h). Each CTA of a cluster runs every cs-th chunk, so a head takes about
+// ceil(nchunks / cs) chunk times plus the hand-off latency, and the heads run in
+// ceil(units / clusters) waves. Pick the size with the smallest estimate (ties: fewer CTAs);
+// the 8% and 0.15-chunk terms are the measured cost of the hand-off per chunk and per head.
+int choose_segments(int units, int nchunks, const DeviceInfo &d) {
+    int best = 1;
+    double best_cost = 1e300;
+    for (int cs = 1; cs <= kMaxSegments; ++cs) {
+        if (d.clusters[cs] <= 0) continue;
+        const double waves = double((units + d.clusters[cs] - 1) / d.clusters[cs]);
+        const double per = double((nchunks + cs - 1) / cs);
+        const double cost = waves * (per * (cs > 1 ? 1.08 : 1.0) + 0.15 * (cs - 1));
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = cs;
+        }
+    }
+    return best;
 }
 
 }  // namespace
@@ -730,10 +816,13 @@ cudaError_t launch_chunk(const FwdArgs &p) {
     a.ln_w = p.ln_w; a.ln_b = p.ln_b; a.r_k = p.r_k; a.gn_eps = p.gn_eps;
     a.err = di->err;
     a.timeout_ns = 2000000000ull;
-    const int units = p.B * p.H;
-    const int grid = units < di->sms ? units : di->sms;
-    chunk_kernel<<<grid, kThreads, SMEM_BYTES, p.stream>>>(maps, a);
-    return cudaGetLastError();
+    const int units = p.B * p.H, nchunks = (p.T + C - 1) / C;
+    const int cs = p.segments > 0 ? p.segments : choose_segments(units, nchunks, *di);
+    if (cs > kMaxSegments || di->clusters[cs] <= 0) return cudaErrorInvalidClusterSize;
+    const int ncl = units < di->clusters[cs] ? units : di->clusters[cs];
+    cudaLaunchAttribute attr;
+    const cudaLaunchConfig_t cfg = launch_config(ncl * cs, cs, p.stream, &attr);
+    return cudaLaunchKernelEx(&cfg, chunk_kernel, maps, a);
 }
 
 cudaError_t read_device_error(cudaStream_t stream, unsigned int *value, bool clear) {

@@ -24,7 +24,7 @@ struct FwdArgs {
     const float *ln_w, *ln_b, *r_k;   // all null = no epilogue
     float gn_eps;
     int chunk;
-    int segments;
+    int segments;          // CTAs per (b, h) on the chunked path; 0 = automatic
     void *ws;
     size_t ws_bytes;
     cudaStream_t stream;

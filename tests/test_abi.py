@@ -75,7 +75,8 @@ def test_forward_rejects_bad_arguments(lib, kw, status):
     assert lib.wkv7_last_error() != b""
 
 
-@pytest.mark.parametrize("field,value", [("algo", 9), ("chunk", 24), ("snap_every", -1), ("segments", -2)])
+@pytest.mark.parametrize("field,value", [("algo", 9), ("chunk", 24), ("snap_every", -1), ("segments", -2),
+                                         ("segments", 9)])
 def test_forward_rejects_bad_options(lib, field, value):
     o = wkv7.Opts()
     lib.wkv7_opts_default(ctypes.byref(o))

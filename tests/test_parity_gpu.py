@@ -12,7 +12,8 @@ from tests.parity_util import TOL, as_np, heads_slice, snaps_err, state_err, y_e
 
 pytestmark = pytest.mark.gpu
 
-ALGOS_ANY = ["seq", "chunk"]      # algorithms that accept bf16 inputs
+ALGOS_ANY = ["seq", "chunk", "split"]   # algorithms that accept bf16 inputs (split: automatic CTAs per head)
+CHUNKED = ("chunk", "split")
 
 
 def _dev(d, device):
@@ -43,8 +44,8 @@ def test_tiny_fp32_workload(cuda_device, algo):
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_ragged_lengths(cuda_device, algo, T, dtype):
     """Lengths that are not multiples of any tile, with a carried-in state."""
-    if dtype == "f32" and algo == "chunk":
-        pytest.skip("the chunked algorithm takes bf16 inputs")
+    if dtype == "f32" and algo in CHUNKED:
+        pytest.skip("the chunked algorithms take bf16 inputs")
     wl = inputs.WORKLOADS[1]
     d = inputs.make_inputs(wl, B=2, T=T, H=3, dtype=dtype, seed=1000 + T)
     y_ref, S_ref, _ = _oracle(d)
@@ -316,4 +317,38 @@ def test_chunk_rejects_unsupported_requests(cuda_device):
 def test_no_device_error_after_runs(cuda_device):
     d = _dev(inputs.make_inputs(inputs.WORKLOADS[1], B=1, T=64, H=2, seed=24), cuda_device)
     _gpu(d, algo="chunk")
+    wkv7.poll_device_error()
+
+
+@pytest.mark.parametrize("segments", [2, 3, 4, 7, 8])
+@pytest.mark.parametrize("T", [130, 64 * 9 + 17, 1024])
+def test_split_matches_oracle_and_single_cta(cuda_device, segments, T):
+    """Chunks of one head spread over a cluster of `segments` CTAs, the state handed on
+    through distributed shared memory: within tolerance of the oracle, and bit-identical
+    to the one-CTA chunked path (same operations in the same order, only the CTA differs).
+    Covers clusters wider than the chunk count (T = 130: three chunks), a ragged last
+    chunk, snapshots and S_T written by different CTAs, and the fused epilogue."""
+    wl = inputs.WORKLOADS[2]
+    d = _dev(inputs.make_inputs(wl, B=2, T=T, H=3, seed=30 + segments), cuda_device)
+    kw = dict(ln_w=d["ln_w"], ln_b=d["ln_b"], r_k=d["r_k"], snap_every=64)
+    y1, S1, sn1 = _gpu(d, algo="chunk", **kw)
+    ys, Ss, sns = _gpu(d, algo="split", segments=segments, **kw)
+    assert torch.equal(ys, y1) and torch.equal(Ss, S1) and torch.equal(sns, sn1)
+    dc = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    y_ref, S_ref, sn_ref = _oracle(dc, snap_every=64)
+    out_ref = native.epilogue(y_ref, dc["r"], dc["k"], dc["v"], dc["ln_w"], dc["ln_b"], dc["r_k"])
+    assert y_err(ys, out_ref) <= TOL["bf16"]
+    assert state_err(Ss, S_ref) <= TOL["bf16"]
+    assert snaps_err(sns, sn_ref) <= TOL["bf16"]
+    wkv7.poll_device_error()
+
+
+def test_split_many_heads_per_cluster(cuda_device):
+    """More heads than clusters: each cluster walks several heads, CTA 0 reloads S0 for
+    every head and the ring of hand-offs restarts at each head's first chunk."""
+    d = _dev(inputs.make_inputs(inputs.WORKLOADS[1], B=8, T=64 * 5 + 3, H=40, seed=31), cuda_device)
+    y1, S1, _ = _gpu(d, algo="chunk")
+    for seg in (2, 3, 8):
+        ys, Ss, _ = _gpu(d, algo="split", segments=seg)
+        assert torch.equal(ys, y1) and torch.equal(Ss, S1), seg
     wkv7.poll_device_error()
