@@ -61,12 +61,13 @@ constexpr int GTS = 68;           // row stride (floats) of the decay table: con
 constexpr int LWS = 68;           // row stride of the inverse workspaces (16-byte aligned rows)
 
 // Shared-memory layout (byte offsets from a 1024-byte aligned base).
-constexpr uint32_t OFF_B1 = 0;        // [Bi; Ki] 128x64 tf32 (B of R1, R1c, R1d; A of R1b); later the inverse workspace
-constexpr uint32_t OFF_B3 = 32768;    // [KKd^T | M_kb^T] 128x64 (B of R3)
+constexpr uint32_t OFF_B1 = 0;        // [Bi; Ki] 128x64 tf32 (B of R1 and of the transpose round); then the
+                                      // inverse workspace; then the y tile of the TMA store (2 x [64][32] fp32)
+constexpr uint32_t OFF_B3 = 32768;    // [M_kb^T; KKd^T] 128x64 (B of R3)
 constexpr uint32_t OFF_B2 = 65536;    // A^T 64x64 (B of R2)
 constexpr uint32_t OFF_B4 = 81920;    // V^T 64x64 (B of R4; exact bf16 values)
 constexpr uint32_t OFF_B5 = 98304;    // S 64x64, row = value channel (B of R5)
-constexpr uint32_t OFF_A1 = 114688;   // [KKd; Rd] 128x64 (A of R1; rows 0-63 are the B of R1b)
+constexpr uint32_t OFF_A1 = 114688;   // [KKd; Rd] 128x64 (A of R1)
 constexpr uint32_t OFF_IN = 147456;   // six bf16 [64][64] input tiles, TMA destination (swizzled)
 constexpr uint32_t OFF_GT = 196608;   // decay table [65][GTS] fp32; later the inverse [64][LWS]
 constexpr uint32_t OFF_SMALL = OFF_GT + 65 * GTS * 4;
@@ -87,24 +88,28 @@ struct Small {
 constexpr uint32_t SMEM_BYTES = OFF_SMALL + sizeof(Small) + 1024;   // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
-// TMEM columns (512 allocated).
-constexpr uint32_t T_D1 = 0;     // Grams [M_ab | M_kb ; Q_b | Q_k] (R1)
-constexpr uint32_t T_D2 = 128;   // transposed Grams [M_ab^T; M_kb^T] (R1b), then Z (R2)
-constexpr uint32_t T_D3 = 192;   // [I | Ki^T ; Rd | Q_k] -> R3 subtracts Z [KKd | M_kb] -> [I - X | Ki^T - X ; R~ | Q~]
+// TMEM columns (512 allocated). A tf32 MMA with N = 64 costs nearly as much issue time as one
+// with N = 128, so products that share an A operand are merged into N = 128 rounds.
+constexpr uint32_t T_D1 = 0;     // Grams [M_ab | M_kb ; Q_b | Q_k] (R1); once read, Z (R2, 64 columns)
+constexpr uint32_t T_A2 = 128;   // A of R2: [Bi^T (transpose round); Q_b]
+constexpr uint32_t T_D3R = 192;  // [Ki^T (transpose round); Q_k] -> R3 subtracts Z M_kb -> [K~; Q~] (A of R4)
+constexpr uint32_t T_D3L = 256;  // [I; Rd] -> R3 subtracts Z KKd -> [I - X; R~] (A of R5)
 constexpr uint32_t T_D4 = 320;   // [S'^T; Y] (R4 + R5); the new state is diag(gC) S'^T
-constexpr uint32_t T_A2 = 384;   // A of R2: [Bi^T (R1c); Q_b]
-constexpr uint32_t T_ID = 448;   // identity (lanes 0-63) over zeros: A of the transposes, written once
+constexpr uint32_t T_ID = 448;   // identity (lanes 0-63) over zeros: A of the transpose round, written once
+static_assert(T_A2 + 64 == T_D3R && T_D3R + 64 == T_D3L, "transpose round and R3 write adjacent blocks");
 
 enum { XR = 0, XW = 1, XK = 2, XV = 3, XKK = 4, XA = 5 };
 
 struct ChunkMaps {
-    CUtensorMap m[6];
+    CUtensorMap m[6];     // inputs r, w, k, v, kk, a: bf16 [B][T][H][64], box 64 tokens x 64 channels
+    CUtensorMap y;        // output y: fp32 [B][T][H][64], box 64 tokens x 32 channels
 };
+constexpr int kStoreThread = 32;   // issues and completes the TMA stores of y (lane 0 of warp 1)
 
 struct ChunkArgs {
     int B, T, H;
     const float *S0;
-    float *y, *S_T, *snaps;
+    float *S_T, *snaps;
     int snap_every, n_snap;
     const float *ln_w, *ln_b, *r_k;
     float gn_eps;
@@ -171,6 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     // rank + cs, ... and hands the state after each of them to CTA rank + 1 (mod cs).
     const int cs = int(cluster_size()), rank = int(cluster_rank());
     const int cid = int(cluster_index()), ncl = int(cluster_count());
+    if (tid < 7) asm volatile("prefetch.tensormap [%0];" ::"l"(tid < 6 ? &maps.m[tid] : &maps.y) : "memory");
     if (tid == 0) {
         mbar_init(&S.bar_tma, 1);
         mbar_init(&S.bar_mma, 1);
@@ -251,6 +257,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         for (int c = rank; c < nchunks && !failed; c += cs) {
             const int c0 = c * C, Lc = min(C, p.T - c0);
             const bool last = c == nchunks - 1;
+            // this CTA's next chunk, whose inputs are prefetched during this one
+            int nu = unit, nc = c + cs;
+            if (nc >= nchunks) { nu = unit + ncl; nc = rank; }
+            const bool more = nu < units && nc < nchunks;
             {   // ---- inputs of this chunk
                 const bool to = !mbar_wait(&S.bar_tma, tma_parity, p.timeout_ns);
                 tma_parity ^= 1u;
@@ -289,10 +299,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                     S.gC[j] = g;
                 }
             }
+            // P3 overwrites the y tile of the previous chunk's TMA store: its reads must be done
+            if (tid == kStoreThread) tma_store_wait_read();
             __syncthreads();
             // ---- P3: token rows. Lanes 0-63 (token t = L): KKd row -> A1 rows 0-63, Ki row -> B1,
-            //      identity row -> T_D3 (start of P). Lanes 64-127 (token t): Rd row -> A1 rows 64-127
-            //      and T_D3 (start of R~), Bi row -> B1, exact current-token Grams.
+            //      identity row -> T_D3L (start of P). Lanes 64-127 (token t): Rd row -> A1 rows 64-127
+            //      and T_D3L (start of R~), Bi row -> B1, exact current-token Grams.
             if (colg) {
                 const int t = L;
                 const float *gp = GT + t * GTS;         // g_{t-1}
@@ -320,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                     st_f4(sm + OFF_B1, sw128_off(64 + t, j0 + 4, 128), ki[4], ki[5], ki[6], ki[7]);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) v[e] = (j0 + e == t) ? 1.f : 0.f;
-                    tmem_st8(tmem_addr(tb, Lq, T_D3 + j0), v);
+                    tmem_st8(tmem_addr(tb, Lq, T_D3L + j0), v);
                 }
             } else {
                 const int t = L - 64;
@@ -348,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                     }
                     st_f4(sm + OFF_A1, sw128_off(64 + t, j0, 128), rd[0], rd[1], rd[2], rd[3]);
                     st_f4(sm + OFF_A1, sw128_off(64 + t, j0 + 4, 128), rd[4], rd[5], rd[6], rd[7]);
-                    tmem_st8(tmem_addr(tb, Lq, T_D3 + j0), rd);
+                    tmem_st8(tmem_addr(tb, Lq, T_D3L + j0), rd);
                     st_f4(sm + OFF_B1, sw128_off(t, j0, 128), bi[0], bi[1], bi[2], bi[3]);
                     st_f4(sm + OFF_B1, sw128_off(t, j0 + 4, 128), bi[4], bi[5], bi[6], bi[7]);
                 }
@@ -358,28 +370,24 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
             }
             sync_for_mma();
             if (tid == 0) {
+                // the next chunk's six input tiles are issued by six warps in P5; their byte count
+                // is registered here, ordered before those issues by the barrier after R1
+                if (more) mbar_arrive_expect_tx(&S.bar_tma, 6 * 8192);
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)   // R1: Grams = [KKd; Rd] [Bi; Ki]^T
                     mma_tf32_ss(tb + T_D1, dA1 + kstep_off(ks, 128), dB1 + kstep_off(ks, 128), idesc_tf32(128, 128), ks > 0);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)   // R1b: transposed Grams [Bi; Ki] KKd^T
-                    mma_tf32_ss(tb + T_D2, dB1 + kstep_off(ks, 128), dA1 + kstep_off(ks, 128), idesc_tf32(128, 64), ks > 0);
-                // transposes on the tensor core (exact: identity times tf32 operands):
-                // lanes 0-63 of T_A2 <- Bi^T (A of R2), of T_D3 cols 64-127 <- Ki^T (start of K~)
+                // transpose round on the tensor core (exact: identity times tf32 operands), N = 128:
+                // lanes 0-63 of T_A2 <- Bi^T (A of R2), of T_D3R <- Ki^T (start of K~)
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_tf32_ts(tb + T_A2, tb + T_ID + 8 * ks, dB1 + kstep_off(ks, 128), idesc_tf32(128, 64), ks > 0);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_tf32_ts(tb + T_D3 + 64, tb + T_ID + 8 * ks, dB1 + (8192 >> 4) + kstep_off(ks, 128),
-                                idesc_tf32(128, 64), ks > 0);
+                    mma_tf32_ts(tb + T_A2, tb + T_ID + 8 * ks, dB1 + kstep_off(ks, 128), idesc_tf32(128, 128), ks > 0);
                 mma_commit(&S.bar_mma);
             }
             mma_pending = true;
             // ---- P4 (while the MMAs run): transposes through shared memory, no arithmetic.
             //      Lanes 0-63 (key/value channel j = L): V^T row j -> B4.
-            //      Lanes 64-127 (key j = L - 64): KKd^T row j -> B3 rows 0-63.
+            //      Lanes 64-127 (key j = L - 64): KKd^T row j -> B3 rows 64-127.
             if (colg) {
                 const int j = L;
                 uint32_t xo[8];
@@ -404,63 +412,67 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                     float kkd[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) kkd[e] = *reinterpret_cast<const float *>(b6 + (t0 + e) * 128 + xo[e]);
-                    st_f4(sm + OFF_B3, sw128_off(j, t0, 128), kkd[0], kkd[1], kkd[2], kkd[3]);
-                    st_f4(sm + OFF_B3, sw128_off(j, t0 + 4, 128), kkd[4], kkd[5], kkd[6], kkd[7]);
+                    st_f4(sm + OFF_B3, sw128_off(64 + j, t0, 128), kkd[0], kkd[1], kkd[2], kkd[3]);
+                    st_f4(sm + OFF_B3, sw128_off(64 + j, t0 + 4, 128), kkd[4], kkd[5], kkd[6], kkd[7]);
                 }
             }
             if (wait_mma()) { failed = true; break; }
-            // ---- P5: masks. Lanes 0-63 (token t): M_ab row -> inverse workspace.
-            //      Lanes 64-127 (token t): Q_b row -> A2 rows 64-127 (T_D3); M_kb^T row t -> B3.
+            // ---- P5: masks. Lanes 0-63 (token t): M_ab row -> inverse workspace; M_kb row t ->
+            //      column t of B3 rows 0-63 (M_kb^T, scalar stores along K: conflict-free).
+            //      Lanes 64-127 (token t): Q_b row -> T_A2 lanes 64-127; Q_k row -> T_D3R lanes 64-127.
+            if (more && lane == 0 && colg && (warp >> 2) < 3) {
+                // the input tiles were last read in P4: six warps each issue one tile of the next chunk
+                const int x = (warp >> 2) * 2 + (warp & 1);
+                tma_load_4d(sm + OFF_IN + x * 8192, &maps.m[x], &S.bar_tma, 0, nu % p.H, nc * C, nu / p.H);
+            }
             if (colg) {
                 const int t = L;
-#pragma unroll 1
+                float m[2][8], mk[2][8];
+                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + c16), m[0]);
+                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + c16 + 8), m[1]);
+                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + 64 + c16), mk[0]);
+                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + 64 + c16 + 8), mk[1]);
+                tmem_ld_wait(m[0], m[1], mk[0], mk[1]);
+                uint32_t xo[8];
+                kcol_offsets(t, 128, xo);
+#pragma unroll
                 for (int g = 0; g < 2; ++g) {
                     const int s0 = c16 + 8 * g;
-                    float m[8];
-                    tmem_ld8(tmem_addr(tb, Lq, T_D1 + s0), m);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) m[e] = (s0 + e < t) ? m[e] : 0.f;
-                    *reinterpret_cast<float4 *>(Lw + t * LWS + s0) = make_float4(m[0], m[1], m[2], m[3]);
-                    *reinterpret_cast<float4 *>(Lw + t * LWS + s0 + 4) = make_float4(m[4], m[5], m[6], m[7]);
+                    for (int e = 0; e < 8; ++e) m[g][e] = (s0 + e < t) ? m[g][e] : 0.f;
+                    *reinterpret_cast<float4 *>(Lw + t * LWS + s0) = make_float4(m[g][0], m[g][1], m[g][2], m[g][3]);
+                    *reinterpret_cast<float4 *>(Lw + t * LWS + s0 + 4) = make_float4(m[g][4], m[g][5], m[g][6], m[g][7]);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)   // B3[s][t] = M_kb[t][s], nonzero for s < t
+                        *reinterpret_cast<float *>(sm + OFF_B3 + (s0 + e) * 128 + xo[e]) =
+                            (s0 + e < t) ? to_tf32(mk[g][e]) : 0.f;
                 }
             } else {
                 const int t = L - 64;
                 // the current-token entries are taken exactly in fp32: they dominate short sequences
                 const float dgb = to_tf32(S.db[0][t] + S.db[1][t] + S.db[2][t] + S.db[3][t]);
                 const float dgk = S.dk[0][t] + S.dk[1][t] + S.dk[2][t] + S.dk[3][t];
-#pragma unroll 1
+                float qb[2][8], qk[2][8];
+                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + c16), qb[0]);            // Q_b row t
+                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + c16 + 8), qb[1]);
+                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + 64 + c16), qk[0]);       // Q_k row t
+                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + 64 + c16 + 8), qk[1]);
+                tmem_ld_wait(qb[0], qb[1], qk[0], qk[1]);
+#pragma unroll
                 for (int g = 0; g < 2; ++g) {
                     const int s0 = c16 + 8 * g;
-                    float m[8];
-                    tmem_ld8(tmem_addr(tb, Lq, T_D1 + s0), m);          // Q_b row t
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int ss = s0 + e;
-                        m[e] = ss < t ? to_tf32(m[e]) : (ss == t ? dgb : 0.f);
+                        qb[g][e] = ss < t ? to_tf32(qb[g][e]) : (ss == t ? dgb : 0.f);
+                        qk[g][e] = ss < t ? qk[g][e] : (ss == t ? dgk : 0.f);
                     }
-                    tmem_st8(tmem_addr(tb, Lq, T_A2 + s0), m);
-                    tmem_ld8(tmem_addr(tb, Lq, T_D1 + 64 + s0), m);     // Q_k row t
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int ss = s0 + e;
-                        m[e] = ss < t ? m[e] : (ss == t ? dgk : 0.f);
-                    }
-                    tmem_st8(tmem_addr(tb, Lq, T_D3 + 64 + s0), m);
-                    // row t of M_kb^T: M_kb[t'][t] for tokens t' = s0..s0+7 (nonzero for t' > t)
-                    tmem_ld8(tmem_addr(tb, Lq, T_D2 + s0), m);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) m[e] = (s0 + e > t) ? to_tf32(m[e]) : 0.f;
-                    st_f4(sm + OFF_B3, sw128_off(64 + t, s0, 128), m[0], m[1], m[2], m[3]);
-                    st_f4(sm + OFF_B3, sw128_off(64 + t, s0 + 4, 128), m[4], m[5], m[6], m[7]);
+                    tmem_st8(tmem_addr(tb, Lq, T_A2 + s0), qb[g]);
+                    tmem_st8(tmem_addr(tb, Lq, T_D3R + s0), qk[g]);
                 }
             }
             sync_for_mma();
-            {   // input tiles and decay table are consumed: prefetch this CTA's next chunk
-                int nu = unit, nc = c + cs;
-                if (nc >= nchunks) { nu = unit + ncl; nc = rank; }
-                tma_pending = nu < units && nc < nchunks;
-                if (tid == 0 && tma_pending) issue_tma(nu, nc);
-            }
+            tma_pending = more;
             // ---- A = (I + M_ab)^{-1}. Diagonal 16x16 blocks: one thread per (block, column)
             //      solves (I + L_dd) x = e_c by forward substitution in registers (warps 2, 3).
             if (tid >= 64 && tid < 128) {
@@ -556,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)   // R2: Z = [Bi^T; Q_b] A
-                    mma_tf32_ts(tb + T_D2, tb + T_A2 + 8 * ks, dB2 + kstep_off(ks, 64), idesc_tf32(128, 64), ks > 0);
+                    mma_tf32_ts(tb + T_D1, tb + T_A2 + 8 * ks, dB2 + kstep_off(ks, 64), idesc_tf32(128, 64), ks > 0);
                 mma_commit(&S.bar_mma);
             }
             mma_pending = true;
@@ -564,8 +576,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
             if (tid == 0) {
                 tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)   // R3: T_D3 -= Z [KKd | M_kb]
-                    mma_tf32_ts(tb + T_D3, tb + T_D2 + 8 * ks, dB3 + kstep_off(ks, 128),
+                for (int ks = 0; ks < 8; ++ks)   // R3: [T_D3R | T_D3L] -= Z [M_kb | KKd]
+                    mma_tf32_ts(tb + T_D3R, tb + T_D1 + 8 * ks, dB3 + kstep_off(ks, 128),
                                 idesc_neg_a(idesc_tf32(128, 128)), 1);
                 mma_commit(&S.bar_mma);
             }
@@ -577,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)   // R4: [Ki^T - X; Q~] V
-                    mma_tf32_ts(tb + T_D4, tb + T_D3 + 64 + 8 * ks, dB4 + kstep_off(ks, 64), idesc_tf32(128, 64), ks > 0);
+                    mma_tf32_ts(tb + T_D4, tb + T_D3R + 8 * ks, dB4 + kstep_off(ks, 64), idesc_tf32(128, 64), ks > 0);
                 if (recv) {
                     // the only wait on another CTA: everything above used this chunk's inputs only
                     state_to = !mbar_wait_cluster(&S.bar_state, state_parity, p.timeout_ns);
@@ -587,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 if (!state_to) {
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks)   // R5: += [I - X; R~] S_0^T
-                        mma_tf32_ts(tb + T_D4, tb + T_D3 + 8 * ks, dB5 + kstep_off(ks, 64), idesc_tf32(128, 64), 1);
+                        mma_tf32_ts(tb + T_D4, tb + T_D3L + 8 * ks, dB5 + kstep_off(ks, 64), idesc_tf32(128, 64), 1);
                 }
                 mma_commit(&S.bar_mma);
             }
@@ -605,11 +617,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 uint8_t *b5 = sm + OFF_B5;
                 // split mode: the state goes straight into the next CTA's B5 (distributed shared memory)
                 const bool send = cs > 1 && c + 1 < nchunks;
-#pragma unroll 1
+                float sv[2][8];
+                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D4 + c16), sv[0]);      // S'[c16+e][j]
+                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D4 + c16 + 8), sv[1]);
+                tmem_ld_wait(sv[0], sv[1]);
+#pragma unroll
                 for (int g = 0; g < 2; ++g) {
                     const int i0 = c16 + 8 * g;
-                    float s8[8];
-                    tmem_ld8(tmem_addr(tb, Lq, T_D4 + i0), s8);    // S'[i0+e][j]
+                    float (&s8)[8] = sv[g];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) s8[e] *= gCj;                // S_C = S' diag(gC)
                     if (send) {
@@ -636,16 +651,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 }
             } else {
                 const int t = L - 64;
-                float *dst = p.y + ((size_t(b) * p.T + c0 + t) * p.H + hh) * 64 + c16;
                 float yv[16];
                 {
-                    float y8[8];
-                    tmem_ld8(tmem_addr(tb, Lq, T_D4 + c16), y8);
+                    float ya[8], yb[8];
+                    tmem_ld8_nowait(tmem_addr(tb, Lq, T_D4 + c16), ya);
+                    tmem_ld8_nowait(tmem_addr(tb, Lq, T_D4 + c16 + 8), yb);
+                    tmem_ld_wait(ya, yb);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) yv[e] = y8[e];
-                    tmem_ld8(tmem_addr(tb, Lq, T_D4 + c16 + 8), y8);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) yv[8 + e] = y8[e];
+                    for (int e = 0; e < 8; ++e) {
+                        yv[e] = ya[e];
+                        yv[8 + e] = yb[e];
+                    }
                 }
                 if (epi) {
                     uint32_t xo[8];
@@ -671,15 +687,23 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                         yv[e] = fmaf((yv[e] - mean) * inv, S.ln_w[ii], S.ln_b[ii]) + bon * v;
                     }
                 }
-                if (t < Lc) {
+                // y row t, channels c16..c16+15 -> the swizzled [64][32] fp32 tile of its channel half
+                // (the layout the y tensor map expects); rows past the end of T are clipped by the store
+                uint8_t *ytile = sm + OFF_B1 + (c16 >> 5) * 8192 + t * 128;
 #pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        *reinterpret_cast<float4 *>(dst + 4 * m) = make_float4(yv[4 * m], yv[4 * m + 1], yv[4 * m + 2], yv[4 * m + 3]);
-                }
+                for (int m = 0; m < 4; ++m)
+                    *reinterpret_cast<float4 *>(ytile + (((((c16 & 31) >> 2) + m) ^ (t & 7)) << 4)) =
+                        make_float4(yv[4 * m], yv[4 * m + 1], yv[4 * m + 2], yv[4 * m + 3]);
             }
             sync_for_mma();
+            if (tid == kStoreThread) {
+                tma_store_4d(&maps.y, sm + OFF_B1, 0, hh, c0, b);
+                tma_store_4d(&maps.y, sm + OFF_B1 + 8192, 32, hh, c0, b);
+                tma_store_commit();
+            }
         }
     }
+    if (tid == kStoreThread) tma_store_wait_all();
 
     if (failed) {
         if (tid == 0) atomicOr(p.err, 1u);
@@ -808,9 +832,18 @@ cudaError_t launch_chunk(const FwdArgs &p) {
                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     }
+    {
+        const cuuint64_t ydims[4] = {cuuint64_t(kN), cuuint64_t(p.H), cuuint64_t(p.T), cuuint64_t(p.B)};
+        const cuuint64_t ystrides[3] = {cuuint64_t(kN) * 4, cuuint64_t(p.H) * kN * 4, cuuint64_t(p.T) * p.H * kN * 4};
+        const cuuint32_t ybox[4] = {32, 1, cuuint32_t(C), 1};
+        const CUresult r = enc(&maps.y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.y, ydims, ystrides, ybox, es,
+                               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
     ChunkArgs a{};
     a.B = p.B; a.T = p.T; a.H = p.H;
-    a.S0 = p.S0; a.y = p.y; a.S_T = p.S_T; a.snaps = p.snaps;
+    a.S0 = p.S0; a.S_T = p.S_T; a.snaps = p.snaps;
     a.snap_every = p.snap_every;
     a.n_snap = p.snap_every > 0 ? p.T / p.snap_every : 0;
     a.ln_w = p.ln_w; a.ln_b = p.ln_b; a.r_k = p.r_k; a.gn_eps = p.gn_eps;

@@ -110,6 +110,25 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
         : "r"(taddr)
         : "memory");
 }
+// Same without the wait: several loads in flight, then one tmem_ld_wait(...) naming every
+// destination array before any use (the operands keep the compiler from moving uses above it).
+__device__ __forceinline__ void tmem_ld8_nowait(uint32_t taddr, float (&v)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : WKV7_R8(0)
+                 : "r"(taddr)
+                 : "memory");
+}
+#define WKV7_RW8(a) "+f"(a[0]), "+f"(a[1]), "+f"(a[2]), "+f"(a[3]), "+f"(a[4]), "+f"(a[5]), "+f"(a[6]), "+f"(a[7])
+__device__ __forceinline__ void tmem_ld_wait(float (&a)[8], float (&b)[8]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : WKV7_RW8(a), WKV7_RW8(b) : : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait(float (&a)[8], float (&b)[8], float (&c)[8]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : WKV7_RW8(a), WKV7_RW8(b), WKV7_RW8(c) : : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait(float (&a)[8], float (&b)[8], float (&c)[8], float (&d)[8]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : WKV7_RW8(a), WKV7_RW8(b), WKV7_RW8(c), WKV7_RW8(d) : : "memory");
+}
+#undef WKV7_RW8
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), WKV7_W8(0)
                  : "memory");
@@ -228,6 +247,19 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, uint64_
         "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
+
+// Shared -> global tile store through a tensor map (bulk-group completion). The source must stay
+// untouched until tma_store_wait_read() in the issuing thread has returned.
+__device__ __forceinline__ void tma_store_4d(const void *tmap, const void *src, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(tmap),
+                 "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// The sources of this thread's committed stores have been read (shared memory reusable).
+__device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// This thread's committed stores are complete.
+__device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // ---- thread-block clusters and distributed shared memory ------------------------------------------
 // A kernel launched without a cluster attribute runs as clusters of one CTA: rank 0 of 1.
