@@ -62,9 +62,11 @@ constexpr int LWS = 68;           // row stride of the inverse workspaces (16-by
 
 // Shared-memory layout (byte offsets from a 1024-byte aligned base).
 constexpr uint32_t OFF_B1 = 0;        // [Bi; Ki] 128x64 tf32 (B of R1 and of the transpose round); then the
-                                      // inverse workspace; then the y tile of the TMA store (2 x [64][32] fp32)
+                                      // inverse workspace
 constexpr uint32_t OFF_B3 = 32768;    // [M_kb^T; KKd^T] 128x64 (B of R3)
-constexpr uint32_t OFF_B2 = 65536;    // A^T 64x64 (B of R2)
+constexpr uint32_t OFF_L21 = 24576;   // inside B1, after the inverse workspace: L21^T 32x32 (B of R2b)
+constexpr uint32_t OFF_B2 = 65536;    // A^T 64x64 (B of R2); after R2, the y tile of the TMA store
+                                      // (2 x [64][32] fp32), stored during the next chunk's R1
 constexpr uint32_t OFF_B4 = 81920;    // V^T 64x64 (B of R4; exact bf16 values)
 constexpr uint32_t OFF_B5 = 98304;    // S 64x64, row = value channel (B of R5)
 constexpr uint32_t OFF_A1 = 114688;   // [KKd; Rd] 128x64 (A of R1)
@@ -95,6 +97,7 @@ constexpr uint32_t T_A2 = 128;   // A of R2: [Bi^T (transpose round); Q_b]
 constexpr uint32_t T_D3R = 192;  // [Ki^T (transpose round); Q_k] -> R3 subtracts Z M_kb -> [K~; Q~] (A of R4)
 constexpr uint32_t T_D3L = 256;  // [I; Rd] -> R3 subtracts Z KKd -> [I - X; R~] (A of R5)
 constexpr uint32_t T_D4 = 320;   // [S'^T; Y] (R4 + R5); the new state is diag(gC) S'^T
+constexpr uint32_t T_V = 384;    // R2b: U[:, 32:64] L21 (32 columns)
 constexpr uint32_t T_ID = 448;   // identity (lanes 0-63) over zeros: A of the transpose round, written once
 static_assert(T_A2 + 64 == T_D3R && T_D3R + 64 == T_D3L, "transpose round and R3 write adjacent blocks");
 
@@ -105,6 +108,13 @@ struct ChunkMaps {
     CUtensorMap y;        // output y: fp32 [B][T][H][64], box 64 tokens x 32 channels
 };
 constexpr int kStoreThread = 32;   // issues and completes the TMA stores of y (lane 0 of warp 1)
+
+// y tile of one chunk (in B2) -> global through the y tensor map; the two channel halves.
+__device__ __forceinline__ void store_y_tile(const ChunkMaps &maps, const uint8_t *tile, int hh, int c0, int b) {
+    tma_store_4d(&maps.y, tile, 0, hh, c0, b);
+    tma_store_4d(&maps.y, tile + 8192, 32, hh, c0, b);
+    tma_store_commit();
+}
 
 struct ChunkArgs {
     int B, T, H;
@@ -159,7 +169,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     float *GT = reinterpret_cast<float *>(sm + OFF_GT);
     float *Lw = reinterpret_cast<float *>(sm + OFF_B1);      // strictly lower M_ab [64][LWS]
     float *Tw = Lw + 64 * LWS;                               // level-1 temps [2][16][20]
-    float *Tw2 = Tw + 2 * 16 * 20;                           // level-2 temp [32][36]
     float *Aw = reinterpret_cast<float *>(sm + OFF_GT);      // inverse [64][LWS]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -199,6 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     const uint64_t dB1 = desc_sw128(smem_u32(sm + OFF_B1)), dB2 = desc_sw128(smem_u32(sm + OFF_B2));
     const uint64_t dB3 = desc_sw128(smem_u32(sm + OFF_B3)), dB4 = desc_sw128(smem_u32(sm + OFF_B4));
     const uint64_t dB5 = desc_sw128(smem_u32(sm + OFF_B5)), dA1 = desc_sw128(smem_u32(sm + OFF_A1));
+    const uint64_t dL21 = desc_sw128(smem_u32(sm + OFF_L21));
     {   // identity over zeros in T_ID (A operand of the transposes; never overwritten)
         float id8[8];
 #pragma unroll 1
@@ -211,6 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         tmem_st_wait();
     }
     uint32_t tma_parity = 0, mma_parity = 0, state_parity = 0;
+    bool y_pending = false;            // the y tile in B2 still has to be stored (uniform)
+    int y_h = 0, y_c0 = 0, y_b = 0;    // its coordinates
     bool tma_pending = false, mma_pending = false, failed = false;
 
     auto issue_tma = [&](int u, int c) {   // thread 0
@@ -299,8 +311,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                     S.gC[j] = g;
                 }
             }
-            // P3 overwrites the y tile of the previous chunk's TMA store: its reads must be done
-            if (tid == kStoreThread) tma_store_wait_read();
             __syncthreads();
             // ---- P3: token rows. Lanes 0-63 (token t = L): KKd row -> A1 rows 0-63, Ki row -> B1,
             //      identity row -> T_D3L (start of P). Lanes 64-127 (token t): Rd row -> A1 rows 64-127
@@ -385,6 +395,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 mma_commit(&S.bar_mma);
             }
             mma_pending = true;
+            // the previous chunk's y tile goes out now: every warp has slack while R1 runs
+            if (y_pending && tid == kStoreThread) store_y_tile(maps, sm + OFF_B2, y_h, y_c0, y_b);
+            y_pending = false;
             // ---- P4 (while the MMAs run): transposes through shared memory, no arithmetic.
             //      Lanes 0-63 (key/value channel j = L): V^T row j -> B4.
             //      Lanes 64-127 (key j = L - 64): KKd^T row j -> B3 rows 64-127.
@@ -447,6 +460,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                         *reinterpret_cast<float *>(sm + OFF_B3 + (s0 + e) * 128 + xo[e]) =
                             (s0 + e < t) ? to_tf32(mk[g][e]) : 0.f;
                 }
+                if (t >= 32 && c16 < 32) {   // L21^T[s][t - 32] = M_ab[t][s] (s < 32 <= t: no mask)
+                    uint32_t xl[8];
+                    kcol_offsets(t - 32, 32, xl);
+#pragma unroll
+                    for (int g = 0; g < 2; ++g)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            *reinterpret_cast<float *>(sm + OFF_L21 + (c16 + 8 * g + e) * 128 + xl[e]) = to_tf32(m[g][e]);
+                }
             } else {
                 const int t = L - 64;
                 // the current-token entries are taken exactly in fp32: they dominate short sequences
@@ -488,16 +510,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 }
 #pragma unroll
                 for (int r = 0; r < 16; ++r) Aw[(16 * d + r) * LWS + 16 * d + cc] = x[r];
-            } else {
-                // zero the blocks above the diagonal: (bi, bj) with bi < bj
-                const int z0 = tid < 64 ? tid : tid - 64;
-#pragma unroll 1
-                for (int e = z0; e < 6 * 256; e += kThreads - 64) {
-                    const int blk = e >> 8, o = e & 255;
-                    const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-                    const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-                    Aw[(16 * bi + (o >> 4)) * LWS + 16 * bj + (o & 15)] = 0.f;
-                }
             }
             __syncthreads();
             // level 1: X[2p+1][2p] = -X[2p+1] (L[2p+1][2p] X[2p]), p = 0, 1. Threads 0-127 each
@@ -528,47 +540,47 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 *reinterpret_cast<float4 *>(Aw + (32 * pp + 16 + i) * LWS + 32 * pp + j4) =
                     make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
             }
+            if (tid == kStoreThread) tma_store_wait_read();   // the y tile in B2 has been read
             __syncthreads();
-            // level 2: Y[1][0] = -Y1 (L[32:64][0:32] Y0). Y0, Y1 are lower triangular, so the
-            // fixed-length sums are exact. Threads 0-255: one row, four adjacent columns each.
-            if (tid < 256) {
-                const int i = tid >> 3, j4 = (tid & 7) * 4;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-                for (int kq = 0; kq < 32; ++kq) {
-                    const float lv = Lw[(32 + i) * LWS + kq];
-                    const float4 yv = *reinterpret_cast<const float4 *>(Aw + kq * LWS + j4);
-                    acc[0] = fmaf(lv, yv.x, acc[0]); acc[1] = fmaf(lv, yv.y, acc[1]);
-                    acc[2] = fmaf(lv, yv.z, acc[2]); acc[3] = fmaf(lv, yv.w, acc[3]);
-                }
-                *reinterpret_cast<float4 *>(Tw2 + i * 36 + j4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            }
-            __syncthreads();
-            if (tid < 256) {
-                const int i = tid >> 3, j4 = (tid & 7) * 4;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-                for (int kq = 0; kq < 32; ++kq) {
-                    const float av = Aw[(32 + i) * LWS + 32 + kq];
-                    const float4 tv = *reinterpret_cast<const float4 *>(Tw2 + kq * 36 + j4);
-                    acc[0] = fmaf(av, tv.x, acc[0]); acc[1] = fmaf(av, tv.y, acc[1]);
-                    acc[2] = fmaf(av, tv.z, acc[2]); acc[3] = fmaf(av, tv.w, acc[3]);
-                }
-                *reinterpret_cast<float4 *>(Aw + (32 + i) * LWS + j4) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
-            }
-            __syncthreads();
-            // B2 = A^T (row s, K = t)
+            // B2 = D^T, D = blockdiag(Y0, Y1) the inverses of the two diagonal 32x32 blocks of
+            // I + M_ab (row s, K = t; entries with t < s or t, s in different halves are zero).
+            // The off-diagonal block of the inverse, -Y1 L21 Y0, is applied by R2b/R2c.
             for (int e = tid; e < 1024; e += kThreads) {
                 const int s = e & 63, t4 = (e >> 6) * 4;
-                st_f4(sm + OFF_B2, sw128_off(s, t4, 64), to_tf32(Aw[t4 * LWS + s]), to_tf32(Aw[(t4 + 1) * LWS + s]),
-                      to_tf32(Aw[(t4 + 2) * LWS + s]), to_tf32(Aw[(t4 + 3) * LWS + s]));
+                float a4[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int t = t4 + q;
+                    a4[q] = (t >= s && ((t ^ s) < 32)) ? to_tf32(Aw[t * LWS + s]) : 0.f;
+                }
+                st_f4(sm + OFF_B2, sw128_off(s, t4, 64), a4[0], a4[1], a4[2], a4[3]);
             }
             sync_for_mma();
             if (tid == 0) {
                 tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)   // R2: Z = [Bi^T; Q_b] A
+                for (int ks = 0; ks < 8; ++ks)   // R2a: U = W D, W = [Bi^T; Q_b]
                     mma_tf32_ts(tb + T_D1, tb + T_A2 + 8 * ks, dB2 + kstep_off(ks, 64), idesc_tf32(128, 64), ks > 0);
+                mma_commit(&S.bar_mma);
+            }
+            mma_pending = true;
+            if (wait_mma()) { failed = true; break; }
+            // Z = W A with A = D - [0 0; Y1 L21 Y0 0]: Z[:, 32:64] = U[:, 32:64] and
+            // Z[:, 0:32] = U[:, 0:32] - (U[:, 32:64] L21) Y0 (block back-substitution on the tensor core)
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)   // R2b: V = U[:, 32:64] L21
+                    mma_tf32_ts(tb + T_V, tb + T_D1 + 32 + 8 * ks, dL21 + kstep_off(ks, 32), idesc_tf32(128, 32), ks > 0);
+                mma_commit(&S.bar_mma);
+            }
+            mma_pending = true;
+            if (wait_mma()) { failed = true; break; }
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)   // R2c: U[:, 0:32] -= V Y0 (B2 rows 0-31 hold Y0^T)
+                    mma_tf32_ts(tb + T_D1, tb + T_V + 8 * ks, dB2 + kstep_off(ks, 64), idesc_neg_a(idesc_tf32(128, 32)), 1);
                 mma_commit(&S.bar_mma);
             }
             mma_pending = true;
@@ -689,21 +701,21 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 }
                 // y row t, channels c16..c16+15 -> the swizzled [64][32] fp32 tile of its channel half
                 // (the layout the y tensor map expects); rows past the end of T are clipped by the store
-                uint8_t *ytile = sm + OFF_B1 + (c16 >> 5) * 8192 + t * 128;
+                uint8_t *ytile = sm + OFF_B2 + (c16 >> 5) * 8192 + t * 128;
 #pragma unroll
                 for (int m = 0; m < 4; ++m)
                     *reinterpret_cast<float4 *>(ytile + (((((c16 & 31) >> 2) + m) ^ (t & 7)) << 4)) =
                         make_float4(yv[4 * m], yv[4 * m + 1], yv[4 * m + 2], yv[4 * m + 3]);
             }
             sync_for_mma();
-            if (tid == kStoreThread) {
-                tma_store_4d(&maps.y, sm + OFF_B1, 0, hh, c0, b);
-                tma_store_4d(&maps.y, sm + OFF_B1 + 8192, 32, hh, c0, b);
-                tma_store_commit();
-            }
+            y_pending = true;
+            y_h = hh; y_c0 = c0; y_b = b;
         }
     }
-    if (tid == kStoreThread) tma_store_wait_all();
+    if (tid == kStoreThread) {
+        if (y_pending && !failed) store_y_tile(maps, sm + OFF_B2, y_h, y_c0, y_b);
+        tma_store_wait_all();
+    }
 
     if (failed) {
         if (tid == 0) atomicOr(p.err, 1u);
