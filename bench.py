@@ -17,9 +17,11 @@ max over ranks.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import sys
 import threading
@@ -43,6 +45,44 @@ WORKLOADS = {
     "long-context": dict(cid=4, default_steps=10),
     "decode": dict(cid=3, default_steps=256),
 }
+
+
+# ---- measured DRAM traffic of the dominant kernel (committed ncu summaries under profiles/) -------
+
+KERNEL_SOURCES = {"chunk_kernel": ("chunk.cu", "tc_util.cuh", "common.cuh"),
+                  "decode_kernel": ("decode.cu", "common.cuh"),
+                  "seq_kernel": ("seq.cu", "common.cuh")}
+PROFILE_TAGS = {"prefill-0.19b": "prefill-0.19B", "prefill-1.5b": "prefill-1.5B",
+                "long-context": "long-context", "decode": "decode-2.9B"}
+
+
+def kernel_digest(kernel: str) -> str:
+    """sha256 (16 hex digits) of the device code a kernel is built from: its .cu file up to the
+    host-side section, plus the headers it includes."""
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "linear_rnn_sequence_rwkv_b200", "csrc", f)) as fh:
+            text = fh.read()
+        cut = text.find("// ---- host side")
+        h.update((text if cut < 0 else text[:cut]).encode())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, workload: str):
+    """dram__bytes_read.sum + dram__bytes_write.sum per launch recorded in
+    profiles/<kernel>_<workload>.md, or None without a capture or when the kernel's device
+    code has changed since it was taken (the summary records the digest it was taken at)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{PROFILE_TAGS.get(workload, workload)}.md")
+    try:
+        with open(path) as f:
+            text = f.read()
+    except OSError:
+        return None
+    t = re.search(r"^traffic_bytes_per_launch:\s*(\d+)\s*$", text, re.M)
+    d = re.search(r"^device_code_sha256_16:\s*([0-9a-f]{16})\s*$", text, re.M)
+    if not (t and d) or d.group(1) != kernel_digest(kernel):
+        return None
+    return int(t.group(1))
 
 
 def _peaks():
@@ -210,6 +250,8 @@ def run_gpu(args, world, rank, local):
         launches_per_step = 1 + (1 if epilogue and _path_name(args) == "seq" else 0)
 
     units_per_step = B * T * H
+    ctas_per_head = None if decode else wkv7.plan(B, T, H, N, torch.bfloat16, algo=args.algo, chunk=args.chunk,
+                                                  snap_every=snap_every)[1]
 
     for i in range(warmup):
         step(i)
@@ -244,12 +286,13 @@ def run_gpu(args, world, rank, local):
         roof = {"bound": "alu", "achieved": round(achieved, 3), "peak": round(fp32_peak, 2),
                 "unit": "TFLOP/s", "frac": round(achieved / fp32_peak, 4),
                 "peak_source": f"148 SMs x 128 FP32 lanes x 2 flop x {sm_max:.0f} MHz (derived)",
-                "traffic": None, "kernel": "seq_kernel",
+                "traffic": measured_traffic("seq_kernel", args.workload), "kernel": "seq_kernel",
                 "hbm_gbs": round(achieved_gbs, 1), "hbm_frac": round(achieved_gbs / hbm_peak, 4)}
     else:
         roof = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved_gbs / hbm_peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
-                "traffic": None, "kernel": "decode_kernel" if decode else "chunk_kernel",
+                "traffic": measured_traffic("decode_kernel" if decode else "chunk_kernel", args.workload),
+                "kernel": "decode_kernel" if decode else "chunk_kernel",
                 "recurrence_tflops": round(flops_per_launch / (launch_ms * 1e-3) / 1e12, 3)}
     roof["algorithmic_bytes_per_launch"] = bytes_per_launch
 
@@ -266,6 +309,7 @@ def run_gpu(args, world, rank, local):
         "data": "synthetic (seeded torch Philox; shapes and value ranges of the RWKV-7 pages' workloads)",
         "config": {"workload": f"{args.workload}: {wl.name}", "B": B, "T": T, "H": H, "N": N,
                    "input_dtype": "bf16", "path": path, "chunk": args.chunk or None,
+                   "ctas_per_head": ctas_per_head,
                    "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world} (independent (b,h) units)",
                    "l2": (f"{n_sets} rotating input sets, {n_sets * B * T * H * N * 12 / 1e6:.0f} MB > 126 MB L2"
                           if not decode else "fp32 state 168 MB > 126 MB L2, 128 rotating token inputs")},

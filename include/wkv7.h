@@ -147,6 +147,18 @@ WKV7_API wkv7_status wkv7_decode_step(int B, int H, int N, wkv7_dtype dt,
  */
 WKV7_API wkv7_status wkv7_poll_device_error(void *stream);
 
+/*
+ * The path wkv7_forward takes for these arguments on the current device, without running
+ * anything: *algo = WKV7_ALGO_SEQ or WKV7_ALGO_CHUNK, and *segments = CTAs per (b, h) of the
+ * chunked path (1: one CTA per head; 2..WKV7_MAX_SEGMENTS: the chunks of a head spread over a
+ * thread-block cluster) or 0 for the scan. Reads the current device's SM count and cluster
+ * occupancy (WKV7_ERR_CUDA without a usable device); argument errors as in wkv7_forward.
+ * T = 0 (state copy only) and the scan report SEQ and 0 without touching the device.
+ * This query has no counterpart on the pages; it reports the dispatch of this library.
+ */
+WKV7_API wkv7_status wkv7_plan(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opts *opts,
+                               int *algo, int *segments);
+
 /* Bytes of device workspace wkv7_forward needs for these arguments (opts may be NULL). */
 WKV7_API size_t wkv7_workspace_bytes(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opts *opts);
 

@@ -100,6 +100,51 @@ bool mul_ok(size_t &acc, long long f) {
 
 }  // namespace
 
+// Sizes and options, shared by wkv7_forward and wkv7_plan; fills `opts` (defaults if NULL).
+wkv7_status check_args(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opts *opts_in, wkv7_opts &opts) {
+    if (N <= 0 || B <= 0 || H <= 0 || T < 0)
+        return fail(WKV7_ERR_ARG, "bad sizes B=%d T=%d H=%d N=%d (need B,H,N >= 1, T >= 0)", B, T, H, N);
+    if (N != wkv7::kN) return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: only N=64 is implemented", N);
+    if (dt != WKV7_F32 && dt != WKV7_BF16) return fail(WKV7_ERR_ARG, "unknown dtype %d", (int)dt);
+    wkv7_opts_default(&opts);
+    if (opts_in) opts = *opts_in;
+    if (opts.algo < WKV7_ALGO_AUTO || opts.algo > WKV7_ALGO_SPLIT)
+        return fail(WKV7_ERR_ARG, "unknown algo %d", opts.algo);
+    if (!(opts.chunk == 0 || opts.chunk == 16 || opts.chunk == 32 || opts.chunk == 64))
+        return fail(WKV7_ERR_ARG, "chunk=%d: must be 0 (default), 16, 32 or 64", opts.chunk);
+    if (opts.snap_every < 0) return fail(WKV7_ERR_ARG, "snap_every=%d < 0", opts.snap_every);
+    if (opts.snap_every > 0 && !opts.snapshots && T >= opts.snap_every)
+        return fail(WKV7_ERR_ARG, "snap_every=%d but snapshots is NULL", opts.snap_every);
+    const int n_epi = (opts.ln_w != nullptr) + (opts.ln_b != nullptr) + (opts.r_k != nullptr);
+    if (n_epi != 0 && n_epi != 3) return fail(WKV7_ERR_ARG, "epilogue needs all of ln_w, ln_b, r_k (or none)");
+    if (n_epi == 3 && !(std::isfinite(opts.gn_eps) && opts.gn_eps >= 0.f))
+        return fail(WKV7_ERR_ARG, "gn_eps must be finite and >= 0");
+    if (opts.segments < 0 || opts.segments > WKV7_MAX_SEGMENTS)
+        return fail(WKV7_ERR_ARG, "segments=%d outside 0..%d", opts.segments, WKV7_MAX_SEGMENTS);
+    return WKV7_OK;
+}
+
+// Whether the chunked kernel runs: forced by CHUNK / SPLIT (UNSUPPORTED if it cannot), chosen
+// by AUTO for bf16 inputs of at least 16 tokens.
+wkv7_status pick_chunk(const wkv7_opts &opts, const wkv7::FwdArgs &p, bool &use_chunk) {
+    const bool chunk_ok = wkv7::chunk_supported(p) && (opts.chunk == 0 || opts.chunk == 64);
+    use_chunk = false;
+    if (opts.algo == WKV7_ALGO_CHUNK || opts.algo == WKV7_ALGO_SPLIT) {
+        if (!chunk_ok)
+            return fail(WKV7_ERR_UNSUPPORTED,
+                        "chunked algorithm needs bf16 inputs, chunk 0 or 64 and snap_every a multiple of 64");
+        use_chunk = true;
+    } else if (opts.algo == WKV7_ALGO_AUTO) {
+        use_chunk = chunk_ok && p.T >= 16;
+    }
+    return WKV7_OK;
+}
+
+// CTAs per (b, h) requested of the chunked path: CHUNK one, SPLIT the caller's count (0 = choose).
+int requested_segments(const wkv7_opts &opts) {
+    return opts.algo == WKV7_ALGO_CHUNK ? 1 : (opts.algo == WKV7_ALGO_SPLIT ? opts.segments : 0);
+}
+
 extern "C" {
 
 void wkv7_opts_default(wkv7_opts *o) {
@@ -136,26 +181,10 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype dt, const void *
                          float *y, float *S_T, const wkv7_opts *opts_in, void *workspace,
                          size_t workspace_bytes, void *stream) {
     g_err[0] = '\0';
-    if (N <= 0 || B <= 0 || H <= 0 || T < 0)
-        return fail(WKV7_ERR_ARG, "bad sizes B=%d T=%d H=%d N=%d (need B,H,N >= 1, T >= 0)", B, T, H, N);
-    if (N != wkv7::kN) return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: only N=64 is implemented", N);
-    if (dt != WKV7_F32 && dt != WKV7_BF16) return fail(WKV7_ERR_ARG, "unknown dtype %d", (int)dt);
     wkv7_opts opts;
-    wkv7_opts_default(&opts);
-    if (opts_in) opts = *opts_in;
-    if (opts.algo < WKV7_ALGO_AUTO || opts.algo > WKV7_ALGO_SPLIT)
-        return fail(WKV7_ERR_ARG, "unknown algo %d", opts.algo);
-    if (!(opts.chunk == 0 || opts.chunk == 16 || opts.chunk == 32 || opts.chunk == 64))
-        return fail(WKV7_ERR_ARG, "chunk=%d: must be 0 (default), 16, 32 or 64", opts.chunk);
-    if (opts.snap_every < 0) return fail(WKV7_ERR_ARG, "snap_every=%d < 0", opts.snap_every);
-    if (opts.snap_every > 0 && !opts.snapshots && T >= opts.snap_every)
-        return fail(WKV7_ERR_ARG, "snap_every=%d but snapshots is NULL", opts.snap_every);
+    const wkv7_status vs = check_args(B, T, H, N, dt, opts_in, opts);
+    if (vs != WKV7_OK) return vs;
     const int n_epi = (opts.ln_w != nullptr) + (opts.ln_b != nullptr) + (opts.r_k != nullptr);
-    if (n_epi != 0 && n_epi != 3) return fail(WKV7_ERR_ARG, "epilogue needs all of ln_w, ln_b, r_k (or none)");
-    if (n_epi == 3 && !(std::isfinite(opts.gn_eps) && opts.gn_eps >= 0.f))
-        return fail(WKV7_ERR_ARG, "gn_eps must be finite and >= 0");
-    if (opts.segments < 0 || opts.segments > WKV7_MAX_SEGMENTS)
-        return fail(WKV7_ERR_ARG, "segments=%d outside 0..%d", opts.segments, WKV7_MAX_SEGMENTS);
 
     size_t tok = 1, st = 1;
     if (!mul_ok(tok, B) || !mul_ok(tok, T) || !mul_ok(tok, H) || !mul_ok(tok, N) || !mul_ok(st, B) ||
@@ -216,7 +245,7 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype dt, const void *
     p.snaps = n_snap ? opts.snapshots : nullptr;
     p.ln_w = opts.ln_w; p.ln_b = opts.ln_b; p.r_k = opts.r_k; p.gn_eps = opts.gn_eps;
     p.chunk = opts.chunk;
-    p.segments = opts.algo == WKV7_ALGO_CHUNK ? 1 : (opts.algo == WKV7_ALGO_SPLIT ? opts.segments : 0);
+    p.segments = requested_segments(opts);
     p.ws = workspace; p.ws_bytes = workspace_bytes;
     p.stream = static_cast<cudaStream_t>(stream);
 
@@ -225,16 +254,9 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype dt, const void *
         e = wkv7::launch_copy_state(p);
         return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "state copy launch");
     }
-    const bool chunk_ok = wkv7::chunk_supported(p) && (opts.chunk == 0 || opts.chunk == 64);
     bool use_chunk = false;
-    if (opts.algo == WKV7_ALGO_CHUNK || opts.algo == WKV7_ALGO_SPLIT) {
-        if (!chunk_ok)
-            return fail(WKV7_ERR_UNSUPPORTED,
-                        "chunked algorithm needs bf16 inputs, chunk 0 or 64 and snap_every a multiple of 64");
-        use_chunk = true;
-    } else if (opts.algo == WKV7_ALGO_AUTO) {
-        use_chunk = chunk_ok && T >= 16;
-    }
+    const wkv7_status ps = pick_chunk(opts, p, use_chunk);
+    if (ps != WKV7_OK) return ps;
     if (use_chunk) {
         e = wkv7::launch_chunk(p);
         if (e != cudaSuccess) return cuda_fail(e, "chunked-prefill launch");
@@ -246,6 +268,37 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype dt, const void *
         e = wkv7::launch_epilogue(p);
         if (e != cudaSuccess) return cuda_fail(e, "epilogue launch");
     }
+    return WKV7_OK;
+}
+
+wkv7_status wkv7_plan(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opts *opts_in, int *algo,
+                      int *segments) {
+    g_err[0] = '\0';
+    if (!algo || !segments) return fail(WKV7_ERR_ARG, "algo and segments must not be NULL");
+    wkv7_opts opts;
+    const wkv7_status vs = check_args(B, T, H, N, dt, opts_in, opts);
+    if (vs != WKV7_OK) return vs;
+    wkv7::FwdArgs p{};
+    p.B = B; p.T = T; p.H = H; p.dt = dt;
+    p.snap_every = (opts.snap_every > 0 && T >= opts.snap_every) ? opts.snap_every : 0;
+    p.chunk = opts.chunk;
+    p.segments = requested_segments(opts);
+    bool use_chunk = false;
+    const wkv7_status ps = pick_chunk(opts, p, use_chunk);
+    if (ps != WKV7_OK) return ps;
+    if (T == 0 || !use_chunk) {
+        *algo = WKV7_ALGO_SEQ;
+        *segments = 0;
+        return WKV7_OK;
+    }
+    int cs = 0;
+    const cudaError_t e = wkv7::chunk_segments(p, &cs);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return cuda_fail(e, "querying the device for the chunked path");
+    }
+    *algo = WKV7_ALGO_CHUNK;
+    *segments = cs;
     return WKV7_OK;
 }
 

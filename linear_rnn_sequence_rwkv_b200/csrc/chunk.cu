@@ -822,6 +822,16 @@ int choose_segments(int units, int nchunks, const DeviceInfo &d) {
 
 }  // namespace
 
+cudaError_t chunk_segments(const FwdArgs &p, int *segments) {
+    DeviceInfo *di = nullptr;
+    const cudaError_t e = device_info(di);
+    if (e != cudaSuccess) return e;
+    const int cs = p.segments > 0 ? p.segments : choose_segments(p.B * p.H, (p.T + C - 1) / C, *di);
+    if (cs > kMaxSegments || di->clusters[cs] <= 0) return cudaErrorInvalidClusterSize;
+    *segments = cs;
+    return cudaSuccess;
+}
+
 bool chunk_supported(const FwdArgs &p) {
     return p.dt == WKV7_BF16 && (p.snap_every == 0 || p.snap_every % C == 0);
 }
@@ -861,9 +871,9 @@ cudaError_t launch_chunk(const FwdArgs &p) {
     a.ln_w = p.ln_w; a.ln_b = p.ln_b; a.r_k = p.r_k; a.gn_eps = p.gn_eps;
     a.err = di->err;
     a.timeout_ns = 2000000000ull;
-    const int units = p.B * p.H, nchunks = (p.T + C - 1) / C;
-    const int cs = p.segments > 0 ? p.segments : choose_segments(units, nchunks, *di);
-    if (cs > kMaxSegments || di->clusters[cs] <= 0) return cudaErrorInvalidClusterSize;
+    const int units = p.B * p.H;
+    int cs = 1;
+    if ((e = chunk_segments(p, &cs)) != cudaSuccess) return e;
     const int ncl = units < di->clusters[cs] ? units : di->clusters[cs];
     cudaLaunchAttribute attr;
     const cudaLaunchConfig_t cfg = launch_config(ncl * cs, cs, p.stream, &attr);

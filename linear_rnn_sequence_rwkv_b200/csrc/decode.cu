@@ -58,6 +58,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecArgs p) {
 
 }  // namespace
 
+// ---- host side ---------------------------------------------------------------------------------------
+
 cudaError_t launch_decode(const DecArgs &p) {
     const unsigned units = unsigned(p.B) * unsigned(p.H);
     if (p.dt == WKV7_BF16)

@@ -28,7 +28,8 @@ F32, BF16 = 0, 1
 ALGOS = {"auto": 0, "seq": 1, "chunk": 2, "split": 3}
 
 EXPORTED = ("wkv7_opts_default", "wkv7_forward", "wkv7_decode_step", "wkv7_workspace_bytes",
-            "wkv7_status_string", "wkv7_last_error", "wkv7_abi_version", "wkv7_poll_device_error")
+            "wkv7_status_string", "wkv7_last_error", "wkv7_abi_version", "wkv7_poll_device_error",
+            "wkv7_plan")
 
 
 class Wkv7Error(RuntimeError):
@@ -79,6 +80,8 @@ def load():
         lib.wkv7_abi_version.restype = ci
         lib.wkv7_poll_device_error.argtypes = [vp]
         lib.wkv7_poll_device_error.restype = ci
+        lib.wkv7_plan.argtypes = [ci, ci, ci, ci, ci, ctypes.POINTER(Opts), ctypes.POINTER(ci), ctypes.POINTER(ci)]
+        lib.wkv7_plan.restype = ci
         _lib = lib
         return lib
 
@@ -121,6 +124,16 @@ def make_opts(algo="auto", chunk=0, snap_every=0, snapshots=None, ln_w=None, ln_
     o.gn_eps = float(gn_eps)
     o.segments = int(segments)
     return o
+
+
+def plan(B, T, H, N=HEAD_SIZE, dtype=torch.bfloat16, **opt_kw):
+    """(algorithm, CTAs per head) wkv7_forward would use on the current device: ("seq", 0) or
+    ("chunk", n) with n = 1 for one CTA per head and n > 1 for a cluster split."""
+    algo, seg = ctypes.c_int(0), ctypes.c_int(0)
+    st = load().wkv7_plan(B, T, H, N, BF16 if dtype == torch.bfloat16 else F32, ctypes.byref(make_opts(**opt_kw)),
+                          ctypes.byref(algo), ctypes.byref(seg))
+    _check(st, "wkv7_plan")
+    return ("seq" if algo.value == ALGOS["seq"] else "chunk"), int(seg.value)
 
 
 def workspace_bytes(B, T, H, N=HEAD_SIZE, dtype=torch.bfloat16, **opt_kw) -> int:

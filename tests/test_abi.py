@@ -115,3 +115,22 @@ def test_decode_rejects_bad_arguments(lib):
 
 def test_workspace_query_is_host_only(lib):
     assert wkv7.workspace_bytes(2, 128, 4) >= 0
+
+
+def test_plan_without_device(lib):
+    """The dispatch query answers the scan cases on the host and reports a CUDA error, not a
+    crash, when the chunked path would need the (absent) device."""
+    import torch
+    assert wkv7.plan(2, 8, 4) == ("seq", 0)                               # AUTO: < 16 tokens -> scan
+    assert wkv7.plan(2, 128, 4, dtype=torch.float32) == ("seq", 0)        # fp32 inputs -> scan
+    assert wkv7.plan(2, 0, 4) == ("seq", 0)                               # T = 0: state copy
+    with pytest.raises(wkv7.Wkv7Error) as e:
+        wkv7.plan(2, 128, 4, algo="split", segments=9)
+    assert e.value.status == wkv7.ERR_ARG
+    with pytest.raises(wkv7.Wkv7Error) as e:
+        wkv7.plan(2, 128, 4, algo="chunk", dtype=torch.float32)
+    assert e.value.status == wkv7.ERR_UNSUPPORTED
+    if not torch.cuda.is_available():
+        with pytest.raises(wkv7.Wkv7Error) as e:
+            wkv7.plan(2, 128, 4)
+        assert e.value.status == wkv7.ERR_CUDA

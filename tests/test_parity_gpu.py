@@ -352,3 +352,14 @@ def test_split_many_heads_per_cluster(cuda_device):
         ys, Ss, _ = _gpu(d, algo="split", segments=seg)
         assert torch.equal(ys, y1) and torch.equal(Ss, S1), seg
     wkv7.poll_device_error()
+
+
+def test_plan_matches_dispatch(cuda_device):
+    """wkv7_plan reports the path wkv7_forward takes: forced sizes are echoed, automatic ones
+    lie in 1..8, and the long-context shape (40 heads) is split across several CTAs."""
+    assert wkv7.plan(1, 1024, 2, algo="chunk") == ("chunk", 1)
+    assert wkv7.plan(1, 1024, 2, algo="split", segments=5) == ("chunk", 5)
+    algo, seg = wkv7.plan(1, 65536, 40)
+    assert algo == "chunk" and 2 <= seg <= 8
+    algo, seg = wkv7.plan(8, 1024, 12)
+    assert algo == "chunk" and 1 <= seg <= 8
