@@ -24,15 +24,16 @@
 //  * TMA (no multicast) stages the six bf16 [64 x 64] input tiles of the next chunk
 //    (128-byte swizzle) while the current chunk is processed.
 //  * Every MMA is tcgen05.mma kind::tf32, M=128, with the A operand in tensor memory
-//    (lane = row) and the B operand in shared memory (K-major, 128-byte swizzle). Five
-//    MMA rounds per chunk: Grams, Z, X, then the two state rounds into one accumulator.
-//  * 512 threads = 16 warps, four per SM sub-partition so that latency is hidden. A warp
-//    reaches only its quarter of the TMEM lanes: lanes 0-63 belong to warps w with w % 4 in
-//    {0, 1} ("column group": a key channel j or a token t, by phase), lanes 64-127 to the
-//    others ("row group": a token t or a key channel). The four warps sharing a lane quarter
-//    split the 64 columns (or tokens) into 16-wide parts.
-//  * The unit-lower-triangular inverse is done in fp32 on the CUDA cores: 16x16
-//    diagonal blocks by warp-shuffle substitution, then two levels of block merges.
+//    (lane = row) or shared memory and the B operand in shared memory (K-major, 128-byte
+//    swizzle); rounds that share an A operand are merged into N = 128.
+//  * 512 threads = 16 warps. A warp reaches only its quarter (warp % 4) of the TMEM lanes:
+//    lanes 0-63 hold key channels or the first 64 rows, lanes 64-127 tokens.
+//  * Software pipeline over the CTA's chunks. After chunk c's inverse, warps 0-3 run the
+//    dependent MMA rounds of chunk c and its output (state, y, epilogue) while warps 4-15
+//    wait for chunk c+1's tiles and compute its decay products and scaled operands
+//    (shared memory only). Everything that writes tensor memory waits for the join.
+//  * The unit-lower-triangular inverse: 16x16 diagonal blocks and one merge level on the
+//    CUDA cores in fp32, the merge of the two 32x32 halves on the tensor core.
 //  * Operands are rounded to tf32 (round to nearest) before the tensor core sees them;
 //    the carried state, the accumulators and all element-wise work stay fp32.
 // Every wait is bounded; a wait that gives up sets the device error word, the CTA
@@ -54,17 +55,19 @@ namespace {
 using namespace tc;
 
 constexpr int C = 64;             // chunk length (tokens)
-constexpr int kThreads = 512;   // 16 warps: 4 per SM sub-partition
-constexpr int kColThreads = 256;  // threads owning TMEM lanes 0-63: they write the next state
+constexpr int kThreads = 512;     // 16 warps
+constexpr int kBackThreads = 128; // warps 0-3: MMA rounds after the inverse, and the output
+constexpr int kFrontThreads = kThreads - kBackThreads;   // warps 4-15: the next chunk's operands
+constexpr int kSendThreads = 64;  // split mode: warps 0-1 write the next CTA's state operand
 constexpr int kMaxSegments = WKV7_MAX_SEGMENTS;   // CTAs per (b, h) in split mode (portable cluster size)
-constexpr int GTS = 68;           // row stride (floats) of the decay table: conflict-free row reads
+constexpr int GTS = 68;           // row stride (floats) of the decay table
 constexpr int LWS = 68;           // row stride of the inverse workspaces (16-byte aligned rows)
+constexpr int BAR_BACK = 1, BAR_FRONT = 2, BAR_SEND = 3;   // named barriers: warps 0-3, 4-15, 0-1
 
 // Shared-memory layout (byte offsets from a 1024-byte aligned base).
 constexpr uint32_t OFF_B1 = 0;        // [Bi; Ki] 128x64 tf32 (B of R1 and of the transpose round); then the
                                       // inverse workspace
 constexpr uint32_t OFF_B3 = 32768;    // [M_kb^T; KKd^T] 128x64 (B of R3)
-constexpr uint32_t OFF_L21 = 24576;   // inside B1, after the inverse workspace: L21^T 32x32 (B of R2b)
 constexpr uint32_t OFF_B2 = 65536;    // A^T 64x64 (B of R2); after R2, the y tile of the TMA store
                                       // (2 x [64][32] fp32), stored during the next chunk's R1
 constexpr uint32_t OFF_B4 = 81920;    // V^T 64x64 (B of R4; exact bf16 values)
@@ -72,19 +75,20 @@ constexpr uint32_t OFF_B5 = 98304;    // S 64x64, row = value channel (B of R5)
 constexpr uint32_t OFF_A1 = 114688;   // [KKd; Rd] 128x64 (A of R1)
 constexpr uint32_t OFF_IN = 147456;   // six bf16 [64][64] input tiles, TMA destination (swizzled)
 constexpr uint32_t OFF_GT = 196608;   // decay table [65][GTS] fp32; later the inverse [64][LWS]
-constexpr uint32_t OFF_SMALL = OFF_GT + 65 * GTS * 4;
+constexpr uint32_t OFF_L21 = (OFF_GT + 65 * GTS * 4 + 1023) & ~1023u;   // L21^T 32x32 (B of R2b)
+constexpr uint32_t OFF_SMALL = OFF_L21 + 4096;
 
 struct Small {
-    float gC[C];
-    float tq[8][C];       // decay product over each eighth of the chunk, per key channel
-    float bon[4][C];
-    float dk[4][C];       // r_t . k_t, partial over each column quarter (exact current-token Gram entry)
-    float db[4][C];       // r_t . (kk_t * a_t)
-    float red[4][C];
-    float ln_w[C], ln_b[C], r_k[C];
+    float gC[2][C];           // decay over the chunk per key channel, by chunk parity
+    float tq[4][C];           // decay product over each quarter of the chunk
+    float bon[2][C];          // epilogue bonus r_t . (k_t * r_k) per token, by chunk parity
+    float dk[C];              // r_t . k_t (exact current-token Gram entry)
+    float db[C];              // r_t . (kk_t * a_t)
+    float ln_w[2][C], ln_b[2][C], r_k[2][C];   // epilogue parameters, by head parity
     uint64_t bar_tma;
     uint64_t bar_mma;
-    uint64_t bar_state;   // split mode: the carried state has arrived in B5 (kColThreads remote arrivals)
+    uint64_t bar_state;       // split mode: the carried state has arrived in B5 (kSendThreads arrivals)
+    uint64_t bar_credit;      // split mode: the next CTA has consumed the state last sent to it
     uint32_t tmem_base;
 };
 constexpr uint32_t SMEM_BYTES = OFF_SMALL + sizeof(Small) + 1024;   // + alignment slack
@@ -158,8 +162,18 @@ __device__ __forceinline__ void in_row8(const uint8_t *tile, int t, int j, float
 __device__ __forceinline__ void st_f4(uint8_t *base, uint32_t off, float a, float b, float c, float d) {
     *reinterpret_cast<float4 *>(base + off) = make_float4(a, b, c, d);
 }
-// Barrier among the warps that own TMEM lanes 64-127 (8 warps).
-__device__ __forceinline__ void named_bar_rows() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void bar_named(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+// Named barrier that also ORs a predicate over its participants (the result is uniform).
+__device__ __forceinline__ bool bar_named_or(int id, int n, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(uint32_t(v)), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
 
 __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constant__ ChunkMaps maps, const ChunkArgs p) {
     extern __shared__ uint8_t smem_raw[];
@@ -177,6 +191,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     const int pq = warp >> 2;               // which 16-wide part of the 64 columns / tokens
     const int c16 = 16 * pq;
     const bool colg = L < 64;
+    const bool back = warp < 4;             // warps 0-3: one per TMEM lane quarter
+    const int ft = tid - kBackThreads;      // index among the front warps 4-15
     const int units = p.B * p.H;
     const int nchunks = (p.T + C - 1) / C;
     const bool epi = p.ln_w != nullptr;
@@ -189,7 +205,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     if (tid == 0) {
         mbar_init(&S.bar_tma, 1);
         mbar_init(&S.bar_mma, 1);
-        mbar_init(&S.bar_state, kColThreads);
+        mbar_init(&S.bar_state, kSendThreads);
+        mbar_init(&S.bar_credit, 1);
         mbar_fence_init();
     }
     if (warp == 0) {
@@ -201,9 +218,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     if (cs > 1) cluster_sync();   // every CTA's barriers are initialised before anyone arrives remotely
     tc_fence_after();
     const uint32_t tb = S.tmem_base;
-    const int next_rank = rank + 1 == cs ? 0 : rank + 1;
+    const int next_rank = rank + 1 == cs ? 0 : rank + 1, prev_rank = rank == 0 ? cs - 1 : rank - 1;
     const uint32_t next_b5 = map_to_rank(smem_u32(sm + OFF_B5), uint32_t(next_rank));
+    const uint32_t own_b5 = map_to_rank(smem_u32(sm + OFF_B5), uint32_t(rank));
     const uint32_t next_bar = map_to_rank(smem_u32(&S.bar_state), uint32_t(next_rank));
+    const uint32_t prev_credit = map_to_rank(smem_u32(&S.bar_credit), uint32_t(prev_rank));
     // matrix descriptors of the shared-memory operands at K-step 0
     const uint64_t dB1 = desc_sw128(smem_u32(sm + OFF_B1)), dB2 = desc_sw128(smem_u32(sm + OFF_B2));
     const uint64_t dB3 = desc_sw128(smem_u32(sm + OFF_B3)), dB4 = desc_sw128(smem_u32(sm + OFF_B4));
@@ -220,24 +239,37 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         }
         tmem_st_wait();
     }
-    uint32_t tma_parity = 0, mma_parity = 0, state_parity = 0;
+    uint32_t tma_parity = 0, mma_parity = 0, state_parity = 0, credit_parity = 0;
+    int sends = 0;                     // states sent to the next CTA (warps 0-1)
     bool y_pending = false;            // the y tile in B2 still has to be stored (uniform)
     int y_h = 0, y_c0 = 0, y_b = 0;    // its coordinates
     bool tma_pending = false, mma_pending = false, failed = false;
 
-    auto issue_tma = [&](int u, int c) {   // thread 0
+    auto issue_tma = [&](int u, int c) {   // one thread: the six tiles of chunk c of head u
         const int b = u / p.H, hh = u % p.H;
         mbar_arrive_expect_tx(&S.bar_tma, 6 * 8192);
 #pragma unroll
         for (int x = 0; x < 6; ++x) tma_load_4d(sm + OFF_IN + x * 8192, &maps.m[x], &S.bar_tma, 0, hh, c * C, b);
     };
-    // all threads; true on timeout here or (`extra`) in any thread (uniform across the CTA)
-    auto wait_mma = [&](bool extra = false) -> bool {
-        const bool to = !mbar_wait(&S.bar_mma, mma_parity, p.timeout_ns);
+    // Waits: one thread polls the mbarrier (bounded, acquire) and the others wait in a hardware
+    // barrier with it; many polling threads would crowd the shared-memory pipe that the other
+    // warp group is using. All threads; true on timeout (uniform across the CTA).
+    auto wait_mma_all = [&]() -> bool {
+        const bool to = tid == 0 && !mbar_wait_spin(&S.bar_mma, mma_parity, p.timeout_ns);
         mma_parity ^= 1u;
         mma_pending = false;
+        const bool f = __syncthreads_or(to) != 0;
         tc_fence_after();
-        return __syncthreads_or(to || extra) != 0;
+        return f;
+    };
+    // warps 0-3 only; true on timeout here or (`extra`) in any of them
+    auto wait_mma_back = [&](bool extra) -> bool {
+        const bool to = tid == 0 && !mbar_wait_spin(&S.bar_mma, mma_parity, p.timeout_ns);
+        mma_parity ^= 1u;
+        const bool f = bar_named_or(BAR_BACK, kBackThreads, to || extra);
+        tc_fence_after();
+        mma_pending = f;   // on a failure the round may still be running: drain it before exit
+        return f;
     };
     auto sync_for_mma = [&]() {            // writes to smem/TMEM -> visible to the next MMA
         fence_proxy_async_smem();
@@ -245,317 +277,449 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         tc_fence_before();
         __syncthreads();
     };
-
-    int unit = cid;
-    tma_pending = unit < units && rank < nchunks;
-    if (tid == 0 && tma_pending) issue_tma(unit, rank);
-
-    for (; unit < units && !failed; unit += ncl) {
-        const int b = unit / p.H, hh = unit % p.H;
-        // state operand S_0 (row = value channel i, K = key channel j), tf32-rounded; in split
-        // mode only the CTA that takes chunk 0 loads it, the others receive their states
-        for (int e = (rank == 0 ? tid : 1024); e < 1024; e += kThreads) {
+    auto load_params = [&](int u, int slot, int i) {   // epilogue parameters of head u, element i
+        const int hh = u % p.H;
+        S.ln_w[slot][i] = epi ? p.ln_w[hh * 64 + i] : 1.f;
+        S.ln_b[slot][i] = epi ? p.ln_b[hh * 64 + i] : 0.f;
+        S.r_k[slot][i] = epi ? p.r_k[hh * 64 + i] : 0.f;
+    };
+    auto load_state = [&](int u) {   // all threads: S_0 of head u (or zeros) -> B5, tf32, row = value channel
+        for (int e = tid; e < 1024; e += kThreads) {
             const int i = e >> 4, j4 = (e & 15) * 4;
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (p.S0) x = __ldg(reinterpret_cast<const float4 *>(p.S0 + size_t(unit) * 4096 + i * 64 + j4));
+            if (p.S0) x = __ldg(reinterpret_cast<const float4 *>(p.S0 + size_t(u) * 4096 + i * 64 + j4));
             st_f4(sm + OFF_B5, sw128_off(i, j4, 64), to_tf32(x.x), to_tf32(x.y), to_tf32(x.z), to_tf32(x.w));
         }
-        if (epi && tid < 64) {
-            S.ln_w[tid] = p.ln_w[hh * 64 + tid];
-            S.ln_b[tid] = p.ln_b[hh * 64 + tid];
-            S.r_k[tid] = p.r_k[hh * 64 + tid];
-        }
+    };
 
-        for (int c = rank; c < nchunks && !failed; c += cs) {
-            const int c0 = c * C, Lc = min(C, p.T - c0);
-            const bool last = c == nchunks - 1;
-            // this CTA's next chunk, whose inputs are prefetched during this one
-            int nu = unit, nc = c + cs;
-            if (nc >= nchunks) { nu = unit + ncl; nc = rank; }
-            const bool more = nu < units && nc < nchunks;
-            {   // ---- inputs of this chunk
-                const bool to = !mbar_wait(&S.bar_tma, tma_parity, p.timeout_ns);
-                tma_parity ^= 1u;
-                tma_pending = false;
-                if (__syncthreads_or(to)) { failed = true; break; }
-            }
-            // ---- P1: decay products per key channel j over each eighth of the chunk (all threads)
-            {
-                const int j = tid & 63, q = tid >> 6;
-                const uint8_t *wt = IN + XW * 8192;
-                uint32_t xo[8];
-                col_offsets(j, xo);
-                float run = 1.f;
+    // ---- front: the operands of chunk c of head u (warps 4-15, shared memory only): decay
+    //      products g_t (table GT, gC[ip]), KKd, Rd -> A1; Bi, Ki -> B1; exact current-token Grams.
+    //      Returns true (uniform over the front warps) if the input tiles did not arrive.
+    auto front = [&](int u, int c, int ip, int us) -> bool {
+        const int Lc = min(C, p.T - c * C);
+        const bool to = ft == 0 && !mbar_wait_spin(&S.bar_tma, tma_parity, p.timeout_ns);
+        tma_parity ^= 1u;
+        if (bar_named_or(BAR_FRONT, kFrontThreads, to)) return true;
+        // P1: decay products per key channel j over each quarter of the chunk (256 threads)
+        if (ft < 256) {
+            const int j = ft & 63, q = ft >> 6;
+            const uint8_t *wt = IN + XW * 8192;
+            uint32_t xo[8];
+            col_offsets(j, xo);
+            float run = 1.f;
+#pragma unroll 1
+            for (int h8 = 0; h8 < 2; ++h8) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const int t = 8 * q + e;
-                    run *= (t < Lc) ? in_col(wt, t, xo, e) : 1.f;   // padded tokens: w = 1
+                    const int t = 16 * q + 8 * h8 + e;
+                    const float w = in_col(wt, t, xo, e);
+                    run *= (t < Lc) ? w : 1.f;   // padded tokens: w = 1
                     GT[(t + 1) * GTS + j] = run;
                 }
-                S.tq[q][j] = run;
             }
-            __syncthreads();
-            // ---- P2: absolute products g_t (the eighths before this one as prefix)
-            {
-                const int j = tid & 63, q = tid >> 6;
+            S.tq[q][j] = run;
+        }
+        bar_named(BAR_FRONT, kFrontThreads);
+        // P2: absolute products g_t (the quarters before this one as prefix)
+        if (ft < 256) {
+            const int j = ft & 63, q = ft >> 6;
+            if (q > 0) {
                 float pre = 1.f;
                 for (int qq = 0; qq < q; ++qq) pre *= S.tq[qq][j];
-                if (q > 0) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) GT[(8 * q + e + 1) * GTS + j] *= pre;
-                } else {
-                    GT[j] = 1.f;
-                    float g = 1.f;
+                for (int e = 0; e < 16; ++e) GT[(16 * q + e + 1) * GTS + j] *= pre;
+            } else {
+                GT[j] = 1.f;
+                S.gC[ip][j] = S.tq[0][j] * S.tq[1][j] * S.tq[2][j] * S.tq[3][j];
+            }
+        }
+        bar_named(BAR_FRONT, kFrontThreads);
+        // P3: one (token t, channel octet o) per thread and pass. In a quarter-warp, token t takes
+        //     octets 0-3 and token t+1 octets 4-7 (or the reverse), so the swizzled bf16 reads, the
+        //     decay-table rows and the tf32 stores of the eight lanes all fall on distinct banks.
+        const int fw = ft >> 5, half = lane >> 4, qa = (lane >> 3) & 1, s8 = lane & 7;
+        const int hi = s8 >> 2, sub = s8 & 3;
+        const int j0 = 8 * (sub + 4 * (qa ^ hi));
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass) {
+            const int tbase = 4 * (fw + 12 * pass);
+            if (tbase >= C) break;   // warp-uniform
+            const int t = tbase + 2 * half + hi;
+            float r8[8], kk8[8], k8[8], a8[8];
+            in_row8(IN + XR * 8192, t, j0, r8);
+            in_row8(IN + XKK * 8192, t, j0, kk8);
+            in_row8(IN + XK * 8192, t, j0, k8);
+            in_row8(IN + XA * 8192, t, j0, a8);
+            const float4 ga = *reinterpret_cast<const float4 *>(GT + t * GTS + j0);         // g_{t-1}
+            const float4 gb = *reinterpret_cast<const float4 *>(GT + t * GTS + j0 + 4);
+            const float4 gc = *reinterpret_cast<const float4 *>(GT + (t + 1) * GTS + j0);   // g_t
+            const float4 gd = *reinterpret_cast<const float4 *>(GT + (t + 1) * GTS + j0 + 4);
+            const float gpv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+            const float gtv[8] = {gc.x, gc.y, gc.z, gc.w, gd.x, gd.y, gd.z, gd.w};
+            float kkd[8], rd[8], bi[8], ki[8], dk = 0.f, db = 0.f, bon = 0.f;
 #pragma unroll
-                    for (int qq = 0; qq < 8; ++qq) g *= S.tq[qq][j];
-                    S.gC[j] = g;
+            for (int e = 0; e < 8; ++e) {
+                const float inv = __fdividef(1.f, gtv[e]);
+                const float bb = kk8[e] * a8[e];
+                kkd[e] = to_tf32(kk8[e] * gpv[e]);
+                rd[e] = to_tf32(r8[e] * gtv[e]);
+                bi[e] = to_tf32(bb * inv);
+                ki[e] = to_tf32(k8[e] * inv);
+                dk = fmaf(r8[e], k8[e], dk);
+                db = fmaf(r8[e], bb, db);
+                bon = fmaf(r8[e] * k8[e], S.r_k[us][j0 + e], bon);   // r_k = 0 without the epilogue
+            }
+            st_f4(sm + OFF_A1, sw128_off(t, j0, 128), kkd[0], kkd[1], kkd[2], kkd[3]);
+            st_f4(sm + OFF_A1, sw128_off(t, j0 + 4, 128), kkd[4], kkd[5], kkd[6], kkd[7]);
+            st_f4(sm + OFF_A1, sw128_off(64 + t, j0, 128), rd[0], rd[1], rd[2], rd[3]);
+            st_f4(sm + OFF_A1, sw128_off(64 + t, j0 + 4, 128), rd[4], rd[5], rd[6], rd[7]);
+            st_f4(sm + OFF_B1, sw128_off(t, j0, 128), bi[0], bi[1], bi[2], bi[3]);
+            st_f4(sm + OFF_B1, sw128_off(t, j0 + 4, 128), bi[4], bi[5], bi[6], bi[7]);
+            st_f4(sm + OFF_B1, sw128_off(64 + t, j0, 128), ki[0], ki[1], ki[2], ki[3]);
+            st_f4(sm + OFF_B1, sw128_off(64 + t, j0 + 4, 128), ki[4], ki[5], ki[6], ki[7]);
+            // the eight octets of token t sit in lanes differing in bits 0, 1 and 3
+#pragma unroll
+            for (int m = 1; m <= 8; m <<= 1) {
+                if (m == 4) continue;
+                dk += __shfl_xor_sync(0xffffffffu, dk, m);
+                db += __shfl_xor_sync(0xffffffffu, db, m);
+                bon += __shfl_xor_sync(0xffffffffu, bon, m);
+            }
+            if (sub == 0 && qa == 0) {
+                S.dk[t] = dk;
+                S.db[t] = db;
+                S.bon[ip][t] = bon;
+            }
+        }
+        return false;
+    };
+
+    // ---- back, second half: the state and y of chunk c of head u (warps 0-3), from T_D4.
+    //      Returns true on a failed wait (uniform over warps 0-3).
+    auto out = [&](int u, int c, int ip, int us) -> bool {
+        const int b = u / p.H, hh = u % p.H, c0 = c * C, done = c0 + min(C, p.T - c0);
+        const bool last = c == nchunks - 1;
+        const bool snap = p.snap_every > 0 && done % p.snap_every == 0;
+        bool fail = false;
+        if (warp < 2) {   // TMEM lane j = key channel: S'[i][j] for all value channels i
+            const int j = L;
+            const float gCj = S.gC[ip][j];
+            uint32_t xo[8];
+            kcol_offsets(j, 64, xo);
+            // split mode: the state goes straight into the next CTA's B5 (distributed shared memory),
+            // once that CTA has consumed the state sent before (its credit)
+            const bool send = cs > 1 && c + 1 < nchunks;
+            if (send && sends > 0) {
+                const bool to = tid == 0 && !mbar_wait_cluster(&S.bar_credit, credit_parity, p.timeout_ns);
+                credit_parity ^= 1u;
+                fail = bar_named_or(BAR_SEND, kSendThreads, to);
+            }
+            const bool write_b5 = cs == 1 || (send && !fail);
+            const uint32_t b5_dst = cs == 1 ? own_b5 : next_b5;
+            float *gdst = nullptr;    // S_T or a snapshot, if this chunk ends one
+            if (last && p.S_T) gdst = p.S_T + size_t(u) * 4096;
+            else if (snap) gdst = p.snaps + ((size_t(b) * p.n_snap + (done / p.snap_every - 1)) * p.H + hh) * 4096;
+            float *sdst = (snap && last && p.S_T)   // the last chunk can also end a snapshot
+                              ? p.snaps + ((size_t(b) * p.n_snap + (done / p.snap_every - 1)) * p.H + hh) * 4096
+                              : nullptr;
+            if (write_b5) {
+#pragma unroll 1
+                for (int h2 = 0; h2 < 64; h2 += 32) {
+                    float v[4][8];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) tmem_ld8_nowait(tmem_addr(tb, Lq, T_D4 + h2 + 8 * q), v[q]);
+                    tmem_ld_wait(v[0], v[1], v[2], v[3]);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)   // S_C = S' diag(gC), this CTA's B5 or the next CTA's
+                            st_cluster(b5_dst + (h2 + 8 * q + e) * 128 + xo[e], to_tf32(v[q][e] * gCj));
                 }
             }
-            __syncthreads();
-            // ---- P3: token rows. Lanes 0-63 (token t = L): KKd row -> A1 rows 0-63, Ki row -> B1,
-            //      identity row -> T_D3L (start of P). Lanes 64-127 (token t): Rd row -> A1 rows 64-127
-            //      and T_D3L (start of R~), Bi row -> B1, exact current-token Grams.
-            if (colg) {
-                const int t = L;
-                const float *gp = GT + t * GTS;         // g_{t-1}
-                const float *gt = GT + (t + 1) * GTS;   // g_t
+            if (gdst || sdst) {   // the end of the sequence or of a snapshot interval: fp32 state out
 #pragma unroll 1
-                for (int g = 0; g < 2; ++g) {
-                    const int j0 = c16 + 8 * g;
-                    float kk8[8], k8[8], v[8], ki[8];
-                    in_row8(IN + XKK * 8192, t, j0, kk8);
-                    in_row8(IN + XK * 8192, t, j0, k8);
-                    const float4 ga = *reinterpret_cast<const float4 *>(gp + j0);
-                    const float4 gb = *reinterpret_cast<const float4 *>(gp + j0 + 4);
-                    const float4 gc = *reinterpret_cast<const float4 *>(gt + j0);
-                    const float4 gd = *reinterpret_cast<const float4 *>(gt + j0 + 4);
-                    const float gpv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-                    const float gtv[8] = {gc.x, gc.y, gc.z, gc.w, gd.x, gd.y, gd.z, gd.w};
+                for (int i0 = 0; i0 < 64; i0 += 8) {
+                    float v[8];
+                    tmem_ld8(tmem_addr(tb, Lq, T_D4 + i0), v);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        v[e] = to_tf32(kk8[e] * gpv[e]);
-                        ki[e] = to_tf32(k8[e] * __fdividef(1.f, gtv[e]));
+                        if (gdst) gdst[(i0 + e) * 64 + j] = v[e] * gCj;
+                        if (sdst) sdst[(i0 + e) * 64 + j] = v[e] * gCj;
                     }
-                    st_f4(sm + OFF_A1, sw128_off(t, j0, 128), v[0], v[1], v[2], v[3]);
-                    st_f4(sm + OFF_A1, sw128_off(t, j0 + 4, 128), v[4], v[5], v[6], v[7]);
-                    st_f4(sm + OFF_B1, sw128_off(64 + t, j0, 128), ki[0], ki[1], ki[2], ki[3]);
-                    st_f4(sm + OFF_B1, sw128_off(64 + t, j0 + 4, 128), ki[4], ki[5], ki[6], ki[7]);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] = (j0 + e == t) ? 1.f : 0.f;
-                    tmem_st8(tmem_addr(tb, Lq, T_D3L + j0), v);
                 }
-            } else {
-                const int t = L - 64;
-                const float *gt = GT + (t + 1) * GTS;   // g_t
-                float bon = 0.f, dk = 0.f, db = 0.f;
+            }
+            if (send) {
+                if (!fail) {
+                    fence_proxy_async_cluster();
+                    mbar_arrive_remote(next_bar);
+                }
+                ++sends;
+            }
+        } else {          // TMEM lane 64 + t: y row t
+            const int t = L - 64;
+            const uint32_t yrow = tmem_addr(tb, Lq, T_D4);
+            float mean = 0.f, inv = 0.f, bon = 0.f;
+            uint32_t xv[8];
+            if (epi) {   // group_norm statistics over the head's 64 channels (two passes over TMEM)
+                float s1 = 0.f, s2 = 0.f;
 #pragma unroll 1
-                for (int g = 0; g < 2; ++g) {
-                    const int j0 = c16 + 8 * g;
-                    float r8[8], kk8[8], a8[8], k8[8], rd[8], bi[8];
-                    in_row8(IN + XR * 8192, t, j0, r8);
-                    in_row8(IN + XKK * 8192, t, j0, kk8);
-                    in_row8(IN + XA * 8192, t, j0, a8);
-                    in_row8(IN + XK * 8192, t, j0, k8);
-                    const float4 ga = *reinterpret_cast<const float4 *>(gt + j0);
-                    const float4 gb = *reinterpret_cast<const float4 *>(gt + j0 + 4);
-                    const float g8v[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                for (int i0 = 0; i0 < 64; i0 += 8) {
+                    float v[8];
+                    tmem_ld8(yrow + i0, v);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) s1 += v[e];
+                }
+                mean = s1 * (1.f / 64.f);
+#pragma unroll 1
+                for (int i0 = 0; i0 < 64; i0 += 8) {
+                    float v[8];
+                    tmem_ld8(yrow + i0, v);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) s2 = fmaf(v[e] - mean, v[e] - mean, s2);
+                }
+                inv = 1.f / sqrtf(s2 * (1.f / 64.f) + p.gn_eps);
+                bon = S.bon[ip][t];
+                kcol_offsets(t, 64, xv);
+            }
+            // y row t -> the swizzled [64][32] fp32 tiles (one per channel half) the y tensor map
+            // expects; rows past the end of T are clipped by the store
+#pragma unroll 1
+            for (int i0 = 0; i0 < 64; i0 += 8) {
+                float v[8];
+                tmem_ld8(yrow + i0, v);
+                if (epi) {   // (y - mean) / sqrt(var + eps) * ln_w + ln_b + (r.(k*r_k)) v
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float bb = kk8[e] * a8[e];
-                        rd[e] = to_tf32(r8[e] * g8v[e]);
-                        bi[e] = to_tf32(bb * __fdividef(1.f, g8v[e]));
-                        dk = fmaf(r8[e], k8[e], dk);
-                        db = fmaf(r8[e], bb, db);
-                        if (epi) bon = fmaf(r8[e] * k8[e], S.r_k[j0 + e], bon);
+                        const int i = i0 + e;
+                        const float vi = *reinterpret_cast<const float *>(sm + OFF_B4 + i * 128 + xv[e]);
+                        v[e] = fmaf((v[e] - mean) * inv, S.ln_w[us][i], S.ln_b[us][i]) + bon * vi;
                     }
-                    st_f4(sm + OFF_A1, sw128_off(64 + t, j0, 128), rd[0], rd[1], rd[2], rd[3]);
-                    st_f4(sm + OFF_A1, sw128_off(64 + t, j0 + 4, 128), rd[4], rd[5], rd[6], rd[7]);
-                    tmem_st8(tmem_addr(tb, Lq, T_D3L + j0), rd);
-                    st_f4(sm + OFF_B1, sw128_off(t, j0, 128), bi[0], bi[1], bi[2], bi[3]);
-                    st_f4(sm + OFF_B1, sw128_off(t, j0 + 4, 128), bi[4], bi[5], bi[6], bi[7]);
                 }
-                S.dk[pq][t] = dk;
-                S.db[pq][t] = db;
-                if (epi) S.bon[pq][t] = bon;
+                uint8_t *row = sm + OFF_B2 + (i0 >> 5) * 8192 + t * 128;
+                const int q = (i0 & 31) >> 2;
+                *reinterpret_cast<float4 *>(row + ((q ^ (t & 7)) << 4)) = make_float4(v[0], v[1], v[2], v[3]);
+                *reinterpret_cast<float4 *>(row + (((q + 1) ^ (t & 7)) << 4)) = make_float4(v[4], v[5], v[6], v[7]);
             }
-            sync_for_mma();
-            if (tid == 0) {
-                // the next chunk's six input tiles are issued by six warps in P5; their byte count
-                // is registered here, ordered before those issues by the barrier after R1
-                if (more) mbar_arrive_expect_tx(&S.bar_tma, 6 * 8192);
-                tc_fence_after();
+        }
+        return bar_named_or(BAR_BACK, kBackThreads, fail);
+    };
+
+    // ---- the CTA's chunks: (head u, chunk c), c = rank, rank + cs, ... of heads cid, cid + ncl, ...
+    int u = cid, c = rank;
+    bool valid = u < units && rank < nchunks;
+    int ip = 0, us = 0;                // parity slots of the current chunk and head
+    if (valid) {
+        if (tid == 0) issue_tma(u, c);
+        tma_pending = true;
+        if (tid < 64) load_params(u, 0, tid);
+        if (rank == 0) load_state(u);
+    }
+    __syncthreads();
+    {
+        const bool f = valid && !back ? front(u, c, 0, 0) : false;
+        failed = __syncthreads_or(f) != 0;
+        if (valid && back) tma_parity ^= 1u;
+        if (!failed) tma_pending = false;
+    }
+
+    while (valid && !failed) {
+        const int b = u / p.H, hh = u % p.H, c0 = c * C;
+        int nu = u, nc = c + cs;
+        if (nc >= nchunks) { nu = u + ncl; nc = rank; }
+        const bool more = nu < units && nc < nchunks;
+        const bool new_unit = more && nu != u;
+        const bool recv = cs > 1 && c > 0;   // split mode: this chunk's start state comes from CTA rank-1
+
+        if (tid == 0) {
+            // the next chunk's six input tiles are issued by six warps in P5; their byte count
+            // is registered here, ordered before those issues by the barrier after R1
+            if (more) mbar_arrive_expect_tx(&S.bar_tma, 6 * 8192);
+            tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)   // R1: Grams = [KKd; Rd] [Bi; Ki]^T
-                    mma_tf32_ss(tb + T_D1, dA1 + kstep_off(ks, 128), dB1 + kstep_off(ks, 128), idesc_tf32(128, 128), ks > 0);
-                // transpose round on the tensor core (exact: identity times tf32 operands), N = 128:
-                // lanes 0-63 of T_A2 <- Bi^T (A of R2), of T_D3R <- Ki^T (start of K~)
+            for (int ks = 0; ks < 8; ++ks)   // R1: Grams = [KKd; Rd] [Bi; Ki]^T
+                mma_tf32_ss(tb + T_D1, dA1 + kstep_off(ks, 128), dB1 + kstep_off(ks, 128), idesc_tf32(128, 128), ks > 0);
+            // transpose round on the tensor core (exact: identity times tf32 operands), N = 128:
+            // lanes 0-63 of T_A2 <- Bi^T (A of R2), of T_D3R <- Ki^T (start of K~)
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_tf32_ts(tb + T_A2, tb + T_ID + 8 * ks, dB1 + kstep_off(ks, 128), idesc_tf32(128, 128), ks > 0);
-                mma_commit(&S.bar_mma);
-            }
-            mma_pending = true;
-            // the previous chunk's y tile goes out now: every warp has slack while R1 runs
-            if (y_pending && tid == kStoreThread) store_y_tile(maps, sm + OFF_B2, y_h, y_c0, y_b);
-            y_pending = false;
-            // ---- P4 (while the MMAs run): transposes through shared memory, no arithmetic.
-            //      Lanes 0-63 (key/value channel j = L): V^T row j -> B4.
-            //      Lanes 64-127 (key j = L - 64): KKd^T row j -> B3 rows 64-127.
-            if (colg) {
-                const int j = L;
-                uint32_t xo[8];
-                col_offsets(j, xo);
+            for (int ks = 0; ks < 8; ++ks)
+                mma_tf32_ts(tb + T_A2, tb + T_ID + 8 * ks, dB1 + kstep_off(ks, 128), idesc_tf32(128, 128), ks > 0);
+            mma_commit(&S.bar_mma);
+        }
+        mma_pending = true;
+        // the previous chunk's y tile goes out now: every warp has slack while R1 runs
+        if (y_pending && tid == kStoreThread) store_y_tile(maps, sm + OFF_B2, y_h, y_c0, y_b);
+        y_pending = false;
+        // ---- P4 (while the MMAs run): transposes through shared memory and the start of
+        //      T_D3L (the previous chunk's R5 has read it).
+        //      Lanes 0-63 (key/value channel j = L): V^T row j -> B4; identity row -> T_D3L.
+        //      Lanes 64-127 (key j = L - 64): KKd^T row j -> B3 rows 64-127; Rd row t = j -> T_D3L.
+        if (colg) {
+            const int j = L;
+            uint32_t xo[8];
+            col_offsets(j, xo);
 #pragma unroll 1
-                for (int g = 0; g < 2; ++g) {
-                    const int t0 = c16 + 8 * g;
-                    float vv[8];
+            for (int g = 0; g < 2; ++g) {
+                const int t0 = c16 + 8 * g;
+                float vv[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) vv[e] = in_col(IN + XV * 8192, t0 + e, xo, e);
-                    st_f4(sm + OFF_B4, sw128_off(j, t0, 64), vv[0], vv[1], vv[2], vv[3]);
-                    st_f4(sm + OFF_B4, sw128_off(j, t0 + 4, 64), vv[4], vv[5], vv[6], vv[7]);
-                }
-            } else {
-                const int j = L - 64;
-                uint32_t xo[8];
-                kcol_offsets(j, 128, xo);
-                const uint8_t *b6 = sm + OFF_A1;
+                for (int e = 0; e < 8; ++e) vv[e] = in_col(IN + XV * 8192, t0 + e, xo, e);
+                st_f4(sm + OFF_B4, sw128_off(j, t0, 64), vv[0], vv[1], vv[2], vv[3]);
+                st_f4(sm + OFF_B4, sw128_off(j, t0 + 4, 64), vv[4], vv[5], vv[6], vv[7]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) vv[e] = (t0 + e == L) ? 1.f : 0.f;
+                tmem_st8(tmem_addr(tb, Lq, T_D3L + t0), vv);
+            }
+        } else {
+            const int j = L - 64;
+            uint32_t xo[8];
+            kcol_offsets(j, 128, xo);
+            const uint8_t *b6 = sm + OFF_A1;
 #pragma unroll 1
-                for (int g = 0; g < 2; ++g) {
-                    const int t0 = c16 + 8 * g;
-                    float kkd[8];
+            for (int g = 0; g < 2; ++g) {
+                const int t0 = c16 + 8 * g;
+                float kkd[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) kkd[e] = *reinterpret_cast<const float *>(b6 + (t0 + e) * 128 + xo[e]);
-                    st_f4(sm + OFF_B3, sw128_off(64 + j, t0, 128), kkd[0], kkd[1], kkd[2], kkd[3]);
-                    st_f4(sm + OFF_B3, sw128_off(64 + j, t0 + 4, 128), kkd[4], kkd[5], kkd[6], kkd[7]);
-                }
+                for (int e = 0; e < 8; ++e) kkd[e] = *reinterpret_cast<const float *>(b6 + (t0 + e) * 128 + xo[e]);
+                st_f4(sm + OFF_B3, sw128_off(64 + j, t0, 128), kkd[0], kkd[1], kkd[2], kkd[3]);
+                st_f4(sm + OFF_B3, sw128_off(64 + j, t0 + 4, 128), kkd[4], kkd[5], kkd[6], kkd[7]);
+                const float4 ra = *reinterpret_cast<const float4 *>(b6 + sw128_off(64 + j, t0, 128));
+                const float4 rb = *reinterpret_cast<const float4 *>(b6 + sw128_off(64 + j, t0 + 4, 128));
+                const float rd[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+                tmem_st8(tmem_addr(tb, Lq, T_D3L + t0), rd);   // Rd row (token j), channels t0..t0+7
             }
-            if (wait_mma()) { failed = true; break; }
-            // ---- P5: masks. Lanes 0-63 (token t): M_ab row -> inverse workspace; M_kb row t ->
-            //      column t of B3 rows 0-63 (M_kb^T, scalar stores along K: conflict-free).
-            //      Lanes 64-127 (token t): Q_b row -> T_A2 lanes 64-127; Q_k row -> T_D3R lanes 64-127.
-            if (more && lane == 0 && colg && (warp >> 2) < 3) {
-                // the input tiles were last read in P4: six warps each issue one tile of the next chunk
-                const int x = (warp >> 2) * 2 + (warp & 1);
-                tma_load_4d(sm + OFF_IN + x * 8192, &maps.m[x], &S.bar_tma, 0, nu % p.H, nc * C, nu / p.H);
+        }
+        if (wait_mma_all()) { failed = true; break; }
+        // ---- P5: masks. Lanes 0-63 (token t): M_ab row -> inverse workspace; M_kb row t ->
+        //      column t of B3 rows 0-63 (M_kb^T, scalar stores along K: conflict-free).
+        //      Lanes 64-127 (token t): Q_b row -> T_A2 lanes 64-127; Q_k row -> T_D3R lanes 64-127.
+        if (more && lane == 0 && colg && (warp >> 2) < 3) {
+            // the input tiles were last read in P4: six warps each issue one tile of the next chunk
+            const int x = (warp >> 2) * 2 + (warp & 1);
+            tma_load_4d(sm + OFF_IN + x * 8192, &maps.m[x], &S.bar_tma, 0, nu % p.H, nc * C, nu / p.H);
+        }
+        if (colg) {
+            const int t = L;
+            float m[2][8], mk[2][8];
+            tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + c16), m[0]);
+            tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + c16 + 8), m[1]);
+            tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + 64 + c16), mk[0]);
+            tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + 64 + c16 + 8), mk[1]);
+            tmem_ld_wait(m[0], m[1], mk[0], mk[1]);
+            uint32_t xo[8];
+            kcol_offsets(t, 128, xo);
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                const int s0 = c16 + 8 * g;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) m[g][e] = (s0 + e < t) ? m[g][e] : 0.f;
+                *reinterpret_cast<float4 *>(Lw + t * LWS + s0) = make_float4(m[g][0], m[g][1], m[g][2], m[g][3]);
+                *reinterpret_cast<float4 *>(Lw + t * LWS + s0 + 4) = make_float4(m[g][4], m[g][5], m[g][6], m[g][7]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)   // B3[s][t] = M_kb[t][s], nonzero for s < t
+                    *reinterpret_cast<float *>(sm + OFF_B3 + (s0 + e) * 128 + xo[e]) =
+                        (s0 + e < t) ? to_tf32(mk[g][e]) : 0.f;
             }
-            if (colg) {
-                const int t = L;
-                float m[2][8], mk[2][8];
-                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + c16), m[0]);
-                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + c16 + 8), m[1]);
-                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + 64 + c16), mk[0]);
-                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + 64 + c16 + 8), mk[1]);
-                tmem_ld_wait(m[0], m[1], mk[0], mk[1]);
-                uint32_t xo[8];
-                kcol_offsets(t, 128, xo);
+            if (t >= 32 && c16 < 32) {   // L21^T[s][t - 32] = M_ab[t][s] (s < 32 <= t: no mask)
+                uint32_t xl[8];
+                kcol_offsets(t - 32, 32, xl);
 #pragma unroll
-                for (int g = 0; g < 2; ++g) {
-                    const int s0 = c16 + 8 * g;
+                for (int g = 0; g < 2; ++g)
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) m[g][e] = (s0 + e < t) ? m[g][e] : 0.f;
-                    *reinterpret_cast<float4 *>(Lw + t * LWS + s0) = make_float4(m[g][0], m[g][1], m[g][2], m[g][3]);
-                    *reinterpret_cast<float4 *>(Lw + t * LWS + s0 + 4) = make_float4(m[g][4], m[g][5], m[g][6], m[g][7]);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)   // B3[s][t] = M_kb[t][s], nonzero for s < t
-                        *reinterpret_cast<float *>(sm + OFF_B3 + (s0 + e) * 128 + xo[e]) =
-                            (s0 + e < t) ? to_tf32(mk[g][e]) : 0.f;
-                }
-                if (t >= 32 && c16 < 32) {   // L21^T[s][t - 32] = M_ab[t][s] (s < 32 <= t: no mask)
-                    uint32_t xl[8];
-                    kcol_offsets(t - 32, 32, xl);
-#pragma unroll
-                    for (int g = 0; g < 2; ++g)
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            *reinterpret_cast<float *>(sm + OFF_L21 + (c16 + 8 * g + e) * 128 + xl[e]) = to_tf32(m[g][e]);
-                }
-            } else {
-                const int t = L - 64;
-                // the current-token entries are taken exactly in fp32: they dominate short sequences
-                const float dgb = to_tf32(S.db[0][t] + S.db[1][t] + S.db[2][t] + S.db[3][t]);
-                const float dgk = S.dk[0][t] + S.dk[1][t] + S.dk[2][t] + S.dk[3][t];
-                float qb[2][8], qk[2][8];
-                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + c16), qb[0]);            // Q_b row t
-                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + c16 + 8), qb[1]);
-                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + 64 + c16), qk[0]);       // Q_k row t
-                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + 64 + c16 + 8), qk[1]);
-                tmem_ld_wait(qb[0], qb[1], qk[0], qk[1]);
-#pragma unroll
-                for (int g = 0; g < 2; ++g) {
-                    const int s0 = c16 + 8 * g;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int ss = s0 + e;
-                        qb[g][e] = ss < t ? to_tf32(qb[g][e]) : (ss == t ? dgb : 0.f);
-                        qk[g][e] = ss < t ? qk[g][e] : (ss == t ? dgk : 0.f);
-                    }
-                    tmem_st8(tmem_addr(tb, Lq, T_A2 + s0), qb[g]);
-                    tmem_st8(tmem_addr(tb, Lq, T_D3R + s0), qk[g]);
-                }
+                    for (int e = 0; e < 8; ++e)
+                        *reinterpret_cast<float *>(sm + OFF_L21 + (c16 + 8 * g + e) * 128 + xl[e]) = to_tf32(m[g][e]);
             }
-            sync_for_mma();
-            tma_pending = more;
-            // ---- A = (I + M_ab)^{-1}. Diagonal 16x16 blocks: one thread per (block, column)
-            //      solves (I + L_dd) x = e_c by forward substitution in registers (warps 2, 3).
-            if (tid >= 64 && tid < 128) {
-                const int d = (tid - 64) >> 4, cc = tid & 15;
-                const float *Lb = Lw + 16 * d * LWS + 16 * d;
-                float x[16];
+        } else {
+            const int t = L - 64;
+            // the current-token entries are taken exactly in fp32: they dominate short sequences
+            const float dgb = to_tf32(S.db[t]);
+            const float dgk = S.dk[t];
+            float qb[2][8], qk[2][8];
+            tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + c16), qb[0]);            // Q_b row t
+            tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + c16 + 8), qb[1]);
+            tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + 64 + c16), qk[0]);       // Q_k row t
+            tmem_ld8_nowait(tmem_addr(tb, Lq, T_D1 + 64 + c16 + 8), qk[1]);
+            tmem_ld_wait(qb[0], qb[1], qk[0], qk[1]);
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    float acc = (r == cc) ? 1.f : 0.f;
+            for (int g = 0; g < 2; ++g) {
+                const int s0 = c16 + 8 * g;
 #pragma unroll
-                    for (int k = 0; k < r; ++k) acc = fmaf(-Lb[r * LWS + k], x[k], acc);
-                    x[r] = acc;
+                for (int e = 0; e < 8; ++e) {
+                    const int ss = s0 + e;
+                    qb[g][e] = ss < t ? to_tf32(qb[g][e]) : (ss == t ? dgb : 0.f);
+                    qk[g][e] = ss < t ? qk[g][e] : (ss == t ? dgk : 0.f);
                 }
-#pragma unroll
-                for (int r = 0; r < 16; ++r) Aw[(16 * d + r) * LWS + 16 * d + cc] = x[r];
+                tmem_st8(tmem_addr(tb, Lq, T_A2 + s0), qb[g]);
+                tmem_st8(tmem_addr(tb, Lq, T_D3R + s0), qk[g]);
             }
-            __syncthreads();
-            // level 1: X[2p+1][2p] = -X[2p+1] (L[2p+1][2p] X[2p]), p = 0, 1. Threads 0-127 each
-            // compute four adjacent outputs from one broadcast scalar and one float4 per step.
-            if (tid < 128) {
-                const int pp = tid >> 6, i = (tid >> 2) & 15, j4 = (tid & 3) * 4;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        }
+        sync_for_mma();
+        tma_pending = more;
+        // ---- A = (I + M_ab)^{-1}. Diagonal 16x16 blocks: one thread per (block, column)
+        //      solves (I + L_dd) x = e_c by forward substitution in registers (warps 2, 3).
+        if (tid >= 64 && tid < 128) {
+            const int d = (tid - 64) >> 4, cc = tid & 15;
+            const float *Lb = Lw + 16 * d * LWS + 16 * d;
+            float x[16];
 #pragma unroll
-                for (int kq = 0; kq < 16; ++kq) {
-                    const float lv = Lw[(32 * pp + 16 + i) * LWS + 32 * pp + kq];
-                    const float4 xv = *reinterpret_cast<const float4 *>(Aw + (32 * pp + kq) * LWS + 32 * pp + j4);
-                    acc[0] = fmaf(lv, xv.x, acc[0]); acc[1] = fmaf(lv, xv.y, acc[1]);
-                    acc[2] = fmaf(lv, xv.z, acc[2]); acc[3] = fmaf(lv, xv.w, acc[3]);
-                }
-                *reinterpret_cast<float4 *>(Tw + (pp * 16 + i) * 20 + j4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            }
-            __syncthreads();
-            if (tid < 128) {
-                const int pp = tid >> 6, i = (tid >> 2) & 15, j4 = (tid & 3) * 4;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int r = 0; r < 16; ++r) {
+                float acc = (r == cc) ? 1.f : 0.f;
 #pragma unroll
-                for (int kq = 0; kq < 16; ++kq) {
-                    const float xv = Aw[(32 * pp + 16 + i) * LWS + 32 * pp + 16 + kq];
-                    const float4 tv = *reinterpret_cast<const float4 *>(Tw + (pp * 16 + kq) * 20 + j4);
-                    acc[0] = fmaf(xv, tv.x, acc[0]); acc[1] = fmaf(xv, tv.y, acc[1]);
-                    acc[2] = fmaf(xv, tv.z, acc[2]); acc[3] = fmaf(xv, tv.w, acc[3]);
-                }
-                *reinterpret_cast<float4 *>(Aw + (32 * pp + 16 + i) * LWS + 32 * pp + j4) =
-                    make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+                for (int k = 0; k < r; ++k) acc = fmaf(-Lb[r * LWS + k], x[k], acc);
+                x[r] = acc;
             }
-            if (tid == kStoreThread) tma_store_wait_read();   // the y tile in B2 has been read
-            __syncthreads();
-            // B2 = D^T, D = blockdiag(Y0, Y1) the inverses of the two diagonal 32x32 blocks of
-            // I + M_ab (row s, K = t; entries with t < s or t, s in different halves are zero).
-            // The off-diagonal block of the inverse, -Y1 L21 Y0, is applied by R2b/R2c.
-            for (int e = tid; e < 1024; e += kThreads) {
-                const int s = e & 63, t4 = (e >> 6) * 4;
-                float a4[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int t = t4 + q;
-                    a4[q] = (t >= s && ((t ^ s) < 32)) ? to_tf32(Aw[t * LWS + s]) : 0.f;
-                }
-                st_f4(sm + OFF_B2, sw128_off(s, t4, 64), a4[0], a4[1], a4[2], a4[3]);
+            for (int r = 0; r < 16; ++r) Aw[(16 * d + r) * LWS + 16 * d + cc] = x[r];
+        }
+        __syncthreads();
+        // level 1: X[2p+1][2p] = -X[2p+1] (L[2p+1][2p] X[2p]), p = 0, 1. Threads 0-127 each
+        // compute four adjacent outputs from one broadcast scalar and one float4 per step.
+        if (tid < 128) {
+            const int pp = tid >> 6, i = (tid >> 2) & 15, j4 = (tid & 3) * 4;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kq = 0; kq < 16; ++kq) {
+                const float lv = Lw[(32 * pp + 16 + i) * LWS + 32 * pp + kq];
+                const float4 xv = *reinterpret_cast<const float4 *>(Aw + (32 * pp + kq) * LWS + 32 * pp + j4);
+                acc[0] = fmaf(lv, xv.x, acc[0]); acc[1] = fmaf(lv, xv.y, acc[1]);
+                acc[2] = fmaf(lv, xv.z, acc[2]); acc[3] = fmaf(lv, xv.w, acc[3]);
             }
-            sync_for_mma();
+            *reinterpret_cast<float4 *>(Tw + (pp * 16 + i) * 20 + j4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        }
+        __syncthreads();
+        if (tid < 128) {
+            const int pp = tid >> 6, i = (tid >> 2) & 15, j4 = (tid & 3) * 4;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kq = 0; kq < 16; ++kq) {
+                const float xv = Aw[(32 * pp + 16 + i) * LWS + 32 * pp + 16 + kq];
+                const float4 tv = *reinterpret_cast<const float4 *>(Tw + (pp * 16 + kq) * 20 + j4);
+                acc[0] = fmaf(xv, tv.x, acc[0]); acc[1] = fmaf(xv, tv.y, acc[1]);
+                acc[2] = fmaf(xv, tv.z, acc[2]); acc[3] = fmaf(xv, tv.w, acc[3]);
+            }
+            *reinterpret_cast<float4 *>(Aw + (32 * pp + 16 + i) * LWS + 32 * pp + j4) =
+                make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+        }
+        if (tid == kStoreThread) tma_store_wait_read();   // the y tile in B2 has been read
+        __syncthreads();
+        // B2 = D^T, D = blockdiag(Y0, Y1) the inverses of the two diagonal 32x32 blocks of
+        // I + M_ab (row s, K = t; entries with t < s or t, s in different halves are zero).
+        // The off-diagonal block of the inverse, -Y1 L21 Y0, is applied by R2b/R2c.
+        for (int e = tid; e < 1024; e += kThreads) {
+            const int s = e & 63, t4 = (e >> 6) * 4;
+            float a4[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int t = t4 + q;
+                a4[q] = (t >= s && ((t ^ s) < 32)) ? to_tf32(Aw[t * LWS + s]) : 0.f;
+            }
+            st_f4(sm + OFF_B2, sw128_off(s, t4, 64), a4[0], a4[1], a4[2], a4[3]);
+        }
+        sync_for_mma();
+
+        // ---- the window: warps 0-3 run this chunk's dependent MMA rounds and its output,
+        //      warps 4-15 prepare the next chunk's operands.
+        bool wfail = false;
+        if (back) {
             if (tid == 0) {
                 tc_fence_after();
 #pragma unroll
@@ -563,154 +727,85 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                     mma_tf32_ts(tb + T_D1, tb + T_A2 + 8 * ks, dB2 + kstep_off(ks, 64), idesc_tf32(128, 64), ks > 0);
                 mma_commit(&S.bar_mma);
             }
-            mma_pending = true;
-            if (wait_mma()) { failed = true; break; }
+            wfail = wait_mma_back(false);
             // Z = W A with A = D - [0 0; Y1 L21 Y0 0]: Z[:, 32:64] = U[:, 32:64] and
             // Z[:, 0:32] = U[:, 0:32] - (U[:, 32:64] L21) Y0 (block back-substitution on the tensor core)
-            if (tid == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)   // R2b: V = U[:, 32:64] L21
-                    mma_tf32_ts(tb + T_V, tb + T_D1 + 32 + 8 * ks, dL21 + kstep_off(ks, 32), idesc_tf32(128, 32), ks > 0);
-                mma_commit(&S.bar_mma);
-            }
-            mma_pending = true;
-            if (wait_mma()) { failed = true; break; }
-            if (tid == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)   // R2c: U[:, 0:32] -= V Y0 (B2 rows 0-31 hold Y0^T)
-                    mma_tf32_ts(tb + T_D1, tb + T_V + 8 * ks, dB2 + kstep_off(ks, 64), idesc_neg_a(idesc_tf32(128, 32)), 1);
-                mma_commit(&S.bar_mma);
-            }
-            mma_pending = true;
-            if (wait_mma()) { failed = true; break; }
-            if (tid == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)   // R3: [T_D3R | T_D3L] -= Z [M_kb | KKd]
-                    mma_tf32_ts(tb + T_D3R, tb + T_D1 + 8 * ks, dB3 + kstep_off(ks, 128),
-                                idesc_neg_a(idesc_tf32(128, 128)), 1);
-                mma_commit(&S.bar_mma);
-            }
-            mma_pending = true;
-            if (wait_mma()) { failed = true; break; }
-            const bool recv = cs > 1 && c > 0;   // split mode: this chunk's start state comes from CTA rank-1
-            bool state_to = false;
-            if (tid == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)   // R4: [Ki^T - X; Q~] V
-                    mma_tf32_ts(tb + T_D4, tb + T_D3R + 8 * ks, dB4 + kstep_off(ks, 64), idesc_tf32(128, 64), ks > 0);
-                if (recv) {
-                    // the only wait on another CTA: everything above used this chunk's inputs only
-                    state_to = !mbar_wait_cluster(&S.bar_state, state_parity, p.timeout_ns);
-                    fence_proxy_async_smem();
+            if (!wfail) {
+                if (tid == 0) {
                     tc_fence_after();
-                }
-                if (!state_to) {
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)   // R5: += [I - X; R~] S_0^T
-                        mma_tf32_ts(tb + T_D4, tb + T_D3L + 8 * ks, dB5 + kstep_off(ks, 64), idesc_tf32(128, 64), 1);
+                    for (int ks = 0; ks < 4; ++ks)   // R2b: V = U[:, 32:64] L21
+                        mma_tf32_ts(tb + T_V, tb + T_D1 + 32 + 8 * ks, dL21 + kstep_off(ks, 32), idesc_tf32(128, 32), ks > 0);
+                    mma_commit(&S.bar_mma);
                 }
-                mma_commit(&S.bar_mma);
+                wfail = wait_mma_back(false);
             }
-            if (recv) state_parity ^= 1u;
-            mma_pending = true;
-            if (wait_mma(state_to)) { failed = true; break; }
-            // ---- new state -> B5 (+ S_T / snapshot); readout -> epilogue -> y
-            const int done = c0 + Lc;
-            const bool snap = p.snap_every > 0 && done % p.snap_every == 0;
-            if (colg) {
-                const int j = L;
-                const float gCj = S.gC[j];
-                uint32_t xo[8];
-                kcol_offsets(j, 64, xo);
-                uint8_t *b5 = sm + OFF_B5;
-                // split mode: the state goes straight into the next CTA's B5 (distributed shared memory)
-                const bool send = cs > 1 && c + 1 < nchunks;
-                float sv[2][8];
-                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D4 + c16), sv[0]);      // S'[c16+e][j]
-                tmem_ld8_nowait(tmem_addr(tb, Lq, T_D4 + c16 + 8), sv[1]);
-                tmem_ld_wait(sv[0], sv[1]);
+            if (!wfail) {
+                if (tid == 0) {
+                    tc_fence_after();
 #pragma unroll
-                for (int g = 0; g < 2; ++g) {
-                    const int i0 = c16 + 8 * g;
-                    float (&s8)[8] = sv[g];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) s8[e] *= gCj;                // S_C = S' diag(gC)
-                    if (send) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) st_cluster(next_b5 + (i0 + e) * 128 + xo[e], to_tf32(s8[e]));
-                        if (g == 1) {
-                            fence_proxy_async_cluster();
-                            mbar_arrive_remote(next_bar);
-                        }
-                    }
-                    if (last && p.S_T) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) p.S_T[size_t(unit) * 4096 + (i0 + e) * 64 + j] = s8[e];
-                    }
-                    if (snap) {
-                        float *dst = p.snaps + ((size_t(b) * p.n_snap + (done / p.snap_every - 1)) * p.H + hh) * 4096;
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) dst[(i0 + e) * 64 + j] = s8[e];
-                    }
-                    if (cs == 1) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) *reinterpret_cast<float *>(b5 + (i0 + e) * 128 + xo[e]) = to_tf32(s8[e]);
-                    }
+                    for (int ks = 0; ks < 4; ++ks)   // R2c: U[:, 0:32] -= V Y0 (B2 rows 0-31 hold Y0^T)
+                        mma_tf32_ts(tb + T_D1, tb + T_V + 8 * ks, dB2 + kstep_off(ks, 64), idesc_neg_a(idesc_tf32(128, 32)), 1);
+                    mma_commit(&S.bar_mma);
                 }
-            } else {
-                const int t = L - 64;
-                float yv[16];
-                {
-                    float ya[8], yb[8];
-                    tmem_ld8_nowait(tmem_addr(tb, Lq, T_D4 + c16), ya);
-                    tmem_ld8_nowait(tmem_addr(tb, Lq, T_D4 + c16 + 8), yb);
-                    tmem_ld_wait(ya, yb);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        yv[e] = ya[e];
-                        yv[8 + e] = yb[e];
-                    }
-                }
-                if (epi) {
-                    uint32_t xo[8];
-                    kcol_offsets(t, 64, xo);
-                    float s1 = 0.f, s2 = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) s1 += yv[e];
-                    S.red[pq][t] = s1;
-                    named_bar_rows();
-                    const float mean = (S.red[0][t] + S.red[1][t] + S.red[2][t] + S.red[3][t]) * (1.f / 64.f);
-                    named_bar_rows();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) s2 = fmaf(yv[e] - mean, yv[e] - mean, s2);
-                    S.red[pq][t] = s2;
-                    named_bar_rows();
-                    const float inv =
-                        1.f / sqrtf((S.red[0][t] + S.red[1][t] + S.red[2][t] + S.red[3][t]) * (1.f / 64.f) + p.gn_eps);
-                    const float bon = S.bon[0][t] + S.bon[1][t] + S.bon[2][t] + S.bon[3][t];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int ii = c16 + e;
-                        const float v = *reinterpret_cast<const float *>(sm + OFF_B4 + ii * 128 + xo[e & 7]);
-                        yv[e] = fmaf((yv[e] - mean) * inv, S.ln_w[ii], S.ln_b[ii]) + bon * v;
-                    }
-                }
-                // y row t, channels c16..c16+15 -> the swizzled [64][32] fp32 tile of its channel half
-                // (the layout the y tensor map expects); rows past the end of T are clipped by the store
-                uint8_t *ytile = sm + OFF_B2 + (c16 >> 5) * 8192 + t * 128;
-#pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    *reinterpret_cast<float4 *>(ytile + (((((c16 & 31) >> 2) + m) ^ (t & 7)) << 4)) =
-                        make_float4(yv[4 * m], yv[4 * m + 1], yv[4 * m + 2], yv[4 * m + 3]);
+                wfail = wait_mma_back(false);
             }
-            sync_for_mma();
-            y_pending = true;
-            y_h = hh; y_c0 = c0; y_b = b;
+            if (!wfail) {
+                if (tid == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)   // R3: [T_D3R | T_D3L] -= Z [M_kb | KKd]
+                        mma_tf32_ts(tb + T_D3R, tb + T_D1 + 8 * ks, dB3 + kstep_off(ks, 128),
+                                    idesc_neg_a(idesc_tf32(128, 128)), 1);
+                    mma_commit(&S.bar_mma);
+                }
+                wfail = wait_mma_back(false);
+            }
+            if (!wfail) {
+                bool state_to = false;
+                if (tid == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)   // R4: [Ki^T - X; Q~] V
+                        mma_tf32_ts(tb + T_D4, tb + T_D3R + 8 * ks, dB4 + kstep_off(ks, 64), idesc_tf32(128, 64), ks > 0);
+                    if (recv) {
+                        // the only wait on another CTA: everything above used this chunk's inputs only
+                        state_to = !mbar_wait_cluster(&S.bar_state, state_parity, p.timeout_ns);
+                        fence_proxy_async_smem();
+                        tc_fence_after();
+                    }
+                    if (!state_to) {
+#pragma unroll
+                        for (int ks = 0; ks < 8; ++ks)   // R5: += [I - X; R~] S_0^T
+                            mma_tf32_ts(tb + T_D4, tb + T_D3L + 8 * ks, dB5 + kstep_off(ks, 64), idesc_tf32(128, 64), 1);
+                    }
+                    mma_commit(&S.bar_mma);
+                }
+                if (recv) state_parity ^= 1u;
+                wfail = wait_mma_back(state_to);
+                // split mode: this CTA's B5 is consumed; the previous CTA may send the next state
+                if (!wfail && recv && tid == 0) mbar_arrive_remote(prev_credit);
+            }
+            if (!wfail) wfail = out(u, c, ip, us);
+        } else if (more) {
+            if (new_unit && ft < 64) load_params(nu, us ^ 1, ft);
+            wfail = front(nu, nc, ip ^ 1, new_unit ? (us ^ 1) : us);
         }
+        tc_fence_before();
+        if (__syncthreads_or(wfail)) { failed = true; break; }
+        tc_fence_after();
+        // keep the barrier parities uniform: warps 0-3 completed five MMA rounds, warps 4-15
+        // consumed the next chunk's tiles
+        if (!back) mma_parity ^= 1u;
+        if (back && more) tma_parity ^= 1u;
+        tma_pending = false;
+        mma_pending = false;
+        y_pending = true;
+        y_h = hh; y_c0 = c0; y_b = b;
+        if (new_unit && rank == 0) load_state(nu);   // R5 of the previous head has read B5
+        u = nu; c = nc; valid = more;
+        ip ^= 1;
+        if (new_unit) us ^= 1;
     }
     if (tid == kStoreThread) {
         if (y_pending && !failed) store_y_tile(maps, sm + OFF_B2, y_h, y_c0, y_b);
