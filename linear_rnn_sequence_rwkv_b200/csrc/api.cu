@@ -101,7 +101,8 @@ bool mul_ok(size_t &acc, long long f) {
 }  // namespace
 
 // Sizes and options, shared by wkv7_forward and wkv7_plan; fills `opts` (defaults if NULL).
-wkv7_status check_args(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opts *opts_in, wkv7_opts &opts) {
+wkv7_status check_args(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opts *opts_in, wkv7_opts &opts,
+                       bool need_buffers = true) {
     if (N <= 0 || B <= 0 || H <= 0 || T < 0)
         return fail(WKV7_ERR_ARG, "bad sizes B=%d T=%d H=%d N=%d (need B,H,N >= 1, T >= 0)", B, T, H, N);
     if (N != wkv7::kN) return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: only N=64 is implemented", N);
@@ -113,7 +114,7 @@ wkv7_status check_args(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opt
     if (!(opts.chunk == 0 || opts.chunk == 16 || opts.chunk == 32 || opts.chunk == 64))
         return fail(WKV7_ERR_ARG, "chunk=%d: must be 0 (default), 16, 32 or 64", opts.chunk);
     if (opts.snap_every < 0) return fail(WKV7_ERR_ARG, "snap_every=%d < 0", opts.snap_every);
-    if (opts.snap_every > 0 && !opts.snapshots && T >= opts.snap_every)
+    if (need_buffers && opts.snap_every > 0 && !opts.snapshots && T >= opts.snap_every)
         return fail(WKV7_ERR_ARG, "snap_every=%d but snapshots is NULL", opts.snap_every);
     const int n_epi = (opts.ln_w != nullptr) + (opts.ln_b != nullptr) + (opts.r_k != nullptr);
     if (n_epi != 0 && n_epi != 3) return fail(WKV7_ERR_ARG, "epilogue needs all of ln_w, ln_b, r_k (or none)");
@@ -276,7 +277,7 @@ wkv7_status wkv7_plan(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opts
     g_err[0] = '\0';
     if (!algo || !segments) return fail(WKV7_ERR_ARG, "algo and segments must not be NULL");
     wkv7_opts opts;
-    const wkv7_status vs = check_args(B, T, H, N, dt, opts_in, opts);
+    const wkv7_status vs = check_args(B, T, H, N, dt, opts_in, opts, false);   // no buffers needed
     if (vs != WKV7_OK) return vs;
     wkv7::FwdArgs p{};
     p.B = B; p.T = T; p.H = H; p.dt = dt;

@@ -58,11 +58,11 @@ constexpr int C = 64;             // chunk length (tokens)
 constexpr int kThreads = 512;     // 16 warps
 constexpr int kBackThreads = 128; // warps 0-3: MMA rounds after the inverse, and the output
 constexpr int kFrontThreads = kThreads - kBackThreads;   // warps 4-15: the next chunk's operands
-constexpr int kSendThreads = 64;  // split mode: warps 0-1 write the next CTA's state operand
+constexpr int kSendThreads = 256; // split mode: the 8 warps of TMEM lanes 0-63 write the next CTA's state
 constexpr int kMaxSegments = WKV7_MAX_SEGMENTS;   // CTAs per (b, h) in split mode (portable cluster size)
 constexpr int GTS = 68;           // row stride (floats) of the decay table
 constexpr int LWS = 68;           // row stride of the inverse workspaces (16-byte aligned rows)
-constexpr int BAR_BACK = 1, BAR_FRONT = 2, BAR_SEND = 3;   // named barriers: warps 0-3, 4-15, 0-1
+constexpr int BAR_BACK = 1, BAR_FRONT = 2, BAR_ROWS = 3;   // named barriers: warps 0-3, 4-15, TMEM lanes 64-127
 
 // Shared-memory layout (byte offsets from a 1024-byte aligned base).
 constexpr uint32_t OFF_B1 = 0;        // [Bi; Ki] 128x64 tf32 (B of R1 and of the transpose round); then the
@@ -82,6 +82,7 @@ struct Small {
     float gC[2][C];           // decay over the chunk per key channel, by chunk parity
     float tq[4][C];           // decay product over each quarter of the chunk
     float bon[2][C];          // epilogue bonus r_t . (k_t * r_k) per token, by chunk parity
+    float red[4][C];          // epilogue: partial sums over the four column parts of each y row
     float dk[C];              // r_t . k_t (exact current-token Gram entry)
     float db[C];              // r_t . (kk_t * a_t)
     float ln_w[2][C], ln_b[2][C], r_k[2][C];   // epilogue parameters, by head parity
@@ -394,114 +395,89 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         return false;
     };
 
-    // ---- back, second half: the state and y of chunk c of head u (warps 0-3), from T_D4.
-    //      Returns true on a failed wait (uniform over warps 0-3).
-    auto out = [&](int u, int c, int ip, int us) -> bool {
-        const int b = u / p.H, hh = u % p.H, c0 = c * C, done = c0 + min(C, p.T - c0);
-        const bool last = c == nchunks - 1;
-        const bool snap = p.snap_every > 0 && done % p.snap_every == 0;
-        bool fail = false;
-        if (warp < 2) {   // TMEM lane j = key channel: S'[i][j] for all value channels i
+    // ---- output of chunk c of head u from T_D4, by all warps (each owns 16 columns of its lane
+    //      quarter). Lanes 0-63 (key channel j): the new state diag(gC) S'^T -> B5, or the next CTA's
+    //      B5 in split mode, and at the end of the sequence or of a snapshot interval fp32 to S_T /
+    //      the snapshot. Lanes 64-127 (token t): y -> epilogue -> the swizzled y tile in B2.
+    auto out = [&](int u, int c, int ip, int us, bool send) {
+        const int b = u / p.H, hh = u % p.H, done = c * C + min(C, p.T - c * C);
+        float v[2][8];
+        tmem_ld8_nowait(tmem_addr(tb, Lq, T_D4 + c16), v[0]);
+        tmem_ld8_nowait(tmem_addr(tb, Lq, T_D4 + c16 + 8), v[1]);
+        tmem_ld_wait(v[0], v[1]);
+        if (colg) {
             const int j = L;
             const float gCj = S.gC[ip][j];
             uint32_t xo[8];
             kcol_offsets(j, 64, xo);
-            // split mode: the state goes straight into the next CTA's B5 (distributed shared memory),
-            // once that CTA has consumed the state sent before (its credit)
-            const bool send = cs > 1 && c + 1 < nchunks;
-            if (send && sends > 0) {
-                const bool to = tid == 0 && !mbar_wait_cluster(&S.bar_credit, credit_parity, p.timeout_ns);
-                credit_parity ^= 1u;
-                fail = bar_named_or(BAR_SEND, kSendThreads, to);
-            }
-            const bool write_b5 = cs == 1 || (send && !fail);
             const uint32_t b5_dst = cs == 1 ? own_b5 : next_b5;
-            float *gdst = nullptr;    // S_T or a snapshot, if this chunk ends one
-            if (last && p.S_T) gdst = p.S_T + size_t(u) * 4096;
-            else if (snap) gdst = p.snaps + ((size_t(b) * p.n_snap + (done / p.snap_every - 1)) * p.H + hh) * 4096;
-            float *sdst = (snap && last && p.S_T)   // the last chunk can also end a snapshot
+            const bool write_b5 = cs == 1 || send;
+#pragma unroll
+            for (int g = 0; g < 2; ++g)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    v[g][e] *= gCj;                                             // S_C = S' diag(gC)
+                    if (write_b5) st_cluster(b5_dst + (c16 + 8 * g + e) * 128 + xo[e], to_tf32(v[g][e]));
+                }
+            if (send) {
+                fence_proxy_async_cluster();
+                mbar_arrive_remote(next_bar);
+            }
+            float *gdst = (c == nchunks - 1 && p.S_T) ? p.S_T + size_t(u) * 4096 : nullptr;
+            float *sdst = (p.snap_every > 0 && done % p.snap_every == 0)
                               ? p.snaps + ((size_t(b) * p.n_snap + (done / p.snap_every - 1)) * p.H + hh) * 4096
                               : nullptr;
-            if (write_b5) {
-#pragma unroll 1
-                for (int h2 = 0; h2 < 64; h2 += 32) {
-                    float v[4][8];
+            if (gdst || sdst) {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) tmem_ld8_nowait(tmem_addr(tb, Lq, T_D4 + h2 + 8 * q), v[q]);
-                    tmem_ld_wait(v[0], v[1], v[2], v[3]);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)   // S_C = S' diag(gC), this CTA's B5 or the next CTA's
-                            st_cluster(b5_dst + (h2 + 8 * q + e) * 128 + xo[e], to_tf32(v[q][e] * gCj));
-                }
-            }
-            if (gdst || sdst) {   // the end of the sequence or of a snapshot interval: fp32 state out
-#pragma unroll 1
-                for (int i0 = 0; i0 < 64; i0 += 8) {
-                    float v[8];
-                    tmem_ld8(tmem_addr(tb, Lq, T_D4 + i0), v);
+                for (int g = 0; g < 2; ++g)
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        if (gdst) gdst[(i0 + e) * 64 + j] = v[e] * gCj;
-                        if (sdst) sdst[(i0 + e) * 64 + j] = v[e] * gCj;
+                        const int i = c16 + 8 * g + e;
+                        if (gdst) gdst[i * 64 + j] = v[g][e];
+                        if (sdst) sdst[i * 64 + j] = v[g][e];
                     }
-                }
             }
-            if (send) {
-                if (!fail) {
-                    fence_proxy_async_cluster();
-                    mbar_arrive_remote(next_bar);
-                }
-                ++sends;
-            }
-        } else {          // TMEM lane 64 + t: y row t
+        } else {
             const int t = L - 64;
-            const uint32_t yrow = tmem_addr(tb, Lq, T_D4);
-            float mean = 0.f, inv = 0.f, bon = 0.f;
-            uint32_t xv[8];
-            if (epi) {   // group_norm statistics over the head's 64 channels (two passes over TMEM)
+            if (epi) {   // group_norm over the head's 64 channels, then the bonus (r.(k*r_k)) v
                 float s1 = 0.f, s2 = 0.f;
-#pragma unroll 1
-                for (int i0 = 0; i0 < 64; i0 += 8) {
-                    float v[8];
-                    tmem_ld8(yrow + i0, v);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) s1 += v[e];
-                }
-                mean = s1 * (1.f / 64.f);
-#pragma unroll 1
-                for (int i0 = 0; i0 < 64; i0 += 8) {
-                    float v[8];
-                    tmem_ld8(yrow + i0, v);
+                for (int e = 0; e < 8; ++e) s1 += v[0][e] + v[1][e];
+                S.red[pq][t] = s1;
+                bar_named(BAR_ROWS, 256);
+                const float mean = (S.red[0][t] + S.red[1][t] + S.red[2][t] + S.red[3][t]) * (1.f / 64.f);
+                bar_named(BAR_ROWS, 256);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) s2 = fmaf(v[e] - mean, v[e] - mean, s2);
+                for (int e = 0; e < 8; ++e) {
+                    s2 = fmaf(v[0][e] - mean, v[0][e] - mean, s2);
+                    s2 = fmaf(v[1][e] - mean, v[1][e] - mean, s2);
                 }
-                inv = 1.f / sqrtf(s2 * (1.f / 64.f) + p.gn_eps);
-                bon = S.bon[ip][t];
+                S.red[pq][t] = s2;
+                bar_named(BAR_ROWS, 256);
+                const float inv =
+                    1.f / sqrtf((S.red[0][t] + S.red[1][t] + S.red[2][t] + S.red[3][t]) * (1.f / 64.f) + p.gn_eps);
+                const float bon = S.bon[ip][t];
+                uint32_t xv[8];
                 kcol_offsets(t, 64, xv);
-            }
-            // y row t -> the swizzled [64][32] fp32 tiles (one per channel half) the y tensor map
-            // expects; rows past the end of T are clipped by the store
-#pragma unroll 1
-            for (int i0 = 0; i0 < 64; i0 += 8) {
-                float v[8];
-                tmem_ld8(yrow + i0, v);
-                if (epi) {   // (y - mean) / sqrt(var + eps) * ln_w + ln_b + (r.(k*r_k)) v
+#pragma unroll
+                for (int g = 0; g < 2; ++g)
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const int i = i0 + e;
+                        const int i = c16 + 8 * g + e;
                         const float vi = *reinterpret_cast<const float *>(sm + OFF_B4 + i * 128 + xv[e]);
-                        v[e] = fmaf((v[e] - mean) * inv, S.ln_w[us][i], S.ln_b[us][i]) + bon * vi;
+                        v[g][e] = fmaf((v[g][e] - mean) * inv, S.ln_w[us][i], S.ln_b[us][i]) + bon * vi;
                     }
-                }
-                uint8_t *row = sm + OFF_B2 + (i0 >> 5) * 8192 + t * 128;
-                const int q = (i0 & 31) >> 2;
-                *reinterpret_cast<float4 *>(row + ((q ^ (t & 7)) << 4)) = make_float4(v[0], v[1], v[2], v[3]);
-                *reinterpret_cast<float4 *>(row + (((q + 1) ^ (t & 7)) << 4)) = make_float4(v[4], v[5], v[6], v[7]);
             }
+            // y row t, channels c16..c16+15 -> the swizzled [64][32] fp32 tile of its channel half
+            // (the layout the y tensor map expects); rows past the end of T are clipped by the store
+            uint8_t *row = sm + OFF_B2 + (c16 >> 5) * 8192 + t * 128;
+            const int q0 = (c16 & 31) >> 2;
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                *reinterpret_cast<float4 *>(row + (((q0 + m) ^ (t & 7)) << 4)) =
+                    make_float4(v[m >> 1][4 * (m & 1)], v[m >> 1][4 * (m & 1) + 1], v[m >> 1][4 * (m & 1) + 2],
+                                v[m >> 1][4 * (m & 1) + 3]);
         }
-        return bar_named_or(BAR_BACK, kBackThreads, fail);
     };
 
     // ---- the CTA's chunks: (head u, chunk c), c = rank, rank + cs, ... of heads cid, cid + ncl, ...
@@ -786,13 +762,23 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 // split mode: this CTA's B5 is consumed; the previous CTA may send the next state
                 if (!wfail && recv && tid == 0) mbar_arrive_remote(prev_credit);
             }
-            if (!wfail) wfail = out(u, c, ip, us);
         } else if (more) {
             if (new_unit && ft < 64) load_params(nu, us ^ 1, ft);
             wfail = front(nu, nc, ip ^ 1, new_unit ? (us ^ 1) : us);
         }
+        // split mode: before writing the next CTA's B5, its credit for the state sent before
+        const bool send = cs > 1 && c + 1 < nchunks;
+        if (send && sends > 0) {
+            if (tid == 0 && !wfail) wfail = !mbar_wait_cluster(&S.bar_credit, credit_parity, p.timeout_ns);
+            credit_parity ^= 1u;
+        }
         tc_fence_before();
         if (__syncthreads_or(wfail)) { failed = true; break; }
+        tc_fence_after();
+        out(u, c, ip, us, send);
+        if (send) ++sends;
+        tc_fence_before();
+        __syncthreads();
         tc_fence_after();
         // keep the barrier parities uniform: warps 0-3 completed five MMA rounds, warps 4-15
         // consumed the next chunk's tiles
@@ -898,7 +884,8 @@ cudaError_t device_info(DeviceInfo *&out) {
 // CTAs per (b, h). Each CTA of a cluster runs every cs-th chunk, so a head takes about
 // ceil(nchunks / cs) chunk times plus the hand-off latency, and the heads run in
 // ceil(units / clusters) waves. Pick the size with the smallest estimate (ties: fewer CTAs);
-// the 8% and 0.15-chunk terms are the measured cost of the hand-off per chunk and per head.
+// the 15.5% and 0.35-chunk terms are the measured cost of the hand-off per chunk and per head
+// (B8 T1024 H12 and B16 T4096 H32 timed with 1-4 CTAs per head).
 int choose_segments(int units, int nchunks, const DeviceInfo &d) {
     int best = 1;
     double best_cost = 1e300;
@@ -906,7 +893,7 @@ int choose_segments(int units, int nchunks, const DeviceInfo &d) {
         if (d.clusters[cs] <= 0) continue;
         const double waves = double((units + d.clusters[cs] - 1) / d.clusters[cs]);
         const double per = double((nchunks + cs - 1) / cs);
-        const double cost = waves * (per * (cs > 1 ? 1.08 : 1.0) + 0.15 * (cs - 1));
+        const double cost = waves * (per * (cs > 1 ? 1.155 : 1.0) + 0.35 * (cs - 1));
         if (cost < best_cost - 1e-9) {
             best_cost = cost;
             best = cs;

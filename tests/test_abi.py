@@ -134,3 +134,16 @@ def test_plan_without_device(lib):
         with pytest.raises(wkv7.Wkv7Error) as e:
             wkv7.plan(2, 128, 4)
         assert e.value.status == wkv7.ERR_CUDA
+
+
+def test_plan_with_snapshot_interval_needs_no_buffer(lib):
+    """The dispatch query takes snap_every without a snapshots buffer (it runs nothing)."""
+    import torch
+    assert wkv7.plan(1, 8, 2, snap_every=4) == ("seq", 0)                 # off chunk boundaries -> scan
+    with pytest.raises(wkv7.Wkv7Error) as e:
+        wkv7.plan(1, 128, 2, algo="chunk", snap_every=10)                  # chunked path cannot take it
+    assert e.value.status == wkv7.ERR_UNSUPPORTED
+    if not torch.cuda.is_available():
+        with pytest.raises(wkv7.Wkv7Error) as e:
+            wkv7.plan(1, 8192, 2, snap_every=4096)                         # chunked: needs the device
+        assert e.value.status == wkv7.ERR_CUDA
