@@ -628,6 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 tmem_st8(tmem_addr(tb, Lq, T_D3R + s0), qk[g]);
             }
         }
+        if (tid == kStoreThread) tma_store_wait_read();   // the y tile in B2 has been read
         sync_for_mma();
         tma_pending = more;
         // ---- A = (I + M_ab)^{-1}. Diagonal 16x16 blocks: one thread per (block, column)
@@ -645,6 +646,21 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
             }
 #pragma unroll
             for (int r = 0; r < 16; ++r) Aw[(16 * d + r) * LWS + 16 * d + cc] = x[r];
+            // column cc of the block is row 16d + cc of B2 = D^T (K = t), tf32
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                st_f4(sm + OFF_B2, sw128_off(16 * d + cc, 16 * d + 4 * m, 64), to_tf32(x[4 * m]), to_tf32(x[4 * m + 1]),
+                      to_tf32(x[4 * m + 2]), to_tf32(x[4 * m + 3]));
+        } else {
+            // B2 = D^T, D = blockdiag(Y0, Y1): zero where t and s lie in different 32-halves or
+            // t's 16-block precedes s's (the diagonal blocks and the level-1 blocks are written by
+            // their producers)
+            const int z = tid < 64 ? tid : tid - 64;
+#pragma unroll 1
+            for (int e = z; e < 1024; e += kThreads - 64) {
+                const int sr = e & 63, t4 = (e >> 6) * 4;
+                if (((t4 ^ sr) >= 32) || ((t4 >> 4) < (sr >> 4))) st_f4(sm + OFF_B2, sw128_off(sr, t4, 64), 0.f, 0.f, 0.f, 0.f);
+            }
         }
         __syncthreads();
         // level 1: X[2p+1][2p] = -X[2p+1] (L[2p+1][2p] X[2p]), p = 0, 1. Threads 0-127 each
@@ -672,24 +688,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 acc[0] = fmaf(xv, tv.x, acc[0]); acc[1] = fmaf(xv, tv.y, acc[1]);
                 acc[2] = fmaf(xv, tv.z, acc[2]); acc[3] = fmaf(xv, tv.w, acc[3]);
             }
-            *reinterpret_cast<float4 *>(Aw + (32 * pp + 16 + i) * LWS + 32 * pp + j4) =
-                make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
-        }
-        if (tid == kStoreThread) tma_store_wait_read();   // the y tile in B2 has been read
-        __syncthreads();
-        // B2 = D^T, D = blockdiag(Y0, Y1) the inverses of the two diagonal 32x32 blocks of
-        // I + M_ab (row s, K = t; entries with t < s or t, s in different halves are zero).
-        // The off-diagonal block of the inverse, -Y1 L21 Y0, is applied by R2b/R2c.
-        for (int e = tid; e < 1024; e += kThreads) {
-            const int s = e & 63, t4 = (e >> 6) * 4;
-            float a4[4];
+            // the block X[2p+1][2p] of D goes transposed into B2 (row s = column of D, K = t), tf32
+            const int t = 32 * pp + 16 + i;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int t = t4 + q;
-                a4[q] = (t >= s && ((t ^ s) < 32)) ? to_tf32(Aw[t * LWS + s]) : 0.f;
-            }
-            st_f4(sm + OFF_B2, sw128_off(s, t4, 64), a4[0], a4[1], a4[2], a4[3]);
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<float *>(sm + OFF_B2 + sw128_off(32 * pp + j4 + q, t, 64)) = to_tf32(-acc[q]);
         }
+        // B2 now holds D^T, D = blockdiag(Y0, Y1) the inverses of the two diagonal 32x32 blocks of
+        // I + M_ab; the off-diagonal block of the inverse, -Y1 L21 Y0, is applied by R2b/R2c.
         sync_for_mma();
 
         // ---- the window: warps 0-3 run this chunk's dependent MMA rounds and its output,
