@@ -151,7 +151,9 @@ WKV7_API wkv7_status wkv7_poll_device_error(void *stream);
  * The path wkv7_forward takes for these arguments on the current device, without running
  * anything: *algo = WKV7_ALGO_SEQ or WKV7_ALGO_CHUNK, and *segments = CTAs per (b, h) of the
  * chunked path (1: one CTA per head; 2..WKV7_MAX_SEGMENTS: the chunks of a head spread over a
- * thread-block cluster) or 0 for the scan. Reads the current device's SM count and cluster
+ * thread-block cluster) or 0 for the scan. When the heads fill whole waves of the GPU and part
+ * of another, AUTO may run the whole waves with one CTA per head and the rest in a second
+ * launch with more; *segments then reports the second launch. Reads the current device's SM count and cluster
  * occupancy (WKV7_ERR_CUDA without a usable device); argument errors as in wkv7_forward.
  * T = 0 (state copy only) and the scan report SEQ and 0 without touching the device.
  * This query has no counterpart on the pages; it reports the dispatch of this library.

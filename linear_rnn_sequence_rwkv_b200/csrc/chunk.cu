@@ -123,6 +123,7 @@ __device__ __forceinline__ void store_y_tile(const ChunkMaps &maps, const uint8_
 
 struct ChunkArgs {
     int B, T, H;
+    int unit0, unit_end;      // the heads (b * H + h) of this launch: [unit0, unit_end)
     const float *S0;
     float *S_T, *snaps;
     int snap_every, n_snap;
@@ -194,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     const bool colg = L < 64;
     const bool back = warp < 4;             // warps 0-3: one per TMEM lane quarter
     const int ft = tid - kBackThreads;      // index among the front warps 4-15
-    const int units = p.B * p.H;
+    const int units = p.unit_end;
     const int nchunks = (p.T + C - 1) / C;
     const bool epi = p.ln_w != nullptr;
 
@@ -481,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     };
 
     // ---- the CTA's chunks: (head u, chunk c), c = rank, rank + cs, ... of heads cid, cid + ncl, ...
-    int u = cid, c = rank;
+    int u = p.unit0 + cid, c = rank;
     bool valid = u < units && rank < nchunks;
     int ip = 0, us = 0;                // parity slots of the current chunk and head
     if (valid) {
@@ -892,20 +893,57 @@ cudaError_t device_info(DeviceInfo *&out) {
 // ceil(units / clusters) waves. Pick the size with the smallest estimate (ties: fewer CTAs);
 // the 15.5% and 0.35-chunk terms are the measured cost of the hand-off per chunk and per head
 // (B8 T1024 H12 and B16 T4096 H32 timed with 1-4 CTAs per head).
-int choose_segments(int units, int nchunks, const DeviceInfo &d) {
+double launch_cost(int units, int nchunks, int cs, const DeviceInfo &d) {
+    const double waves = double((units + d.clusters[cs] - 1) / d.clusters[cs]);
+    const double per = double((nchunks + cs - 1) / cs);
+    return waves * (per * (cs > 1 ? 1.155 : 1.0) + 0.35 * (cs - 1));
+}
+int choose_segments(int units, int nchunks, const DeviceInfo &d, double *cost_out = nullptr) {
     int best = 1;
     double best_cost = 1e300;
     for (int cs = 1; cs <= kMaxSegments; ++cs) {
         if (d.clusters[cs] <= 0) continue;
-        const double waves = double((units + d.clusters[cs] - 1) / d.clusters[cs]);
-        const double per = double((nchunks + cs - 1) / cs);
-        const double cost = waves * (per * (cs > 1 ? 1.155 : 1.0) + 0.35 * (cs - 1));
+        const double cost = launch_cost(units, nchunks, cs, d);
         if (cost < best_cost - 1e-9) {
             best_cost = cost;
             best = cs;
         }
     }
+    if (cost_out) *cost_out = best_cost;
     return best;
+}
+
+// The launches of one forward call: the heads that fill whole waves of one CTA per head, then
+// the rest with the CTAs per head that suit them (a partial last wave would otherwise leave
+// SMs idle), when that is cheaper than one launch; the second launch costs about half a chunk.
+struct ChunkPlan {
+    int n = 1;
+    int units[2] = {0, 0};   // heads per launch
+    int cs[2] = {1, 1};
+};
+ChunkPlan plan_launches(const FwdArgs &p, const DeviceInfo &d) {
+    const int units = p.B * p.H, nchunks = (p.T + C - 1) / C;
+    ChunkPlan pl;
+    pl.units[0] = units;
+    if (p.segments > 0) {
+        pl.cs[0] = p.segments;
+        return pl;
+    }
+    double one = 0.0, tail_cost = 0.0;
+    pl.cs[0] = choose_segments(units, nchunks, d, &one);
+    const int full = (units / d.clusters[1]) * d.clusters[1];
+    if (full > 0 && full < units) {
+        const int tail_cs = choose_segments(units - full, nchunks, d, &tail_cost);
+        const double two = double(full / d.clusters[1]) * nchunks + tail_cost + 0.5;
+        if (tail_cs > 1 && two < one - 1e-9) {
+            pl.n = 2;
+            pl.units[0] = full;
+            pl.cs[0] = 1;
+            pl.units[1] = units - full;
+            pl.cs[1] = tail_cs;
+        }
+    }
+    return pl;
 }
 
 }  // namespace
@@ -914,9 +952,10 @@ cudaError_t chunk_segments(const FwdArgs &p, int *segments) {
     DeviceInfo *di = nullptr;
     const cudaError_t e = device_info(di);
     if (e != cudaSuccess) return e;
-    const int cs = p.segments > 0 ? p.segments : choose_segments(p.B * p.H, (p.T + C - 1) / C, *di);
-    if (cs > kMaxSegments || di->clusters[cs] <= 0) return cudaErrorInvalidClusterSize;
-    *segments = cs;
+    const ChunkPlan pl = plan_launches(p, *di);
+    for (int i = 0; i < pl.n; ++i)
+        if (pl.cs[i] > kMaxSegments || di->clusters[pl.cs[i]] <= 0) return cudaErrorInvalidClusterSize;
+    *segments = pl.cs[pl.n - 1];   // the CTAs per head of the last launch (the first is 1 when there are two)
     return cudaSuccess;
 }
 
@@ -959,13 +998,19 @@ cudaError_t launch_chunk(const FwdArgs &p) {
     a.ln_w = p.ln_w; a.ln_b = p.ln_b; a.r_k = p.r_k; a.gn_eps = p.gn_eps;
     a.err = di->err;
     a.timeout_ns = 2000000000ull;
-    const int units = p.B * p.H;
     int cs = 1;
     if ((e = chunk_segments(p, &cs)) != cudaSuccess) return e;
-    const int ncl = units < di->clusters[cs] ? units : di->clusters[cs];
-    cudaLaunchAttribute attr;
-    const cudaLaunchConfig_t cfg = launch_config(ncl * cs, cs, p.stream, &attr);
-    return cudaLaunchKernelEx(&cfg, chunk_kernel, maps, a);
+    const ChunkPlan pl = plan_launches(p, *di);
+    a.unit0 = 0;
+    for (int i = 0; i < pl.n; ++i) {
+        a.unit_end = a.unit0 + pl.units[i];
+        const int ncl = pl.units[i] < di->clusters[pl.cs[i]] ? pl.units[i] : di->clusters[pl.cs[i]];
+        cudaLaunchAttribute attr;
+        const cudaLaunchConfig_t cfg = launch_config(ncl * pl.cs[i], pl.cs[i], p.stream, &attr);
+        if ((e = cudaLaunchKernelEx(&cfg, chunk_kernel, maps, a)) != cudaSuccess) return e;
+        a.unit0 = a.unit_end;
+    }
+    return cudaSuccess;
 }
 
 cudaError_t read_device_error(cudaStream_t stream, unsigned int *value, bool clear) {

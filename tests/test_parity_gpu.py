@@ -363,3 +363,16 @@ def test_plan_matches_dispatch(cuda_device):
     assert algo == "chunk" and 2 <= seg <= 8
     algo, seg = wkv7.plan(8, 1024, 12)
     assert algo == "chunk" and 1 <= seg <= 8
+
+
+def test_partial_wave_tail_launch(cuda_device):
+    """320 heads of 6 chunks: two whole waves run with one CTA per head, the 24 heads left over
+    run in a second launch with several CTAs per head. Bit-identical to one CTA per head, and
+    the plan reports the second launch's CTAs per head."""
+    d = _dev(inputs.make_inputs(inputs.WORKLOADS[1], B=8, T=64 * 5 + 3, H=40, seed=32), cuda_device)
+    algo, seg = wkv7.plan(8, 64 * 5 + 3, 40)
+    assert algo == "chunk" and seg >= 1
+    y1, S1, _ = _gpu(d, algo="chunk")
+    ya, Sa, _ = _gpu(d)
+    assert torch.equal(ya, y1) and torch.equal(Sa, S1)
+    wkv7.poll_device_error()
