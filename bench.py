@@ -250,8 +250,11 @@ def run_gpu(args, world, rank, local):
         launches_per_step = 1 + (1 if epilogue and _path_name(args) == "seq" else 0)
 
     units_per_step = B * T * H
-    ctas_per_head = None if decode else wkv7.plan(B, T, H, N, torch.bfloat16, algo=args.algo, chunk=args.chunk,
-                                                  snap_every=snap_every)[1]
+    ctas_per_head = None
+    if not decode:
+        ep = dict(ln_w=sets[0]["ln_w"], ln_b=sets[0]["ln_b"], r_k=sets[0]["r_k"]) if epilogue else {}
+        _, ctas_per_head, launches_per_step = wkv7.plan(B, T, H, N, torch.bfloat16, launches=True, algo=args.algo,
+                                                        chunk=args.chunk, snap_every=snap_every, **ep)
 
     for i in range(warmup):
         step(i)

@@ -52,7 +52,7 @@ extern "C" {
 #define WKV7_API
 #endif
 
-#define WKV7_ABI_VERSION 1
+#define WKV7_ABI_VERSION 2
 #define WKV7_HEAD_SIZE 64
 #define WKV7_MAX_SEGMENTS 8   /* CTAs per (b, h) of WKV7_ALGO_SPLIT (one thread-block cluster) */
 
@@ -151,15 +151,16 @@ WKV7_API wkv7_status wkv7_poll_device_error(void *stream);
  * The path wkv7_forward takes for these arguments on the current device, without running
  * anything: *algo = WKV7_ALGO_SEQ or WKV7_ALGO_CHUNK, and *segments = CTAs per (b, h) of the
  * chunked path (1: one CTA per head; 2..WKV7_MAX_SEGMENTS: the chunks of a head spread over a
- * thread-block cluster) or 0 for the scan. When the heads fill whole waves of the GPU and part
- * of another, AUTO may run the whole waves with one CTA per head and the rest in a second
- * launch with more; *segments then reports the second launch. Reads the current device's SM count and cluster
+ * thread-block cluster) or 0 for the scan; *launches = kernel launches of the call (1 or 2;
+ * 0 for T = 0 without a state copy). When the heads fill whole waves of the GPU and part of
+ * another, AUTO may run the whole waves with one CTA per head and the rest in a second launch
+ * with more; *segments then reports the second launch. Reads the current device's SM count and cluster
  * occupancy (WKV7_ERR_CUDA without a usable device); argument errors as in wkv7_forward.
  * T = 0 (state copy only) and the scan report SEQ and 0 without touching the device.
  * This query has no counterpart on the pages; it reports the dispatch of this library.
  */
 WKV7_API wkv7_status wkv7_plan(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opts *opts,
-                               int *algo, int *segments);
+                               int *algo, int *segments, int *launches);
 
 /* Bytes of device workspace wkv7_forward needs for these arguments (opts may be NULL). */
 WKV7_API size_t wkv7_workspace_bytes(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opts *opts);

@@ -273,9 +273,9 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype dt, const void *
 }
 
 wkv7_status wkv7_plan(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opts *opts_in, int *algo,
-                      int *segments) {
+                      int *segments, int *launches) {
     g_err[0] = '\0';
-    if (!algo || !segments) return fail(WKV7_ERR_ARG, "algo and segments must not be NULL");
+    if (!algo || !segments || !launches) return fail(WKV7_ERR_ARG, "algo, segments and launches must not be NULL");
     wkv7_opts opts;
     const wkv7_status vs = check_args(B, T, H, N, dt, opts_in, opts, false);   // no buffers needed
     if (vs != WKV7_OK) return vs;
@@ -287,19 +287,26 @@ wkv7_status wkv7_plan(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opts
     bool use_chunk = false;
     const wkv7_status ps = pick_chunk(opts, p, use_chunk);
     if (ps != WKV7_OK) return ps;
-    if (T == 0 || !use_chunk) {
-        *algo = WKV7_ALGO_SEQ;
-        *segments = 0;
+    *algo = WKV7_ALGO_SEQ;
+    *segments = 0;
+    if (T == 0) {   // the state copy (one launch) unless S_T is not requested; counted as one here
+        *launches = 1;
         return WKV7_OK;
     }
-    int cs = 0;
-    const cudaError_t e = wkv7::chunk_segments(p, &cs);
+    if (!use_chunk) {   // the scan, plus the stand-alone epilogue when it is on
+        const int n_epi = (opts.ln_w != nullptr) + (opts.ln_b != nullptr) + (opts.r_k != nullptr);
+        *launches = n_epi == 3 ? 2 : 1;
+        return WKV7_OK;
+    }
+    int cs = 0, n = 0;
+    const cudaError_t e = wkv7::chunk_segments(p, &cs, &n);
     if (e != cudaSuccess) {
         cudaGetLastError();
         return cuda_fail(e, "querying the device for the chunked path");
     }
     *algo = WKV7_ALGO_CHUNK;
     *segments = cs;
+    *launches = n;
     return WKV7_OK;
 }
 

@@ -948,7 +948,7 @@ ChunkPlan plan_launches(const FwdArgs &p, const DeviceInfo &d) {
 
 }  // namespace
 
-cudaError_t chunk_segments(const FwdArgs &p, int *segments) {
+cudaError_t chunk_segments(const FwdArgs &p, int *segments, int *launches) {
     DeviceInfo *di = nullptr;
     const cudaError_t e = device_info(di);
     if (e != cudaSuccess) return e;
@@ -956,6 +956,7 @@ cudaError_t chunk_segments(const FwdArgs &p, int *segments) {
     for (int i = 0; i < pl.n; ++i)
         if (pl.cs[i] > kMaxSegments || di->clusters[pl.cs[i]] <= 0) return cudaErrorInvalidClusterSize;
     *segments = pl.cs[pl.n - 1];   // the CTAs per head of the last launch (the first is 1 when there are two)
+    if (launches) *launches = pl.n;
     return cudaSuccess;
 }
 

@@ -46,7 +46,8 @@ cudaError_t launch_decode(const DecArgs &p);
 cudaError_t launch_copy_state(const FwdArgs &p);   // T == 0: S_T <- S0 (or zeros)
 bool chunk_supported(const FwdArgs &p);            // bf16 inputs, snapshots on chunk boundaries
 cudaError_t launch_chunk(const FwdArgs &p);        // chunked prefill on tcgen05 (epilogue fused)
-cudaError_t chunk_segments(const FwdArgs &p, int *segments);   // CTAs per (b, h) launch_chunk uses
+// CTAs per (b, h) of launch_chunk's last launch, and its number of launches (1 or 2)
+cudaError_t chunk_segments(const FwdArgs &p, int *segments, int *launches = nullptr);
 // Synchronises `stream` and reads the device error word (bounded waits that gave up).
 cudaError_t read_device_error(cudaStream_t stream, unsigned int *value, bool clear);
 

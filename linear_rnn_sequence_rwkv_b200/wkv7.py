@@ -19,6 +19,7 @@ import torch
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libwkv7.so")
 HEAD_SIZE = 64
+ABI_VERSION = 2          # WKV7_ABI_VERSION of include/wkv7.h this binding follows
 
 # wkv7_status
 OK, ERR_ARG, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(7)
@@ -80,8 +81,12 @@ def load():
         lib.wkv7_abi_version.restype = ci
         lib.wkv7_poll_device_error.argtypes = [vp]
         lib.wkv7_poll_device_error.restype = ci
-        lib.wkv7_plan.argtypes = [ci, ci, ci, ci, ci, ctypes.POINTER(Opts), ctypes.POINTER(ci), ctypes.POINTER(ci)]
+        lib.wkv7_plan.argtypes = [ci, ci, ci, ci, ci, ctypes.POINTER(Opts), ctypes.POINTER(ci), ctypes.POINTER(ci),
+                                  ctypes.POINTER(ci)]
         lib.wkv7_plan.restype = ci
+        if lib.wkv7_abi_version() != ABI_VERSION:
+            raise RuntimeError(f"{_LIB_PATH} has ABI version {lib.wkv7_abi_version()}, the binding expects "
+                               f"{ABI_VERSION}: rebuild it")
         _lib = lib
         return lib
 
@@ -126,14 +131,16 @@ def make_opts(algo="auto", chunk=0, snap_every=0, snapshots=None, ln_w=None, ln_
     return o
 
 
-def plan(B, T, H, N=HEAD_SIZE, dtype=torch.bfloat16, **opt_kw):
+def plan(B, T, H, N=HEAD_SIZE, dtype=torch.bfloat16, launches=False, **opt_kw):
     """(algorithm, CTAs per head) wkv7_forward would use on the current device: ("seq", 0) or
-    ("chunk", n) with n = 1 for one CTA per head and n > 1 for a cluster split."""
-    algo, seg = ctypes.c_int(0), ctypes.c_int(0)
+    ("chunk", n) with n = 1 for one CTA per head and n > 1 for a cluster split; with
+    launches=True also the number of kernel launches of the call."""
+    algo, seg, n = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
     st = load().wkv7_plan(B, T, H, N, BF16 if dtype == torch.bfloat16 else F32, ctypes.byref(make_opts(**opt_kw)),
-                          ctypes.byref(algo), ctypes.byref(seg))
+                          ctypes.byref(algo), ctypes.byref(seg), ctypes.byref(n))
     _check(st, "wkv7_plan")
-    return ("seq" if algo.value == ALGOS["seq"] else "chunk"), int(seg.value)
+    out = ("seq" if algo.value == ALGOS["seq"] else "chunk"), int(seg.value)
+    return out + (int(n.value),) if launches else out
 
 
 def workspace_bytes(B, T, H, N=HEAD_SIZE, dtype=torch.bfloat16, **opt_kw) -> int:

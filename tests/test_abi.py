@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_strings(lib):
-    assert lib.wkv7_abi_version() == 1
+    assert lib.wkv7_abi_version() == 2
     assert lib.wkv7_status_string(0) == b"WKV7_OK"
     assert lib.wkv7_status_string(3) == b"WKV7_ERR_ALIGN"
     assert lib.wkv7_status_string(99) == b"WKV7_ERR_UNKNOWN"
@@ -147,3 +147,13 @@ def test_plan_with_snapshot_interval_needs_no_buffer(lib):
         with pytest.raises(wkv7.Wkv7Error) as e:
             wkv7.plan(1, 8192, 2, snap_every=4096)                         # chunked: needs the device
         assert e.value.status == wkv7.ERR_CUDA
+
+
+def test_plan_counts_launches(lib):
+    """The launch count the bench reports: the scan is one launch, plus one for the stand-alone
+    epilogue; T = 0 is the state copy."""
+    import torch
+    assert wkv7.plan(2, 8, 4, launches=True) == ("seq", 0, 1)
+    ln = torch.zeros(4, 64)
+    assert wkv7.plan(2, 8, 4, launches=True, ln_w=ln, ln_b=ln, r_k=ln) == ("seq", 0, 2)
+    assert wkv7.plan(2, 0, 4, launches=True) == ("seq", 0, 1)

@@ -376,3 +376,10 @@ def test_partial_wave_tail_launch(cuda_device):
     ya, Sa, _ = _gpu(d)
     assert torch.equal(ya, y1) and torch.equal(Sa, S1)
     wkv7.poll_device_error()
+
+
+def test_plan_launch_counts_on_device(cuda_device):
+    """One launch per forward call, except the partial-wave split (two)."""
+    assert wkv7.plan(8, 1024, 12, launches=True)[2] == 1
+    algo, seg, n = wkv7.plan(16, 4096, 32, launches=True)
+    assert algo == "chunk" and n in (1, 2) and (n == 1 or seg > 1)
