@@ -124,3 +124,47 @@ def make_inputs(wl: Workload, *, seed: int | None = None, device: str = "cpu",
         out["ln_b"] = (0.1 * randn(H, N)).contiguous()
         out["r_k"] = (0.5 * randn(H, N)).contiguous()
     return out
+
+
+def make_raw_inputs(wl: Workload, *, seed: int | None = None, device: str = "cpu",
+                    B: int | None = None, T: int | None = None, H: int | None = None,
+                    s0: str | None = None, dtype: str | None = None, k_a: bool = True) -> dict:
+    """The same workload's draws *before* the pre-processing, for the path that fuses it
+    into the kernel: r, w_logit (= z), k, v, a_logit ([B, T, H, N] in the workload dtype),
+    k_k ~ U(0.5, 1.5) and k_a ~ U(0, 1) (zeros if ``k_a`` is False) as [H, N] fp32, S0 and
+    the epilogue parameters as in ``make_inputs``. No arithmetic of the method is applied.
+    """
+    B = wl.B if B is None else B
+    T = wl.T if T is None else T
+    H = wl.H if H is None else H
+    N = wl.N
+    s0 = wl.s0 if s0 is None else s0
+    dt = torch_dtype(wl.dtype if dtype is None else dtype)
+    g = torch.Generator(device=device)
+    g.manual_seed(SEED_BASE + 500 + wl.cid if seed is None else seed)
+    shape = (B, T, H, N)
+
+    def randn(*s):
+        return torch.randn(*s, generator=g, device=device, dtype=torch.float32)
+
+    def rand(*s):
+        return torch.rand(*s, generator=g, device=device, dtype=torch.float32)
+
+    out = {}
+    for name in ("r", "k", "v"):
+        out[name] = randn(*shape).to(dt).contiguous()
+    out["w_logit"] = (randn(*shape) + wl.z_mean).to(dt).contiguous()
+    out["a_logit"] = randn(*shape).to(dt).contiguous()
+    out["k_k"] = (0.5 + rand(H, N)).contiguous()
+    out["k_a"] = rand(H, N).contiguous() if k_a else torch.zeros(H, N, device=device)
+    if s0 == "normal":
+        out["S0"] = (0.1 * randn(B, H, N, N)).contiguous()
+    elif s0 == "zeros":
+        out["S0"] = None
+    else:
+        raise ValueError(f"unknown S0 recipe {s0!r}")
+    if wl.epilogue:
+        out["ln_w"] = (1.0 + 0.1 * randn(H, N)).contiguous()
+        out["ln_b"] = (0.1 * randn(H, N)).contiguous()
+        out["r_k"] = (0.5 * randn(H, N)).contiguous()
+    return out

@@ -22,7 +22,9 @@ Readings taken where the pages leave a step open (each listed in the design doc):
   S_{t-1} kk with kk*a (``@`` and ``*`` share precedence, left to right).
 * The readout uses the updated state S_t (the current token is included).
 * kk arrives already L2-normalised, k is the replacement key, w is the decay
-  multiplier itself; nothing is renormalised here.
+  multiplier itself; nothing is renormalised in the recurrence. ``prepare_inputs``
+  states the pre-processing that produces them from the raw time-mixing values
+  (the path that fuses it into the kernel's load stage).
 
 Parity pins: every function here is pinned in tests/test_oracle.py against closed
 forms, brute-force transition products, the paper's elementary-transition
@@ -79,6 +81,28 @@ def group_norm_bonus(y, r, k, v, ln_w, ln_b, r_k, eps=64e-5):
     normed = (y - mean) / np.sqrt(var + eps) * ln_w + ln_b
     bonus = (r * k * r_k).sum(axis=-1, keepdims=True) * v
     return normed + bonus
+
+
+def prepare_inputs(w_logit, a_logit, k, k_k, k_a=None):
+    """The pre-processing the pages place before the update, in fp64 (the rebuttal page's
+    ``time_mixing`` listing: the decay line, the ``a = sigmoid(...)`` line, ``kk = k * k_k``,
+    ``k += k * (a-1) * k_a`` and ``kk /= max(norm(kk), 1e-12)``).
+
+    w_logit, a_logit, k: [B, T, H, N]; k_k, k_a: [H, N] (k_a None = 0).
+    Returns (w, a, kk, k_tilde), each [B, T, H, N] fp64:
+      w = exp(-sigmoid(w_logit) / sqrt(e)), a = sigmoid(a_logit),
+      kk = (k * k_k) / max(||k * k_k||_2, 1e-12) over the head's N channels (from the key
+      before its update), k_tilde = k + k * (a - 1) * k_a.
+    """
+    w_logit, a_logit, k, k_k = (_f64(x) for x in (w_logit, a_logit, k, k_k))
+    k_a = np.zeros_like(k_k) if k_a is None else _f64(k_a)
+    sig = lambda x: 1.0 / (1.0 + np.exp(-x))
+    w = np.exp(-sig(w_logit) / np.e ** 0.5)
+    a = sig(a_logit)
+    kk = k * k_k
+    k_tilde = k + k * (a - 1.0) * k_a
+    kk = kk / np.maximum(np.linalg.norm(kk, axis=-1, keepdims=True), 1e-12)
+    return w, a, kk, k_tilde
 
 
 def transition_matrix(w_t, kk_t, a_t):

@@ -428,3 +428,63 @@ def test_golden_elementary_transitions(impl):
     _close(snaps[0, :, 0], g["S_expected"], 1e-13)
     _close(y[0, :, 0], g["y_expected"], 1e-13)
     _close(S[0, 0], g["S_expected"][-1], 1e-13)
+
+
+# ---- the input pre-processing (fused into the kernel's load stage on the raw path) ----------
+
+def test_prepare_inputs_closed_forms():
+    """Decay and rate at known logits, the decay range, and the removal key's norm."""
+    B, T, H, N = 1, 3, 2, 8
+    rng = np.random.default_rng(7)
+    k = rng.standard_normal((B, T, H, N))
+    k_k = 0.5 + rng.random((H, N))
+    z = np.zeros((B, T, H, N))
+    w, a, kk, kt = reference.prepare_inputs(z, z, k, k_k)
+    assert np.allclose(w, math.exp(-0.5 / math.sqrt(math.e)), rtol=0, atol=1e-15)
+    assert np.allclose(a, 0.5, rtol=0, atol=1e-15)
+    big = np.full((B, T, H, N), 20.0)
+    w_hi, a_hi, _, _ = reference.prepare_inputs(-big, big, k, k_k)             # sigmoid -> 0 / 1
+    w_lo, a_lo, _, _ = reference.prepare_inputs(big, -big, k, k_k)
+    lo = math.exp(-math.exp(-0.5))                                              # w in (e^-e^-1/2, 1)
+    assert np.all(w_hi < 1.0) and np.all(w_hi > 1.0 - 1e-8)
+    assert np.all(w_lo > lo) and np.all(w_lo < lo + 1e-8)
+    assert np.allclose(a_hi, 1.0, atol=1e-8) and np.allclose(a_lo, 0.0, atol=1e-8)
+    assert np.allclose(np.linalg.norm(kk, axis=-1), 1.0, atol=1e-14)
+    assert np.allclose(kt, k, rtol=0, atol=0)                                 # k_a = 0: k unchanged
+
+
+def test_prepare_inputs_removal_key_uses_the_key_before_its_update():
+    """kk is the normalised k * k_k of the raw key whatever k_a is; k_tilde = k * (1 + (a-1) k_a)."""
+    B, T, H, N = 2, 4, 3, 16
+    rng = np.random.default_rng(8)
+    k = rng.standard_normal((B, T, H, N))
+    k_k = 0.5 + rng.random((H, N))
+    k_a = rng.random((H, N))
+    zw, za = rng.standard_normal((B, T, H, N)), rng.standard_normal((B, T, H, N))
+    w, a, kk, kt = reference.prepare_inputs(zw, za, k, k_k, k_a)
+    _, _, kk0, _ = reference.prepare_inputs(zw, za, k, k_k, None)
+    assert np.array_equal(kk, kk0)
+    direction = (k * k_k) / np.linalg.norm(k * k_k, axis=-1, keepdims=True)
+    assert np.allclose(kk, direction, atol=1e-14)
+    assert np.allclose(kt, k * (1.0 + (a - 1.0) * k_a), atol=1e-14)
+    _, a1, _, kt1 = reference.prepare_inputs(zw, np.full_like(za, 60.0), k, k_k, k_a)   # a -> 1
+    assert np.allclose(kt1, k, atol=1e-12)
+    _, _, _, kt2 = reference.prepare_inputs(zw, za, k, k_k, np.ones((H, N)))            # k_a = 1
+    assert np.allclose(kt2, k * a, atol=1e-14)
+
+
+def test_prepare_inputs_zero_key_is_finite():
+    """A zero key gives a zero removal key (the 1e-12 floor), not a division by zero."""
+    k = np.zeros((1, 1, 1, 64))
+    _, _, kk, _ = reference.prepare_inputs(np.zeros_like(k), np.zeros_like(k), k, np.ones((1, 64)))
+    assert np.all(np.isfinite(kk)) and np.all(kk == 0.0)
+
+
+def test_raw_generator_matches_prepared_recipe_ranges():
+    """The raw draws, prepared by the oracle, land in the ranges the prepared recipe states."""
+    d = inputs.make_raw_inputs(inputs.WORKLOADS[1], B=1, T=40, H=2, seed=11)
+    w, a, kk, kt = reference.prepare_inputs(d["w_logit"], d["a_logit"], d["k"], d["k_k"], d["k_a"])
+    assert np.all((w > math.exp(-math.exp(-0.5))) & (w <= 1.0))
+    assert np.all((a > 0.0) & (a < 1.0))
+    assert np.allclose(np.linalg.norm(kk, axis=-1), 1.0, atol=1e-12)
+    assert np.all(np.abs(kt) <= np.abs(reference._f64(d["k"])) + 1e-12)        # 0 < 1 + (a-1) k_a <= 1
