@@ -38,6 +38,7 @@ METRIC = "WKV-7 Mtokens·heads/s (prefill, decode) at N=64 bf16; % of HBM/FP32/T
 UNIT = "Mtoken·heads/s"
 L2_BYTES = 126 * 2 ** 20
 NAMES = ("r", "w", "k", "v", "kk", "a")
+RAW_NAMES = ("r", "w_logit", "k", "v", "a_logit")   # raw time-mixing values (pre-processing fused)
 
 WORKLOADS = {
     "prefill-0.19b": dict(cid=1, default_steps=200),
@@ -68,11 +69,12 @@ def kernel_digest(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def measured_traffic(kernel: str, workload: str):
+def measured_traffic(kernel: str, workload: str, raw: bool = False):
     """dram__bytes_read.sum + dram__bytes_write.sum per launch recorded in
     profiles/<kernel>_<workload>.md, or None without a capture or when the kernel's device
     code has changed since it was taken (the summary records the digest it was taken at)."""
-    path = os.path.join(ROOT, "profiles", f"{kernel}_{PROFILE_TAGS.get(workload, workload)}.md")
+    tag = PROFILE_TAGS.get(workload, workload) + ("-raw-inputs" if raw else "")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{tag}.md")
     try:
         with open(path) as f:
             text = f.read()
@@ -187,12 +189,14 @@ def max_over_ranks(x: float, world: int, device) -> float:
 
 # ---- workload set-up ---------------------------------------------------------------------------
 
-def algorithmic_bytes(wl, B, T, H, dt_bytes, s0: bool, s_out: bool, snaps: int, epilogue: bool) -> int:
-    """Bytes one forward must move at minimum: inputs once, y once, states once."""
+def algorithmic_bytes(wl, B, T, H, dt_bytes, s0: bool, s_out: bool, snaps: int, epilogue: bool,
+                      raw: bool = False) -> int:
+    """Bytes one forward must move at minimum: inputs once, y once, states once (raw inputs:
+    five token vectors instead of six, plus the per-head k_k and k_a)."""
     N = wl.N
-    per_tok = 6 * N * dt_bytes + N * 4
+    per_tok = (5 if raw else 6) * N * dt_bytes + N * 4
     st = N * N * 4
-    extra = (H * N * 3 * 4) if epilogue else 0
+    extra = (H * N * 3 * 4 if epilogue else 0) + (H * N * 2 * 4 if raw else 0)
     return B * T * H * per_tok + B * H * st * (int(s0) + int(s_out) + snaps) + extra
 
 
@@ -207,6 +211,9 @@ def run_gpu(args, world, rank, local):
     peaks, peak_kind = _peaks()
     stream = torch.cuda.current_stream(dev)
     decode = args.workload == "decode"
+    raw = args.inputs == "raw"
+    if decode and raw:
+        raise SystemExit("--inputs raw applies to the prefill workloads")
     snap_every = wl.snap_every
 
     # independent batches per rank (seed offset), rotating input sets larger than L2
@@ -229,9 +236,11 @@ def run_gpu(args, world, rank, local):
         epilogue = False
     else:
         B, T, H, N = wl.B, wl.T, wl.H, wl.N
-        set_bytes = B * T * H * N * (6 * 2)
+        n_vec = 5 if raw else 6
+        set_bytes = B * T * H * N * (n_vec * 2)
         n_sets = max(1, min(8, math.ceil(2 * L2_BYTES / set_bytes)))
-        sets = [inputs.make_inputs(wl, device=str(dev), seed=seed0 + 17 * i) for i in range(n_sets)]
+        make = inputs.make_raw_inputs if raw else inputs.make_inputs
+        sets = [make(wl, device=str(dev), seed=seed0 + 17 * i) for i in range(n_sets)]
         y = torch.empty(B, T, H, N, device=dev)
         S_T = torch.empty(B, H, N, N, device=dev)
         snaps = torch.empty(B, T // snap_every, H, N, N, device=dev) if snap_every else None
@@ -243,10 +252,15 @@ def run_gpu(args, world, rank, local):
         def step(i):
             s = sets[i % n_sets]
             ep = dict(ln_w=s["ln_w"], ln_b=s["ln_b"], r_k=s["r_k"]) if epilogue else {}
-            wkv7.forward(*(s[n] for n in NAMES), s["S0"], algo=args.algo, chunk=args.chunk, y=y, S_T=S_T,
-                         snap_every=snap_every, snapshots=snaps, workspace=ws, **ep)
+            if raw:
+                wkv7.forward_raw(*(s[n] for n in RAW_NAMES), s["k_k"], s["k_a"], s["S0"], algo=args.algo,
+                                 chunk=args.chunk, y=y, S_T=S_T, snap_every=snap_every, snapshots=snaps,
+                                 workspace=ws, **ep)
+            else:
+                wkv7.forward(*(s[n] for n in NAMES), s["S0"], algo=args.algo, chunk=args.chunk, y=y, S_T=S_T,
+                             snap_every=snap_every, snapshots=snaps, workspace=ws, **ep)
         bytes_per_launch = algorithmic_bytes(wl, B, T, H, 2, sets[0]["S0"] is not None, True,
-                                             T // snap_every if snap_every else 0, epilogue)
+                                             T // snap_every if snap_every else 0, epilogue, raw)
         launches_per_step = 1 + (1 if epilogue and _path_name(args) == "seq" else 0)
 
     units_per_step = B * T * H
@@ -289,12 +303,12 @@ def run_gpu(args, world, rank, local):
         roof = {"bound": "alu", "achieved": round(achieved, 3), "peak": round(fp32_peak, 2),
                 "unit": "TFLOP/s", "frac": round(achieved / fp32_peak, 4),
                 "peak_source": f"148 SMs x 128 FP32 lanes x 2 flop x {sm_max:.0f} MHz (derived)",
-                "traffic": measured_traffic("seq_kernel", args.workload), "kernel": "seq_kernel",
+                "traffic": measured_traffic("seq_kernel", args.workload, raw), "kernel": "seq_kernel",
                 "hbm_gbs": round(achieved_gbs, 1), "hbm_frac": round(achieved_gbs / hbm_peak, 4)}
     else:
         roof = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved_gbs / hbm_peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
-                "traffic": measured_traffic("decode_kernel" if decode else "chunk_kernel", args.workload),
+                "traffic": measured_traffic("decode_kernel" if decode else "chunk_kernel", args.workload, raw),
                 "kernel": "decode_kernel" if decode else "chunk_kernel",
                 "recurrence_tflops": round(flops_per_launch / (launch_ms * 1e-3) / 1e12, 3)}
     roof["algorithmic_bytes_per_launch"] = bytes_per_launch
@@ -303,7 +317,7 @@ def run_gpu(args, world, rank, local):
     e2e = None
     if not decode:
         e2e = run_e2e(args, wl, dev, stream, B, T, H, N, seed0, epilogue, snap_every, warmup,
-                      max(1, min(steps, 10)), world)
+                      max(1, min(steps, 10)), world, raw)
 
     out = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": steps,
@@ -312,9 +326,11 @@ def run_gpu(args, world, rank, local):
         "data": "synthetic (seeded torch Philox; shapes and value ranges of the RWKV-7 pages' workloads)",
         "config": {"workload": f"{args.workload}: {wl.name}", "B": B, "T": T, "H": H, "N": N,
                    "input_dtype": "bf16", "path": path, "chunk": args.chunk or None,
+                   "inputs": ("raw: decay/rate logits and the key before its update, pre-processing fused"
+                              if raw else "prepared: w, a, kk, k~"),
                    "ctas_per_head": ctas_per_head,
                    "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world} (independent (b,h) units)",
-                   "l2": (f"{n_sets} rotating input sets, {n_sets * B * T * H * N * 12 / 1e6:.0f} MB > 126 MB L2"
+                   "l2": (f"{n_sets} rotating input sets, {n_sets * set_bytes / 1e6:.0f} MB > 126 MB L2"
                           if not decode else "fp32 state 168 MB > 126 MB L2, 128 rotating token inputs")},
         "roofline": roof,
         "e2e": e2e,
@@ -331,22 +347,33 @@ def _path_name(args):
     return {"auto": "chunk", "seq": "seq", "chunk": "chunk", "split": "chunk"}[args.algo]
 
 
-def run_e2e(args, wl, dev, stream, B, T, H, N, seed, epilogue, snap_every, warmup, steps, world):
-    """Same metric through wkv7.forward with pinned HOST tensors: H2D of the inputs,
-    the kernels and D2H of y and S_T are all inside the timed region."""
+def run_e2e(args, wl, dev, stream, B, T, H, N, seed, epilogue, snap_every, warmup, steps, world, raw=False):
+    """Same metric through wkv7.forward (or forward_raw) with pinned HOST tensors: H2D of the
+    inputs, the kernels and D2H of y and S_T are all inside the timed region."""
     from linear_rnn_sequence_rwkv_b200 import wkv7
-    d = inputs.make_inputs(wl, device="cpu", seed=seed + 999)
+    d = (inputs.make_raw_inputs if raw else inputs.make_inputs)(wl, device="cpu", seed=seed + 999)
     host = {n: (v.pin_memory() if isinstance(v, torch.Tensor) else v) for n, v in d.items()}
-    h2d = sum(host[n].numel() * host[n].element_size() for n in NAMES)
+    h2d = sum(host[n].numel() * host[n].element_size() for n in (RAW_NAMES if raw else NAMES))
     h2d += 0 if host["S0"] is None else host["S0"].numel() * 4
     if epilogue:
         h2d += 3 * H * N * 4
+    if raw:
+        h2d += 2 * H * N * 4
     d2h = B * T * H * N * 4 + B * H * N * N * 4 + (B * (T // snap_every) * H * N * N * 4 if snap_every else 0)
     y_h = torch.empty(B, T, H, N).pin_memory()
     S_h = torch.empty(B, H, N, N).pin_memory()
 
     def once():
         ep = {n: host[n] for n in ("ln_w", "ln_b", "r_k")} if epilogue else {}
+        if raw:   # the raw entry takes device tensors: copy in, run, copy out, all on this stream
+            dv = {n: (None if host[n] is None else host[n].to(dev, non_blocking=True))
+                  for n in RAW_NAMES + ("k_k", "k_a", "S0")}
+            dep = {n: v.to(dev, non_blocking=True) for n, v in ep.items()}
+            y, S, _ = wkv7.forward_raw(*(dv[n] for n in RAW_NAMES), dv["k_k"], dv["k_a"], dv["S0"], algo=args.algo,
+                                       chunk=args.chunk, snap_every=snap_every, **dep)
+            y_h.copy_(y, non_blocking=True)
+            S_h.copy_(S, non_blocking=True)
+            return y_h, S_h
         y, S, _ = wkv7.forward(*(host[n] for n in NAMES), host["S0"], algo=args.algo, chunk=args.chunk,
                                snap_every=snap_every, out_host=(y_h, S_h), **ep)
         return y, S
@@ -440,6 +467,8 @@ def main(argv=None):
     ap.add_argument("--algo", choices=["auto", "seq", "chunk", "split"], default="auto")
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--inputs", choices=["prepared", "raw"], default="prepared",
+                    help="raw: decay/rate logits and the key before its update, pre-processing fused")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -126,6 +126,31 @@ WKV7_API wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype dt,
                          void *stream);
 
 /*
+ * Prefill / full-sequence forward from the raw time-mixing values: the pre-processing the
+ * pages place before the update (rebuttal page, the numpy time_mixing listing: the decay, the
+ * in-context learning rate, the removal key and its normalisation, the key update) is
+ * done on the device in the load stage of whichever kernel runs (chunked or scan, and in the
+ * separate epilogue kernel for the bonus), then the same recurrence and epilogue as
+ * wkv7_forward:
+ *     w  = exp(-sigmoid(w_logit) / sqrt(e))          a  = sigmoid(a_logit)
+ *     kk = (k * k_k) / max(||k * k_k||_2, 1e-12)     (per head, over its N channels)
+ *     k~ = k + k * (a - 1) * k_a                     (kk uses k, the update and bonus use k~)
+ *
+ * Inputs  r, w_logit, k, v, a_logit : [B][T][H][N] of dtype dt (k is the key before its
+ *                                     update).
+ *         k_k                       : [H][N] fp32, required.   k_a : [H][N] fp32 or NULL (= 0).
+ * Everything else (S0, y, S_T, opts, workspace, errors) as wkv7_forward; the prepared values
+ * are never written to memory. WKV7_ERR_ARG also when k_k is NULL (T > 0).
+ */
+WKV7_API wkv7_status wkv7_forward_raw(int B, int T, int H, int N, wkv7_dtype dt,
+                             const void *r, const void *w_logit, const void *k, const void *v,
+                             const void *a_logit, const float *k_k, const float *k_a,
+                             const float *S0, float *y, float *S_T,
+                             const wkv7_opts *opts,
+                             void *workspace, size_t workspace_bytes,
+                             void *stream);
+
+/*
  * One decode step for every (b, h): the recurrence for a single token, with the
  * state read and written in place.
  *

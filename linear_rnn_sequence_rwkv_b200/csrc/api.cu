@@ -177,10 +177,16 @@ size_t wkv7_workspace_bytes(int B, int T, int H, int N, wkv7_dtype dt, const wkv
     return 0;
 }
 
-wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype dt, const void *r, const void *w,
-                         const void *k, const void *v, const void *kk, const void *a, const float *S0,
-                         float *y, float *S_T, const wkv7_opts *opts_in, void *workspace,
-                         size_t workspace_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// wkv7_forward and wkv7_forward_raw. raw: w and a are the decay and rate logits, k the key
+// before its update, kk is unused, k_k (required) and k_a (nullable) are the [H][N] parameters.
+wkv7_status forward_impl(bool raw, int B, int T, int H, int N, wkv7_dtype dt, const void *r, const void *w,
+                         const void *k, const void *v, const void *kk, const void *a, const float *k_k,
+                         const float *k_a, const float *S0, float *y, float *S_T, const wkv7_opts *opts_in,
+                         void *workspace, size_t workspace_bytes, void *stream) {
     g_err[0] = '\0';
     wkv7_opts opts;
     const wkv7_status vs = check_args(B, T, H, N, dt, opts_in, opts);
@@ -194,20 +200,23 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype dt, const void *
     const size_t in_bytes = tok * elem_bytes(dt), y_bytes = tok * 4, st_bytes = st * 4;
     const int n_snap = opts.snap_every > 0 ? T / opts.snap_every : 0;
     const size_t snap_bytes = st_bytes * static_cast<size_t>(n_snap);
+    const size_t par_bytes = size_t(H) * N * 4;
+    const char *wn = raw ? "w_logit" : "w", *an = raw ? "a_logit" : "a";
 
     if (T > 0) {
-        const void *req[] = {r, w, k, v, kk, a, y};
-        const char *names[] = {"r", "w", "k", "v", "kk", "a", "y"};
+        const void *req[] = {r, w, k, v, raw ? k_k : kk, a, y};
+        const char *names[] = {"r", wn, "k", "v", raw ? "k_k" : "kk", an, "y"};
         for (int i = 0; i < 7; ++i)
             if (!req[i]) return fail(WKV7_ERR_ARG, "%s is NULL", names[i]);
     }
-    const Buf bufs[] = {{"r", r, T ? in_bytes : 0},      {"w", w, T ? in_bytes : 0},
+    const Buf bufs[] = {{"r", r, T ? in_bytes : 0},      {wn, w, T ? in_bytes : 0},
                         {"k", k, T ? in_bytes : 0},      {"v", v, T ? in_bytes : 0},
-                        {"kk", kk, T ? in_bytes : 0},    {"a", a, T ? in_bytes : 0},
+                        {"kk", raw ? nullptr : kk, T ? in_bytes : 0}, {an, a, T ? in_bytes : 0},
                         {"S0", S0, st_bytes},            {"y", y, T ? y_bytes : 0},
                         {"S_T", S_T, st_bytes},          {"snapshots", n_snap ? opts.snapshots : nullptr, snap_bytes},
-                        {"ln_w", opts.ln_w, size_t(H) * N * 4}, {"ln_b", opts.ln_b, size_t(H) * N * 4},
-                        {"r_k", opts.r_k, size_t(H) * N * 4},   {"workspace", workspace, workspace_bytes}};
+                        {"ln_w", opts.ln_w, par_bytes},  {"ln_b", opts.ln_b, par_bytes},
+                        {"r_k", opts.r_k, par_bytes},    {"workspace", workspace, workspace_bytes},
+                        {"k_k", raw ? k_k : nullptr, par_bytes}, {"k_a", raw ? k_a : nullptr, par_bytes}};
     constexpr int nb = sizeof(bufs) / sizeof(bufs[0]);
     for (int i = 0; i < nb; ++i)
         if (bufs[i].ptr && !aligned16(bufs[i].ptr))
@@ -240,11 +249,12 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype dt, const void *
 
     wkv7::FwdArgs p{};
     p.B = B; p.T = T; p.H = H; p.dt = dt;
-    p.r = r; p.w = w; p.k = k; p.v = v; p.kk = kk; p.a = a;
+    p.r = r; p.w = w; p.k = k; p.v = v; p.kk = raw ? nullptr : kk; p.a = a;
     p.S0 = S0; p.y = y; p.S_T = S_T;
     p.snap_every = n_snap ? opts.snap_every : 0;
     p.snaps = n_snap ? opts.snapshots : nullptr;
     p.ln_w = opts.ln_w; p.ln_b = opts.ln_b; p.r_k = opts.r_k; p.gn_eps = opts.gn_eps;
+    p.raw = raw; p.k_k = raw ? k_k : nullptr; p.k_a = raw ? k_a : nullptr;
     p.chunk = opts.chunk;
     p.segments = requested_segments(opts);
     p.ws = workspace; p.ws_bytes = workspace_bytes;
@@ -258,7 +268,7 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype dt, const void *
     bool use_chunk = false;
     const wkv7_status ps = pick_chunk(opts, p, use_chunk);
     if (ps != WKV7_OK) return ps;
-    if (use_chunk) {
+    if (use_chunk) {   // raw inputs are prepared in each kernel's load stage
         e = wkv7::launch_chunk(p);
         if (e != cudaSuccess) return cuda_fail(e, "chunked-prefill launch");
         return WKV7_OK;
@@ -270,6 +280,26 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype dt, const void *
         if (e != cudaSuccess) return cuda_fail(e, "epilogue launch");
     }
     return WKV7_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype dt, const void *r, const void *w,
+                         const void *k, const void *v, const void *kk, const void *a, const float *S0,
+                         float *y, float *S_T, const wkv7_opts *opts_in, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+    return forward_impl(false, B, T, H, N, dt, r, w, k, v, kk, a, nullptr, nullptr, S0, y, S_T, opts_in,
+                        workspace, workspace_bytes, stream);
+}
+
+wkv7_status wkv7_forward_raw(int B, int T, int H, int N, wkv7_dtype dt, const void *r, const void *w_logit,
+                             const void *k, const void *v, const void *a_logit, const float *k_k,
+                             const float *k_a, const float *S0, float *y, float *S_T, const wkv7_opts *opts_in,
+                             void *workspace, size_t workspace_bytes, void *stream) {
+    return forward_impl(true, B, T, H, N, dt, r, w_logit, k, v, nullptr, a_logit, k_k, k_a, S0, y, S_T, opts_in,
+                        workspace, workspace_bytes, stream);
 }
 
 wkv7_status wkv7_plan(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opts *opts_in, int *algo,

@@ -86,6 +86,8 @@ struct Small {
     float dk[C];              // r_t . k_t (exact current-token Gram entry)
     float db[C];              // r_t . (kk_t * a_t)
     float ln_w[2][C], ln_b[2][C], r_k[2][C];   // epilogue parameters, by head parity
+    float k_k[2][C], k_a[2][C];                 // raw inputs: removal-key scale, key-update rate
+    float inv_norm[C];                          // raw inputs: 1 / max(||k_t * k_k||, 1e-12) per token
     uint64_t bar_tma;
     uint64_t bar_mma;
     uint64_t bar_state;       // split mode: the carried state has arrived in B5 (kSendThreads arrivals)
@@ -129,6 +131,7 @@ struct ChunkArgs {
     int snap_every, n_snap;
     const float *ln_w, *ln_b, *r_k;
     float gn_eps;
+    const float *k_k, *k_a;   // raw inputs: the removal-key scale and the key-update rate ([H][64]; k_a nullable)
     unsigned int *err;
     unsigned long long timeout_ns;
 };
@@ -177,6 +180,12 @@ __device__ __forceinline__ bool bar_named_or(int id, int n, bool v) {
     return r != 0;
 }
 
+// RAW: the inputs are the pages' time-mixing values before their pre-processing (the decay and
+// rate logits, the raw key, the per-head removal-key scale k_k and key-update rate k_a); the
+// load stage computes w = exp(-sigmoid(w_logit) / sqrt(e)), a = sigmoid(a_logit),
+// kk = (k * k_k) / max(||k * k_k||, 1e-12) and k~ = k + k (a - 1) k_a (rebuttal page, the
+// time_mixing listing) in fp32. Otherwise the inputs are r, w, k~, v, kk, a themselves.
+template <bool RAW>
 __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constant__ ChunkMaps maps, const ChunkArgs p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
@@ -247,11 +256,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     int y_h = 0, y_c0 = 0, y_b = 0;    // its coordinates
     bool tma_pending = false, mma_pending = false, failed = false;
 
-    auto issue_tma = [&](int u, int c) {   // one thread: the six tiles of chunk c of head u
+    constexpr uint32_t kTileBytes = (RAW ? 5 : 6) * 8192;   // RAW has no kk tile
+    auto issue_tma = [&](int u, int c) {   // one thread: the input tiles of chunk c of head u
         const int b = u / p.H, hh = u % p.H;
-        mbar_arrive_expect_tx(&S.bar_tma, 6 * 8192);
+        mbar_arrive_expect_tx(&S.bar_tma, kTileBytes);
 #pragma unroll
-        for (int x = 0; x < 6; ++x) tma_load_4d(sm + OFF_IN + x * 8192, &maps.m[x], &S.bar_tma, 0, hh, c * C, b);
+        for (int x = 0; x < 6; ++x)
+            if (!(RAW && x == XKK)) tma_load_4d(sm + OFF_IN + x * 8192, &maps.m[x], &S.bar_tma, 0, hh, c * C, b);
     };
     // Waits: one thread polls the mbarrier (bounded, acquire) and the others wait in a hardware
     // barrier with it; many polling threads would crowd the shared-memory pipe that the other
@@ -279,11 +290,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         tc_fence_before();
         __syncthreads();
     };
-    auto load_params = [&](int u, int slot, int i) {   // epilogue parameters of head u, element i
+    auto load_params = [&](int u, int slot, int i) {   // per-head parameters of head u, element i
         const int hh = u % p.H;
         S.ln_w[slot][i] = epi ? p.ln_w[hh * 64 + i] : 1.f;
         S.ln_b[slot][i] = epi ? p.ln_b[hh * 64 + i] : 0.f;
         S.r_k[slot][i] = epi ? p.r_k[hh * 64 + i] : 0.f;
+        if (RAW) {
+            S.k_k[slot][i] = p.k_k[hh * 64 + i];
+            S.k_a[slot][i] = p.k_a ? p.k_a[hh * 64 + i] : 0.f;
+        }
     };
     auto load_state = [&](int u) {   // all threads: S_0 of head u (or zeros) -> B5, tf32, row = value channel
         for (int e = tid; e < 1024; e += kThreads) {
@@ -314,7 +329,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int t = 16 * q + 8 * h8 + e;
-                    const float w = in_col(wt, t, xo, e);
+                    float w = in_col(wt, t, xo, e);
+                    if (RAW) w = __expf(__fdividef(-0.60653065971263342f, 1.f + __expf(-w)));   // exp(-sigmoid(z)/sqrt(e))
                     run *= (t < Lc) ? w : 1.f;   // padded tokens: w = 1
                     GT[(t + 1) * GTS + j] = run;
                 }
@@ -334,6 +350,22 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 GT[j] = 1.f;
                 S.gC[ip][j] = S.tq[0][j] * S.tq[1][j] * S.tq[2][j] * S.tq[3][j];
             }
+            if (RAW) {   // removal-key norms: four threads per token, sixteen channels each
+                const int t = ft >> 2, j0 = 16 * (ft & 3);
+                float k8[8], ss = 0.f;
+#pragma unroll
+                for (int hlf = 0; hlf < 2; ++hlf) {
+                    in_row8(IN + XK * 8192, t, j0 + 8 * hlf, k8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float x = k8[e] * S.k_k[us][j0 + 8 * hlf + e];
+                        ss = fmaf(x, x, ss);
+                    }
+                }
+                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+                if ((ft & 3) == 0) S.inv_norm[t] = rsqrtf(fmaxf(ss, 1e-24f));   // 1 / max(||.||, 1e-12)
+            }
         }
         bar_named(BAR_FRONT, kFrontThreads);
         // P3: one (token t, channel octet o) per thread and pass. In a quarter-warp, token t takes
@@ -349,9 +381,26 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
             const int t = tbase + 2 * half + hi;
             float r8[8], kk8[8], k8[8], a8[8];
             in_row8(IN + XR * 8192, t, j0, r8);
-            in_row8(IN + XKK * 8192, t, j0, kk8);
             in_row8(IN + XK * 8192, t, j0, k8);
             in_row8(IN + XA * 8192, t, j0, a8);
+            if (RAW) {
+                // a = sigmoid(a_logit); kk = k*k_k / max(||k*k_k||, 1e-12) with the norm from P2;
+                // k~ = k + k (a - 1) k_a, from the key before its update
+                const float inv_norm = S.inv_norm[t];
+                float kkp[8], kap[8];
+                *reinterpret_cast<float4 *>(kkp) = *reinterpret_cast<const float4 *>(&S.k_k[us][j0]);
+                *reinterpret_cast<float4 *>(kkp + 4) = *reinterpret_cast<const float4 *>(&S.k_k[us][j0 + 4]);
+                *reinterpret_cast<float4 *>(kap) = *reinterpret_cast<const float4 *>(&S.k_a[us][j0]);
+                *reinterpret_cast<float4 *>(kap + 4) = *reinterpret_cast<const float4 *>(&S.k_a[us][j0 + 4]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    a8[e] = __fdividef(1.f, 1.f + __expf(-a8[e]));   // exp overflow -> 0, the limit
+                    kk8[e] = k8[e] * kkp[e] * inv_norm;
+                    k8[e] = fmaf(k8[e] * (a8[e] - 1.f), kap[e], k8[e]);
+                }
+            } else {
+                in_row8(IN + XKK * 8192, t, j0, kk8);
+            }
             const float4 ga = *reinterpret_cast<const float4 *>(GT + t * GTS + j0);         // g_{t-1}
             const float4 gb = *reinterpret_cast<const float4 *>(GT + t * GTS + j0 + 4);
             const float4 gc = *reinterpret_cast<const float4 *>(GT + (t + 1) * GTS + j0);   // g_t
@@ -510,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         if (tid == 0) {
             // the next chunk's six input tiles are issued by six warps in P5; their byte count
             // is registered here, ordered before those issues by the barrier after R1
-            if (more) mbar_arrive_expect_tx(&S.bar_tma, 6 * 8192);
+            if (more) mbar_arrive_expect_tx(&S.bar_tma, kTileBytes);
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)   // R1: Grams = [KKd; Rd] [Bi; Ki]^T
@@ -572,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         if (more && lane == 0 && colg && (warp >> 2) < 3) {
             // the input tiles were last read in P4: six warps each issue one tile of the next chunk
             const int x = (warp >> 2) * 2 + (warp & 1);
-            tma_load_4d(sm + OFF_IN + x * 8192, &maps.m[x], &S.bar_tma, 0, nu % p.H, nc * C, nu / p.H);
+            if (!(RAW && x == XKK)) tma_load_4d(sm + OFF_IN + x * 8192, &maps.m[x], &S.bar_tma, 0, nu % p.H, nc * C, nu / p.H);
         }
         if (colg) {
             const int t = L;
@@ -868,15 +917,17 @@ cudaError_t device_info(DeviceInfo *&out) {
     if (!d.attr_set) {
         if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
         if ((e = cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_device_error)) != cudaSuccess) return e;
-        if ((e = cudaFuncSetAttribute(chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_BYTES))) !=
-            cudaSuccess)
+        if ((e = cudaFuncSetAttribute(chunk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(SMEM_BYTES))) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(chunk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(SMEM_BYTES))) != cudaSuccess)
             return e;
         d.clusters[1] = d.sms;
         for (int cs = 2; cs <= kMaxSegments; ++cs) {
             cudaLaunchAttribute attr;
             const cudaLaunchConfig_t cfg = launch_config(cs * (d.sms / cs), cs, nullptr, &attr);
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, chunk_kernel, &cfg) != cudaSuccess) {
+            if (cudaOccupancyMaxActiveClusters(&n, chunk_kernel<false>, &cfg) != cudaSuccess) {
                 cudaGetLastError();
                 n = 0;
             }
@@ -971,7 +1022,8 @@ cudaError_t launch_chunk(const FwdArgs &p) {
     cudaError_t e = device_info(di);
     if (e != cudaSuccess) return e;
     ChunkMaps maps;
-    const void *src[6] = {p.r, p.w, p.k, p.v, p.kk, p.a};
+    // raw inputs: slot XW holds the decay logit, XA the rate logit, and the kk slot is not loaded
+    const void *src[6] = {p.r, p.w, p.k, p.v, p.raw ? p.k : p.kk, p.a};
     const cuuint64_t dims[4] = {cuuint64_t(kN), cuuint64_t(p.H), cuuint64_t(p.T), cuuint64_t(p.B)};
     const cuuint64_t strides[3] = {cuuint64_t(kN) * 2, cuuint64_t(p.H) * kN * 2, cuuint64_t(p.T) * p.H * kN * 2};
     const cuuint32_t box[4] = {cuuint32_t(kN), 1, cuuint32_t(C), 1};
@@ -997,6 +1049,7 @@ cudaError_t launch_chunk(const FwdArgs &p) {
     a.snap_every = p.snap_every;
     a.n_snap = p.snap_every > 0 ? p.T / p.snap_every : 0;
     a.ln_w = p.ln_w; a.ln_b = p.ln_b; a.r_k = p.r_k; a.gn_eps = p.gn_eps;
+    a.k_k = p.k_k; a.k_a = p.k_a;
     a.err = di->err;
     a.timeout_ns = 2000000000ull;
     int cs = 1;
@@ -1008,7 +1061,8 @@ cudaError_t launch_chunk(const FwdArgs &p) {
         const int ncl = pl.units[i] < di->clusters[pl.cs[i]] ? pl.units[i] : di->clusters[pl.cs[i]];
         cudaLaunchAttribute attr;
         const cudaLaunchConfig_t cfg = launch_config(ncl * pl.cs[i], pl.cs[i], p.stream, &attr);
-        if ((e = cudaLaunchKernelEx(&cfg, chunk_kernel, maps, a)) != cudaSuccess) return e;
+        e = p.raw ? cudaLaunchKernelEx(&cfg, chunk_kernel<true>, maps, a) : cudaLaunchKernelEx(&cfg, chunk_kernel<false>, maps, a);
+        if (e != cudaSuccess) return e;
         a.unit0 = a.unit_end;
     }
     return cudaSuccess;

@@ -22,6 +22,8 @@ struct FwdArgs {
     int snap_every;        // 0 = off
     float *snaps;          // [B][T/snap_every][H][N][N]
     const float *ln_w, *ln_b, *r_k;   // all null = no epilogue
+    bool raw;              // w and a hold the decay / rate logits, k the raw key; kk unused
+    const float *k_k, *k_a;   // raw: [H][N] removal-key scale and key-update rate (k_a nullable)
     float gn_eps;
     int chunk;
     int segments;          // CTAs per (b, h) on the chunked path; 0 = automatic

@@ -51,7 +51,11 @@ __device__ __forceinline__ void store_vals(float *dst, const float (&o)[E]) {
     for (int j = 0; j < E; j += 4) *reinterpret_cast<float4 *>(dst + j) = make_float4(o[j], o[j + 1], o[j + 2], o[j + 3]);
 }
 
-template <class Tin, int RPT>
+// RAW: w and a hold the decay and rate logits, k the key before its update and kk is not read;
+// the staging step turns them into w, b = kk * a, k~ and the unit-norm removal key (rebuttal
+// page, the time_mixing listing: decay, learning rate, removal key with its 1e-12 norm floor,
+// key update), with the formulas of the chunked kernel's load stage.
+template <class Tin, int RPT, bool RAW>
 __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const FwdArgs p) {
     using Sm = SeqSmem<Tin, RPT>;
     constexpr int TB = Sm::TB, ROWS = Sm::ROWS;
@@ -94,6 +98,7 @@ __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const FwdArgs p) {
         for (int x = 0; x < 5; ++x)
 #pragma unroll
             for (int i = 0; i < VEC_CH; ++i) {
+                if (RAW && x == 1) continue;   // the removal key is derived from k
                 const int c = threadIdx.x + kSeqThreads * i, t = c / CPT, e = (c % CPT) * EPC;
                 raw[x][i] = t0 + t < T ? __ldg(reinterpret_cast<const uint4 *>(src[x] + tok_off(t0 + t) + e))
                                        : make_uint4(0, 0, 0, 0);
@@ -113,10 +118,29 @@ __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const FwdArgs p) {
             const int c = threadIdx.x + kSeqThreads * i, t = c / CPT, e = (c % CPT) * EPC;
             float w_[EPC], kk_[EPC], a_[EPC], k_[EPC], r_[EPC], b_[EPC];
             unpack16(raw[0][i], tag, w_);
-            unpack16(raw[1][i], tag, kk_);
             unpack16(raw[2][i], tag, a_);
             unpack16(raw[3][i], tag, k_);
             unpack16(raw[4][i], tag, r_);
+            if (RAW) {
+                // the CPT consecutive threads that hold one token reduce ||k * k_k|| by shuffles
+                const float *kk_p = p.k_k + h * kN + e, *ka_p = p.k_a ? p.k_a + h * kN + e : nullptr;
+                float ss = 0.f;
+#pragma unroll
+                for (int j = 0; j < EPC; ++j) {
+                    w_[j] = __expf(-0.60653065971263342f / (1.f + __expf(-w_[j])));   // e^-1/2 = 1/sqrt(e)
+                    a_[j] = 1.f / (1.f + __expf(-a_[j]));
+                    kk_[j] = k_[j] * __ldg(kk_p + j);
+                    ss = fmaf(kk_[j], kk_[j], ss);
+                    if (ka_p) k_[j] = fmaf(k_[j] * (a_[j] - 1.f), __ldg(ka_p + j), k_[j]);
+                }
+#pragma unroll
+                for (int o = 1; o < CPT; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                const float inv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+#pragma unroll
+                for (int j = 0; j < EPC; ++j) kk_[j] *= inv;
+            } else {
+                unpack16(raw[1][i], tag, kk_);
+            }
 #pragma unroll
             for (int j = 0; j < EPC; ++j) b_[j] = kk_[j] * a_[j];
             store_vals(&sm.vec[kW][t][e], w_);
@@ -221,15 +245,20 @@ __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const FwdArgs p) {
     }
 }
 
-template <class Tin, int RPT>
+template <class Tin, int RPT, bool RAW>
 cudaError_t launch_seq_t(const FwdArgs &p) {
     const size_t smem = sizeof(SeqSmem<Tin, RPT>);
-    static cudaError_t attr = cudaFuncSetAttribute(seq_kernel<Tin, RPT>,
+    static cudaError_t attr = cudaFuncSetAttribute(seq_kernel<Tin, RPT, RAW>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (attr != cudaSuccess) return attr;
     dim3 grid(p.B * p.H, kN / (16 * RPT));
-    seq_kernel<Tin, RPT><<<grid, kSeqThreads, smem, p.stream>>>(p);
+    seq_kernel<Tin, RPT, RAW><<<grid, kSeqThreads, smem, p.stream>>>(p);
     return cudaGetLastError();
+}
+
+template <class Tin, int RPT>
+cudaError_t launch_seq_r(const FwdArgs &p) {
+    return p.raw ? launch_seq_t<Tin, RPT, true>(p) : launch_seq_t<Tin, RPT, false>(p);
 }
 
 // ---- T = 0: S_T <- S0 (or zeros) -------------------------------------------------------------
@@ -239,7 +268,8 @@ __global__ void copy_state_kernel(const float4 *__restrict__ src, float4 *__rest
 }
 
 // ---- group_norm + bonus epilogue (one warp per (b, t, h) row of 64 channels) ---------------
-template <class Tin>
+// RAW: k is the key before its update and a the rate logit; the bonus uses k~ = k + k (a-1) k_a.
+template <class Tin, bool RAW>
 __global__ void __launch_bounds__(256) epilogue_kernel(const FwdArgs p, size_t rows) {
     const size_t row = blockIdx.x * size_t(8) + (threadIdx.x >> 5);
     if (row >= rows) return;
@@ -248,7 +278,14 @@ __global__ void __launch_bounds__(256) epilogue_kernel(const FwdArgs p, size_t r
     const int pc = h * kN + 2 * lane;
     float2 yv = *reinterpret_cast<const float2 *>(p.y + base);
     const Tin *r = static_cast<const Tin *>(p.r), *k = static_cast<const Tin *>(p.k), *v = static_cast<const Tin *>(p.v);
-    float bon = load1(r + base) * load1(k + base) * p.r_k[pc] + load1(r + base + 1) * load1(k + base + 1) * p.r_k[pc + 1];
+    float k0 = load1(k + base), k1 = load1(k + base + 1);
+    if (RAW && p.k_a) {
+        const Tin *al = static_cast<const Tin *>(p.a);
+        const float a0 = 1.f / (1.f + __expf(-load1(al + base))), a1 = 1.f / (1.f + __expf(-load1(al + base + 1)));
+        k0 = fmaf(k0 * (a0 - 1.f), p.k_a[pc], k0);
+        k1 = fmaf(k1 * (a1 - 1.f), p.k_a[pc + 1], k1);
+    }
+    float bon = load1(r + base) * k0 * p.r_k[pc] + load1(r + base + 1) * k1 * p.r_k[pc + 1];
     float sum = yv.x + yv.y;
 #pragma unroll
     for (int o = 16; o; o >>= 1) {
@@ -272,8 +309,8 @@ __global__ void __launch_bounds__(256) epilogue_kernel(const FwdArgs p, size_t r
 cudaError_t launch_seq(const FwdArgs &p) {
     const bool wide = size_t(p.B) * p.H >= 2 * 148;   // enough (b, h) units: 32 rows per CTA
     if (p.dt == WKV7_BF16)
-        return wide ? launch_seq_t<__nv_bfloat16, 2>(p) : launch_seq_t<__nv_bfloat16, 1>(p);
-    return wide ? launch_seq_t<float, 2>(p) : launch_seq_t<float, 1>(p);
+        return wide ? launch_seq_r<__nv_bfloat16, 2>(p) : launch_seq_r<__nv_bfloat16, 1>(p);
+    return wide ? launch_seq_r<float, 2>(p) : launch_seq_r<float, 1>(p);
 }
 
 cudaError_t launch_copy_state(const FwdArgs &p) {
@@ -287,10 +324,13 @@ cudaError_t launch_copy_state(const FwdArgs &p) {
 cudaError_t launch_epilogue(const FwdArgs &p) {
     const size_t rows = size_t(p.B) * p.T * p.H;
     const unsigned blocks = unsigned((rows + 7) / 8);
-    if (p.dt == WKV7_BF16)
-        epilogue_kernel<__nv_bfloat16><<<blocks, 256, 0, p.stream>>>(p, rows);
-    else
-        epilogue_kernel<float><<<blocks, 256, 0, p.stream>>>(p, rows);
+    if (p.dt == WKV7_BF16) {
+        if (p.raw) epilogue_kernel<__nv_bfloat16, true><<<blocks, 256, 0, p.stream>>>(p, rows);
+        else epilogue_kernel<__nv_bfloat16, false><<<blocks, 256, 0, p.stream>>>(p, rows);
+    } else {
+        if (p.raw) epilogue_kernel<float, true><<<blocks, 256, 0, p.stream>>>(p, rows);
+        else epilogue_kernel<float, false><<<blocks, 256, 0, p.stream>>>(p, rows);
+    }
     return cudaGetLastError();
 }
 

@@ -30,7 +30,7 @@ ALGOS = {"auto": 0, "seq": 1, "chunk": 2, "split": 3}
 
 EXPORTED = ("wkv7_opts_default", "wkv7_forward", "wkv7_decode_step", "wkv7_workspace_bytes",
             "wkv7_status_string", "wkv7_last_error", "wkv7_abi_version", "wkv7_poll_device_error",
-            "wkv7_plan")
+            "wkv7_plan", "wkv7_forward_raw")
 
 
 class Wkv7Error(RuntimeError):
@@ -84,6 +84,9 @@ def load():
         lib.wkv7_plan.argtypes = [ci, ci, ci, ci, ci, ctypes.POINTER(Opts), ctypes.POINTER(ci), ctypes.POINTER(ci),
                                   ctypes.POINTER(ci)]
         lib.wkv7_plan.restype = ci
+        lib.wkv7_forward_raw.argtypes = [ci, ci, ci, ci, ci] + [vp] * 5 + [vp, vp] + [vp, vp, vp, ctypes.POINTER(Opts),
+                                                                               vp, ctypes.c_size_t, vp]
+        lib.wkv7_forward_raw.restype = ci
         if lib.wkv7_abi_version() != ABI_VERSION:
             raise RuntimeError(f"{_LIB_PATH} has ABI version {lib.wkv7_abi_version()}, the binding expects "
                                f"{ABI_VERSION}: rebuild it")
@@ -184,6 +187,35 @@ def forward(r, w, k, v, kk, a, S0=None, *, algo="auto", chunk=0, snap_every=0, l
                               _ptr(S0), _ptr(y), _ptr(S_T), ctypes.byref(opts), _ptr(workspace),
                               ws_bytes, _stream_handle(dev, stream))
     _check(st, "wkv7_forward")
+    return y, S_T, snapshots
+
+
+def forward_raw(r, w_logit, k, v, a_logit, k_k, k_a=None, S0=None, *, algo="auto", chunk=0, snap_every=0,
+                ln_w=None, ln_b=None, r_k=None, gn_eps=64e-5, segments=0, y=None, S_T=None, snapshots=None,
+                workspace=None, return_state=True, stream=None):
+    """WKV-7 forward from the raw time-mixing values (decay and rate logits, the key before its
+    update, the per-head k_k and k_a): the pre-processing runs on the device (see
+    wkv7_forward_raw in include/wkv7.h). Same outputs as ``forward``; device tensors only."""
+    lib = load()
+    B, T, H, N = r.shape
+    dev = r.device
+    if y is None:
+        y = torch.empty((B, T, H, N), device=dev, dtype=torch.float32)
+    if S_T is None and return_state:
+        S_T = torch.empty((B, H, N, N), device=dev, dtype=torch.float32)
+    n_snap = T // snap_every if snap_every else 0
+    if snapshots is None and n_snap:
+        snapshots = torch.empty((B, n_snap, H, N, N), device=dev, dtype=torch.float32)
+    opts = make_opts(algo, chunk, snap_every, snapshots, ln_w, ln_b, r_k, gn_eps, segments)
+    need = int(lib.wkv7_workspace_bytes(B, T, H, N, _dt(r), ctypes.byref(opts)))
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = lib.wkv7_forward_raw(B, T, H, N, _dt(r), _ptr(r), _ptr(w_logit), _ptr(k), _ptr(v), _ptr(a_logit),
+                                  _ptr(k_k), _ptr(k_a), _ptr(S0), _ptr(y), _ptr(S_T), ctypes.byref(opts),
+                                  _ptr(workspace), ws_bytes, _stream_handle(dev, stream))
+    _check(st, "wkv7_forward_raw")
     return y, S_T, snapshots
 
 

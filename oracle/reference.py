@@ -85,8 +85,8 @@ def group_norm_bonus(y, r, k, v, ln_w, ln_b, r_k, eps=64e-5):
 
 def prepare_inputs(w_logit, a_logit, k, k_k, k_a=None):
     """The pre-processing the pages place before the update, in fp64 (the rebuttal page's
-    ``time_mixing`` listing: the decay line, the ``a = sigmoid(...)`` line, ``kk = k * k_k``,
-    ``k += k * (a-1) * k_a`` and ``kk /= max(norm(kk), 1e-12)``).
+    ``time_mixing`` listing: the decay, the in-context learning rate, the removal key formed
+    from the key before its update and normalised with a 1e-12 floor, and the key update).
 
     w_logit, a_logit, k: [B, T, H, N]; k_k, k_a: [H, N] (k_a None = 0).
     Returns (w, a, kk, k_tilde), each [B, T, H, N] fp64:

@@ -157,3 +157,29 @@ def test_plan_counts_launches(lib):
     ln = torch.zeros(4, 64)
     assert wkv7.plan(2, 8, 4, launches=True, ln_w=ln, ln_b=ln, r_k=ln) == ("seq", 0, 2)
     assert wkv7.plan(2, 0, 4, launches=True) == ("seq", 0, 1)
+
+
+def _fwd_raw(lib, ptrs=None, B=1, T=4, H=1, N=64, dt=1):
+    p = ptrs or {}
+    get = lambda n, d=FAKE: ctypes.c_void_p(p.get(n, d)) if p.get(n, d) is not None else None
+    return lib.wkv7_forward_raw(B, T, H, N, dt, *(get(n) for n in ("r", "w_logit", "k", "v", "a_logit", "k_k")),
+                                get("k_a", None), get("S0", None), get("y", FAKE + 0x100000), get("S_T", None),
+                                None, None, 0, None)
+
+
+@pytest.mark.parametrize("ptrs,status,word", [
+    ({"k_k": None}, wkv7.ERR_ARG, b"k_k"),
+    ({"a_logit": None}, wkv7.ERR_ARG, b"a_logit"),
+    ({"w_logit": None}, wkv7.ERR_ARG, b"w_logit"),
+    ({"k_a": FAKE + 0x200004}, wkv7.ERR_ALIGN, b"k_a"),
+    ({"k_k": FAKE + 0x200008}, wkv7.ERR_ALIGN, b"k_k"),
+])
+def test_forward_raw_rejects_bad_arguments(lib, ptrs, status, word):
+    assert _fwd_raw(lib, ptrs) == status
+    assert word in lib.wkv7_last_error()
+
+
+def test_forward_raw_shares_the_size_checks(lib):
+    assert _fwd_raw(lib, N=32) == wkv7.ERR_UNSUPPORTED
+    assert _fwd_raw(lib, B=0) == wkv7.ERR_ARG
+    assert _fwd_raw(lib, {"y": FAKE}) == wkv7.ERR_ARG   # y overlapping r
