@@ -4,22 +4,25 @@ TEST INFRASTRUCTURE ONLY. Nothing in the product path may import this module;
 only tests, the graft smoke check and the benchmark's CPU-baseline leg do.
 
 Sources (RWKV-7 "Goose"):
-* State update and readout: the rebuttal page's numpy ``time_mixing`` listing, the
-  update line ``S = S*w.mT - S@kk*(kk*a).mT + v*k.mT`` and readout ``y = S@r``; the
-  same update in row-vector form in the ARWKV verdict page (``key_machinery``):
+* State update and readout: the rebuttal page's numpy ``time_mixing`` listing (its
+  state-update line and its readout line): S_t = S_{t-1} diag(w_t) - (S_{t-1} kk_t)
+  (kk_t * a_t)^T + v_t k_t^T and y_t = S_t r_t with column vectors; the same update in
+  row-vector form in the ARWKV verdict page (``key_machinery``):
   S_t = S_{t-1}(diag(w_t) - kk_t^T (a_t * kk_t)) + v_t^T k_t.
 * Per-head group_norm (population variance, eps 64e-5 inside the square root, then
   a per-channel affine) and the bonus term sum_j(r_j k_j r_k[j]) * v added after the
   norm: same listing, the ``group_norm`` lambda and the two lines after the readout.
 
 Readings taken where the pages leave a step open (each listed in the design doc):
-* S is N x N with row i = value channel, column j = key channel (the listing's
-  column vectors make ``S*w.mT`` scale columns and ``S@r`` contract the key index).
+* S is N x N with row i = value channel, column j = key channel (with the listing's
+  column vectors the decay multiplies the key columns and the readout contracts the
+  key index).
 * The removal term uses the state *before* this token's update, S_{t-1}: the
   right-hand side is evaluated before assignment, and the row-vector form factors
   S_{t-1} out of both terms.
-* ``S@kk*(kk*a).mT`` is ``(S@kk) * (kk*a)^T``: the outer product of the removed value
-  S_{t-1} kk with kk*a (``@`` and ``*`` share precedence, left to right).
+* The removal term, a matrix product followed by an elementwise product of equal
+  precedence, evaluates left to right: (S kk)(kk*a)^T, the outer product of the removed
+  value S_{t-1} kk with kk*a.
 * The readout uses the updated state S_t (the current token is included).
 * kk arrives already L2-normalised, k is the replacement key, w is the decay
   multiplier itself; nothing is renormalised in the recurrence. ``prepare_inputs``
@@ -68,6 +71,53 @@ def wkv7_recurrence(r, w, k, v, kk, a, S0=None, snap_every=0):
         if n_snap and (t + 1) % snap_every == 0:
             snaps[:, (t + 1) // snap_every - 1] = S
     return y, S, snaps
+
+
+def wkv7_backward(r, w, k, v, kk, a, S0=None, dy=None, dS_T=None):
+    """Gradients of the recurrence, in fp64: reverse-mode differentiation of
+    ``wkv7_recurrence`` for the scalar L = <dy, y> + <dS_T, S_T> (dy, dS_T: the
+    gradients arriving from above; None = 0). The pages time a backward pass and quote its
+    fp32 precision (rebuttal page, the answer on numerical precision; paper summary, the
+    speed figures for the forward that keeps its states and for the backward) but do not
+    print it; this is the chain rule through the update and the readout, one token at a
+    time in reverse, with every state kept from a forward sweep.
+
+    For one token, with b = kk * a, s = S_{t-1} kk and dS the gradient of S_t:
+      y_t = S_t r_t                      -> dS += dy_t r_t^T, dr_t = S_t^T dy_t
+      + v_t k_t^T                        -> dv_t = dS k_t, dk_t = dS^T v_t
+      S_{t-1} diag(w_t)                  -> dw_t[j] = sum_i S_{t-1}[i, j] dS[i, j]
+      - s b^T                            -> db = -dS^T s, ds = -dS b
+      s = S_{t-1} kk, b = kk * a         -> dkk_t = S_{t-1}^T ds + db * a_t, da_t = db * kk_t
+      dS_{t-1} = dS diag(w_t) + ds kk_t^T.
+    Returns dict of dr, dw, dk, dv, dkk, da ([B, T, H, N]) and dS0 ([B, H, N, N]), fp64.
+    """
+    r, w, k, v, kk, a = (_f64(x) for x in (r, w, k, v, kk, a))
+    B, T, H, N = r.shape
+    states = np.empty((T + 1, B, H, N, N))
+    states[0] = 0.0 if S0 is None else _f64(S0)
+    if T:
+        _, _, snaps = wkv7_recurrence(r, w, k, v, kk, a, states[0], snap_every=1)
+        states[1:] = np.moveaxis(snaps, 1, 0)
+    dy = np.zeros((B, T, H, N)) if dy is None else _f64(dy)
+    dS = np.zeros((B, H, N, N)) if dS_T is None else _f64(dS_T).copy()
+    out = {n: np.zeros((B, T, H, N)) for n in ("dr", "dw", "dk", "dv", "dkk", "da")}
+    for t in range(T - 1, -1, -1):
+        S_prev, S_t = states[t], states[t + 1]
+        w_t, k_t, v_t, kk_t, a_t, r_t, dy_t = (x[:, t] for x in (w, k, v, kk, a, r, dy))
+        dS = dS + dy_t[:, :, :, None] * r_t[:, :, None, :]
+        out["dr"][:, t] = np.einsum("bhij,bhi->bhj", S_t, dy_t)
+        out["dv"][:, t] = np.einsum("bhij,bhj->bhi", dS, k_t)
+        out["dk"][:, t] = np.einsum("bhij,bhi->bhj", dS, v_t)
+        out["dw"][:, t] = np.sum(S_prev * dS, axis=-2)
+        b_t = kk_t * a_t
+        s = np.einsum("bhij,bhj->bhi", S_prev, kk_t)
+        db = -np.einsum("bhij,bhi->bhj", dS, s)
+        ds = -np.einsum("bhij,bhj->bhi", dS, b_t)
+        out["dkk"][:, t] = np.einsum("bhij,bhi->bhj", S_prev, ds) + db * a_t
+        out["da"][:, t] = db * kk_t
+        dS = dS * w_t[:, :, None, :] + ds[:, :, :, None] * kk_t[:, :, None, :]
+    out["dS0"] = dS
+    return out
 
 
 def group_norm_bonus(y, r, k, v, ln_w, ln_b, r_k, eps=64e-5):
