@@ -51,6 +51,7 @@ WORKLOADS = {
 # ---- measured DRAM traffic of the dominant kernel (committed ncu summaries under profiles/) -------
 
 KERNEL_SOURCES = {"chunk_kernel": ("chunk.cu", "tc_util.cuh", "common.cuh"),
+                  "bwd_kernel": ("backward.cu", "common.cuh"),
                   "decode_kernel": ("decode.cu", "common.cuh"),
                   "seq_kernel": ("seq.cu", "common.cuh")}
 PROFILE_TAGS = {"prefill-0.19b": "prefill-0.19B", "prefill-1.5b": "prefill-1.5B",
@@ -342,6 +343,138 @@ def run_gpu(args, world, rank, local):
     return out
 
 
+BWD_FLOPS_PER_UNIT = 21 * 64 * 64   # gradient arithmetic per token-head (recomputation not counted)
+
+
+def run_backward(args, world, rank, local):
+    """Backward pass on the prefill workload: one step = wkv7.backward over the batch, with
+    the snapshots (every 64 tokens) of a forward that kept its states, dy and dS_T resident."""
+    from linear_rnn_sequence_rwkv_b200 import wkv7
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    spec = WORKLOADS[args.workload]
+    wl = inputs.WORKLOADS[spec["cid"]]
+    steps = args.steps if args.steps is not None else max(5, spec["default_steps"] // 10)
+    warmup = args.warmup
+    peaks, _ = _peaks()
+    stream = torch.cuda.current_stream(dev)
+    B, T, H, N = wl.B, wl.T, wl.H, wl.N
+    snap = 64
+    seed0 = inputs.SEED_BASE + wl.cid + 1000 * rank + 77
+    set_bytes = B * T * H * N * (6 * 2 + 4) + B * (T // snap) * H * N * N * 4
+    n_sets = max(1, min(4, math.ceil(2 * L2_BYTES / set_bytes)))
+    sets = []
+    for i in range(n_sets):
+        d = inputs.make_inputs(wl, device=str(dev), seed=seed0 + 17 * i)
+        g = torch.Generator(device=dev).manual_seed(seed0 + 17 * i + 1)
+        d["dy"] = torch.randn(B, T, H, N, device=dev, generator=g)
+        d["dS_T"] = 0.1 * torch.randn(B, H, N, N, device=dev, generator=g)
+        _, _, d["snaps"] = wkv7.forward(*(d[n] for n in NAMES), d["S0"], snap_every=snap)
+        sets.append(d)
+    grads = {n: torch.empty(B, T, H, N, device=dev) for n in wkv7.GRAD_NAMES}
+    dS0 = torch.empty(B, H, N, N, device=dev)
+    ws = torch.empty(wkv7.backward_workspace_bytes(B, T, H, N, snap), dtype=torch.uint8, device=dev)
+
+    def step(i):
+        s = sets[i % n_sets]
+        wkv7.backward(*(s[n] for n in NAMES), s["dy"], s["S0"], s["dS_T"], snapshots=s["snaps"],
+                      snap_every=snap, grads=grads, dS0=dS0, workspace=ws)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        ev[0].record(stream)
+        for i in range(steps):
+            step(warmup + i)
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    per_step_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[steps]), world, dev)
+    units = B * T * H
+    value = units * steps * world / (total_ms * 1e-3) / 1e6
+    launch_ms = statistics.mean(per_step_ms)
+    sm_max = float(peaks.get("sm_max_mhz", 1965.0))
+    fp32_peak = 148 * 128 * 2 * sm_max * 1e6 / 1e12
+    achieved = BWD_FLOPS_PER_UNIT * units / (launch_ms * 1e-3) / 1e12
+    hbm_bytes = units * (6 * N * 2 + N * 4 + 6 * N * 4) + B * H * N * N * 4 * (3 + T // snap)
+    roof = {"bound": "alu", "achieved": round(achieved, 3), "peak": round(fp32_peak, 2), "unit": "TFLOP/s",
+            "frac": round(achieved / fp32_peak, 4),
+            "peak_source": f"148 SMs x 128 FP32 lanes x 2 flop x {sm_max:.0f} MHz (derived)",
+            "traffic": measured_traffic("bwd_kernel", args.workload), "kernel": "bwd_kernel",
+            "flops_per_unit": BWD_FLOPS_PER_UNIT, "algorithmic_bytes_per_launch": hbm_bytes,
+            "hbm_gbs": round(hbm_bytes / (launch_ms * 1e-3) / 1e9, 1),
+            "hbm_frac": round(hbm_bytes / (launch_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]), 4)}
+
+    # end to end: host inputs (pinned) -> device, backward, gradients -> host, all timed
+    hd = {n: (v.to("cpu").pin_memory() if isinstance(v, torch.Tensor) else v) for n, v in sets[0].items()}
+    host_out = {n: torch.empty(B, T, H, N).pin_memory() for n in wkv7.GRAD_NAMES}
+    host_ds0 = torch.empty(B, H, N, N).pin_memory()
+    in_names = NAMES + ("S0", "dy", "dS_T", "snaps")
+    h2d = sum(hd[n].numel() * hd[n].element_size() for n in in_names if hd[n] is not None)
+    d2h = sum(t.numel() * 4 for t in host_out.values()) + host_ds0.numel() * 4
+
+    def once():
+        dv = {n: (None if hd[n] is None else hd[n].to(dev, non_blocking=True)) for n in in_names}
+        out = wkv7.backward(*(dv[n] for n in NAMES), dv["dy"], dv["S0"], dv["dS_T"], snapshots=dv["snaps"],
+                            snap_every=snap, workspace=ws)
+        for n in wkv7.GRAD_NAMES:
+            host_out[n].copy_(out[n], non_blocking=True)
+        host_ds0.copy_(out["dS0"], non_blocking=True)
+
+    once()
+    torch.cuda.synchronize(dev)
+    e_steps = max(1, min(steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record(stream)
+    for _ in range(e_steps):
+        once()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e = {"value": round(units * e_steps * world / (e_ms * 1e-3) / 1e6, 3), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
+           "ms_per_step": round(e_ms / e_steps, 4)}
+    out = {
+        "metric": METRIC.replace("(prefill, decode)", "(backward)"), "value": round(value, 3), "unit": UNIT,
+        "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": round(total_ms / steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded torch Philox; shapes and value ranges of the RWKV-7 pages' workloads)",
+        "config": {"workload": f"{args.workload} backward: {wl.name}", "B": B, "T": T, "H": H, "N": N,
+                   "input_dtype": "bf16", "path": "backward", "snap_every": snap,
+                   "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world} (independent (b,h) units)",
+                   "l2": f"{n_sets} rotating input sets, {n_sets * set_bytes / 1e6:.0f} MB"},
+        "roofline": roof, "e2e": e2e, "gpu_launches": steps, "clocks": clocks.summary(),
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_backward(wl)
+    return out
+
+
+def cpu_baseline_backward(wl, budget_s: float = 12.0):
+    """The fp64 oracle's backward (numpy, vectorised over (b, h)) on a bounded sample."""
+    from oracle import reference
+    B, T, H = 1, min(wl.T, 1024), wl.H
+    d = inputs.make_inputs(wl, B=B, T=T, H=H)
+    g = torch.Generator().manual_seed(5)
+    dy = torch.randn(B, T, H, wl.N, generator=g)
+    dS_T = 0.1 * torch.randn(B, H, wl.N, wl.N, generator=g)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        reference.wkv7_backward(*(d[n] for n in NAMES), d["S0"], dy, dS_T)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el > budget_s / 4 or reps >= 50:
+            break
+    return {"value": round(B * T * H * reps / el / 1e6, 5), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"B{B} T{T} H{H} of the workload (numpy fp64 backward); {reps} run(s), {el:.1f} s wall"}
+
+
 def _path_name(args):
     """Kernel the library dispatches to for the bf16 workloads (AUTO picks the chunked one)."""
     return {"auto": "chunk", "seq": "seq", "chunk": "chunk", "split": "chunk"}[args.algo]
@@ -467,6 +600,8 @@ def main(argv=None):
     ap.add_argument("--algo", choices=["auto", "seq", "chunk", "split"], default="auto")
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="pass_", choices=["forward", "backward"], default="forward",
+                    help="backward: gradients of every input from a forward's snapshots")
     ap.add_argument("--inputs", choices=["prepared", "raw"], default="prepared",
                     help="raw: decay/rate logits and the key before its update, pre-processing fused")
     args = ap.parse_args(argv)
@@ -485,7 +620,12 @@ def main(argv=None):
     if world != args.gpus and rank == 0:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
     try:
-        out = run_gpu(args, world, rank, local)
+        if args.pass_ == "backward":
+            if args.workload == "decode" or args.inputs == "raw":
+                raise SystemExit("--pass backward takes a prefill workload with prepared inputs")
+            out = run_backward(args, world, rank, local)
+        else:
+            out = run_gpu(args, world, rank, local)
         if rank == 0:
             print(json.dumps(out))
     finally:

@@ -151,6 +151,49 @@ WKV7_API wkv7_status wkv7_forward_raw(int B, int T, int H, int N, wkv7_dtype dt,
                              void *stream);
 
 /*
+ * Backward pass of wkv7_forward (no epilogue): the gradients of every input for the scalar
+ * L = <dy, y> + <dS_T, S_T>, in fp32. The pages time a backward pass and state the precision
+ * of an fp32 one (RWKV-7 rebuttal page, the answer on numerical precision; paper summary,
+ * the speed figures for the forward that keeps its states and for the backward); the
+ * operation is the chain rule through the update and readout of the rebuttal page's numpy
+ * time_mixing listing, token by token in reverse:
+ *     dS += dy_t r_t^T, dr_t = S_t^T dy_t, dv_t = dS k_t, dk_t = dS^T v_t,
+ *     dw_t = column sums of S_{t-1} (.) dS, db = -dS^T (S_{t-1} kk_t), ds = -dS (kk_t a_t),
+ *     dkk_t = S_{t-1}^T ds + db (.) a_t, da_t = db (.) kk_t, dS_{t-1} = dS diag(w_t) + ds kk_t^T.
+ * The states S_{t-1} are recomputed on the device, starting from S0 and from the forward's
+ * snapshots when given: pass the snapshots a wkv7_forward call wrote with
+ * the same snap_every (the states after tokens snap_every, 2 snap_every, ...) to bound the
+ * recomputation and the workspace; snap_every = 0 recomputes from S0 alone.
+ *
+ * Inputs  r, w, k, v, kk, a : [B][T][H][N] of dtype dt, the forward's inputs.
+ *         S0                : [B][H][N][N] fp32 or NULL (zeros).
+ *         snapshots         : [B][T/snap_every][H][N][N] fp32; required when snap_every > 0
+ *                             and T >= snap_every, else ignored.
+ *         dy                : [B][T][H][N] fp32 gradient of y (required when T > 0).
+ *         dS_T              : [B][H][N][N] fp32 or NULL (zero gradient on the final state).
+ * Outputs dr, dw, dk, dv, dkk, da : [B][T][H][N] fp32 (required when T > 0).
+ *         dS0               : [B][H][N][N] fp32 or NULL; may equal dS_T exactly (in place).
+ * Workspace: at least wkv7_backward_workspace_bytes(B, T, H, N, snap_every) bytes of device
+ * memory (the recomputation's checkpoints, one state per 4 tokens of a segment); it must not
+ * overlap any other argument and its contents need no initialisation.
+ * Errors as wkv7_forward: WKV7_ERR_ARG for sizes, NULL required pointers, snap_every < 0,
+ * missing snapshots, overlapping outputs, host or too-small buffers; WKV7_ERR_ALIGN;
+ * WKV7_ERR_UNSUPPORTED for N != 64; WKV7_ERR_WORKSPACE. T = 0 copies dS_T (or zeros) to dS0.
+ */
+WKV7_API wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype dt,
+                          const void *r, const void *w, const void *k, const void *v,
+                          const void *kk, const void *a, const float *S0,
+                          const float *snapshots, int snap_every,
+                          const float *dy, const float *dS_T,
+                          float *dr, float *dw, float *dk, float *dv, float *dkk, float *da,
+                          float *dS0, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace wkv7_backward needs: B * H * ceil(K / 4) * N * N * 4 with K the
+ * snapshot interval (or T when snap_every is 0 or >= T); 0 when T = 0 or an argument is
+ * invalid. Host only. */
+WKV7_API size_t wkv7_backward_workspace_bytes(int B, int T, int H, int N, int snap_every);
+
+/*
  * One decode step for every (b, h): the recurrence for a single token, with the
  * state read and written in place.
  *

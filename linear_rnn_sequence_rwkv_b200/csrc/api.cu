@@ -387,4 +387,88 @@ wkv7_status wkv7_decode_step(int B, int H, int N, wkv7_dtype dt, const void *r, 
     return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "decode launch");
 }
 
+size_t wkv7_backward_workspace_bytes(int B, int T, int H, int N, int snap_every) {
+    if (B <= 0 || T <= 0 || H <= 0 || N != wkv7::kN || snap_every < 0) return 0;
+    size_t n = 1;
+    if (!mul_ok(n, B) || !mul_ok(n, H) || !mul_ok(n, T)) return 0;
+    return wkv7::backward_checkpoint_bytes(B, T, H, snap_every);
+}
+
+wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype dt, const void *r, const void *w,
+                          const void *k, const void *v, const void *kk, const void *a, const float *S0,
+                          const float *snapshots, int snap_every, const float *dy, const float *dS_T,
+                          float *dr, float *dw, float *dk, float *dv, float *dkk, float *da, float *dS0,
+                          void *workspace, size_t workspace_bytes, void *stream) {
+    g_err[0] = '\0';
+    if (N <= 0 || B <= 0 || H <= 0 || T < 0)
+        return fail(WKV7_ERR_ARG, "bad sizes B=%d T=%d H=%d N=%d (need B,H,N >= 1, T >= 0)", B, T, H, N);
+    if (N != wkv7::kN) return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: only N=64 is implemented", N);
+    if (dt != WKV7_F32 && dt != WKV7_BF16) return fail(WKV7_ERR_ARG, "unknown dtype %d", (int)dt);
+    if (snap_every < 0) return fail(WKV7_ERR_ARG, "snap_every=%d < 0", snap_every);
+    const int n_snap = snap_every > 0 ? T / snap_every : 0;
+    if (n_snap > 0 && !snapshots) return fail(WKV7_ERR_ARG, "snap_every=%d but snapshots is NULL", snap_every);
+    size_t tok = 1, st = 1;
+    if (!mul_ok(tok, B) || !mul_ok(tok, T) || !mul_ok(tok, H) || !mul_ok(tok, N) || !mul_ok(st, B) ||
+        !mul_ok(st, H) || !mul_ok(st, N) || !mul_ok(st, N) || tok > (size_t(1) << 40))
+        return fail(WKV7_ERR_ARG, "sizes overflow");
+    const size_t in_bytes = T ? tok * elem_bytes(dt) : 0, g_bytes = T ? tok * 4 : 0, st_bytes = st * 4;
+    if (T > 0) {
+        const void *req[] = {r, w, k, v, kk, a, dy, dr, dw, dk, dv, dkk, da};
+        const char *names[] = {"r", "w", "k", "v", "kk", "a", "dy", "dr", "dw", "dk", "dv", "dkk", "da"};
+        for (int i = 0; i < 13; ++i)
+            if (!req[i]) return fail(WKV7_ERR_ARG, "%s is NULL", names[i]);
+    }
+    // inputs 0-9, outputs 10-16, workspace 17
+    const Buf bufs[] = {{"r", r, in_bytes},   {"w", w, in_bytes},   {"k", k, in_bytes},
+                        {"v", v, in_bytes},   {"kk", kk, in_bytes}, {"a", a, in_bytes},
+                        {"S0", S0, st_bytes}, {"snapshots", n_snap ? snapshots : nullptr, st_bytes * n_snap},
+                        {"dy", dy, g_bytes},  {"dS_T", dS_T, st_bytes},
+                        {"dr", dr, g_bytes},  {"dw", dw, g_bytes},  {"dk", dk, g_bytes},
+                        {"dv", dv, g_bytes},  {"dkk", dkk, g_bytes}, {"da", da, g_bytes},
+                        {"dS0", dS0, st_bytes}, {"workspace", workspace, workspace_bytes}};
+    constexpr int nb = sizeof(bufs) / sizeof(bufs[0]);
+    for (int i = 0; i < nb; ++i)
+        if (bufs[i].ptr && !aligned16(bufs[i].ptr))
+            return fail(WKV7_ERR_ALIGN, "%s is not 16-byte aligned", bufs[i].name);
+    const size_t need_ws = wkv7_backward_workspace_bytes(B, T, H, N, snap_every);
+    if (need_ws > 0 && (!workspace || workspace_bytes < need_ws))
+        return fail(WKV7_ERR_WORKSPACE, "workspace of %zu bytes required, %zu given", need_ws,
+                    workspace ? workspace_bytes : 0);
+    const Buf ws_used{"workspace", workspace, need_ws};
+    for (int o = 10; o < nb; ++o) {   // outputs (and the workspace) overlap nothing else
+        const Buf &ob = o == nb - 1 ? ws_used : bufs[o];
+        for (int i = 0; i < nb - 1; ++i)
+            if (i != o && overlaps(ob, bufs[i]) && !(o == 16 && i == 9 && dS0 == dS_T))   // dS0 = dS_T in place
+                return fail(WKV7_ERR_ARG, "%s overlaps %s", ob.name, bufs[i].name);
+    }
+    int device = 0;
+    cudaError_t e = cudaGetDevice(&device);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return cuda_fail(e, "cudaGetDevice");
+    }
+    for (int i = 0; i < nb; ++i) {
+        const wkv7_status s = check_device_buffer(i == nb - 1 ? ws_used : bufs[i], device);
+        if (s != WKV7_OK) return s;
+    }
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (T == 0) {   // dS0 <- dS_T (or zeros)
+        if (!dS0) return WKV7_OK;
+        wkv7::FwdArgs c{};
+        c.B = B; c.H = H; c.S0 = dS_T; c.S_T = dS0; c.stream = cs;
+        e = wkv7::launch_copy_state(c);
+        return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "state-gradient copy launch");
+    }
+    wkv7::BwdArgs p{};
+    p.B = B; p.T = T; p.H = H; p.dt = dt;
+    p.r = r; p.w = w; p.k = k; p.v = v; p.kk = kk; p.a = a;
+    p.S0 = S0; p.snaps = n_snap ? snapshots : nullptr; p.snap_every = n_snap ? snap_every : 0;
+    p.dy = dy; p.dS_T = dS_T;
+    p.dr = dr; p.dw = dw; p.dk = dk; p.dv = dv; p.dkk = dkk; p.da = da; p.dS0 = dS0;
+    p.ws = static_cast<float *>(workspace);
+    p.stream = cs;
+    e = wkv7::launch_backward(p);
+    return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "backward launch");
+}
+
 }  // extern "C"

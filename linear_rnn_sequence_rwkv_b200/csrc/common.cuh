@@ -41,11 +41,29 @@ struct DecArgs {
     cudaStream_t stream;
 };
 
+// Arguments of one backward call after validation.
+struct BwdArgs {
+    int B, T, H;
+    wkv7_dtype dt;
+    const void *r, *w, *k, *v, *kk, *a;
+    const float *S0;        // nullable: zero initial state
+    const float *snaps;     // the forward's states every snap_every tokens, or null (snap_every 0)
+    int snap_every;
+    const float *dy;        // [B][T][H][N] gradient of y
+    const float *dS_T;      // nullable: no gradient on the final state
+    float *dr, *dw, *dk, *dv, *dkk, *da;   // [B][T][H][N]
+    float *dS0;             // nullable
+    float *ws;              // backward_checkpoint_bytes(...) of scratch
+    cudaStream_t stream;
+};
+
 // Launchers (each returns the launch status; no synchronisation).
 cudaError_t launch_seq(const FwdArgs &p);
 cudaError_t launch_epilogue(const FwdArgs &p);
 cudaError_t launch_decode(const DecArgs &p);
 cudaError_t launch_copy_state(const FwdArgs &p);   // T == 0: S_T <- S0 (or zeros)
+cudaError_t launch_backward(const BwdArgs &p);     // T >= 1
+size_t backward_checkpoint_bytes(int B, int T, int H, int snap_every);
 bool chunk_supported(const FwdArgs &p);            // bf16 inputs, snapshots on chunk boundaries
 cudaError_t launch_chunk(const FwdArgs &p);        // chunked prefill on tcgen05 (epilogue fused)
 // CTAs per (b, h) of launch_chunk's last launch, and its number of launches (1 or 2)

@@ -30,7 +30,7 @@ ALGOS = {"auto": 0, "seq": 1, "chunk": 2, "split": 3}
 
 EXPORTED = ("wkv7_opts_default", "wkv7_forward", "wkv7_decode_step", "wkv7_workspace_bytes",
             "wkv7_status_string", "wkv7_last_error", "wkv7_abi_version", "wkv7_poll_device_error",
-            "wkv7_plan", "wkv7_forward_raw")
+            "wkv7_plan", "wkv7_forward_raw", "wkv7_backward", "wkv7_backward_workspace_bytes")
 
 
 class Wkv7Error(RuntimeError):
@@ -71,6 +71,11 @@ def load():
         lib.wkv7_forward.restype = ci
         lib.wkv7_decode_step.argtypes = [ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp]
         lib.wkv7_decode_step.restype = ci
+        lib.wkv7_backward.argtypes = [ci, ci, ci, ci, ci] + [vp] * 6 + [vp, vp, ci, vp, vp] + [vp] * 7 + [
+            vp, ctypes.c_size_t, vp]
+        lib.wkv7_backward.restype = ci
+        lib.wkv7_backward_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
+        lib.wkv7_backward_workspace_bytes.restype = ctypes.c_size_t
         lib.wkv7_workspace_bytes.argtypes = [ci, ci, ci, ci, ci, ctypes.POINTER(Opts)]
         lib.wkv7_workspace_bytes.restype = ctypes.c_size_t
         lib.wkv7_status_string.argtypes = [ci]
@@ -217,6 +222,41 @@ def forward_raw(r, w_logit, k, v, a_logit, k_k, k_a=None, S0=None, *, algo="auto
                                   _ptr(workspace), ws_bytes, _stream_handle(dev, stream))
     _check(st, "wkv7_forward_raw")
     return y, S_T, snapshots
+
+
+GRAD_NAMES = ("dr", "dw", "dk", "dv", "dkk", "da")
+
+
+def backward_workspace_bytes(B, T, H, N=HEAD_SIZE, snap_every=0) -> int:
+    return int(load().wkv7_backward_workspace_bytes(B, T, H, N, snap_every))
+
+
+def backward(r, w, k, v, kk, a, dy, S0=None, dS_T=None, *, snapshots=None, snap_every=0, grads=None,
+             dS0=None, return_state_grad=True, workspace=None, stream=None):
+    """Gradients of <dy, y> + <dS_T, S_T> with respect to the forward's inputs (see
+    wkv7_backward in include/wkv7.h). ``snapshots``/``snap_every``: the states a forward with
+    the same ``snap_every`` wrote, bounding the recomputation. Device tensors only. Returns a
+    dict of dr, dw, dk, dv, dkk, da ([B, T, H, 64] fp32) and dS0 ([B, H, 64, 64] or None)."""
+    lib = load()
+    B, T, H, N = r.shape
+    dev = r.device
+    if grads is None:
+        grads = {n: torch.empty((B, T, H, N), device=dev, dtype=torch.float32) for n in GRAD_NAMES}
+    if dS0 is None and return_state_grad:
+        dS0 = torch.empty((B, H, N, N), device=dev, dtype=torch.float32)
+    need = int(lib.wkv7_backward_workspace_bytes(B, T, H, N, snap_every))
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = lib.wkv7_backward(B, T, H, N, _dt(r), _ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(kk), _ptr(a),
+                               _ptr(S0), _ptr(snapshots), int(snap_every), _ptr(dy), _ptr(dS_T),
+                               *(_ptr(grads[n]) for n in GRAD_NAMES), _ptr(dS0), _ptr(workspace), ws_bytes,
+                               _stream_handle(dev, stream))
+    _check(st, "wkv7_backward")
+    out = dict(grads)
+    out["dS0"] = dS0
+    return out
 
 
 def decode_step(r, w, k, v, kk, a, S, *, y=None, stream=None):

@@ -183,3 +183,51 @@ def test_forward_raw_shares_the_size_checks(lib):
     assert _fwd_raw(lib, N=32) == wkv7.ERR_UNSUPPORTED
     assert _fwd_raw(lib, B=0) == wkv7.ERR_ARG
     assert _fwd_raw(lib, {"y": FAKE}) == wkv7.ERR_ARG   # y overlapping r
+
+
+def _bwd(lib, ptrs=None, B=1, T=4, H=1, N=64, dt=1, snap_every=0, ws=None, ws_bytes=0):
+    p = ptrs or {}
+    names_in = ("r", "w", "k", "v", "kk", "a")
+    names_out = ("dr", "dw", "dk", "dv", "dkk", "da")
+    base = {n: FAKE + 0x100000 * (i + 1) for i, n in enumerate(names_in + ("dy",) + names_out)}
+    get = lambda n: (ctypes.c_void_p(p.get(n, base.get(n))) if p.get(n, base.get(n)) is not None else None)
+    return lib.wkv7_backward(B, T, H, N, dt, *(get(n) for n in names_in), get("S0"), get("snapshots"),
+                             snap_every, get("dy"), get("dS_T"), *(get(n) for n in names_out), get("dS0"),
+                             ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status,word", [
+    (dict(N=32), wkv7.ERR_UNSUPPORTED, b"N=32"),
+    (dict(T=-1), wkv7.ERR_ARG, b"bad sizes"),
+    (dict(dt=5), wkv7.ERR_ARG, b"dtype"),
+    (dict(snap_every=-1), wkv7.ERR_ARG, b"snap_every"),
+    (dict(snap_every=2), wkv7.ERR_ARG, b"snapshots"),
+    (dict(ptrs={"dy": None}), wkv7.ERR_ARG, b"dy"),
+    (dict(ptrs={"dkk": None}), wkv7.ERR_ARG, b"dkk"),
+    (dict(ptrs={"kk": None}), wkv7.ERR_ARG, b"kk"),
+    (dict(ptrs={"dr": FAKE + 0x100000 * 8 + 4}), wkv7.ERR_ALIGN, b"dr"),
+    (dict(ptrs={"dS0": FAKE + 0x40000004}), wkv7.ERR_ALIGN, b"dS0"),
+])
+def test_backward_rejects_bad_arguments(lib, kw, status, word):
+    assert _bwd(lib, **kw) == status
+    assert word in lib.wkv7_last_error()
+
+
+def test_backward_rejects_overlaps_and_small_workspace(lib):
+    need = wkv7.backward_workspace_bytes(1, 4, 1)
+    ws = ctypes.c_void_p(FAKE + 0x10000000)
+    assert _bwd(lib, {"dw": FAKE + 0x100000 * 8}, ws=ws, ws_bytes=need) == wkv7.ERR_ARG   # dw on top of dr
+    assert b"overlaps" in lib.wkv7_last_error()
+    assert _bwd(lib, {"dr": FAKE + 0x100000}, ws=ws, ws_bytes=need) == wkv7.ERR_ARG       # dr on top of r
+    assert _bwd(lib, ws=ctypes.c_void_p(FAKE + 0x100000 * 9), ws_bytes=need) == wkv7.ERR_ARG   # ws on dw
+    assert need == 64 * 64 * 4                                              # one checkpoint per 4 tokens
+    assert _bwd(lib, ws=ctypes.c_void_p(FAKE + 0x10000000), ws_bytes=need - 16) == wkv7.ERR_WORKSPACE
+    assert _bwd(lib, ws=None, ws_bytes=0) == wkv7.ERR_WORKSPACE
+
+
+def test_backward_workspace_query():
+    assert wkv7.backward_workspace_bytes(2, 0, 3) == 0
+    assert wkv7.backward_workspace_bytes(2, 10, 3) == 2 * 3 * 3 * 16384           # ceil(10 / 4) states
+    assert wkv7.backward_workspace_bytes(2, 100, 3, snap_every=16) == 2 * 3 * 4 * 16384
+    assert wkv7.backward_workspace_bytes(2, 100, 3, snap_every=200) == 2 * 3 * 25 * 16384
+    assert wkv7.backward_workspace_bytes(2, 100, 3, N=32) == 0
