@@ -194,6 +194,28 @@ WKV7_API wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype dt,
 WKV7_API size_t wkv7_backward_workspace_bytes(int B, int T, int H, int N, int snap_every);
 
 /*
+ * wkv7_backward without a workspace argument and without any allocation: the checkpoints go
+ * to a scratch array of 32 MiB (33,554,432 bytes) that the library's device code holds at
+ * module scope; its address is looked up once per device. This entry has no counterpart on
+ * the pages; it serves callers that cannot provide device memory.
+ * Limit: wkv7_backward_workspace_bytes(B, T, H, N, snap_every) must be at most 32 MiB
+ * (2048 checkpoints: B * H * ceil(K / 4) <= 2048, K the snapshot interval, or T without
+ * snapshots); larger requests return WKV7_ERR_WORKSPACE before anything is enqueued.
+ * Nothing in the scratch needs to start at zero (every checkpoint is written before it is read).
+ * The scratch is shared by every call on a device: calls that may overlap in time (different
+ * streams, or host threads without ordering between them) race on it and corrupt each other's
+ * results; order such calls on one stream. Arguments, outputs and errors otherwise as
+ * wkv7_backward.
+ */
+WKV7_API wkv7_status wkv7_backward_static(int B, int T, int H, int N, wkv7_dtype dt,
+                          const void *r, const void *w, const void *k, const void *v,
+                          const void *kk, const void *a, const float *S0,
+                          const float *snapshots, int snap_every,
+                          const float *dy, const float *dS_T,
+                          float *dr, float *dw, float *dk, float *dv, float *dkk, float *da,
+                          float *dS0, void *stream);
+
+/*
  * One decode step for every (b, h): the recurrence for a single token, with the
  * state read and written in place.
  *

@@ -387,6 +387,29 @@ wkv7_status wkv7_decode_step(int B, int H, int N, wkv7_dtype dt, const void *r, 
     return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "decode launch");
 }
 
+wkv7_status wkv7_backward_static(int B, int T, int H, int N, wkv7_dtype dt, const void *r, const void *w,
+                                 const void *k, const void *v, const void *kk, const void *a, const float *S0,
+                                 const float *snapshots, int snap_every, const float *dy, const float *dS_T,
+                                 float *dr, float *dw, float *dk, float *dv, float *dkk, float *da, float *dS0,
+                                 void *stream) {
+    g_err[0] = '\0';
+    const size_t need = wkv7_backward_workspace_bytes(B, T, H, N, snap_every);
+    const size_t cap = wkv7::backward_static_scratch_bytes();
+    if (need > cap)
+        return fail(WKV7_ERR_WORKSPACE, "needs %zu bytes of scratch; the static scratch holds %zu (use wkv7_backward)",
+                    need, cap);
+    void *scratch = nullptr;
+    if (need > 0) {
+        const cudaError_t e = wkv7::backward_static_scratch(&scratch);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return cuda_fail(e, "static scratch address");
+        }
+    }
+    return wkv7_backward(B, T, H, N, dt, r, w, k, v, kk, a, S0, snapshots, snap_every, dy, dS_T, dr, dw, dk, dv,
+                         dkk, da, dS0, scratch, need ? cap : 0, stream);
+}
+
 size_t wkv7_backward_workspace_bytes(int B, int T, int H, int N, int snap_every) {
     if (B <= 0 || T <= 0 || H <= 0 || N != wkv7::kN || snap_every < 0) return 0;
     size_t n = 1;

@@ -27,10 +27,18 @@
 //                two shuffles.
 // Shared rows are 80 floats apart (320 B = 64 mod 128), so the row owners' float4 stores
 // and the column pass's float4 loads are both free of bank conflicts.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace wkv7 {
 namespace {
+
+// Scratch of the allocation-free backward entry: the recomputation checkpoints live in this
+// module-scope array instead of a caller's workspace. Every checkpoint is written before it is
+// read, so nothing in it needs to start at zero.
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;   // 2048 states of 64 x 64 fp32
+static __device__ __align__(256) float g_bwd_scratch[kStaticScratchBytes / sizeof(float)];
 
 constexpr int kBwdThreads = 256;
 constexpr int kLb = 4;          // tokens per block
@@ -297,6 +305,23 @@ size_t backward_checkpoint_bytes(int B, int T, int H, int snap_every) {
     if (T <= 0) return 0;
     const int K = segment_length(T, snap_every);
     return size_t(B) * H * size_t((K + kLb - 1) / kLb) * kN * kN * sizeof(float);
+}
+
+size_t backward_static_scratch_bytes() { return kStaticScratchBytes; }
+
+// Device address of the static scratch on the current device, looked up once per device.
+cudaError_t backward_static_scratch(void **ptr) {
+    constexpr int kMaxDevices = 64;
+    static std::once_flag once[kMaxDevices];
+    static void *addr[kMaxDevices];
+    static cudaError_t err[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::call_once(once[dev], [dev] { err[dev] = cudaGetSymbolAddress(&addr[dev], g_bwd_scratch); });
+    *ptr = addr[dev];
+    return err[dev];
 }
 
 cudaError_t launch_backward(const BwdArgs &p) {

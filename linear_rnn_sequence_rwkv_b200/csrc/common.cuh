@@ -64,6 +64,8 @@ cudaError_t launch_decode(const DecArgs &p);
 cudaError_t launch_copy_state(const FwdArgs &p);   // T == 0: S_T <- S0 (or zeros)
 cudaError_t launch_backward(const BwdArgs &p);     // T >= 1
 size_t backward_checkpoint_bytes(int B, int T, int H, int snap_every);
+size_t backward_static_scratch_bytes();             // capacity of the module's static scratch
+cudaError_t backward_static_scratch(void **ptr);    // its address on the current device
 bool chunk_supported(const FwdArgs &p);            // bf16 inputs, snapshots on chunk boundaries
 cudaError_t launch_chunk(const FwdArgs &p);        // chunked prefill on tcgen05 (epilogue fused)
 // CTAs per (b, h) of launch_chunk's last launch, and its number of launches (1 or 2)

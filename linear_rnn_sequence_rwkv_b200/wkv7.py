@@ -30,7 +30,8 @@ ALGOS = {"auto": 0, "seq": 1, "chunk": 2, "split": 3}
 
 EXPORTED = ("wkv7_opts_default", "wkv7_forward", "wkv7_decode_step", "wkv7_workspace_bytes",
             "wkv7_status_string", "wkv7_last_error", "wkv7_abi_version", "wkv7_poll_device_error",
-            "wkv7_plan", "wkv7_forward_raw", "wkv7_backward", "wkv7_backward_workspace_bytes")
+            "wkv7_plan", "wkv7_forward_raw", "wkv7_backward", "wkv7_backward_workspace_bytes",
+            "wkv7_backward_static")
 
 
 class Wkv7Error(RuntimeError):
@@ -74,6 +75,8 @@ def load():
         lib.wkv7_backward.argtypes = [ci, ci, ci, ci, ci] + [vp] * 6 + [vp, vp, ci, vp, vp] + [vp] * 7 + [
             vp, ctypes.c_size_t, vp]
         lib.wkv7_backward.restype = ci
+        lib.wkv7_backward_static.argtypes = [ci, ci, ci, ci, ci] + [vp] * 6 + [vp, vp, ci, vp, vp] + [vp] * 7 + [vp]
+        lib.wkv7_backward_static.restype = ci
         lib.wkv7_backward_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
         lib.wkv7_backward_workspace_bytes.restype = ctypes.c_size_t
         lib.wkv7_workspace_bytes.argtypes = [ci, ci, ci, ci, ci, ctypes.POINTER(Opts)]
@@ -254,6 +257,30 @@ def backward(r, w, k, v, kk, a, dy, S0=None, dS_T=None, *, snapshots=None, snap_
                                *(_ptr(grads[n]) for n in GRAD_NAMES), _ptr(dS0), _ptr(workspace), ws_bytes,
                                _stream_handle(dev, stream))
     _check(st, "wkv7_backward")
+    out = dict(grads)
+    out["dS0"] = dS0
+    return out
+
+
+STATIC_SCRATCH_BYTES = 32 << 20   # capacity of the library's static backward scratch
+
+
+def backward_static(r, w, k, v, kk, a, dy, S0=None, dS_T=None, *, snapshots=None, snap_every=0, grads=None,
+                    dS0=None, return_state_grad=True, stream=None):
+    """``backward`` through the allocation-free entry (wkv7_backward_static): the library's
+    static scratch replaces the workspace; calls on one device must not overlap in time."""
+    lib = load()
+    B, T, H, N = r.shape
+    dev = r.device
+    if grads is None:
+        grads = {n: torch.empty((B, T, H, N), device=dev, dtype=torch.float32) for n in GRAD_NAMES}
+    if dS0 is None and return_state_grad:
+        dS0 = torch.empty((B, H, N, N), device=dev, dtype=torch.float32)
+    with torch.cuda.device(dev):
+        st = lib.wkv7_backward_static(B, T, H, N, _dt(r), _ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(kk), _ptr(a),
+                                      _ptr(S0), _ptr(snapshots), int(snap_every), _ptr(dy), _ptr(dS_T),
+                                      *(_ptr(grads[n]) for n in GRAD_NAMES), _ptr(dS0), _stream_handle(dev, stream))
+    _check(st, "wkv7_backward_static")
     out = dict(grads)
     out["dS0"] = dS0
     return out
