@@ -17,6 +17,7 @@ max over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -207,6 +208,9 @@ def run_gpu(args, world, rank, local):
     torch.cuda.set_device(dev)
     spec = WORKLOADS[args.workload]
     wl = inputs.WORKLOADS[spec["cid"]]
+    if args.head_size != wl.N:   # same channel count per token, wider heads
+        wl = dataclasses.replace(wl, N=args.head_size, H=max(1, wl.H * wl.N // args.head_size),
+                                 name=f"{wl.name} as N={args.head_size}")
     steps = args.steps if args.steps is not None else spec["default_steps"]
     warmup = args.warmup
     peaks, peak_kind = _peaks()
@@ -268,8 +272,8 @@ def run_gpu(args, world, rank, local):
     ctas_per_head = None
     if not decode:
         ep = dict(ln_w=sets[0]["ln_w"], ln_b=sets[0]["ln_b"], r_k=sets[0]["r_k"]) if epilogue else {}
-        _, ctas_per_head, launches_per_step = wkv7.plan(B, T, H, N, torch.bfloat16, launches=True, algo=args.algo,
-                                                        chunk=args.chunk, snap_every=snap_every, **ep)
+        plan_algo, ctas_per_head, launches_per_step = wkv7.plan(
+            B, T, H, N, torch.bfloat16, launches=True, algo=args.algo, chunk=args.chunk, snap_every=snap_every, **ep)
 
     for i in range(warmup):
         step(i)
@@ -295,8 +299,9 @@ def run_gpu(args, world, rank, local):
     # roofline of the dominant kernel
     hbm_peak = float(peaks["hbm_gbs"])
     achieved_gbs = bytes_per_launch / (launch_ms * 1e-3) / 1e9
-    flops_per_launch = 36864 * units_per_step   # 9 N^2 per token-head: the exact recurrence
-    path = "decode" if decode else _path_name(args)
+    flops_per_launch = 9 * N * N * units_per_step   # 9 N^2 per token-head: the exact recurrence
+    wtag = args.workload if N == 64 else f"{args.workload}-N{N}"   # profiles are per head size
+    path = "decode" if decode else plan_algo
     if path == "seq":
         sm_max = float(peaks.get("sm_max_mhz", 1965.0))
         fp32_peak = 148 * 128 * 2 * sm_max * 1e6 / 1e12
@@ -304,12 +309,12 @@ def run_gpu(args, world, rank, local):
         roof = {"bound": "alu", "achieved": round(achieved, 3), "peak": round(fp32_peak, 2),
                 "unit": "TFLOP/s", "frac": round(achieved / fp32_peak, 4),
                 "peak_source": f"148 SMs x 128 FP32 lanes x 2 flop x {sm_max:.0f} MHz (derived)",
-                "traffic": measured_traffic("seq_kernel", args.workload, raw), "kernel": "seq_kernel",
+                "traffic": measured_traffic("seq_kernel", wtag, raw), "kernel": "seq_kernel",
                 "hbm_gbs": round(achieved_gbs, 1), "hbm_frac": round(achieved_gbs / hbm_peak, 4)}
     else:
         roof = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved_gbs / hbm_peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
-                "traffic": measured_traffic("decode_kernel" if decode else "chunk_kernel", args.workload, raw),
+                "traffic": measured_traffic("decode_kernel" if decode else "chunk_kernel", wtag, raw),
                 "kernel": "decode_kernel" if decode else "chunk_kernel",
                 "recurrence_tflops": round(flops_per_launch / (launch_ms * 1e-3) / 1e12, 3)}
     roof["algorithmic_bytes_per_launch"] = bytes_per_launch
@@ -600,6 +605,8 @@ def main(argv=None):
     ap.add_argument("--algo", choices=["auto", "seq", "chunk", "split"], default="auto")
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--head-size", type=int, choices=[64, 128], default=64,
+                    help="128: the same channels per token in heads of 128 (scan path)")
     ap.add_argument("--pass", dest="pass_", choices=["forward", "backward"], default="forward",
                     help="backward: gradients of every input from a forward's snapshots")
     ap.add_argument("--inputs", choices=["prepared", "raw"], default="prepared",

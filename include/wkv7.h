@@ -19,7 +19,11 @@
  * with the population variance over the N channels of the head.
  *
  * Conventions for every entry point:
- *   - N must be 64 (the head size the kernels are written for).
+ *   - N is 64 on every path, or 128 (the larger head size the pages name as the next
+ *     one) on the sequential scan, its epilogue and the decode step. The chunked
+ *     algorithms and the backward pass take N = 64 only: WKV7_ALGO_CHUNK / SPLIT with
+ *     N = 128 and wkv7_backward with N != 64 return WKV7_ERR_UNSUPPORTED, and
+ *     WKV7_ALGO_AUTO runs N = 128 on the scan.
  *   - Token tensors r, w, k, v, kk, a are [B][T][H][N] row-major (decode: [B][H][N]),
  *     all of the dtype given by `dt`. States are [B][H][N][N] fp32 row-major.
  *     y is fp32 with the layout of the token tensors.
@@ -52,14 +56,15 @@ extern "C" {
 #define WKV7_API
 #endif
 
-#define WKV7_ABI_VERSION 2
+#define WKV7_ABI_VERSION 3
 #define WKV7_HEAD_SIZE 64
 #define WKV7_MAX_SEGMENTS 8   /* CTAs per (b, h) of WKV7_ALGO_SPLIT (one thread-block cluster) */
 
 typedef enum wkv7_status {
     WKV7_OK = 0,
     WKV7_ERR_ARG = 1,          /* null / host / too-small pointer, bad size or option   */
-    WKV7_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement (N != 64) */
+    WKV7_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement (N not 64 or 128,
+                                  or 128 on a path that takes 64 only) */
     WKV7_ERR_ALIGN = 3,        /* a pointer is not 16-byte aligned                       */
     WKV7_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed                    */
     WKV7_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up (see poll below)    */

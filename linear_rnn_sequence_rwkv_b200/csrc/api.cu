@@ -105,7 +105,8 @@ wkv7_status check_args(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opt
                        bool need_buffers = true) {
     if (N <= 0 || B <= 0 || H <= 0 || T < 0)
         return fail(WKV7_ERR_ARG, "bad sizes B=%d T=%d H=%d N=%d (need B,H,N >= 1, T >= 0)", B, T, H, N);
-    if (N != wkv7::kN) return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: only N=64 is implemented", N);
+    if (N != wkv7::kN && N != 128)
+        return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: N=64 and N=128 (scan path) are implemented", N);
     if (dt != WKV7_F32 && dt != WKV7_BF16) return fail(WKV7_ERR_ARG, "unknown dtype %d", (int)dt);
     wkv7_opts_default(&opts);
     if (opts_in) opts = *opts_in;
@@ -248,7 +249,7 @@ wkv7_status forward_impl(bool raw, int B, int T, int H, int N, wkv7_dtype dt, co
     }
 
     wkv7::FwdArgs p{};
-    p.B = B; p.T = T; p.H = H; p.dt = dt;
+    p.B = B; p.T = T; p.H = H; p.N = N; p.dt = dt;
     p.r = r; p.w = w; p.k = k; p.v = v; p.kk = raw ? nullptr : kk; p.a = a;
     p.S0 = S0; p.y = y; p.S_T = S_T;
     p.snap_every = n_snap ? opts.snap_every : 0;
@@ -310,7 +311,7 @@ wkv7_status wkv7_plan(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opts
     const wkv7_status vs = check_args(B, T, H, N, dt, opts_in, opts, false);   // no buffers needed
     if (vs != WKV7_OK) return vs;
     wkv7::FwdArgs p{};
-    p.B = B; p.T = T; p.H = H; p.dt = dt;
+    p.B = B; p.T = T; p.H = H; p.N = N; p.dt = dt;
     p.snap_every = (opts.snap_every > 0 && T >= opts.snap_every) ? opts.snap_every : 0;
     p.chunk = opts.chunk;
     p.segments = requested_segments(opts);
@@ -353,7 +354,8 @@ wkv7_status wkv7_decode_step(int B, int H, int N, wkv7_dtype dt, const void *r, 
                              const void *v, const void *kk, const void *a, float *S, float *y, void *stream) {
     g_err[0] = '\0';
     if (N <= 0 || B <= 0 || H <= 0) return fail(WKV7_ERR_ARG, "bad sizes B=%d H=%d N=%d", B, H, N);
-    if (N != wkv7::kN) return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: only N=64 is implemented", N);
+    if (N != wkv7::kN && N != 128)
+        return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: N=64 and N=128 are implemented", N);
     if (dt != WKV7_F32 && dt != WKV7_BF16) return fail(WKV7_ERR_ARG, "unknown dtype %d", (int)dt);
     size_t tok = 1;
     if (!mul_ok(tok, B) || !mul_ok(tok, H) || !mul_ok(tok, N) || tok > (size_t(1) << 36))
@@ -382,7 +384,7 @@ wkv7_status wkv7_decode_step(int B, int H, int N, wkv7_dtype dt, const void *r, 
         const wkv7_status s = check_device_buffer(Buf{names[i], req[i], bytes[i]}, device);
         if (s != WKV7_OK) return s;
     }
-    wkv7::DecArgs p{B, H, dt, r, w, k, v, kk, a, S, y, static_cast<cudaStream_t>(stream)};
+    wkv7::DecArgs p{B, H, N, dt, r, w, k, v, kk, a, S, y, static_cast<cudaStream_t>(stream)};
     e = wkv7::launch_decode(p);
     return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "decode launch");
 }
@@ -425,7 +427,7 @@ wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype dt, const void 
     g_err[0] = '\0';
     if (N <= 0 || B <= 0 || H <= 0 || T < 0)
         return fail(WKV7_ERR_ARG, "bad sizes B=%d T=%d H=%d N=%d (need B,H,N >= 1, T >= 0)", B, T, H, N);
-    if (N != wkv7::kN) return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: only N=64 is implemented", N);
+    if (N != wkv7::kN) return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: the backward pass is implemented for N=64", N);
     if (dt != WKV7_F32 && dt != WKV7_BF16) return fail(WKV7_ERR_ARG, "unknown dtype %d", (int)dt);
     if (snap_every < 0) return fail(WKV7_ERR_ARG, "snap_every=%d < 0", snap_every);
     const int n_snap = snap_every > 0 ? T / snap_every : 0;
@@ -478,7 +480,7 @@ wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype dt, const void 
     if (T == 0) {   // dS0 <- dS_T (or zeros)
         if (!dS0) return WKV7_OK;
         wkv7::FwdArgs c{};
-        c.B = B; c.H = H; c.S0 = dS_T; c.S_T = dS0; c.stream = cs;
+        c.B = B; c.H = H; c.N = N; c.S0 = dS_T; c.S_T = dS0; c.stream = cs;
         e = wkv7::launch_copy_state(c);
         return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "state-gradient copy launch");
     }

@@ -1012,7 +1012,7 @@ cudaError_t chunk_segments(const FwdArgs &p, int *segments, int *launches) {
 }
 
 bool chunk_supported(const FwdArgs &p) {
-    return p.dt == WKV7_BF16 && (p.snap_every == 0 || p.snap_every % C == 0);
+    return p.N == kN && p.dt == WKV7_BF16 && (p.snap_every == 0 || p.snap_every % C == 0);
 }
 
 cudaError_t launch_chunk(const FwdArgs &p) {

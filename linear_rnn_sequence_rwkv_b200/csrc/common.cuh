@@ -14,6 +14,7 @@ constexpr int kN = WKV7_HEAD_SIZE;   // head size: the state of one (b, h) is kN
 // Arguments of one forward call after validation (device pointers, caller's stream).
 struct FwdArgs {
     int B, T, H;
+    int N;                 // head size: 64, or 128 on the scan path
     wkv7_dtype dt;
     const void *r, *w, *k, *v, *kk, *a;
     const float *S0;       // nullable: zero initial state
@@ -34,6 +35,7 @@ struct FwdArgs {
 
 struct DecArgs {
     int B, H;
+    int N;                 // head size: 64 or 128
     wkv7_dtype dt;
     const void *r, *w, *k, *v, *kk, *a;
     float *S;

@@ -17,32 +17,37 @@ namespace {
 
 constexpr int kDecThreads = 256;
 
-template <class Tin>
+// NN = 64: the layout above. NN = 128: a warp covers one 512-byte row (32 float4 columns) and
+// a thread holds rows t/32 + 8m, m = 0..15; the row dot products reduce over the 32 lanes.
+template <class Tin, int NN>
 __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecArgs p) {
+    constexpr int CL = NN / 4;                  // lanes per row (one float4 each)
+    constexpr int RS = kDecThreads / CL;        // row stride between a thread's rows
+    constexpr int RPT = NN / RS;                // rows per thread
     const int unit = blockIdx.x;
-    const int c4 = threadIdx.x & 15, rbase = threadIdx.x >> 4;
-    float *S = p.S + size_t(unit) * kN * kN;
-    const size_t vo = size_t(unit) * kN;
+    const int c4 = threadIdx.x % CL, rbase = threadIdx.x / CL;
+    float *S = p.S + size_t(unit) * NN * NN;
+    const size_t vo = size_t(unit) * NN;
 
-    float4 s[4];
+    float4 s[RPT];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) s[m] = __ldcs(reinterpret_cast<const float4 *>(S + (rbase + 16 * m) * kN + 4 * c4));
+    for (int m = 0; m < RPT; ++m) s[m] = __ldcs(reinterpret_cast<const float4 *>(S + (rbase + RS * m) * NN + 4 * c4));
 
     const Tin *r = static_cast<const Tin *>(p.r), *w = static_cast<const Tin *>(p.w);
     const Tin *k = static_cast<const Tin *>(p.k), *v = static_cast<const Tin *>(p.v);
     const Tin *kk = static_cast<const Tin *>(p.kk), *a = static_cast<const Tin *>(p.a);
     const float4 w4 = load4(w + vo + 4 * c4), kk4 = load4(kk + vo + 4 * c4), a4 = load4(a + vo + 4 * c4);
     const float4 k4 = load4(k + vo + 4 * c4), r4 = load4(r + vo + 4 * c4);
-    float vi[4];
+    float vi[RPT];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) vi[m] = load1(v + vo + rbase + 16 * m);
+    for (int m = 0; m < RPT; ++m) vi[m] = load1(v + vo + rbase + RS * m);
     const float4 b4 = make_float4(kk4.x * a4.x, kk4.y * a4.y, kk4.z * a4.z, kk4.w * a4.w);
 
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
+    for (int m = 0; m < RPT; ++m) {
         float sk = dot4(s[m], kk4);
 #pragma unroll
-        for (int o = 8; o; o >>= 1) sk += __shfl_xor_sync(0xffffffffu, sk, o);
+        for (int o = CL / 2; o; o >>= 1) sk += __shfl_xor_sync(0xffffffffu, sk, o);
         float4 x;
         x.x = fmaf(vi[m], k4.x, fmaf(-sk, b4.x, s[m].x * w4.x));
         x.y = fmaf(vi[m], k4.y, fmaf(-sk, b4.y, s[m].y * w4.y));
@@ -50,9 +55,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecArgs p) {
         x.w = fmaf(vi[m], k4.w, fmaf(-sk, b4.w, s[m].w * w4.w));
         float yv = dot4(x, r4);
 #pragma unroll
-        for (int o = 8; o; o >>= 1) yv += __shfl_xor_sync(0xffffffffu, yv, o);
-        __stcs(reinterpret_cast<float4 *>(S + (rbase + 16 * m) * kN + 4 * c4), x);
-        if (c4 == 0) p.y[vo + rbase + 16 * m] = yv;
+        for (int o = CL / 2; o; o >>= 1) yv += __shfl_xor_sync(0xffffffffu, yv, o);
+        __stcs(reinterpret_cast<float4 *>(S + (rbase + RS * m) * NN + 4 * c4), x);
+        if (c4 == 0) p.y[vo + rbase + RS * m] = yv;
     }
 }
 
@@ -62,10 +67,16 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecArgs p) {
 
 cudaError_t launch_decode(const DecArgs &p) {
     const unsigned units = unsigned(p.B) * unsigned(p.H);
-    if (p.dt == WKV7_BF16)
-        decode_kernel<__nv_bfloat16><<<units, kDecThreads, 0, p.stream>>>(p);
-    else
-        decode_kernel<float><<<units, kDecThreads, 0, p.stream>>>(p);
+    if (p.N == 128) {
+        if (p.dt == WKV7_BF16)
+            decode_kernel<__nv_bfloat16, 128><<<units, kDecThreads, 0, p.stream>>>(p);
+        else
+            decode_kernel<float, 128><<<units, kDecThreads, 0, p.stream>>>(p);
+    } else if (p.dt == WKV7_BF16) {
+        decode_kernel<__nv_bfloat16, 64><<<units, kDecThreads, 0, p.stream>>>(p);
+    } else {
+        decode_kernel<float, 64><<<units, kDecThreads, 0, p.stream>>>(p);
+    }
     return cudaGetLastError();
 }
 

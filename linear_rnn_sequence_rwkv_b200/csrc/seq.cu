@@ -29,11 +29,11 @@ template <> struct SeqTile<float> { static constexpr int TB = 16; };
 // Shared-memory slots of the key-side vectors.
 enum { kW = 0, kB = 1, kK = 2, kKK = 3, kR = 4, kSlots = 5 };
 
-template <class Tin, int RPT>
+template <class Tin, int RPT, int NN>
 struct SeqSmem {
-    static constexpr int TB = SeqTile<Tin>::TB;
+    static constexpr int TB = SeqTile<Tin>::TB * 64 / NN;   // the same prefetch registers at any NN
     static constexpr int ROWS = 16 * RPT;
-    float vec[kSlots][TB][kN];
+    float vec[kSlots][TB][NN];
     float v[TB][ROWS];
 };
 
@@ -55,12 +55,13 @@ __device__ __forceinline__ void store_vals(float *dst, const float (&o)[E]) {
 // the staging step turns them into w, b = kk * a, k~ and the unit-norm removal key (rebuttal
 // page, the time_mixing listing: decay, learning rate, removal key with its 1e-12 norm floor,
 // key update), with the formulas of the chunked kernel's load stage.
-template <class Tin, int RPT, bool RAW>
+template <class Tin, int RPT, bool RAW, int NN>
 __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const FwdArgs p) {
-    using Sm = SeqSmem<Tin, RPT>;
+    using Sm = SeqSmem<Tin, RPT, NN>;
+    constexpr int NM = NN / 16;                           // float4 column groups per thread
     constexpr int TB = Sm::TB, ROWS = Sm::ROWS;
     constexpr int EPC = 16 / sizeof(Tin);                 // elements per 16-byte chunk
-    constexpr int CPT = kN / EPC;                         // chunks per token vector
+    constexpr int CPT = NN / EPC;                         // chunks per token vector
     constexpr int VEC_CH = TB * CPT / kSeqThreads;        // chunks per thread per vector
     constexpr int VCPT = ROWS / EPC;                      // v chunks per token
     constexpr int V_CH = (TB * VCPT + kSeqThreads - 1) / kSeqThreads;
@@ -76,17 +77,17 @@ __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const FwdArgs p) {
     const Tin *src[6] = {static_cast<const Tin *>(p.w), static_cast<const Tin *>(p.kk),
                          static_cast<const Tin *>(p.a), static_cast<const Tin *>(p.k),
                          static_cast<const Tin *>(p.r), static_cast<const Tin *>(p.v)};
-    auto tok_off = [&](int t) { return ((size_t(b) * T + t) * H + h) * kN; };
+    auto tok_off = [&](int t) { return ((size_t(b) * T + t) * H + h) * NN; };
 
     // state: s[rr][4m + c] = S[row(rr)][4q + 16m + c]
-    float s[RPT][16];
+    float s[RPT][4 * NM];
 #pragma unroll
     for (int rr = 0; rr < RPT; ++rr) {
         const int row = row0 + rg * RPT + rr;
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
+        for (int m = 0; m < NM; ++m) {
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (p.S0) x = __ldg(reinterpret_cast<const float4 *>(p.S0 + (size_t(unit) * kN + row) * kN + 4 * q + 16 * m));
+            if (p.S0) x = __ldg(reinterpret_cast<const float4 *>(p.S0 + (size_t(unit) * NN + row) * NN + 4 * q + 16 * m));
             s[rr][4 * m + 0] = x.x; s[rr][4 * m + 1] = x.y; s[rr][4 * m + 2] = x.z; s[rr][4 * m + 3] = x.w;
         }
     }
@@ -123,7 +124,7 @@ __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const FwdArgs p) {
             unpack16(raw[4][i], tag, r_);
             if (RAW) {
                 // the CPT consecutive threads that hold one token reduce ||k * k_k|| by shuffles
-                const float *kk_p = p.k_k + h * kN + e, *ka_p = p.k_a ? p.k_a + h * kN + e : nullptr;
+                const float *kk_p = p.k_k + h * NN + e, *ka_p = p.k_a ? p.k_a + h * NN + e : nullptr;
                 float ss = 0.f;
 #pragma unroll
                 for (int j = 0; j < EPC; ++j) {
@@ -167,15 +168,15 @@ __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const FwdArgs p) {
         if (t0 + TB < T) issue_loads(t0 + TB);
         const int tn = min(TB, T - t0);
         for (int t = 0; t < tn; ++t) {
-            float4 kk4[4];
+            float4 kk4[NM];
 #pragma unroll
-            for (int m = 0; m < 4; ++m) kk4[m] = reinterpret_cast<const float4 *>(&sm.vec[kKK][t][0])[q + 4 * m];
+            for (int m = 0; m < NM; ++m) kk4[m] = reinterpret_cast<const float4 *>(&sm.vec[kKK][t][0])[q + 4 * m];
             float sk[RPT];
 #pragma unroll
             for (int rr = 0; rr < RPT; ++rr) {
                 float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-                for (int m = 0; m < 4; m += 2) {
+                for (int m = 0; m < NM; m += 2) {
                     acc0 = fmaf(s[rr][4 * m + 0], kk4[m].x, acc0);
                     acc0 = fmaf(s[rr][4 * m + 1], kk4[m].y, acc0);
                     acc0 = fmaf(s[rr][4 * m + 2], kk4[m].z, acc0);
@@ -196,7 +197,7 @@ __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const FwdArgs p) {
 #pragma unroll
             for (int rr = 0; rr < RPT; ++rr) yv[rr] = 0.f;
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
+            for (int m = 0; m < NM; ++m) {
                 const float4 w4 = reinterpret_cast<const float4 *>(&sm.vec[kW][t][0])[q + 4 * m];
                 const float4 b4 = reinterpret_cast<const float4 *>(&sm.vec[kB][t][0])[q + 4 * m];
                 const float4 k4 = reinterpret_cast<const float4 *>(&sm.vec[kK][t][0])[q + 4 * m];
@@ -225,12 +226,12 @@ __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const FwdArgs p) {
             const int tt = t0 + t + 1;
             if (n_snap && tt % p.snap_every == 0) {
                 const int m_idx = tt / p.snap_every - 1;
-                float *dst = p.snaps + (((size_t(b) * n_snap + m_idx) * H + h) * kN) * kN;
+                float *dst = p.snaps + (((size_t(b) * n_snap + m_idx) * H + h) * NN) * NN;
 #pragma unroll
                 for (int rr = 0; rr < RPT; ++rr)
 #pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        *reinterpret_cast<float4 *>(dst + (row0 + rg * RPT + rr) * kN + 4 * q + 16 * m) =
+                    for (int m = 0; m < NM; ++m)
+                        *reinterpret_cast<float4 *>(dst + (row0 + rg * RPT + rr) * NN + 4 * q + 16 * m) =
                             make_float4(s[rr][4 * m], s[rr][4 * m + 1], s[rr][4 * m + 2], s[rr][4 * m + 3]);
             }
         }
@@ -239,26 +240,28 @@ __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const FwdArgs p) {
 #pragma unroll
         for (int rr = 0; rr < RPT; ++rr)
 #pragma unroll
-            for (int m = 0; m < 4; ++m)
-                *reinterpret_cast<float4 *>(p.S_T + (size_t(unit) * kN + row0 + rg * RPT + rr) * kN + 4 * q + 16 * m) =
+            for (int m = 0; m < NM; ++m)
+                *reinterpret_cast<float4 *>(p.S_T + (size_t(unit) * NN + row0 + rg * RPT + rr) * NN + 4 * q + 16 * m) =
                     make_float4(s[rr][4 * m], s[rr][4 * m + 1], s[rr][4 * m + 2], s[rr][4 * m + 3]);
     }
 }
 
-template <class Tin, int RPT, bool RAW>
+template <class Tin, int RPT, bool RAW, int NN>
 cudaError_t launch_seq_t(const FwdArgs &p) {
-    const size_t smem = sizeof(SeqSmem<Tin, RPT>);
-    static cudaError_t attr = cudaFuncSetAttribute(seq_kernel<Tin, RPT, RAW>,
+    const size_t smem = sizeof(SeqSmem<Tin, RPT, NN>);
+    static cudaError_t attr = cudaFuncSetAttribute(seq_kernel<Tin, RPT, RAW, NN>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (attr != cudaSuccess) return attr;
-    dim3 grid(p.B * p.H, kN / (16 * RPT));
-    seq_kernel<Tin, RPT, RAW><<<grid, kSeqThreads, smem, p.stream>>>(p);
+    dim3 grid(p.B * p.H, NN / (16 * RPT));
+    seq_kernel<Tin, RPT, RAW, NN><<<grid, kSeqThreads, smem, p.stream>>>(p);
     return cudaGetLastError();
 }
 
 template <class Tin, int RPT>
 cudaError_t launch_seq_r(const FwdArgs &p) {
-    return p.raw ? launch_seq_t<Tin, RPT, true>(p) : launch_seq_t<Tin, RPT, false>(p);
+    if (p.N == 128)
+        return p.raw ? launch_seq_t<Tin, RPT, true, 128>(p) : launch_seq_t<Tin, RPT, false, 128>(p);
+    return p.raw ? launch_seq_t<Tin, RPT, true, 64>(p) : launch_seq_t<Tin, RPT, false, 64>(p);
 }
 
 // ---- T = 0: S_T <- S0 (or zeros) -------------------------------------------------------------
@@ -267,41 +270,47 @@ __global__ void copy_state_kernel(const float4 *__restrict__ src, float4 *__rest
         dst[i] = src ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// ---- group_norm + bonus epilogue (one warp per (b, t, h) row of 64 channels) ---------------
+// ---- group_norm + bonus epilogue (one warp per (b, t, h) row of NN channels) ----------------
 // RAW: k is the key before its update and a the rate logit; the bonus uses k~ = k + k (a-1) k_a.
-template <class Tin, bool RAW>
+template <class Tin, bool RAW, int NN>
 __global__ void __launch_bounds__(256) epilogue_kernel(const FwdArgs p, size_t rows) {
+    constexpr int E = NN / 32;   // channels per lane
     const size_t row = blockIdx.x * size_t(8) + (threadIdx.x >> 5);
     if (row >= rows) return;
     const int lane = threadIdx.x & 31, h = int(row % p.H);
-    const size_t base = row * kN + 2 * lane;
-    const int pc = h * kN + 2 * lane;
-    float2 yv = *reinterpret_cast<const float2 *>(p.y + base);
+    const size_t base = row * NN + E * lane;
+    const int pc = h * NN + E * lane;
     const Tin *r = static_cast<const Tin *>(p.r), *k = static_cast<const Tin *>(p.k), *v = static_cast<const Tin *>(p.v);
-    float k0 = load1(k + base), k1 = load1(k + base + 1);
-    if (RAW && p.k_a) {
-        const Tin *al = static_cast<const Tin *>(p.a);
-        const float a0 = 1.f / (1.f + __expf(-load1(al + base))), a1 = 1.f / (1.f + __expf(-load1(al + base + 1)));
-        k0 = fmaf(k0 * (a0 - 1.f), p.k_a[pc], k0);
-        k1 = fmaf(k1 * (a1 - 1.f), p.k_a[pc + 1], k1);
+    float yv[E], bon = 0.f, sum = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        yv[e] = p.y[base + e];
+        float ke = load1(k + base + e);
+        if (RAW && p.k_a) {
+            const float ae = 1.f / (1.f + __expf(-load1(static_cast<const Tin *>(p.a) + base + e)));
+            ke = fmaf(ke * (ae - 1.f), p.k_a[pc + e], ke);
+        }
+        bon = fmaf(load1(r + base + e) * ke, p.r_k[pc + e], bon);
+        sum += yv[e];
     }
-    float bon = load1(r + base) * k0 * p.r_k[pc] + load1(r + base + 1) * k1 * p.r_k[pc + 1];
-    float sum = yv.x + yv.y;
 #pragma unroll
     for (int o = 16; o; o >>= 1) {
         sum += __shfl_xor_sync(0xffffffffu, sum, o);
         bon += __shfl_xor_sync(0xffffffffu, bon, o);
     }
-    const float mean = sum * (1.f / kN);
-    const float d0 = yv.x - mean, d1 = yv.y - mean;
-    float sq = d0 * d0 + d1 * d1;
+    const float mean = sum * (1.f / NN);
+    float sq = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        yv[e] -= mean;
+        sq = fmaf(yv[e], yv[e], sq);
+    }
 #pragma unroll
     for (int o = 16; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-    const float inv = 1.f / sqrtf(sq * (1.f / kN) + p.gn_eps);
-    float2 out;
-    out.x = d0 * inv * p.ln_w[pc] + p.ln_b[pc] + bon * load1(v + base);
-    out.y = d1 * inv * p.ln_w[pc + 1] + p.ln_b[pc + 1] + bon * load1(v + base + 1);
-    *reinterpret_cast<float2 *>(p.y + base) = out;
+    const float inv = 1.f / sqrtf(sq * (1.f / NN) + p.gn_eps);
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+        p.y[base + e] = yv[e] * inv * p.ln_w[pc + e] + p.ln_b[pc + e] + bon * load1(v + base + e);
 }
 
 }  // namespace
@@ -314,22 +323,30 @@ cudaError_t launch_seq(const FwdArgs &p) {
 }
 
 cudaError_t launch_copy_state(const FwdArgs &p) {
-    const size_t n4 = size_t(p.B) * p.H * kN * kN / 4;
+    const size_t n4 = size_t(p.B) * p.H * p.N * p.N / 4;
     const int blocks = int(std::min<size_t>((n4 + 255) / 256, 148 * 8));
     copy_state_kernel<<<blocks, 256, 0, p.stream>>>(reinterpret_cast<const float4 *>(p.S0),
                                                     reinterpret_cast<float4 *>(p.S_T), n4);
     return cudaGetLastError();
 }
 
+template <class Tin, bool RAW>
+void launch_epilogue_t(const FwdArgs &p, size_t rows, unsigned blocks) {
+    if (p.N == 128)
+        epilogue_kernel<Tin, RAW, 128><<<blocks, 256, 0, p.stream>>>(p, rows);
+    else
+        epilogue_kernel<Tin, RAW, 64><<<blocks, 256, 0, p.stream>>>(p, rows);
+}
+
 cudaError_t launch_epilogue(const FwdArgs &p) {
     const size_t rows = size_t(p.B) * p.T * p.H;
     const unsigned blocks = unsigned((rows + 7) / 8);
     if (p.dt == WKV7_BF16) {
-        if (p.raw) epilogue_kernel<__nv_bfloat16, true><<<blocks, 256, 0, p.stream>>>(p, rows);
-        else epilogue_kernel<__nv_bfloat16, false><<<blocks, 256, 0, p.stream>>>(p, rows);
+        if (p.raw) launch_epilogue_t<__nv_bfloat16, true>(p, rows, blocks);
+        else launch_epilogue_t<__nv_bfloat16, false>(p, rows, blocks);
     } else {
-        if (p.raw) epilogue_kernel<float, true><<<blocks, 256, 0, p.stream>>>(p, rows);
-        else epilogue_kernel<float, false><<<blocks, 256, 0, p.stream>>>(p, rows);
+        if (p.raw) launch_epilogue_t<float, true>(p, rows, blocks);
+        else launch_epilogue_t<float, false>(p, rows, blocks);
     }
     return cudaGetLastError();
 }

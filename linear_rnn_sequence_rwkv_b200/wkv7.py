@@ -19,7 +19,7 @@ import torch
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libwkv7.so")
 HEAD_SIZE = 64
-ABI_VERSION = 2          # WKV7_ABI_VERSION of include/wkv7.h this binding follows
+ABI_VERSION = 3          # WKV7_ABI_VERSION of include/wkv7.h this binding follows
 
 # wkv7_status
 OK, ERR_ARG, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(7)

@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from linear_rnn_sequence_rwkv_b200 import build, wkv7
 
@@ -36,7 +37,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_strings(lib):
-    assert lib.wkv7_abi_version() == 2
+    assert lib.wkv7_abi_version() == 3
     assert lib.wkv7_status_string(0) == b"WKV7_OK"
     assert lib.wkv7_status_string(3) == b"WKV7_ERR_ALIGN"
     assert lib.wkv7_status_string(99) == b"WKV7_ERR_UNKNOWN"
@@ -58,7 +59,8 @@ def _fwd(lib, B=1, T=4, H=1, N=64, dt=1, ptrs=None, opts=None, ws=None, ws_bytes
 
 @pytest.mark.parametrize("kw,status", [
     (dict(N=63), wkv7.ERR_UNSUPPORTED),
-    (dict(N=128), wkv7.ERR_UNSUPPORTED),
+    (dict(N=96), wkv7.ERR_UNSUPPORTED),
+    (dict(N=256), wkv7.ERR_UNSUPPORTED),
     (dict(N=0), wkv7.ERR_ARG),
     (dict(B=0), wkv7.ERR_ARG),
     (dict(H=-1), wkv7.ERR_ARG),
@@ -231,3 +233,13 @@ def test_backward_workspace_query():
     assert wkv7.backward_workspace_bytes(2, 100, 3, snap_every=16) == 2 * 3 * 4 * 16384
     assert wkv7.backward_workspace_bytes(2, 100, 3, snap_every=200) == 2 * 3 * 25 * 16384
     assert wkv7.backward_workspace_bytes(2, 100, 3, N=32) == 0
+
+
+def test_head_size_128_runs_on_the_scan():
+    """N = 128: AUTO plans the scan; the chunked algorithms and the backward refuse it."""
+    assert wkv7.plan(2, 300, 4, 128, torch.bfloat16) == ("seq", 0)
+    assert wkv7.plan(2, 300, 4, 128, torch.float32, algo="seq") == ("seq", 0)
+    with pytest.raises(wkv7.Wkv7Error) as e:
+        wkv7.plan(2, 300, 4, 128, torch.bfloat16, algo="chunk")
+    assert e.value.status == wkv7.ERR_UNSUPPORTED
+    assert wkv7.backward_workspace_bytes(2, 300, 4, N=128) == 0
