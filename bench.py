@@ -174,6 +174,12 @@ def dist_setup():
     return world, rank, local
 
 
+def rank_seed(wl, rank: int, salt: int = 0) -> int:
+    """Seed of rank `rank`'s batch: every rank draws its own batch of the workload (weak
+    scaling over independent (b, h) units; no data crosses ranks)."""
+    return inputs.SEED_BASE + wl.cid + 1000 * rank + salt
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -222,7 +228,7 @@ def run_gpu(args, world, rank, local):
     snap_every = wl.snap_every
 
     # independent batches per rank (seed offset), rotating input sets larger than L2
-    seed0 = inputs.SEED_BASE + wl.cid + 1000 * rank
+    seed0 = rank_seed(wl, rank)
     if decode:
         n_tok = 128
         d = inputs.make_inputs(wl, device=str(dev), seed=seed0, T=n_tok)
@@ -365,7 +371,7 @@ def run_backward(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     B, T, H, N = wl.B, wl.T, wl.H, wl.N
     snap = 64
-    seed0 = inputs.SEED_BASE + wl.cid + 1000 * rank + 77
+    seed0 = rank_seed(wl, rank, 77)
     set_bytes = B * T * H * N * (6 * 2 + 4) + B * (T // snap) * H * N * N * 4
     n_sets = max(1, min(4, math.ceil(2 * L2_BYTES / set_bytes)))
     sets = []
