@@ -306,19 +306,72 @@ def poll_device_error(stream=None):
     _check(load().wkv7_poll_device_error(_stream_handle(dev, stream)), "wkv7_poll_device_error")
 
 
+_copy_streams = {}
+
+
+def _side_streams(dev):
+    """Two copy streams per device (host->device and device->host), made once."""
+    if dev not in _copy_streams:
+        _copy_streams[dev] = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+    return _copy_streams[dev]
+
+
 def _forward_host(r, w, k, v, kk, a, S0, *, return_state, out_host, **kw):
-    """End-to-end path for host tensors: H2D copies, the kernels, D2H copies, all on
-    the current stream, which is synchronised before returning."""
+    """End-to-end path for host tensors. The batch is cut into up to eight slices of whole
+    sequences (at least 24 MB of input each, so per-copy overheads stay small); slice i's host->device copies (one stream), its forward (the current stream)
+    and its device->host copies (another stream) overlap with those of the other slices, so
+    the two copy directions and the kernels run at the same time. Returns after the
+    current stream has waited for everything and been synchronised."""
     dev = torch.device("cuda", torch.cuda.current_device())
-    stream = torch.cuda.current_stream(dev)
-    to = lambda t: None if t is None else t.to(dev, non_blocking=True)
-    ep = {n: to(kw.pop(n)) for n in ("ln_w", "ln_b", "r_k")}
-    y, S_T, snaps = forward(*(to(t) for t in (r, w, k, v, kk, a)), to(S0), return_state=return_state,
-                            **ep, **kw)
+    main = torch.cuda.current_stream(dev)
+    s_in, s_out = _side_streams(dev)
+    B, T, H, N = r.shape
+    snap_every = kw.get("snap_every", 0)
+    n_snap = T // snap_every if snap_every else 0
+    ins = {"r": r, "w": w, "k": k, "v": v, "kk": kk, "a": a, "S0": S0}
+    dv = {n: None if t is None else torch.empty(t.shape, dtype=t.dtype, device=dev) for n, t in ins.items()}
+    y_d = torch.empty((B, T, H, N), device=dev, dtype=torch.float32)
+    S_d = torch.empty((B, H, N, N), device=dev, dtype=torch.float32) if return_state else None
+    sn_d = torch.empty((B, n_snap, H, N, N), device=dev, dtype=torch.float32) if n_snap else None
     y_h, S_h = out_host if out_host is not None else (None, None)
-    y_h = y.to("cpu") if y_h is None else y_h.copy_(y, non_blocking=True)
-    if S_T is not None:
-        S_h = S_T.to("cpu") if S_h is None else S_h.copy_(S_T, non_blocking=True)
-    sn_h = None if snaps is None else snaps.to("cpu")
-    stream.synchronize()
-    return y_h, S_h, sn_h
+    if y_h is None:
+        y_h = torch.empty((B, T, H, N), dtype=torch.float32, pin_memory=True)
+    if S_d is not None and S_h is None:
+        S_h = torch.empty((B, H, N, N), dtype=torch.float32, pin_memory=True)
+    sn_h = torch.empty((B, n_snap, H, N, N), dtype=torch.float32, pin_memory=True) if n_snap else None
+    s_in.wait_stream(main)   # the device buffers above were made on the current stream
+    ep = {}
+    with torch.cuda.stream(s_in):
+        for n in ("ln_w", "ln_b", "r_k"):
+            t = kw.pop(n, None)
+            ep[n] = None if t is None else t.to(dev, non_blocking=True)
+    for t in [*dv.values(), *ep.values()]:
+        if t is not None:
+            t.record_stream(s_in)
+    in_bytes = sum(t.numel() * t.element_size() for t in ins.values() if t is not None)
+    pieces = max(1, min(B, 8, in_bytes // (24 << 20))) if T > 0 else 1   # slices of >= 24 MB of input
+    cuts = [B * i // pieces for i in range(pieces + 1)]
+    for b0, b1 in zip(cuts[:-1], cuts[1:]):
+        if b0 == b1:
+            continue
+        with torch.cuda.stream(s_in):
+            for n, t in ins.items():
+                if t is not None:
+                    dv[n][b0:b1].copy_(t[b0:b1], non_blocking=True)
+        main.wait_stream(s_in)
+        sl = lambda t: None if t is None else t[b0:b1]
+        forward(*(dv[n][b0:b1] for n in ("r", "w", "k", "v", "kk", "a")), sl(dv["S0"]), y=y_d[b0:b1],
+                S_T=sl(S_d), snapshots=sl(sn_d), return_state=return_state, **ep, **kw)
+        s_out.wait_stream(main)
+        with torch.cuda.stream(s_out):
+            y_h[b0:b1].copy_(y_d[b0:b1], non_blocking=True)
+            if S_d is not None:
+                S_h[b0:b1].copy_(S_d[b0:b1], non_blocking=True)
+            if sn_d is not None:
+                sn_h[b0:b1].copy_(sn_d[b0:b1], non_blocking=True)
+    for t in (y_d, S_d, sn_d):
+        if t is not None:
+            t.record_stream(s_out)
+    main.wait_stream(s_out)
+    main.synchronize()
+    return y_h, (S_h if return_state else None), sn_h
