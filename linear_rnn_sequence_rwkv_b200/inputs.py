@@ -168,3 +168,47 @@ def make_raw_inputs(wl: Workload, *, seed: int | None = None, device: str = "cpu
         out["ln_b"] = (0.1 * randn(H, N)).contiguous()
         out["r_k"] = (0.5 * randn(H, N)).contiguous()
     return out
+
+
+LAYER_RANKS = {"d_w": 64, "d_a": 64, "d_v": 32, "d_g": 128}   # low-rank widths of the synthetic layer
+
+
+def make_layer(B: int, T: int, H: int, N: int = HEAD_SIZE, *, seed: int = SEED_BASE + 900, device: str = "cpu",
+               dtype: str = "bf16", first_layer: bool = False, ranks: dict | None = None) -> dict:
+    """Synthetic weights and activations for one time-mixing layer (no trained weights are
+    available): x, last_x, v0 ([B, T, C] / [B, C], C = H * N) and the projections in the layer
+    dtype; mixes, biases and the per-head parameters fp32. Scales keep every projection's
+    output near unit variance: square projections N(0, 1/C), low-rank factors N(0, 1/fan_in).
+    No arithmetic of the method is applied."""
+    rk = dict(LAYER_RANKS if ranks is None else ranks)
+    C = H * N
+    dt = torch_dtype(dtype)
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+
+    def randn(*s, std=1.0):
+        return std * torch.randn(*s, generator=g, device=device, dtype=torch.float32)
+
+    def rand(*s):
+        return torch.rand(*s, generator=g, device=device, dtype=torch.float32)
+
+    out = {"x": randn(B, T, C).to(dt), "last_x": randn(B, C).to(dt)}
+    out["v0"] = None if first_layer else randn(B, T, C).to(dt)
+    for m in ("mr", "mw", "mk", "mv", "ma", "mg"):
+        out[m] = rand(C)
+    out["w_bias"] = randn(C, std=0.5)
+    out["a_bias"] = randn(C, std=0.5)
+    out["v_bias"] = randn(C, std=0.5)
+    out["r_k"] = randn(H, N, std=0.5)
+    out["k_k"] = 0.5 + rand(H, N)
+    out["k_a"] = rand(H, N)
+    out["ln_w"] = 1.0 + randn(H, N, std=0.1)
+    out["ln_b"] = randn(H, N, std=0.1)
+    for n in ("Wr", "Wk", "Wv", "Wo"):
+        out[n] = randn(C, C, std=C ** -0.5).to(dt)
+    for lo, hi, d in (("Ww1", "Ww2", rk["d_w"]), ("Wa1", "Wa2", rk["d_a"]), ("Wv1", "Wv2", rk["d_v"]),
+                      ("Wg1", "Wg2", rk["d_g"])):
+        out[lo] = randn(C, d, std=C ** -0.5).to(dt)
+        out[hi] = randn(d, C, std=d ** -0.5).to(dt)
+    out["S0"] = randn(B, H, N, N, std=0.1)
+    return out

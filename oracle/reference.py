@@ -155,6 +155,57 @@ def prepare_inputs(w_logit, a_logit, k, k_k, k_a=None):
     return w, a, kk, k_tilde
 
 
+LAYER_PARAM_NAMES = ("mr", "mw", "mk", "mv", "ma", "mg", "w_bias", "a_bias", "v_bias", "r_k", "k_k", "k_a",
+                     "ln_w", "ln_b", "Wr", "Wk", "Wv", "Wo", "Ww1", "Ww2", "Wa1", "Wa2", "Wv1", "Wv2", "Wg1", "Wg2")
+
+
+def time_mixing_layer(x, params, last_x=None, v0=None, S0=None, eps=64e-5):
+    """One RWKV-7 time-mixing layer over a sequence, in fp64 (the rebuttal page's numpy
+    ``time_mixing`` listing, applied token after token with the state, the previous token
+    and the first layer's values carried along).
+
+    x: [B, T, C] with C = H * N. params (arrays, fp64-convertible): token-shift mixes
+    mr, mw, mk, mv, ma, mg [C]; biases w_bias, a_bias, v_bias [C]; r_k, k_k, k_a, ln_w, ln_b
+    [H, N]; square projections Wr, Wk, Wv, Wo [C_out, C_in] applied as W x; low-rank factors
+    Ww1 [C, Dw], Ww2 [Dw, C], Wa1, Wa2, Wv1, Wv2, Wg1, Wg2 likewise, applied as x W.
+    last_x: [B, C] (the token before x[:, 0]; None = zeros). v0: [B, T, C] values of the
+    first layer (None: this is the first layer, and its own v is returned as v0).
+    S0: [B, H, N, N] or None. Returns (out [B, T, C], v0 [B, T, C], last x [B, C], S_T).
+
+    Per token, with x_p the previous token (last_x for the first):
+      x_m = x + m (x_p - x) for the six mixes m
+      r = Wr x_r, k = Wk x_k, v = Wv x_v
+      w = exp(-sigmoid(tanh(x_w Ww1) Ww2 + w_bias) / sqrt(e))
+      v <- v + (v0 - v) sigmoid(x_v Wv1 Wv2 + v_bias)        (layers after the first)
+      a = sigmoid(x_a Wa1 Wa2 + a_bias), g = sigmoid(x_g Wg1) Wg2
+      kk = normalised (k * k_k) per head, k <- k + k (a - 1) k_a
+      the recurrence and readout per head, group_norm + bonus, out = Wo (y * g).
+    """
+    P = {n: _f64(params[n]) for n in LAYER_PARAM_NAMES}
+    x = _f64(x)
+    B, T, C = x.shape
+    H, N = P["r_k"].shape
+    prev = np.concatenate([np.zeros((B, 1, C)) if last_x is None else _f64(last_x)[:, None], x[:, :-1]], axis=1)
+    mix = {m: x + P[m] * (prev - x) for m in ("mr", "mw", "mk", "mv", "ma", "mg")}
+    sig = lambda z: 1.0 / (1.0 + np.exp(-z))
+    r = mix["mr"] @ P["Wr"].T
+    k = mix["mk"] @ P["Wk"].T
+    v = mix["mv"] @ P["Wv"].T
+    w_logit = np.tanh(mix["mw"] @ P["Ww1"]) @ P["Ww2"] + P["w_bias"]
+    if v0 is None:
+        v0 = v
+    else:
+        v = v + (_f64(v0) - v) * sig(mix["mv"] @ P["Wv1"] @ P["Wv2"] + P["v_bias"])
+    a_logit = mix["ma"] @ P["Wa1"] @ P["Wa2"] + P["a_bias"]
+    g = sig(mix["mg"] @ P["Wg1"]) @ P["Wg2"]
+    heads = lambda z: z.reshape(B, T, H, N)
+    w, a, kk, k_t = prepare_inputs(heads(w_logit), heads(a_logit), heads(k), P["k_k"], P["k_a"])
+    y, S_T, _ = wkv7_recurrence(heads(r), w, k_t, heads(v), kk, a, S0)
+    y = group_norm_bonus(y, heads(r), k_t, heads(v), P["ln_w"], P["ln_b"], P["r_k"], eps)
+    out = (y.reshape(B, T, C) * g) @ P["Wo"].T
+    return out, v0, x[:, -1].copy(), S_T
+
+
 def transition_matrix(w_t, kk_t, a_t):
     """A_t = diag(w_t) - kk_t (kk_t * a_t)^T for one head (vectors of length N)."""
     w_t, kk_t, a_t = (_f64(x) for x in (w_t, kk_t, a_t))

@@ -191,3 +191,57 @@ BACKWARD_PINS = [
 def test_backward_mutant_is_caught(monkeypatch, kind):
     monkeypatch.setattr(reference, "wkv7_backward", _backward(kind))
     assert _failures(BACKWARD_PINS) >= 1
+
+
+# ---- layer mutants --------------------------------------------------------------------------
+
+from tests import test_oracle_layer as PL   # noqa: E402
+
+
+def _layer_mutant(kind):
+    def run(x, params, last_x=None, v0=None, S0=None, eps=64e-5):
+        P = {n: _f64(params[n]) for n in reference.LAYER_PARAM_NAMES}
+        x = _f64(x)
+        B, T, C = x.shape
+        H, N = P["r_k"].shape
+        first = np.zeros((B, 1, C)) if (last_x is None or kind == "ignores_last_x") else _f64(last_x)[:, None]
+        prev = np.concatenate([first, x[:, :-1]], axis=1)
+        sgn = -1.0 if kind == "mix_sign" else 1.0
+        mix = {m: x + sgn * P[m] * (prev - x) for m in ("mr", "mw", "mk", "mv", "ma", "mg")}
+        sig = lambda z: 1.0 / (1.0 + np.exp(-z))
+        r = mix["mr"] @ P["Wr"].T
+        k = mix["mk"] @ P["Wk"].T
+        v = mix["mv"] @ P["Wv"].T
+        w_logit = np.tanh(mix["mw"] @ P["Ww1"]) @ P["Ww2"] + P["w_bias"]
+        if v0 is None:
+            v0 = v
+        else:
+            lerp = sig(mix["mv"] @ P["Wv1"] @ P["Wv2"] + P["v_bias"])
+            v = v + ((v - _f64(v0)) if kind == "residual_sign" else (_f64(v0) - v)) * lerp
+        a_logit = mix["ma"] @ P["Wa1"] @ P["Wa2"] + P["a_bias"]
+        g = sig(mix["mg"] @ P["Wg1"] @ P["Wg2"]) if kind == "gate_sigmoid_outside" else sig(mix["mg"] @ P["Wg1"]) @ P["Wg2"]
+        heads = lambda z: z.reshape(B, T, H, N)
+        w, a, kk, k_t = reference.prepare_inputs(heads(w_logit), heads(a_logit), heads(k), P["k_k"], P["k_a"])
+        y, S_T, _ = reference.wkv7_recurrence(heads(r), w, k_t, heads(v), kk, a, S0)
+        y = reference.group_norm_bonus(y, heads(r), k_t, heads(v), P["ln_w"], P["ln_b"], P["r_k"], eps)
+        return (y.reshape(B, T, C) * g) @ P["Wo"].T, v0, x[:, -1].copy(), S_T
+    return run
+
+
+LAYER_PINS = [
+    PL.test_reduces_to_the_recurrence_and_epilogue,
+    PL.test_full_mix_reads_only_the_previous_token,
+    PL.test_value_residual_limits,
+    PL.test_linear_in_output_projection_and_gate_output_factor,
+    lambda: PL.test_sequence_split_carries_state_and_previous_token(3),
+]
+
+
+@pytest.mark.parametrize("kind", ["mix_sign", "residual_sign", "gate_sigmoid_outside", "ignores_last_x"])
+def test_layer_mutant_is_caught(monkeypatch, kind):
+    monkeypatch.setattr(reference, "time_mixing_layer", _layer_mutant(kind))
+    assert _failures(LAYER_PINS) >= 1
+
+
+def test_unmutated_layer_passes_its_pins():
+    assert _failures(LAYER_PINS) == 0
