@@ -221,6 +221,60 @@ WKV7_API wkv7_status wkv7_backward_static(int B, int T, int H, int N, wkv7_dtype
                           float *dS0, void *stream);
 
 /*
+ * One RWKV-7 time-mixing layer over a sequence (RWKV-7 rebuttal page, the numpy time_mixing
+ * listing, applied token after token with state, previous token and the first layer's values
+ * carried along). With C = H * N channels, M = B * T token rows, x_p the previous token
+ * (last_x for t = 0) and every vector below per token:
+ *     x_m = x + m (x_p - x) for the six mixes m in {mr, mw, mk, mv, ma, mg}
+ *     r = Wr x_r, k = Wk x_k, v = Wv x_v
+ *     w_logit = tanh(x_w Ww1) Ww2 + w_bias, a_logit = x_a Wa1 Wa2 + a_bias
+ *     v <- v + (v0 - v) sigmoid(x_v Wv1 Wv2 + v_bias)          (only when v0 is given)
+ *     g = sigmoid(x_g Wg1) Wg2
+ *     y = wkv7_forward_raw(r, w_logit, k, v, a_logit, k_k, k_a) with the epilogue (ln_w, ln_b, r_k)
+ *     out = Wo (y * g)
+ * The GEMMs run in cuBLASLt (fp32 accumulation; bf16 tensor cores for WKV7_BF16, fp32 for
+ * WKV7_F32) on the caller's workspace; the element-wise steps and the recurrence are this
+ * library's kernels. Intermediates are stored in dt (the logits' and gate's GEMMs in fp32).
+ *
+ * dims:   H, N (64, or 128 on the scan), low-rank widths d_w, d_a, d_v, d_g (>= 1).
+ * params: fp32 mixes and biases [C]; fp32 r_k, k_k, k_a, ln_w, ln_b [H][N] (k_a may be NULL);
+ *         Wr, Wk, Wv, Wo [C][C] of dt applied as W x (row = output channel);
+ *         Ww1, Wa1, Wv1, Wg1 [C][d] and Ww2, Wa2, Wv2, Wg2 [d][C] of dt applied as x W
+ *         (Wv1, Wv2, v_bias unused when v0 is NULL).
+ * x       [B][T][C] dt.     last_x [B][C] dt or NULL (zeros).
+ * v0      [B][T][C] dt: the first layer's values; NULL means this is the first layer.
+ * S       [B][H][N][N] fp32, read and updated in place (NULL: zero state, not returned).
+ * out     [B][T][C] fp32.   v0_out [B][T][C] dt or NULL: receives v when v0 is NULL.
+ * last_x_out [B][C] dt or NULL: receives x[:, T-1].
+ * opts: algorithm, chunk, segments and snapshots of the recurrence (its epilogue fields are
+ *       replaced by params'); NULL = defaults.
+ * Workspace: wkv7_layer_workspace_bytes(B, T, dt, dims) bytes, not overlapping any argument.
+ * Errors: WKV7_ERR_ARG (sizes, NULL required pointers, C != H * N), WKV7_ERR_ALIGN (every
+ * pointer 16-byte aligned), WKV7_ERR_UNSUPPORTED (N), WKV7_ERR_WORKSPACE, WKV7_ERR_CUDA (a launch
+ * or a cuBLASLt call failed; the message names the step). T = 0 only copies last_x.
+ */
+typedef struct {
+    int H, N;
+    int d_w, d_a, d_v, d_g;
+} wkv7_layer_dims;
+
+typedef struct {
+    const float *mr, *mw, *mk, *mv, *ma, *mg;
+    const float *w_bias, *a_bias, *v_bias;
+    const float *r_k, *k_k, *k_a, *ln_w, *ln_b;
+    const void *Wr, *Wk, *Wv, *Wo;
+    const void *Ww1, *Ww2, *Wa1, *Wa2, *Wv1, *Wv2, *Wg1, *Wg2;
+} wkv7_layer_params;
+
+WKV7_API wkv7_status wkv7_layer_forward(int B, int T, wkv7_dtype dt, const wkv7_layer_dims *dims,
+                          const wkv7_layer_params *params, const void *x, const void *last_x,
+                          const void *v0, float *S, float *out, void *v0_out, void *last_x_out,
+                          const wkv7_opts *opts, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes of wkv7_layer_forward (0 when T = 0 or the arguments are invalid). Host only. */
+WKV7_API size_t wkv7_layer_workspace_bytes(int B, int T, wkv7_dtype dt, const wkv7_layer_dims *dims);
+
+/*
  * One decode step for every (b, h): the recurrence for a single token, with the
  * state read and written in place.
  *

@@ -412,6 +412,103 @@ wkv7_status wkv7_backward_static(int B, int T, int H, int N, wkv7_dtype dt, cons
                          dkk, da, dS0, scratch, need ? cap : 0, stream);
 }
 
+static bool layer_dims_ok(const wkv7_layer_dims *d) {
+    return d && d->H > 0 && (d->N == wkv7::kN || d->N == 128) && d->d_w > 0 && d->d_a > 0 && d->d_v > 0 &&
+           d->d_g > 0 && size_t(d->H) * d->N <= (size_t(1) << 20);
+}
+
+size_t wkv7_layer_workspace_bytes(int B, int T, wkv7_dtype dt, const wkv7_layer_dims *dims) {
+    if (B <= 0 || T <= 0 || !layer_dims_ok(dims) || (dt != WKV7_F32 && dt != WKV7_BF16)) return 0;
+    size_t m = 1;
+    if (!mul_ok(m, B) || !mul_ok(m, T) || !mul_ok(m, dims->H) || !mul_ok(m, dims->N) || m > (size_t(1) << 36)) return 0;
+    return wkv7::layer_workspace(B, T, dt, *dims);
+}
+
+wkv7_status wkv7_layer_forward(int B, int T, wkv7_dtype dt, const wkv7_layer_dims *dims,
+                               const wkv7_layer_params *params, const void *x, const void *last_x, const void *v0,
+                               float *S, float *out, void *v0_out, void *last_x_out, const wkv7_opts *opts_in,
+                               void *workspace, size_t workspace_bytes, void *stream) {
+    g_err[0] = '\0';
+    if (B <= 0 || T < 0) return fail(WKV7_ERR_ARG, "bad sizes B=%d T=%d", B, T);
+    if (dt != WKV7_F32 && dt != WKV7_BF16) return fail(WKV7_ERR_ARG, "unknown dtype %d", (int)dt);
+    if (!dims || !params) return fail(WKV7_ERR_ARG, "dims and params are required");
+    if (dims->N != wkv7::kN && dims->N != 128)
+        return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: N=64 and N=128 are implemented", dims->N);
+    if (!layer_dims_ok(dims)) return fail(WKV7_ERR_ARG, "bad layer dims (H, low-rank widths >= 1)");
+    const wkv7_layer_params &P = *params;
+    const int C = dims->H * dims->N;
+    const size_t e = elem_bytes(dt), bc = size_t(B) * C;
+    size_t mc = bc;
+    if (!mul_ok(mc, T) || mc > (size_t(1) << 36)) return fail(WKV7_ERR_ARG, "sizes overflow");
+    wkv7_opts opts;
+    wkv7_opts_default(&opts);
+    if (opts_in) opts = *opts_in;
+    // required pointers and their sizes (bytes); optional ones may be NULL
+    const size_t pc = size_t(C) * 4, ph = size_t(dims->H) * dims->N * 4, sq = size_t(C) * C * e;
+    const Buf bufs[] = {
+        {"mr", P.mr, pc}, {"mw", P.mw, pc}, {"mk", P.mk, pc}, {"mv", P.mv, pc}, {"ma", P.ma, pc}, {"mg", P.mg, pc},
+        {"w_bias", P.w_bias, pc}, {"a_bias", P.a_bias, pc}, {"r_k", P.r_k, ph}, {"k_k", P.k_k, ph},
+        {"ln_w", P.ln_w, ph}, {"ln_b", P.ln_b, ph}, {"Wr", P.Wr, sq}, {"Wk", P.Wk, sq}, {"Wv", P.Wv, sq},
+        {"Wo", P.Wo, sq}, {"Ww1", P.Ww1, size_t(C) * dims->d_w * e}, {"Ww2", P.Ww2, size_t(C) * dims->d_w * e},
+        {"Wa1", P.Wa1, size_t(C) * dims->d_a * e}, {"Wa2", P.Wa2, size_t(C) * dims->d_a * e},
+        {"Wg1", P.Wg1, size_t(C) * dims->d_g * e}, {"Wg2", P.Wg2, size_t(C) * dims->d_g * e},
+        {"x", x, mc * e}, {"out", out, mc * 4}};
+    const Buf opt[] = {{"k_a", P.k_a, ph}, {"v_bias", v0 ? P.v_bias : nullptr, pc},
+                       {"Wv1", v0 ? P.Wv1 : nullptr, size_t(C) * dims->d_v * e},
+                       {"Wv2", v0 ? P.Wv2 : nullptr, size_t(C) * dims->d_v * e},
+                       {"last_x", last_x, bc * e}, {"v0", v0, mc * e}, {"S", S, size_t(B) * dims->H * dims->N * dims->N * 4},
+                       {"v0_out", v0_out, mc * e}, {"last_x_out", last_x_out, bc * e},
+                       {"workspace", workspace, workspace_bytes}};
+    for (const Buf &b : bufs) {
+        if (!b.ptr && T > 0) return fail(WKV7_ERR_ARG, "%s is NULL", b.name);
+        if (b.ptr && !aligned16(b.ptr)) return fail(WKV7_ERR_ALIGN, "%s is not 16-byte aligned", b.name);
+    }
+    if (v0 && (!P.v_bias || !P.Wv1 || !P.Wv2)) return fail(WKV7_ERR_ARG, "v0 given but v_bias / Wv1 / Wv2 is NULL");
+    for (const Buf &b : opt)
+        if (b.ptr && !aligned16(b.ptr)) return fail(WKV7_ERR_ALIGN, "%s is not 16-byte aligned", b.name);
+    const size_t need = wkv7_layer_workspace_bytes(B, T, dt, dims);
+    if (need > 0 && (!workspace || workspace_bytes < need))
+        return fail(WKV7_ERR_WORKSPACE, "workspace of %zu bytes required, %zu given", need, workspace ? workspace_bytes : 0);
+    const Buf outs[] = {{"out", out, T ? mc * 4 : 0}, {"v0_out", v0_out, T ? mc * e : 0},
+                        {"last_x_out", last_x_out, bc * e}, {"S", S, size_t(B) * dims->H * dims->N * dims->N * 4},
+                        {"workspace", workspace, need}};
+    const Buf ins[] = {{"x", x, mc * e}, {"last_x", last_x, bc * e}, {"v0", v0, mc * e}};
+    for (const Buf &o : outs) {
+        for (const Buf &i : ins)
+            if (overlaps(o, i)) return fail(WKV7_ERR_ARG, "%s overlaps %s", o.name, i.name);
+        for (const Buf &o2 : outs)
+            if (&o2 != &o && overlaps(o, o2)) return fail(WKV7_ERR_ARG, "%s overlaps %s", o.name, o2.name);
+    }
+    int device = 0;
+    cudaError_t ce = cudaGetDevice(&device);
+    if (ce != cudaSuccess) {
+        cudaGetLastError();
+        return cuda_fail(ce, "cudaGetDevice");
+    }
+    for (const Buf &b : bufs) {
+        const wkv7_status s = check_device_buffer(b, device);
+        if (s != WKV7_OK) return s;
+    }
+    for (const Buf &b : opt) {
+        const wkv7_status s = check_device_buffer(b, device);
+        if (s != WKV7_OK) return s;
+    }
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (T == 0) {   // nothing to mix: the previous token passes through
+        if (last_x_out) {
+            ce = last_x ? cudaMemcpyAsync(last_x_out, last_x, bc * e, cudaMemcpyDeviceToDevice, cs)
+                        : cudaMemsetAsync(last_x_out, 0, bc * e, cs);
+            if (ce != cudaSuccess) return cuda_fail(ce, "last_x copy");
+        }
+        return WKV7_OK;
+    }
+    char err[400] = "";
+    const wkv7_status s = wkv7::layer_dispatch(B, T, dt, *dims, P, x, last_x, v0, S, out, v0_out, last_x_out, opts,
+                                               workspace, cs, err, sizeof(err));
+    if (s != WKV7_OK) return fail(s, "%s", err);
+    return WKV7_OK;
+}
+
 size_t wkv7_backward_workspace_bytes(int B, int T, int H, int N, int snap_every) {
     if (B <= 0 || T <= 0 || H <= 0 || N != wkv7::kN || snap_every < 0) return 0;
     size_t n = 1;

@@ -67,6 +67,12 @@ cudaError_t launch_copy_state(const FwdArgs &p);   // T == 0: S_T <- S0 (or zero
 cudaError_t launch_backward(const BwdArgs &p);     // T >= 1
 size_t backward_checkpoint_bytes(int B, int T, int H, int snap_every);
 size_t backward_static_scratch_bytes();             // capacity of the module's static scratch
+// One time-mixing layer (validated arguments): launches on `stream`, error text into err.
+size_t layer_workspace(int B, int T, wkv7_dtype dt, const wkv7_layer_dims &d);
+wkv7_status layer_dispatch(int B, int T, wkv7_dtype dt, const wkv7_layer_dims &d, const wkv7_layer_params &P,
+                           const void *x, const void *last_x, const void *v0, float *S, float *out, void *v0_out,
+                           void *last_x_out, const wkv7_opts &opts, void *ws, cudaStream_t stream, char *err,
+                           size_t err_len);
 cudaError_t backward_static_scratch(void **ptr);    // its address on the current device
 bool chunk_supported(const FwdArgs &p);            // bf16 inputs, snapshots on chunk boundaries
 cudaError_t launch_chunk(const FwdArgs &p);        // chunked prefill on tcgen05 (epilogue fused)

@@ -31,13 +31,26 @@ ALGOS = {"auto": 0, "seq": 1, "chunk": 2, "split": 3}
 EXPORTED = ("wkv7_opts_default", "wkv7_forward", "wkv7_decode_step", "wkv7_workspace_bytes",
             "wkv7_status_string", "wkv7_last_error", "wkv7_abi_version", "wkv7_poll_device_error",
             "wkv7_plan", "wkv7_forward_raw", "wkv7_backward", "wkv7_backward_workspace_bytes",
-            "wkv7_backward_static")
+            "wkv7_backward_static", "wkv7_layer_forward", "wkv7_layer_workspace_bytes")
 
 
 class Wkv7Error(RuntimeError):
     def __init__(self, status: int, where: str, detail: str):
         super().__init__(f"{where}: status {status} ({detail})")
         self.status = status
+
+
+class LayerDims(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int), ("N", ctypes.c_int), ("d_w", ctypes.c_int), ("d_a", ctypes.c_int),
+                ("d_v", ctypes.c_int), ("d_g", ctypes.c_int)]
+
+
+LAYER_PARAMS = ("mr", "mw", "mk", "mv", "ma", "mg", "w_bias", "a_bias", "v_bias", "r_k", "k_k", "k_a", "ln_w",
+                "ln_b", "Wr", "Wk", "Wv", "Wo", "Ww1", "Ww2", "Wa1", "Wa2", "Wv1", "Wv2", "Wg1", "Wg2")
+
+
+class LayerParams(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in LAYER_PARAMS]
 
 
 class Opts(ctypes.Structure):
@@ -77,6 +90,11 @@ def load():
         lib.wkv7_backward.restype = ci
         lib.wkv7_backward_static.argtypes = [ci, ci, ci, ci, ci] + [vp] * 6 + [vp, vp, ci, vp, vp] + [vp] * 7 + [vp]
         lib.wkv7_backward_static.restype = ci
+        lib.wkv7_layer_forward.argtypes = [ci, ci, ci, ctypes.POINTER(LayerDims), ctypes.POINTER(LayerParams)] + [
+            vp] * 7 + [ctypes.POINTER(Opts), vp, ctypes.c_size_t, vp]
+        lib.wkv7_layer_forward.restype = ci
+        lib.wkv7_layer_workspace_bytes.argtypes = [ci, ci, ci, ctypes.POINTER(LayerDims)]
+        lib.wkv7_layer_workspace_bytes.restype = ctypes.c_size_t
         lib.wkv7_backward_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
         lib.wkv7_backward_workspace_bytes.restype = ctypes.c_size_t
         lib.wkv7_workspace_bytes.argtypes = [ci, ci, ci, ci, ci, ctypes.POINTER(Opts)]
@@ -284,6 +302,46 @@ def backward_static(r, w, k, v, kk, a, dy, S0=None, dS_T=None, *, snapshots=None
     out = dict(grads)
     out["dS0"] = dS0
     return out
+
+
+def layer_dims(params, H, N=HEAD_SIZE):
+    return LayerDims(H, N, params["Ww1"].shape[1], params["Wa1"].shape[1], params["Wv1"].shape[1],
+                     params["Wg1"].shape[1])
+
+
+def layer_forward(x, params, H, *, N=HEAD_SIZE, last_x=None, v0=None, S=None, out=None, v0_out=None,
+                  last_x_out=None, algo="auto", chunk=0, segments=0, workspace=None, stream=None):
+    """One time-mixing layer over x [B, T, C] (bf16 or fp32; C = H * N) with the weights in
+    ``params`` (names as in LAYER_PARAMS; see wkv7_layer_forward in include/wkv7.h). S
+    [B, H, N, N] fp32 is updated in place. Returns (out, v0_out, last_x_out, S): v0_out is the
+    layer's v when v0 is None (the first layer), else None."""
+    lib = load()
+    B, T, C = x.shape
+    dev = x.device
+    dims = layer_dims(params, H, N)
+    if out is None:
+        out = torch.empty((B, T, C), device=dev, dtype=torch.float32)
+    if v0 is None and v0_out is None:
+        v0_out = torch.empty((B, T, C), device=dev, dtype=x.dtype)
+    if last_x_out is None:
+        last_x_out = torch.empty((B, C), device=dev, dtype=x.dtype)
+    lp = LayerParams(*(None if params.get(n) is None else params[n].data_ptr() for n in LAYER_PARAMS))
+    opts = make_opts(algo, chunk, 0, None, None, None, None, 64e-5, segments)
+    need = int(lib.wkv7_layer_workspace_bytes(B, T, _dt(x), ctypes.byref(dims)))
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = lib.wkv7_layer_forward(B, T, _dt(x), ctypes.byref(dims), ctypes.byref(lp), _ptr(x), _ptr(last_x),
+                                    _ptr(v0), _ptr(S), _ptr(out), _ptr(v0_out), _ptr(last_x_out), ctypes.byref(opts),
+                                    _ptr(workspace), ws_bytes, _stream_handle(dev, stream))
+    _check(st, "wkv7_layer_forward")
+    return out, (v0_out if v0 is None else None), last_x_out, S
+
+
+def layer_workspace_bytes(B, T, params, H, N=HEAD_SIZE, dtype=torch.bfloat16) -> int:
+    return int(load().wkv7_layer_workspace_bytes(B, T, BF16 if dtype == torch.bfloat16 else F32,
+                                                 ctypes.byref(layer_dims(params, H, N))))
 
 
 def decode_step(r, w, k, v, kk, a, S, *, y=None, stream=None):

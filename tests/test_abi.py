@@ -243,3 +243,28 @@ def test_head_size_128_runs_on_the_scan():
         wkv7.plan(2, 300, 4, 128, torch.bfloat16, algo="chunk")
     assert e.value.status == wkv7.ERR_UNSUPPORTED
     assert wkv7.backward_workspace_bytes(2, 300, 4, N=128) == 0
+
+
+def _layer_call(lib, B=1, T=4, H=1, N=64, dt=1, drop=None, over=None, ws=None, ws_bytes=0, v0=None):
+    dims = wkv7.LayerDims(H, N, 8, 8, 8, 8)
+    vals = {n: FAKE + 0x100000 * (i + 1) for i, n in enumerate(wkv7.LAYER_PARAMS)}
+    vals.update(over or {})
+    if drop:
+        vals[drop] = None
+    lp = wkv7.LayerParams(*(vals[n] for n in wkv7.LAYER_PARAMS))
+    P = lambda a: None if a is None else ctypes.c_void_p(a)
+    base = FAKE + 0x10000000
+    return lib.wkv7_layer_forward(B, T, dt, ctypes.byref(dims), ctypes.byref(lp), P(base), None, P(v0), None,
+                                  P(base + 0x1000000), None, None, None, ws, ws_bytes, None)
+
+
+def test_layer_rejects_bad_arguments(lib):
+    assert _layer_call(lib, N=96) == wkv7.ERR_UNSUPPORTED
+    assert _layer_call(lib, drop="Wr") == wkv7.ERR_ARG and b"Wr" in lib.wkv7_last_error()
+    assert _layer_call(lib, drop="ln_b") == wkv7.ERR_ARG
+    assert _layer_call(lib, over={"Wg2": FAKE + 0x100000 * 30 + 8}) == wkv7.ERR_ALIGN
+    assert _layer_call(lib, v0=FAKE + 0x20000000, drop="Wv1") == wkv7.ERR_ARG   # a later layer needs Wv1
+    assert _layer_call(lib) == wkv7.ERR_WORKSPACE
+    dims = wkv7.LayerDims(2, 64, 8, 8, 8, 8)
+    assert lib.wkv7_layer_workspace_bytes(2, 0, 1, ctypes.byref(dims)) == 0
+    assert lib.wkv7_layer_workspace_bytes(2, 10, 1, ctypes.byref(dims)) > 32 << 20

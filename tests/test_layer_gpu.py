@@ -1,0 +1,76 @@
+"""GPU parity of the full time-mixing layer (cuBLASLt GEMMs, this library's element-wise
+kernels and recurrence) against the oracle's fp64 layer.
+
+Bounds (max relative error per (b, h) slice of the output, as everywhere):
+* fp32 layer: 1e-4. The GEMMs accumulate in fp32 over at most C = 256 products (first-order
+  relative error near C * 2^-24 = 1.5e-5 each), the fp32 recurrence stays within its 1e-5
+  bound, and a few such steps lie in series.
+* bf16 layer: 2.2e-2. Every intermediate stored in bf16 is a relative rounding of at most
+  2^-9 = 1.95e-3. The readout y = S r sees, to first order and in the worst case, r's two
+  roundings (mixed input, projection), v's two, k's two, the decay's three (mixed input,
+  low-rank hidden value, logit) and then the gated readout's one: 10 * 1.95e-3 = 1.95e-2,
+  plus the tf32 recurrence's 2e-3 bound.
+"""
+import pytest
+import torch
+
+from linear_rnn_sequence_rwkv_b200 import inputs, wkv7
+from oracle import reference
+from tests.parity_util import slice_rel_err, state_err
+
+pytestmark = pytest.mark.gpu
+
+TOL_LAYER = {"f32": 1e-4, "bf16": 2.2e-2}
+RANKS = {"d_w": 16, "d_a": 16, "d_v": 8, "d_g": 32}
+
+
+def _out_err(got, ref, H):
+    B, T, C = ref.shape
+    return slice_rel_err(got.reshape(B, T, H, C // H), ref.reshape(B, T, H, C // H), (0, 2))
+
+
+def _case(B, T, H, dtype, first, seed):
+    d = inputs.make_layer(B, T, H, seed=seed, dtype=dtype, first_layer=first, ranks=RANKS)
+    ref = reference.time_mixing_layer(d["x"], d, d["last_x"], d["v0"], d["S0"])
+    return d, ref
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("first", [True, False])
+@pytest.mark.parametrize("T", [1, 37, 130])
+def test_layer_matches_oracle(cuda_device, dtype, first, T):
+    H = 4
+    d, (out_ref, v0_ref, last_ref, S_ref) = _case(2, T, H, dtype, first, seed=900 + T + 7 * first)
+    dd = {k: (None if v is None else v.to(cuda_device)) for k, v in d.items()}
+    S = dd["S0"].clone()
+    out, v0_out, last_out, S = wkv7.layer_forward(dd["x"], dd, H, last_x=dd["last_x"], v0=dd["v0"], S=S)
+    assert _out_err(out, out_ref, H) <= TOL_LAYER[dtype]
+    assert state_err(S, S_ref) <= TOL_LAYER[dtype]
+    assert torch.equal(last_out.cpu(), d["x"][:, -1])
+    if first:
+        v_err = _out_err(v0_out.float(), torch.as_tensor(v0_ref), H)
+        assert v_err <= TOL_LAYER[dtype]
+    else:
+        assert v0_out is None
+
+
+def test_layer_two_calls_carry_state_and_previous_token(cuda_device):
+    """Two calls (the second fed the first's state and last token) equal the oracle's layer
+    over the whole sequence."""
+    H, T1 = 4, 40
+    d, (out_ref, _, _, S_ref) = _case(2, 100, H, "f32", False, seed=950)
+    dd = {k: (None if v is None else v.to(cuda_device)) for k, v in d.items()}
+    S = dd["S0"].clone()
+    o1, _, last1, S = wkv7.layer_forward(dd["x"][:, :T1].contiguous(), dd, H, last_x=dd["last_x"],
+                                         v0=dd["v0"][:, :T1].contiguous(), S=S)
+    o2, _, _, S = wkv7.layer_forward(dd["x"][:, T1:].contiguous(), dd, H, last_x=last1,
+                                     v0=dd["v0"][:, T1:].contiguous(), S=S)
+    assert _out_err(torch.cat([o1, o2], dim=1), out_ref, H) <= TOL_LAYER["f32"]
+    assert state_err(S, S_ref) <= TOL_LAYER["f32"]
+
+
+def test_layer_empty_sequence_passes_last_token(cuda_device):
+    d = inputs.make_layer(2, 0, 2, seed=960, dtype="bf16", ranks=RANKS)
+    dd = {k: (None if v is None else v.to(cuda_device)) for k, v in d.items()}
+    _, _, last_out, _ = wkv7.layer_forward(dd["x"], dd, 2, last_x=dd["last_x"], v0=dd["v0"], S=dd["S0"])
+    assert torch.equal(last_out, dd["last_x"])
