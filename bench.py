@@ -467,6 +467,71 @@ def run_backward(args, world, rank, local):
     return out
 
 
+def run_layer(args, world, rank, local):
+    """Full time-mixing layer (a layer after the first: value residual on) with synthetic
+    weights over the prefill workload's batch: one step = wkv7.layer_forward over the batch."""
+    from linear_rnn_sequence_rwkv_b200 import wkv7
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    spec = WORKLOADS[args.workload]
+    wl = inputs.WORKLOADS[spec["cid"]]
+    steps = args.steps if args.steps is not None else max(5, spec["default_steps"] // 4)
+    warmup = args.warmup
+    B, T, H, N = wl.B, wl.T, wl.H, wl.N
+    C = H * N
+    d = inputs.make_layer(B, T, H, N, seed=rank_seed(wl, rank, 55), device=str(dev), dtype="bf16")
+    S = d["S0"].clone()
+    out = torch.empty(B, T, C, device=dev)
+    last = torch.empty(B, C, device=dev, dtype=torch.bfloat16)
+    ws = torch.empty(wkv7.layer_workspace_bytes(B, T, d, H, N), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        S.copy_(d["S0"])
+        wkv7.layer_forward(d["x"], d, H, N=N, last_x=d["last_x"], v0=d["v0"], S=S, out=out, last_x_out=last,
+                           workspace=ws)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        ev[0].record(stream)
+        for i in range(steps):
+            step(warmup + i)
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[steps]), world, dev)
+    ms = total_ms / steps
+    units = B * T * H
+    rk = inputs.LAYER_RANKS
+    gemm_flops = 2 * B * T * C * (4 * C + 2 * (rk["d_w"] + rk["d_a"] + rk["d_v"] + rk["d_g"]))
+    peaks, peak_kind = _peaks()
+    tc_peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops", 1590.0)))
+    achieved = gemm_flops / (ms * 1e-3) / 1e12
+    return {
+        "metric": METRIC.replace("(prefill, decode)", "(time-mixing layer)"), "value": round(units * steps * world /
+                                                                                             (total_ms * 1e-3) / 1e6, 3),
+        "unit": UNIT, "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16+f32",
+        "data": "synthetic weights and activations (seeded torch Philox)",
+        "config": {"workload": f"{args.workload} layer: {wl.name}, C={C}, low-rank {rk}", "B": B, "T": T, "H": H,
+                   "N": N, "path": "layer", "global_batch": B * world, "seq_len": T,
+                   "parallelism": f"dp{world} (independent sequences)"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": tc_peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / tc_peak, 4), "traffic": None,
+                     "kernel": "whole layer step (GEMM flops over the step time; the recurrence runs inside it)",
+                     "peak_source": f"{peak_kind} bf16 (sustained)", "gemm_flops_per_step": gemm_flops},
+        "e2e": None, "clocks": clocks.summary(),
+        # this library's kernels per step: token shift, 2 activations, 2 bias adds, residual, the
+        # recurrence, gate, last token (the 12 GEMMs are cuBLASLt's and not counted)
+        "gpu_launches": steps * 9,
+    }
+
+
 def cpu_baseline_backward(wl, budget_s: float = 12.0):
     """The fp64 oracle's backward (numpy, vectorised over (b, h)) on a bounded sample."""
     from oracle import reference
@@ -613,7 +678,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--head-size", type=int, choices=[64, 128], default=64,
                     help="128: the same channels per token in heads of 128 (scan path)")
-    ap.add_argument("--pass", dest="pass_", choices=["forward", "backward"], default="forward",
+    ap.add_argument("--pass", dest="pass_", choices=["forward", "backward", "layer"], default="forward",
                     help="backward: gradients of every input from a forward's snapshots")
     ap.add_argument("--inputs", choices=["prepared", "raw"], default="prepared",
                     help="raw: decay/rate logits and the key before its update, pre-processing fused")
@@ -633,7 +698,9 @@ def main(argv=None):
     if world != args.gpus and rank == 0:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
     try:
-        if args.pass_ == "backward":
+        if args.pass_ == "layer":
+            out = run_layer(args, world, rank, local)
+        elif args.pass_ == "backward":
             if args.workload == "decode" or args.inputs == "raw":
                 raise SystemExit("--pass backward takes a prefill workload with prepared inputs")
             out = run_backward(args, world, rank, local)
