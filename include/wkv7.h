@@ -92,7 +92,8 @@ typedef enum wkv7_algo {
 /* Options of wkv7_forward. Obtain defaults with wkv7_opts_default(). */
 typedef struct wkv7_opts {
     int algo;             /* wkv7_algo                                                   */
-    int chunk;            /* chunk length of the chunked algorithms; 0 = default         */
+    int chunk;            /* 0 (default) or 64: the chunked kernel's chunk; 16 and 32 are */
+                          /* accepted and run on the scan under AUTO (CHUNK/SPLIT refuse) */
     int snap_every;       /* 0 = no snapshots; else store S after every snap_every tokens */
     float *snapshots;     /* [B][T / snap_every][H][N][N] fp32, required if snap_every>0 */
     const float *ln_w;    /* epilogue: all three NULL (off) or all three [H][N] fp32     */
