@@ -285,19 +285,34 @@ def run_gpu(args, world, rank, local):
         step(i)
     torch.cuda.synchronize(dev)
 
-    # timed region: K steps, one event pair per step on the launching stream
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    # decode: the 128 token steps are captured once in a CUDA graph and replayed (a step is
+    # launch-bound at this size); each replay is timed and divided by its 128 steps
+    graph = None
+    if decode:
+        graph = _decode_graph(lambda: [step(j) for j in range(n_tok)], dev)
+        if graph is not None:
+            reps = max(1, -(-steps // n_tok))
+            steps = reps * n_tok
+            graph.replay()   # warm-up replay (128 steps)
+            torch.cuda.synchronize(dev)
+
+    # timed region: K steps, one event pair per step (per replay for decode) on the launching stream
+    n_ev = steps if graph is None else steps // n_tok
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev + 1)]
     barrier(world)
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index) as clocks:
         ev[0].record(stream)
-        for i in range(steps):
-            step(warmup + i)
+        for i in range(n_ev):
+            if graph is None:
+                step(warmup + i)
+            else:
+                graph.replay()
             ev[i + 1].record(stream)
         torch.cuda.synchronize(dev)
     barrier(world)
-    per_step_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
-    total_ms = ev[0].elapsed_time(ev[steps])
+    per_step_ms = [ev[i].elapsed_time(ev[i + 1]) / (1 if graph is None else n_tok) for i in range(n_ev)]
+    total_ms = ev[0].elapsed_time(ev[n_ev])
     total_ms = max_over_ranks(total_ms, world, dev)
     value = units_per_step * steps * world / (total_ms * 1e-3) / 1e6
     launch_ms = statistics.mean(per_step_ms)
@@ -343,7 +358,9 @@ def run_gpu(args, world, rank, local):
                    "ctas_per_head": ctas_per_head,
                    "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world} (independent (b,h) units)",
                    "l2": (f"{n_sets} rotating input sets, {n_sets * set_bytes / 1e6:.0f} MB > 126 MB L2"
-                          if not decode else "fp32 state 168 MB > 126 MB L2, 128 rotating token inputs")},
+                          if not decode else "fp32 state 168 MB > 126 MB L2, 128 rotating token inputs"),
+                   "timing": ("CUDA graph of the 128 decode steps, replay time / 128" if graph is not None
+                              else "one event pair per step")},
         "roofline": roof,
         "e2e": e2e,
         "gpu_launches": steps * launches_per_step,
@@ -549,6 +566,25 @@ def cpu_baseline_backward(wl, budget_s: float = 12.0):
             break
     return {"value": round(B * T * H * reps / el / 1e6, 5), "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"B{B} T{T} H{H} of the workload (numpy fp64 backward); {reps} run(s), {el:.1f} s wall"}
+
+
+def _decode_graph(body, dev):
+    """CUDA graph of `body` (the 128 decode steps) captured on a side stream, or None when the
+    capture is refused (the eager loop is timed instead)."""
+    try:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                body()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize(dev)
+        return g
+    except Exception as e:   # pragma: no cover - depends on the driver
+        print(f"decode graph capture refused ({e}); timing the eager loop", file=sys.stderr)
+        torch.cuda.synchronize(dev)
+        return None
 
 
 def _path_name(args):
