@@ -17,7 +17,9 @@
 #include <cublasLt.h>
 
 #include <cstdio>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "common.cuh"
 
@@ -118,45 +120,63 @@ struct Gemm {
     cudaDataType_t in_t, out_t;
 };
 
-cublasStatus_t run_gemm(const Gemm &g, void *ws, size_t ws_bytes, cudaStream_t stream) {
-    cublasStatus_t st;
-    cublasLtHandle_t h = lt_handle(&st);
-    if (st != CUBLAS_STATUS_SUCCESS) return st;
-    // column-major view: Y^T[Nout][M] = op(A)[Nout][K] * X^T[K][M]
+// A GEMM shape's cuBLASLt descriptors and chosen algorithm, made once per process and shape
+// (descriptor creation and the heuristic query cost more host time than a small GEMM runs).
+struct GemmPlan {
     cublasLtMatmulDesc_t desc = nullptr;
     cublasLtMatrixLayout_t la = nullptr, lb = nullptr, ld = nullptr;
-    cublasLtMatmulPreference_t pref = nullptr;
+    cublasLtMatmulAlgo_t algo{};
+    cublasStatus_t status = CUBLAS_STATUS_NOT_INITIALIZED;
+};
+
+cublasStatus_t make_plan(cublasLtHandle_t h, const Gemm &g, size_t ws_bytes, GemmPlan &p) {
     const cublasOperation_t ta = g.w_out_major ? CUBLAS_OP_T : CUBLAS_OP_N, tb = CUBLAS_OP_N;
-    float alpha = 1.f, beta = 0.f;
+    cublasLtMatmulPreference_t pref = nullptr;
     cublasLtMatmulHeuristicResult_t heur{};
     int found = 0;
+    cublasStatus_t st;
     do {
-        if ((st = cublasLtMatmulDescCreate(&desc, CUBLAS_COMPUTE_32F, CUDA_R_32F))) break;
-        if ((st = cublasLtMatmulDescSetAttribute(desc, CUBLASLT_MATMUL_DESC_TRANSA, &ta, sizeof(ta)))) break;
-        if ((st = cublasLtMatmulDescSetAttribute(desc, CUBLASLT_MATMUL_DESC_TRANSB, &tb, sizeof(tb)))) break;
-        if (g.w_out_major) st = cublasLtMatrixLayoutCreate(&la, g.in_t, g.K, g.Nout, g.K);
-        else st = cublasLtMatrixLayoutCreate(&la, g.in_t, g.Nout, g.K, g.Nout);
+        if ((st = cublasLtMatmulDescCreate(&p.desc, CUBLAS_COMPUTE_32F, CUDA_R_32F))) break;
+        if ((st = cublasLtMatmulDescSetAttribute(p.desc, CUBLASLT_MATMUL_DESC_TRANSA, &ta, sizeof(ta)))) break;
+        if ((st = cublasLtMatmulDescSetAttribute(p.desc, CUBLASLT_MATMUL_DESC_TRANSB, &tb, sizeof(tb)))) break;
+        // column-major view: Y^T[Nout][M] = op(A)[Nout][K] * X^T[K][M]
+        if (g.w_out_major) st = cublasLtMatrixLayoutCreate(&p.la, g.in_t, g.K, g.Nout, g.K);
+        else st = cublasLtMatrixLayoutCreate(&p.la, g.in_t, g.Nout, g.K, g.Nout);
         if (st) break;
-        if ((st = cublasLtMatrixLayoutCreate(&lb, g.in_t, g.K, g.M, g.K))) break;
-        if ((st = cublasLtMatrixLayoutCreate(&ld, g.out_t, g.Nout, g.M, g.Nout))) break;
+        if ((st = cublasLtMatrixLayoutCreate(&p.lb, g.in_t, g.K, g.M, g.K))) break;
+        if ((st = cublasLtMatrixLayoutCreate(&p.ld, g.out_t, g.Nout, g.M, g.Nout))) break;
         if ((st = cublasLtMatmulPreferenceCreate(&pref))) break;
         if ((st = cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws_bytes,
                                                        sizeof(ws_bytes))))
             break;
-        if ((st = cublasLtMatmulAlgoGetHeuristic(h, desc, la, lb, ld, ld, pref, 1, &heur, &found))) break;
-        if (found == 0) {
-            st = CUBLAS_STATUS_NOT_SUPPORTED;
-            break;
-        }
-        st = cublasLtMatmul(h, desc, &alpha, g.W, la, g.X, lb, &beta, g.Y, ld, g.Y, ld, &heur.algo, ws, ws_bytes,
-                            stream);
+        if ((st = cublasLtMatmulAlgoGetHeuristic(h, p.desc, p.la, p.lb, p.ld, p.ld, pref, 1, &heur, &found))) break;
+        if (found == 0) st = CUBLAS_STATUS_NOT_SUPPORTED;
+        else p.algo = heur.algo;
     } while (false);
     if (pref) cublasLtMatmulPreferenceDestroy(pref);
-    if (ld) cublasLtMatrixLayoutDestroy(ld);
-    if (lb) cublasLtMatrixLayoutDestroy(lb);
-    if (la) cublasLtMatrixLayoutDestroy(la);
-    if (desc) cublasLtMatmulDescDestroy(desc);
     return st;
+}
+
+cublasStatus_t run_gemm(const Gemm &g, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    cublasStatus_t st;
+    cublasLtHandle_t h = lt_handle(&st);
+    if (st != CUBLAS_STATUS_SUCCESS) return st;
+    typedef std::tuple<int, int, int, bool, int, int, int> Key;   // shape, types, device
+    static std::mutex mu;
+    static std::map<Key, GemmPlan> plans;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const Key key(g.M, g.K, g.Nout, g.w_out_major, int(g.in_t), int(g.out_t), dev);
+    GemmPlan *p;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        p = &plans[key];
+        if (p->status == CUBLAS_STATUS_NOT_INITIALIZED) p->status = make_plan(h, g, ws_bytes, *p);
+    }
+    if (p->status != CUBLAS_STATUS_SUCCESS) return p->status;
+    const float alpha = 1.f, beta = 0.f;
+    return cublasLtMatmul(h, p->desc, &alpha, g.W, p->la, g.X, p->lb, &beta, g.Y, p->ld, g.Y, p->ld, &p->algo, ws,
+                          ws_bytes, stream);
 }
 
 constexpr size_t kGemmWorkspace = size_t(32) << 20;
