@@ -74,3 +74,27 @@ def test_layer_empty_sequence_passes_last_token(cuda_device):
     dd = {k: (None if v is None else v.to(cuda_device)) for k, v in d.items()}
     _, _, last_out, _ = wkv7.layer_forward(dd["x"], dd, 2, last_x=dd["last_x"], v0=dd["v0"], S=dd["S0"])
     assert torch.equal(last_out, dd["last_x"])
+
+
+def test_layer_head_size_128(cuda_device):
+    """N = 128 heads (the recurrence on the scan) in the fp32 layer."""
+    H, N = 2, 128
+    d = inputs.make_layer(2, 33, H, N, seed=970, dtype="f32", ranks=RANKS)
+    out_ref, _, _, S_ref = reference.time_mixing_layer(d["x"], d, d["last_x"], d["v0"], d["S0"])
+    dd = {k: (None if v is None else v.to(cuda_device)) for k, v in d.items()}
+    S = dd["S0"].clone()
+    out, _, _, S = wkv7.layer_forward(dd["x"], dd, H, N=N, last_x=dd["last_x"], v0=dd["v0"], S=S)
+    assert _out_err(out, out_ref, H) <= TOL_LAYER["f32"]
+    assert state_err(S, S_ref) <= TOL_LAYER["f32"]
+
+
+def test_layer_bench_shape_bf16(cuda_device):
+    """The bench's layer: B8 T1024 H12 N64 (C = 768), bf16, default low-rank widths, a layer
+    after the first; every output slice against the fp64 oracle layer."""
+    d = inputs.make_layer(8, 1024, 12, seed=980, dtype="bf16")
+    out_ref, _, _, S_ref = reference.time_mixing_layer(d["x"], d, d["last_x"], d["v0"], d["S0"])
+    dd = {k: (None if v is None else v.to(cuda_device)) for k, v in d.items()}
+    S = dd["S0"].clone()
+    out, _, _, S = wkv7.layer_forward(dd["x"], dd, 12, last_x=dd["last_x"], v0=dd["v0"], S=S)
+    assert _out_err(out, out_ref, 12) <= TOL_LAYER["bf16"]
+    assert state_err(S, S_ref) <= TOL_LAYER["bf16"]
