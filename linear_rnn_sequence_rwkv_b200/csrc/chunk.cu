@@ -317,6 +317,22 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         const bool to = ft == 0 && !mbar_wait_spin(&S.bar_tma, tma_parity, p.timeout_ns);
         tma_parity ^= 1u;
         if (bar_named_or(BAR_FRONT, kFrontThreads, to)) return true;
+        if (RAW) {
+            // P0: the decay multipliers w = exp(-sigmoid(z)/sqrt(e)) of the whole tile into the decay
+            //     table's rows, four channels per item over all front threads (independent items,
+            //     so the transcendental latencies overlap), before the products run over them
+            for (int it = ft; it < C * 16; it += kFrontThreads) {
+                const int t = it >> 4, j0 = (it & 15) * 4;
+                const uint2 u = *reinterpret_cast<const uint2 *>(IN + XW * 8192 + t * 128 +
+                                                                 ((((j0 >> 3) ^ (t & 7))) << 4) + (j0 & 4) * 2);
+                const float z[4] = {bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y)};
+                float wv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) wv[e] = __expf(__fdividef(-0.60653065971263342f, 1.f + __expf(-z[e])));
+                *reinterpret_cast<float4 *>(GT + (t + 1) * GTS + j0) = make_float4(wv[0], wv[1], wv[2], wv[3]);
+            }
+            bar_named(BAR_FRONT, kFrontThreads);
+        }
         // P1: decay products per key channel j over each quarter of the chunk (256 threads)
         if (ft < 256) {
             const int j = ft & 63, q = ft >> 6;
@@ -329,8 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int t = 16 * q + 8 * h8 + e;
-                    float w = in_col(wt, t, xo, e);
-                    if (RAW) w = __expf(__fdividef(-0.60653065971263342f, 1.f + __expf(-w)));   // exp(-sigmoid(z)/sqrt(e))
+                    const float w = RAW ? GT[(t + 1) * GTS + j] : in_col(wt, t, xo, e);
                     run *= (t < Lc) ? w : 1.f;   // padded tokens: w = 1
                     GT[(t + 1) * GTS + j] = run;
                 }
