@@ -63,7 +63,7 @@ extern "C" {
 typedef enum wkv7_status {
     WKV7_OK = 0,
     WKV7_ERR_ARG = 1,          /* null / host / too-small pointer, bad size or option   */
-    WKV7_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement (N not 64 or 128,
+    WKV7_ERR_UNSUPPORTED = 2,  /* valid request the library does not implement (N not 64 or 128,
                                   or 128 on a path that takes 64 only) */
     WKV7_ERR_ALIGN = 3,        /* a pointer is not 16-byte aligned                       */
     WKV7_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed                    */

@@ -13,7 +13,7 @@ Sources (RWKV-7 "Goose"):
   a per-channel affine) and the bonus term sum_j(r_j k_j r_k[j]) * v added after the
   norm: same listing, the ``group_norm`` lambda and the two lines after the readout.
 
-Readings taken where the pages leave a step open (each listed in the design doc):
+Readings taken where the pages leave a step open:
 * S is N x N with row i = value channel, column j = key channel (with the listing's
   column vectors the decay multiplies the key columns and the readout contracts the
   key index).
