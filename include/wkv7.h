@@ -250,7 +250,8 @@ WKV7_API wkv7_status wkv7_backward_static(int B, int T, int H, int N, wkv7_dtype
  * opts: algorithm, chunk, segments and snapshots of the recurrence (its epilogue fields are
  *       replaced by params'); NULL = defaults.
  * Workspace: wkv7_layer_workspace_bytes(B, T, dt, dims) bytes, not overlapping any argument.
- * Errors: WKV7_ERR_ARG (sizes, NULL required pointers, C != H * N), WKV7_ERR_ALIGN (every
+ * Errors: WKV7_ERR_ARG (sizes, NULL dims / params / required pointers, overlapping outputs,
+ * host or too-small buffers, v0 without Wv1 / Wv2 / v_bias), WKV7_ERR_ALIGN (every
  * pointer 16-byte aligned), WKV7_ERR_UNSUPPORTED (N), WKV7_ERR_WORKSPACE, WKV7_ERR_CUDA (a launch
  * or a cuBLASLt call failed; the message names the step). T = 0 only copies last_x.
  */
