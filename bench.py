@@ -59,15 +59,39 @@ PROFILE_TAGS = {"prefill-0.19b": "prefill-0.19B", "prefill-1.5b": "prefill-1.5B"
                 "long-context": "long-context", "decode": "decode-2.9B"}
 
 
+def _strip_comments(text: str) -> str:
+    """C/C++ source without its comments and blank lines (string and character literals kept),
+    so that a comment edit does not count as a change of the compiled code."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            i = text.find("\n", i)
+            i = n if i < 0 else i
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return "\n".join(l.rstrip() for l in "".join(out).splitlines() if l.strip())
+
+
 def kernel_digest(kernel: str) -> str:
     """sha256 (16 hex digits) of the device code a kernel is built from: its .cu file up to the
-    host-side section, plus the headers it includes."""
+    host-side section, plus the headers it includes, comments removed."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "linear_rnn_sequence_rwkv_b200", "csrc", f)) as fh:
             text = fh.read()
         cut = text.find("// ---- host side")
-        h.update((text if cut < 0 else text[:cut]).encode())
+        h.update(_strip_comments(text if cut < 0 else text[:cut]).encode())
     return h.hexdigest()[:16]
 
 

@@ -2,8 +2,8 @@
 // with the state carried from chunk to chunk in fp32.
 //
 // The recurrence (RWKV-7 rebuttal page, numpy time_mixing listing, update and
-// readout lines; the paper summary, section 4: the transition stays "diagonal plus
-// rank one", which keeps the model parallelisable over time) is, per (b, h),
+// readout lines; the paper summary, section 4: the transition is a diagonal matrix plus a
+// rank-one one, so products over time can be formed in parallel) is, per (b, h),
 //     S_t = S_{t-1} diag(w_t) + u_t b_t^T + v_t k_t^T,  u_t = -S_{t-1} kk_t,  b_t = kk_t*a_t,
 //     y_t = S_t r_t.
 // Over a chunk of C tokens with start state S_0, let g_t = prod_{s<=t} w_s (per key

@@ -207,7 +207,7 @@ __device__ __forceinline__ uint64_t kstep_off(int ks, int rows) {
 }
 
 // ---- MN-major operand layout (128-byte swizzle, tf32) ----------------------------------------------
-// A K x MN operand stored "MN-major": for each K index (a "row" here) 32 consecutive MN elements
+// A K x MN operand stored MN-major: for each K index (a row here) 32 consecutive MN elements
 // fill one 128-byte line; 8 consecutive K rows form a 1024-byte swizzle atom (16-byte chunk c of
 // row r at chunk position c ^ (r % 8)). Atoms of successive K groups are MN_SBO bytes apart and
 // blocks of 32 MN elements are `kdim/8 * 1024` bytes apart. A thread owning one K row writes its
