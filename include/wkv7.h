@@ -246,7 +246,7 @@ WKV7_API wkv7_status wkv7_backward_static(int B, int T, int H, int N, wkv7_dtype
  * v0      [B][T][C] dt: the first layer's values; NULL means this is the first layer.
  * S       [B][H][N][N] fp32, read and updated in place (NULL: zero state, not returned).
  * out     [B][T][C] fp32.   v0_out [B][T][C] dt or NULL: receives v when v0 is NULL.
- * last_x_out [B][C] dt or NULL: receives x[:, T-1].
+ * last_x_out [B][C] dt or NULL: receives x[:, T-1]; may be last_x itself (in place).
  * opts: algorithm, chunk, segments and snapshots of the recurrence (its epilogue fields are
  *       replaced by params'); NULL = defaults.
  * Workspace: wkv7_layer_workspace_bytes(B, T, dt, dims) bytes, not overlapping any argument.

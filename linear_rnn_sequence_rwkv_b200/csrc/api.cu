@@ -474,8 +474,12 @@ wkv7_status wkv7_layer_forward(int B, int T, wkv7_dtype dt, const wkv7_layer_dim
                         {"workspace", workspace, need}};
     const Buf ins[] = {{"x", x, mc * e}, {"last_x", last_x, bc * e}, {"v0", v0, mc * e}};
     for (const Buf &o : outs) {
-        for (const Buf &i : ins)
+        for (const Buf &i : ins) {
+            // last_x_out == last_x in place is allowed: last_x is read by the first kernel,
+            // x[:, T-1] is written by the last one
+            if (o.ptr == last_x_out && i.ptr == last_x && last_x_out == last_x) continue;
             if (overlaps(o, i)) return fail(WKV7_ERR_ARG, "%s overlaps %s", o.name, i.name);
+        }
         for (const Buf &o2 : outs)
             if (&o2 != &o && overlaps(o, o2)) return fail(WKV7_ERR_ARG, "%s overlaps %s", o.name, o2.name);
     }

@@ -98,3 +98,14 @@ def test_layer_bench_shape_bf16(cuda_device):
     out, _, _, S = wkv7.layer_forward(dd["x"], dd, 12, last_x=dd["last_x"], v0=dd["v0"], S=S)
     assert _out_err(out, out_ref, 12) <= TOL_LAYER["bf16"]
     assert state_err(S, S_ref) <= TOL_LAYER["bf16"]
+
+
+def test_layer_previous_token_in_place(cuda_device):
+    """last_x_out may be last_x itself: the next call's previous token is updated in place."""
+    d, (out_ref, _, last_ref, _) = _case(2, 20, 4, "f32", False, seed=990)
+    dd = {k: (None if v is None else v.to(cuda_device)) for k, v in d.items()}
+    last = dd["last_x"].clone()
+    out, _, last_out, _ = wkv7.layer_forward(dd["x"], dd, 4, last_x=last, v0=dd["v0"], S=dd["S0"].clone(),
+                                             last_x_out=last)
+    assert last_out is last and torch.equal(last.cpu(), d["x"][:, -1])
+    assert _out_err(out, out_ref, 4) <= TOL_LAYER["f32"]
