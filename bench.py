@@ -60,8 +60,8 @@ PROFILE_TAGS = {"prefill-0.19b": "prefill-0.19B", "prefill-1.5b": "prefill-1.5B"
 
 
 def _strip_comments(text: str) -> str:
-    """C/C++ source without its comments and blank lines (string and character literals kept),
-    so that a comment edit does not count as a change of the compiled code."""
+    """C/C++ source without its comments, blank lines and indentation (string and character
+    literals kept), so that a comment edit does not count as a change of the compiled code."""
     out, i, n = [], 0, len(text)
     while i < n:
         c = text[i]
@@ -80,7 +80,7 @@ def _strip_comments(text: str) -> str:
         else:
             out.append(c)
             i += 1
-    return "\n".join(l.rstrip() for l in "".join(out).splitlines() if l.strip())
+    return "\n".join(l.strip() for l in "".join(out).splitlines() if l.strip())
 
 
 def kernel_digest(kernel: str) -> str:
