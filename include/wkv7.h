@@ -210,8 +210,10 @@ WKV7_API size_t wkv7_backward_workspace_bytes(int B, int T, int H, int N, int sn
  * Nothing in the scratch needs to start at zero (every checkpoint is written before it is read).
  * The scratch is shared by every call on a device: calls that may overlap in time (different
  * streams, or host threads without ordering between them) race on it and corrupt each other's
- * results; order such calls on one stream. Arguments, outputs and errors otherwise as
- * wkv7_backward.
+ * results; order such calls on one stream. The first call on a device looks up the scratch's
+ * device address (make it before any stream capture); the address is kept for later calls
+ * and belongs to that device's context, so it is not valid after cudaDeviceReset. Arguments,
+ * outputs and errors otherwise as wkv7_backward.
  */
 WKV7_API wkv7_status wkv7_backward_static(int B, int T, int H, int N, wkv7_dtype dt,
                           const void *r, const void *w, const void *k, const void *v,

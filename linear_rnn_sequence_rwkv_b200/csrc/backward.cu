@@ -328,11 +328,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs p) {
     if (p.dS0) store_rows(p.dS0 + size_t(unit) * kN * kN, d);
 }
 
+// ---- host side ---------------------------------------------------------------------------------------
+
 template <class Tin>
 cudaError_t launch_bwd_t(const BwdArgs &p) {
     const int smem = int(sizeof(BwdSmem));
-    static const cudaError_t attr =
-        cudaFuncSetAttribute(bwd_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const cudaError_t attr = allow_dynamic_smem(reinterpret_cast<const void *>(bwd_kernel<Tin>), smem);
     if (attr != cudaSuccess) return attr;
     bwd_kernel<Tin><<<p.B * p.H, kBwdThreads, smem, p.stream>>>(p);
     return cudaGetLastError();
@@ -348,19 +349,25 @@ size_t backward_checkpoint_bytes(int B, int T, int H, int snap_every) {
 
 size_t backward_static_scratch_bytes() { return kStaticScratchBytes; }
 
-// Device address of the static scratch on the current device, looked up once per device.
+// Device address of the static scratch on the current device. A successful lookup is kept per
+// device; a failed one is not, so the next call tries again. The kept address belongs to the
+// device's current context and is not valid after cudaDeviceReset.
 cudaError_t backward_static_scratch(void **ptr) {
     constexpr int kMaxDevices = 64;
-    static std::once_flag once[kMaxDevices];
+    static std::mutex mu;
     static void *addr[kMaxDevices];
-    static cudaError_t err[kMaxDevices];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::call_once(once[dev], [dev] { err[dev] = cudaGetSymbolAddress(&addr[dev], g_bwd_scratch); });
+    std::lock_guard<std::mutex> lk(mu);
+    if (!addr[dev]) {
+        void *a = nullptr;
+        if ((e = cudaGetSymbolAddress(&a, g_bwd_scratch)) != cudaSuccess) return e;
+        addr[dev] = a;
+    }
     *ptr = addr[dev];
-    return err[dev];
+    return cudaSuccess;
 }
 
 cudaError_t launch_backward(const BwdArgs &p) {

@@ -80,6 +80,10 @@ cudaError_t launch_chunk(const FwdArgs &p);        // chunked prefill on tcgen05
 cudaError_t chunk_segments(const FwdArgs &p, int *segments, int *launches = nullptr);
 // Synchronises `stream` and reads the device error word (bounded waits that gave up).
 cudaError_t read_device_error(cudaStream_t stream, unsigned int *value, bool clear);
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` on the current device. The attribute
+// belongs to the device's context, so it is set once per (device, kernel); failures are not
+// remembered (the next call tries again).
+cudaError_t allow_dynamic_smem(const void *kernel, int bytes);
 
 // ---- device helpers -------------------------------------------------------------------------
 

@@ -246,11 +246,13 @@ __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const FwdArgs p) {
     }
 }
 
+// ---- host side ---------------------------------------------------------------------------------------
+
 template <class Tin, int RPT, bool RAW, int NN>
 cudaError_t launch_seq_t(const FwdArgs &p) {
     const size_t smem = sizeof(SeqSmem<Tin, RPT, NN>);
-    static cudaError_t attr = cudaFuncSetAttribute(seq_kernel<Tin, RPT, RAW, NN>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    const cudaError_t attr =
+        allow_dynamic_smem(reinterpret_cast<const void *>(seq_kernel<Tin, RPT, RAW, NN>), int(smem));
     if (attr != cudaSuccess) return attr;
     dim3 grid(p.B * p.H, NN / (16 * RPT));
     seq_kernel<Tin, RPT, RAW, NN><<<grid, kSeqThreads, smem, p.stream>>>(p);

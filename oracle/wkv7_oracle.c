@@ -147,3 +147,166 @@ int wkv7_oracle_epilogue(int B, int T, int H, int N, const double *y,
     }
     return 0;
 }
+
+/*
+ * One RWKV-7 time-mixing layer, a second transcription independent of the numpy oracle:
+ * the rebuttal page's numpy time_mixing listing taken one token at a time with plain loops,
+ * every vector 1-D of length C = H * N and every step in the listing's order:
+ *   token-shift mixes x_m = x + m (x_prev - x);
+ *   r = Wr x_r (W stored [out][in]);
+ *   w = exp(-sigmoid(tanh(x_w Ww1) Ww2 + w_bias) / sqrt(e)) (low-rank factors [in][out]);
+ *   k = Wk x_k, v = Wv x_v;
+ *   first layer: v0 = v; later layers: v += (v0 - v) sigmoid(x_v Wv1 Wv2 + v_bias);
+ *   a = sigmoid(x_a Wa1 Wa2 + a_bias); g = sigmoid(x_g Wg1) Wg2;
+ *   kk = k * k_k; k += k (a - 1) k_a; kk normalised per head (floor 1e-12 on the norm);
+ *   S = S diag(w) - (S kk)(kk a)^T + v k^T per head; y = S r;
+ *   group_norm per head (population variance, eps inside the root), * ln_w + ln_b;
+ *   y += (sum_j r_j k_j r_k_j) v per head; out = Wo (y * g).
+ * Layouts: x, v0, out, v0_out [B][T][C]; last_x, last_out [B][C]; S0, S_T [B][H][N][N];
+ * square projections [C][C]; Ww1 [C][dw], Ww2 [dw][C] and likewise for a, v, g;
+ * mixes and biases [C]; r_k, k_k, k_a, ln_w, ln_b [H][N] (= [C]). last_x, v0, S0 may be NULL
+ * (zeros / first layer / zero state; Wv1, Wv2, v_bias are then unused). Single-threaded.
+ * Returns 0, -1 on bad arguments, -2 on allocation failure.
+ */
+static double sigm(double z) { return 1.0 / (1.0 + exp(-z)); }
+
+int wkv7_oracle_layer(int B, int T, int H, int N, int dw, int da, int dv, int dg,
+                      const double *x, const double *last_x, const double *v0, const double *S0,
+                      const double *mr, const double *mw, const double *mk, const double *mv,
+                      const double *ma, const double *mg, const double *w_bias, const double *a_bias,
+                      const double *v_bias, const double *r_k, const double *k_k, const double *k_a,
+                      const double *ln_w, const double *ln_b, const double *Wr, const double *Wk,
+                      const double *Wv, const double *Wo, const double *Ww1, const double *Ww2,
+                      const double *Wa1, const double *Wa2, const double *Wv1, const double *Wv2,
+                      const double *Wg1, const double *Wg2, double eps,
+                      double *out, double *v0_out, double *last_out, double *S_T) {
+    if (B < 0 || T < 0 || H <= 0 || N <= 0 || dw <= 0 || da <= 0 || dv <= 0 || dg <= 0 || !x || !out ||
+        !v0_out || !last_out || !S_T)
+        return -1;
+    const int C = H * N;
+    const int dmax = dw > da ? (dw > dv ? (dw > dg ? dw : dg) : (dv > dg ? dv : dg))
+                             : (da > dv ? (da > dg ? da : dg) : (dv > dg ? dv : dg));
+    double *buf = (double *)malloc(sizeof(double) * ((size_t)C * 17 + dmax));
+    if (!buf) return -2;
+    double *xp = buf, *xr = xp + C, *xw = xr + C, *xk = xw + C, *xv = xk + C, *xa = xv + C, *xg = xa + C;
+    double *r = xg + C, *w = r + C, *k = w + C, *v = k + C, *a = v + C, *g = a + C, *kk = g + C;
+    double *y = kk + C, *tmp = y + C, *sk = tmp + C, *hid = sk + C;
+    const double *mixes[6] = {mr, mw, mk, mv, ma, mg};
+    double *xs[6] = {xr, xw, xk, xv, xa, xg};
+    for (int b = 0; b < B; ++b) {
+        double *Sb = S_T + (size_t)b * H * N * N;
+        for (size_t e = 0; e < (size_t)H * N * N; ++e) Sb[e] = S0 ? S0[(size_t)b * H * N * N + e] : 0.0;
+        for (int c = 0; c < C; ++c) xp[c] = last_x ? last_x[(size_t)b * C + c] : 0.0;
+        for (int t = 0; t < T; ++t) {
+            const double *xt = x + ((size_t)b * T + t) * C;
+            for (int m = 0; m < 6; ++m)
+                for (int c = 0; c < C; ++c) xs[m][c] = xt[c] + mixes[m][c] * (xp[c] - xt[c]);
+            for (int o = 0; o < C; ++o) {   /* square projections: W @ x */
+                double sr = 0.0, sk2 = 0.0, sv = 0.0;
+                for (int i = 0; i < C; ++i) {
+                    sr += Wr[(size_t)o * C + i] * xr[i];
+                    sk2 += Wk[(size_t)o * C + i] * xk[i];
+                    sv += Wv[(size_t)o * C + i] * xv[i];
+                }
+                r[o] = sr;
+                k[o] = sk2;
+                v[o] = sv;
+            }
+            /* decay: hidden = tanh(x_w @ Ww1), logit = hidden @ Ww2 + w_bias */
+            for (int d = 0; d < dw; ++d) {
+                double s = 0.0;
+                for (int c = 0; c < C; ++c) s += xw[c] * Ww1[(size_t)c * dw + d];
+                hid[d] = tanh(s);
+            }
+            for (int c = 0; c < C; ++c) {
+                double s = w_bias[c];
+                for (int d = 0; d < dw; ++d) s += hid[d] * Ww2[(size_t)d * C + c];
+                w[c] = exp(-sigm(s) / sqrt(exp(1.0)));
+            }
+            double *v0t = v0_out + ((size_t)b * T + t) * C;
+            if (!v0) {
+                for (int c = 0; c < C; ++c) v0t[c] = v[c];
+            } else {
+                const double *v0i = v0 + ((size_t)b * T + t) * C;
+                for (int d = 0; d < dv; ++d) {
+                    double s = 0.0;
+                    for (int c = 0; c < C; ++c) s += xv[c] * Wv1[(size_t)c * dv + d];
+                    hid[d] = s;
+                }
+                for (int c = 0; c < C; ++c) {
+                    double s = v_bias[c];
+                    for (int d = 0; d < dv; ++d) s += hid[d] * Wv2[(size_t)d * C + c];
+                    v[c] += (v0i[c] - v[c]) * sigm(s);
+                    v0t[c] = v0i[c];
+                }
+            }
+            for (int d = 0; d < da; ++d) {   /* rate: no activation between the two factors */
+                double s = 0.0;
+                for (int c = 0; c < C; ++c) s += xa[c] * Wa1[(size_t)c * da + d];
+                hid[d] = s;
+            }
+            for (int c = 0; c < C; ++c) {
+                double s = a_bias[c];
+                for (int d = 0; d < da; ++d) s += hid[d] * Wa2[(size_t)d * C + c];
+                a[c] = sigm(s);
+            }
+            for (int d = 0; d < dg; ++d) {   /* gate: sigmoid on the hidden value, then Wg2 */
+                double s = 0.0;
+                for (int c = 0; c < C; ++c) s += xg[c] * Wg1[(size_t)c * dg + d];
+                hid[d] = sigm(s);
+            }
+            for (int c = 0; c < C; ++c) {
+                double s = 0.0;
+                for (int d = 0; d < dg; ++d) s += hid[d] * Wg2[(size_t)d * C + c];
+                g[c] = s;
+            }
+            for (int c = 0; c < C; ++c) kk[c] = k[c] * k_k[c];
+            for (int c = 0; c < C; ++c) k[c] += k[c] * (a[c] - 1.0) * k_a[c];
+            for (int h = 0; h < H; ++h) {
+                double ss = 0.0;
+                for (int j = 0; j < N; ++j) ss += kk[h * N + j] * kk[h * N + j];
+                double nrm = sqrt(ss);
+                if (nrm < 1e-12) nrm = 1e-12;
+                for (int j = 0; j < N; ++j) kk[h * N + j] /= nrm;
+            }
+            for (int h = 0; h < H; ++h) {
+                double *Sh = Sb + (size_t)h * N * N;
+                const double *wh = w + h * N, *kh = k + h * N, *vh = v + h * N, *kkh = kk + h * N;
+                const double *ah = a + h * N, *rh = r + h * N;
+                for (int i = 0; i < N; ++i) {
+                    double s = 0.0;
+                    for (int j = 0; j < N; ++j) s += Sh[i * N + j] * kkh[j];
+                    sk[i] = s;
+                }
+                for (int i = 0; i < N; ++i)
+                    for (int j = 0; j < N; ++j)
+                        Sh[i * N + j] = Sh[i * N + j] * wh[j] - sk[i] * (kkh[j] * ah[j]) + vh[i] * kh[j];
+                for (int i = 0; i < N; ++i) {
+                    double s = 0.0;
+                    for (int j = 0; j < N; ++j) s += Sh[i * N + j] * rh[j];
+                    y[h * N + i] = s;
+                }
+                double mean = 0.0, var = 0.0, bonus = 0.0;
+                for (int i = 0; i < N; ++i) mean += y[h * N + i];
+                mean /= N;
+                for (int i = 0; i < N; ++i) var += (y[h * N + i] - mean) * (y[h * N + i] - mean);
+                var /= N;
+                for (int i = 0; i < N; ++i)
+                    y[h * N + i] = (y[h * N + i] - mean) / sqrt(var + eps) * ln_w[h * N + i] + ln_b[h * N + i];
+                for (int j = 0; j < N; ++j) bonus += rh[j] * kh[j] * r_k[h * N + j];
+                for (int i = 0; i < N; ++i) y[h * N + i] += bonus * vh[i];
+            }
+            for (int c = 0; c < C; ++c) tmp[c] = y[c] * g[c];
+            double *ot = out + ((size_t)b * T + t) * C;
+            for (int o = 0; o < C; ++o) {
+                double s = 0.0;
+                for (int i = 0; i < C; ++i) s += Wo[(size_t)o * C + i] * tmp[i];
+                ot[o] = s;
+            }
+            for (int c = 0; c < C; ++c) xp[c] = xt[c];
+        }
+        for (int c = 0; c < C; ++c) last_out[(size_t)b * C + c] = xp[c];
+    }
+    free(buf);
+    return 0;
+}

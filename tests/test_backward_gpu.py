@@ -118,9 +118,11 @@ def test_backward_prefill_019b_sampled_heads(cuda_device):
     _check(sel, ref)
 
 
-def test_backward_matches_finite_difference_of_the_gpu_forward(cuda_device):
-    """A directional derivative of the GPU forward (fp32 scan, central difference along a
-    random direction of every input) equals the GPU gradients contracted with it."""
+def test_gpu_gradients_match_finite_difference_of_the_oracle_forward(cuda_device):
+    """A directional derivative of the oracle's fp64 forward (central difference along a
+    random direction of every input) equals the GPU gradients contracted with that direction.
+    The fp64 oracle is differentiated, not the GPU forward: an fp32 forward's rounding would
+    swamp a central difference."""
     d = _case(1, 24, 2, dtype="f32", seed=560)
     dd = _dev(d, cuda_device)
     got = wkv7.backward(*(dd[n] for n in NAMES), dd["dy"], dd["S0"], dd["dS_T"])

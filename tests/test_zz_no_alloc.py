@@ -49,3 +49,37 @@ def test_static_entry_matches_workspace_entry_on_consecutive_calls(cuda_device, 
                             snap_every=snap_every)
         for n in wkv7.GRAD_NAMES + ("dS0",):
             assert torch.equal(got[n], ref[n]), n
+
+
+@pytest.mark.gpu
+def test_static_entry_takes_no_device_memory(cuda_device):
+    """With every argument allocated up front, further calls leave the device's free memory
+    unchanged: the entry itself allocates nothing (its scratch is part of the loaded module)."""
+    B, T, H = 2, 200, 3
+    d = {k: (None if v is None else v.to(cuda_device)) for k, v in _case(B, T, H, 950).items()}
+    grads = {n: torch.empty(B, T, H, 64, device=cuda_device) for n in wkv7.GRAD_NAMES}
+    dS0 = torch.empty(B, H, 64, 64, device=cuda_device)
+    call = lambda: wkv7.backward_static(*(d[n] for n in NAMES), d["dy"], d["S0"], d["dS_T"], grads=grads,
+                                        dS0=dS0)
+    call()                                   # first call on the device: the scratch address lookup
+    torch.cuda.synchronize(cuda_device)
+    free0 = torch.cuda.mem_get_info(cuda_device)[0]
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(cuda_device)
+    assert torch.cuda.mem_get_info(cuda_device)[0] == free0
+
+
+@pytest.mark.gpu
+def test_static_and_workspace_entries_on_a_second_device(cuda_device):
+    """Kernel attributes and the scratch address are per device: the backward runs on device 1
+    after device 0 in the same process (skipped with one visible device)."""
+    if torch.cuda.device_count() < 2:
+        pytest.skip("one visible CUDA device")
+    B, T, H = 1, 130, 2
+    for dev in (torch.device("cuda:0"), torch.device("cuda:1")):
+        d = {k: (None if v is None else v.to(dev)) for k, v in _case(B, T, H, 960).items()}
+        got = wkv7.backward_static(*(d[n] for n in NAMES), d["dy"], d["S0"], d["dS_T"])
+        ref = wkv7.backward(*(d[n] for n in NAMES), d["dy"], d["S0"], d["dS_T"])
+        for n in wkv7.GRAD_NAMES + ("dS0",):
+            assert torch.equal(got[n], ref[n]), (dev, n)
