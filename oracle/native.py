@@ -43,6 +43,8 @@ def _load():
             lib.wkv7_oracle_forward.restype = ctypes.c_int
             lib.wkv7_oracle_epilogue.argtypes = [ctypes.c_int] * 4 + [d] * 7 + [ctypes.c_double, d]
             lib.wkv7_oracle_epilogue.restype = ctypes.c_int
+            lib.wkv7_oracle_layer.argtypes = [ctypes.c_int] * 8 + [d] * 30 + [ctypes.c_double] + [d] * 4
+            lib.wkv7_oracle_layer.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -89,3 +91,31 @@ def epilogue(y, r, k, v, ln_w, ln_b, r_k, eps=64e-5):
     if rc != 0:
         raise RuntimeError(f"wkv7_oracle_epilogue failed with {rc}")
     return out
+
+
+_LAYER_ORDER = ("mr", "mw", "mk", "mv", "ma", "mg", "w_bias", "a_bias", "v_bias", "r_k", "k_k", "k_a", "ln_w",
+                "ln_b", "Wr", "Wk", "Wv", "Wo", "Ww1", "Ww2", "Wa1", "Wa2", "Wv1", "Wv2", "Wg1", "Wg2")
+
+
+def time_mixing_layer(x, params, last_x=None, v0=None, S0=None, eps=64e-5):
+    """The C transcription of one time-mixing layer (wkv7_oracle_layer: the listing token by
+    token with plain loops). Same contract as reference.time_mixing_layer; k_a must be given."""
+    lib = _load()
+    P = {n: np.ascontiguousarray(_f64(params[n])) for n in _LAYER_ORDER}
+    xs = np.ascontiguousarray(_f64(x))
+    B, T, C = xs.shape
+    H, N = P["r_k"].shape
+    dims = [P[n].shape[1] for n in ("Ww1", "Wa1", "Wv1", "Wg1")]
+    lx = None if last_x is None else np.ascontiguousarray(_f64(last_x))
+    v0s = None if v0 is None else np.ascontiguousarray(_f64(v0))
+    s0 = None if S0 is None else np.ascontiguousarray(_f64(S0))
+    out = np.empty((B, T, C))
+    v0_out = np.empty((B, T, C))
+    last = np.empty((B, C))
+    S_T = np.empty((B, H, N, N))
+    rc = lib.wkv7_oracle_layer(B, T, H, N, *dims, _ptr(xs), _ptr(lx), _ptr(v0s), _ptr(s0),
+                               *(_ptr(P[n]) for n in _LAYER_ORDER), float(eps), _ptr(out), _ptr(v0_out),
+                               _ptr(last), _ptr(S_T))
+    if rc != 0:
+        raise RuntimeError(f"wkv7_oracle_layer failed with {rc}")
+    return out, v0_out, last, S_T

@@ -31,7 +31,12 @@ Readings taken where the pages leave a step open:
 
 Parity pins: every function here is pinned in tests/test_oracle.py against closed
 forms, brute-force transition products, the paper's elementary-transition
-constructions and a finite-difference SGD reading of the delta rule.
+constructions and a finite-difference SGD reading of the delta rule; the backward in
+tests/test_oracle_backward.py by finite differences; the layer (``layer_projections`` and
+``time_mixing_layer``) in tests/test_oracle_layer.py by a second transcription in plain C
+(oracle/wkv7_oracle.c, ``wkv7_oracle_layer``) and by properties of each activation (tanh
+saturation and slope on the decay path, linearity of the rate and value-residual paths
+between their factors, the gate's sigmoid limits, the orientation of the projections).
 """
 from __future__ import annotations
 
@@ -159,6 +164,39 @@ LAYER_PARAM_NAMES = ("mr", "mw", "mk", "mv", "ma", "mg", "w_bias", "a_bias", "v_
                      "ln_w", "ln_b", "Wr", "Wk", "Wv", "Wo", "Ww1", "Ww2", "Wa1", "Wa2", "Wv1", "Wv2", "Wg1", "Wg2")
 
 
+def layer_projections(x, P, last_x=None, v0=None):
+    """The per-token values one time-mixing layer feeds to its recurrence, in fp64 (the rebuttal
+    page's numpy ``time_mixing`` listing, from the token shift to the gate), for a whole
+    sequence at once.
+
+    x: [B, T, C]; P: dict of fp64 parameters as in ``time_mixing_layer``; last_x [B, C] or None
+    (zeros); v0 [B, T, C] or None (first layer). Returns a dict of [B, T, C] arrays: r, k, v (v
+    after the value residual), w_logit, a_logit, g, and v0 (the first layer's values). Per token,
+    with x_p the previous token (last_x for the first):
+      x_m = x + m (x_p - x) for the six mixes m
+      r = Wr x_r, k = Wk x_k, v = Wv x_v                      (W stored [out][in])
+      w_logit = tanh(x_w Ww1) Ww2 + w_bias                    (low-rank factors [in][out])
+      v <- v + (v0 - v) sigmoid(x_v Wv1 Wv2 + v_bias)         (layers after the first)
+      a_logit = x_a Wa1 Wa2 + a_bias                          (no activation between the factors)
+      g = sigmoid(x_g Wg1) Wg2
+    """
+    B, T, C = x.shape
+    prev = np.concatenate([np.zeros((B, 1, C)) if last_x is None else _f64(last_x)[:, None], x[:, :-1]], axis=1)
+    mix = {m: x + P[m] * (prev - x) for m in ("mr", "mw", "mk", "mv", "ma", "mg")}
+    sig = lambda z: 1.0 / (1.0 + np.exp(-z))
+    out = {"r": mix["mr"] @ P["Wr"].T, "k": mix["mk"] @ P["Wk"].T}
+    v = mix["mv"] @ P["Wv"].T
+    out["w_logit"] = np.tanh(mix["mw"] @ P["Ww1"]) @ P["Ww2"] + P["w_bias"]
+    if v0 is None:
+        v0 = v
+    else:
+        v = v + (_f64(v0) - v) * sig(mix["mv"] @ P["Wv1"] @ P["Wv2"] + P["v_bias"])
+    out["v"], out["v0"] = v, v0
+    out["a_logit"] = mix["ma"] @ P["Wa1"] @ P["Wa2"] + P["a_bias"]
+    out["g"] = sig(mix["mg"] @ P["Wg1"]) @ P["Wg2"]
+    return out
+
+
 def time_mixing_layer(x, params, last_x=None, v0=None, S0=None, eps=64e-5):
     """One RWKV-7 time-mixing layer over a sequence, in fp64 (the rebuttal page's numpy
     ``time_mixing`` listing, applied token after token with the state, the previous token
@@ -172,38 +210,22 @@ def time_mixing_layer(x, params, last_x=None, v0=None, S0=None, eps=64e-5):
     first layer (None: this is the first layer, and its own v is returned as v0).
     S0: [B, H, N, N] or None. Returns (out [B, T, C], v0 [B, T, C], last x [B, C], S_T).
 
-    Per token, with x_p the previous token (last_x for the first):
-      x_m = x + m (x_p - x) for the six mixes m
-      r = Wr x_r, k = Wk x_k, v = Wv x_v
-      w = exp(-sigmoid(tanh(x_w Ww1) Ww2 + w_bias) / sqrt(e))
-      v <- v + (v0 - v) sigmoid(x_v Wv1 Wv2 + v_bias)        (layers after the first)
-      a = sigmoid(x_a Wa1 Wa2 + a_bias), g = sigmoid(x_g Wg1) Wg2
-      kk = normalised (k * k_k) per head, k <- k + k (a - 1) k_a
-      the recurrence and readout per head, group_norm + bonus, out = Wo (y * g).
+    The per-token values come from ``layer_projections``; then the pre-processing
+    (w = exp(-sigmoid(w_logit) / sqrt(e)), a = sigmoid(a_logit), kk = normalised (k * k_k) per
+    head, k <- k + k (a - 1) k_a), the recurrence and readout per head, group_norm + bonus, and
+    out = Wo (y * g).
     """
     P = {n: _f64(params[n]) for n in LAYER_PARAM_NAMES}
     x = _f64(x)
     B, T, C = x.shape
     H, N = P["r_k"].shape
-    prev = np.concatenate([np.zeros((B, 1, C)) if last_x is None else _f64(last_x)[:, None], x[:, :-1]], axis=1)
-    mix = {m: x + P[m] * (prev - x) for m in ("mr", "mw", "mk", "mv", "ma", "mg")}
-    sig = lambda z: 1.0 / (1.0 + np.exp(-z))
-    r = mix["mr"] @ P["Wr"].T
-    k = mix["mk"] @ P["Wk"].T
-    v = mix["mv"] @ P["Wv"].T
-    w_logit = np.tanh(mix["mw"] @ P["Ww1"]) @ P["Ww2"] + P["w_bias"]
-    if v0 is None:
-        v0 = v
-    else:
-        v = v + (_f64(v0) - v) * sig(mix["mv"] @ P["Wv1"] @ P["Wv2"] + P["v_bias"])
-    a_logit = mix["ma"] @ P["Wa1"] @ P["Wa2"] + P["a_bias"]
-    g = sig(mix["mg"] @ P["Wg1"]) @ P["Wg2"]
-    heads = lambda z: z.reshape(B, T, H, N)
-    w, a, kk, k_t = prepare_inputs(heads(w_logit), heads(a_logit), heads(k), P["k_k"], P["k_a"])
-    y, S_T, _ = wkv7_recurrence(heads(r), w, k_t, heads(v), kk, a, S0)
-    y = group_norm_bonus(y, heads(r), k_t, heads(v), P["ln_w"], P["ln_b"], P["r_k"], eps)
-    out = (y.reshape(B, T, C) * g) @ P["Wo"].T
-    return out, v0, x[:, -1].copy(), S_T
+    z = layer_projections(x, P, last_x, v0)
+    heads = lambda u: u.reshape(B, T, H, N)
+    w, a, kk, k_t = prepare_inputs(heads(z["w_logit"]), heads(z["a_logit"]), heads(z["k"]), P["k_k"], P["k_a"])
+    y, S_T, _ = wkv7_recurrence(heads(z["r"]), w, k_t, heads(z["v"]), kk, a, S0)
+    y = group_norm_bonus(y, heads(z["r"]), k_t, heads(z["v"]), P["ln_w"], P["ln_b"], P["r_k"], eps)
+    out = (y.reshape(B, T, C) * z["g"]) @ P["Wo"].T
+    return out, z["v0"], x[:, -1].copy(), S_T
 
 
 def transition_matrix(w_t, kk_t, a_t):

@@ -20,6 +20,8 @@
  * [B][T/snap_every][H][N][N]; epilogue parameters [H][N]. All fp64.
  * Units (b, h) are independent and are spread over POSIX threads; within a unit
  * the token loop runs in order, so the result does not depend on the thread count.
+ * wkv7_oracle_layer (at the end) is a second, independent transcription of the whole
+ * time-mixing layer, against which the numpy layer is checked.
  */
 #include <math.h>
 #include <pthread.h>

@@ -91,3 +91,90 @@ def test_sequence_split_carries_state_and_previous_token(T1):
     np.testing.assert_allclose(np.concatenate([a[0], b[0]], axis=1), out, rtol=0, atol=1e-12)
     np.testing.assert_allclose(b[3], S_T, rtol=0, atol=1e-12)
     np.testing.assert_array_equal(b[2], last)
+
+
+# ---- second transcription and the activations of the low-rank paths ----------------------------
+
+from oracle import native  # noqa: E402
+
+
+@pytest.mark.parametrize("first,with_last,with_s0", [(True, True, True), (False, True, True), (False, False, False)])
+def test_numpy_layer_matches_the_c_transcription(first, with_last, with_s0):
+    """The numpy layer (whole sequences at once) equals the plain-C transcription of the
+    listing (one token at a time, plain loops) with every low-rank factor non-zero."""
+    d = _layer(B=2, T=5, H=2, N=4, seed=11 + int(first), first=first)
+    p = {n: d[n] for n in P_NAMES}
+    args = (d["x"], p, d["last_x"] if with_last else None, d["v0"], d["S0"] if with_s0 else None)
+    a = reference.time_mixing_layer(*args)
+    b = native.time_mixing_layer(*args)
+    for u, v, name in zip(a, b, ("out", "v0", "last_x", "S_T")):
+        np.testing.assert_allclose(u, v, rtol=0, atol=1e-11 * max(1.0, np.max(np.abs(v))), err_msg=name)
+
+
+def _proj(d, **over):
+    P = {n: over.get(n, d[n]) for n in P_NAMES}
+    return reference.layer_projections(over.get("x", d["x"]), P, over.get("last_x", d["last_x"]),
+                                       over.get("v0", d["v0"]))
+
+
+def _mixed(d, m):
+    prev = np.concatenate([d["last_x"][:, None], d["x"][:, :-1]], axis=1)
+    return d["x"] + d[m] * (prev - d["x"])
+
+
+def test_decay_path_is_tanh_between_its_factors():
+    """tanh saturates at +-1 for a large first factor, so the logit minus its bias becomes
+    sign(x_w Ww1) Ww2; for a tiny first factor tanh is the identity to first order."""
+    d = _layer()
+    xw = _mixed(d, "mw")
+    big = _proj(d, Ww1=1e4 * d["Ww1"])["w_logit"] - d["w_bias"]
+    np.testing.assert_allclose(big, np.sign(xw @ d["Ww1"]) @ d["Ww2"], rtol=0, atol=1e-9)
+    eps = 1e-6
+    small = (_proj(d, Ww1=eps * d["Ww1"])["w_logit"] - d["w_bias"]) / eps
+    np.testing.assert_allclose(small, (xw @ d["Ww1"]) @ d["Ww2"], rtol=0, atol=1e-6)
+
+
+def test_rate_path_is_linear_between_its_factors():
+    """Nothing sits between Wa1 and Wa2: the logit minus its bias is linear in Wa1."""
+    d = _layer()
+    base = _proj(d)["a_logit"] - d["a_bias"]
+    for alpha in (3.0, -2.0):
+        np.testing.assert_allclose(_proj(d, Wa1=alpha * d["Wa1"])["a_logit"] - d["a_bias"], alpha * base,
+                                   rtol=0, atol=1e-12)
+    np.testing.assert_allclose(base, _mixed(d, "ma") @ d["Wa1"] @ d["Wa2"], rtol=0, atol=1e-12)
+
+
+def test_value_residual_path_is_linear_between_its_factors():
+    """The residual's mixing weight is sigmoid(x_v Wv1 Wv2 + v_bias): recovered from v, v0 and
+    the first-layer v, its logit minus the bias is x_v Wv1 Wv2 (no activation in between)."""
+    d = _layer()
+    v_lin = _proj(d, v0=None)["v"]
+    got = _proj(d)
+    lam = (got["v"] - v_lin) / (d["v0"] - v_lin)
+    logit = np.log(lam / (1.0 - lam))
+    np.testing.assert_allclose(logit - d["v_bias"], _mixed(d, "mv") @ d["Wv1"] @ d["Wv2"], rtol=0, atol=1e-8)
+
+
+def test_gate_is_sigmoid_of_the_hidden_value_then_the_second_factor():
+    """g = sigmoid(x_g Wg1) Wg2: with Wg1 = 0 every hidden unit is 1/2; with a large Wg1 the
+    hidden units become the step of x_g Wg1."""
+    d = _layer()
+    g0 = _proj(d, Wg1=np.zeros_like(d["Wg1"]))["g"]
+    np.testing.assert_allclose(g0, np.broadcast_to(0.5 * d["Wg2"].sum(axis=0), g0.shape), rtol=0, atol=1e-14)
+    gb = _proj(d, Wg1=1e4 * d["Wg1"])["g"]
+    np.testing.assert_allclose(gb, (_mixed(d, "mg") @ d["Wg1"] > 0) @ d["Wg2"], rtol=0, atol=1e-9)
+
+
+def test_square_projections_take_the_stored_row_as_output_channel():
+    """W x with W stored [out][in]: a one-hot token at channel i (no mixing, first layer) gives
+    column i of Wr, Wk and Wv; the matrices are not symmetric, so a transposed use fails."""
+    d = _layer(B=1, T=1)
+    C = d["x"].shape[-1]
+    i = 3
+    x = np.zeros((1, 1, C))
+    x[0, 0, i] = 1.0
+    zero = {m: np.zeros(C) for m in ("mr", "mw", "mk", "mv", "ma", "mg")}
+    z = _proj(d, x=x, last_x=np.zeros((1, C)), v0=None, **zero)
+    for name, W in (("r", "Wr"), ("k", "Wk"), ("v", "Wv")):
+        assert np.max(np.abs(d[W] - d[W].T)) > 1e-3
+        np.testing.assert_allclose(z[name][0, 0], d[W][:, i], rtol=0, atol=1e-15)

@@ -234,12 +234,64 @@ LAYER_PINS = [
     PL.test_value_residual_limits,
     PL.test_linear_in_output_projection_and_gate_output_factor,
     lambda: PL.test_sequence_split_carries_state_and_previous_token(3),
+    lambda: PL.test_numpy_layer_matches_the_c_transcription(False, True, True),
+    lambda: PL.test_numpy_layer_matches_the_c_transcription(True, True, True),
+    PL.test_decay_path_is_tanh_between_its_factors,
+    PL.test_rate_path_is_linear_between_its_factors,
+    PL.test_value_residual_path_is_linear_between_its_factors,
+    PL.test_gate_is_sigmoid_of_the_hidden_value_then_the_second_factor,
+    PL.test_square_projections_take_the_stored_row_as_output_channel,
 ]
 
 
 @pytest.mark.parametrize("kind", ["mix_sign", "residual_sign", "gate_sigmoid_outside", "ignores_last_x"])
 def test_layer_mutant_is_caught(monkeypatch, kind):
     monkeypatch.setattr(reference, "time_mixing_layer", _layer_mutant(kind))
+    assert _failures(LAYER_PINS) >= 1
+
+
+def _projection_mutant(kind):
+    """reference.layer_projections with one activation or one operand orientation changed."""
+    def run(x, P, last_x=None, v0=None):
+        B, T, C = x.shape
+        prev = np.concatenate([np.zeros((B, 1, C)) if last_x is None else _f64(last_x)[:, None], x[:, :-1]], axis=1)
+        mix = {m: x + P[m] * (prev - x) for m in ("mr", "mw", "mk", "mv", "ma", "mg")}
+        sig = lambda z: 1.0 / (1.0 + np.exp(-z))
+        ident = lambda z: z
+        sq = (lambda xm, W: xm @ W) if kind == "transposed_square_projection" else (lambda xm, W: xm @ W.T)
+        out = {"r": sq(mix["mr"], P["Wr"]), "k": sq(mix["mk"], P["Wk"])}
+        v = sq(mix["mv"], P["Wv"])
+        act_w = {"decay_no_tanh": ident, "decay_sigmoid": sig}.get(kind, np.tanh)
+        out["w_logit"] = act_w(mix["mw"] @ P["Ww1"]) @ P["Ww2"] + P["w_bias"]
+        if v0 is None:
+            v0 = v
+        else:
+            act_v = np.tanh if kind == "residual_tanh" else ident
+            v = v + (_f64(v0) - v) * sig(act_v(mix["mv"] @ P["Wv1"]) @ P["Wv2"] + P["v_bias"])
+        out["v"], out["v0"] = v, v0
+        act_a = {"rate_tanh": np.tanh, "rate_sigmoid": sig}.get(kind, ident)
+        out["a_logit"] = act_a(mix["ma"] @ P["Wa1"]) @ P["Wa2"] + P["a_bias"]
+        act_g = {"gate_no_sigmoid": ident, "gate_tanh": np.tanh}.get(kind, sig)
+        out["g"] = act_g(mix["mg"] @ P["Wg1"]) @ P["Wg2"]
+        return out
+    return run
+
+
+@pytest.mark.parametrize("kind", ["decay_no_tanh", "decay_sigmoid", "rate_tanh", "rate_sigmoid", "residual_tanh",
+                                  "gate_no_sigmoid", "gate_tanh", "transposed_square_projection"])
+def test_layer_projection_mutant_is_caught(monkeypatch, kind):
+    monkeypatch.setattr(reference, "layer_projections", _projection_mutant(kind))
+    assert _failures(LAYER_PINS) >= 1
+
+
+def test_layer_with_transposed_output_projection_is_caught(monkeypatch):
+    orig = reference.time_mixing_layer
+
+    def run(x, params, last_x=None, v0=None, S0=None, eps=64e-5):
+        p = dict(params)
+        p["Wo"] = _f64(params["Wo"]).T
+        return orig(x, p, last_x, v0, S0, eps)
+    monkeypatch.setattr(reference, "time_mixing_layer", run)
     assert _failures(LAYER_PINS) >= 1
 
 
