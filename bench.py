@@ -4,9 +4,11 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
 One step = one pass of the hot path over one batch of the workload:
-  prefill-0.19b (default): wkv7_forward on B8 T1024 H12 N64, bf16 inputs, fp32
-      state carried in (S0 ~ N(0, 0.1^2)) and out, y fp32;
-  prefill-1.5b: B16 T4096 H32 with the fused group_norm + bonus epilogue;
+  prefill-1.5b (default): wkv7_forward on B16 T4096 H32 N64, bf16 inputs, fp32 state out,
+      y fp32 with the fused group_norm + bonus epilogue (the largest prefill shape that
+      fits one GPU). The same line carries a `decode` record (B256 H40, 128 steps replayed
+      from a CUDA graph) and a `chunk_sweep` record (the same shape at chunk 16, 32, 64);
+  prefill-0.19b: B8 T1024 H12, state carried in (S0 ~ N(0, 0.1^2)) and out;
   long-context: B1 T65536 H40, decay logits ~ N(2, 1), snapshots every 4096 tokens;
   decode: one wkv7_decode_step on B256 H40 (fp32 state in HBM).
 Prints ONE JSON line (rank 0). Under torchrun every rank runs its own independent
@@ -119,6 +121,31 @@ def _peaks():
             return json.load(f), "measured"
     except OSError:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+_PIPE_PEAKS = {}
+
+
+def pipe_peaks(dev):
+    """FP32 FMA and tf32 tensor-core rates measured on this device in this run (the library's
+    peak probes, CUDA-event timed): the denominators of the "alu" and "tensor" rooflines."""
+    key = str(dev)
+    if key not in _PIPE_PEAKS:
+        from linear_rnn_sequence_rwkv_b200 import wkv7
+        with torch.cuda.device(dev):
+            _PIPE_PEAKS[key] = {"fp32_fma_tflops": round(wkv7.probe_peak("fp32_fma"), 2),
+                                "tf32_mma_tflops": {str(n): round(wkv7.probe_peak("tf32_mma", n=n), 1)
+                                                    for n in (64, 128, 256)},
+                                "source": "wkv7_probe_fp32_fma / wkv7_probe_tf32_mma, CUDA events, this run"}
+    return _PIPE_PEAKS[key]
+
+
+def fp32_roof(flops_per_launch, launch_ms, dev):
+    pk = pipe_peaks(dev)
+    peak = pk["fp32_fma_tflops"]
+    achieved = flops_per_launch / (launch_ms * 1e-3) / 1e12
+    return {"bound": "alu", "achieved": round(achieved, 3), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "peak_source": "measured FP32 FMA rate (" + pk["source"] + ")"}
 
 
 # ---- clocks sampled during the timed region (NVML, polled from a thread) -------------------------
@@ -348,14 +375,9 @@ def run_gpu(args, world, rank, local):
     wtag = args.workload if N == 64 else f"{args.workload}-N{N}"   # profiles are per head size
     path = "decode" if decode else plan_algo
     if path == "seq":
-        sm_max = float(peaks.get("sm_max_mhz", 1965.0))
-        fp32_peak = 148 * 128 * 2 * sm_max * 1e6 / 1e12
-        achieved = flops_per_launch / (launch_ms * 1e-3) / 1e12
-        roof = {"bound": "alu", "achieved": round(achieved, 3), "peak": round(fp32_peak, 2),
-                "unit": "TFLOP/s", "frac": round(achieved / fp32_peak, 4),
-                "peak_source": f"148 SMs x 128 FP32 lanes x 2 flop x {sm_max:.0f} MHz (derived)",
-                "traffic": measured_traffic("seq_kernel", wtag, raw), "kernel": "seq_kernel",
-                "hbm_gbs": round(achieved_gbs, 1), "hbm_frac": round(achieved_gbs / hbm_peak, 4)}
+        roof = fp32_roof(flops_per_launch, launch_ms, dev)
+        roof.update({"traffic": measured_traffic("seq_kernel", wtag, raw), "kernel": "seq_kernel",
+                     "hbm_gbs": round(achieved_gbs, 1), "hbm_frac": round(achieved_gbs / hbm_peak, 4)})
     else:
         roof = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved_gbs / hbm_peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
@@ -366,9 +388,8 @@ def run_gpu(args, world, rank, local):
 
     # end to end through the public API with pinned host buffers (copies inside the timed region)
     e2e = None
-    if not decode:
-        e2e = run_e2e(args, wl, dev, stream, B, T, H, N, seed0, epilogue, snap_every, warmup,
-                      max(1, min(steps, 10)), world, raw)
+    if not decode and not getattr(args, "no_e2e", False):
+        e2e = run_e2e(args, wl, dev, stream, B, T, H, N, seed0, epilogue, snap_every, warmup, steps, world, raw)
 
     out = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": steps,
@@ -386,13 +407,46 @@ def run_gpu(args, world, rank, local):
                    "timing": ("CUDA graph of the 128 decode steps, replay time / 128" if graph is not None
                               else "one event pair per step")},
         "roofline": roof,
+        "pipe_peaks": pipe_peaks(dev),
         "e2e": e2e,
         "gpu_launches": steps * launches_per_step,
         "clocks": clocks.summary(),
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, decode)
+    if (args.workload == "prefill-1.5b" and not args.no_extras and not raw and N == 64 and args.algo == "auto"
+            and not args.chunk):
+        out["decode"] = run_decode_record(args, world, rank, local)
+        out["chunk_sweep"] = run_chunk_sweep(args, world, rank, local, steps)
     return out
+
+
+def _sub_args(args, **over):
+    d = dict(vars(args))
+    d.update(no_cpu_baseline=True, no_extras=True, no_e2e=True)
+    d.update(over)
+    return argparse.Namespace(**d)
+
+
+def run_decode_record(args, world, rank, local):
+    """The decode half of the metric on its own workload (B256 H40, fp32 state in HBM, 128 steps
+    per CUDA graph replay), measured in the same run as the prefill line."""
+    d = run_gpu(_sub_args(args, workload="decode", steps=256), world, rank, local)
+    keep = ("value", "unit", "ms_per_step", "steps", "warmup", "dtype", "config", "roofline", "gpu_launches", "clocks")
+    return {k: d[k] for k in keep}
+
+
+def run_chunk_sweep(args, world, rank, local, steps):
+    """The prefill workload at the three chunk lengths the option takes (16, 32, 64): the path
+    the library dispatches each to, and its time."""
+    rows = []
+    for c in (16, 32, 64):
+        d = run_gpu(_sub_args(args, chunk=c, steps=max(3, min(steps, 10))), world, rank, local)
+        rows.append({"chunk": c, "path": d["config"]["path"], "ctas_per_head": d["config"]["ctas_per_head"],
+                     "ms_per_step": d["ms_per_step"], "value": d["value"], "unit": d["unit"],
+                     "bound": d["roofline"]["bound"], "frac": d["roofline"]["frac"],
+                     "hbm_frac": d["roofline"].get("hbm_frac", d["roofline"]["frac"]), "clocks": d["clocks"]})
+    return rows
 
 
 BWD_FLOPS_PER_UNIT = 21 * 64 * 64   # gradient arithmetic per token-head (recomputation not counted)
@@ -450,17 +504,12 @@ def run_backward(args, world, rank, local):
     units = B * T * H
     value = units * steps * world / (total_ms * 1e-3) / 1e6
     launch_ms = statistics.mean(per_step_ms)
-    sm_max = float(peaks.get("sm_max_mhz", 1965.0))
-    fp32_peak = 148 * 128 * 2 * sm_max * 1e6 / 1e12
-    achieved = BWD_FLOPS_PER_UNIT * units / (launch_ms * 1e-3) / 1e12
     hbm_bytes = units * (6 * N * 2 + N * 4 + 6 * N * 4) + B * H * N * N * 4 * (3 + T // snap)
-    roof = {"bound": "alu", "achieved": round(achieved, 3), "peak": round(fp32_peak, 2), "unit": "TFLOP/s",
-            "frac": round(achieved / fp32_peak, 4),
-            "peak_source": f"148 SMs x 128 FP32 lanes x 2 flop x {sm_max:.0f} MHz (derived)",
-            "traffic": measured_traffic("bwd_kernel", args.workload), "kernel": "bwd_kernel",
+    roof = fp32_roof(BWD_FLOPS_PER_UNIT * units, launch_ms, dev)
+    roof.update({"traffic": measured_traffic("bwd_kernel", args.workload), "kernel": "bwd_kernel",
             "flops_per_unit": BWD_FLOPS_PER_UNIT, "algorithmic_bytes_per_launch": hbm_bytes,
             "hbm_gbs": round(hbm_bytes / (launch_ms * 1e-3) / 1e9, 1),
-            "hbm_frac": round(hbm_bytes / (launch_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]), 4)}
+            "hbm_frac": round(hbm_bytes / (launch_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]), 4)})
 
     # end to end: host inputs (pinned) -> device, backward, gradients -> host, all timed
     hd = {n: (v.to("cpu").pin_memory() if isinstance(v, torch.Tensor) else v) for n, v in sets[0].items()}
@@ -731,7 +780,9 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="prefill-0.19b")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="prefill-1.5b")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="prefill-1.5b: leave out the decode and chunk-sweep records")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--algo", choices=["auto", "seq", "chunk", "split"], default="auto")
     ap.add_argument("--chunk", type=int, default=0)

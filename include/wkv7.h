@@ -56,7 +56,7 @@ extern "C" {
 #define WKV7_API
 #endif
 
-#define WKV7_ABI_VERSION 3
+#define WKV7_ABI_VERSION 4
 #define WKV7_HEAD_SIZE 64
 #define WKV7_MAX_SEGMENTS 8   /* CTAs per (b, h) of WKV7_ALGO_SPLIT (one thread-block cluster) */
 
@@ -102,10 +102,19 @@ typedef struct wkv7_opts {
     float gn_eps;         /* epilogue epsilon added to the variance (default 64e-5)      */
     int segments;         /* WKV7_ALGO_SPLIT: CTAs per (b, h), 1..WKV7_MAX_SEGMENTS, or  */
                           /* 0 = automatic (AUTO always chooses; CHUNK uses one)         */
+    unsigned int handoff_wait_us;   /* limit of each wait for a state (or for its receipt)    */
+                          /* between the CTAs of one head in split mode, in microseconds; */
+                          /* 0 = the default 2 s. Every other device-side wait keeps 2 s. */
+    int withhold_handoff; /* failure-path test only: 1 = in split mode the first CTA of   */
+                          /* each head withholds its first state hand-off, so the waiting */
+                          /* CTA's bounded wait runs out, the kernel records the error    */
+                          /* and returns (wkv7_poll_device_error then gives               */
+                          /* WKV7_ERR_TIMEOUT; y and S_T are incomplete). Accepted only   */
+                          /* with WKV7_ALGO_SPLIT and segments >= 2; 0 = normal.          */
 } wkv7_opts;
 
 /* Fills *opts with the defaults: AUTO, default chunk, no snapshots, no epilogue,
- * gn_eps = 64e-5, automatic segments. */
+ * gn_eps = 64e-5, automatic segments, default hand-off wait limit, no withheld hand-off. */
 WKV7_API void wkv7_opts_default(wkv7_opts *opts);
 
 /*
@@ -323,6 +332,21 @@ WKV7_API const char *wkv7_status_string(wkv7_status status);
 
 /* Detail of the last error returned on the calling thread ("" if none). */
 WKV7_API const char *wkv7_last_error(void);
+
+/*
+ * Peak-rate probes (no counterpart on the pages): kernels that keep one pipe busy and nothing
+ * else, for measuring the roofline denominators on the device at hand. Each enqueues one launch
+ * on `stream` and stores in *flops the floating-point operations it performs; time the launch
+ * with CUDA events on that stream and divide.
+ *   wkv7_probe_fp32_fma: `blocks` CTAs of 256 threads, each thread `iters` x 128 fused
+ *     multiply-adds on 8 independent chains (2 flops each). blocks, iters >= 1.
+ *   wkv7_probe_tf32_mma: one CTA per SM issuing `iters` x 4 tcgen05.mma kind::tf32 of
+ *     M = 128, N = n (64, 128 or 256), K = 8 back to back into tensor memory. iters >= 1.
+ * WKV7_ERR_ARG for other values, WKV7_ERR_CUDA for a failed launch; a bounded wait that gives
+ * up is reported by wkv7_poll_device_error. Host pointers only for `flops`.
+ */
+WKV7_API wkv7_status wkv7_probe_fp32_fma(int blocks, int iters, void *stream, double *flops);
+WKV7_API wkv7_status wkv7_probe_tf32_mma(int n, int iters, void *stream, double *flops);
 
 /* WKV7_ABI_VERSION of the loaded library. */
 WKV7_API int wkv7_abi_version(void);

@@ -142,6 +142,10 @@ wkv7_status check_args(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opt
         return fail(WKV7_ERR_ARG, "gn_eps must be finite and >= 0");
     if (opts.segments < 0 || opts.segments > WKV7_MAX_SEGMENTS)
         return fail(WKV7_ERR_ARG, "segments=%d outside 0..%d", opts.segments, WKV7_MAX_SEGMENTS);
+    if (opts.withhold_handoff != 0 &&
+        (opts.withhold_handoff != 1 || opts.algo != WKV7_ALGO_SPLIT || opts.segments < 2))
+        return fail(WKV7_ERR_ARG, "withhold_handoff=%d: only 1, with WKV7_ALGO_SPLIT and segments >= 2",
+                    opts.withhold_handoff);
     return WKV7_OK;
 }
 
@@ -191,6 +195,19 @@ const char *wkv7_status_string(wkv7_status s) {
 const char *wkv7_last_error(void) { return g_err; }
 
 int wkv7_abi_version(void) { return WKV7_ABI_VERSION; }
+
+wkv7_status wkv7_probe_fp32_fma(int blocks, int iters, void *stream, double *flops) {
+    if (blocks < 1 || iters < 1 || !flops) return fail(WKV7_ERR_ARG, "blocks and iters must be >= 1, flops non-NULL");
+    const cudaError_t e = wkv7::launch_fma_peak(blocks, iters, static_cast<cudaStream_t>(stream), flops);
+    return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "FMA peak probe");
+}
+
+wkv7_status wkv7_probe_tf32_mma(int n, int iters, void *stream, double *flops) {
+    if (!(n == 64 || n == 128 || n == 256) || iters < 1 || !flops)
+        return fail(WKV7_ERR_ARG, "n must be 64, 128 or 256, iters >= 1, flops non-NULL");
+    const cudaError_t e = wkv7::launch_tf32_mma_peak(n, iters, static_cast<cudaStream_t>(stream), flops);
+    return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "tf32 MMA peak probe");
+}
 
 size_t wkv7_workspace_bytes(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opts *opts) {
     (void)B; (void)T; (void)H; (void)N; (void)dt; (void)opts;
@@ -277,6 +294,8 @@ wkv7_status forward_impl(bool raw, int B, int T, int H, int N, wkv7_dtype dt, co
     p.raw = raw; p.k_k = raw ? k_k : nullptr; p.k_a = raw ? k_a : nullptr;
     p.chunk = opts.chunk;
     p.segments = requested_segments(opts);
+    p.handoff_wait_us = opts.handoff_wait_us;
+    p.withhold_handoff = opts.withhold_handoff;
     p.ws = workspace; p.ws_bytes = workspace_bytes;
     p.stream = static_cast<cudaStream_t>(stream);
 

@@ -133,7 +133,9 @@ struct ChunkArgs {
     float gn_eps;
     const float *k_k, *k_a;   // raw inputs: the removal-key scale and the key-update rate ([H][64]; k_a nullable)
     unsigned int *err;
-    unsigned long long timeout_ns;
+    unsigned long long timeout_ns;           // every bounded wait but the split-mode hand-off
+    unsigned long long handoff_timeout_ns;   // split mode: waits for a state and for its receipt
+    int withhold_handoff;     // failure-path test: CTA 0 of each cluster does not send its first state
 };
 
 // bf16 element (t, j) of a 128-byte-swizzled [64][64] tile.
@@ -267,10 +269,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     // Waits: one thread polls the mbarrier (bounded, acquire) and the others wait in a hardware
     // barrier with it; many polling threads would crowd the shared-memory pipe that the other
     // warp group is using. All threads; true on timeout (uniform across the CTA).
+    // On a timeout the issuing thread keeps the parity of the phase that did not complete and
+    // stays `mma_pending`, so the drain on the way out waits (bounded) for that phase.
     auto wait_mma_all = [&]() -> bool {
         const bool to = tid == 0 && !mbar_wait_spin(&S.bar_mma, mma_parity, p.timeout_ns);
-        mma_parity ^= 1u;
-        mma_pending = false;
+        if (!to) mma_parity ^= 1u;
+        mma_pending = to;
         const bool f = __syncthreads_or(to) != 0;
         tc_fence_after();
         return f;
@@ -278,10 +282,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     // warps 0-3 only; true on timeout here or (`extra`) in any of them
     auto wait_mma_back = [&](bool extra) -> bool {
         const bool to = tid == 0 && !mbar_wait_spin(&S.bar_mma, mma_parity, p.timeout_ns);
-        mma_parity ^= 1u;
+        if (!to) mma_parity ^= 1u;
         const bool f = bar_named_or(BAR_BACK, kBackThreads, to || extra);
         tc_fence_after();
-        mma_pending = f;   // on a failure the round may still be running: drain it before exit
+        mma_pending = to;   // a round that did not complete may still be running: drain it before exit
         return f;
     };
     auto sync_for_mma = [&]() {            // writes to smem/TMEM -> visible to the next MMA
@@ -476,7 +480,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
             uint32_t xo[8];
             kcol_offsets(j, 64, xo);
             const uint32_t b5_dst = cs == 1 ? own_b5 : next_b5;
-            const bool write_b5 = cs == 1 || send;
+            // failure-path test: CTA 0 of the cluster keeps its first state to itself, so the next
+            // CTA's bounded wait for it runs out
+            const bool deliver = send && !(p.withhold_handoff && rank == 0 && sends == 0);
+            const bool write_b5 = cs == 1 || deliver;
 #pragma unroll
             for (int g = 0; g < 2; ++g)
 #pragma unroll
@@ -484,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                     v[g][e] *= gCj;                                             // S_C = S' diag(gC)
                     if (write_b5) st_cluster(b5_dst + (c16 + 8 * g + e) * 128 + xo[e], to_tf32(v[g][e]));
                 }
-            if (send) {
+            if (deliver) {
                 fence_proxy_async_cluster();
                 mbar_arrive_remote(next_bar);
             }
@@ -817,7 +824,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                         mma_tf32_ts(tb + T_D4, tb + T_D3R + 8 * ks, dB4 + kstep_off(ks, 64), idesc_tf32(128, 64), ks > 0);
                     if (recv) {
                         // the only wait on another CTA: everything above used this chunk's inputs only
-                        state_to = !mbar_wait_cluster(&S.bar_state, state_parity, p.timeout_ns);
+                        state_to = !mbar_wait_cluster(&S.bar_state, state_parity, p.handoff_timeout_ns);
                         fence_proxy_async_smem();
                         tc_fence_after();
                     }
@@ -836,11 +843,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         } else if (more) {
             if (new_unit && ft < 64) load_params(nu, us ^ 1, ft);
             wfail = front(nu, nc, ip ^ 1, new_unit ? (us ^ 1) : us);
+            if (!wfail) tma_pending = false;   // these threads saw the tiles arrive
         }
         // split mode: before writing the next CTA's B5, its credit for the state sent before
         const bool send = cs > 1 && c + 1 < nchunks;
         if (send && sends > 0) {
-            if (tid == 0 && !wfail) wfail = !mbar_wait_cluster(&S.bar_credit, credit_parity, p.timeout_ns);
+            if (tid == 0 && !wfail) wfail = !mbar_wait_cluster(&S.bar_credit, credit_parity, p.handoff_timeout_ns);
             credit_parity ^= 1u;
         }
         tc_fence_before();
@@ -1067,6 +1075,8 @@ cudaError_t launch_chunk(const FwdArgs &p) {
     a.k_k = p.k_k; a.k_a = p.k_a;
     a.err = di->err;
     a.timeout_ns = 2000000000ull;
+    a.handoff_timeout_ns = p.handoff_wait_us ? 1000ull * p.handoff_wait_us : a.timeout_ns;
+    a.withhold_handoff = p.withhold_handoff;
     int cs = 1;
     if ((e = chunk_segments(p, &cs)) != cudaSuccess) return e;
     const ChunkPlan pl = plan_launches(p, *di);
@@ -1081,6 +1091,13 @@ cudaError_t launch_chunk(const FwdArgs &p) {
         a.unit0 = a.unit_end;
     }
     return cudaSuccess;
+}
+
+cudaError_t device_error_word(unsigned int **ptr) {
+    DeviceInfo *di = nullptr;
+    const cudaError_t e = device_info(di);
+    if (e == cudaSuccess) *ptr = di->err;
+    return e;
 }
 
 cudaError_t read_device_error(cudaStream_t stream, unsigned int *value, bool clear) {

@@ -28,6 +28,8 @@ struct FwdArgs {
     float gn_eps;
     int chunk;
     int segments;          // CTAs per (b, h) on the chunked path; 0 = automatic
+    unsigned int handoff_wait_us;   // split mode: limit of the hand-off waits (0 = default)
+    int withhold_handoff;  // split mode, failure-path test: withhold the first hand-off of each head
     void *ws;
     size_t ws_bytes;
     cudaStream_t stream;
@@ -80,6 +82,11 @@ cudaError_t launch_chunk(const FwdArgs &p);        // chunked prefill on tcgen05
 cudaError_t chunk_segments(const FwdArgs &p, int *segments, int *launches = nullptr);
 // Synchronises `stream` and reads the device error word (bounded waits that gave up).
 cudaError_t read_device_error(cudaStream_t stream, unsigned int *value, bool clear);
+// The device error word of the current device (set by a bounded wait that gave up).
+cudaError_t device_error_word(unsigned int **ptr);
+// Peak-rate probes: launch on `stream`, *flops = the floating-point operations of the launch.
+cudaError_t launch_fma_peak(int blocks, int iters, cudaStream_t stream, double *flops);
+cudaError_t launch_tf32_mma_peak(int n, int iters, cudaStream_t stream, double *flops);
 // Raises `kernel`'s dynamic shared-memory limit to `bytes` on the current device. The attribute
 // belongs to the device's context, so it is set once per (device, kernel); failures are not
 // remembered (the next call tries again).

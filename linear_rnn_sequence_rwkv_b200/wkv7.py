@@ -19,7 +19,7 @@ import torch
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libwkv7.so")
 HEAD_SIZE = 64
-ABI_VERSION = 3          # WKV7_ABI_VERSION of include/wkv7.h this binding follows
+ABI_VERSION = 4          # WKV7_ABI_VERSION of include/wkv7.h this binding follows
 
 # wkv7_status
 OK, ERR_ARG, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(7)
@@ -31,7 +31,8 @@ ALGOS = {"auto": 0, "seq": 1, "chunk": 2, "split": 3}
 EXPORTED = ("wkv7_opts_default", "wkv7_forward", "wkv7_decode_step", "wkv7_workspace_bytes",
             "wkv7_status_string", "wkv7_last_error", "wkv7_abi_version", "wkv7_poll_device_error",
             "wkv7_plan", "wkv7_forward_raw", "wkv7_backward", "wkv7_backward_workspace_bytes",
-            "wkv7_backward_static", "wkv7_layer_forward", "wkv7_layer_workspace_bytes")
+            "wkv7_backward_static", "wkv7_layer_forward", "wkv7_layer_workspace_bytes", "wkv7_probe_fp32_fma",
+            "wkv7_probe_tf32_mma")
 
 
 class Wkv7Error(RuntimeError):
@@ -56,7 +57,8 @@ class LayerParams(ctypes.Structure):
 class Opts(ctypes.Structure):
     _fields_ = [("algo", ctypes.c_int), ("chunk", ctypes.c_int), ("snap_every", ctypes.c_int),
                 ("snapshots", ctypes.c_void_p), ("ln_w", ctypes.c_void_p), ("ln_b", ctypes.c_void_p),
-                ("r_k", ctypes.c_void_p), ("gn_eps", ctypes.c_float), ("segments", ctypes.c_int)]
+                ("r_k", ctypes.c_void_p), ("gn_eps", ctypes.c_float), ("segments", ctypes.c_int),
+                ("handoff_wait_us", ctypes.c_uint), ("withhold_handoff", ctypes.c_int)]
 
 
 _lock = threading.Lock()
@@ -113,6 +115,10 @@ def load():
         lib.wkv7_forward_raw.argtypes = [ci, ci, ci, ci, ci] + [vp] * 5 + [vp, vp] + [vp, vp, vp, ctypes.POINTER(Opts),
                                                                                vp, ctypes.c_size_t, vp]
         lib.wkv7_forward_raw.restype = ci
+        lib.wkv7_probe_fp32_fma.argtypes = [ci, ci, vp, ctypes.POINTER(ctypes.c_double)]
+        lib.wkv7_probe_fp32_fma.restype = ci
+        lib.wkv7_probe_tf32_mma.argtypes = [ci, ci, vp, ctypes.POINTER(ctypes.c_double)]
+        lib.wkv7_probe_tf32_mma.restype = ci
         if lib.wkv7_abi_version() != ABI_VERSION:
             raise RuntimeError(f"{_LIB_PATH} has ABI version {lib.wkv7_abi_version()}, the binding expects "
                                f"{ABI_VERSION}: rebuild it")
@@ -145,7 +151,7 @@ def _stream_handle(device, stream):
 
 
 def make_opts(algo="auto", chunk=0, snap_every=0, snapshots=None, ln_w=None, ln_b=None, r_k=None,
-              gn_eps=64e-5, segments=0) -> Opts:
+              gn_eps=64e-5, segments=0, handoff_wait_us=0, withhold_handoff=0) -> Opts:
     o = Opts()
     load().wkv7_opts_default(ctypes.byref(o))
     o.algo = ALGOS[algo] if isinstance(algo, str) else int(algo)
@@ -157,6 +163,8 @@ def make_opts(algo="auto", chunk=0, snap_every=0, snapshots=None, ln_w=None, ln_
     o.r_k = None if r_k is None else r_k.data_ptr()
     o.gn_eps = float(gn_eps)
     o.segments = int(segments)
+    o.handoff_wait_us = int(handoff_wait_us)
+    o.withhold_handoff = int(withhold_handoff)
     return o
 
 
@@ -179,7 +187,7 @@ def workspace_bytes(B, T, H, N=HEAD_SIZE, dtype=torch.bfloat16, **opt_kw) -> int
 
 def forward(r, w, k, v, kk, a, S0=None, *, algo="auto", chunk=0, snap_every=0, ln_w=None, ln_b=None,
             r_k=None, gn_eps=64e-5, segments=0, y=None, S_T=None, snapshots=None, workspace=None,
-            return_state=True, stream=None, out_host=None):
+            return_state=True, stream=None, out_host=None, handoff_wait_us=0, withhold_handoff=0):
     """WKV-7 forward over [B, T, H, 64] inputs (bf16 or fp32, all the same dtype).
 
     Returns (y, S_T, snapshots): y [B, T, H, 64] fp32, S_T [B, H, 64, 64] fp32
@@ -203,7 +211,8 @@ def forward(r, w, k, v, kk, a, S0=None, *, algo="auto", chunk=0, snap_every=0, l
     n_snap = T // snap_every if snap_every else 0
     if snapshots is None and n_snap:
         snapshots = torch.empty((B, n_snap, H, N, N), device=dev, dtype=torch.float32)
-    opts = make_opts(algo, chunk, snap_every, snapshots, ln_w, ln_b, r_k, gn_eps, segments)
+    opts = make_opts(algo, chunk, snap_every, snapshots, ln_w, ln_b, r_k, gn_eps, segments, handoff_wait_us,
+                     withhold_handoff)
     need = int(lib.wkv7_workspace_bytes(B, T, H, N, _dt(r), ctypes.byref(opts)))
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, device=dev, dtype=torch.uint8)
@@ -433,3 +442,39 @@ def _forward_host(r, w, k, v, kk, a, S0, *, return_state, out_host, **kw):
     main.wait_stream(s_out)
     main.synchronize()
     return y_h, (S_h if return_state else None), sn_h
+
+
+def probe_peak(kind, *, n=256, iters=None, blocks=None, reps=5, device=None):
+    """Measured rate (TFLOP/s) of one pipe: kind "fp32_fma" (the FMA pipe, all SMs) or
+    "tf32_mma" (tcgen05 kind::tf32, M = 128 and N = n, one CTA per SM). Each of `reps` launches
+    is timed with CUDA events on the current stream after a warm-up launch; the median is kept."""
+    lib = load()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    stream = torch.cuda.current_stream(dev)
+    flops = ctypes.c_double(0.0)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+
+    def launch():
+        if kind == "fp32_fma":
+            st = lib.wkv7_probe_fp32_fma(blocks or 8 * sms, iters or 4096, ctypes.c_void_p(stream.cuda_stream),
+                                         ctypes.byref(flops))
+        elif kind == "tf32_mma":
+            st = lib.wkv7_probe_tf32_mma(int(n), iters or 20000, ctypes.c_void_p(stream.cuda_stream),
+                                         ctypes.byref(flops))
+        else:
+            raise ValueError(kind)
+        _check(st, "wkv7_probe_" + kind)
+
+    with torch.cuda.device(dev):
+        launch()
+        times = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            launch()
+            e1.record(stream)
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+        poll_device_error()
+    times.sort()
+    return flops.value / (times[len(times) // 2] * 1e-3) / 1e12

@@ -37,13 +37,14 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_strings(lib):
-    assert lib.wkv7_abi_version() == 3
+    assert lib.wkv7_abi_version() == 4
     assert lib.wkv7_status_string(0) == b"WKV7_OK"
     assert lib.wkv7_status_string(3) == b"WKV7_ERR_ALIGN"
     assert lib.wkv7_status_string(99) == b"WKV7_ERR_UNKNOWN"
     o = wkv7.Opts()
     lib.wkv7_opts_default(ctypes.byref(o))
     assert o.algo == 0 and o.chunk == 0 and o.snap_every == 0 and abs(o.gn_eps - 64e-5) < 1e-9
+    assert o.handoff_wait_us == 0 and o.withhold_handoff == 0
 
 
 FAKE = 0x10000   # 16-byte aligned, never dereferenced: validation fails first
@@ -84,6 +85,17 @@ def test_forward_rejects_bad_options(lib, field, value):
     lib.wkv7_opts_default(ctypes.byref(o))
     setattr(o, field, value)
     assert _fwd(lib, opts=o) == wkv7.ERR_ARG
+
+
+@pytest.mark.parametrize("algo,segments,value", [(0, 0, 1), (2, 0, 1), (3, 1, 1), (3, 2, 2), (3, 2, -1)])
+def test_withheld_handoff_only_in_split_mode(lib, algo, segments, value):
+    """The failure-path switch is refused unless the chunks of a head are spread over at
+    least two CTAs (the only place a hand-off happens)."""
+    o = wkv7.Opts()
+    lib.wkv7_opts_default(ctypes.byref(o))
+    o.algo, o.segments, o.withhold_handoff = algo, segments, value
+    assert _fwd(lib, opts=o) == wkv7.ERR_ARG
+    assert b"withhold_handoff" in lib.wkv7_last_error()
 
 
 def test_forward_rejects_partial_epilogue_and_missing_snapshots(lib):

@@ -320,6 +320,26 @@ def test_no_device_error_after_runs(cuda_device):
     wkv7.poll_device_error()
 
 
+def test_handoff_wait_runs_out_and_reports_timeout(cuda_device):
+    """Split mode with each head's first state hand-off withheld: the receiving CTA's bounded
+    wait (2 ms here) runs out, the kernel records the error, drains what it issued and
+    returns. wkv7_poll_device_error reports WKV7_ERR_TIMEOUT once and clears it; the context
+    stays usable, and a normal forward afterwards matches the oracle."""
+    d = inputs.make_inputs(inputs.WORKLOADS[1], B=1, T=256, H=2, seed=4242)
+    dd = _dev(d, cuda_device)
+    wkv7.poll_device_error()                       # nothing pending before
+    _gpu(dd, algo="split", segments=2, handoff_wait_us=2000, withhold_handoff=1)
+    with pytest.raises(wkv7.Wkv7Error) as e:
+        wkv7.poll_device_error()
+    assert e.value.status == wkv7.ERR_TIMEOUT
+    wkv7.poll_device_error()                       # cleared by the poll
+    y, S, _ = _gpu(dd, algo="split", segments=2)
+    wkv7.poll_device_error()
+    y_ref, S_ref, _ = _oracle(d)
+    assert y_err(y, y_ref) <= TOL["bf16"]
+    assert state_err(S, S_ref) <= TOL["bf16"]
+
+
 @pytest.mark.parametrize("segments", [2, 3, 4, 7, 8])
 @pytest.mark.parametrize("T", [130, 64 * 9 + 17, 1024])
 def test_split_matches_oracle_and_single_cta(cuda_device, segments, T):
@@ -383,3 +403,38 @@ def test_plan_launch_counts_on_device(cuda_device):
     assert wkv7.plan(8, 1024, 12, launches=True)[2] == 1
     algo, seg, n = wkv7.plan(16, 4096, 32, launches=True)
     assert algo == "chunk" and n in (1, 2) and (n == 1 or seg > 1)
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+@pytest.mark.parametrize("T", [1, 15, 33, 100, 257])
+def test_chunk_option_with_epilogue(cuda_device, chunk, T):
+    """The chunk-length option (16, 32, 64) under AUTO on ragged lengths, with the fused
+    group_norm + bonus epilogue and a carried-in state, against the oracle recurrence and
+    epilogue; the path AUTO picks is whichever the library dispatches the option to."""
+    wl = inputs.WORKLOADS[2]
+    d = inputs.make_inputs(wl, B=2, T=T, H=3, seed=1500 + 7 * T + chunk, s0="normal")
+    y_ref, S_ref, _ = _oracle(d)
+    y_ref = native.epilogue(y_ref, d["r"], d["k"], d["v"], d["ln_w"], d["ln_b"], d["r_k"])
+    dd = _dev(d, cuda_device)
+    y, S, _ = _gpu(dd, chunk=chunk, ln_w=dd["ln_w"], ln_b=dd["ln_b"], r_k=dd["r_k"])
+    assert y_err(y, y_ref) <= TOL["bf16"]
+    assert state_err(S, S_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("chunk", [16, 32])
+def test_chunk_option_on_the_prefill_15b_shape_sampled(cuda_device, chunk):
+    """The 1.5B prefill shape (B16 T4096 H32, epilogue) at chunk 16 and 32; the oracle runs
+    on four sampled (b, h) pairs."""
+    wl = inputs.WORKLOADS[2]
+    d = inputs.make_inputs(wl)
+    dd = _dev(d, cuda_device)
+    y, S, _ = _gpu(dd, chunk=chunk, ln_w=dd["ln_w"], ln_b=dd["ln_b"], r_k=dd["r_k"])
+    pairs = [(0, 0), (5, 31), (11, 17), (15, 3)]
+    for b, h in pairs:
+        sub = {n: d[n][b:b + 1, :, h:h + 1] for n in ("r", "w", "k", "v", "kk", "a")}
+        sub["S0"] = None if d["S0"] is None else d["S0"][b:b + 1, h:h + 1]
+        y_ref, S_ref, _ = _oracle(sub)
+        y_ref = native.epilogue(y_ref, sub["r"], sub["k"], sub["v"], d["ln_w"][h:h + 1], d["ln_b"][h:h + 1],
+                                d["r_k"][h:h + 1])
+        assert y_err(y[b:b + 1, :, h:h + 1], y_ref) <= TOL["bf16"], (b, h)
+        assert state_err(S[b:b + 1, h:h + 1], S_ref) <= TOL["bf16"], (b, h)
