@@ -666,8 +666,10 @@ def _path_name(args):
 
 
 def run_e2e(args, wl, dev, stream, B, T, H, N, seed, epilogue, snap_every, warmup, steps, world, raw=False):
-    """Same metric through wkv7.forward (or forward_raw) with pinned HOST tensors: H2D of the
-    inputs, the kernels and D2H of y and S_T are all inside the timed region."""
+    """Same metric through the C ABI's host-buffer entry (wkv7_forward_host) with pinned HOST
+    tensors: every step's host-to-device copies of the inputs, the kernels and the
+    device-to-host copies of y and S_T are inside the timed region. The raw-input workload has
+    no host-buffer entry; it copies through torch around wkv7_forward_raw instead."""
     from linear_rnn_sequence_rwkv_b200 import wkv7
     d = (inputs.make_raw_inputs if raw else inputs.make_inputs)(wl, device="cpu", seed=seed + 999)
     host = {n: (v.pin_memory() if isinstance(v, torch.Tensor) else v) for n, v in d.items()}
@@ -680,10 +682,16 @@ def run_e2e(args, wl, dev, stream, B, T, H, N, seed, epilogue, snap_every, warmu
     d2h = B * T * H * N * 4 + B * H * N * N * 4 + (B * (T // snap_every) * H * N * N * 4 if snap_every else 0)
     y_h = torch.empty(B, T, H, N).pin_memory()
     S_h = torch.empty(B, H, N, N).pin_memory()
+    sn_h = torch.empty(B, T // snap_every, H, N, N).pin_memory() if snap_every else None
+    ep = {n: host[n] for n in ("ln_w", "ln_b", "r_k")} if epilogue else {}
+    ws = None
+    if not raw:
+        ws = torch.empty(wkv7.forward_host_workspace_bytes(B, T, H, N, torch.bfloat16, snap_every=snap_every,
+                                                           epilogue=epilogue, algo=args.algo, chunk=args.chunk),
+                         dtype=torch.uint8, device=dev)
 
     def once():
-        ep = {n: host[n] for n in ("ln_w", "ln_b", "r_k")} if epilogue else {}
-        if raw:   # the raw entry takes device tensors: copy in, run, copy out, all on this stream
+        if raw:   # copy in, run, copy out, all on this stream
             dv = {n: (None if host[n] is None else host[n].to(dev, non_blocking=True))
                   for n in RAW_NAMES + ("k_k", "k_a", "S0")}
             dep = {n: v.to(dev, non_blocking=True) for n, v in ep.items()}
@@ -691,10 +699,9 @@ def run_e2e(args, wl, dev, stream, B, T, H, N, seed, epilogue, snap_every, warmu
                                        chunk=args.chunk, snap_every=snap_every, **dep)
             y_h.copy_(y, non_blocking=True)
             S_h.copy_(S, non_blocking=True)
-            return y_h, S_h
-        y, S, _ = wkv7.forward(*(host[n] for n in NAMES), host["S0"], algo=args.algo, chunk=args.chunk,
-                               snap_every=snap_every, out_host=(y_h, S_h), **ep)
-        return y, S
+            return
+        wkv7.forward_host(*(host[n] for n in NAMES), host["S0"], y_h, S_h, ws, algo=args.algo, chunk=args.chunk,
+                          snap_every=snap_every, snapshots=sn_h, **ep)
 
     for _ in range(max(1, min(warmup, 3))):
         once()
@@ -709,7 +716,8 @@ def run_e2e(args, wl, dev, stream, B, T, H, N, seed, epilogue, snap_every, warmu
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     return {"value": round(B * T * H * steps * world / (ms * 1e-3) / 1e6, 3), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": round(ms / steps, 4)}
+            "ms_per_step": round(ms / steps, 4),
+            "api": "wkv7_forward_raw with torch copies" if raw else "wkv7_forward_host (C ABI, pinned host buffers)"}
 
 
 def cpu_baseline(wl, decode: bool, budget_s: float = 12.0):

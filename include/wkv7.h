@@ -166,6 +166,38 @@ WKV7_API wkv7_status wkv7_forward_raw(int B, int T, int H, int N, wkv7_dtype dt,
                              void *stream);
 
 /*
+ * wkv7_forward on HOST buffers: the end-to-end path for a caller whose inputs and results live
+ * in host memory. Every pointer argument (r, w, k, v, kk, a, S0, y, S_T, opts->snapshots and the
+ * epilogue parameters opts->ln_w, ln_b, r_k) is a host pointer with the layout of wkv7_forward;
+ * page-locked (pinned) memory lets the copies run asynchronously and overlap. The batch is cut
+ * into slices of whole sequences (up to 8, at least 24 MB of input each); each slice's
+ * host-to-device copies run on a copy stream of the library, its forward on `stream`, its
+ * device-to-host copies on a second copy stream, so copies in both directions overlap the
+ * kernels of the other slices. The device copies live in `workspace` (device memory of at least
+ * wkv7_forward_host_workspace_bytes(...) bytes, 256-byte aligned): nothing is allocated. The
+ * library makes its two copy streams and their events once per device (first call on a device:
+ * make it before any stream capture).
+ * Returns once everything is enqueued; the host outputs are complete when `stream` is
+ * (cudaStreamSynchronize). Calls on one device are serialised while they enqueue; a call's
+ * copies start after all work already on `stream`, so the workspace may be reused by the next
+ * call on the same stream. Host output buffers must not overlap the inputs.
+ * Errors as wkv7_forward, plus WKV7_ERR_ARG for device or managed pointers (use wkv7_forward),
+ * WKV7_ERR_WORKSPACE, WKV7_ERR_ALIGN for a workspace not 256-byte aligned.
+ * (RWKV-7 paper summary, section 8: the forward over a sequence; the host path itself has no
+ * counterpart on the pages.)
+ */
+WKV7_API wkv7_status wkv7_forward_host(int B, int T, int H, int N, wkv7_dtype dt,
+                              const void *r, const void *w, const void *k, const void *v,
+                              const void *kk, const void *a, const float *S0, float *y, float *S_T,
+                              const wkv7_opts *opts, void *workspace, size_t workspace_bytes,
+                              void *stream);
+
+/* Device workspace bytes of wkv7_forward_host: device copies of every input and output of the
+ * whole batch (S0 and S_T always counted) plus wkv7_workspace_bytes. 0 for invalid sizes. */
+WKV7_API size_t wkv7_forward_host_workspace_bytes(int B, int T, int H, int N, wkv7_dtype dt,
+                                                  const wkv7_opts *opts);
+
+/*
  * Backward pass of wkv7_forward (no epilogue): the gradients of every input for the scalar
  * L = <dy, y> + <dS_T, S_T>, in fp32. The pages time a backward pass and state the precision
  * of an fp32 one (RWKV-7 rebuttal page, the answer on numerical precision; paper summary,

@@ -32,6 +32,8 @@ cudaError_t allow_dynamic_smem(const void *kernel, int bytes) {
     return e;
 }
 
+wkv7_status set_error(wkv7_status s, const char *fmt, ...);
+
 }  // namespace wkv7
 
 namespace {
@@ -45,6 +47,18 @@ wkv7_status fail(wkv7_status s, const char *fmt, ...) {
     va_end(ap);
     return s;
 }
+
+}  // namespace
+
+wkv7_status wkv7::set_error(wkv7_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+namespace {
 
 wkv7_status cuda_fail(cudaError_t e, const char *what) {
     return fail(WKV7_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));

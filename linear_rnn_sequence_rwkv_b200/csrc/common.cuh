@@ -82,6 +82,8 @@ cudaError_t launch_chunk(const FwdArgs &p);        // chunked prefill on tcgen05
 cudaError_t chunk_segments(const FwdArgs &p, int *segments, int *launches = nullptr);
 // Synchronises `stream` and reads the device error word (bounded waits that gave up).
 cudaError_t read_device_error(cudaStream_t stream, unsigned int *value, bool clear);
+// Records the calling thread's error text (wkv7_last_error) and returns s.
+wkv7_status set_error(wkv7_status s, const char *fmt, ...);
 // The device error word of the current device (set by a bounded wait that gave up).
 cudaError_t device_error_word(unsigned int **ptr);
 // Peak-rate probes: launch on `stream`, *flops = the floating-point operations of the launch.

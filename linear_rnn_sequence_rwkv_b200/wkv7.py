@@ -32,7 +32,7 @@ EXPORTED = ("wkv7_opts_default", "wkv7_forward", "wkv7_decode_step", "wkv7_works
             "wkv7_status_string", "wkv7_last_error", "wkv7_abi_version", "wkv7_poll_device_error",
             "wkv7_plan", "wkv7_forward_raw", "wkv7_backward", "wkv7_backward_workspace_bytes",
             "wkv7_backward_static", "wkv7_layer_forward", "wkv7_layer_workspace_bytes", "wkv7_probe_fp32_fma",
-            "wkv7_probe_tf32_mma")
+            "wkv7_probe_tf32_mma", "wkv7_forward_host", "wkv7_forward_host_workspace_bytes")
 
 
 class Wkv7Error(RuntimeError):
@@ -115,6 +115,10 @@ def load():
         lib.wkv7_forward_raw.argtypes = [ci, ci, ci, ci, ci] + [vp] * 5 + [vp, vp] + [vp, vp, vp, ctypes.POINTER(Opts),
                                                                                vp, ctypes.c_size_t, vp]
         lib.wkv7_forward_raw.restype = ci
+        lib.wkv7_forward_host.argtypes = lib.wkv7_forward.argtypes
+        lib.wkv7_forward_host.restype = ci
+        lib.wkv7_forward_host_workspace_bytes.argtypes = [ci, ci, ci, ci, ci, ctypes.POINTER(Opts)]
+        lib.wkv7_forward_host_workspace_bytes.restype = ctypes.c_size_t
         lib.wkv7_probe_fp32_fma.argtypes = [ci, ci, vp, ctypes.POINTER(ctypes.c_double)]
         lib.wkv7_probe_fp32_fma.restype = ci
         lib.wkv7_probe_tf32_mma.argtypes = [ci, ci, vp, ctypes.POINTER(ctypes.c_double)]
@@ -478,3 +482,47 @@ def probe_peak(kind, *, n=256, iters=None, blocks=None, reps=5, device=None):
         poll_device_error()
     times.sort()
     return flops.value / (times[len(times) // 2] * 1e-3) / 1e12
+
+
+def _host_ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _host_opts(algo, chunk, snap_every, snapshots, ln_w, ln_b, r_k, gn_eps, segments):
+    o = make_opts(algo, chunk, snap_every, None, None, None, None, gn_eps, segments)
+    o.snapshots = None if snapshots is None else snapshots.data_ptr()
+    o.ln_w = None if ln_w is None else ln_w.data_ptr()
+    o.ln_b = None if ln_b is None else ln_b.data_ptr()
+    o.r_k = None if r_k is None else r_k.data_ptr()
+    return o
+
+
+def forward_host_workspace_bytes(B, T, H, N=HEAD_SIZE, dtype=torch.bfloat16, *, snap_every=0, epilogue=False,
+                                 algo="auto", chunk=0, segments=0) -> int:
+    o = make_opts(algo, chunk, snap_every, None, None, None, None, 64e-5, segments)
+    if epilogue:   # any non-null value marks the epilogue as on for the size query
+        o.ln_w = o.ln_b = o.r_k = 16
+    return int(load().wkv7_forward_host_workspace_bytes(B, T, H, N, _dt_of(dtype), ctypes.byref(o)))
+
+
+def _dt_of(dtype):
+    return BF16 if dtype == torch.bfloat16 else F32
+
+
+def forward_host(r, w, k, v, kk, a, S0, y, S_T, workspace, *, algo="auto", chunk=0, snap_every=0,
+                 snapshots=None, ln_w=None, ln_b=None, r_k=None, gn_eps=64e-5, segments=0, stream=None):
+    """wkv7_forward_host: every tensor but ``workspace`` is a host (CPU) tensor, pinned for
+    asynchronous copies; ``workspace`` is a device uint8 tensor of at least
+    ``forward_host_workspace_bytes`` bytes. Enqueues the copies and kernels on the current
+    stream of the workspace's device and returns; synchronise that stream before reading y,
+    S_T and the snapshots."""
+    lib = load()
+    B, T, H, N = r.shape
+    dev = workspace.device
+    opts = _host_opts(algo, chunk, snap_every, snapshots, ln_w, ln_b, r_k, gn_eps, segments)
+    with torch.cuda.device(dev):
+        st = lib.wkv7_forward_host(B, T, H, N, _dt(r), *(_host_ptr(t) for t in (r, w, k, v, kk, a, S0, y, S_T)),
+                                   ctypes.byref(opts), ctypes.c_void_p(workspace.data_ptr()),
+                                   workspace.numel() * workspace.element_size(), _stream_handle(dev, stream))
+    _check(st, "wkv7_forward_host")
+    return y, S_T, snapshots
