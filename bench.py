@@ -598,6 +598,8 @@ def run_layer(args, world, rank, local):
     ms = total_ms / steps
     units = B * T * H
     rk = inputs.LAYER_RANKS
+    rec_launches = wkv7.plan(B, T, H, N, torch.bfloat16, launches=True, ln_w=d["ln_w"], ln_b=d["ln_b"],
+                             r_k=d["r_k"])[2]
     gemm_flops = 2 * B * T * C * (4 * C + 2 * (rk["d_w"] + rk["d_a"] + rk["d_v"] + rk["d_g"]))
     peaks, peak_kind = _peaks()
     tc_peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops", 1590.0)))
@@ -616,9 +618,9 @@ def run_layer(args, world, rank, local):
                      "kernel": "whole layer step (GEMM flops over the step time; the recurrence runs inside it)",
                      "peak_source": f"{peak_kind} bf16 (sustained)", "gemm_flops_per_step": gemm_flops},
         "e2e": None, "clocks": clocks.summary(),
-        # this library's kernels per step: token shift, 2 activations, 2 bias adds, residual, the
-        # recurrence, gate, last token (the 12 GEMMs are cuBLASLt's and not counted)
-        "gpu_launches": steps * 9,
+        # this library's kernels per step: 8 low-rank factor copies, 12 GEMMs (mixes, activations,
+        # biases, residual and gate fused into them), the recurrence, the last-token copy
+        "gpu_launches": steps * (8 + 12 + rec_launches + 1),
     }
 
 

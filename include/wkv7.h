@@ -276,9 +276,12 @@ WKV7_API wkv7_status wkv7_backward_static(int B, int T, int H, int N, wkv7_dtype
  *     g = sigmoid(x_g Wg1) Wg2
  *     y = wkv7_forward_raw(r, w_logit, k, v, a_logit, k_k, k_a) with the epilogue (ln_w, ln_b, r_k)
  *     out = Wo (y * g)
- * The GEMMs run in cuBLASLt (fp32 accumulation; bf16 tensor cores for WKV7_BF16, fp32 for
- * WKV7_F32) on the caller's workspace; the element-wise steps and the recurrence are this
- * library's kernels. Intermediates are stored in dt (the logits' and gate's GEMMs in fp32).
+ * Every projection is this library's GEMM: tcgen05 tensor cores with bf16 operands and fp32
+ * accumulation for WKV7_BF16, the fp32 FMA pipe for WKV7_F32. The token-shift mixes are formed in
+ * each GEMM's operand load and tanh, sigmoid, the biases and the value residual in its store;
+ * r, k, v, the two logits and the low-rank hidden values are stored in dt, g and y in fp32, and the
+ * gate multiplies y inside the output projection's operand load. Each call also copies the
+ * low-rank factors, transposed and zero-padded to multiples of 64, into the workspace.
  *
  * dims:   H, N (64, or 128 on the scan), low-rank widths d_w, d_a, d_v, d_g (>= 1).
  * params: fp32 mixes and biases [C]; fp32 r_k, k_k, k_a, ln_w, ln_b [H][N] (k_a may be NULL);
@@ -296,7 +299,7 @@ WKV7_API wkv7_status wkv7_backward_static(int B, int T, int H, int N, wkv7_dtype
  * Errors: WKV7_ERR_ARG (sizes, NULL dims / params / required pointers, overlapping outputs,
  * host or too-small buffers, v0 without Wv1 / Wv2 / v_bias), WKV7_ERR_ALIGN (every
  * pointer 16-byte aligned), WKV7_ERR_UNSUPPORTED (N), WKV7_ERR_WORKSPACE, WKV7_ERR_CUDA (a launch
- * or a cuBLASLt call failed; the message names the step). T = 0 only copies last_x.
+ * failed; the message names the step). T = 0 only copies last_x.
  */
 typedef struct {
     int H, N;

@@ -76,9 +76,7 @@ def build(verbose: bool = False, extra_flags=()) -> str:
     stamp = LIB + ".stamp"
     if not os.path.exists(LIB) or not os.path.exists(stamp) or open(stamp).read() != link_tag:
         tmp = LIB + f".tmp{os.getpid()}"
-        # cuBLASLt for the time-mixing layer's GEMMs (resolved by soname at load time)
-        cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-cudart", "static", "-lcublasLt",
-               "-Xlinker", "-rpath,/usr/local/cuda/lib64"]
+        cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-cudart", "static"]
         res = subprocess.run(cmd, capture_output=True, text=True)
         if verbose or res.returncode:
             sys.stderr.write(" ".join(cmd) + "\n" + res.stdout + res.stderr)

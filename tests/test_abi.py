@@ -279,4 +279,9 @@ def test_layer_rejects_bad_arguments(lib):
     assert _layer_call(lib) == wkv7.ERR_WORKSPACE
     dims = wkv7.LayerDims(2, 64, 8, 8, 8, 8)
     assert lib.wkv7_layer_workspace_bytes(2, 0, 1, ctypes.byref(dims)) == 0
-    assert lib.wkv7_layer_workspace_bytes(2, 10, 1, ctypes.byref(dims)) > 32 << 20
+    # B2 T10, C = 128 channels, bf16, low-rank widths 8 (padded to 64): r, k, v and the two logits
+    # (bf16), four hidden values (bf16, 64 wide), g and y (fp32), and the transposed factors
+    up = lambda n: (n + 255) // 256 * 256
+    M, C = 20, 128
+    want = 5 * up(M * C * 2) + 4 * up(M * 64 * 2) + 2 * up(M * C * 4) + 8 * up(64 * C * 2)
+    assert lib.wkv7_layer_workspace_bytes(2, 10, 1, ctypes.byref(dims)) == want

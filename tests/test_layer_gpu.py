@@ -1,5 +1,6 @@
-"""GPU parity of the full time-mixing layer (cuBLASLt GEMMs, this library's element-wise
-kernels and recurrence) against the oracle's fp64 layer.
+"""GPU parity of the full time-mixing layer (this library's GEMMs with the token-shift mixes,
+activations, biases, value residual and gate fused into them, and its recurrence) against the
+oracle's fp64 layer.
 
 Bounds (max relative error per (b, h) slice of the output, as everywhere):
 * fp32 layer: 1e-4. The GEMMs accumulate in fp32 over at most C = 256 products (first-order
@@ -9,7 +10,8 @@ Bounds (max relative error per (b, h) slice of the output, as everywhere):
   2^-9 = 1.95e-3. The readout y = S r sees, to first order and in the worst case, r's two
   roundings (mixed input, projection), v's two, k's two, the decay's three (mixed input,
   low-rank hidden value, logit) and then the gated readout's one: 10 * 1.95e-3 = 1.95e-2,
-  plus the tf32 recurrence's 2e-3 bound.
+  plus the tf32 recurrence's 2e-3 bound. (g and y stay fp32; y * g is rounded once, as the
+  output projection's bf16 operand.)
 """
 import pytest
 import torch
