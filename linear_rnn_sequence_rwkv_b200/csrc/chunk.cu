@@ -88,14 +88,8 @@ struct Small {
     float ln_w[2][C], ln_b[2][C], r_k[2][C];   // epilogue parameters, by head parity
     float k_k[2][C], k_a[2][C];                 // raw inputs: removal-key scale, key-update rate
     float inv_norm[C];                          // raw inputs: 1 / max(||k_t * k_k||, 1e-12) per token
-    uint64_t bar_tma;         // the key-side input tiles (all but v) of the next chunk to prepare
-    uint64_t bar_tmav;        // the v tile of the next chunk (read by P4)
-    uint32_t tmaf_inflight;   // key-side tiles issued and not yet waited for (the first front thread)
-    uint32_t tmav_inflight;   // a v tile issued and not yet waited for (thread 0)
-    uint64_t bar_mma;         // the dependent rounds R2a-R5 (issued by thread 0)
-    uint64_t bar_r1;          // R1 (issued by the first front thread for the chunk it prepared)
-    uint64_t bar_r3;          // R3 has completed: T_D1 may take the next chunk's Grams
-    uint32_t r1_inflight;     // an R1 has been issued and not yet waited for
+    uint64_t bar_tma;
+    uint64_t bar_mma;
     uint64_t bar_state;       // split mode: the carried state has arrived in B5 (kSendThreads arrivals)
     uint64_t bar_credit;      // split mode: the next CTA has consumed the state last sent to it
     uint32_t tmem_base;
@@ -106,12 +100,13 @@ static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 // TMEM columns (512 allocated). A tf32 MMA with N = 64 costs nearly as much issue time as one
 // with N = 128, so products that share an A operand are merged into N = 128 rounds.
 constexpr uint32_t T_D1 = 0;     // Grams [M_ab | M_kb ; Q_b | Q_k] (R1); once read, Z (R2, 64 columns)
-constexpr uint32_t T_A2 = 128;   // A of R2: [Bi^T; Q_b]
-constexpr uint32_t T_D3R = 192;  // [Ki^T; Q_k] -> R3 subtracts Z M_kb -> [K~; Q~] (A of R4)
+constexpr uint32_t T_A2 = 128;   // A of R2: [Bi^T (transpose round); Q_b]
+constexpr uint32_t T_D3R = 192;  // [Ki^T (transpose round); Q_k] -> R3 subtracts Z M_kb -> [K~; Q~] (A of R4)
 constexpr uint32_t T_D3L = 256;  // [I; Rd] -> R3 subtracts Z KKd -> [I - X; R~] (A of R5)
 constexpr uint32_t T_D4 = 320;   // [S'^T; Y] (R4 + R5); the new state is diag(gC) S'^T
 constexpr uint32_t T_V = 384;    // R2b: U[:, 32:64] L21 (32 columns)
-static_assert(T_D3R + 64 == T_D3L, "R3 writes adjacent blocks");
+constexpr uint32_t T_ID = 448;   // identity (lanes 0-63) over zeros: A of the transpose round, written once
+static_assert(T_A2 + 64 == T_D3R && T_D3R + 64 == T_D3L, "transpose round and R3 write adjacent blocks");
 
 enum { XR = 0, XW = 1, XK = 2, XV = 3, XKK = 4, XA = 5 };
 
@@ -222,13 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     if (tid < 7) asm volatile("prefetch.tensormap [%0];" ::"l"(tid < 6 ? &maps.m[tid] : &maps.y) : "memory");
     if (tid == 0) {
         mbar_init(&S.bar_tma, 1);
-        mbar_init(&S.bar_tmav, 1);
-        S.tmaf_inflight = 0u;
-        S.tmav_inflight = 0u;
         mbar_init(&S.bar_mma, 1);
-        mbar_init(&S.bar_r1, 1);
-        mbar_init(&S.bar_r3, 1);
-        S.r1_inflight = 0u;
         mbar_init(&S.bar_state, kSendThreads);
         mbar_init(&S.bar_credit, 1);
         mbar_fence_init();
@@ -251,63 +240,45 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     const uint64_t dB1 = desc_sw128(smem_u32(sm + OFF_B1)), dB2 = desc_sw128(smem_u32(sm + OFF_B2));
     const uint64_t dB3 = desc_sw128(smem_u32(sm + OFF_B3)), dB4 = desc_sw128(smem_u32(sm + OFF_B4));
     const uint64_t dB5 = desc_sw128(smem_u32(sm + OFF_B5)), dA1 = desc_sw128(smem_u32(sm + OFF_A1));
-    uint32_t tma_parity = 0, tmav_parity = 0, mma_parity = 0, state_parity = 0, credit_parity = 0, r1_parity = 0,
-             r3_parity = 0;
+    const uint64_t dL21 = desc_sw128(smem_u32(sm + OFF_L21));
+    {   // identity over zeros in T_ID (A operand of the transposes; never overwritten)
+        float id8[8];
+#pragma unroll 1
+        for (int g = 0; g < 2; ++g) {
+            const int c8 = c16 + 8 * g;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) id8[e] = (c8 + e == L) ? 1.f : 0.f;
+            tmem_st8(tmem_addr(tb, Lq, T_ID + c8), id8);
+        }
+        tmem_st_wait();
+    }
+    uint32_t tma_parity = 0, mma_parity = 0, state_parity = 0, credit_parity = 0;
     int sends = 0;                     // states sent to the next CTA (warps 0-1)
     bool y_pending = false;            // the y tile in B2 still has to be stored (uniform)
     int y_h = 0, y_c0 = 0, y_b = 0;    // its coordinates
-    bool mma_pending = false, failed = false;
+    bool tma_pending = false, mma_pending = false, failed = false;
 
-    // The input tiles of a chunk arrive in two groups: the key-side tiles (all but v), read only by
-    // the front warps, and the v tile, read by P4. The key-side tiles of the chunk after next are
-    // loaded as soon as the front has finished with the current ones (end of the window); the v
-    // tile once P4 has read the current one.
-    constexpr uint32_t kFrontBytes = (RAW ? 4 : 5) * 8192;   // RAW has no kk tile
-    auto front_tile = [&](int x) { return x != XV && !(RAW && x == XKK); };
-    auto issue_front_tiles = [&](int u, int c) {   // one thread
+    constexpr uint32_t kTileBytes = (RAW ? 5 : 6) * 8192;   // RAW has no kk tile
+    auto issue_tma = [&](int u, int c) {   // one thread: the input tiles of chunk c of head u
         const int b = u / p.H, hh = u % p.H;
-        mbar_arrive_expect_tx(&S.bar_tma, kFrontBytes);
-        S.tmaf_inflight = 1u;
+        mbar_arrive_expect_tx(&S.bar_tma, kTileBytes);
 #pragma unroll
         for (int x = 0; x < 6; ++x)
-            if (front_tile(x)) tma_load_4d(sm + OFF_IN + x * 8192, &maps.m[x], &S.bar_tma, 0, hh, c * C, b);
-    };
-    auto issue_v_tile = [&](int u, int c) {   // one thread
-        mbar_arrive_expect_tx(&S.bar_tmav, 8192);
-        S.tmav_inflight = 1u;
-        tma_load_4d(sm + OFF_IN + XV * 8192, &maps.m[XV], &S.bar_tmav, 0, u % p.H, c * C, u / p.H);
-    };
-    // thread 0: the v tile of the chunk P4 is about to read has arrived (false: the wait gave up)
-    auto wait_v_tile = [&]() -> bool {
-        if (!mbar_wait_spin(&S.bar_tmav, tmav_parity, p.timeout_ns)) return false;
-        tmav_parity ^= 1u;
-        S.tmav_inflight = 0u;
-        return true;
-    };
-    // the chunk after (u, c) in this CTA's order, and whether it exists
-    auto advance = [&](int u, int c, int &nu, int &nc) -> bool {
-        nu = u; nc = c + cs;
-        if (nc >= nchunks) { nu = u + ncl; nc = rank; }
-        return nu < units && nc < nchunks;
+            if (!(RAW && x == XKK)) tma_load_4d(sm + OFF_IN + x * 8192, &maps.m[x], &S.bar_tma, 0, hh, c * C, b);
     };
     // Waits: one thread polls the mbarrier (bounded, acquire) and the others wait in a hardware
     // barrier with it; many polling threads would crowd the shared-memory pipe that the other
     // warp group is using. All threads; true on timeout (uniform across the CTA).
-    // All threads: R1 of the current chunk has completed. On a timeout the polling thread keeps
-    // the parity of the phase that did not complete, so the drain on the way out waits (bounded)
-    // for that phase; `S.r1_inflight` stays set.
-    auto wait_r1_all = [&]() -> bool {
-        const bool to = tid == 0 && !mbar_wait_spin(&S.bar_r1, r1_parity, p.timeout_ns);
-        if (tid == 0 && !to) {
-            r1_parity ^= 1u;
-            S.r1_inflight = 0u;
-        }
+    // On a timeout the issuing thread keeps the parity of the phase that did not complete and
+    // stays `mma_pending`, so the drain on the way out waits (bounded) for that phase.
+    auto wait_mma_all = [&]() -> bool {
+        const bool to = tid == 0 && !mbar_wait_spin(&S.bar_mma, mma_parity, p.timeout_ns);
+        if (!to) mma_parity ^= 1u;
+        mma_pending = to;
         const bool f = __syncthreads_or(to) != 0;
         tc_fence_after();
         return f;
     };
-    // On a timeout the issuing thread keeps the parity of the phase that did not complete and
-    // stays `mma_pending`, so the drain on the way out waits (bounded) for that phase.
     // warps 0-3 only; true on timeout here or (`extra`) in any of them
     auto wait_mma_back = [&](bool extra) -> bool {
         const bool to = tid == 0 && !mbar_wait_spin(&S.bar_mma, mma_parity, p.timeout_ns);
@@ -322,23 +293,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         tmem_st_wait();
         tc_fence_before();
         __syncthreads();
-    };
-    // R1 of the chunk whose operands the front warps have just written, issued by the first front
-    // thread after their barrier: Grams = [KKd; Rd] [Bi; Ki]^T into T_D1, committed to bar_r1.
-    // T_D1 last held Z, which R3 of the chunk before reads: with `after_r3` the thread first waits
-    // for R3's completion. True if that wait gave up (nothing issued then).
-    auto issue_r1 = [&](bool after_r3) -> bool {
-        if (after_r3) {
-            if (!mbar_wait_spin(&S.bar_r3, r3_parity, p.timeout_ns)) return true;
-            r3_parity ^= 1u;
-        }
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-            mma_tf32_ss(tb + T_D1, dA1 + kstep_off(ks, 128), dB1 + kstep_off(ks, 128), idesc_tf32(128, 128), ks > 0);
-        mma_commit(&S.bar_r1);
-        S.r1_inflight = 1u;
-        return false;
     };
     auto load_params = [&](int u, int slot, int i) {   // per-head parameters of head u, element i
         const int hh = u % p.H;
@@ -365,10 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     auto front = [&](int u, int c, int ip, int us) -> bool {
         const int Lc = min(C, p.T - c * C);
         const bool to = ft == 0 && !mbar_wait_spin(&S.bar_tma, tma_parity, p.timeout_ns);
-        if (ft == 0 && !to) {
-            tma_parity ^= 1u;
-            S.tmaf_inflight = 0u;
-        }
+        tma_parity ^= 1u;
         if (bar_named_or(BAR_FRONT, kFrontThreads, to)) return true;
         if (RAW) {
             // P0: the decay multipliers w = exp(-sigmoid(z)/sqrt(e)) of the whole tile into the decay
@@ -510,57 +461,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 S.bon[ip][t] = bon;
             }
         }
+        // the operand tiles are read next by the tensor core (R1 and the transpose round at the
+        // top of the chunk): generic-proxy writes -> visible to the async proxy
+        fence_proxy_async_smem();
         return false;
-    };
-
-    // ---- P4: the rest of a chunk's operand set, by all warps, from the tiles the front wrote
-    //      (shared memory) into the layouts the later rounds read.
-    //      Lanes 0-63 (key/value channel j = L): V^T row j -> B4; Bi^T and Ki^T row j -> lanes 0-63
-    //      of T_A2 and T_D3R (A operands of R2 and of R3/R4); identity row -> T_D3L.
-    //      Lanes 64-127 (key j = L - 64): KKd^T row j -> B3 rows 64-127; Rd row t = j -> T_D3L.
-    auto p4 = [&]() {
-        if (colg) {
-            const int j = L;
-            uint32_t xo[8], xk[8];
-            col_offsets(j, xo);
-            kcol_offsets(j, 128, xk);
-#pragma unroll 1
-            for (int g = 0; g < 2; ++g) {
-                const int t0 = c16 + 8 * g;
-                float vv[8], bi[8], ki[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    vv[e] = in_col(IN + XV * 8192, t0 + e, xo, e);
-                    bi[e] = *reinterpret_cast<const float *>(sm + OFF_B1 + (t0 + e) * 128 + xk[e]);
-                    ki[e] = *reinterpret_cast<const float *>(sm + OFF_B1 + (64 + t0 + e) * 128 + xk[e]);
-                }
-                st_f4(sm + OFF_B4, sw128_off(j, t0, 64), vv[0], vv[1], vv[2], vv[3]);
-                st_f4(sm + OFF_B4, sw128_off(j, t0 + 4, 64), vv[4], vv[5], vv[6], vv[7]);
-                tmem_st8(tmem_addr(tb, Lq, T_A2 + t0), bi);
-                tmem_st8(tmem_addr(tb, Lq, T_D3R + t0), ki);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) vv[e] = (t0 + e == L) ? 1.f : 0.f;
-                tmem_st8(tmem_addr(tb, Lq, T_D3L + t0), vv);
-            }
-        } else {
-            const int j = L - 64;
-            uint32_t xo[8];
-            kcol_offsets(j, 128, xo);
-            const uint8_t *b6 = sm + OFF_A1;
-#pragma unroll 1
-            for (int g = 0; g < 2; ++g) {
-                const int t0 = c16 + 8 * g;
-                float kkd[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) kkd[e] = *reinterpret_cast<const float *>(b6 + (t0 + e) * 128 + xo[e]);
-                st_f4(sm + OFF_B3, sw128_off(64 + j, t0, 128), kkd[0], kkd[1], kkd[2], kkd[3]);
-                st_f4(sm + OFF_B3, sw128_off(64 + j, t0 + 4, 128), kkd[4], kkd[5], kkd[6], kkd[7]);
-                const float4 ra = *reinterpret_cast<const float4 *>(b6 + sw128_off(64 + j, t0, 128));
-                const float4 rb = *reinterpret_cast<const float4 *>(b6 + sw128_off(64 + j, t0 + 4, 128));
-                const float rd[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
-                tmem_st8(tmem_addr(tb, Lq, T_D3L + t0), rd);   // Rd row (token j), channels t0..t0+7
-            }
-        }
     };
 
     // ---- output of chunk c of head u from T_D4, by all warps (each owns 16 columns of its lane
@@ -652,61 +556,98 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     };
 
     // ---- the CTA's chunks: (head u, chunk c), c = rank, rank + cs, ... of heads cid, cid + ncl, ...
-    // Per chunk, after the operands of the chunk (front warps) and its R1 and P4 are done:
-    //   masks and inverse (all warps) -> window: warps 0-3 run the dependent rounds R2a-R5 while
-    //   warps 4-15 prepare the next chunk's operands and then issue its R1 -> output of this chunk
-    //   and P4 of the next (all warps).
     int u = p.unit0 + cid, c = rank;
     bool valid = u < units && rank < nchunks;
     int ip = 0, us = 0;                // parity slots of the current chunk and head
     if (valid) {
-        if (ft == 0) issue_front_tiles(u, c);
-        if (tid == 0) issue_v_tile(u, c);
+        if (tid == 0) issue_tma(u, c);
+        tma_pending = true;
         if (tid < 64) load_params(u, 0, tid);
         if (rank == 0) load_state(u);
     }
     __syncthreads();
     {
-        bool f = false;
-        if (valid && !back) {
-            f = front(u, c, 0, 0);
-            if (!f) {
-                int u2, c2;
-                const bool more2 = advance(u, c, u2, c2);
-                fence_proxy_async_smem();   // the operand tiles -> visible to R1
-                bar_named(BAR_FRONT, kFrontThreads);
-                if (ft == 0) {
-                    if (more2) issue_front_tiles(u2, c2);   // the key-side tiles have been read
-                    f = issue_r1(false);
-                }
-            }
-        }
-        if (valid && tid == 0 && !wait_v_tile()) f = true;
+        const bool f = valid && !back ? front(u, c, 0, 0) : false;
         failed = __syncthreads_or(f) != 0;
-        if (valid && !failed) {
-            tc_fence_after();
-            p4();
-            sync_for_mma();
-            tc_fence_after();
-        }
+        if (valid && back) tma_parity ^= 1u;
+        if (!failed) tma_pending = false;
     }
 
     while (valid && !failed) {
         const int b = u / p.H, hh = u % p.H, c0 = c * C;
-        int nu, nc;
-        const bool more = advance(u, c, nu, nc);
+        int nu = u, nc = c + cs;
+        if (nc >= nchunks) { nu = u + ncl; nc = rank; }
+        const bool more = nu < units && nc < nchunks;
         const bool new_unit = more && nu != u;
         const bool recv = cs > 1 && c > 0;   // split mode: this chunk's start state comes from CTA rank-1
 
-        if (wait_r1_all()) { failed = true; break; }
-        // the previous chunk's y tile goes out now; the next chunk's v tile comes in (P4 of this
-        // chunk, the last reader of the v tile, is done)
+        if (tid == 0) {
+            // the next chunk's six input tiles are issued by six warps in P5; their byte count
+            // is registered here, ordered before those issues by the barrier after R1
+            if (more) mbar_arrive_expect_tx(&S.bar_tma, kTileBytes);
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)   // R1: Grams = [KKd; Rd] [Bi; Ki]^T
+                mma_tf32_ss(tb + T_D1, dA1 + kstep_off(ks, 128), dB1 + kstep_off(ks, 128), idesc_tf32(128, 128), ks > 0);
+            // transpose round on the tensor core (exact: identity times tf32 operands), N = 128:
+            // lanes 0-63 of T_A2 <- Bi^T (A of R2), of T_D3R <- Ki^T (start of K~)
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_tf32_ts(tb + T_A2, tb + T_ID + 8 * ks, dB1 + kstep_off(ks, 128), idesc_tf32(128, 128), ks > 0);
+            mma_commit(&S.bar_mma);
+        }
+        mma_pending = true;
+        // the previous chunk's y tile goes out now: every warp has slack while R1 runs
         if (y_pending && tid == kStoreThread) store_y_tile(maps, sm + OFF_B2, y_h, y_c0, y_b);
         y_pending = false;
-        if (more && tid == 0) issue_v_tile(nu, nc);
+        // ---- P4 (while the MMAs run): transposes through shared memory and the start of
+        //      T_D3L (the previous chunk's R5 has read it).
+        //      Lanes 0-63 (key/value channel j = L): V^T row j -> B4; identity row -> T_D3L.
+        //      Lanes 64-127 (key j = L - 64): KKd^T row j -> B3 rows 64-127; Rd row t = j -> T_D3L.
+        if (colg) {
+            const int j = L;
+            uint32_t xo[8];
+            col_offsets(j, xo);
+#pragma unroll 1
+            for (int g = 0; g < 2; ++g) {
+                const int t0 = c16 + 8 * g;
+                float vv[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) vv[e] = in_col(IN + XV * 8192, t0 + e, xo, e);
+                st_f4(sm + OFF_B4, sw128_off(j, t0, 64), vv[0], vv[1], vv[2], vv[3]);
+                st_f4(sm + OFF_B4, sw128_off(j, t0 + 4, 64), vv[4], vv[5], vv[6], vv[7]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) vv[e] = (t0 + e == L) ? 1.f : 0.f;
+                tmem_st8(tmem_addr(tb, Lq, T_D3L + t0), vv);
+            }
+        } else {
+            const int j = L - 64;
+            uint32_t xo[8];
+            kcol_offsets(j, 128, xo);
+            const uint8_t *b6 = sm + OFF_A1;
+#pragma unroll 1
+            for (int g = 0; g < 2; ++g) {
+                const int t0 = c16 + 8 * g;
+                float kkd[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) kkd[e] = *reinterpret_cast<const float *>(b6 + (t0 + e) * 128 + xo[e]);
+                st_f4(sm + OFF_B3, sw128_off(64 + j, t0, 128), kkd[0], kkd[1], kkd[2], kkd[3]);
+                st_f4(sm + OFF_B3, sw128_off(64 + j, t0 + 4, 128), kkd[4], kkd[5], kkd[6], kkd[7]);
+                const float4 ra = *reinterpret_cast<const float4 *>(b6 + sw128_off(64 + j, t0, 128));
+                const float4 rb = *reinterpret_cast<const float4 *>(b6 + sw128_off(64 + j, t0 + 4, 128));
+                const float rd[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+                tmem_st8(tmem_addr(tb, Lq, T_D3L + t0), rd);   // Rd row (token j), channels t0..t0+7
+            }
+        }
+        if (wait_mma_all()) { failed = true; break; }
         // ---- P5: masks. Lanes 0-63 (token t): M_ab row -> inverse workspace; M_kb row t ->
         //      column t of B3 rows 0-63 (M_kb^T, scalar stores along K: conflict-free).
         //      Lanes 64-127 (token t): Q_b row -> T_A2 lanes 64-127; Q_k row -> T_D3R lanes 64-127.
+        if (more && lane == 0 && colg && (warp >> 2) < 3) {
+            // the input tiles were last read in P4: six warps each issue one tile of the next chunk
+            const int x = (warp >> 2) * 2 + (warp & 1);
+            if (!(RAW && x == XKK)) tma_load_4d(sm + OFF_IN + x * 8192, &maps.m[x], &S.bar_tma, 0, nu % p.H, nc * C, nu / p.H);
+        }
         if (colg) {
             const int t = L;
             float m[2][8], mk[2][8];
@@ -728,6 +669,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 for (int e = 0; e < 8; ++e)   // B3[s][t] = M_kb[t][s], nonzero for s < t
                     *reinterpret_cast<float *>(sm + OFF_B3 + (s0 + e) * 128 + xo[e]) =
                         (s0 + e < t) ? to_tf32(mk[g][e]) : 0.f;
+            }
+            if (t >= 32 && c16 < 32) {   // L21^T[s][t - 32] = M_ab[t][s] (s < 32 <= t: no mask)
+                uint32_t xl[8];
+                kcol_offsets(t - 32, 32, xl);
+#pragma unroll
+                for (int g = 0; g < 2; ++g)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        *reinterpret_cast<float *>(sm + OFF_L21 + (c16 + 8 * g + e) * 128 + xl[e]) = to_tf32(m[g][e]);
             }
         } else {
             const int t = L - 64;
@@ -755,6 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         }
         if (tid == kStoreThread) tma_store_wait_read();   // the y tile in B2 has been read
         sync_for_mma();
+        tma_pending = more;
         // ---- A = (I + M_ab)^{-1}. Diagonal 16x16 blocks: one thread per (block, column)
         //      solves (I + L_dd) x = e_c by forward substitution in registers (warps 2, 3).
         if (tid >= 64 && tid < 128) {
@@ -776,15 +727,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 st_f4(sm + OFF_B2, sw128_off(16 * d + cc, 16 * d + 4 * m, 64), to_tf32(x[4 * m]), to_tf32(x[4 * m + 1]),
                       to_tf32(x[4 * m + 2]), to_tf32(x[4 * m + 3]));
         } else {
-            // B2 = A^T (row n, K = s holds A[s][n]): zero where A is, i.e. above its diagonal: s in
-            // the first 32-half and n in the second, or both in one half with s's 16-block before
-            // n's (the diagonal, level-1 and level-2 blocks are written by their producers)
+            // B2 = D^T, D = blockdiag(Y0, Y1): zero where t and s lie in different 32-halves or
+            // t's 16-block precedes s's (the diagonal blocks and the level-1 blocks are written by
+            // their producers)
             const int z = tid < 64 ? tid : tid - 64;
 #pragma unroll 1
             for (int e = z; e < 1024; e += kThreads - 64) {
                 const int sr = e & 63, t4 = (e >> 6) * 4;
-                if ((sr >= 32 && t4 < 32) || (((t4 ^ sr) < 32) && ((t4 >> 4) < (sr >> 4))))
-                    st_f4(sm + OFF_B2, sw128_off(sr, t4, 64), 0.f, 0.f, 0.f, 0.f);
+                if (((t4 ^ sr) >= 32) || ((t4 >> 4) < (sr >> 4))) st_f4(sm + OFF_B2, sw128_off(sr, t4, 64), 0.f, 0.f, 0.f, 0.f);
             }
         }
         __syncthreads();
@@ -801,8 +751,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 acc[2] = fmaf(lv, xv.z, acc[2]); acc[3] = fmaf(lv, xv.w, acc[3]);
             }
             *reinterpret_cast<float4 *>(Tw + (pp * 16 + i) * 20 + j4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            // Y_p's block above its diagonal is zero (level 2 reads Y_p whole)
-            *reinterpret_cast<float4 *>(Aw + (32 * pp + i) * LWS + 32 * pp + 16 + j4) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         __syncthreads();
         if (tid < 128) {
@@ -815,47 +763,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                 acc[0] = fmaf(xv, tv.x, acc[0]); acc[1] = fmaf(xv, tv.y, acc[1]);
                 acc[2] = fmaf(xv, tv.z, acc[2]); acc[3] = fmaf(xv, tv.w, acc[3]);
             }
-            // the block X[2p+1][2p] goes to Aw (fp32, for level 2) and transposed into B2 (row = column
-            // of A, K = row of A), tf32
+            // the block X[2p+1][2p] of D goes transposed into B2 (row s = column of D, K = t), tf32
             const int t = 32 * pp + 16 + i;
-            *reinterpret_cast<float4 *>(Aw + t * LWS + 32 * pp + j4) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 *reinterpret_cast<float *>(sm + OFF_B2 + sw128_off(32 * pp + j4 + q, t, 64)) = to_tf32(-acc[q]);
         }
-        __syncthreads();
-        // level 2: the off-diagonal block of A = (I + M_ab)^{-1}, X21 = -Y1 (L21 Y0), with Y0, Y1 the
-        // inverses of the diagonal 32x32 blocks and L21 = M_ab[32:64][0:32]. Threads 0-255 each
-        // compute four adjacent outputs; T2 = L21 Y0 is kept in Aw's (otherwise unused) block
-        // above the diagonal.
-        if (tid < 256) {
-            const int i = tid >> 3, j4 = (tid & 7) * 4;
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-            for (int k = 0; k < 32; ++k) {
-                const float lv = Lw[(32 + i) * LWS + k];
-                const float4 yv = *reinterpret_cast<const float4 *>(Aw + k * LWS + j4);
-                acc[0] = fmaf(lv, yv.x, acc[0]); acc[1] = fmaf(lv, yv.y, acc[1]);
-                acc[2] = fmaf(lv, yv.z, acc[2]); acc[3] = fmaf(lv, yv.w, acc[3]);
-            }
-            *reinterpret_cast<float4 *>(Aw + i * LWS + 32 + j4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        }
-        __syncthreads();
-        if (tid < 256) {
-            const int i = tid >> 3, j4 = (tid & 7) * 4;
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-            for (int k = 0; k < 32; ++k) {
-                const float yv = Aw[(32 + i) * LWS + 32 + k];
-                const float4 tv = *reinterpret_cast<const float4 *>(Aw + k * LWS + 32 + j4);
-                acc[0] = fmaf(yv, tv.x, acc[0]); acc[1] = fmaf(yv, tv.y, acc[1]);
-                acc[2] = fmaf(yv, tv.z, acc[2]); acc[3] = fmaf(yv, tv.w, acc[3]);
-            }
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<float *>(sm + OFF_B2 + sw128_off(j4 + q, 32 + i, 64)) = to_tf32(-acc[q]);
-        }
-        // B2 now holds A^T, the whole inverse
+        // B2 now holds D^T, D = blockdiag(Y0, Y1) the inverses of the two diagonal 32x32 blocks of
+        // I + M_ab; the off-diagonal block of the inverse, -Y1 L21 Y0, is applied by R2b/R2c.
         sync_for_mma();
 
         // ---- the window: warps 0-3 run this chunk's dependent MMA rounds and its output,
@@ -865,11 +780,33 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
             if (tid == 0) {
                 tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)   // R2: Z = W A, W = [Bi^T; Q_b]
+                for (int ks = 0; ks < 8; ++ks)   // R2a: U = W D, W = [Bi^T; Q_b]
                     mma_tf32_ts(tb + T_D1, tb + T_A2 + 8 * ks, dB2 + kstep_off(ks, 64), idesc_tf32(128, 64), ks > 0);
                 mma_commit(&S.bar_mma);
             }
             wfail = wait_mma_back(false);
+            // Z = W A with A = D - [0 0; Y1 L21 Y0 0]: Z[:, 32:64] = U[:, 32:64] and
+            // Z[:, 0:32] = U[:, 0:32] - (U[:, 32:64] L21) Y0 (block back-substitution on the tensor core)
+            if (!wfail) {
+                if (tid == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)   // R2b: V = U[:, 32:64] L21
+                        mma_tf32_ts(tb + T_V, tb + T_D1 + 32 + 8 * ks, dL21 + kstep_off(ks, 32), idesc_tf32(128, 32), ks > 0);
+                    mma_commit(&S.bar_mma);
+                }
+                wfail = wait_mma_back(false);
+            }
+            if (!wfail) {
+                if (tid == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)   // R2c: U[:, 0:32] -= V Y0 (B2 rows 0-31 hold Y0^T)
+                        mma_tf32_ts(tb + T_D1, tb + T_V + 8 * ks, dB2 + kstep_off(ks, 64), idesc_neg_a(idesc_tf32(128, 32)), 1);
+                    mma_commit(&S.bar_mma);
+                }
+                wfail = wait_mma_back(false);
+            }
             if (!wfail) {
                 if (tid == 0) {
                     tc_fence_after();
@@ -878,7 +815,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                         mma_tf32_ts(tb + T_D3R, tb + T_D1 + 8 * ks, dB3 + kstep_off(ks, 128),
                                     idesc_neg_a(idesc_tf32(128, 128)), 1);
                     mma_commit(&S.bar_mma);
-                    if (more) mma_commit(&S.bar_r3);   // Z has been read: T_D1 may take the next Grams
                 }
                 wfail = wait_mma_back(false);
             }
@@ -910,16 +846,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         } else if (more) {
             if (new_unit && ft < 64) load_params(nu, us ^ 1, ft);
             wfail = front(nu, nc, ip ^ 1, new_unit ? (us ^ 1) : us);
-            if (!wfail) {
-                int u2, c2;
-                const bool more2 = advance(nu, nc, u2, c2);
-                fence_proxy_async_smem();     // the operand tiles -> visible to R1
-                bar_named(BAR_FRONT, kFrontThreads);
-                if (ft == 0) {
-                    if (more2) issue_front_tiles(u2, c2);   // the key-side tiles have been read
-                    wfail = issue_r1(true);
-                }
-            }
+            if (!wfail) tma_pending = false;   // these threads saw the tiles arrive
         }
         // split mode: before writing the next CTA's B5, its credit for the state sent before
         const bool send = cs > 1 && c + 1 < nchunks;
@@ -927,15 +854,19 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
             if (tid == 0 && !wfail) wfail = !mbar_wait_cluster(&S.bar_credit, credit_parity, p.handoff_timeout_ns);
             credit_parity ^= 1u;
         }
-        if (more && tid == 0 && !wfail) wfail = !wait_v_tile();   // P4 below reads it
         tc_fence_before();
         if (__syncthreads_or(wfail)) { failed = true; break; }
         tc_fence_after();
         out(u, c, ip, us, send);
         if (send) ++sends;
-        if (more) p4();   // the next chunk's transposes, while its R1 runs
-        sync_for_mma();
+        tc_fence_before();
+        __syncthreads();
         tc_fence_after();
+        // keep the barrier parities uniform: warps 0-3 completed five MMA rounds, warps 4-15
+        // consumed the next chunk's tiles
+        if (!back) mma_parity ^= 1u;
+        if (back && more) tma_parity ^= 1u;
+        tma_pending = false;
         mma_pending = false;
         y_pending = true;
         y_h = hh; y_c0 = c0; y_b = b;
@@ -953,14 +884,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         if (tid == 0) atomicOr(p.err, 1u);
         // drain what this CTA issued (bounded), then release tensor memory
         if (mma_pending) mbar_wait(&S.bar_mma, mma_parity, p.timeout_ns);
+        if (tma_pending) mbar_wait(&S.bar_tma, tma_parity, p.timeout_ns);
     }
-    tc_fence_before();
-    __syncthreads();
-    // loads and an R1 issued for chunks that were never processed (a failure in between) are
-    // drained by the thread that polls their barrier, with the parity of that phase
-    if (tid == 0 && S.r1_inflight) mbar_wait(&S.bar_r1, r1_parity, p.timeout_ns);
-    if (tid == 0 && S.tmav_inflight) mbar_wait(&S.bar_tmav, tmav_parity, p.timeout_ns);
-    if (ft == 0 && S.tmaf_inflight) mbar_wait(&S.bar_tma, tma_parity, p.timeout_ns);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tb, 512);

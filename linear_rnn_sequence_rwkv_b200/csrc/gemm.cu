@@ -21,6 +21,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -32,6 +33,18 @@ namespace {
 using namespace tc;
 
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + __expf(-z)); }
+
+// Named barrier over `n` threads that also ORs a predicate (the result is uniform).
+__device__ __forceinline__ bool bar_or(int id, int n, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(uint32_t(v)), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
 
 __device__ __forceinline__ float apply_epi(int epi, float z, float bias, float v, float v0) {
     switch (epi) {
@@ -52,67 +65,77 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 }
 
 // ---- bf16 on tcgen05 -------------------------------------------------------------------------------
-constexpr int kProdThreads = 256;                 // warps 0-7: A preparation, then the store
-constexpr int kGemmThreads = kProdThreads + 64;   // warp 8: TMA of W; warp 9: MMA issue and TMEM
-constexpr int kStages = 3;
+constexpr int kProdThreads = 256;                 // warps 0-7: A preparation (MIX, GATE), then the store
+constexpr int kGemmThreads = kProdThreads + 64;   // warp 8: TMA; warp 9: MMA issue and TMEM
+constexpr int kStages = 4;
 
+// One stage: the A tile (128 rows x 64 K, bf16, 128-byte swizzle), the previous-token tile of the
+// mix (the same rows shifted by one token), and the W tile (BN rows).
 template <int BN>
 struct GemmSmem {
-    static constexpr uint32_t A = 128 * 128, B = BN * 128;   // bytes of one stage's A and W tiles
-    static constexpr uint32_t bytes = kStages * (A + B) + 1024 + 256;
+    static constexpr uint32_t A = 128 * 128, XP = 128 * 128, B = BN * 128, STAGE = A + XP + B;
+    static constexpr uint32_t bytes = kStages * STAGE + 1024 + 256;
 };
 
-// Eight bf16 values of A's row m, columns k..k+7 (k a multiple of 8), prepared as `pro` says.
-__device__ __forceinline__ uint4 prep_a8(const GemmArgs &a, int m, int k) {
+// GATE: eight bf16 values of A's row m, columns k..k+7 (k a multiple of 8): y * g from fp32.
+__device__ __forceinline__ uint4 gate_a8(const GemmArgs &a, int m, int k) {
     if (m >= a.M) return make_uint4(0u, 0u, 0u, 0u);
-    float o[8];
-    if (a.pro == GEMM_PLAIN) {
-        return __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.A) + size_t(m) * a.lda + k));
-    } else if (a.pro == GEMM_MIX) {
-        const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(a.x);
-        const uint4 xc = __ldg(reinterpret_cast<const uint4 *>(x + size_t(m) * a.K + k));
-        uint4 xp = make_uint4(0u, 0u, 0u, 0u);
-        if (m % a.T != 0) xp = __ldg(reinterpret_cast<const uint4 *>(x + size_t(m - 1) * a.K + k));
-        else if (a.last_x)
-            xp = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.last_x) +
-                                                       size_t(m / a.T) * a.K + k));
-        const float4 m0 = __ldg(reinterpret_cast<const float4 *>(a.mix + k));
-        const float4 m1 = __ldg(reinterpret_cast<const float4 *>(a.mix + k + 4));
-        const float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-        const uint32_t xcw[4] = {xc.x, xc.y, xc.z, xc.w}, xpw[4] = {xp.x, xp.y, xp.z, xp.w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float xi = bf(xcw[e >> 1], e & 1), pi = bf(xpw[e >> 1], e & 1);
-            o[e] = fmaf(mv[e], pi - xi, xi);
-        }
-    } else {   // GATE: y * g, both fp32
-        const float *yr = a.y + size_t(m) * a.K + k, *gr = static_cast<const float *>(a.g) + size_t(m) * a.K + k;
-        const float4 y0 = __ldg(reinterpret_cast<const float4 *>(yr)), y1 = __ldg(reinterpret_cast<const float4 *>(yr + 4));
-        const float4 g0 = __ldg(reinterpret_cast<const float4 *>(gr)), g1 = __ldg(reinterpret_cast<const float4 *>(gr + 4));
-        o[0] = y0.x * g0.x; o[1] = y0.y * g0.y; o[2] = y0.z * g0.z; o[3] = y0.w * g0.w;
-        o[4] = y1.x * g1.x; o[5] = y1.y * g1.y; o[6] = y1.z * g1.z; o[7] = y1.w * g1.w;
-    }
-    return make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
+    const float *yr = a.y + size_t(m) * a.K + k, *gr = static_cast<const float *>(a.g) + size_t(m) * a.K + k;
+    const float4 y0 = __ldg(reinterpret_cast<const float4 *>(yr)), y1 = __ldg(reinterpret_cast<const float4 *>(yr + 4));
+    const float4 g0 = __ldg(reinterpret_cast<const float4 *>(gr)), g1 = __ldg(reinterpret_cast<const float4 *>(gr + 4));
+    return make_uint4(pack_bf16(y0.x * g0.x, y0.y * g0.y), pack_bf16(y0.z * g0.z, y0.w * g0.w),
+                      pack_bf16(y1.x * g1.x, y1.y * g1.y), pack_bf16(y1.z * g1.z, y1.w * g1.w));
 }
 
+// MIX, in place in the stage: A chunk (row r, 16-byte chunk at byte `off` of the swizzled tile)
+// <- x + m (x_prev - x), with x_prev from the shifted tile, or last_x (0 without it) when row
+// m0 + r starts a sequence.
+__device__ __forceinline__ void mix_chunk(const GemmArgs &a, uint8_t *at, const uint8_t *xpt, int m, int k,
+                                          uint32_t off) {
+    if (m >= a.M) return;
+    uint4 xc = *reinterpret_cast<const uint4 *>(at + off), xp;
+    if (m % a.T != 0) xp = *reinterpret_cast<const uint4 *>(xpt + off);
+    else if (a.last_x)
+        xp = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.last_x) + size_t(m / a.T) * a.K + k));
+    else xp = make_uint4(0u, 0u, 0u, 0u);
+    const float4 m0 = __ldg(reinterpret_cast<const float4 *>(a.mix + k));
+    const float4 m1 = __ldg(reinterpret_cast<const float4 *>(a.mix + k + 4));
+    const float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+    const uint32_t xcw[4] = {xc.x, xc.y, xc.z, xc.w}, xpw[4] = {xp.x, xp.y, xp.z, xp.w};
+    float o[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const float xi = bf(xcw[e >> 1], e & 1), pi = bf(xpw[e >> 1], e & 1);
+        o[e] = fmaf(mv[e], pi - xi, xi);
+    }
+    *reinterpret_cast<uint4 *>(at + off) =
+        make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
+}
+
+// PLAIN: A by TMA straight into the stage. MIX: x and the previous-token rows by TMA, mixed in
+// place by warps 0-7. GATE: A formed by warps 0-7 from global memory. W always by TMA.
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_kernel(const __grid_constant__ CUtensorMap wmap,
+                                                                    const __grid_constant__ CUtensorMap amap,
                                                                     const GemmArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
     using L = GemmSmem<BN>;
-    uint8_t *sA = sm, *sB = sm + kStages * L::A;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kStages * (L::A + L::B));
-    uint64_t *full_a = bars, *full_b = bars + kStages, *empty = bars + 2 * kStages, *acc_full = bars + 3 * kStages;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kStages * L::STAGE);
+    uint64_t *full_t = bars, *full_a = bars + kStages, *empty = bars + 2 * kStages, *acc_full = bars + 3 * kStages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * kStages + 1);
+    auto stA = [&](int s) { return sm + s * L::STAGE; };
+    auto stXP = [&](int s) { return sm + s * L::STAGE + L::A; };
+    auto stB = [&](int s) { return sm + s * L::STAGE + L::A + L::XP; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int m0 = blockIdx.x * 128, n0 = blockIdx.y * BN, nkb = a.K / 64;
+    const bool tma_a = a.pro != GEMM_GATE, mix = a.pro == GEMM_MIX, prod = a.pro != GEMM_PLAIN;
     const uint64_t tmo = 2000000000ull;
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full_t[s], 1);
             mbar_init(&full_a[s], kProdThreads);
-            mbar_init(&full_b[s], 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(acc_full, 1);
@@ -129,39 +152,46 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_kernel(const __grid
     bool bad = false;
 
     if (warp < 8) {
-        // ---- A preparation: 1024 16-byte chunks per stage, four per thread; chunk q of row r goes
-        //      to chunk position q ^ (r % 8) of the row (128-byte swizzle, K-major)
-        for (int kb = 0; kb < nkb && !bad; ++kb) {
-            const int s = kb % kStages;
-            if (!mbar_wait(&empty[s], ((kb / kStages) & 1) ^ 1, tmo)) { bad = true; break; }
-            uint8_t *dst = sA + s * L::A;
+        if (prod) {
+            // 1024 16-byte chunks per stage, four per thread; chunk q of row r sits at chunk position
+            // q ^ (r % 8) of the row (128-byte swizzle, K-major). Thread 0 polls the stage's barrier,
+            // the others wait for it in a named barrier.
+            for (int kb = 0; kb < nkb && !bad; ++kb) {
+                const int s = kb % kStages;
+                const uint32_t ph = (kb / kStages) & 1;
+                const bool to = tid == 0 && (mix ? !mbar_wait_spin(&full_t[s], ph, tmo) : !mbar_wait_spin(&empty[s], ph ^ 1, tmo));
+                if (bar_or(1, kProdThreads, to)) { bad = true; break; }
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int idx = tid + kProdThreads * i, r = idx >> 3, q = idx & 7;
-                const uint4 v = prep_a8(a, m0 + r, kb * 64 + q * 8);
-                *reinterpret_cast<uint4 *>(dst + r * 128 + ((q ^ (r & 7)) << 4)) = v;
+                for (int i = 0; i < 4; ++i) {
+                    const int idx = tid + kProdThreads * i, r = idx >> 3, q = idx & 7;
+                    const uint32_t off = r * 128 + ((q ^ (r & 7)) << 4);
+                    if (mix) mix_chunk(a, stA(s), stXP(s), m0 + r, kb * 64 + q * 8, off);
+                    else *reinterpret_cast<uint4 *>(stA(s) + off) = gate_a8(a, m0 + r, kb * 64 + q * 8);
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&full_a[s]);
             }
-            fence_proxy_async_smem();
-            mbar_arrive(&full_a[s]);
         }
     } else if (warp == 8) {
         if (lane == 0) {
+            const uint32_t bytes = L::B + (tma_a ? L::A : 0u) + (mix ? L::XP : 0u);
             for (int kb = 0; kb < nkb; ++kb) {
                 const int s = kb % kStages;
-                if (!mbar_wait(&empty[s], ((kb / kStages) & 1) ^ 1, tmo)) { bad = true; break; }
-                mbar_arrive_expect_tx(&full_b[s], L::B);
-                tma_load_2d(sB + s * L::B, &wmap, &full_b[s], kb * 64, n0);
+                if (!mbar_wait_spin(&empty[s], ((kb / kStages) & 1) ^ 1, tmo)) { bad = true; break; }
+                mbar_arrive_expect_tx(&full_t[s], bytes);
+                tma_load_2d(stB(s), &wmap, &full_t[s], kb * 64, n0);
+                if (tma_a) tma_load_2d(stA(s), &amap, &full_t[s], kb * 64, m0);
+                if (mix) tma_load_2d(stXP(s), &amap, &full_t[s], kb * 64, m0 - 1);   // row -1: zeros
             }
         }
     } else if (lane == 0) {
         // ---- MMA issue: four K = 16 steps per stage, then the stage goes back to its producers
-        int kb = 0;
-        for (; kb < nkb; ++kb) {
+        for (int kb = 0; kb < nkb; ++kb) {
             const int s = kb % kStages;
             const uint32_t ph = (kb / kStages) & 1;
-            if (!mbar_wait(&full_a[s], ph, tmo) || !mbar_wait(&full_b[s], ph, tmo)) { bad = true; break; }
+            if (!mbar_wait_spin(&full_t[s], ph, tmo) || (prod && !mbar_wait_spin(&full_a[s], ph, tmo))) { bad = true; break; }
             tc_fence_after();
-            const uint64_t dA = desc_sw128(smem_u32(sA + s * L::A)), dB = desc_sw128(smem_u32(sB + s * L::B));
+            const uint64_t dA = desc_sw128(smem_u32(stA(s))), dB = desc_sw128(smem_u32(stB(s)));
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16_ss(tb, dA + uint64_t(2 * ks), dB + uint64_t(2 * ks), idesc_bf16(128, BN), (kb | ks) != 0);
@@ -172,7 +202,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_kernel(const __grid
 
     // ---- store: warp w reads TMEM lanes 32 (w % 4) .. + 31 (rows), columns of its half
     if (warp < 8) {
-        const bool ok = mbar_wait(acc_full, 0, tmo);
+        const bool ok = !bar_or(1, kProdThreads, tid == 0 && !mbar_wait_spin(acc_full, 0, tmo));
         if (!ok) bad = true;
         tc_fence_after();
         const int q = warp & 3, h = warp >> 2, m = m0 + 32 * q + lane;
@@ -309,23 +339,29 @@ PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
     return fn;
 }
 
+bool encode_bf16_2d(CUtensorMap *map, const void *base, int cols, int rows, int ld, int box_rows) {
+    auto enc = tmap_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+    const cuuint64_t strides[1] = {cuuint64_t(ld) * 2};
+    const cuuint32_t box[2] = {64, cuuint32_t(box_rows)}, es[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int BN>
 cudaError_t launch_bf16(const GemmArgs &a, cudaStream_t stream) {
-    auto enc = tmap_encoder();
-    if (!enc) return cudaErrorNotSupported;
-    CUtensorMap map;
-    const cuuint64_t dims[2] = {cuuint64_t(a.K), cuuint64_t(a.N)};
-    const cuuint64_t strides[1] = {cuuint64_t(a.K) * 2};
-    const cuuint32_t box[2] = {64, cuuint32_t(BN)}, es[2] = {1, 1};
-    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.W), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return cudaErrorInvalidValue;
+    CUtensorMap wmap, amap;
+    std::memset(&amap, 0, sizeof(amap));
+    if (!encode_bf16_2d(&wmap, a.W, a.K, a.N, a.K, BN)) return cudaErrorInvalidValue;
+    if (a.pro == GEMM_PLAIN && !encode_bf16_2d(&amap, a.A, a.K, a.M, a.lda, 128)) return cudaErrorInvalidValue;
+    if (a.pro == GEMM_MIX && !encode_bf16_2d(&amap, a.x, a.K, a.M, a.K, 128)) return cudaErrorInvalidValue;
     const int smem = int(GemmSmem<BN>::bytes);
     cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void *>(gemm_bf16_kernel<BN>), smem);
     if (e != cudaSuccess) return e;
     const dim3 grid(unsigned((a.M + 127) / 128), unsigned(a.N / BN));
-    gemm_bf16_kernel<BN><<<grid, kGemmThreads, smem, stream>>>(map, a);
+    gemm_bf16_kernel<BN><<<grid, kGemmThreads, smem, stream>>>(wmap, amap, a);
     return cudaGetLastError();
 }
 
