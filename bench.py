@@ -618,9 +618,10 @@ def run_layer(args, world, rank, local):
                      "kernel": "whole layer step (GEMM flops over the step time; the recurrence runs inside it)",
                      "peak_source": f"{peak_kind} bf16 (sustained)", "gemm_flops_per_step": gemm_flops},
         "e2e": None, "clocks": clocks.summary(),
-        # this library's kernels per step: 8 low-rank factor copies, 12 GEMMs (mixes, activations,
-        # biases, residual and gate fused into them), the recurrence, the last-token copy
-        "gpu_launches": steps * (8 + 12 + rec_launches + 1),
+        # this library's kernels per step: the low-rank factor copies, the grouped GEMM over the
+        # mixed x (7 products), the grouped second factors (4), the recurrence, the output
+        # projection (gate fused into its operand), the last-token copy
+        "gpu_launches": steps * (1 + 1 + 1 + rec_launches + 1 + 1),
     }
 
 

@@ -61,36 +61,6 @@ struct BwdArgs {
     cudaStream_t stream;
 };
 
-// One projection of the time-mixing layer (gemm.cu): D[M][N] = op(A)[M][K] * W[N][K]^T, all
-// matrices row-major in the layer dtype unless noted; op prepares A (GEMM_PLAIN / MIX / GATE)
-// and the store applies GEMM_STORE / TANH / SIGMOID / BIAS / RESIDUAL (dtype out) or GEMM_F32.
-enum { GEMM_PLAIN = 0, GEMM_MIX = 1, GEMM_GATE = 2 };
-enum { GEMM_STORE = 0, GEMM_TANH = 1, GEMM_SIGMOID = 2, GEMM_BIAS = 3, GEMM_RESIDUAL = 4, GEMM_F32 = 5 };
-struct GemmArgs {
-    int M, N, K;            // bf16: K and N multiples of 64
-    int pro;
-    const void *A;          // PLAIN: [M][lda]
-    int lda;
-    const void *x;          // MIX: x [M][K] (rows b * T + t), last_x [M / T][K] or null, mix [K] fp32
-    const void *last_x;
-    const float *mix;
-    int T;
-    const float *y;         // GATE: y [M][K] fp32 times g [M][K] fp32
-    const void *g;
-    const void *W;          // [N][K]
-    int epi;
-    void *D;                // [M][ldd]; RESIDUAL reads v from it
-    int ldd;
-    const float *bias;      // [N] (BIAS, RESIDUAL)
-    const void *v0;         // RESIDUAL: [M][ldd]
-    void *D2;               // optional second copy of the result
-    unsigned int *err;      // device error word (a bounded wait that gave up)
-};
-cudaError_t launch_gemm(const GemmArgs &a, wkv7_dtype dt, cudaStream_t stream);
-// out [out_rows][out_cols] = transpose of in [rows][cols], zero outside it.
-cudaError_t launch_transpose_pad(const void *in, void *out, int rows, int cols, int out_rows, int out_cols,
-                                 wkv7_dtype dt, cudaStream_t stream);
-
 // Launchers (each returns the launch status; no synchronisation).
 cudaError_t launch_seq(const FwdArgs &p);
 cudaError_t launch_epilogue(const FwdArgs &p);

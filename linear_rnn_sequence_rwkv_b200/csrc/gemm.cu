@@ -1,30 +1,34 @@
-// The projections of the time-mixing layer: D[M][N] = op(A)[M][K] * W[N][K]^T with the operand's
-// preparation fused into its load and the element-wise step after the product fused into the
-// store (RWKV-7 rebuttal page, numpy time_mixing listing: the token-shift mixes feed the square
-// projections and the low-rank first factors; tanh, sigmoid, the biases and the value residual
-// follow them; the gate multiplies the readout before the output projection).
+// The projections of the time-mixing layer: D_i[M][N_i] = op(A)[M][K_i] * W_i[N_i][K_i]^T for up to
+// seven products per launch, with the operand's preparation fused into its load and the
+// element-wise step after each product fused into its store (RWKV-7 rebuttal page, numpy
+// time_mixing listing: the token-shift mixes feed the square projections and the low-rank first
+// factors; tanh, sigmoid, the biases and the value residual follow them).
 //
-// Operand preparation (A, per element, in fp32, then rounded to the layer dtype):
-//   PLAIN  A itself;
-//   MIX    x + m (x_prev - x), x_prev the previous token of the same sequence (last_x, or 0,
-//          for the first token);
-//   GATE   y * g (both fp32).
-// Store (per element of the fp32 accumulator z, column n):
+// Operand preparation (per element, in fp32, then rounded to the layer dtype):
+//   PLAIN  A_i itself;
+//   MIX    x + m_i (x_prev - x), x_prev the previous token of the same sequence (last_x, or 0,
+//          for the first token).
+// Store (per element of the fp32 accumulator z, column n of problem i):
 //   STORE z;  TANH tanh(z);  SIGMOID sigmoid(z);  BIAS z + bias[n];
 //   RESIDUAL v + (v0 - v) sigmoid(z + bias[n]) with v the value already in D;  F32 z in fp32.
 //
-// bf16 layers: tcgen05.mma kind::f16 (bf16 operands, fp32 accumulation in tensor memory), a
-// 128 x BN output tile per CTA, K in blocks of 64. W arrives by TMA (128-byte swizzle); eight
-// warps prepare A into the same swizzled layout and later read the accumulator back; one thread
-// issues the MMAs. fp32 layers: a shared-memory tiled FMA GEMM with the same preparation and
-// store steps (exact fp32 products, fp32 accumulation).
+// bf16: a persistent kernel, one CTA per SM, walking 128-row output tiles (all the launch's
+// problems for one row block, then the next block, so that a block of x is read from HBM once).
+// Warp 12 streams W (and A or x) by TMA into a ring of shared-memory stages (128-byte swizzle);
+// warps 0-7 prepare the MIX operand into the stage; warp 13 issues tcgen05.mma (bf16
+// operands, fp32 accumulation) into one of two tensor-memory accumulators of up to 256 columns;
+// warps 8-11 read the other accumulator back (one TMEM lane quarter each) and store it, so that
+// a tile's store overlaps the next tile's products. fp32: a shared-memory tiled FMA GEMM with the
+// same preparation and store steps (exact fp32 products, fp32 accumulation), one launch per
+// problem.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
-#include "common.cuh"
+#include "gemm.cuh"
 #include "tc_util.cuh"
 
 namespace wkv7 {
@@ -32,29 +36,9 @@ namespace {
 
 using namespace tc;
 
-__device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + __expf(-z)); }
-
-// Named barrier over `n` threads that also ORs a predicate (the result is uniform).
-__device__ __forceinline__ bool bar_or(int id, int n, bool v) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"(uint32_t(v)), "r"(id), "r"(n)
-        : "memory");
-    return r != 0;
-}
-
-__device__ __forceinline__ float apply_epi(int epi, float z, float bias, float v, float v0) {
-    switch (epi) {
-        case GEMM_TANH: return tanhf(z);
-        case GEMM_SIGMOID: return sigmoidf_(z);
-        case GEMM_BIAS: return z + bias;
-        case GEMM_RESIDUAL: return fmaf(v0 - v, sigmoidf_(z + bias), v);
-        default: return z;
-    }
-}
+// 1 / (1 + e^-z) with the hardware reciprocal: no slow path for large or non-finite arguments
+// (e^-z = inf gives 0, the limit).
+__device__ __forceinline__ float sigmoidf_(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
 
 __device__ __forceinline__ float bf(uint32_t packed, int hi) {
     return __uint_as_float(hi ? (packed & 0xffff0000u) : (packed << 16));
@@ -64,221 +48,483 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     return *reinterpret_cast<const uint32_t *>(&h);
 }
 
+// Shared-memory accesses with an explicit state space (the staging tiles are addressed as
+// 32-bit shared addresses).
+__device__ __forceinline__ void st_shared_f4(uint32_t a, float4 v) {
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
+}
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t a) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a) : "memory");
+    return v;
+}
 // ---- bf16 on tcgen05 -------------------------------------------------------------------------------
-constexpr int kProdThreads = 256;                 // warps 0-7: A preparation (MIX, GATE), then the store
-constexpr int kGemmThreads = kProdThreads + 64;   // warp 8: TMA; warp 9: MMA issue and TMEM
-constexpr int kStages = 4;
+constexpr int kProdWarps = 8;                 // warps 0-7: MIX operand preparation
+constexpr int kEpiWarp0 = 8;                  // warps 8-11: accumulator read-back and store
+constexpr int kTmaWarp = 12, kMmaWarp = 13;
+constexpr int kGemmThreads = 14 * 32;
+constexpr int kAccCols = 256;                 // one accumulator: 128 lanes x up to 256 fp32 columns
+constexpr uint32_t kTileA = 128 * 128;        // 128 rows x 64 bf16
+constexpr uint32_t kTileB = 256 * 128;        // up to 256 rows x 64 bf16
+constexpr uint64_t kWaitNs = 2000000000ull;
 
-// One stage: the A tile (128 rows x 64 K, bf16, 128-byte swizzle), the previous-token tile of the
-// mix (the same rows shifted by one token), and the W tile (BN rows).
-template <int BN>
-struct GemmSmem {
-    static constexpr uint32_t A = 128 * 128, XP = 128 * 128, B = BN * 128, STAGE = A + XP + B;
-    static constexpr uint32_t bytes = kStages * STAGE + 1024 + 256;
+// One stage: the W tile, the A tile as loaded (x for the mix), and for MIX the prepared operand
+// (OP: where the products read A).
+// After the ring: per store warp two 4 KB output staging tiles, and for PLAIN two pairs of 2 KB
+// tiles for the value residual's v and v0.
+template <int PRO>
+struct Ring {
+    static constexpr uint32_t B = 0, A = kTileB, P = kTileB + kTileA, OP = PRO == GEMM_MIX ? P : A;
+    static constexpr uint32_t stage = kTileB + kTileA + (PRO == GEMM_MIX ? kTileA : 0u);
+    static constexpr int stages = 3;
+    static constexpr uint32_t out_off = stages * stage;             // [warp][2] x 4096
+    static constexpr uint32_t res_off = out_off + 4 * 2 * 4096;     // PLAIN: [warp][2] x (v 2048, v0 2048)
+    static constexpr uint32_t bar_off = res_off + (PRO == GEMM_PLAIN ? 4 * 2 * 4096 : 0u);
+    static constexpr uint32_t bytes = bar_off + 256 + 1024;   // + barriers, + 1 KB alignment slack
 };
 
-// GATE: eight bf16 values of A's row m, columns k..k+7 (k a multiple of 8): y * g from fp32.
-__device__ __forceinline__ uint4 gate_a8(const GemmArgs &a, int m, int k) {
-    if (m >= a.M) return make_uint4(0u, 0u, 0u, 0u);
-    const float *yr = a.y + size_t(m) * a.K + k, *gr = static_cast<const float *>(a.g) + size_t(m) * a.K + k;
-    const float4 y0 = __ldg(reinterpret_cast<const float4 *>(yr)), y1 = __ldg(reinterpret_cast<const float4 *>(yr + 4));
-    const float4 g0 = __ldg(reinterpret_cast<const float4 *>(gr)), g1 = __ldg(reinterpret_cast<const float4 *>(gr + 4));
-    return make_uint4(pack_bf16(y0.x * g0.x, y0.y * g0.y), pack_bf16(y0.z * g0.z, y0.w * g0.w),
-                      pack_bf16(y1.x * g1.x, y1.y * g1.y), pack_bf16(y1.z * g1.z, y1.w * g1.w));
+struct GemmProb {
+    int N, K, bn, tile0;   // bn: columns per tile (64, 128 or 256); tile0: first column tile of the problem
+    int epi, ldd, Kx;      // Kx: row length of x (MIX)
+    const float *mix, *bias;
+    const void *v0;
+    void *D;
+};
+struct GemmDev {
+    int M, T, nprob, ntn, ntiles;   // ntn: column tiles per row block over all problems
+    const void *x, *last_x;
+    unsigned int *err;
+    GemmProb p[kGemmMaxProblems];
+};
+struct GemmParams {
+    CUtensorMap wmap[kGemmMaxProblems];
+    CUtensorMap amap[kGemmMaxProblems];   // PLAIN: problem i's A; MIX: amap[0] is x
+    CUtensorMap dmap[kGemmMaxProblems];   // D in boxes of 32 x 32 (the stores; RESIDUAL also loads v)
+    CUtensorMap v0map;                    // RESIDUAL: v0, same boxes
+    GemmDev d;
+};
+
+struct Tile {
+    int m0, pi, n0;
+};
+__device__ __forceinline__ Tile tile_of(const GemmDev &d, int t) {
+    const int mt = t / d.ntn, nt = t - mt * d.ntn;
+    int i = 0;
+    while (i + 1 < d.nprob && nt >= d.p[i + 1].tile0) ++i;
+    return Tile{mt * 128, i, (nt - d.p[i].tile0) * d.p[i].bn};
 }
 
-// MIX, in place in the stage: A chunk (row r, 16-byte chunk at byte `off` of the swizzled tile)
-// <- x + m (x_prev - x), with x_prev from the shifted tile, or last_x (0 without it) when row
-// m0 + r starts a sequence.
-__device__ __forceinline__ void mix_chunk(const GemmArgs &a, uint8_t *at, const uint8_t *xpt, int m, int k,
-                                          uint32_t off) {
-    if (m >= a.M) return;
-    uint4 xc = *reinterpret_cast<const uint4 *>(at + off), xp;
-    if (m % a.T != 0) xp = *reinterpret_cast<const uint4 *>(xpt + off);
-    else if (a.last_x)
-        xp = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.last_x) + size_t(m / a.T) * a.K + k));
-    else xp = make_uint4(0u, 0u, 0u, 0u);
-    const float4 m0 = __ldg(reinterpret_cast<const float4 *>(a.mix + k));
-    const float4 m1 = __ldg(reinterpret_cast<const float4 *>(a.mix + k + 4));
-    const float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-    const uint32_t xcw[4] = {xc.x, xc.y, xc.z, xc.w}, xpw[4] = {xp.x, xp.y, xp.z, xp.w};
-    float o[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const float xi = bf(xcw[e >> 1], e & 1), pi = bf(xpw[e >> 1], e & 1);
-        o[e] = fmaf(mv[e], pi - xi, xi);
+// Wait for a phase: at most kWaitNs, and not past an abort raised by another role.
+__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    if (mbar_test_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_test_wait(bar, parity)) return true;
+        if ((i & 255u) == 0 && (*abort || globaltimer_ns() - t0 > kWaitNs)) {
+            *abort = 1;
+            return false;
+        }
     }
-    *reinterpret_cast<uint4 *>(at + off) =
-        make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
+}
+// The same with a pause between polls, for waits that are long and not on the critical path:
+// a tight poll takes issue slots from the warps that share the scheduler.
+__device__ __forceinline__ bool wait_phase_idle(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    if (mbar_test_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        __nanosleep(100);
+        if (mbar_test_wait(bar, parity)) return true;
+        if ((i & 15u) == 0 && (*abort || globaltimer_ns() - t0 > kWaitNs)) {
+            *abort = 1;
+            return false;
+        }
+    }
+}
+// Lane 0 waits, the warp learns the outcome.
+__device__ __forceinline__ bool warp_wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort, int lane,
+                                                bool idle = false) {
+    int ok = 0;
+    if (lane == 0) ok = idle ? wait_phase_idle(bar, parity, abort) : wait_phase(bar, parity, abort);
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-// PLAIN: A by TMA straight into the stage. MIX: x and the previous-token rows by TMA, mixed in
-// place by warps 0-7. GATE: A formed by warps 0-7 from global memory. W always by TMA.
-template <int BN>
-__global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_kernel(const __grid_constant__ CUtensorMap wmap,
-                                                                    const __grid_constant__ CUtensorMap amap,
-                                                                    const GemmArgs a) {
+// The store warps. Each owns 32 accumulator rows (its TMEM lane quarter, token rows m0 .. m0 + 31)
+// and moves them out 32 columns at a time: tcgen05.ld puts row `lane` in the lane's registers,
+// the element-wise step runs there, the lane writes its row into a staging tile in the layout
+// of the output's tensor map (bf16: 64-byte rows, 16-byte chunk c at c ^ ((row >> 1) & 3), the
+// 64-byte swizzle; fp32: 128-byte rows, chunk c at c ^ (row & 7), the 128-byte swizzle), and one
+// lane hands the tile to a TMA store. The value residual's v (the current D) and v0 arrive the
+// same way, by TMA loads into the same 64-byte-swizzled layout, one chunk ahead.
+struct StoreCtx {
+    uint8_t *out;               // two 4 KB staging tiles
+    uint8_t *res;               // two (v, v0) pairs of 2 KB tiles (PLAIN)
+    uint64_t *vbar;             // two barriers, one per pair
+    uint32_t vuse[2];           // completed phases of each barrier
+    volatile int *abort;        // raised when a wait gives up
+};
+
+template <int EPI>
+__device__ __noinline__ void store_tile(const GemmProb p, const CUtensorMap *dmap, const CUtensorMap *v0map,
+                                        uint32_t tacc, int m0, int n0, StoreCtx &cx, int lane) {
+    const int nch = p.bn / 32;
+    const float *const bias_p = p.bias;
+    auto fetch_res = [&](int j) {   // v and v0 of chunk j into pair j & 1
+        if (lane == 0) {
+            uint8_t *r = cx.res + (j & 1) * 4096;
+            mbar_arrive_expect_tx(&cx.vbar[j & 1], 4096);
+            tma_load_2d(r, dmap, &cx.vbar[j & 1], n0 + 32 * j, m0);
+            tma_load_2d(r + 2048, v0map, &cx.vbar[j & 1], n0 + 32 * j, m0);
+        }
+    };
+    if constexpr (EPI == GEMM_RESIDUAL) fetch_res(0);
+#pragma unroll 1
+    for (int j = 0; j < nch; ++j) {
+        if constexpr (EPI == GEMM_RESIDUAL)
+            if (j + 1 < nch) fetch_res(j + 1);   // its pair was last read in chunk j - 1
+        float z[32];
+        tmem_ld32(tacc + uint32_t(32 * j), z);
+        const int n = n0 + 32 * j;
+        if constexpr (EPI == GEMM_BIAS || EPI == GEMM_RESIDUAL) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+                const float4 b = __ldg(reinterpret_cast<const float4 *>(bias_p + n + e));
+                z[e] += b.x; z[e + 1] += b.y; z[e + 2] += b.z; z[e + 3] += b.w;
+            }
+        }
+        if constexpr (EPI == GEMM_TANH) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) z[e] = tanhf(z[e]);
+        } else if constexpr (EPI == GEMM_SIGMOID) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) z[e] = sigmoidf_(z[e]);
+        } else if constexpr (EPI == GEMM_RESIDUAL) {
+            const int b = j & 1;
+            int ok = 1;
+            if (lane == 0) ok = wait_phase(&cx.vbar[b], cx.vuse[b] & 1, cx.abort);   // polled: wakes on time
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            ++cx.vuse[b];
+            const uint32_t rv = smem_u32(cx.res + b * 4096) + uint32_t(lane * 64);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint32_t off = uint32_t((c ^ ((lane >> 1) & 3)) << 4);
+                const float4 va = ld_shared_f4(rv + off), v0a = ld_shared_f4(rv + 2048 + off);
+                const uint32_t vw[4] = {__float_as_uint(va.x), __float_as_uint(va.y), __float_as_uint(va.z),
+                                        __float_as_uint(va.w)};
+                const uint32_t v0w[4] = {__float_as_uint(v0a.x), __float_as_uint(v0a.y), __float_as_uint(v0a.z),
+                                         __float_as_uint(v0a.w)};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float v = bf(vw[e >> 1], e & 1);
+                    z[8 * c + e] = ok ? fmaf(bf(v0w[e >> 1], e & 1) - v, sigmoidf_(z[8 * c + e]), v) : 0.f;
+                }
+            }
+        }
+        // staging tile j & 1: its store from chunk j - 2 has finished reading it
+        uint8_t *o = cx.out + (j & 1) * 4096;
+        if (lane == 0) tma_store_wait_read1();
+        __syncwarp();
+        if constexpr (EPI == GEMM_F32) {
+            const uint32_t ro = smem_u32(o) + uint32_t(lane * 128);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                st_shared_f4(ro + uint32_t((c ^ (lane & 7)) << 4), make_float4(z[4 * c], z[4 * c + 1], z[4 * c + 2], z[4 * c + 3]));
+        } else {
+            const uint32_t ro = smem_u32(o) + uint32_t(lane * 64);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float4 w = make_float4(__uint_as_float(pack_bf16(z[8 * c], z[8 * c + 1])),
+                                             __uint_as_float(pack_bf16(z[8 * c + 2], z[8 * c + 3])),
+                                             __uint_as_float(pack_bf16(z[8 * c + 4], z[8 * c + 5])),
+                                             __uint_as_float(pack_bf16(z[8 * c + 6], z[8 * c + 7])));
+                st_shared_f4(ro + uint32_t((c ^ ((lane >> 1) & 3)) << 4), w);
+            }
+        }
+        fence_proxy_async_smem();   // the staging writes -> visible to the TMA unit
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(dmap, o, n, m0);   // rows past M are clipped by the tensor map
+            tma_store_commit();
+        }
+    }
+}
+
+// MIX: the thread's four chunks (rows rb + 32 i, 16-byte chunk q) of the prepared operand, from
+// the loaded x tile (the row before comes from the same tile, except for tile row 0 and the
+// first token of a sequence: those come from global memory, loaded by mix_fetch before the
+// stage's wait).
+struct MixFetch {
+    float mv[8];
+    uint4 xp[4];
+};
+// The operand sources, copied out of the kernel parameters into registers once (reads through a
+// reference to the parameters would be repeated after every shared-memory store).
+struct Src {
+    const __nv_bfloat16 *x, *last_x;
+    const float *mix;
+    int M, T, K;
+};
+__device__ __forceinline__ void mix_fetch(MixFetch &f, const Src &d, int m0, int kb, int rb, int q,
+                                          uint32_t first_mask) {
+    const int k = kb * 64 + q * 8;
+    const float4 mA = __ldg(reinterpret_cast<const float4 *>(d.mix + k));
+    const float4 mB = __ldg(reinterpret_cast<const float4 *>(d.mix + k + 4));
+    f.mv[0] = mA.x; f.mv[1] = mA.y; f.mv[2] = mA.z; f.mv[3] = mA.w;
+    f.mv[4] = mB.x; f.mv[5] = mB.y; f.mv[6] = mB.z; f.mv[7] = mB.w;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = rb + 32 * i, m = m0 + r;
+        f.xp[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (first_mask >> i & 1u) {   // the row starts a sequence: last_x of its sequence, or zeros
+            if (d.last_x) f.xp[i] = __ldg(reinterpret_cast<const uint4 *>(d.last_x + size_t(m / d.T) * d.K + k));
+        } else if (r == 0 && m < d.M) {
+            f.xp[i] = __ldg(reinterpret_cast<const uint4 *>(d.x + size_t(m - 1) * d.K + k));
+        }
+    }
+}
+__device__ __forceinline__ void mix_stage(const MixFetch &f, const uint8_t *xt, uint8_t *pt, int rb, int q,
+                                          uint32_t first_mask) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = rb + 32 * i;
+        const uint32_t off = uint32_t(r) * 128u + (uint32_t(q ^ (r & 7)) << 4);
+        const uint4 xp = ((first_mask >> i & 1u) || r == 0)
+                             ? f.xp[i]
+                             : *reinterpret_cast<const uint4 *>(xt + uint32_t(r - 1) * 128u + (uint32_t(q ^ ((r - 1) & 7)) << 4));
+        const uint4 xc = *reinterpret_cast<const uint4 *>(xt + off);
+        const uint32_t xcw[4] = {xc.x, xc.y, xc.z, xc.w}, xpw[4] = {xp.x, xp.y, xp.z, xp.w};
+        float o[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float xi = bf(xcw[e >> 1], e & 1), pi = bf(xpw[e >> 1], e & 1);
+            o[e] = fmaf(f.mv[e], pi - xi, xi);
+        }
+        *reinterpret_cast<uint4 *>(pt + off) =
+            make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
+    }
+}
+
+template <int PRO>
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_kernel(const __grid_constant__ GemmParams P) {
+    using R = Ring<PRO>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
-    using L = GemmSmem<BN>;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kStages * L::STAGE);
-    uint64_t *full_t = bars, *full_a = bars + kStages, *empty = bars + 2 * kStages, *acc_full = bars + 3 * kStages;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * kStages + 1);
-    auto stA = [&](int s) { return sm + s * L::STAGE; };
-    auto stXP = [&](int s) { return sm + s * L::STAGE + L::A; };
-    auto stB = [&](int s) { return sm + s * L::STAGE + L::A + L::XP; };
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + R::bar_off);
+    uint64_t *full_t = bars, *full_a = bars + 4, *empty = bars + 8, *acc_full = bars + 12, *acc_empty = bars + 14;
+    uint64_t *drain = bars + 16, *vbars = bars + 17;   // vbars: [store warp][2]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 25);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 26);
+    auto stage = [&](int s) { return sm + s * R::stage; };
 
+    const GemmDev &d = P.d;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int m0 = blockIdx.x * 128, n0 = blockIdx.y * BN, nkb = a.K / 64;
-    const bool tma_a = a.pro != GEMM_GATE, mix = a.pro == GEMM_MIX, prod = a.pro != GEMM_PLAIN;
-    const uint64_t tmo = 2000000000ull;
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < R::stages; ++s) {
             mbar_init(&full_t[s], 1);
-            mbar_init(&full_a[s], kProdThreads);
+            mbar_init(&full_a[s], kProdWarps);   // one arrival per preparing warp
             mbar_init(&empty[s], 1);
         }
-        mbar_init(acc_full, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);         // one arrival per store warp
+        }
+        mbar_init(drain, 1);
+        for (int i = 0; i < 8; ++i) mbar_init(&vbars[i], 1);
+        *abort = 0;
         mbar_fence_init();
     }
-    if (warp == 9) {
-        tmem_alloc(tmem_slot, BN);
+    if (warp == kMmaWarp) {
+        tmem_alloc(tmem_slot, 2 * kAccCols);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tb = *tmem_slot;
-    bool bad = false;
 
-    if (warp < 8) {
-        if (prod) {
-            // 1024 16-byte chunks per stage, four per thread; chunk q of row r sits at chunk position
-            // q ^ (r % 8) of the row (128-byte swizzle, K-major). Thread 0 polls the stage's barrier,
-            // the others wait for it in a named barrier.
-            for (int kb = 0; kb < nkb && !bad; ++kb) {
-                const int s = kb % kStages;
-                const uint32_t ph = (kb / kStages) & 1;
-                const bool to = tid == 0 && (mix ? !mbar_wait_spin(&full_t[s], ph, tmo) : !mbar_wait_spin(&empty[s], ph ^ 1, tmo));
-                if (bar_or(1, kProdThreads, to)) { bad = true; break; }
+    if (warp == kTmaWarp) {
+        if (lane == 0) {
+            for (int i = 0; i < d.nprob; ++i) {
+                prefetch_tensormap(&P.wmap[i]);
+                if (PRO == GEMM_PLAIN || (PRO == GEMM_MIX && i == 0)) prefetch_tensormap(&P.amap[i]);
+            }
+            int it = 0;
+            for (int t = blockIdx.x; t < d.ntiles && !*abort; t += gridDim.x) {
+                const Tile tl = tile_of(d, t);
+                const GemmProb &p = d.p[tl.pi];
+                const uint32_t bytes = uint32_t(p.bn) * 128u + kTileA;
+                const CUtensorMap *am = &P.amap[PRO == GEMM_PLAIN ? tl.pi : 0];
+                for (int kb = 0; kb < p.K / 64; ++kb, ++it) {
+                    const int s = it % R::stages;
+                    if (!wait_phase(&empty[s], ((it / R::stages) & 1) ^ 1, abort)) break;
+                    mbar_arrive_expect_tx(&full_t[s], bytes);
+                    tma_load_2d(stage(s) + R::B, &P.wmap[tl.pi], &full_t[s], kb * 64, tl.n0);
+                    tma_load_2d(stage(s) + R::A, am, &full_t[s], kb * 64, tl.m0);
+                }
+            }
+            // the loads still in flight land before the CTA leaves
+            for (int j = std::max(0, it - R::stages); j < it; ++j)
+                mbar_wait_spin(&full_t[j % R::stages], (j / R::stages) & 1, kWaitNs);
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            int it = 0, lt = 0;
+            for (int t = blockIdx.x; t < d.ntiles && !*abort; t += gridDim.x, ++lt) {
+                const Tile tl = tile_of(d, t);
+                const GemmProb &p = d.p[tl.pi];
+                const int b = lt & 1;
+                if (!wait_phase(&acc_empty[b], ((lt >> 1) & 1) ^ 1, abort)) break;
+                tc_fence_after();
+                const uint32_t tacc = tb + uint32_t(b * kAccCols), idesc = idesc_bf16(128, p.bn);
+                bool ok = true;
+                for (int kb = 0; kb < p.K / 64; ++kb, ++it) {
+                    const int s = it % R::stages;
+                    const uint32_t ph = (it / R::stages) & 1;
+                    if (!wait_phase(&full_t[s], ph, abort) || (PRO != GEMM_PLAIN && !wait_phase(&full_a[s], ph, abort))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint8_t *a_op = stage(s) + R::OP;
+                    const uint64_t dA = desc_sw128(smem_u32(a_op)), dB = desc_sw128(smem_u32(stage(s) + R::B));
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16_ss(tacc, dA + uint64_t(2 * ks), dB + uint64_t(2 * ks), idesc, (kb | ks) != 0);
+                    mma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                mma_commit(&acc_full[b]);
+            }
+            // every product issued has completed before the accumulators are freed
+            mma_commit(drain);
+            mbar_wait_spin(drain, 0, kWaitNs);   // polled: a suspended wait can wake late
+        }
+    } else if (warp >= kEpiWarp0) {
+        const int quarter = warp & 3, ew = warp - kEpiWarp0;
+        StoreCtx cx{sm + R::out_off + ew * 8192, sm + R::res_off + ew * 8192, vbars + 2 * ew, {0u, 0u}, abort};
+        if (lane == 0) {
+            for (int i = 0; i < d.nprob; ++i) prefetch_tensormap(&P.dmap[i]);
+        }
+        int lt = 0;
+        for (int t = blockIdx.x; t < d.ntiles; t += gridDim.x, ++lt) {
+            const Tile tl = tile_of(d, t);
+            const GemmProb p = d.p[tl.pi];
+            const int b = lt & 1;
+            if (!warp_wait_phase(&acc_full[b], (lt >> 1) & 1, abort, lane, true)) break;
+            tc_fence_after();
+            const uint32_t tacc = tmem_addr(tb, 32 * quarter, b * kAccCols);
+            const int m0 = tl.m0 + 32 * quarter;
+            const CUtensorMap *dm = &P.dmap[tl.pi];
+            switch (p.epi) {
+                case GEMM_TANH: store_tile<GEMM_TANH>(p, dm, &P.v0map, tacc, m0, tl.n0, cx, lane); break;
+                case GEMM_SIGMOID: store_tile<GEMM_SIGMOID>(p, dm, &P.v0map, tacc, m0, tl.n0, cx, lane); break;
+                case GEMM_BIAS: store_tile<GEMM_BIAS>(p, dm, &P.v0map, tacc, m0, tl.n0, cx, lane); break;
+                case GEMM_RESIDUAL:
+                    if (PRO == GEMM_PLAIN) store_tile<GEMM_RESIDUAL>(p, dm, &P.v0map, tacc, m0, tl.n0, cx, lane);
+                    break;
+                case GEMM_F32: store_tile<GEMM_F32>(p, dm, &P.v0map, tacc, m0, tl.n0, cx, lane); break;
+                default: store_tile<GEMM_STORE>(p, dm, &P.v0map, tacc, m0, tl.n0, cx, lane); break;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[b]);
+        }
+        if (lane == 0) tma_store_wait_all();   // the stores have landed before the CTA leaves
+    } else if (PRO == GEMM_MIX) {
+        // operand preparation: the thread owns chunk q of rows rb, rb + 32, rb + 64, rb + 96. The
+        // global operands of a stage (its mix values, and the rows before the tile or a sequence)
+        // are fetched one stage ahead, so that their latency overlaps the previous stage's work.
+        const int q = tid & 7, rb = tid >> 3;
+        const int ntiles = d.ntiles;
+        Src src{static_cast<const __nv_bfloat16 *>(d.x), static_cast<const __nv_bfloat16 *>(d.last_x), nullptr, d.M,
+                d.T, 0};
+        struct Pos {
+            int t, kb, nkb, m0;
+            uint32_t first_mask;
+            const float *mix;
+            int K;
+        };
+        auto tile_pos = [&](int t) {
+            Pos ps{t, 0, 0, 0, 0u, nullptr, 0};
+            if (t < ntiles) {
+                const Tile tl = tile_of(d, t);
+                ps.nkb = d.p[tl.pi].K / 64;
+                ps.m0 = tl.m0;
+                ps.mix = d.p[tl.pi].mix;
+                ps.K = d.p[tl.pi].Kx;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int idx = tid + kProdThreads * i, r = idx >> 3, q = idx & 7;
-                    const uint32_t off = r * 128 + ((q ^ (r & 7)) << 4);
-                    if (mix) mix_chunk(a, stA(s), stXP(s), m0 + r, kb * 64 + q * 8, off);
-                    else *reinterpret_cast<uint4 *>(stA(s) + off) = gate_a8(a, m0 + r, kb * 64 + q * 8);
+                    const int m = tl.m0 + rb + 32 * i;
+                    if (m < src.M && m % src.T == 0) ps.first_mask |= 1u << i;
                 }
-                fence_proxy_async_smem();
-                mbar_arrive(&full_a[s]);
             }
+            return ps;
+        };
+        auto fetch = [&](MixFetch &f, const Pos &ps) {
+            src.mix = ps.mix;
+            src.K = ps.K;
+            mix_fetch(f, src, ps.m0, ps.kb, rb, q, ps.first_mask);
+        };
+        Pos cur = tile_pos(blockIdx.x);
+        MixFetch fc, fn;
+        if (cur.t < ntiles) fetch(fc, cur);
+        for (int it = 0; cur.t < ntiles; ++it) {
+            Pos nxt = cur;
+            if (++nxt.kb == cur.nkb) nxt = tile_pos(cur.t + gridDim.x);
+            if (nxt.t < ntiles) fetch(fn, nxt);
+            const int s = it % R::stages;
+            if (!warp_wait_phase(&full_t[s], (it / R::stages) & 1, abort, lane)) break;
+            mix_stage(fc, stage(s) + R::A, stage(s) + R::OP, rb, q, cur.first_mask);
+            fence_proxy_async_smem();   // generic-proxy writes -> visible to the tensor core
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full_a[s]);
+            cur = nxt;
+            fc = fn;
         }
-    } else if (warp == 8) {
-        if (lane == 0) {
-            const uint32_t bytes = L::B + (tma_a ? L::A : 0u) + (mix ? L::XP : 0u);
-            for (int kb = 0; kb < nkb; ++kb) {
-                const int s = kb % kStages;
-                if (!mbar_wait_spin(&empty[s], ((kb / kStages) & 1) ^ 1, tmo)) { bad = true; break; }
-                mbar_arrive_expect_tx(&full_t[s], bytes);
-                tma_load_2d(stB(s), &wmap, &full_t[s], kb * 64, n0);
-                if (tma_a) tma_load_2d(stA(s), &amap, &full_t[s], kb * 64, m0);
-                if (mix) tma_load_2d(stXP(s), &amap, &full_t[s], kb * 64, m0 - 1);   // row -1: zeros
-            }
-        }
-    } else if (lane == 0) {
-        // ---- MMA issue: four K = 16 steps per stage, then the stage goes back to its producers
-        for (int kb = 0; kb < nkb; ++kb) {
-            const int s = kb % kStages;
-            const uint32_t ph = (kb / kStages) & 1;
-            if (!mbar_wait_spin(&full_t[s], ph, tmo) || (prod && !mbar_wait_spin(&full_a[s], ph, tmo))) { bad = true; break; }
-            tc_fence_after();
-            const uint64_t dA = desc_sw128(smem_u32(stA(s))), dB = desc_sw128(smem_u32(stB(s)));
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16_ss(tb, dA + uint64_t(2 * ks), dB + uint64_t(2 * ks), idesc_bf16(128, BN), (kb | ks) != 0);
-            mma_commit(&empty[s]);
-        }
-        mma_commit(acc_full);   // also after a failure: the store side waits for what was issued
     }
 
-    // ---- store: warp w reads TMEM lanes 32 (w % 4) .. + 31 (rows), columns of its half
-    if (warp < 8) {
-        const bool ok = !bar_or(1, kProdThreads, tid == 0 && !mbar_wait_spin(acc_full, 0, tmo));
-        if (!ok) bad = true;
-        tc_fence_after();
-        const int q = warp & 3, h = warp >> 2, m = m0 + 32 * q + lane;
-        constexpr int HALF = BN / 2;
-#pragma unroll 1
-        for (int c0 = 0; c0 < HALF && ok; c0 += 32) {
-            float z[32];
-            tmem_ld32(tmem_addr(tb, 32 * q, h * HALF + c0), z);
-            const int n = n0 + h * HALF + c0;
-            if (m < a.M) {
-                if (a.epi == GEMM_F32) {
-                    float *d = static_cast<float *>(a.D) + size_t(m) * a.ldd + n;
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4 *>(d + e) = make_float4(z[e], z[e + 1], z[e + 2], z[e + 3]);
-                } else {
-                    __nv_bfloat16 *d = static_cast<__nv_bfloat16 *>(a.D) + size_t(m) * a.ldd + n;
-#pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        float o[8];
-                        uint4 vv = make_uint4(0u, 0u, 0u, 0u), v0 = make_uint4(0u, 0u, 0u, 0u);
-                        if (a.epi == GEMM_RESIDUAL) {
-                            vv = *reinterpret_cast<const uint4 *>(d + e);
-                            v0 = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.v0) +
-                                                                       size_t(m) * a.ldd + n + e));
-                        }
-                        const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w}, v0w[4] = {v0.x, v0.y, v0.z, v0.w};
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            o[j] = apply_epi(a.epi, z[e + j], a.bias ? __ldg(a.bias + n + e + j) : 0.f, bf(vw[j >> 1], j & 1),
-                                             bf(v0w[j >> 1], j & 1));
-                        const uint4 w = make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]),
-                                                   pack_bf16(o[6], o[7]));
-                        *reinterpret_cast<uint4 *>(d + e) = w;
-                        if (a.D2)
-                            *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.D2) + size_t(m) * a.ldd + n + e) = w;
-                    }
-                }
-            }
-        }
-    }
-    if (bad && a.err) atomicOr(a.err, 1u);
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) tmem_dealloc(tb, BN);
+    if (tid == 0 && *abort && d.err) atomicOr(d.err, 1u);
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tb, 2 * kAccCols);
+    }
 }
 
 // ---- fp32 on the FMA pipe ---------------------------------------------------------------------------
 constexpr int kFT = 64, kFK = 16;   // 64 x 64 output tile, K in steps of 16; 256 threads, 4 x 4 each
 
-__device__ __forceinline__ float prep_a1(const GemmArgs &a, int m, int k) {
-    if (m >= a.M || k >= a.K) return 0.f;
-    if (a.pro == GEMM_PLAIN) return static_cast<const float *>(a.A)[size_t(m) * a.lda + k];
-    if (a.pro == GEMM_MIX) {
-        const float *x = static_cast<const float *>(a.x);
-        const float xi = x[size_t(m) * a.K + k];
-        float xp = 0.f;
-        if (m % a.T != 0) xp = x[size_t(m - 1) * a.K + k];
-        else if (a.last_x) xp = static_cast<const float *>(a.last_x)[size_t(m / a.T) * a.K + k];
-        return fmaf(a.mix[k], xp - xi, xi);
-    }
-    return a.y[size_t(m) * a.K + k] * static_cast<const float *>(a.g)[size_t(m) * a.K + k];
+struct F32Args {
+    int M, T, pro;
+    const float *x, *last_x;
+    GemmProblem p;
+};
+
+__device__ __forceinline__ float prep_a1(const F32Args &a, int m, int k) {
+    const int K = a.p.K;
+    if (m >= a.M || k >= K) return 0.f;
+    if (a.pro == GEMM_PLAIN) return static_cast<const float *>(a.p.A)[size_t(m) * a.p.lda + k];
+    const float xi = a.x[size_t(m) * K + k];
+    float xp = 0.f;
+    if (m % a.T != 0) xp = a.x[size_t(m - 1) * K + k];
+    else if (a.last_x) xp = a.last_x[size_t(m / a.T) * K + k];
+    return fmaf(a.p.mix[k], xp - xi, xi);
 }
 
-__global__ void __launch_bounds__(256) gemm_f32_kernel(const GemmArgs a) {
+__global__ void __launch_bounds__(256) gemm_f32_kernel(const F32Args a) {
     __shared__ float As[kFK][kFT + 4], Bs[kFK][kFT + 4];
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     const int m0 = blockIdx.x * kFT, n0 = blockIdx.y * kFT;
-    const float *W = static_cast<const float *>(a.W);
+    const GemmProblem &p = a.p;
+    const float *W = static_cast<const float *>(p.W);
     float acc[4][4] = {};
-    for (int k0 = 0; k0 < a.K; k0 += kFK) {
+    for (int k0 = 0; k0 < p.K; k0 += kFK) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int e = tid + 256 * i, r = e >> 4, k = e & 15;
             As[k][r] = prep_a1(a, m0 + r, k0 + k);
             const int n = n0 + r;
-            Bs[k][r] = (n < a.N && k0 + k < a.K) ? W[size_t(n) * a.K + k0 + k] : 0.f;
+            Bs[k][r] = (n < p.N && k0 + k < p.K) ? W[size_t(n) * p.K + k0 + k] : 0.f;
         }
         __syncthreads();
 #pragma unroll
@@ -303,25 +549,41 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const GemmArgs a) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int n = n0 + tx * 4 + j;
-            if (n >= a.N) continue;
-            float *d = static_cast<float *>(a.D) + size_t(m) * a.ldd + n;
-            const float v = a.epi == GEMM_RESIDUAL ? *d : 0.f;
-            const float v0 = a.epi == GEMM_RESIDUAL ? static_cast<const float *>(a.v0)[size_t(m) * a.ldd + n] : 0.f;
-            const float o = apply_epi(a.epi, acc[i][j], a.bias ? a.bias[n] : 0.f, v, v0);
-            *d = o;
-            if (a.D2) static_cast<float *>(a.D2)[size_t(m) * a.ldd + n] = o;
+            if (n >= p.N) continue;
+            float *dp = static_cast<float *>(p.D) + size_t(m) * p.ldd + n;
+            const float z = acc[i][j], bias = p.bias ? p.bias[n] : 0.f;
+            float o = z;
+            switch (p.epi) {
+                case GEMM_TANH: o = tanhf(z); break;
+                case GEMM_SIGMOID: o = sigmoidf_(z); break;
+                case GEMM_BIAS: o = z + bias; break;
+                case GEMM_RESIDUAL: {
+                    const float v = *dp, v0 = static_cast<const float *>(p.v0)[size_t(m) * p.ldd + n];
+                    o = fmaf(v0 - v, sigmoidf_(z + bias), v);
+                    break;
+                }
+                default: break;
+            }
+            *dp = o;
         }
     }
 }
 
 // ---- transposed, zero-padded copies of the low-rank factors ------------------------------------------
+struct PadCopies {
+    PadCopy c[kMaxPadCopies];
+};
+
 template <class T>
-__global__ void transpose_pad_kernel(const T *in, T *out, int rows, int cols, int out_rows, int out_cols) {
-    // in [rows][cols] -> out [out_rows][out_cols], out[i][j] = in[j][i] inside, 0 in the padding
-    const size_t n = size_t(out_rows) * out_cols;
+__global__ void transpose_pad_kernel(const PadCopies cs) {
+    // blockIdx.y selects the copy: out[i][j] = in[j][i] inside, 0 in the padding
+    const PadCopy &c = cs.c[blockIdx.y];
+    const T *in = static_cast<const T *>(c.in);
+    T *out = static_cast<T *>(c.out);
+    const size_t n = size_t(c.out_rows) * c.out_cols;
     for (size_t e = blockIdx.x * size_t(blockDim.x) + threadIdx.x; e < n; e += size_t(gridDim.x) * blockDim.x) {
-        const int i = int(e / out_cols), j = int(e % out_cols);
-        out[e] = (i < cols && j < rows) ? in[size_t(j) * cols + i] : T(0.f);
+        const int i = int(e / c.out_cols), j = int(e % c.out_cols);
+        out[e] = (i < c.cols && j < c.rows) ? in[size_t(j) * c.cols + i] : T(0.f);
     }
 }
 
@@ -339,29 +601,75 @@ PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
     return fn;
 }
 
-bool encode_bf16_2d(CUtensorMap *map, const void *base, int cols, int rows, int ld, int box_rows) {
+// A [rows][cols] matrix (bf16, or fp32 when f32) with row stride ld elements, moved in boxes of
+// box_cols x box_rows.
+bool encode_2d(CUtensorMap *map, bool f32, const void *base, int cols, int rows, int ld, int box_cols, int box_rows,
+               CUtensorMapSwizzle swz) {
     auto enc = tmap_encoder();
     if (!enc) return false;
     const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
-    const cuuint64_t strides[1] = {cuuint64_t(ld) * 2};
-    const cuuint32_t box[2] = {64, cuuint32_t(box_rows)}, es[2] = {1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    const cuuint64_t strides[1] = {cuuint64_t(ld) * (f32 ? 4 : 2)};
+    const cuuint32_t box[2] = {cuuint32_t(box_cols), cuuint32_t(box_rows)}, es[2] = {1, 1};
+    return enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base),
+               dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+// Operand tiles: 64 bf16 columns (128 bytes, the 128-byte swizzle) x box_rows rows.
+bool encode_operand(CUtensorMap *map, const void *base, int cols, int rows, int ld, int box_rows) {
+    return encode_2d(map, false, base, cols, rows, ld, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+// Store-side tiles: 32 x 32, bf16 rows of 64 bytes (64-byte swizzle) or fp32 rows of 128 bytes
+// (128-byte swizzle), the layouts the store warps write.
+bool encode_out(CUtensorMap *map, bool f32, const void *base, int cols, int rows, int ld) {
+    return encode_2d(map, f32, base, cols, rows, ld, 32, 32, f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+}
 
-template <int BN>
-cudaError_t launch_bf16(const GemmArgs &a, cudaStream_t stream) {
-    CUtensorMap wmap, amap;
-    std::memset(&amap, 0, sizeof(amap));
-    if (!encode_bf16_2d(&wmap, a.W, a.K, a.N, a.K, BN)) return cudaErrorInvalidValue;
-    if (a.pro == GEMM_PLAIN && !encode_bf16_2d(&amap, a.A, a.K, a.M, a.lda, 128)) return cudaErrorInvalidValue;
-    if (a.pro == GEMM_MIX && !encode_bf16_2d(&amap, a.x, a.K, a.M, a.K, 128)) return cudaErrorInvalidValue;
-    const int smem = int(GemmSmem<BN>::bytes);
-    cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void *>(gemm_bf16_kernel<BN>), smem);
+int tile_cols(int N) { return N % 256 == 0 ? 256 : N % 128 == 0 ? 128 : 64; }
+
+template <int PRO>
+cudaError_t launch_bf16(const GemmGroup &g, cudaStream_t stream) {
+    GemmParams P;
+    std::memset(&P, 0, sizeof(P));
+    GemmDev &d = P.d;
+    d.M = g.M; d.T = g.T; d.nprob = g.nprob;
+    d.x = g.x; d.last_x = g.last_x; d.err = g.err;
+    int ntn = 0;
+    const void *v0 = nullptr;
+    for (int i = 0; i < g.nprob; ++i) {
+        const GemmProblem &q = g.p[i];
+        if (q.K <= 0 || q.N <= 0 || q.K % 64 != 0 || q.N % 64 != 0) return cudaErrorInvalidValue;
+        GemmProb &p = d.p[i];
+        p.N = q.N; p.K = q.K; p.bn = tile_cols(q.N); p.tile0 = ntn;
+        p.epi = q.epi; p.ldd = q.ldd; p.Kx = q.K;
+        p.mix = q.mix; p.bias = q.bias; p.v0 = q.v0; p.D = q.D;
+        ntn += q.N / p.bn;
+        if (!encode_operand(&P.wmap[i], q.W, q.K, q.N, q.K, p.bn)) return cudaErrorInvalidValue;
+        if (PRO == GEMM_PLAIN && !encode_operand(&P.amap[i], q.A, q.K, g.M, q.lda, 128)) return cudaErrorInvalidValue;
+        if (!encode_out(&P.dmap[i], q.epi == GEMM_F32, q.D, q.N, g.M, q.ldd)) return cudaErrorInvalidValue;
+        if (q.epi == GEMM_RESIDUAL) {
+            // the value residual: PLAIN launches only (the others have no room for its tiles), one v0
+            if (PRO != GEMM_PLAIN || !q.v0 || (v0 && v0 != q.v0)) return cudaErrorInvalidValue;
+            v0 = q.v0;
+            if (!encode_out(&P.v0map, false, q.v0, q.N, g.M, q.ldd)) return cudaErrorInvalidValue;
+        }
+    }
+    if (PRO == GEMM_MIX) {
+        for (int i = 1; i < g.nprob; ++i)
+            if (g.p[i].K != g.p[0].K) return cudaErrorInvalidValue;   // every mix reads the same x
+        if (!encode_operand(&P.amap[0], g.x, g.p[0].K, g.M, g.p[0].K, 128)) return cudaErrorInvalidValue;
+    }
+    d.ntn = ntn;
+    const long long ntiles = (long long)((g.M + 127) / 128) * ntn;
+    if (ntiles > INT32_MAX) return cudaErrorInvalidValue;
+    d.ntiles = int(ntiles);
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    const dim3 grid(unsigned((a.M + 127) / 128), unsigned(a.N / BN));
-    gemm_bf16_kernel<BN><<<grid, kGemmThreads, smem, stream>>>(wmap, amap, a);
+    const int smem = int(Ring<PRO>::bytes);
+    if ((e = allow_dynamic_smem(reinterpret_cast<const void *>(gemm_bf16_kernel<PRO>), smem)) != cudaSuccess) return e;
+    const unsigned grid = unsigned(std::min<long long>(ntiles, sms));
+    gemm_bf16_kernel<PRO><<<grid, kGemmThreads, smem, stream>>>(P);
     return cudaGetLastError();
 }
 
@@ -369,29 +677,43 @@ cudaError_t launch_bf16(const GemmArgs &a, cudaStream_t stream) {
 
 // ---- host side ---------------------------------------------------------------------------------------
 
-cudaError_t launch_gemm(const GemmArgs &a, wkv7_dtype dt, cudaStream_t stream) {
-    if (a.M <= 0 || a.N <= 0 || a.K <= 0) return cudaSuccess;
+cudaError_t launch_gemm_group(const GemmGroup &g, wkv7_dtype dt, cudaStream_t stream) {
+    if (g.nprob < 1 || g.nprob > kGemmMaxProblems) return cudaErrorInvalidValue;
+    if (g.M <= 0) return cudaSuccess;
+    if (g.pro == GEMM_MIX && g.T <= 0) return cudaErrorInvalidValue;
     if (dt == WKV7_F32) {
-        const dim3 grid(unsigned((a.M + kFT - 1) / kFT), unsigned((a.N + kFT - 1) / kFT));
-        gemm_f32_kernel<<<grid, 256, 0, stream>>>(a);
-        return cudaGetLastError();
+        for (int i = 0; i < g.nprob; ++i) {
+            F32Args a{};
+            a.M = g.M; a.T = g.T; a.pro = g.pro;
+            a.x = static_cast<const float *>(g.x); a.last_x = static_cast<const float *>(g.last_x);
+            a.p = g.p[i];
+            if (a.p.N <= 0 || a.p.K <= 0) return cudaErrorInvalidValue;
+            const dim3 grid(unsigned((g.M + kFT - 1) / kFT), unsigned((a.p.N + kFT - 1) / kFT));
+            gemm_f32_kernel<<<grid, 256, 0, stream>>>(a);
+            const cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
     }
-    if (a.K % 64 != 0 || a.N % 64 != 0) return cudaErrorInvalidValue;
-    if (a.N % 128 == 0) return launch_bf16<128>(a, stream);
-    return launch_bf16<64>(a, stream);
+    switch (g.pro) {
+        case GEMM_PLAIN: return launch_bf16<GEMM_PLAIN>(g, stream);
+        case GEMM_MIX: return launch_bf16<GEMM_MIX>(g, stream);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
-cudaError_t launch_transpose_pad(const void *in, void *out, int rows, int cols, int out_rows, int out_cols,
-                                 wkv7_dtype dt, cudaStream_t stream) {
-    const size_t n = size_t(out_rows) * out_cols;
-    const unsigned grid = unsigned(std::min<size_t>((n + 255) / 256, 148 * 8));
-    if (dt == WKV7_BF16)
-        transpose_pad_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(in),
-                                                                     static_cast<__nv_bfloat16 *>(out), rows, cols,
-                                                                     out_rows, out_cols);
-    else
-        transpose_pad_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float *>(in), static_cast<float *>(out),
-                                                             rows, cols, out_rows, out_cols);
+cudaError_t launch_transpose_pad(const PadCopy *copies, int n, wkv7_dtype dt, cudaStream_t stream) {
+    if (n <= 0) return cudaSuccess;
+    if (n > kMaxPadCopies) return cudaErrorInvalidValue;
+    PadCopies cs{};
+    size_t most = 0;
+    for (int i = 0; i < n; ++i) {
+        cs.c[i] = copies[i];
+        most = std::max(most, size_t(copies[i].out_rows) * copies[i].out_cols);
+    }
+    const dim3 grid(unsigned(std::min<size_t>((most + 255) / 256, 148 * 4)), unsigned(n));
+    if (dt == WKV7_BF16) transpose_pad_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(cs);
+    else transpose_pad_kernel<float><<<grid, 256, 0, stream>>>(cs);
     return cudaGetLastError();
 }
 
