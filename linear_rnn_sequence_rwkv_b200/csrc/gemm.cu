@@ -4,10 +4,10 @@
 // time_mixing listing: the token-shift mixes feed the square projections and the low-rank first
 // factors; tanh, sigmoid, the biases and the value residual follow them).
 //
-// Operand preparation (per element, in fp32, then rounded to the layer dtype):
+// Operand preparation:
 //   PLAIN  A_i itself;
 //   MIX    x + m_i (x_prev - x), x_prev the previous token of the same sequence (last_x, or 0,
-//          for the first token).
+//          for the first token), in fp32 and rounded once to the layer dtype.
 // Store (per element of the fp32 accumulator z, column n of problem i):
 //   STORE z;  TANH tanh(z);  SIGMOID sigmoid(z);  BIAS z + bias[n];
 //   RESIDUAL v + (v0 - v) sigmoid(z + bias[n]) with v the value already in D;  F32 z in fp32.
@@ -70,8 +70,9 @@ constexpr uint64_t kWaitNs = 2000000000ull;
 
 // One stage: the W tile, the A tile as loaded (x for the mix), and for MIX the prepared operand
 // (OP: where the products read A).
-// After the ring: per store warp two 4 KB output staging tiles, and for PLAIN two pairs of 2 KB
-// tiles for the value residual's v and v0.
+// After the ring: per store warp two 4 KB output staging tiles; for PLAIN two pairs of 2 KB tiles
+// for the value residual's v and v0, for MIX per stage the mix values of its 64 columns (256
+// bytes) and the x row before the tile (128 bytes), loaded with the stage.
 template <int PRO>
 struct Ring {
     static constexpr uint32_t B = 0, A = kTileB, P = kTileB + kTileA, OP = PRO == GEMM_MIX ? P : A;
@@ -79,7 +80,8 @@ struct Ring {
     static constexpr int stages = 3;
     static constexpr uint32_t out_off = stages * stage;             // [warp][2] x 4096
     static constexpr uint32_t res_off = out_off + 4 * 2 * 4096;     // PLAIN: [warp][2] x (v 2048, v0 2048)
-    static constexpr uint32_t bar_off = res_off + (PRO == GEMM_PLAIN ? 4 * 2 * 4096 : 0u);
+    static constexpr uint32_t mix_off = res_off;                     // MIX: [stage] x 384
+    static constexpr uint32_t bar_off = res_off + (PRO == GEMM_PLAIN ? 4 * 2 * 4096u : stages * 384u);
     static constexpr uint32_t bytes = bar_off + 256 + 1024;   // + barriers, + 1 KB alignment slack
 };
 
@@ -155,25 +157,22 @@ __device__ __forceinline__ bool warp_wait_phase(uint64_t *bar, uint32_t parity, 
 // 64-byte swizzle; fp32: 128-byte rows, chunk c at c ^ (row & 7), the 128-byte swizzle), and one
 // lane hands the tile to a TMA store. The value residual's v (the current D) and v0 arrive the
 // same way, by TMA loads into the same 64-byte-swizzled layout, one chunk ahead.
-struct StoreCtx {
-    uint8_t *out;               // two 4 KB staging tiles
-    uint8_t *res;               // two (v, v0) pairs of 2 KB tiles (PLAIN)
-    uint64_t *vbar;             // two barriers, one per pair
-    uint32_t vuse[2];           // completed phases of each barrier
-    volatile int *abort;        // raised when a wait gives up
-};
-
+// out: the warp's two 4 KB staging tiles; res: its two (v, v0) pairs of 2 KB tiles (PLAIN) with
+// one barrier each in vbar; vpar: bit b = parity of the next phase of vbar[b]. Everything is
+// passed by value (a context struct passed by reference would live in local memory and cost a
+// round trip to the cache for every field read). Returns the updated vpar.
 template <int EPI>
-__device__ __noinline__ void store_tile(const GemmProb p, const CUtensorMap *dmap, const CUtensorMap *v0map,
-                                        uint32_t tacc, int m0, int n0, StoreCtx &cx, int lane) {
+__device__ __noinline__ uint32_t store_tile(const GemmProb p, const CUtensorMap *dmap, const CUtensorMap *v0map,
+                                            uint32_t tacc, int m0, int n0, uint8_t *const out, uint8_t *const res,
+                                            uint64_t *const vbar, uint32_t vpar, volatile int *abort, int lane) {
     const int nch = p.bn / 32;
     const float *const bias_p = p.bias;
     auto fetch_res = [&](int j) {   // v and v0 of chunk j into pair j & 1
         if (lane == 0) {
-            uint8_t *r = cx.res + (j & 1) * 4096;
-            mbar_arrive_expect_tx(&cx.vbar[j & 1], 4096);
-            tma_load_2d(r, dmap, &cx.vbar[j & 1], n0 + 32 * j, m0);
-            tma_load_2d(r + 2048, v0map, &cx.vbar[j & 1], n0 + 32 * j, m0);
+            uint8_t *r = res + (j & 1) * 4096;
+            mbar_arrive_expect_tx(&vbar[j & 1], 4096);
+            tma_load_2d(r, dmap, &vbar[j & 1], n0 + 32 * j, m0);
+            tma_load_2d(r + 2048, v0map, &vbar[j & 1], n0 + 32 * j, m0);
         }
     };
     if constexpr (EPI == GEMM_RESIDUAL) fetch_res(0);
@@ -200,10 +199,10 @@ __device__ __noinline__ void store_tile(const GemmProb p, const CUtensorMap *dma
         } else if constexpr (EPI == GEMM_RESIDUAL) {
             const int b = j & 1;
             int ok = 1;
-            if (lane == 0) ok = wait_phase(&cx.vbar[b], cx.vuse[b] & 1, cx.abort);   // polled: wakes on time
+            if (lane == 0) ok = wait_phase(&vbar[b], vpar >> b & 1u, abort);   // polled: wakes on time
             ok = __shfl_sync(0xffffffffu, ok, 0);
-            ++cx.vuse[b];
-            const uint32_t rv = smem_u32(cx.res + b * 4096) + uint32_t(lane * 64);
+            vpar ^= 1u << b;
+            const uint32_t rv = smem_u32(res + b * 4096) + uint32_t(lane * 64);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const uint32_t off = uint32_t((c ^ ((lane >> 1) & 3)) << 4);
@@ -220,7 +219,7 @@ __device__ __noinline__ void store_tile(const GemmProb p, const CUtensorMap *dma
             }
         }
         // staging tile j & 1: its store from chunk j - 2 has finished reading it
-        uint8_t *o = cx.out + (j & 1) * 4096;
+        uint8_t *o = out + (j & 1) * 4096;
         if (lane == 0) tma_store_wait_read1();
         __syncwarp();
         if constexpr (EPI == GEMM_F32) {
@@ -246,59 +245,52 @@ __device__ __noinline__ void store_tile(const GemmProb p, const CUtensorMap *dma
             tma_store_commit();
         }
     }
+    return vpar;
 }
 
-// MIX: the thread's four chunks (rows rb + 32 i, 16-byte chunk q) of the prepared operand, from
-// the loaded x tile (the row before comes from the same tile, except for tile row 0 and the
-// first token of a sequence: those come from global memory, loaded by mix_fetch before the
-// stage's wait).
-struct MixFetch {
-    float mv[8];
-    uint4 xp[4];
-};
+// MIX: the thread's four chunks (rows rb + 32 i, 16-byte chunk q) of the prepared operand,
+// x + m (x_prev - x) in fp32, rounded once to bf16. The row before comes from the loaded x tile,
+// for tile row 0 from the stage's copy of the row before the tile, and for the first token of a
+// sequence from last_x (or zeros), read from global memory (rare unless sequences are short).
 // The operand sources, copied out of the kernel parameters into registers once (reads through a
 // reference to the parameters would be repeated after every shared-memory store).
 struct Src {
-    const __nv_bfloat16 *x, *last_x;
-    const float *mix;
+    const __nv_bfloat16 *last_x;
     int M, T, K;
 };
-__device__ __forceinline__ void mix_fetch(MixFetch &f, const Src &d, int m0, int kb, int rb, int q,
-                                          uint32_t first_mask) {
-    const int k = kb * 64 + q * 8;
-    const float4 mA = __ldg(reinterpret_cast<const float4 *>(d.mix + k));
-    const float4 mB = __ldg(reinterpret_cast<const float4 *>(d.mix + k + 4));
-    f.mv[0] = mA.x; f.mv[1] = mA.y; f.mv[2] = mA.z; f.mv[3] = mA.w;
-    f.mv[4] = mB.x; f.mv[5] = mB.y; f.mv[6] = mB.z; f.mv[7] = mB.w;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int r = rb + 32 * i, m = m0 + r;
-        f.xp[i] = make_uint4(0u, 0u, 0u, 0u);
-        if (first_mask >> i & 1u) {   // the row starts a sequence: last_x of its sequence, or zeros
-            if (d.last_x) f.xp[i] = __ldg(reinterpret_cast<const uint4 *>(d.last_x + size_t(m / d.T) * d.K + k));
-        } else if (r == 0 && m < d.M) {
-            f.xp[i] = __ldg(reinterpret_cast<const uint4 *>(d.x + size_t(m - 1) * d.K + k));
-        }
-    }
-}
-__device__ __forceinline__ void mix_stage(const MixFetch &f, const uint8_t *xt, uint8_t *pt, int rb, int q,
-                                          uint32_t first_mask) {
+__device__ __forceinline__ void mix_stage(const Src &d, const uint8_t *xt, const uint8_t *extra, uint8_t *pt, int m0,
+                                          int k, int rb, int q, uint32_t first_mask) {
+    // extra: the stage's 64 mix values (256 bytes), then the row before the tile (128 bytes)
+    const float4 mA = *reinterpret_cast<const float4 *>(extra + q * 32), mB = *reinterpret_cast<const float4 *>(extra + q * 32 + 16);
+    const float mv[8] = {mA.x, mA.y, mA.z, mA.w, mB.x, mB.y, mB.z, mB.w};
+    uint4 xc[4], xp[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int r = rb + 32 * i;
-        const uint32_t off = uint32_t(r) * 128u + (uint32_t(q ^ (r & 7)) << 4);
-        const uint4 xp = ((first_mask >> i & 1u) || r == 0)
-                             ? f.xp[i]
-                             : *reinterpret_cast<const uint4 *>(xt + uint32_t(r - 1) * 128u + (uint32_t(q ^ ((r - 1) & 7)) << 4));
-        const uint4 xc = *reinterpret_cast<const uint4 *>(xt + off);
-        const uint32_t xcw[4] = {xc.x, xc.y, xc.z, xc.w}, xpw[4] = {xp.x, xp.y, xp.z, xp.w};
+        xc[i] = *reinterpret_cast<const uint4 *>(xt + uint32_t(r) * 128u + (uint32_t(q ^ (r & 7)) << 4));
+        xp[i] = r > 0 ? *reinterpret_cast<const uint4 *>(xt + uint32_t(r - 1) * 128u + (uint32_t(q ^ ((r - 1) & 7)) << 4))
+                      : *reinterpret_cast<const uint4 *>(extra + 256 + q * 16);
+    }
+    if (first_mask) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (first_mask >> i & 1u) {
+                const int m = m0 + rb + 32 * i;
+                xp[i] = d.last_x ? __ldg(reinterpret_cast<const uint4 *>(d.last_x + size_t(m / d.T) * d.K + k))
+                                 : make_uint4(0u, 0u, 0u, 0u);
+            }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = rb + 32 * i;
+        const uint32_t cw[4] = {xc[i].x, xc[i].y, xc[i].z, xc[i].w}, pw[4] = {xp[i].x, xp[i].y, xp[i].z, xp[i].w};
         float o[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            const float xi = bf(xcw[e >> 1], e & 1), pi = bf(xpw[e >> 1], e & 1);
-            o[e] = fmaf(f.mv[e], pi - xi, xi);
+            const float xi = bf(cw[e >> 1], e & 1), pi = bf(pw[e >> 1], e & 1);
+            o[e] = fmaf(mv[e], pi - xi, xi);
         }
-        *reinterpret_cast<uint4 *>(pt + off) =
+        *reinterpret_cast<uint4 *>(pt + uint32_t(r) * 128u + (uint32_t(q ^ (r & 7)) << 4)) =
             make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
     }
 }
@@ -351,7 +343,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_kernel(const __grid
             for (int t = blockIdx.x; t < d.ntiles && !*abort; t += gridDim.x) {
                 const Tile tl = tile_of(d, t);
                 const GemmProb &p = d.p[tl.pi];
-                const uint32_t bytes = uint32_t(p.bn) * 128u + kTileA;
+                // MIX: the mix values, and the row before the tile unless the tile starts at row 0
+                const uint32_t bytes = uint32_t(p.bn) * 128u + kTileA + (PRO == GEMM_MIX ? (tl.m0 > 0 ? 384u : 256u) : 0u);
                 const CUtensorMap *am = &P.amap[PRO == GEMM_PLAIN ? tl.pi : 0];
                 for (int kb = 0; kb < p.K / 64; ++kb, ++it) {
                     const int s = it % R::stages;
@@ -359,6 +352,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_kernel(const __grid
                     mbar_arrive_expect_tx(&full_t[s], bytes);
                     tma_load_2d(stage(s) + R::B, &P.wmap[tl.pi], &full_t[s], kb * 64, tl.n0);
                     tma_load_2d(stage(s) + R::A, am, &full_t[s], kb * 64, tl.m0);
+                    if (PRO == GEMM_MIX) {
+                        uint8_t *ex = sm + R::mix_off + s * 384;
+                        bulk_load_1d(ex, p.mix + kb * 64, 256u, &full_t[s]);
+                        if (tl.m0 > 0)
+                            bulk_load_1d(ex + 256, static_cast<const __nv_bfloat16 *>(d.x) + size_t(tl.m0 - 1) * p.Kx + kb * 64,
+                                         128u, &full_t[s]);
+                    }
                 }
             }
             // the loads still in flight land before the CTA leaves
@@ -400,7 +400,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_kernel(const __grid
         }
     } else if (warp >= kEpiWarp0) {
         const int quarter = warp & 3, ew = warp - kEpiWarp0;
-        StoreCtx cx{sm + R::out_off + ew * 8192, sm + R::res_off + ew * 8192, vbars + 2 * ew, {0u, 0u}, abort};
+        uint8_t *const out = sm + R::out_off + ew * 8192, *const res = sm + R::res_off + ew * 8192;
+        uint64_t *const vbar = vbars + 2 * ew;
+        uint32_t vpar = 0;
         if (lane == 0) {
             for (int i = 0; i < d.nprob; ++i) prefetch_tensormap(&P.dmap[i]);
         }
@@ -415,14 +417,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_kernel(const __grid
             const int m0 = tl.m0 + 32 * quarter;
             const CUtensorMap *dm = &P.dmap[tl.pi];
             switch (p.epi) {
-                case GEMM_TANH: store_tile<GEMM_TANH>(p, dm, &P.v0map, tacc, m0, tl.n0, cx, lane); break;
-                case GEMM_SIGMOID: store_tile<GEMM_SIGMOID>(p, dm, &P.v0map, tacc, m0, tl.n0, cx, lane); break;
-                case GEMM_BIAS: store_tile<GEMM_BIAS>(p, dm, &P.v0map, tacc, m0, tl.n0, cx, lane); break;
+                case GEMM_TANH: vpar = store_tile<GEMM_TANH>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, vpar, abort, lane); break;
+                case GEMM_SIGMOID: vpar = store_tile<GEMM_SIGMOID>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, vpar, abort, lane); break;
+                case GEMM_BIAS: vpar = store_tile<GEMM_BIAS>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, vpar, abort, lane); break;
                 case GEMM_RESIDUAL:
-                    if (PRO == GEMM_PLAIN) store_tile<GEMM_RESIDUAL>(p, dm, &P.v0map, tacc, m0, tl.n0, cx, lane);
+                    if (PRO == GEMM_PLAIN) vpar = store_tile<GEMM_RESIDUAL>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, vpar, abort, lane);
                     break;
-                case GEMM_F32: store_tile<GEMM_F32>(p, dm, &P.v0map, tacc, m0, tl.n0, cx, lane); break;
-                default: store_tile<GEMM_STORE>(p, dm, &P.v0map, tacc, m0, tl.n0, cx, lane); break;
+                case GEMM_F32: vpar = store_tile<GEMM_F32>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, vpar, abort, lane); break;
+                default: vpar = store_tile<GEMM_STORE>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, vpar, abort, lane); break;
             }
             tc_fence_before();
             __syncwarp();
@@ -430,55 +432,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_kernel(const __grid
         }
         if (lane == 0) tma_store_wait_all();   // the stores have landed before the CTA leaves
     } else if (PRO == GEMM_MIX) {
-        // operand preparation: the thread owns chunk q of rows rb, rb + 32, rb + 64, rb + 96. The
-        // global operands of a stage (its mix values, and the rows before the tile or a sequence)
-        // are fetched one stage ahead, so that their latency overlaps the previous stage's work.
+        // operand preparation: the thread owns chunk q of rows rb, rb + 32, rb + 64, rb + 96
         const int q = tid & 7, rb = tid >> 3;
-        const int ntiles = d.ntiles;
-        Src src{static_cast<const __nv_bfloat16 *>(d.x), static_cast<const __nv_bfloat16 *>(d.last_x), nullptr, d.M,
-                d.T, 0};
-        struct Pos {
-            int t, kb, nkb, m0;
-            uint32_t first_mask;
-            const float *mix;
-            int K;
-        };
-        auto tile_pos = [&](int t) {
-            Pos ps{t, 0, 0, 0, 0u, nullptr, 0};
-            if (t < ntiles) {
-                const Tile tl = tile_of(d, t);
-                ps.nkb = d.p[tl.pi].K / 64;
-                ps.m0 = tl.m0;
-                ps.mix = d.p[tl.pi].mix;
-                ps.K = d.p[tl.pi].Kx;
+        const Src src{static_cast<const __nv_bfloat16 *>(d.last_x), d.M, d.T, 0};
+        int it = 0;
+        for (int t = blockIdx.x; t < d.ntiles; t += gridDim.x) {
+            const Tile tl = tile_of(d, t);
+            Src sd = src;
+            sd.K = d.p[tl.pi].Kx;
+            const int nkb = d.p[tl.pi].K / 64;
+            uint32_t first_mask = 0;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int m = tl.m0 + rb + 32 * i;
-                    if (m < src.M && m % src.T == 0) ps.first_mask |= 1u << i;
-                }
+            for (int i = 0; i < 4; ++i) {
+                const int m = tl.m0 + rb + 32 * i;
+                if (m < sd.M && m % sd.T == 0) first_mask |= 1u << i;
             }
-            return ps;
-        };
-        auto fetch = [&](MixFetch &f, const Pos &ps) {
-            src.mix = ps.mix;
-            src.K = ps.K;
-            mix_fetch(f, src, ps.m0, ps.kb, rb, q, ps.first_mask);
-        };
-        Pos cur = tile_pos(blockIdx.x);
-        MixFetch fc, fn;
-        if (cur.t < ntiles) fetch(fc, cur);
-        for (int it = 0; cur.t < ntiles; ++it) {
-            Pos nxt = cur;
-            if (++nxt.kb == cur.nkb) nxt = tile_pos(cur.t + gridDim.x);
-            if (nxt.t < ntiles) fetch(fn, nxt);
-            const int s = it % R::stages;
-            if (!warp_wait_phase(&full_t[s], (it / R::stages) & 1, abort, lane)) break;
-            mix_stage(fc, stage(s) + R::A, stage(s) + R::OP, rb, q, cur.first_mask);
-            fence_proxy_async_smem();   // generic-proxy writes -> visible to the tensor core
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&full_a[s]);
-            cur = nxt;
-            fc = fn;
+            bool ok = true;
+            for (int kb = 0; kb < nkb; ++kb, ++it) {
+                const int s = it % R::stages;
+                if (!warp_wait_phase(&full_t[s], (it / R::stages) & 1, abort, lane)) {
+                    ok = false;
+                    break;
+                }
+                mix_stage(sd, stage(s) + R::A, sm + R::mix_off + s * 384, stage(s) + R::OP, tl.m0, kb * 64 + q * 8, rb, q,
+                          first_mask);
+                fence_proxy_async_smem();   // generic-proxy writes -> visible to the tensor core
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full_a[s]);
+            }
+            if (!ok) break;
         }
     }
 
@@ -656,6 +638,8 @@ cudaError_t launch_bf16(const GemmGroup &g, cudaStream_t stream) {
     if (PRO == GEMM_MIX) {
         for (int i = 1; i < g.nprob; ++i)
             if (g.p[i].K != g.p[0].K) return cudaErrorInvalidValue;   // every mix reads the same x
+        for (int i = 0; i < g.nprob; ++i)   // the mix values are copied in 256-byte pieces
+            if (!g.p[i].mix || reinterpret_cast<uintptr_t>(g.p[i].mix) % 16 != 0) return cudaErrorInvalidValue;
         if (!encode_operand(&P.amap[0], g.x, g.p[0].K, g.M, g.p[0].K, 128)) return cudaErrorInvalidValue;
     }
     d.ntn = ntn;
