@@ -277,10 +277,12 @@ WKV7_API wkv7_status wkv7_backward_static(int B, int T, int H, int N, wkv7_dtype
  *     y = wkv7_forward_raw(r, w_logit, k, v, a_logit, k_k, k_a) with the epilogue (ln_w, ln_b, r_k)
  *     out = Wo (y * g)
  * Every projection is this library's GEMM: tcgen05 tensor cores with bf16 operands and fp32
- * accumulation for WKV7_BF16, the fp32 FMA pipe for WKV7_F32. The token-shift mixes are formed in
- * each GEMM's operand load and tanh, sigmoid, the biases and the value residual in its store;
- * r, k, v, the two logits and the low-rank hidden values are stored in dt, g and y in fp32, and the
- * gate multiplies y inside the output projection's operand load. Each call also copies the
+ * accumulation for WKV7_BF16, the fp32 FMA pipe for WKV7_F32. The seven products of the mixed x
+ * (r, k, v and the four low-rank first factors) run as one launch and the four second factors as
+ * another; the token-shift mixes are formed in the operand load (fp32 arithmetic, rounded once to
+ * dt) and tanh, sigmoid, the biases and the value residual in the store. r, k, v, the two logits
+ * and the low-rank hidden values are stored in dt, g and y in fp32; y * g is formed in one
+ * element-wise pass, rounded to dt, before the output projection. Each call also copies the
  * low-rank factors, transposed and zero-padded to multiples of 64, into the workspace.
  *
  * dims:   H, N (64, or 128 on the scan), low-rank widths d_w, d_a, d_v, d_g (>= 1).

@@ -106,6 +106,9 @@ struct GemmParams {
     GemmDev d;
 };
 
+static_assert(sizeof(GemmParams) <= 4096, "kernel parameters");
+static_assert(Ring<GEMM_MIX>::bytes <= 232448 && Ring<GEMM_PLAIN>::bytes <= 232448, "shared memory per CTA");
+
 struct Tile {
     int m0, pi, n0;
 };
