@@ -111,3 +111,20 @@ def test_layer_previous_token_in_place(cuda_device):
                                              last_x_out=last)
     assert last_out is last and torch.equal(last.cpu(), d["x"][:, -1])
     assert _out_err(out, out_ref, 4) <= TOL_LAYER["f32"]
+
+
+def test_layer_at_the_large_shape_sampled(cuda_device):
+    """B16 T4096 H32 (C 2048): the whole batch runs on the GPU; the first and the last sequence
+    are checked against the oracle run on those two sequences alone (sequences are independent)."""
+    H = 32
+    d = inputs.make_layer(16, 4096, H, seed=971, dtype="bf16")
+    rows = [0, 15]
+    pick = {k: v for k, v in d.items()}
+    for k in ("x", "last_x", "v0", "S0"):
+        pick[k] = d[k][rows]
+    out_ref, _, _, S_ref = reference.time_mixing_layer(pick["x"], pick, pick["last_x"], pick["v0"], pick["S0"])
+    dd = {k: (None if v is None else v.to(cuda_device)) for k, v in d.items()}
+    S = dd["S0"].clone()
+    out, _, _, S = wkv7.layer_forward(dd["x"], dd, H, last_x=dd["last_x"], v0=dd["v0"], S=S)
+    assert _out_err(out[rows], out_ref, H) <= TOL_LAYER["bf16"]
+    assert state_err(S[rows], S_ref) <= TOL_LAYER["bf16"]
