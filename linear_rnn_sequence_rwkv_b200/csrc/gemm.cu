@@ -70,18 +70,18 @@ constexpr uint64_t kWaitNs = 2000000000ull;
 
 // One stage: the W tile, the A tile as loaded (x for the mix), and for MIX the prepared operand
 // (OP: where the products read A).
-// After the ring: per store warp two 4 KB output staging tiles; for PLAIN two pairs of 2 KB tiles
-// for the value residual's v and v0, for MIX per stage the mix values of its 64 columns (256
-// bytes) and the x row before the tile (128 bytes), loaded with the stage.
+// After the ring: per store warp two 4 KB output staging tiles; for PLAIN three pairs of 2 KB
+// tiles for the value residual's v and v0, for MIX per stage the mix values of its 64 columns
+// (256 bytes) and the x row before the tile (128 bytes), loaded with the stage.
 template <int PRO>
 struct Ring {
     static constexpr uint32_t B = 0, A = kTileB, P = kTileB + kTileA, OP = PRO == GEMM_MIX ? P : A;
     static constexpr uint32_t stage = kTileB + kTileA + (PRO == GEMM_MIX ? kTileA : 0u);
     static constexpr int stages = 3;
     static constexpr uint32_t out_off = stages * stage;             // [warp][2] x 4096
-    static constexpr uint32_t res_off = out_off + 4 * 2 * 4096;     // PLAIN: [warp][2] x (v 2048, v0 2048)
+    static constexpr uint32_t res_off = out_off + 4 * 2 * 4096;     // PLAIN: [warp][3] x (v 2048, v0 2048)
     static constexpr uint32_t mix_off = res_off;                     // MIX: [stage] x 384
-    static constexpr uint32_t bar_off = res_off + (PRO == GEMM_PLAIN ? 4 * 2 * 4096u : stages * 384u);
+    static constexpr uint32_t bar_off = res_off + (PRO == GEMM_PLAIN ? 4 * 3 * 4096u : stages * 384u);
     static constexpr uint32_t bytes = bar_off + 256 + 1024;   // + barriers, + 1 KB alignment slack
 };
 
@@ -160,29 +160,35 @@ __device__ __forceinline__ bool warp_wait_phase(uint64_t *bar, uint32_t parity, 
 // 64-byte swizzle; fp32: 128-byte rows, chunk c at c ^ (row & 7), the 128-byte swizzle), and one
 // lane hands the tile to a TMA store. The value residual's v (the current D) and v0 arrive the
 // same way, by TMA loads into the same 64-byte-swizzled layout, one chunk ahead.
-// out: the warp's two 4 KB staging tiles; res: its two (v, v0) pairs of 2 KB tiles (PLAIN) with
-// one barrier each in vbar; vpar: bit b = parity of the next phase of vbar[b]. Everything is
-// passed by value (a context struct passed by reference would live in local memory and cost a
-// round trip to the cache for every field read). Returns the updated vpar.
+// out: the warp's two 4 KB staging tiles; res: its three (v, v0) pairs of 2 KB tiles (PLAIN), with
+// one barrier each in vbar, used in turn by the value residual's blocks (two blocks are in
+// flight while a third is read); rc: the residual blocks this warp has taken so far (block a
+// uses pair a % 3, whose barrier is then in its (a / 3)-th phase). Everything is passed by
+// value (a context struct passed by reference would live in local memory and cost a round trip
+// to the cache for every field read). Returns the updated rc.
 template <int EPI>
 __device__ __noinline__ uint32_t store_tile(const GemmProb p, const CUtensorMap *dmap, const CUtensorMap *v0map,
                                             uint32_t tacc, int m0, int n0, uint8_t *const out, uint8_t *const res,
-                                            uint64_t *const vbar, uint32_t vpar, volatile int *abort, int lane) {
+                                            uint64_t *const vbar, uint32_t rc, volatile int *abort, int lane) {
     const int nch = p.bn / 32;
     const float *const bias_p = p.bias;
-    auto fetch_res = [&](int j) {   // v and v0 of chunk j into pair j & 1
+    auto fetch_res = [&](int j) {   // v and v0 of chunk j (block rc + j) into pair (rc + j) % 3
         if (lane == 0) {
-            uint8_t *r = res + (j & 1) * 4096;
-            mbar_arrive_expect_tx(&vbar[j & 1], 4096);
-            tma_load_2d(r, dmap, &vbar[j & 1], n0 + 32 * j, m0);
-            tma_load_2d(r + 2048, v0map, &vbar[j & 1], n0 + 32 * j, m0);
+            const uint32_t sl = (rc + uint32_t(j)) % 3u;
+            uint8_t *r = res + sl * 4096;
+            mbar_arrive_expect_tx(&vbar[sl], 4096);
+            tma_load_2d(r, dmap, &vbar[sl], n0 + 32 * j, m0);
+            tma_load_2d(r + 2048, v0map, &vbar[sl], n0 + 32 * j, m0);
         }
     };
-    if constexpr (EPI == GEMM_RESIDUAL) fetch_res(0);
+    if constexpr (EPI == GEMM_RESIDUAL) {
+        fetch_res(0);
+        if (nch > 1) fetch_res(1);
+    }
 #pragma unroll 1
     for (int j = 0; j < nch; ++j) {
         if constexpr (EPI == GEMM_RESIDUAL)
-            if (j + 1 < nch) fetch_res(j + 1);   // its pair was last read in chunk j - 1
+            if (j + 2 < nch) fetch_res(j + 2);   // its pair was last read in chunk j - 1
         float z[32];
         tmem_ld32(tacc + uint32_t(32 * j), z);
         const int n = n0 + 32 * j;
@@ -200,11 +206,10 @@ __device__ __noinline__ uint32_t store_tile(const GemmProb p, const CUtensorMap 
 #pragma unroll
             for (int e = 0; e < 32; ++e) z[e] = sigmoidf_(z[e]);
         } else if constexpr (EPI == GEMM_RESIDUAL) {
-            const int b = j & 1;
+            const uint32_t a = rc + uint32_t(j), b = a % 3u;
             int ok = 1;
-            if (lane == 0) ok = wait_phase(&vbar[b], vpar >> b & 1u, abort);   // polled: wakes on time
+            if (lane == 0) ok = wait_phase(&vbar[b], (a / 3u) & 1u, abort);   // polled: wakes on time
             ok = __shfl_sync(0xffffffffu, ok, 0);
-            vpar ^= 1u << b;
             const uint32_t rv = smem_u32(res + b * 4096) + uint32_t(lane * 64);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -248,7 +253,7 @@ __device__ __noinline__ uint32_t store_tile(const GemmProb p, const CUtensorMap 
             tma_store_commit();
         }
     }
-    return vpar;
+    return EPI == GEMM_RESIDUAL ? rc + uint32_t(nch) : rc;
 }
 
 // MIX: the thread's four chunks (rows rb + 32 i, 16-byte chunk q) of the prepared operand,
@@ -305,9 +310,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_kernel(const __grid
     uint8_t *sm = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + R::bar_off);
     uint64_t *full_t = bars, *full_a = bars + 4, *empty = bars + 8, *acc_full = bars + 12, *acc_empty = bars + 14;
-    uint64_t *drain = bars + 16, *vbars = bars + 17;   // vbars: [store warp][2]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 25);
-    volatile int *abort = reinterpret_cast<volatile int *>(bars + 26);
+    uint64_t *drain = bars + 16, *vbars = bars + 17;   // vbars: [store warp][3]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 29);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 30);
     auto stage = [&](int s) { return sm + s * R::stage; };
 
     const GemmDev &d = P.d;
@@ -323,7 +328,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_kernel(const __grid
             mbar_init(&acc_empty[b], 4);         // one arrival per store warp
         }
         mbar_init(drain, 1);
-        for (int i = 0; i < 8; ++i) mbar_init(&vbars[i], 1);
+        for (int i = 0; i < 12; ++i) mbar_init(&vbars[i], 1);
         *abort = 0;
         mbar_fence_init();
     }
@@ -403,9 +408,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_kernel(const __grid
         }
     } else if (warp >= kEpiWarp0) {
         const int quarter = warp & 3, ew = warp - kEpiWarp0;
-        uint8_t *const out = sm + R::out_off + ew * 8192, *const res = sm + R::res_off + ew * 8192;
-        uint64_t *const vbar = vbars + 2 * ew;
-        uint32_t vpar = 0;
+        uint8_t *const out = sm + R::out_off + ew * 8192, *const res = sm + R::res_off + ew * 12288;
+        uint64_t *const vbar = vbars + 3 * ew;
+        uint32_t rc = 0;
         if (lane == 0) {
             for (int i = 0; i < d.nprob; ++i) prefetch_tensormap(&P.dmap[i]);
         }
@@ -420,14 +425,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_kernel(const __grid
             const int m0 = tl.m0 + 32 * quarter;
             const CUtensorMap *dm = &P.dmap[tl.pi];
             switch (p.epi) {
-                case GEMM_TANH: vpar = store_tile<GEMM_TANH>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, vpar, abort, lane); break;
-                case GEMM_SIGMOID: vpar = store_tile<GEMM_SIGMOID>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, vpar, abort, lane); break;
-                case GEMM_BIAS: vpar = store_tile<GEMM_BIAS>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, vpar, abort, lane); break;
+                case GEMM_TANH: rc = store_tile<GEMM_TANH>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, rc, abort, lane); break;
+                case GEMM_SIGMOID: rc = store_tile<GEMM_SIGMOID>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, rc, abort, lane); break;
+                case GEMM_BIAS: rc = store_tile<GEMM_BIAS>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, rc, abort, lane); break;
                 case GEMM_RESIDUAL:
-                    if (PRO == GEMM_PLAIN) vpar = store_tile<GEMM_RESIDUAL>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, vpar, abort, lane);
+                    if (PRO == GEMM_PLAIN) rc = store_tile<GEMM_RESIDUAL>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, rc, abort, lane);
                     break;
-                case GEMM_F32: vpar = store_tile<GEMM_F32>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, vpar, abort, lane); break;
-                default: vpar = store_tile<GEMM_STORE>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, vpar, abort, lane); break;
+                case GEMM_F32: rc = store_tile<GEMM_F32>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, rc, abort, lane); break;
+                default: rc = store_tile<GEMM_STORE>(p, dm, &P.v0map, tacc, m0, tl.n0, out, res, vbar, rc, abort, lane); break;
             }
             tc_fence_before();
             __syncwarp();
