@@ -138,6 +138,31 @@ def group_norm_bonus(y, r, k, v, ln_w, ln_b, r_k, eps=64e-5):
     return normed + bonus
 
 
+def group_norm_bonus_backward(y, r, k, v, ln_w, ln_b, r_k, dout, eps=64e-5):
+    """Gradients of L = <dout, group_norm_bonus(y, r, k, v, ln_w, ln_b, r_k)> in fp64: the
+    chain rule through the per-head group_norm and the bonus (the pages print the forward
+    only; same listing as ``group_norm_bonus``). With yc = y - mean(y), inv = (mean(yc^2) +
+    eps)^(-1/2), yn = yc inv and beta = sum_j r_j k_j r_k[j], per (b, t, h):
+      out = yn ln_w + ln_b + beta v
+      -> dv = beta dout, dbeta = sum_i dout_i v_i, dr = dbeta k r_k, dk = dbeta r r_k,
+         dr_k += dbeta r k, dln_w += dout yn, dln_b += dout,
+         g = dout ln_w, dy = inv (g - mean(g) - yn mean(g yn)).
+    y, r, k, v, dout: [B, T, H, N]; ln_w, ln_b, r_k: [H, N]. Returns a dict of fp64 arrays:
+    dy, dr, dk, dv [B, T, H, N] and dln_w, dln_b, dr_k [H, N] (summed over B and T).
+    """
+    y, r, k, v, ln_w, ln_b, r_k, dout = (_f64(x) for x in (y, r, k, v, ln_w, ln_b, r_k, dout))
+    yc = y - y.mean(axis=-1, keepdims=True)
+    inv = 1.0 / np.sqrt((yc ** 2).mean(axis=-1, keepdims=True) + eps)
+    yn = yc * inv
+    beta = (r * k * r_k).sum(axis=-1, keepdims=True)
+    dbeta = (dout * v).sum(axis=-1, keepdims=True)
+    g = dout * ln_w
+    dy = inv * (g - g.mean(axis=-1, keepdims=True) - yn * (g * yn).mean(axis=-1, keepdims=True))
+    return {"dy": dy, "dr": dbeta * k * r_k, "dk": dbeta * r * r_k, "dv": beta * dout,
+            "dln_w": (dout * yn).sum(axis=(0, 1)), "dln_b": dout.sum(axis=(0, 1)),
+            "dr_k": (dbeta * r * k).sum(axis=(0, 1))}
+
+
 def prepare_inputs(w_logit, a_logit, k, k_k, k_a=None):
     """The pre-processing the pages place before the update, in fp64 (the rebuttal page's
     ``time_mixing`` listing: the decay, the in-context learning rate, the removal key formed

@@ -297,3 +297,46 @@ def test_layer_with_transposed_output_projection_is_caught(monkeypatch):
 
 def test_unmutated_layer_passes_its_pins():
     assert _failures(LAYER_PINS) == 0
+
+
+# ---- epilogue backward mutants -----------------------------------------------------------
+
+from tests import test_oracle_epilogue_backward as PE  # noqa: E402
+
+
+def _epilogue_backward(kind):
+    def run(y, r, k, v, ln_w, ln_b, r_k, dout, eps=64e-5):
+        y, r, k, v, ln_w, ln_b, r_k, dout = (_f64(x) for x in (y, r, k, v, ln_w, ln_b, r_k, dout))
+        N = y.shape[-1]
+        yc = y - y.mean(axis=-1, keepdims=True)
+        var = (yc ** 2).sum(axis=-1, keepdims=True) / (N - 1 if kind == "sample_variance" else N)
+        inv = 1.0 / np.sqrt(var + eps)
+        yn = yc * inv
+        beta = (r * k * r_k).sum(axis=-1, keepdims=True)
+        dbeta = (dout * v).sum(axis=-1, keepdims=True)
+        g = dout * ln_w
+        corr = 0.0 if kind == "no_variance_term" else yn * (g * yn).mean(axis=-1, keepdims=True)
+        dy = inv * (g - (0.0 if kind == "no_mean_term" else g.mean(axis=-1, keepdims=True)) - corr)
+        dk = dbeta * (r if kind != "dk_uses_k" else k) * r_k
+        return {"dy": dy, "dr": dbeta * k * r_k, "dk": dk, "dv": beta * dout,
+                "dln_w": (dout * (yc if kind == "dln_w_unnormalised" else yn)).sum(axis=(0, 1)),
+                "dln_b": dout.sum(axis=(0, 1)), "dr_k": (dbeta * r * k).sum(axis=(0, 1))}
+    return run
+
+
+@pytest.mark.parametrize("kind", ["sample_variance", "no_variance_term", "no_mean_term", "dk_uses_k",
+                                  "dln_w_unnormalised"])
+def test_epilogue_backward_mutant_is_caught(monkeypatch, kind):
+    monkeypatch.setattr(reference, "group_norm_bonus_backward", _epilogue_backward(kind))
+    failures = 0
+    for name in ("y", "r", "k", "v", "ln_w", "ln_b", "r_k"):
+        try:
+            PE.test_matches_central_differences(name)
+        except AssertionError:
+            failures += 1
+    for pin in (PE.test_normalisation_invariants, PE.test_branches_cut_off):
+        try:
+            pin()
+        except AssertionError:
+            failures += 1
+    assert failures > 0, f"mutant {kind} passed every pin"
