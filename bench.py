@@ -475,7 +475,7 @@ def run_backward(args, world, rank, local):
         g = torch.Generator(device=dev).manual_seed(seed0 + 17 * i + 1)
         d["dy"] = torch.randn(B, T, H, N, device=dev, generator=g)
         d["dS_T"] = 0.1 * torch.randn(B, H, N, N, device=dev, generator=g)
-        _, _, d["snaps"] = wkv7.forward(*(d[n] for n in NAMES), d["S0"], snap_every=snap)
+        d["y"], _, d["snaps"] = wkv7.forward(*(d[n] for n in NAMES), d["S0"], snap_every=snap)
         sets.append(d)
     grads = {n: torch.empty(B, T, H, N, device=dev) for n in wkv7.GRAD_NAMES}
     dS0 = torch.empty(B, H, N, N, device=dev)
@@ -541,6 +541,7 @@ def run_backward(args, world, rank, local):
     e2e = {"value": round(units * e_steps * world / (e_ms * 1e-3) / 1e6, 3), "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
            "ms_per_step": round(e_ms / e_steps, 4)}
+    epi = run_epilogue_backward_record(sets, wl, steps, warmup, world, dev, stream, peaks)
     out = {
         "metric": METRIC.replace("(prefill, decode)", "(backward)"), "value": round(value, 3), "unit": UNIT,
         "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": round(total_ms / steps, 5),
@@ -551,10 +552,56 @@ def run_backward(args, world, rank, local):
                    "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world} (independent (b,h) units)",
                    "l2": f"{n_sets} rotating input sets, {n_sets * set_bytes / 1e6:.0f} MB"},
         "roofline": roof, "e2e": e2e, "gpu_launches": steps, "clocks": clocks.summary(),
+        "epilogue_backward": epi,
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline_backward(wl)
     return out
+
+
+def run_epilogue_backward_record(sets, wl, steps, warmup, world, dev, stream, peaks):
+    """The epilogue's backward (wkv7.epilogue_backward) over the same batch, the forward's
+    readout as y and dy as the gradient arriving at the epilogue: a record of the backward line.
+    HBM-bound: per token-head it reads y and dout (fp32) and r, k, v, and writes dy, dr, dk, dv
+    (fp32)."""
+    from linear_rnn_sequence_rwkv_b200 import wkv7
+    B, T, H, N = wl.B, wl.T, wl.H, wl.N
+    g = torch.Generator(device=dev).manual_seed(4242)
+    ln_w = 1.0 + 0.1 * torch.randn(H, N, device=dev, generator=g)
+    ln_b = 0.1 * torch.randn(H, N, device=dev, generator=g)
+    r_k = 0.5 * torch.randn(H, N, device=dev, generator=g)
+    grads = {n: torch.empty((B, T, H, N) if n in ("dy", "dr", "dk", "dv") else (H, N), device=dev)
+             for n in wkv7.EPILOGUE_GRAD_NAMES}
+    ws = torch.empty(max(1, int(wkv7.load().wkv7_epilogue_backward_workspace_bytes(B, T, H, N))), dtype=torch.uint8,
+                     device=dev)
+
+    def step(i):
+        s = sets[i % len(sets)]
+        wkv7.epilogue_backward(s["y"], s["r"], s["k"], s["v"], ln_w, ln_b, r_k, s["dy"], grads=grads, workspace=ws)
+
+    for i in range(max(3, warmup)):
+        step(i)
+    torch.cuda.synchronize(dev)
+    n = max(steps, 20)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    with ClockSampler(dev.index) as clocks:
+        e0.record(stream)
+        for i in range(n):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / n
+    units = B * T * H
+    elem = sets[0]["r"].element_size()
+    nbytes = units * N * (4 + 3 * elem + 4 + 4 * 4)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"ms_per_step": round(ms, 5), "value": round(units * world / (ms * 1e-3) / 1e6, 3), "unit": UNIT,
+            "steps": n, "gpu_launches_per_step": 2,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                         "frac": round(gbs / float(peaks["hbm_gbs"]), 4), "traffic": None,
+                         "kernel": "epilogue_bwd_kernel", "algorithmic_bytes_per_launch": nbytes},
+            "clocks": clocks.summary()}
 
 
 def run_layer(args, world, rank, local):

@@ -56,7 +56,7 @@ extern "C" {
 #define WKV7_API
 #endif
 
-#define WKV7_ABI_VERSION 4
+#define WKV7_ABI_VERSION 5
 #define WKV7_HEAD_SIZE 64
 #define WKV7_MAX_SEGMENTS 8   /* CTAs per (b, h) of WKV7_ALGO_SPLIT (one thread-block cluster) */
 
@@ -323,6 +323,46 @@ WKV7_API wkv7_status wkv7_layer_forward(int B, int T, wkv7_dtype dt, const wkv7_
 
 /* Workspace bytes of wkv7_layer_forward (0 when T = 0 or the arguments are invalid). Host only. */
 WKV7_API size_t wkv7_layer_workspace_bytes(int B, int T, wkv7_dtype dt, const wkv7_layer_dims *dims);
+
+/*
+ * The epilogue on its own, out of place (RWKV-7 rebuttal page, numpy time_mixing listing: the
+ * group_norm lambda and the bonus line after the readout): per (b, t, h) row of N channels
+ *     out = (y - mean(y)) / sqrt(var(y) + gn_eps) * ln_w + ln_b + (sum_j r_j k_j r_k[j]) v
+ * with the population variance: the operation wkv7_forward applies when opts carries ln_w, ln_b
+ * and r_k. A training step runs wkv7_forward without the epilogue, keeps its readout y for the
+ * backward, and applies this.
+ * y, out  [B][T][H][N] fp32 (out may be y: in place; otherwise they must not overlap).
+ * r, k, v [B][T][H][N] of dt (prepared inputs: k is the replacement key).
+ * ln_w, ln_b, r_k [H][N] fp32; gn_eps > 0 (64e-5 in the pages). N 64 or 128.
+ * Errors: WKV7_ERR_ARG, WKV7_ERR_ALIGN (every pointer 16-byte aligned), WKV7_ERR_UNSUPPORTED (N),
+ * WKV7_ERR_CUDA. T = 0 does nothing.
+ */
+WKV7_API wkv7_status wkv7_epilogue(int B, int T, int H, int N, wkv7_dtype dt, const float *y, const void *r,
+                                   const void *k, const void *v, const float *ln_w, const float *ln_b,
+                                   const float *r_k, float gn_eps, float *out, void *stream);
+
+/*
+ * Backward of wkv7_epilogue for L = <dout, out>. The pages print the forward only; this is its
+ * chain rule. With yn the normalised row, inv its inverse standard deviation and
+ * beta = sum_j r_j k_j r_k[j], per row:
+ *     dv = beta dout,  dbeta = sum_i dout_i v_i,  dr = dbeta k r_k,  dk = dbeta r r_k,
+ *     dy = inv (g - mean(g) - yn mean(g yn))  with g = dout ln_w,
+ * and over all rows dr_k = sum dbeta r k, dln_w = sum dout yn, dln_b = sum dout.
+ * Inputs as wkv7_epilogue (y: the readout before the epilogue) plus dout [B][T][H][N] fp32.
+ * Outputs (fp32, overwritten, no overlap with each other or the inputs): dy (the gradient that
+ * wkv7_backward takes as its dy), the bonus's share of dr, dk, dv [B][T][H][N] (add them to
+ * wkv7_backward's), dln_w, dln_b, dr_k [H][N]. The parameter sums run in a fixed order, so
+ * repeated calls give identical results.
+ * Workspace: wkv7_epilogue_backward_workspace_bytes(B, T, H, N) bytes. Errors as wkv7_epilogue,
+ * plus WKV7_ERR_WORKSPACE. T = 0 writes zero parameter gradients.
+ */
+WKV7_API size_t wkv7_epilogue_backward_workspace_bytes(int B, int T, int H, int N);
+WKV7_API wkv7_status wkv7_epilogue_backward(int B, int T, int H, int N, wkv7_dtype dt, const float *y,
+                                            const void *r, const void *k, const void *v, const float *ln_w,
+                                            const float *ln_b, const float *r_k, float gn_eps, const float *dout,
+                                            float *dy, float *dr, float *dk, float *dv, float *dln_w,
+                                            float *dln_b, float *dr_k, void *workspace, size_t workspace_bytes,
+                                            void *stream);
 
 /*
  * One decode step for every (b, h): the recurrence for a single token, with the

@@ -16,6 +16,7 @@
 #include <utility>
 
 #include "common.cuh"
+#include "epilogue.cuh"
 
 namespace wkv7 {
 
@@ -647,6 +648,113 @@ wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype dt, const void 
     p.stream = cs;
     e = wkv7::launch_backward(p);
     return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "backward launch");
+}
+
+}  // extern "C"
+
+namespace {
+
+// Shared checks of the epilogue entries: sizes, dtype, head size, the epilogue's inputs.
+wkv7_status epilogue_args(int B, int T, int H, int N, wkv7_dtype dt, float gn_eps, size_t &tok) {
+    if (B <= 0 || H <= 0 || N <= 0 || T < 0) return fail(WKV7_ERR_ARG, "bad sizes B=%d T=%d H=%d N=%d", B, T, H, N);
+    if (N != wkv7::kN && N != 128) return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: N=64 and N=128 are implemented", N);
+    if (dt != WKV7_F32 && dt != WKV7_BF16) return fail(WKV7_ERR_ARG, "unknown dtype %d", (int)dt);
+    if (!(gn_eps > 0.f) || !std::isfinite(gn_eps)) return fail(WKV7_ERR_ARG, "gn_eps must be finite and > 0");
+    tok = 1;
+    if (!mul_ok(tok, B) || !mul_ok(tok, T) || !mul_ok(tok, H) || !mul_ok(tok, N) || tok > (size_t(1) << 40))
+        return fail(WKV7_ERR_ARG, "sizes overflow");
+    return WKV7_OK;
+}
+
+// Alignment, device placement and overlaps of bufs[0 .. n): entries from `first_out` on are outputs
+// and may overlap nothing else, except the pairs the caller allows through `allowed`.
+template <class Allowed>
+wkv7_status check_buffers(const Buf *bufs, int n, int first_out, Allowed allowed) {
+    for (int i = 0; i < n; ++i) {
+        if (bufs[i].bytes && !bufs[i].ptr) return fail(WKV7_ERR_ARG, "%s is NULL", bufs[i].name);
+        if (bufs[i].ptr && !aligned16(bufs[i].ptr)) return fail(WKV7_ERR_ALIGN, "%s is not 16-byte aligned", bufs[i].name);
+    }
+    for (int o = first_out; o < n; ++o)
+        for (int i = 0; i < n; ++i)
+            if (i != o && overlaps(bufs[o], bufs[i]) && !allowed(o, i))
+                return fail(WKV7_ERR_ARG, "%s overlaps %s", bufs[o].name, bufs[i].name);
+    int device = 0;
+    cudaError_t e = cudaGetDevice(&device);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return cuda_fail(e, "cudaGetDevice");
+    }
+    for (int i = 0; i < n; ++i) {
+        const wkv7_status s = check_device_buffer(bufs[i], device);
+        if (s != WKV7_OK) return s;
+    }
+    return WKV7_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+wkv7_status wkv7_epilogue(int B, int T, int H, int N, wkv7_dtype dt, const float *y, const void *r, const void *k,
+                          const void *v, const float *ln_w, const float *ln_b, const float *r_k, float gn_eps,
+                          float *out, void *stream) {
+    g_err[0] = '\0';
+    size_t tok = 0;
+    wkv7_status st = epilogue_args(B, T, H, N, dt, gn_eps, tok);
+    if (st != WKV7_OK) return st;
+    if (T == 0) return WKV7_OK;
+    const size_t in = tok * elem_bytes(dt), f = tok * 4, ph = size_t(H) * N * 4;
+    const Buf bufs[] = {{"y", y, f},         {"r", r, in},       {"k", k, in},     {"v", v, in},
+                        {"ln_w", ln_w, ph},  {"ln_b", ln_b, ph}, {"r_k", r_k, ph}, {"out", out, f}};
+    st = check_buffers(bufs, 8, 7, [&](int o, int i) { return o == 7 && i == 0 && out == y; });
+    if (st != WKV7_OK) return st;
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    if (out != y && (e = cudaMemcpyAsync(out, y, f, cudaMemcpyDeviceToDevice, cs)) != cudaSuccess)
+        return cuda_fail(e, "copy of y");
+    wkv7::FwdArgs p{};
+    p.B = B; p.T = T; p.H = H; p.N = N; p.dt = dt;
+    p.r = r; p.k = k; p.v = v; p.y = out;
+    p.ln_w = ln_w; p.ln_b = ln_b; p.r_k = r_k; p.gn_eps = gn_eps; p.raw = false; p.stream = cs;
+    e = wkv7::launch_epilogue(p);
+    return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "epilogue launch");
+}
+
+size_t wkv7_epilogue_backward_workspace_bytes(int B, int T, int H, int N) {
+    if (B <= 0 || T < 0 || H <= 0 || (N != wkv7::kN && N != 128)) return 0;
+    size_t tok = 1;
+    if (!mul_ok(tok, B) || !mul_ok(tok, T) || !mul_ok(tok, H) || !mul_ok(tok, N) || tok > (size_t(1) << 40)) return 0;
+    return wkv7::epilogue_backward_partials(B, T, H, N) * sizeof(float);
+}
+
+wkv7_status wkv7_epilogue_backward(int B, int T, int H, int N, wkv7_dtype dt, const float *y, const void *r,
+                                   const void *k, const void *v, const float *ln_w, const float *ln_b,
+                                   const float *r_k, float gn_eps, const float *dout, float *dy, float *dr,
+                                   float *dk, float *dv, float *dln_w, float *dln_b, float *dr_k, void *workspace,
+                                   size_t workspace_bytes, void *stream) {
+    g_err[0] = '\0';
+    size_t tok = 0;
+    wkv7_status st = epilogue_args(B, T, H, N, dt, gn_eps, tok);
+    if (st != WKV7_OK) return st;
+    const size_t in = tok * elem_bytes(dt), f = tok * 4, ph = size_t(H) * N * 4;
+    const size_t need = wkv7_epilogue_backward_workspace_bytes(B, T, H, N);
+    if (need > 0 && (!workspace || workspace_bytes < need))
+        return fail(WKV7_ERR_WORKSPACE, "workspace of %zu bytes required, %zu given", need, workspace ? workspace_bytes : 0);
+    // inputs 0-7, outputs 8-14, workspace 15
+    const Buf bufs[] = {{"y", y, f},          {"r", r, in},         {"k", k, in},         {"v", v, in},
+                        {"ln_w", ln_w, ph},   {"ln_b", ln_b, ph},   {"r_k", r_k, ph},     {"dout", dout, f},
+                        {"dy", dy, f},        {"dr", dr, f},        {"dk", dk, f},        {"dv", dv, f},
+                        {"dln_w", dln_w, ph}, {"dln_b", dln_b, ph}, {"dr_k", dr_k, ph},   {"workspace", workspace, need}};
+    st = check_buffers(bufs, 16, 8, [](int, int) { return false; });
+    if (st != WKV7_OK) return st;
+    wkv7::EpiBwdArgs a{};
+    a.B = B; a.T = T; a.H = H; a.N = N; a.dt = dt;
+    a.y = y; a.r = r; a.k = k; a.v = v; a.ln_w = ln_w; a.ln_b = ln_b; a.r_k = r_k; a.eps = gn_eps;
+    a.dout = dout; a.dy = dy; a.dr = dr; a.dk = dk; a.dv = dv; a.dln_w = dln_w; a.dln_b = dln_b; a.dr_k = dr_k;
+    a.ws = static_cast<float *>(workspace);
+    a.stream = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = wkv7::launch_epilogue_backward(a);
+    return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "epilogue backward launch");
 }
 
 }  // extern "C"

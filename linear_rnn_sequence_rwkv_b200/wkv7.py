@@ -19,7 +19,7 @@ import torch
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libwkv7.so")
 HEAD_SIZE = 64
-ABI_VERSION = 4          # WKV7_ABI_VERSION of include/wkv7.h this binding follows
+ABI_VERSION = 5          # WKV7_ABI_VERSION of include/wkv7.h this binding follows
 
 # wkv7_status
 OK, ERR_ARG, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(7)
@@ -32,7 +32,8 @@ EXPORTED = ("wkv7_opts_default", "wkv7_forward", "wkv7_decode_step", "wkv7_works
             "wkv7_status_string", "wkv7_last_error", "wkv7_abi_version", "wkv7_poll_device_error",
             "wkv7_plan", "wkv7_forward_raw", "wkv7_backward", "wkv7_backward_workspace_bytes",
             "wkv7_backward_static", "wkv7_layer_forward", "wkv7_layer_workspace_bytes", "wkv7_probe_fp32_fma",
-            "wkv7_probe_tf32_mma", "wkv7_forward_host", "wkv7_forward_host_workspace_bytes")
+            "wkv7_probe_tf32_mma", "wkv7_forward_host", "wkv7_forward_host_workspace_bytes", "wkv7_epilogue",
+            "wkv7_epilogue_backward", "wkv7_epilogue_backward_workspace_bytes")
 
 
 class Wkv7Error(RuntimeError):
@@ -92,6 +93,13 @@ def load():
         lib.wkv7_backward.restype = ci
         lib.wkv7_backward_static.argtypes = [ci, ci, ci, ci, ci] + [vp] * 6 + [vp, vp, ci, vp, vp] + [vp] * 7 + [vp]
         lib.wkv7_backward_static.restype = ci
+        lib.wkv7_epilogue.argtypes = [ci, ci, ci, ci, ci] + [vp] * 7 + [ctypes.c_float, vp, vp]
+        lib.wkv7_epilogue.restype = ci
+        lib.wkv7_epilogue_backward_workspace_bytes.argtypes = [ci, ci, ci, ci]
+        lib.wkv7_epilogue_backward_workspace_bytes.restype = ctypes.c_size_t
+        lib.wkv7_epilogue_backward.argtypes = [ci, ci, ci, ci, ci] + [vp] * 7 + [ctypes.c_float] + [vp] * 8 + [
+            vp, ctypes.c_size_t, vp]
+        lib.wkv7_epilogue_backward.restype = ci
         lib.wkv7_layer_forward.argtypes = [ci, ci, ci, ctypes.POINTER(LayerDims), ctypes.POINTER(LayerParams)] + [
             vp] * 7 + [ctypes.POINTER(Opts), vp, ctypes.c_size_t, vp]
         lib.wkv7_layer_forward.restype = ci
@@ -291,6 +299,47 @@ def backward(r, w, k, v, kk, a, dy, S0=None, dS_T=None, *, snapshots=None, snap_
     out = dict(grads)
     out["dS0"] = dS0
     return out
+
+
+def epilogue(y, r, k, v, ln_w, ln_b, r_k, *, gn_eps=64e-5, out=None, stream=None):
+    """The group_norm + bonus epilogue on its own (wkv7_epilogue): returns out [B, T, H, N] fp32;
+    ``out=y`` applies it in place. Device tensors only; r, k, v prepared inputs of one dtype."""
+    lib = load()
+    B, T, H, N = y.shape
+    if out is None:
+        out = torch.empty_like(y)
+    with torch.cuda.device(y.device):
+        st = lib.wkv7_epilogue(B, T, H, N, _dt(r), _ptr(y), _ptr(r), _ptr(k), _ptr(v), _ptr(ln_w), _ptr(ln_b),
+                               _ptr(r_k), float(gn_eps), _ptr(out), _stream_handle(y.device, stream))
+    _check(st, "wkv7_epilogue")
+    return out
+
+
+EPILOGUE_GRAD_NAMES = ("dy", "dr", "dk", "dv", "dln_w", "dln_b", "dr_k")
+
+
+def epilogue_backward(y, r, k, v, ln_w, ln_b, r_k, dout, *, gn_eps=64e-5, grads=None, workspace=None, stream=None):
+    """Backward of the epilogue (wkv7_epilogue_backward) for <dout, out>: returns a dict of dy,
+    and the bonus's dr, dk, dv ([B, T, H, N] fp32) and dln_w, dln_b, dr_k ([H, N] fp32). y is
+    the readout before the epilogue; dy is what ``backward`` takes, and its dr, dk, dv add to
+    these."""
+    lib = load()
+    B, T, H, N = y.shape
+    dev = y.device
+    if grads is None:
+        grads = {n: torch.empty((B, T, H, N) if n in ("dy", "dr", "dk", "dv") else (H, N), device=dev,
+                                dtype=torch.float32) for n in EPILOGUE_GRAD_NAMES}
+    need = int(lib.wkv7_epilogue_backward_workspace_bytes(B, T, H, N))
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = lib.wkv7_epilogue_backward(B, T, H, N, _dt(r), _ptr(y), _ptr(r), _ptr(k), _ptr(v), _ptr(ln_w),
+                                        _ptr(ln_b), _ptr(r_k), float(gn_eps), _ptr(dout),
+                                        *(_ptr(grads[n]) for n in EPILOGUE_GRAD_NAMES), _ptr(workspace), ws_bytes,
+                                        _stream_handle(dev, stream))
+    _check(st, "wkv7_epilogue_backward")
+    return dict(grads)
 
 
 STATIC_SCRATCH_BYTES = 32 << 20   # capacity of the library's static backward scratch

@@ -37,7 +37,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_strings(lib):
-    assert lib.wkv7_abi_version() == 4
+    assert lib.wkv7_abi_version() == 5
     assert lib.wkv7_status_string(0) == b"WKV7_OK"
     assert lib.wkv7_status_string(3) == b"WKV7_ERR_ALIGN"
     assert lib.wkv7_status_string(99) == b"WKV7_ERR_UNKNOWN"
@@ -285,3 +285,45 @@ def test_layer_rejects_bad_arguments(lib):
     M, C = 20, 128
     want = 5 * up(M * C * 2) + 4 * up(M * 64 * 2) + 2 * up(M * C * 4) + 8 * up(64 * C * 2)
     assert lib.wkv7_layer_workspace_bytes(2, 10, 1, ctypes.byref(dims)) == want
+
+
+def _epi(lib, B=1, T=4, H=1, N=64, dt=1, eps=64e-5, ptrs=None):
+    p = ptrs or {}
+    get = lambda n: ctypes.c_void_p(p.get(n, FAKE)) if p.get(n, FAKE) is not None else None
+    return lib.wkv7_epilogue(B, T, H, N, dt, *(get(n) for n in ("y", "r", "k", "v", "ln_w", "ln_b", "r_k")),
+                             ctypes.c_float(eps), get("out"), None)
+
+
+def _epi_bwd(lib, B=1, T=4, H=1, N=64, dt=1, ptrs=None, ws=None, ws_bytes=0):
+    p = ptrs or {}
+    names = ("y", "r", "k", "v", "ln_w", "ln_b", "r_k")
+    outs = ("dy", "dr", "dk", "dv", "dln_w", "dln_b", "dr_k")
+    # distinct fake addresses far apart, so that only the overlaps a test asks for exist
+    base = {n: FAKE + (i + 1) * (1 << 24) for i, n in enumerate(names + ("dout",) + outs)}
+    get = lambda n: ctypes.c_void_p(p.get(n, base[n]))
+    return lib.wkv7_epilogue_backward(B, T, H, N, dt, *(get(n) for n in names), ctypes.c_float(64e-5), get("dout"),
+                                      *(get(n) for n in outs), ws, ws_bytes, None)
+
+
+def test_epilogue_entries_validate_before_touching_memory(lib):
+    assert _epi(lib, N=32) == wkv7.ERR_UNSUPPORTED
+    assert _epi(lib, eps=0.0) == wkv7.ERR_ARG
+    assert _epi(lib, eps=float("nan")) == wkv7.ERR_ARG
+    assert _epi(lib, dt=7) == wkv7.ERR_ARG
+    assert _epi(lib, ptrs={"y": FAKE + 4}) == wkv7.ERR_ALIGN
+    assert _epi(lib, ptrs={"r": None}) == wkv7.ERR_ARG
+    assert _epi(lib, T=0, ptrs={n: None for n in ("y", "r", "k", "v", "ln_w", "ln_b", "r_k", "out")}) == wkv7.OK
+    assert _epi_bwd(lib, N=96) == wkv7.ERR_UNSUPPORTED
+    assert _epi_bwd(lib) == wkv7.ERR_WORKSPACE                      # one partial block needed, none given
+    need = lib.wkv7_epilogue_backward_workspace_bytes(1, 4, 1, 64)
+    ws = ctypes.c_void_p(FAKE + (1 << 30))
+    assert _epi_bwd(lib, ptrs={"dr": FAKE + 8 * (1 << 24)}, ws=ws, ws_bytes=need) == wkv7.ERR_ARG   # dr on dout
+
+
+def test_epilogue_backward_workspace_formula(lib):
+    """One partial sum of the three parameter gradients (fp32, [3][N]) per head and per block of
+    64 (b, t) rows."""
+    assert lib.wkv7_epilogue_backward_workspace_bytes(2, 100, 3, 64) == 4 * 3 * 3 * 64 * 4
+    assert lib.wkv7_epilogue_backward_workspace_bytes(1, 64, 2, 128) == 1 * 2 * 3 * 128 * 4
+    assert lib.wkv7_epilogue_backward_workspace_bytes(1, 0, 2, 64) == 0
+    assert lib.wkv7_epilogue_backward_workspace_bytes(1, 4, 2, 32) == 0
