@@ -128,3 +128,19 @@ def test_layer_at_the_large_shape_sampled(cuda_device):
     out, _, _, S = wkv7.layer_forward(dd["x"], dd, H, last_x=dd["last_x"], v0=dd["v0"], S=S)
     assert _out_err(out[rows], out_ref, H) <= TOL_LAYER["bf16"]
     assert state_err(S[rows], S_ref) <= TOL_LAYER["bf16"]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_layer_odd_widths(cuda_device, dtype):
+    """C = 192 (three heads) and low-rank widths 70, 130, 1, 257 (padded to 128, 192, 64, 320):
+    column tiles of 64 and 128 next to each other in one launch, second-factor K of 64 to 320,
+    and 3 x 101 = 303 token rows (a partial last row block)."""
+    H = 3
+    ranks = {"d_w": 70, "d_a": 130, "d_v": 1, "d_g": 257}
+    d = inputs.make_layer(3, 101, H, seed=990 + (dtype == "f32"), dtype=dtype, ranks=ranks)
+    out_ref, _, _, S_ref = reference.time_mixing_layer(d["x"], d, d["last_x"], d["v0"], d["S0"])
+    dd = {k: (None if v is None else v.to(cuda_device)) for k, v in d.items()}
+    S = dd["S0"].clone()
+    out, _, _, S = wkv7.layer_forward(dd["x"], dd, H, last_x=dd["last_x"], v0=dd["v0"], S=S)
+    assert _out_err(out, out_ref, H) <= TOL_LAYER[dtype]
+    assert state_err(S, S_ref) <= TOL_LAYER[dtype]
