@@ -31,6 +31,7 @@
 // Shared rows are 80 floats apart (320 B = 64 mod 128), so the column pass's float4 loads
 // are free of bank conflicts (the row owners' stores are: eight lanes write one row's 128 B).
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -53,26 +54,101 @@ __host__ __device__ inline int segment_length(int T, int snap_every) {
     return (snap_every > 0 && snap_every < T) ? snap_every : (T > 0 ? T : 1);
 }
 
-enum { VW = 0, VKK, VB, VK, VR, VV, VDY, VA, kVecs };
+// Token vectors indexed by column (the key index); v and dy, indexed by row, go to BwdSmem::sc.
+enum { VW = 0, VKK, VA, VK, VR, VB, kVecs };
 enum { GU = 0, GZ, GK, GB, GW, kGrads };   // partial sums: S_t^T dy, S_{t-1}^T ds, dS^T v, db, dw
 
-struct BwdSmem {
-    float S[kLb + 1][kRows][kRS];    // S_{t0} .. S_{t0 + L}, this CTA's rows
-    float D[kLb][kRows][kRS];        // the gradient reaching S_t, t in the block
-    float vec[kVecs][kLb][kN];       // w, kk, b = kk*a, k, r, v, dy, a (fp32, all 64 channels)
-    float sa[kLb][kRows];            // s_i = S_{t-1}[i, :] . kk_t
-    float ds[kLb][kRows];            // ds_i = -dS_t[i, :] . b_t
+// The staged column vectors of a block. Each row-owner thread reads its eight columns
+// 4q + 32m + c of every vector, once per row group, so the bytes a lane reads per token set the
+// shared-memory traffic of the recurrence phases.
+//   fp32 inputs: w, kk, a, k, r and b = kk * a in fp32, in column order.
+//   bf16 inputs: w, kk, a, k, r as loaded (bf16 is exact in fp32, so nothing is lost), with the
+//                columns permuted so that a thread's eight sit in one 16-byte word (column j at
+//                8 ((j / 4) % 8) + 4 (j / 32) + j % 4); b is formed in registers as kk * a, the
+//                same fp32 product the fp32 layout stores.
+template <class Tin> struct VecTile;
+template <> struct VecTile<float> {
+    float x[kVecs][kLb][kN];
+    __device__ __forceinline__ void put(int slot, int tt, int c, float2 v) {
+        *reinterpret_cast<float2 *>(&x[slot][tt][c]) = v;
+    }
+    __device__ __forceinline__ void get8(int slot, int tt, int q, float (&o)[8]) const {
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            const float4 v = *reinterpret_cast<const float4 *>(&x[slot][tt][4 * q + 32 * m]);
+            o[4 * m] = v.x; o[4 * m + 1] = v.y; o[4 * m + 2] = v.z; o[4 * m + 3] = v.w;
+        }
+    }
+    __device__ __forceinline__ void b8(int tt, int q, const float (&)[8], float (&o)[8]) const { get8(VB, tt, q, o); }
+    __device__ __forceinline__ float4 get4(int slot, int tt, int cq) const {
+        return *reinterpret_cast<const float4 *>(&x[slot][tt][4 * cq]);
+    }
+};
+template <> struct VecTile<__nv_bfloat16> {
+    unsigned short x[VB][kLb][kN];
+    static __device__ __forceinline__ int perm(int j) { return 8 * ((j >> 2) & 7) + 4 * (j >> 5) + (j & 3); }
+    static __device__ __forceinline__ float lo(unsigned int u) { return __uint_as_float(u << 16); }
+    static __device__ __forceinline__ float hi(unsigned int u) { return __uint_as_float(u & 0xffff0000u); }
+    __device__ __forceinline__ void put(int slot, int tt, int c, unsigned int bits) {   // channels c, c + 1 (c even)
+        *reinterpret_cast<unsigned int *>(&x[slot][tt][perm(c)]) = bits;
+    }
+    __device__ __forceinline__ void get8(int slot, int tt, int q, float (&o)[8]) const {
+        const uint4 u = *reinterpret_cast<const uint4 *>(&x[slot][tt][8 * q]);
+        o[0] = lo(u.x); o[1] = hi(u.x); o[2] = lo(u.y); o[3] = hi(u.y);
+        o[4] = lo(u.z); o[5] = hi(u.z); o[6] = lo(u.w); o[7] = hi(u.w);
+    }
+    __device__ __forceinline__ void b8(int tt, int q, const float (&kk)[8], float (&o)[8]) const {
+        get8(VA, tt, q, o);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) o[c] = kk[c] * o[c];
+    }
+    __device__ __forceinline__ float4 get4(int slot, int tt, int cq) const {
+        const uint2 u = *reinterpret_cast<const uint2 *>(&x[slot][tt][perm(4 * cq)]);
+        return make_float4(lo(u.x), hi(u.x), lo(u.y), hi(u.y));
+    }
 };
 
 template <class Tin>
-__device__ __forceinline__ float ld_in(const void *p, size_t i) {
-    return load1(static_cast<const Tin *>(p) + i);
+struct BwdSmem {
+    float S[kLb + 1][kRows][kRS];    // S_{t0} .. S_{t0 + L}, this CTA's rows
+    float D[kLb][kRows][kRS];        // the gradient reaching S_t, t in the block
+    float4 sc[kLb][kRows];           // per row i: dy_i, v_i, s_i = S_{t-1}[i, :] . kk_t, ds_i = -dS_t[i, :] . b_t
+    VecTile<Tin> vec;
+};
+
+// Two adjacent channels as loaded; converted to fp32 only when staged, so that the loads of
+// the next block stay in flight across the current one.
+template <class Tin> struct Pair;
+template <> struct Pair<float> {
+    float2 x;
+    __device__ __forceinline__ void load(const void *p, size_t i) {
+        x = __ldg(reinterpret_cast<const float2 *>(static_cast<const float *>(p) + i));
+    }
+    __device__ __forceinline__ float2 get() const { return x; }
+};
+template <> struct Pair<__nv_bfloat16> {
+    unsigned int x;
+    __device__ __forceinline__ void load(const void *p, size_t i) {
+        x = __ldg(reinterpret_cast<const unsigned int *>(static_cast<const __nv_bfloat16 *>(p) + i));
+    }
+    __device__ __forceinline__ float2 get() const {   // bf16 -> fp32 is exact: the bits move up
+        return make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xffff0000u));
+    }
+};
+
+template <class Tin> __device__ __forceinline__ void put_pair(VecTile<Tin> &t, int slot, int tt, int c, const Pair<Tin> &v);
+template <> __device__ __forceinline__ void put_pair(VecTile<float> &t, int slot, int tt, int c, const Pair<float> &v) {
+    t.put(slot, tt, c, v.get());
+}
+template <> __device__ __forceinline__ void put_pair(VecTile<__nv_bfloat16> &t, int slot, int tt, int c,
+                                                     const Pair<__nv_bfloat16> &v) {
+    t.put(slot, tt, c, v.x);
 }
 
 template <class Tin>
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs p) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    BwdSmem &sm = *reinterpret_cast<BwdSmem *>(smem_raw);
+    BwdSmem<Tin> &sm = *reinterpret_cast<BwdSmem<Tin> *>(smem_raw);
     const int T = p.T, H = p.H;
     const int unit = blockIdx.x, b = unit / H, h = unit % H;
     const int tid = threadIdx.x;
@@ -109,13 +185,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs p) {
                     make_float4(x[rr][4 * m], x[rr][4 * m + 1], x[rr][4 * m + 2], x[rr][4 * m + 3]);
     };
     // this thread's eight columns of a staged token vector
-    auto vec8 = [&](int slot, int tt, float (&o)[8]) {
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
-            const float4 v = *reinterpret_cast<const float4 *>(&sm.vec[slot][tt][4 * q + 32 * m]);
-            o[4 * m] = v.x; o[4 * m + 1] = v.y; o[4 * m + 2] = v.z; o[4 * m + 3] = v.w;
-        }
-    };
+    auto vec8 = [&](int slot, int tt, float (&o)[8]) { sm.vec.get8(slot, tt, q, o); };
     auto rowsum = [&](float x) {   // over the eight lanes of a row group
         x += __shfl_xor_sync(0xffffffffu, x, 1);
         x += __shfl_xor_sync(0xffffffffu, x, 2);
@@ -124,40 +194,41 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs p) {
 
     // Token vectors of [t0, t0 + L) -> shared fp32: thread (tt = tid / 32) takes channels
     // 2 (tid % 32) and the next. `full` also loads r and dy (the backward block).
-    float pre[kVecs][2];
+    Pair<Tin> pre[VB], pre_v;
+    float2 pre_dy;
     auto fetch = [&](int t0, int L, bool full) {
         const int tt = tid >> 5, c = 2 * (tid & 31);
         if (tt < L) {
             const size_t o = tok(t0 + tt) + c;
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                pre[VW][e] = ld_in<Tin>(p.w, o + e);
-                pre[VKK][e] = ld_in<Tin>(p.kk, o + e);
-                pre[VA][e] = ld_in<Tin>(p.a, o + e);
-                pre[VK][e] = ld_in<Tin>(p.k, o + e);
-                pre[VV][e] = ld_in<Tin>(p.v, o + e);
-                if (full) {
-                    pre[VR][e] = ld_in<Tin>(p.r, o + e);
-                    pre[VDY][e] = __ldg(p.dy + o + e);
-                }
+            pre[VW].load(p.w, o);
+            pre[VKK].load(p.kk, o);
+            pre[VA].load(p.a, o);
+            pre[VK].load(p.k, o);
+            pre_v.load(p.v, o);
+            if (full) {
+                pre[VR].load(p.r, o);
+                pre_dy = __ldg(reinterpret_cast<const float2 *>(p.dy + o));
             }
         }
     };
     auto stage = [&](int L, bool full) {
         const int tt = tid >> 5, c = 2 * (tid & 31);
         if (tt < L) {
-            auto put = [&](int slot, float x0, float x1) {
-                *reinterpret_cast<float2 *>(&sm.vec[slot][tt][c]) = make_float2(x0, x1);
-            };
-            put(VW, pre[VW][0], pre[VW][1]);
-            put(VKK, pre[VKK][0], pre[VKK][1]);
-            put(VB, pre[VKK][0] * pre[VA][0], pre[VKK][1] * pre[VA][1]);
-            put(VA, pre[VA][0], pre[VA][1]);
-            put(VK, pre[VK][0], pre[VK][1]);
-            put(VV, pre[VV][0], pre[VV][1]);
+            put_pair(sm.vec, VW, tt, c, pre[VW]);
+            put_pair(sm.vec, VKK, tt, c, pre[VKK]);
+            put_pair(sm.vec, VA, tt, c, pre[VA]);
+            put_pair(sm.vec, VK, tt, c, pre[VK]);
+            if constexpr (std::is_same<Tin, float>::value) {
+                const float2 kk = pre[VKK].get(), a = pre[VA].get();
+                sm.vec.put(VB, tt, c, make_float2(kk.x * a.x, kk.y * a.y));
+            }
+            const float2 v = pre_v.get();
+            sm.sc[tt][c].y = v.x;
+            sm.sc[tt][c + 1].y = v.y;
             if (full) {
-                put(VR, pre[VR][0], pre[VR][1]);
-                put(VDY, pre[VDY][0], pre[VDY][1]);
+                put_pair(sm.vec, VR, tt, c, pre[VR]);
+                sm.sc[tt][c].x = pre_dy.x;
+                sm.sc[tt][c + 1].x = pre_dy.y;
             }
         }
     };
@@ -174,9 +245,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs p) {
         sa[0] = rowsum(acc[0][0] + acc[0][1]);
         sa[1] = rowsum(acc[1][0] + acc[1][1]);
         vec8(VW, tt, w);
-        vec8(VB, tt, bb);
+        sm.vec.b8(tt, q, kk, bb);
         vec8(VK, tt, kv);
-        const float v0 = sm.vec[VV][tt][row0 + rg], v1 = sm.vec[VV][tt][row0 + rg + 32];
+        const float v0 = sm.sc[tt][row0 + rg].y, v1 = sm.sc[tt][row0 + rg + 32].y;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             s[0][c] = fmaf(v0, kv[c], fmaf(-sa[0], bb[c], s[0][c] * w[c]));
@@ -205,9 +276,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs p) {
             stage(L, false);
             __syncthreads();
             if (t0 + kLb + kLb < te) fetch(t0 + kLb, min(kLb, te - t0 - kLb), false);
-            for (int tt = 0; tt < L; ++tt) {
+            auto seg_tok = [&](int tt) {
                 float sa[2];
                 forward_step(tt, sa);
+            };
+            if (L == kLb) {
+#pragma unroll
+                for (int tt = 0; tt < kLb; ++tt) seg_tok(tt);
+            } else {
+                for (int tt = 0; tt < L; ++tt) seg_tok(tt);
             }
         }
         // ---- blocks in reverse; each block's checkpoint is loaded one block ahead
@@ -229,23 +306,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs p) {
                 load_rows(ck + size_t((t0 - kLb - tb) / kLb) * kN * kN, cnext);
             }
             // recompute S_{t0} .. S_{t0 + L} (this CTA's rows) into shared memory
-            for (int tt = 0; tt < L; ++tt) {
+            auto rec_tok = [&](int tt) {
                 store_rows_sm(sm.S[tt], s);
                 float sa[2];
                 forward_step(tt, sa);
                 if (q == 0) {
-                    sm.sa[tt][rg] = sa[0];
-                    sm.sa[tt][rg + 32] = sa[1];
+                    sm.sc[tt][rg].z = sa[0];
+                    sm.sc[tt][rg + 32].z = sa[1];
                 }
+            };
+            if (L == kLb) {
+#pragma unroll
+                for (int tt = 0; tt < kLb; ++tt) rec_tok(tt);
+            } else {
+                for (int tt = 0; tt < L; ++tt) rec_tok(tt);
             }
             store_rows_sm(sm.S[L], s);
             // reverse recurrence over the block on the row owner's registers
-            for (int tt = L - 1; tt >= 0; --tt) {
-                float rv[8], kv[8], bb[8];
+            auto rev_tok = [&](int tt) {
+                float rv[8], kv[8], bb[8], kk[8];
                 vec8(VR, tt, rv);
                 vec8(VK, tt, kv);
-                vec8(VB, tt, bb);
-                const float dy0 = sm.vec[VDY][tt][row0 + rg], dy1 = sm.vec[VDY][tt][row0 + rg + 32];
+                vec8(VKK, tt, kk);
+                sm.vec.b8(tt, q, kk, bb);
+                const float dy0 = sm.sc[tt][row0 + rg].x, dy1 = sm.sc[tt][row0 + rg + 32].x;
                 float av[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, ab[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
@@ -261,18 +345,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs p) {
                 if (q == 0) {
                     p.dv[tok(t0 + tt) + row0 + rg] = dv0;
                     p.dv[tok(t0 + tt) + row0 + rg + 32] = dv1;
-                    sm.ds[tt][rg] = ds0;
-                    sm.ds[tt][rg + 32] = ds1;
+                    sm.sc[tt][rg].w = ds0;
+                    sm.sc[tt][rg + 32].w = ds1;
                 }
                 store_rows_sm(sm.D[tt], d);
-                float w[8], kk[8];
+                float w[8];
                 vec8(VW, tt, w);
-                vec8(VKK, tt, kk);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     d[0][c] = fmaf(ds0, kk[c], d[0][c] * w[c]);
                     d[1][c] = fmaf(ds1, kk[c], d[1][c] * w[c]);
                 }
+            };
+            if (L == kLb) {
+#pragma unroll
+                for (int tt = kLb - 1; tt >= 0; --tt) rev_tok(tt);
+            } else {
+                for (int tt = L - 1; tt >= 0; --tt) rev_tok(tt);
             }
             __syncthreads();
             // ---- column pass: the per-token gradient vectors, summed over the 64 rows
@@ -288,8 +377,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs p) {
                         const float4 sp = *reinterpret_cast<const float4 *>(&sm.S[tt][i][4 * cq]);
                         const float4 sn = *reinterpret_cast<const float4 *>(&sm.S[tt + 1][i][4 * cq]);
                         const float4 dd = *reinterpret_cast<const float4 *>(&sm.D[tt][i][4 * cq]);
-                        const float cdy = sm.vec[VDY][tt][i], cv = sm.vec[VV][tt][i];
-                        const float csa = sm.sa[tt][i], cds = sm.ds[tt][i];
+                        const float4 sc = sm.sc[tt][i];   // one 16-byte load for the row's four scalars
+                        const float cdy = sc.x, cv = sc.y, csa = sc.z, cds = sc.w;
                         const float spv[4] = {sp.x, sp.y, sp.z, sp.w}, snv[4] = {sn.x, sn.y, sn.z, sn.w};
                         const float ddv[4] = {dd.x, dd.y, dd.z, dd.w};
 #pragma unroll
@@ -310,8 +399,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs p) {
                         }
                     if (rq == 0) {
                         const size_t o = tok(t0 + tt) + 4 * cq;
-                        const float4 a4 = *reinterpret_cast<const float4 *>(&sm.vec[VA][tt][4 * cq]);
-                        const float4 kk4 = *reinterpret_cast<const float4 *>(&sm.vec[VKK][tt][4 * cq]);
+                        const float4 a4 = sm.vec.get4(VA, tt, cq);
+                        const float4 kk4 = sm.vec.get4(VKK, tt, cq);
                         *reinterpret_cast<float4 *>(p.dr + o) = make_float4(g[GU][0], g[GU][1], g[GU][2], g[GU][3]);
                         *reinterpret_cast<float4 *>(p.dk + o) = make_float4(g[GK][0], g[GK][1], g[GK][2], g[GK][3]);
                         *reinterpret_cast<float4 *>(p.dw + o) = make_float4(g[GW][0], g[GW][1], g[GW][2], g[GW][3]);
@@ -332,7 +421,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs p) {
 
 template <class Tin>
 cudaError_t launch_bwd_t(const BwdArgs &p) {
-    const int smem = int(sizeof(BwdSmem));
+    const int smem = int(sizeof(BwdSmem<Tin>));
     const cudaError_t attr = allow_dynamic_smem(reinterpret_cast<const void *>(bwd_kernel<Tin>), smem);
     if (attr != cudaSuccess) return attr;
     bwd_kernel<Tin><<<p.B * p.H, kBwdThreads, smem, p.stream>>>(p);
