@@ -167,6 +167,9 @@ __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const FwdArgs p) {
         __syncthreads();
         if (t0 + TB < T) issue_loads(t0 + TB);
         const int tn = min(TB, T - t0);
+        // Two rows per thread: two tokens per loop pass let the next token's loads start early
+        // (measured faster); one row per thread: faster rolled.
+#pragma unroll (RPT)
         for (int t = 0; t < tn; ++t) {
             float4 kk4[NM];
 #pragma unroll
