@@ -118,6 +118,29 @@ def test_backward_prefill_019b_sampled_heads(cuda_device):
     _check(sel, ref)
 
 
+def test_backward_prefill_15b_sampled_heads(cuda_device):
+    """The backward bench's launch: B16 T4096 H32 bf16 with S0 and dS_T, snapshots every 64
+    tokens from the fp32 scan forward, all 512 heads in one launch (3.5 waves of CTAs). Inputs
+    are drawn on the device; the oracle runs on four sampled (b, h) pairs, one from each wave."""
+    wl = inputs.WORKLOADS[2]
+    d = inputs.make_inputs(wl, device=str(cuda_device), seed=560)
+    g = torch.Generator(device=cuda_device).manual_seed(561)
+    d["dy"] = torch.randn(wl.B, wl.T, wl.H, 64, device=cuda_device, generator=g)
+    d["dS_T"] = 0.1 * torch.randn(wl.B, wl.H, 64, 64, device=cuda_device, generator=g)
+    if d["S0"] is None:
+        d["S0"] = 0.1 * torch.randn(wl.B, wl.H, 64, 64, device=cuda_device, generator=g)
+    _, _, snaps = wkv7.forward(*(d[n] for n in NAMES), d["S0"], snap_every=64, algo="seq")
+    got = wkv7.backward(*(d[n] for n in NAMES), d["dy"], d["S0"], d["dS_T"], snapshots=snaps, snap_every=64)
+    pairs = [(0, 0), (4, 20), (9, 17), (15, 31)]   # units b*H + h = 0, 148, 305, 511
+    sub = {n: torch.stack([d[n][b, :, h] for b, h in pairs])[:, :, None].cpu() for n in NAMES + ("dy",)}
+    sub["S0"] = torch.stack([d["S0"][b, h] for b, h in pairs])[:, None].cpu()
+    sub["dS_T"] = torch.stack([d["dS_T"][b, h] for b, h in pairs])[:, None].cpu()
+    ref = _oracle(sub)
+    sel = {n: torch.stack([got[n][b, :, h] for b, h in pairs])[:, :, None].cpu() for n in wkv7.GRAD_NAMES}
+    sel["dS0"] = torch.stack([got["dS0"][b, h] for b, h in pairs])[:, None].cpu()
+    _check(sel, ref)
+
+
 def test_gpu_gradients_match_finite_difference_of_the_oracle_forward(cuda_device):
     """A directional derivative of the oracle's fp64 forward (central difference along a
     random direction of every input) equals the GPU gradients contracted with that direction.
