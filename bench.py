@@ -10,7 +10,8 @@ One step = one pass of the hot path over one batch of the workload:
       from a CUDA graph) and a `chunk_sweep` record (the same shape at chunk 16, 32, 64);
   prefill-0.19b: B8 T1024 H12, state carried in (S0 ~ N(0, 0.1^2)) and out;
   long-context: B1 T65536 H40, decay logits ~ N(2, 1), snapshots every 4096 tokens;
-  decode: one wkv7_decode_step on B256 H40 (fp32 state in HBM).
+  decode: one wkv7_decode_step on B256 H40 (fp32 state in HBM); with --inputs raw, one
+      wkv7_decode_step_raw with the epilogue (the pre-processing and group_norm + bonus fused).
 Prints ONE JSON line (rank 0). Under torchrun every rank runs its own independent
 batch (weak scaling over (b, h) units, no collective on the data path); the timed
 region is bracketed by a barrier and a device synchronisation, and the time is the
@@ -55,7 +56,7 @@ WORKLOADS = {
 
 KERNEL_SOURCES = {"chunk_kernel": ("chunk.cu", "tc_util.cuh", "common.cuh"),
                   "bwd_kernel": ("backward.cu", "common.cuh"),
-                  "decode_kernel": ("decode.cu", "common.cuh"),
+                  "decode_kernel": ("decode.cu", "decode.cuh", "common.cuh"),
                   "seq_kernel": ("seq.cu", "common.cuh")}
 PROFILE_TAGS = {"prefill-0.19b": "prefill-0.19B", "prefill-1.5b": "prefill-1.5B",
                 "long-context": "long-context", "decode": "decode-2.9B"}
@@ -274,17 +275,19 @@ def run_gpu(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     decode = args.workload == "decode"
     raw = args.inputs == "raw"
-    if decode and raw:
-        raise SystemExit("--inputs raw applies to the prefill workloads")
     snap_every = wl.snap_every
 
     # independent batches per rank (seed offset), rotating input sets larger than L2
     seed0 = rank_seed(wl, rank)
     if decode:
+        # raw: the fused step (raw inputs pre-processed in the load, group_norm + bonus epilogue)
         n_tok = 128
-        d = inputs.make_inputs(wl, device=str(dev), seed=seed0, T=n_tok)
+        if raw:
+            d = inputs.make_raw_inputs(dataclasses.replace(wl, epilogue=True), device=str(dev), seed=seed0, T=n_tok)
+        else:
+            d = inputs.make_inputs(wl, device=str(dev), seed=seed0, T=n_tok)
         B, H, N = wl.B, wl.H, wl.N
-        steps_in = {n: d[n].transpose(0, 1).contiguous() for n in NAMES}      # [128, B, H, N]
+        steps_in = {n: d[n].transpose(0, 1).contiguous() for n in (RAW_NAMES if raw else NAMES)}   # [128, B, H, N]
         S = torch.zeros(B, H, N, N, device=dev)
         y = torch.empty(B, H, N, device=dev)
         T = 1
@@ -292,10 +295,15 @@ def run_gpu(args, world, rank, local):
 
         def step(i):
             j = i % n_tok
-            wkv7.decode_step(*(steps_in[n][j] for n in NAMES), S, y=y)
-        bytes_per_launch = B * H * (6 * N * 2 + N * 4 + 2 * N * N * 4)
+            if raw:
+                wkv7.decode_step_raw(*(steps_in[n][j] for n in RAW_NAMES), d["k_k"], S, k_a=d["k_a"], y=y,
+                                     ln_w=d["ln_w"], ln_b=d["ln_b"], r_k=d["r_k"])
+            else:
+                wkv7.decode_step(*(steps_in[n][j] for n in NAMES), S, y=y)
+        n_in = 5 if raw else 6
+        bytes_per_launch = B * H * (n_in * N * 2 + N * 4 + 2 * N * N * 4) + (H * N * 5 * 4 if raw else 0)
         launches_per_step = 1
-        epilogue = False
+        epilogue = raw
     else:
         B, T, H, N = wl.B, wl.T, wl.H, wl.N
         n_vec = 5 if raw else 6
@@ -433,7 +441,11 @@ def run_decode_record(args, world, rank, local):
     per CUDA graph replay), measured in the same run as the prefill line."""
     d = run_gpu(_sub_args(args, workload="decode", steps=256), world, rank, local)
     keep = ("value", "unit", "ms_per_step", "steps", "warmup", "dtype", "config", "roofline", "gpu_launches", "clocks")
-    return {k: d[k] for k in keep}
+    rec = {k: d[k] for k in keep}
+    # the same steps from raw inputs with the epilogue fused (wkv7_decode_step_raw)
+    f = run_gpu(_sub_args(args, workload="decode", steps=256, inputs="raw"), world, rank, local)
+    rec["raw_inputs_with_epilogue"] = {k: f[k] for k in ("value", "ms_per_step", "roofline", "gpu_launches", "clocks")}
+    return rec
 
 
 def run_chunk_sweep(args, world, rank, local, steps):
@@ -850,7 +862,8 @@ def main(argv=None):
     ap.add_argument("--pass", dest="pass_", choices=["forward", "backward", "layer"], default="forward",
                     help="backward: gradients of every input from a forward's snapshots")
     ap.add_argument("--inputs", choices=["prepared", "raw"], default="prepared",
-                    help="raw: decay/rate logits and the key before its update, pre-processing fused")
+                    help="raw: decay/rate logits and the key before its update, pre-processing fused "
+                         "(decode: with the epilogue too)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -56,7 +56,7 @@ extern "C" {
 #define WKV7_API
 #endif
 
-#define WKV7_ABI_VERSION 5
+#define WKV7_ABI_VERSION 6
 #define WKV7_HEAD_SIZE 64
 #define WKV7_MAX_SEGMENTS 8   /* CTAs per (b, h) of WKV7_ALGO_SPLIT (one thread-block cluster) */
 
@@ -377,6 +377,35 @@ WKV7_API wkv7_status wkv7_decode_step(int B, int H, int N, wkv7_dtype dt,
                              const void *r, const void *w, const void *k, const void *v,
                              const void *kk, const void *a,
                              float *S, float *y, void *stream);
+
+/*
+ * wkv7_decode_step with the fused group_norm + bonus epilogue of wkv7_forward: the head's N
+ * readouts are normalised over the head (population variance plus gn_eps), scaled by ln_w and
+ * shifted by ln_b, and (sum_j r_j k_j r_k[j]) v is added; y receives the result. ln_w, ln_b,
+ * r_k: [H][N] fp32, all three or none (none = wkv7_decode_step); gn_eps > 0 when they are given
+ * (64e-5 in the pages). Other arguments and errors as wkv7_decode_step; the parameters must be
+ * 16-byte aligned device memory. (Rebuttal page, the numpy time_mixing listing, output lines.)
+ */
+WKV7_API wkv7_status wkv7_decode_step_ex(int B, int H, int N, wkv7_dtype dt,
+                                         const void *r, const void *w, const void *k, const void *v,
+                                         const void *kk, const void *a, float *S, float *y,
+                                         const float *ln_w, const float *ln_b, const float *r_k,
+                                         float gn_eps, void *stream);
+
+/*
+ * One decode step from the raw time-mixing values, the pre-processing of wkv7_forward_raw done in
+ * the step's load (w = exp(-sigmoid(w_logit) / sqrt(e)), a = sigmoid(a_logit),
+ * kk = (k * k_k) / max(||k * k_k||_2, 1e-12) over the head's channels, k~ = k + k (a - 1) k_a;
+ * kk uses k, the update and the bonus use k~), with the optional epilogue of
+ * wkv7_decode_step_ex. Inputs r, w_logit, k, v, a_logit: [B][H][N] of dtype dt; k_k [H][N] fp32
+ * required, k_a [H][N] fp32 or NULL (= 0). S, y, the epilogue arguments and the errors as
+ * wkv7_decode_step_ex; WKV7_ERR_ARG also when k_k is NULL.
+ */
+WKV7_API wkv7_status wkv7_decode_step_raw(int B, int H, int N, wkv7_dtype dt,
+                                          const void *r, const void *w_logit, const void *k, const void *v,
+                                          const void *a_logit, const float *k_k, const float *k_a,
+                                          float *S, float *y, const float *ln_w, const float *ln_b,
+                                          const float *r_k, float gn_eps, void *stream);
 
 /*
  * Synchronises `stream`, then reports whether a kernel of this library gave up one

@@ -16,6 +16,7 @@
 #include <utility>
 
 #include "common.cuh"
+#include "decode.cuh"
 #include "epilogue.cuh"
 
 namespace wkv7 {
@@ -336,6 +337,12 @@ wkv7_status forward_impl(bool raw, int B, int T, int H, int N, wkv7_dtype dt, co
     return WKV7_OK;
 }
 
+// Defined with the other shared checks below.
+wkv7_status decode_impl(int B, int H, int N, wkv7_dtype dt, const void *r, const void *w, const void *k,
+                        const void *v, const void *kk, const void *a, float *S, float *y, bool raw,
+                        const float *k_k, const float *k_a, const float *ln_w, const float *ln_b,
+                        const float *r_k, float gn_eps, void *stream);
+
 }  // namespace
 
 extern "C" {
@@ -406,40 +413,26 @@ wkv7_status wkv7_poll_device_error(void *stream) {
 wkv7_status wkv7_decode_step(int B, int H, int N, wkv7_dtype dt, const void *r, const void *w, const void *k,
                              const void *v, const void *kk, const void *a, float *S, float *y, void *stream) {
     g_err[0] = '\0';
-    if (N <= 0 || B <= 0 || H <= 0) return fail(WKV7_ERR_ARG, "bad sizes B=%d H=%d N=%d", B, H, N);
-    if (N != wkv7::kN && N != 128)
-        return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: N=64 and N=128 are implemented", N);
-    if (dt != WKV7_F32 && dt != WKV7_BF16) return fail(WKV7_ERR_ARG, "unknown dtype %d", (int)dt);
-    size_t tok = 1;
-    if (!mul_ok(tok, B) || !mul_ok(tok, H) || !mul_ok(tok, N) || tok > (size_t(1) << 36))
-        return fail(WKV7_ERR_ARG, "sizes overflow");
-    const void *req[] = {r, w, k, v, kk, a, S, y};
-    const char *names[] = {"r", "w", "k", "v", "kk", "a", "S", "y"};
-    const size_t in_bytes = tok * elem_bytes(dt);
-    const size_t bytes[] = {in_bytes, in_bytes, in_bytes, in_bytes, in_bytes, in_bytes, tok * N * 4, tok * 4};
-    for (int i = 0; i < 8; ++i) {
-        if (!req[i]) return fail(WKV7_ERR_ARG, "%s is NULL", names[i]);
-        if (!aligned16(req[i])) return fail(WKV7_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
-    }
-    const Buf sb{"S", S, bytes[6]}, yb{"y", y, bytes[7]};
-    for (int i = 0; i < 6; ++i) {
-        const Buf ib{names[i], req[i], in_bytes};
-        if (overlaps(sb, ib) || overlaps(yb, ib)) return fail(WKV7_ERR_ARG, "output overlaps %s", names[i]);
-    }
-    if (overlaps(sb, yb)) return fail(WKV7_ERR_ARG, "y overlaps S");
-    int device = 0;
-    cudaError_t e = cudaGetDevice(&device);
-    if (e != cudaSuccess) {
-        cudaGetLastError();
-        return cuda_fail(e, "cudaGetDevice");
-    }
-    for (int i = 0; i < 8; ++i) {
-        const wkv7_status s = check_device_buffer(Buf{names[i], req[i], bytes[i]}, device);
-        if (s != WKV7_OK) return s;
-    }
-    wkv7::DecArgs p{B, H, N, dt, r, w, k, v, kk, a, S, y, static_cast<cudaStream_t>(stream)};
-    e = wkv7::launch_decode(p);
-    return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "decode launch");
+    return decode_impl(B, H, N, dt, r, w, k, v, kk, a, S, y, false, nullptr, nullptr, nullptr, nullptr, nullptr,
+                       64e-5f, stream);
+}
+
+wkv7_status wkv7_decode_step_ex(int B, int H, int N, wkv7_dtype dt, const void *r, const void *w, const void *k,
+                                const void *v, const void *kk, const void *a, float *S, float *y,
+                                const float *ln_w, const float *ln_b, const float *r_k, float gn_eps,
+                                void *stream) {
+    g_err[0] = '\0';
+    return decode_impl(B, H, N, dt, r, w, k, v, kk, a, S, y, false, nullptr, nullptr, ln_w, ln_b, r_k, gn_eps,
+                       stream);
+}
+
+wkv7_status wkv7_decode_step_raw(int B, int H, int N, wkv7_dtype dt, const void *r, const void *w_logit,
+                                 const void *k, const void *v, const void *a_logit, const float *k_k,
+                                 const float *k_a, float *S, float *y, const float *ln_w, const float *ln_b,
+                                 const float *r_k, float gn_eps, void *stream) {
+    g_err[0] = '\0';
+    return decode_impl(B, H, N, dt, r, w_logit, k, v, nullptr, a_logit, S, y, true, k_k, k_a, ln_w, ln_b, r_k,
+                       gn_eps, stream);
 }
 
 wkv7_status wkv7_backward_static(int B, int T, int H, int N, wkv7_dtype dt, const void *r, const void *w,
@@ -689,6 +682,56 @@ wkv7_status check_buffers(const Buf *bufs, int n, int first_out, Allowed allowed
         if (s != WKV7_OK) return s;
     }
     return WKV7_OK;
+}
+
+// The decode entries: sizes, the epilogue and raw-input arguments, then every buffer (inputs,
+// per-head parameters, the in/out state S and y) checked before the launch.
+wkv7_status decode_impl(int B, int H, int N, wkv7_dtype dt, const void *r, const void *w, const void *k,
+                        const void *v, const void *kk, const void *a, float *S, float *y, bool raw,
+                        const float *k_k, const float *k_a, const float *ln_w, const float *ln_b,
+                        const float *r_k, float gn_eps, void *stream) {
+    if (N <= 0 || B <= 0 || H <= 0) return fail(WKV7_ERR_ARG, "bad sizes B=%d H=%d N=%d", B, H, N);
+    if (N != wkv7::kN && N != 128)
+        return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: N=64 and N=128 are implemented", N);
+    if (dt != WKV7_F32 && dt != WKV7_BF16) return fail(WKV7_ERR_ARG, "unknown dtype %d", (int)dt);
+    size_t tok = 1;
+    if (!mul_ok(tok, B) || !mul_ok(tok, H) || !mul_ok(tok, N) || tok > (size_t(1) << 36))
+        return fail(WKV7_ERR_ARG, "sizes overflow");
+    const int n_epi = (ln_w != nullptr) + (ln_b != nullptr) + (r_k != nullptr);
+    if (n_epi != 0 && n_epi != 3) return fail(WKV7_ERR_ARG, "epilogue needs ln_w, ln_b and r_k (or none)");
+    if (n_epi == 3 && (!(gn_eps > 0.f) || !std::isfinite(gn_eps)))
+        return fail(WKV7_ERR_ARG, "gn_eps must be finite and > 0");
+    if (raw && !k_k) return fail(WKV7_ERR_ARG, "k_k is NULL");
+    const size_t in = tok * elem_bytes(dt), ph = size_t(H) * N * 4, pe = n_epi ? ph : 0;
+    const Buf bufs[] = {{"r", r, in},
+                        {raw ? "w_logit" : "w", w, in},
+                        {"k", k, in},
+                        {"v", v, in},
+                        {"kk", kk, raw ? 0 : in},
+                        {raw ? "a_logit" : "a", a, in},
+                        {"k_k", k_k, raw ? ph : 0},
+                        {"k_a", k_a, k_a ? ph : 0},
+                        {"ln_w", ln_w, pe},
+                        {"ln_b", ln_b, pe},
+                        {"r_k", r_k, pe},
+                        {"S", S, tok * N * 4},
+                        {"y", y, tok * 4}};
+    const wkv7_status st = check_buffers(bufs, 13, 11, [](int, int) { return false; });
+    if (st != WKV7_OK) return st;
+    wkv7::DecArgs p{B, H, N, dt, r, w, k, v, raw ? nullptr : kk, a, S, y, static_cast<cudaStream_t>(stream)};
+    wkv7::DecOpts o;
+    if (raw) {
+        o.k_k = k_k;
+        o.k_a = k_a;
+    }
+    if (n_epi) {
+        o.ln_w = ln_w;
+        o.ln_b = ln_b;
+        o.r_k = r_k;
+        o.gn_eps = gn_eps;
+    }
+    const cudaError_t e = wkv7::launch_decode_ex(p, o);
+    return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "decode launch");
 }
 
 }  // namespace

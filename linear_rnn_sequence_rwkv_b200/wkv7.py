@@ -5,9 +5,9 @@ CUDA stream; every step of the computation runs in the library's CUDA kernels.
 There is no CPU fallback: without the built library or a CUDA device these
 functions raise.
 
-Host (CPU) tensors are accepted by ``forward`` and ``decode_step`` for callers
-that keep their data on the host: the inputs are copied to the device, the
-kernels run, and the outputs are copied back (the end-to-end path).
+Host (CPU) tensors are accepted by ``forward`` for callers that keep their data
+on the host: the inputs are copied to the device, the kernels run, and the
+outputs are copied back (the end-to-end path).
 """
 from __future__ import annotations
 
@@ -19,7 +19,7 @@ import torch
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libwkv7.so")
 HEAD_SIZE = 64
-ABI_VERSION = 5          # WKV7_ABI_VERSION of include/wkv7.h this binding follows
+ABI_VERSION = 6          # WKV7_ABI_VERSION of include/wkv7.h this binding follows
 
 # wkv7_status
 OK, ERR_ARG, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(7)
@@ -33,7 +33,8 @@ EXPORTED = ("wkv7_opts_default", "wkv7_forward", "wkv7_decode_step", "wkv7_works
             "wkv7_plan", "wkv7_forward_raw", "wkv7_backward", "wkv7_backward_workspace_bytes",
             "wkv7_backward_static", "wkv7_layer_forward", "wkv7_layer_workspace_bytes", "wkv7_probe_fp32_fma",
             "wkv7_probe_tf32_mma", "wkv7_forward_host", "wkv7_forward_host_workspace_bytes", "wkv7_epilogue",
-            "wkv7_epilogue_backward", "wkv7_epilogue_backward_workspace_bytes")
+            "wkv7_epilogue_backward", "wkv7_epilogue_backward_workspace_bytes", "wkv7_decode_step_ex",
+            "wkv7_decode_step_raw")
 
 
 class Wkv7Error(RuntimeError):
@@ -88,6 +89,11 @@ def load():
         lib.wkv7_forward.restype = ci
         lib.wkv7_decode_step.argtypes = [ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp]
         lib.wkv7_decode_step.restype = ci
+        lib.wkv7_decode_step_ex.argtypes = [ci, ci, ci, ci] + [vp] * 6 + [vp, vp] + [vp] * 3 + [ctypes.c_float, vp]
+        lib.wkv7_decode_step_ex.restype = ci
+        lib.wkv7_decode_step_raw.argtypes = [ci, ci, ci, ci] + [vp] * 5 + [vp, vp] + [vp, vp] + [vp] * 3 + [
+            ctypes.c_float, vp]
+        lib.wkv7_decode_step_raw.restype = ci
         lib.wkv7_backward.argtypes = [ci, ci, ci, ci, ci] + [vp] * 6 + [vp, vp, ci, vp, vp] + [vp] * 7 + [
             vp, ctypes.c_size_t, vp]
         lib.wkv7_backward.restype = ci
@@ -406,16 +412,38 @@ def layer_workspace_bytes(B, T, params, H, N=HEAD_SIZE, dtype=torch.bfloat16) ->
                                                  ctypes.byref(layer_dims(params, H, N))))
 
 
-def decode_step(r, w, k, v, kk, a, S, *, y=None, stream=None):
-    """One decode step; inputs [B, H, 64]; S [B, H, 64, 64] fp32 updated in place. Returns y."""
+def decode_step(r, w, k, v, kk, a, S, *, y=None, ln_w=None, ln_b=None, r_k=None, gn_eps=64e-5, stream=None):
+    """One decode step; inputs [B, H, N]; S [B, H, N, N] fp32 updated in place. Returns y
+    ([B, H, N] fp32), with the group_norm + bonus epilogue applied when ln_w, ln_b, r_k are given."""
+    lib = load()
+    B, H, N = r.shape
+    if y is None:
+        y = torch.empty((B, H, N), device=r.device, dtype=torch.float32)
+    args = (B, H, N, _dt(r), _ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(kk), _ptr(a), _ptr(S), _ptr(y))
+    with torch.cuda.device(r.device):
+        if ln_w is None and ln_b is None and r_k is None:
+            st, name = lib.wkv7_decode_step(*args, _stream_handle(r.device, stream)), "wkv7_decode_step"
+        else:
+            st = lib.wkv7_decode_step_ex(*args, _ptr(ln_w), _ptr(ln_b), _ptr(r_k), ctypes.c_float(gn_eps),
+                                         _stream_handle(r.device, stream))
+            name = "wkv7_decode_step_ex"
+    _check(st, name)
+    return y
+
+
+def decode_step_raw(r, w_logit, k, v, a_logit, k_k, S, *, k_a=None, y=None, ln_w=None, ln_b=None, r_k=None,
+                    gn_eps=64e-5, stream=None):
+    """One decode step from the raw time-mixing values (decay and rate logits, the key before its
+    update; per-head k_k [H, N] and optional k_a), optionally with the epilogue. Returns y."""
     lib = load()
     B, H, N = r.shape
     if y is None:
         y = torch.empty((B, H, N), device=r.device, dtype=torch.float32)
     with torch.cuda.device(r.device):
-        st = lib.wkv7_decode_step(B, H, N, _dt(r), _ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(kk), _ptr(a),
-                                  _ptr(S), _ptr(y), _stream_handle(r.device, stream))
-    _check(st, "wkv7_decode_step")
+        st = lib.wkv7_decode_step_raw(B, H, N, _dt(r), _ptr(r), _ptr(w_logit), _ptr(k), _ptr(v), _ptr(a_logit),
+                                      _ptr(k_k), _ptr(k_a), _ptr(S), _ptr(y), _ptr(ln_w), _ptr(ln_b), _ptr(r_k),
+                                      ctypes.c_float(gn_eps), _stream_handle(r.device, stream))
+    _check(st, "wkv7_decode_step_raw")
     return y
 
 

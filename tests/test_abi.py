@@ -37,7 +37,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_strings(lib):
-    assert lib.wkv7_abi_version() == 5
+    assert lib.wkv7_abi_version() == 6
     assert lib.wkv7_status_string(0) == b"WKV7_OK"
     assert lib.wkv7_status_string(3) == b"WKV7_ERR_ALIGN"
     assert lib.wkv7_status_string(99) == b"WKV7_ERR_UNKNOWN"
@@ -327,3 +327,31 @@ def test_epilogue_backward_workspace_formula(lib):
     assert lib.wkv7_epilogue_backward_workspace_bytes(1, 64, 2, 128) == 1 * 2 * 3 * 128 * 4
     assert lib.wkv7_epilogue_backward_workspace_bytes(1, 0, 2, 64) == 0
     assert lib.wkv7_epilogue_backward_workspace_bytes(1, 4, 2, 32) == 0
+
+
+def _dec(lib, raw=False, N=64, eps=64e-5, ptrs=None, B=1, H=1):
+    """A decode entry with distinct fake addresses far apart (host checks only)."""
+    p = ptrs or {}
+    ins = ("r", "w", "k", "v", "kk", "a") if not raw else ("r", "w_logit", "k", "v", "a_logit", "k_k", "k_a")
+    names = ins + ("S", "y", "ln_w", "ln_b", "r_k")
+    base = {n: FAKE + (i + 1) * (1 << 24) for i, n in enumerate(names)}
+    get = lambda n: (lambda x: None if x is None else ctypes.c_void_p(x))(p.get(n, base[n]))
+    if raw:
+        return lib.wkv7_decode_step_raw(B, H, N, 1, *(get(n) for n in names), ctypes.c_float(eps), None)
+    return lib.wkv7_decode_step_ex(B, H, N, 1, *(get(n) for n in names), ctypes.c_float(eps), None)
+
+
+@pytest.mark.parametrize("raw", [False, True])
+def test_decode_options_validate_before_touching_memory(lib, raw):
+    assert _dec(lib, raw, N=32) == wkv7.ERR_UNSUPPORTED
+    assert _dec(lib, raw, B=0) == wkv7.ERR_ARG
+    assert _dec(lib, raw, ptrs={"ln_b": None}) == wkv7.ERR_ARG            # partial epilogue
+    assert _dec(lib, raw, eps=0.0) == wkv7.ERR_ARG
+    assert _dec(lib, raw, eps=float("inf")) == wkv7.ERR_ARG
+    assert _dec(lib, raw, ptrs={"ln_w": FAKE + (1 << 30) + 4}) == wkv7.ERR_ALIGN
+    s_base = FAKE + (8 if raw else 7) * (1 << 24)                            # where _dec puts S
+    assert _dec(lib, raw, ptrs={"y": s_base + 256}) == wkv7.ERR_ARG          # y inside S
+    assert b"overlaps" in lib.wkv7_last_error()
+    if raw:
+        assert _dec(lib, raw, ptrs={"k_k": None}) == wkv7.ERR_ARG
+        assert b"k_k" in lib.wkv7_last_error()
