@@ -132,8 +132,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecArgs p) {
     decode_body<Tin, NN, false, false>(p, DecOpts{});
 }
 template <class Tin, int NN, bool RAW, bool EPI>
-__global__ void __launch_bounds__(kDecThreads, NN == 64 ? 4 : 1) decode_fused_kernel(const DecArgs p,
-                                                                                                   const DecOpts o) {
+__global__ void __launch_bounds__(kDecThreads, NN == 64 ? 4 : 1)
+    decode_fused_kernel(const DecArgs p, const DecOpts o) {
     decode_body<Tin, NN, RAW, EPI>(p, o);
 }
 
