@@ -28,7 +28,9 @@ template <class Tin, int NN>
 __global__ void __launch_bounds__(kWarps * 32) epilogue_bwd_kernel(const EpiBwdArgs a) {
     constexpr int E = NN / 32;
     __shared__ float red[kWarps][3][NN];
-    const int h = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // one CTA per (block of kEpiRows rows, head); the heads of a row block are adjacent CTAs
+    const size_t part = blockIdx.x / unsigned(a.H);
+    const int h = int(blockIdx.x % unsigned(a.H)), warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t rows = size_t(a.B) * a.T;
     const int j0 = lane * E;
     const Tin *r = static_cast<const Tin *>(a.r), *k = static_cast<const Tin *>(a.k), *v = static_cast<const Tin *>(a.v);
@@ -48,7 +50,7 @@ __global__ void __launch_bounds__(kWarps * 32) epilogue_bwd_kernel(const EpiBwdA
         bool live[G];
 #pragma unroll
         for (int gI = 0; gI < G; ++gI) {
-            const size_t rr = size_t(blockIdx.x) * kEpiRows + i0 + gI * kWarps;
+            const size_t rr = part * kEpiRows + i0 + gI * kWarps;
             live[gI] = rr < rows;
             base[gI] = (rr * a.H + h) * NN + j0;   // row (b, t) = rr of head h
 #pragma unroll
@@ -109,13 +111,13 @@ __global__ void __launch_bounds__(kWarps * 32) epilogue_bwd_kernel(const EpiBwdA
         red[warp][2][j0 + e] = acc_k[e];
     }
     __syncthreads();
-    float *part = a.ws + (size_t(blockIdx.x) * a.H + h) * 3 * NN;
+    float *ws = a.ws + (part * a.H + h) * 3 * NN;
     for (int q = threadIdx.x; q < 3 * NN; q += blockDim.x) {
         const int which = q / NN, j = q % NN;
         float s = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) s += red[w][which][j];
-        part[q] = s;
+        ws[q] = s;
     }
 }
 
@@ -153,7 +155,8 @@ cudaError_t launch_t(const EpiBwdArgs &a) {
     const size_t rows = size_t(a.B) * a.T;
     const int parts = int((rows + kEpiRows - 1) / kEpiRows);
     if (parts > 0) {
-        epilogue_bwd_kernel<Tin, NN><<<dim3(unsigned(parts), unsigned(a.H)), kWarps * 32, 0, a.stream>>>(a);
+        // parts * H: at most 2^29 under the size limit B * T * H * N <= 2^40 (H alone when B * T <= 64)
+        epilogue_bwd_kernel<Tin, NN><<<unsigned(size_t(parts) * a.H), kWarps * 32, 0, a.stream>>>(a);
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -48,6 +48,17 @@ def test_epilogue_backward_matches_oracle(cuda_device, dtype, N, T):
         assert _param_err(got[n], ref[n]) <= TOL_PARAM, n
 
 
+def test_epilogue_backward_more_heads_than_a_grid_row(cuda_device):
+    """H = 70,000 heads, more than a grid's y extent: one CTA per (row block, head) in x."""
+    x, d = _case(1, 3, 70000, 64, "bf16", seed=1090, dev=cuda_device)
+    ref = reference.group_norm_bonus_backward(x["y"], x["r"], x["k"], x["v"], x["ln_w"], x["ln_b"], x["r_k"], x["dout"])
+    got = wkv7.epilogue_backward(d["y"], d["r"], d["k"], d["v"], d["ln_w"], d["ln_b"], d["r_k"], d["dout"])
+    for n in ("dy", "dr", "dk", "dv"):
+        assert slice_rel_err(got[n], ref[n], (0, 2)) <= TOL_ROW, n
+    for n in ("dln_w", "dln_b", "dr_k"):
+        assert _param_err(got[n], ref[n]) <= TOL_PARAM, n
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_epilogue_out_of_place_matches_oracle_and_fused(cuda_device, dtype):
     """wkv7_epilogue equals the oracle, leaves y untouched, and equals the epilogue fused into
