@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cmath>
 #include <cstdarg>
 #include <cstdint>
@@ -140,6 +141,7 @@ wkv7_status check_args(int B, int T, int H, int N, wkv7_dtype dt, const wkv7_opt
                        bool need_buffers = true) {
     if (N <= 0 || B <= 0 || H <= 0 || T < 0)
         return fail(WKV7_ERR_ARG, "bad sizes B=%d T=%d H=%d N=%d (need B,H,N >= 1, T >= 0)", B, T, H, N);
+    if (static_cast<long long>(B) * H > INT_MAX) return fail(WKV7_ERR_ARG, "B*H=%lld heads: at most %d", static_cast<long long>(B) * H, INT_MAX);
     if (N != wkv7::kN && N != 128)
         return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: N=64 and N=128 (scan path) are implemented", N);
     if (dt != WKV7_F32 && dt != WKV7_BF16) return fail(WKV7_ERR_ARG, "unknown dtype %d", (int)dt);
@@ -574,6 +576,7 @@ wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype dt, const void 
     g_err[0] = '\0';
     if (N <= 0 || B <= 0 || H <= 0 || T < 0)
         return fail(WKV7_ERR_ARG, "bad sizes B=%d T=%d H=%d N=%d (need B,H,N >= 1, T >= 0)", B, T, H, N);
+    if (static_cast<long long>(B) * H > INT_MAX) return fail(WKV7_ERR_ARG, "B*H=%lld heads: at most %d", static_cast<long long>(B) * H, INT_MAX);
     if (N != wkv7::kN) return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: the backward pass is implemented for N=64", N);
     if (dt != WKV7_F32 && dt != WKV7_BF16) return fail(WKV7_ERR_ARG, "unknown dtype %d", (int)dt);
     if (snap_every < 0) return fail(WKV7_ERR_ARG, "snap_every=%d < 0", snap_every);

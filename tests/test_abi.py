@@ -355,3 +355,9 @@ def test_decode_options_validate_before_touching_memory(lib, raw):
     if raw:
         assert _dec(lib, raw, ptrs={"k_k": None}) == wkv7.ERR_ARG
         assert b"k_k" in lib.wkv7_last_error()
+
+
+def test_head_count_bound(lib):
+    """B * H heads index the grids of the scan and the backward: more than INT_MAX is refused."""
+    assert _fwd(lib, B=1 << 16, H=1 << 15, T=1) == wkv7.ERR_ARG
+    assert b"heads" in lib.wkv7_last_error()
