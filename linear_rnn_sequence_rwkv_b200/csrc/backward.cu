@@ -87,15 +87,13 @@ template <> struct VecTile<float> {
 template <> struct VecTile<__nv_bfloat16> {
     unsigned short x[VB][kLb][kN];
     static __device__ __forceinline__ int perm(int j) { return 8 * ((j >> 2) & 7) + 4 * (j >> 5) + (j & 3); }
-    static __device__ __forceinline__ float lo(unsigned int u) { return __uint_as_float(u << 16); }
-    static __device__ __forceinline__ float hi(unsigned int u) { return __uint_as_float(u & 0xffff0000u); }
     __device__ __forceinline__ void put(int slot, int tt, int c, unsigned int bits) {   // channels c, c + 1 (c even)
         *reinterpret_cast<unsigned int *>(&x[slot][tt][perm(c)]) = bits;
     }
     __device__ __forceinline__ void get8(int slot, int tt, int q, float (&o)[8]) const {
         const uint4 u = *reinterpret_cast<const uint4 *>(&x[slot][tt][8 * q]);
-        o[0] = lo(u.x); o[1] = hi(u.x); o[2] = lo(u.y); o[3] = hi(u.y);
-        o[4] = lo(u.z); o[5] = hi(u.z); o[6] = lo(u.w); o[7] = hi(u.w);
+        o[0] = bf16_lo(u.x); o[1] = bf16_hi(u.x); o[2] = bf16_lo(u.y); o[3] = bf16_hi(u.y);
+        o[4] = bf16_lo(u.z); o[5] = bf16_hi(u.z); o[6] = bf16_lo(u.w); o[7] = bf16_hi(u.w);
     }
     __device__ __forceinline__ void b8(int tt, int q, const float (&kk)[8], float (&o)[8]) const {
         get8(VA, tt, q, o);
@@ -104,7 +102,7 @@ template <> struct VecTile<__nv_bfloat16> {
     }
     __device__ __forceinline__ float4 get4(int slot, int tt, int cq) const {
         const uint2 u = *reinterpret_cast<const uint2 *>(&x[slot][tt][perm(4 * cq)]);
-        return make_float4(lo(u.x), hi(u.x), lo(u.y), hi(u.y));
+        return make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
     }
 };
 
@@ -131,9 +129,7 @@ template <> struct Pair<__nv_bfloat16> {
     __device__ __forceinline__ void load(const void *p, size_t i) {
         x = __ldg(reinterpret_cast<const unsigned int *>(static_cast<const __nv_bfloat16 *>(p) + i));
     }
-    __device__ __forceinline__ float2 get() const {   // bf16 -> fp32 is exact: the bits move up
-        return make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xffff0000u));
-    }
+    __device__ __forceinline__ float2 get() const { return make_float2(bf16_lo(x), bf16_hi(x)); }   // exact
 };
 
 template <class Tin> __device__ __forceinline__ void put_pair(VecTile<Tin> &t, int slot, int tt, int c, const Pair<Tin> &v);

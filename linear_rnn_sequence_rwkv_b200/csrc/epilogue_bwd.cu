@@ -42,66 +42,56 @@ __global__ void __launch_bounds__(kWarps * 32) epilogue_bwd_kernel(const EpiBwdA
         acc_w[e] = acc_b[e] = acc_k[e] = 0.f;
     }
     const float inv_n = 1.f / NN;
-    // the warp's rows one at a time (G rows per batch: batching more cost occupancy)
-    constexpr int G = 1;
-    for (int i0 = warp; i0 < kEpiRows; i0 += G * kWarps) {
-        float y[G][E], rv[G][E], kv[G][E], vv[G][E], d[G][E];
-        size_t base[G];
-        bool live[G];
+    // the warp's rows one at a time (batching two or four rows per warp cost more in occupancy)
+    for (int i0 = warp; i0 < kEpiRows; i0 += kWarps) {
+        const size_t rr = part * kEpiRows + i0;
+        if (rr >= rows) break;                          // uniform over the warp
+        const size_t base = (rr * a.H + h) * NN + j0;   // row (b, t) = rr of head h
+        float y[E], rv[E], kv[E], vv[E], d[E];
 #pragma unroll
-        for (int gI = 0; gI < G; ++gI) {
-            const size_t rr = part * kEpiRows + i0 + gI * kWarps;
-            live[gI] = rr < rows;
-            base[gI] = (rr * a.H + h) * NN + j0;   // row (b, t) = rr of head h
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                y[gI][e] = live[gI] ? a.y[base[gI] + e] : 0.f;
-                rv[gI][e] = live[gI] ? load1(r + base[gI] + e) : 0.f;
-                kv[gI][e] = live[gI] ? load1(k + base[gI] + e) : 0.f;
-                vv[gI][e] = live[gI] ? load1(v + base[gI] + e) : 0.f;
-                d[gI][e] = live[gI] ? a.dout[base[gI] + e] : 0.f;
-            }
+        for (int e = 0; e < E; ++e) {
+            y[e] = a.y[base + e];
+            rv[e] = load1(r + base + e);
+            kv[e] = load1(k + base + e);
+            vv[e] = load1(v + base + e);
+            d[e] = a.dout[base + e];
         }
+        float sy = 0.f, beta = 0.f, dbeta = 0.f;
 #pragma unroll
-        for (int gI = 0; gI < G; ++gI) {
-            if (!live[gI]) continue;   // uniform over the warp
-            float sy = 0.f, beta = 0.f, dbeta = 0.f;
+        for (int e = 0; e < E; ++e) {
+            sy += y[e];
+            beta = fmaf(rv[e] * kv[e], rk[e], beta);
+            dbeta = fmaf(d[e], vv[e], dbeta);
+        }
+        sy = warp_sum(sy);
+        beta = warp_sum(beta);
+        dbeta = warp_sum(dbeta);
+        const float mean = sy * inv_n;
+        float sq = 0.f;
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
-                sy += y[gI][e];
-                beta = fmaf(rv[gI][e] * kv[gI][e], rk[e], beta);
-                dbeta = fmaf(d[gI][e], vv[gI][e], dbeta);
-            }
-            sy = warp_sum(sy);
-            beta = warp_sum(beta);
-            dbeta = warp_sum(dbeta);
-            const float mean = sy * inv_n;
-            float sq = 0.f;
+        for (int e = 0; e < E; ++e) {
+            y[e] -= mean;
+            sq = fmaf(y[e], y[e], sq);
+        }
+        const float inv = 1.f / sqrtf(warp_sum(sq) * inv_n + a.eps);
+        float g[E], sg = 0.f, sgy = 0.f;
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
-                y[gI][e] -= mean;
-                sq = fmaf(y[gI][e], y[gI][e], sq);
-            }
-            const float inv = 1.f / sqrtf(warp_sum(sq) * inv_n + a.eps);
-            float g[E], sg = 0.f, sgy = 0.f;
+        for (int e = 0; e < E; ++e) {
+            y[e] *= inv;   // yn
+            g[e] = d[e] * lw[e];
+            sg += g[e];
+            sgy = fmaf(g[e], y[e], sgy);
+            acc_w[e] = fmaf(d[e], y[e], acc_w[e]);
+            acc_b[e] += d[e];
+            acc_k[e] = fmaf(dbeta * rv[e], kv[e], acc_k[e]);
+        }
+        const float mg = warp_sum(sg) * inv_n, mgy = warp_sum(sgy) * inv_n;
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
-                y[gI][e] *= inv;   // yn
-                g[e] = d[gI][e] * lw[e];
-                sg += g[e];
-                sgy = fmaf(g[e], y[gI][e], sgy);
-                acc_w[e] = fmaf(d[gI][e], y[gI][e], acc_w[e]);
-                acc_b[e] += d[gI][e];
-                acc_k[e] = fmaf(dbeta * rv[gI][e], kv[gI][e], acc_k[e]);
-            }
-            const float mg = warp_sum(sg) * inv_n, mgy = warp_sum(sgy) * inv_n;
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                a.dy[base[gI] + e] = inv * (g[e] - mg - y[gI][e] * mgy);
-                a.dr[base[gI] + e] = dbeta * kv[gI][e] * rk[e];
-                a.dk[base[gI] + e] = dbeta * rv[gI][e] * rk[e];
-                a.dv[base[gI] + e] = beta * d[gI][e];
-            }
+        for (int e = 0; e < E; ++e) {
+            a.dy[base + e] = inv * (g[e] - mg - y[e] * mgy);
+            a.dr[base + e] = dbeta * kv[e] * rk[e];
+            a.dk[base + e] = dbeta * rv[e] * rk[e];
+            a.dv[base + e] = beta * d[e];
         }
     }
 #pragma unroll
