@@ -55,7 +55,7 @@ WORKLOADS = {
 # ---- measured DRAM traffic of the dominant kernel (committed ncu summaries under profiles/) -------
 
 KERNEL_SOURCES = {"chunk_kernel": ("chunk.cu", "tc_util.cuh", "common.cuh"),
-                  "bwd_kernel": ("backward.cu", "common.cuh"),
+                  "bwd_kernel": ("backward.cu", "backward.cuh", "tc_util.cuh", "common.cuh"),
                   "decode_kernel": ("decode.cu", "decode.cuh", "common.cuh"),
                   "seq_kernel": ("seq.cu", "common.cuh")}
 PROFILE_TAGS = {"prefill-0.19b": "prefill-0.19B", "prefill-1.5b": "prefill-1.5B",
@@ -461,7 +461,7 @@ def run_chunk_sweep(args, world, rank, local, steps):
     return rows
 
 
-BWD_FLOPS_PER_UNIT = 21 * 64 * 64   # gradient arithmetic per token-head (recomputation not counted)
+BWD_FLOPS_PER_UNIT = 21 * 64 * 64   # gradient arithmetic per token-head at N = 64 (21 N^2; recomputation not counted)
 
 
 def run_backward(args, world, rank, local):
@@ -472,6 +472,9 @@ def run_backward(args, world, rank, local):
     torch.cuda.set_device(dev)
     spec = WORKLOADS[args.workload]
     wl = inputs.WORKLOADS[spec["cid"]]
+    if args.head_size != wl.N:   # same channel count per token, wider heads
+        wl = dataclasses.replace(wl, N=args.head_size, H=max(1, wl.H * wl.N // args.head_size),
+                                 name=f"{wl.name} as N={args.head_size}")
     steps = args.steps if args.steps is not None else max(5, spec["default_steps"] // 10)
     warmup = args.warmup
     peaks, _ = _peaks()
@@ -517,9 +520,10 @@ def run_backward(args, world, rank, local):
     value = units * steps * world / (total_ms * 1e-3) / 1e6
     launch_ms = statistics.mean(per_step_ms)
     hbm_bytes = units * (6 * N * 2 + N * 4 + 6 * N * 4) + B * H * N * N * 4 * (3 + T // snap)
-    roof = fp32_roof(BWD_FLOPS_PER_UNIT * units, launch_ms, dev)
-    roof.update({"traffic": measured_traffic("bwd_kernel", args.workload), "kernel": "bwd_kernel",
-            "flops_per_unit": BWD_FLOPS_PER_UNIT, "algorithmic_bytes_per_launch": hbm_bytes,
+    flops_per_unit = BWD_FLOPS_PER_UNIT * (N // 64) ** 2
+    roof = fp32_roof(flops_per_unit * units, launch_ms, dev)
+    roof.update({"traffic": measured_traffic("bwd_kernel", args.workload) if N == 64 else None, "kernel": "bwd_kernel",
+            "flops_per_unit": flops_per_unit, "algorithmic_bytes_per_launch": hbm_bytes,
             "hbm_gbs": round(hbm_bytes / (launch_ms * 1e-3) / 1e9, 1),
             "hbm_frac": round(hbm_bytes / (launch_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]), 4)})
 

@@ -20,10 +20,9 @@
  *
  * Conventions for every entry point:
  *   - N is 64 on every path, or 128 (the larger head size the pages name as the next
- *     one) on the sequential scan, its epilogue and the decode step. The chunked
- *     algorithms and the backward pass take N = 64 only: WKV7_ALGO_CHUNK / SPLIT with
- *     N = 128 and wkv7_backward with N != 64 return WKV7_ERR_UNSUPPORTED, and
- *     WKV7_ALGO_AUTO runs N = 128 on the scan.
+ *     one) on the sequential scan, its epilogue, the decode step and the backward pass.
+ *     The chunked algorithms take N = 64 only: WKV7_ALGO_CHUNK / SPLIT with N = 128
+ *     return WKV7_ERR_UNSUPPORTED, and WKV7_ALGO_AUTO runs N = 128 on the scan.
  *   - Token tensors r, w, k, v, kk, a are [B][T][H][N] row-major (decode: [B][H][N]),
  *     all of the dtype given by `dt`. States are [B][H][N][N] fp32 row-major.
  *     y is fp32 with the layout of the token tensors.
@@ -221,11 +220,13 @@ WKV7_API size_t wkv7_forward_host_workspace_bytes(int B, int T, int H, int N, wk
  * Outputs dr, dw, dk, dv, dkk, da : [B][T][H][N] fp32 (required when T > 0).
  *         dS0               : [B][H][N][N] fp32 or NULL; may equal dS_T exactly (in place).
  * Workspace: at least wkv7_backward_workspace_bytes(B, T, H, N, snap_every) bytes of device
- * memory (the recomputation's checkpoints, one state per 4 tokens of a segment); it must not
- * overlap any other argument and its contents need no initialisation.
+ * memory (the recomputation's checkpoints, one state per 4 tokens of a segment at N = 64, per 2
+ * tokens at N = 128); it must not overlap any other argument and its contents need no
+ * initialisation.
  * Errors as wkv7_forward: WKV7_ERR_ARG for sizes, NULL required pointers, snap_every < 0,
  * missing snapshots, overlapping outputs, host or too-small buffers; WKV7_ERR_ALIGN;
- * WKV7_ERR_UNSUPPORTED for N != 64; WKV7_ERR_WORKSPACE. T = 0 copies dS_T (or zeros) to dS0.
+ * WKV7_ERR_UNSUPPORTED for N other than 64 and 128; WKV7_ERR_WORKSPACE. T = 0 copies dS_T (or
+ * zeros) to dS0.
  */
 WKV7_API wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype dt,
                           const void *r, const void *w, const void *k, const void *v,
@@ -235,9 +236,9 @@ WKV7_API wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype dt,
                           float *dr, float *dw, float *dk, float *dv, float *dkk, float *da,
                           float *dS0, void *workspace, size_t workspace_bytes, void *stream);
 
-/* Bytes of workspace wkv7_backward needs: B * H * ceil(K / 4) * N * N * 4 with K the
- * snapshot interval (or T when snap_every is 0 or >= T); 0 when T = 0 or an argument is
- * invalid. Host only. */
+/* Bytes of workspace wkv7_backward needs: B * H * ceil(K / 4) * N * N * 4 at N = 64 and
+ * B * H * ceil(K / 2) * N * N * 4 at N = 128, with K the snapshot interval (or T when snap_every
+ * is 0 or >= T); 0 when T = 0 or an argument is invalid. Host only. */
 WKV7_API size_t wkv7_backward_workspace_bytes(int B, int T, int H, int N, int snap_every);
 
 /*

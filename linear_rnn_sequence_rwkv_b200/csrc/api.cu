@@ -17,6 +17,7 @@
 #include <utility>
 
 #include "common.cuh"
+#include "backward.cuh"
 #include "decode.cuh"
 #include "epilogue.cuh"
 
@@ -562,10 +563,10 @@ wkv7_status wkv7_layer_forward(int B, int T, wkv7_dtype dt, const wkv7_layer_dim
 }
 
 size_t wkv7_backward_workspace_bytes(int B, int T, int H, int N, int snap_every) {
-    if (B <= 0 || T <= 0 || H <= 0 || N != wkv7::kN || snap_every < 0) return 0;
+    if (B <= 0 || T <= 0 || H <= 0 || (N != wkv7::kN && N != 128) || snap_every < 0) return 0;
     size_t n = 1;
     if (!mul_ok(n, B) || !mul_ok(n, H) || !mul_ok(n, T)) return 0;
-    return wkv7::backward_checkpoint_bytes(B, T, H, snap_every);
+    return wkv7::backward_checkpoint_bytes_n(B, T, H, N, snap_every);
 }
 
 wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype dt, const void *r, const void *w,
@@ -577,7 +578,8 @@ wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype dt, const void 
     if (N <= 0 || B <= 0 || H <= 0 || T < 0)
         return fail(WKV7_ERR_ARG, "bad sizes B=%d T=%d H=%d N=%d (need B,H,N >= 1, T >= 0)", B, T, H, N);
     if (static_cast<long long>(B) * H > INT_MAX) return fail(WKV7_ERR_ARG, "B*H=%lld heads: at most %d", static_cast<long long>(B) * H, INT_MAX);
-    if (N != wkv7::kN) return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: the backward pass is implemented for N=64", N);
+    if (N != wkv7::kN && N != 128)
+        return fail(WKV7_ERR_UNSUPPORTED, "head size N=%d: the backward pass is implemented for N=64 and N=128", N);
     if (dt != WKV7_F32 && dt != WKV7_BF16) return fail(WKV7_ERR_ARG, "unknown dtype %d", (int)dt);
     if (snap_every < 0) return fail(WKV7_ERR_ARG, "snap_every=%d < 0", snap_every);
     const int n_snap = snap_every > 0 ? T / snap_every : 0;
@@ -642,7 +644,7 @@ wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype dt, const void 
     p.dr = dr; p.dw = dw; p.dk = dk; p.dv = dv; p.dkk = dkk; p.da = da; p.dS0 = dS0;
     p.ws = static_cast<float *>(workspace);
     p.stream = cs;
-    e = wkv7::launch_backward(p);
+    e = wkv7::launch_backward_n(p, N);
     return e == cudaSuccess ? WKV7_OK : cuda_fail(e, "backward launch");
 }
 

@@ -248,13 +248,16 @@ def test_backward_workspace_query():
 
 
 def test_head_size_128_runs_on_the_scan():
-    """N = 128: AUTO plans the scan; the chunked algorithms and the backward refuse it."""
+    """N = 128: AUTO plans the scan and the chunked algorithms refuse it; the backward takes it
+    (checkpoints every 2 tokens: B * H * ceil(K / 2) * N * N * 4 bytes)."""
     assert wkv7.plan(2, 300, 4, 128, torch.bfloat16) == ("seq", 0)
     assert wkv7.plan(2, 300, 4, 128, torch.float32, algo="seq") == ("seq", 0)
     with pytest.raises(wkv7.Wkv7Error) as e:
         wkv7.plan(2, 300, 4, 128, torch.bfloat16, algo="chunk")
     assert e.value.status == wkv7.ERR_UNSUPPORTED
-    assert wkv7.backward_workspace_bytes(2, 300, 4, N=128) == 0
+    assert wkv7.backward_workspace_bytes(2, 300, 4, N=128) == 2 * 4 * 150 * 128 * 128 * 4
+    assert wkv7.backward_workspace_bytes(2, 300, 4, N=128, snap_every=64) == 2 * 4 * 32 * 128 * 128 * 4
+    assert wkv7.backward_workspace_bytes(2, 300, 4, N=96) == 0
 
 
 def _layer_call(lib, B=1, T=4, H=1, N=64, dt=1, drop=None, over=None, ws=None, ws_bytes=0, v0=None):

@@ -2,6 +2,8 @@
 sweep on the same seeded inputs. The kernel works in fp32 from inputs that are exact in
 fp32 (bf16 or fp32), so one bound serves both: max relative error per (b, h) slice
 <= 9e-5, the precision the pages report for their fp32 backward."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -16,11 +18,12 @@ TOL_BWD = 9e-5
 NAMES = ("r", "w", "k", "v", "kk", "a")
 
 
-def _case(B, T, H, *, dtype="bf16", seed=0, s0="normal", ds_t=True, wl=1):
-    d = inputs.make_inputs(inputs.WORKLOADS[wl], B=B, T=T, H=H, dtype=dtype, seed=seed, s0=s0)
+def _case(B, T, H, *, dtype="bf16", seed=0, s0="normal", ds_t=True, wl=1, N=64):
+    work = dataclasses.replace(inputs.WORKLOADS[wl], N=N)
+    d = inputs.make_inputs(work, B=B, T=T, H=H, dtype=dtype, seed=seed, s0=s0)
     g = torch.Generator().manual_seed(seed + 1)
-    d["dy"] = torch.randn(B, T, H, 64, generator=g)
-    d["dS_T"] = 0.1 * torch.randn(B, H, 64, 64, generator=g) if ds_t else None
+    d["dy"] = torch.randn(B, T, H, N, generator=g)
+    d["dS_T"] = 0.1 * torch.randn(B, H, N, N, generator=g) if ds_t else None
     return d
 
 
@@ -160,3 +163,53 @@ def test_gpu_gradients_match_finite_difference_of_the_oracle_forward(cuda_device
     fd = (loss(1) - loss(-1)) / (2 * eps)
     lin = sum(float((got["d" + n].double().cpu() * dirs[n]).sum()) for n in NAMES)
     assert abs(fd - lin) <= 1e-4 * max(1.0, abs(fd))
+
+
+# ---- head size 128: the rows of a head split over a cluster of two CTAs, two-token blocks ----
+
+@pytest.mark.parametrize("T", [1, 2, 3, 5, 37, 130])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_backward_n128_ragged_lengths(cuda_device, T, dtype):
+    d = _case(2, T, 3, dtype=dtype, seed=1700 + T, N=128)
+    ref = _oracle(d)
+    dd = _dev(d, cuda_device)
+    got = wkv7.backward(*(dd[n] for n in NAMES), dd["dy"], dd["S0"], dd["dS_T"])
+    _check(got, ref)
+
+
+@pytest.mark.parametrize("snap_every", [7, 64])
+def test_backward_n128_from_forward_snapshots(cuda_device, snap_every):
+    d = _case(2, 150, 2, seed=1750 + snap_every, N=128)
+    ref = _oracle(d)
+    dd = _dev(d, cuda_device)
+    _, _, snaps = wkv7.forward(*(dd[n] for n in NAMES), dd["S0"], snap_every=snap_every, algo="seq")
+    got = wkv7.backward(*(dd[n] for n in NAMES), dd["dy"], dd["S0"], dd["dS_T"], snapshots=snaps,
+                        snap_every=snap_every)
+    _check(got, ref)
+
+
+def test_backward_n128_no_state_and_in_place_state_gradient(cuda_device):
+    d = _case(1, 20, 2, seed=1770, s0="zeros", N=128)
+    ref = _oracle(d)
+    dd = _dev(d, cuda_device)
+    dS = dd["dS_T"].clone()
+    got = wkv7.backward(*(dd[n] for n in NAMES), dd["dy"], None, dS, dS0=dS)
+    _check(got, ref)
+    assert got["dS0"].data_ptr() == dS.data_ptr()
+
+
+def test_backward_n128_sampled_heads(cuda_device):
+    """B8 T1024 H6 N128 (the 0.19B channel count in 128-wide heads, bf16, S0), snapshots every 64
+    tokens from the scan forward; the oracle runs on four sampled (b, h) pairs."""
+    d = _case(8, 1024, 6, seed=1790, N=128)
+    dd = _dev(d, cuda_device)
+    _, _, snaps = wkv7.forward(*(dd[n] for n in NAMES), dd["S0"], snap_every=64, algo="seq")
+    got = wkv7.backward(*(dd[n] for n in NAMES), dd["dy"], dd["S0"], dd["dS_T"], snapshots=snaps, snap_every=64)
+    pairs = [(0, 0), (3, 5), (6, 2), (7, 5)]
+    sub = {n: torch.stack([d[n][b, :, h] for b, h in pairs])[:, :, None] for n in NAMES + ("dy",)}
+    sub["S0"] = torch.stack([d["S0"][b, h] for b, h in pairs])[:, None]
+    sub["dS_T"] = torch.stack([d["dS_T"][b, h] for b, h in pairs])[:, None]
+    ref = _oracle(sub)
+    sel = {n: torch.stack([got[n][b, :, h] for b, h in pairs])[:, :, None] for n in wkv7.GRAD_NAMES}
+    sel["dS0"] = torch.stack([got["dS0"][b, h] for b, h in pairs])[:, None]
+    _check(sel, ref)

@@ -102,7 +102,3 @@ def test_n128_refused_where_unsupported(cuda_device):
     with pytest.raises(wkv7.Wkv7Error) as e:
         wkv7.forward(*(d[n] for n in NAMES), algo="chunk")
     assert e.value.status == wkv7.ERR_UNSUPPORTED
-    dy = torch.zeros(1, 64, 1, 128, device=cuda_device)
-    with pytest.raises(wkv7.Wkv7Error) as e:
-        wkv7.backward(*(d[n] for n in NAMES), dy)
-    assert e.value.status == wkv7.ERR_UNSUPPORTED

@@ -2,6 +2,7 @@
 in place of a caller's workspace. Collected last, so that it also runs after every other
 test has used the device; it must pass alone as well."""
 import ctypes
+import dataclasses
 
 import pytest
 import torch
@@ -12,11 +13,11 @@ NAMES = ("r", "w", "k", "v", "kk", "a")
 FAKE = 0x10000
 
 
-def _case(B, T, H, seed):
-    d = inputs.make_inputs(inputs.WORKLOADS[1], B=B, T=T, H=H, seed=seed, s0="normal")
+def _case(B, T, H, seed, N=64):
+    d = inputs.make_inputs(dataclasses.replace(inputs.WORKLOADS[1], N=N), B=B, T=T, H=H, seed=seed, s0="normal")
     g = torch.Generator().manual_seed(seed + 1)
-    d["dy"] = torch.randn(B, T, H, 64, generator=g)
-    d["dS_T"] = 0.1 * torch.randn(B, H, 64, 64, generator=g)
+    d["dy"] = torch.randn(B, T, H, N, generator=g)
+    d["dS_T"] = 0.1 * torch.randn(B, H, N, N, generator=g)
     return d
 
 
@@ -34,12 +35,13 @@ def test_static_entry_rejects_requests_above_its_capacity():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("B,T,H,snap_every", [(2, 130, 3, 0), (2, 1024, 4, 0), (3, 300, 2, 64)])
-def test_static_entry_matches_workspace_entry_on_consecutive_calls(cuda_device, B, T, H, snap_every):
+@pytest.mark.parametrize("B,T,H,snap_every,N", [(2, 130, 3, 0, 64), (2, 1024, 4, 0, 64), (3, 300, 2, 64, 64),
+                                                (2, 130, 2, 0, 128), (2, 300, 3, 64, 128)])
+def test_static_entry_matches_workspace_entry_on_consecutive_calls(cuda_device, B, T, H, snap_every, N):
     """Two calls in a row with different inputs: each equals wkv7_backward bit for bit (the
     second call sees the first one's leftovers in the scratch and must not depend on them)."""
     for seed in (900 + T, 901 + T):
-        d = {k: (None if v is None else v.to(cuda_device)) for k, v in _case(B, T, H, seed).items()}
+        d = {k: (None if v is None else v.to(cuda_device)) for k, v in _case(B, T, H, seed, N).items()}
         snaps = None
         if snap_every:
             _, _, snaps = wkv7.forward(*(d[n] for n in NAMES), d["S0"], snap_every=snap_every, algo="seq")
