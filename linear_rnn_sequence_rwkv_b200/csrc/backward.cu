@@ -191,6 +191,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdArgs p) {
     const int T = p.T, H = p.H;
     const int unit = blockIdx.x / CPH, b = unit / H, h = unit % H;
     const int rank = CPH > 1 ? int(tc::cluster_rank()) : 0;   // which 64 rows of the head
+    if constexpr (CPH > 1) tc::cluster_sync();   // both CTAs running before any remote store
     const int row0 = kRows * rank;
     const int tid = threadIdx.x;
     // row owner: rows rg + NRG rr (rr < RPT), columns 4q + (N/2) m + c (m < 2, c < 4)
