@@ -264,8 +264,10 @@ cudaError_t launch_seq_t(const FwdArgs &p) {
 
 template <class Tin, int RPT>
 cudaError_t launch_seq_r(const FwdArgs &p) {
-    if (p.N == 128)
-        return p.raw ? launch_seq_t<Tin, RPT, true, 128>(p) : launch_seq_t<Tin, RPT, false, 128>(p);
+    if constexpr (RPT <= 2) {   // four rows of 32 columns would not fit the registers at N = 128
+        if (p.N == 128)
+            return p.raw ? launch_seq_t<Tin, RPT, true, 128>(p) : launch_seq_t<Tin, RPT, false, 128>(p);
+    }
     return p.raw ? launch_seq_t<Tin, RPT, true, 64>(p) : launch_seq_t<Tin, RPT, false, 64>(p);
 }
 
@@ -321,14 +323,18 @@ __global__ void __launch_bounds__(256) epilogue_kernel(const FwdArgs p, size_t r
 }  // namespace
 
 cudaError_t launch_seq(const FwdArgs &p) {
-    // 32 rows per CTA (two per thread: each token-vector read serves two rows) from 128 heads on,
-    // and always at N = 128; 16 rows per CTA only for fewer heads, where four CTAs per head keep
-    // more warps per SM (measured: 96 heads 0.389 against 0.401 ms; 128 heads 1.81 against 1.54
-    // ms and 256 heads 0.95 against 0.52 ms the other way; N = 128, 48 heads: 0.69 against 0.59 ms)
-    const bool wide = p.N == 128 || size_t(p.B) * p.H >= 128;
+    // Rows per thread (a CTA holds 16 of them per thread): more rows let each token-vector read
+    // serve more rows, fewer give a head more CTAs and an SM more warps. Measured at N = 64,
+    // B8 T1024: 96 heads one row 0.389 ms against two 0.401; 128 heads two rows 0.395 against
+    // four 0.414; 160 heads four rows 0.414 against two 0.467 and 512 heads (T4096) 2.61 against
+    // 4.08 ms, from the head count at which one CTA per head fills the 148 SMs. N = 128 takes two
+    // rows (0.59 against 0.69 ms at 48 heads; four would spill).
+    const size_t heads = size_t(p.B) * p.H;
+    const int rpt = p.N == 128 ? 2 : heads >= 148 ? 4 : heads >= 128 ? 2 : 1;
     if (p.dt == WKV7_BF16)
-        return wide ? launch_seq_r<__nv_bfloat16, 2>(p) : launch_seq_r<__nv_bfloat16, 1>(p);
-    return wide ? launch_seq_r<float, 2>(p) : launch_seq_r<float, 1>(p);
+        return rpt == 4 ? launch_seq_r<__nv_bfloat16, 4>(p)
+                        : rpt == 2 ? launch_seq_r<__nv_bfloat16, 2>(p) : launch_seq_r<__nv_bfloat16, 1>(p);
+    return rpt == 4 ? launch_seq_r<float, 4>(p) : rpt == 2 ? launch_seq_r<float, 2>(p) : launch_seq_r<float, 1>(p);
 }
 
 cudaError_t launch_copy_state(const FwdArgs &p) {

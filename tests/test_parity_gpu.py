@@ -6,7 +6,7 @@ import pytest
 import torch
 
 from linear_rnn_sequence_rwkv_b200 import inputs, wkv7
-from oracle import native
+from oracle import native, reference
 from tests.golden_util import elementary_transitions
 from tests.parity_util import TOL, as_np, heads_slice, snaps_err, state_err, y_err
 
@@ -438,3 +438,33 @@ def test_chunk_option_on_the_prefill_15b_shape_sampled(cuda_device, chunk):
                                 d["r_k"][h:h + 1])
         assert y_err(y[b:b + 1, :, h:h + 1], y_ref) <= TOL["bf16"], (b, h)
         assert state_err(S[b:b + 1, h:h + 1], S_ref) <= TOL["bf16"], (b, h)
+
+
+@pytest.mark.parametrize("B,H", [(4, 32), (4, 37), (8, 20)])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_scan_launch_shapes_by_head_count(cuda_device, B, H, dtype):
+    """The scan's launch by head count: 128 heads (two rows per thread, two CTAs per head), 148
+    and 160 (four rows per thread, one CTA per head); ragged T, S0, snapshots and the epilogue."""
+    wl = inputs.WORKLOADS[2]   # with the epilogue parameters
+    T, snap = 45, 9
+    d = inputs.make_inputs(wl, B=B, T=T, H=H, dtype=dtype, seed=1800 + B * H, s0="normal")
+    y_ref, S_ref, sn_ref = _oracle(d, snap_every=snap)
+    out_ref = native.epilogue(y_ref, d["r"], d["k"], d["v"], d["ln_w"], d["ln_b"], d["r_k"])
+    dd = _dev(d, cuda_device)
+    y, S, sn = _gpu(dd, algo="seq", snap_every=snap, ln_w=dd["ln_w"], ln_b=dd["ln_b"], r_k=dd["r_k"])
+    assert y_err(y, out_ref) <= TOL[dtype]
+    assert state_err(S, S_ref) <= TOL[dtype]
+    assert snaps_err(sn, sn_ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("H", [32, 40])
+def test_scan_raw_inputs_by_head_count(cuda_device, H):
+    """Raw inputs on the scan at 128 and 160 heads (two and four rows per thread)."""
+    d = inputs.make_raw_inputs(inputs.WORKLOADS[1], B=4, T=33, H=H, s0="normal", seed=1900 + H)
+    w, a, kk, kt = reference.prepare_inputs(d["w_logit"], d["a_logit"], d["k"], d["k_k"], d["k_a"])
+    y_ref, S_ref, _ = native.forward(d["r"], w, kt, d["v"], kk, a, d["S0"])
+    dd = _dev(d, cuda_device)
+    y, S, _ = wkv7.forward_raw(dd["r"], dd["w_logit"], dd["k"], dd["v"], dd["a_logit"], dd["k_k"], dd["k_a"],
+                               dd["S0"], algo="seq")
+    assert y_err(y, y_ref) <= TOL["bf16"]
+    assert state_err(S, S_ref) <= TOL["bf16"]
