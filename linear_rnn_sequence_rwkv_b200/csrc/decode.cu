@@ -26,10 +26,10 @@ constexpr int kDecThreads = 256;
 // EPI: the head's N readouts meet in shared memory; the first N threads normalise them over
 // the head (group_norm, population variance plus gn_eps) and add the bonus
 // (sum_j r_j k_j r_k[j]) v_i (rebuttal page, the listing's output lines).
-template <class Tin, int NN, bool RAW, bool EPI>
+template <class Tin, int NN, bool RAW, bool EPI, int THREADS = kDecThreads>
 __device__ __forceinline__ void decode_body(const DecArgs &p, const DecOpts &o) {
     constexpr int CL = NN / 4;                  // lanes per row (one float4 each)
-    constexpr int RS = kDecThreads / CL;        // row stride between a thread's rows
+    constexpr int RS = THREADS / CL;            // row stride between a thread's rows
     constexpr int RPT = NN / RS;                // rows per thread
     __shared__ float ys[EPI ? NN : 1];
     const int unit = blockIdx.x, h = unit % p.H;
@@ -125,16 +125,21 @@ __device__ __forceinline__ void decode_body(const DecArgs &p, const DecOpts &o) 
     }
 }
 
-// The prepared-input step, and the steps with raw inputs and/or the epilogue. The fused steps' bound
-// (four CTAs per SM at N = 64) measured faster than the tighter register budgets of five or six.
+// The prepared-input step, and the steps with raw inputs and/or the epilogue. At N = 64 the fused
+// steps run 128 threads per head (eight rows each): half as many row groups repeat the
+// pre-processing and the bonus. Measured on B256 H40 against 256 threads: raw inputs with the
+// epilogue 54.4 against 66.5 us (bound of eight CTAs per SM), raw inputs 55.9 against 58.1 and the
+// epilogue alone 58.4 against 59.1 us (bound of six).
+template <int NN> constexpr int kFusedThreads = NN == 64 ? 128 : kDecThreads;
+template <int NN, bool RAW, bool EPI> constexpr int kFusedMinCtas = NN == 64 ? (RAW && EPI ? 8 : 6) : 1;
 template <class Tin, int NN>
 __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecArgs p) {
     decode_body<Tin, NN, false, false>(p, DecOpts{});
 }
 template <class Tin, int NN, bool RAW, bool EPI>
-__global__ void __launch_bounds__(kDecThreads, NN == 64 ? 4 : 1)
+__global__ void __launch_bounds__(kFusedThreads<NN>, (kFusedMinCtas<NN, RAW, EPI>))
     decode_fused_kernel(const DecArgs p, const DecOpts o) {
-    decode_body<Tin, NN, RAW, EPI>(p, o);
+    decode_body<Tin, NN, RAW, EPI, kFusedThreads<NN>>(p, o);
 }
 
 template <class Tin, int NN>
@@ -142,11 +147,11 @@ cudaError_t launch_dec_t(const DecArgs &p, const DecOpts &o) {
     const unsigned units = unsigned(p.B) * unsigned(p.H);
     const bool raw = o.k_k != nullptr, epi = o.ln_w != nullptr;
     if (raw && epi)
-        decode_fused_kernel<Tin, NN, true, true><<<units, kDecThreads, 0, p.stream>>>(p, o);
+        decode_fused_kernel<Tin, NN, true, true><<<units, kFusedThreads<NN>, 0, p.stream>>>(p, o);
     else if (raw)
-        decode_fused_kernel<Tin, NN, true, false><<<units, kDecThreads, 0, p.stream>>>(p, o);
+        decode_fused_kernel<Tin, NN, true, false><<<units, kFusedThreads<NN>, 0, p.stream>>>(p, o);
     else if (epi)
-        decode_fused_kernel<Tin, NN, false, true><<<units, kDecThreads, 0, p.stream>>>(p, o);
+        decode_fused_kernel<Tin, NN, false, true><<<units, kFusedThreads<NN>, 0, p.stream>>>(p, o);
     else
         decode_kernel<Tin, NN><<<units, kDecThreads, 0, p.stream>>>(p);
     return cudaGetLastError();
