@@ -131,7 +131,7 @@ __device__ __forceinline__ void decode_body(const DecArgs &p, const DecOpts &o) 
 // epilogue 54.4 against 66.5 us (bound of eight CTAs per SM), raw inputs 55.9 against 58.1 and the
 // epilogue alone 58.4 against 59.1 us (bound of six).
 template <int NN> constexpr int kFusedThreads = NN == 64 ? 128 : kDecThreads;
-template <int NN, bool RAW, bool EPI> constexpr int kFusedMinCtas = NN == 64 ? (RAW && EPI ? 8 : 6) : 1;
+template <int NN, bool RAW, bool EPI> constexpr int kFusedMinCtas = NN == 64 ? (RAW && EPI ? 8 : 6) : 2;
 template <class Tin, int NN>
 __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecArgs p) {
     decode_body<Tin, NN, false, false>(p, DecOpts{});
