@@ -17,8 +17,9 @@ namespace {
 
 constexpr int kDecThreads = 256;
 
-// NN = 64: the layout above. NN = 128: a warp covers one 512-byte row (32 float4 columns) and
-// a thread holds rows t/32 + 8m, m = 0..15; the row dot products reduce over the 32 lanes.
+// NN = 64: the layout above (THREADS = 128, as the fused steps run: rows t/16 + 8m, m = 0..7).
+// NN = 128: a warp covers one 512-byte row (32 float4 columns) and a thread holds rows
+// t/32 + 8m, m = 0..15; the row dot products reduce over the 32 lanes.
 // RAW: w and a hold the decay and rate logits and k the key before its update; the load turns
 // them into w, a, the unit-norm removal key kk (its norm reduced over the CL lanes that hold
 // one row's channels) and the updated key k~ (rebuttal page, the time_mixing listing: decay,
