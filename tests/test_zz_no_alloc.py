@@ -32,6 +32,11 @@ def test_static_entry_rejects_requests_above_its_capacity():
                                   *(P(i) for i in range(8, 14)), None, None)
     assert st == wkv7.ERR_WORKSPACE
     assert b"static scratch" in lib.wkv7_last_error()
+    # N = 128: a head's two CTAs hold 64 KB states, one per two tokens of a segment
+    assert wkv7.backward_workspace_bytes(1, 1024, 1, N=128) == wkv7.STATIC_SCRATCH_BYTES   # exactly full
+    st = lib.wkv7_backward_static(1, 1026, 1, 128, 1, *(P(i) for i in range(1, 7)), None, None, 0, P(7), None,
+                                  *(P(i) for i in range(8, 14)), None, None)
+    assert st == wkv7.ERR_WORKSPACE
 
 
 @pytest.mark.gpu
