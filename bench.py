@@ -400,7 +400,7 @@ def run_gpu(args, world, rank, local):
         e2e = run_e2e(args, wl, dev, stream, B, T, H, N, seed0, epilogue, snap_every, warmup, steps, world, raw)
 
     out = {
-        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": steps,
+        "metric": METRIC.replace("N=64", f"N={N}"), "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": steps,
         "warmup": warmup, "ms_per_step": round(total_ms / steps, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32" if path in ("seq", "decode") else "tf32+f32",
         "data": "synthetic (seeded torch Philox; shapes and value ranges of the RWKV-7 pages' workloads)",
@@ -559,7 +559,8 @@ def run_backward(args, world, rank, local):
            "ms_per_step": round(e_ms / e_steps, 4)}
     epi = run_epilogue_backward_record(sets, wl, steps, warmup, world, dev, stream, peaks)
     out = {
-        "metric": METRIC.replace("(prefill, decode)", "(backward)"), "value": round(value, 3), "unit": UNIT,
+        "metric": METRIC.replace("(prefill, decode)", "(backward)").replace("N=64", f"N={N}"), "value": round(value, 3),
+        "unit": UNIT,
         "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": round(total_ms / steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded torch Philox; shapes and value ranges of the RWKV-7 pages' workloads)",
